@@ -1,0 +1,394 @@
+"""CPU oracle for the image half of the Mistral 3 / Pixtral multimodal forward.
+
+TEST INFRASTRUCTURE. Only the tests, `__graft_entry__.smoke()` and the
+`cpu_baseline` / reference leg of `bench.py` may import or run this module.
+The product path (the C-ABI library and its Python binding) never calls it
+and shares no code with it.
+
+What it computes, step by step, as plain numpy in float64 (matmul is the only
+library primitive used as a step):
+
+  vision tower ("Mistral 3", KerasFormers, API: `Mistral3VisionModel`:
+  conv patch embed -> RMS pre-norm -> 2D-rotary blocks over a packed
+  variable-resolution patch sequence)
+    a1  pixel normalisation with the processor's mean/std
+        ("Mistral 3", API: `Mistral3ImageProcessor`)
+    a2  patch embedding: a convolution with kernel = stride = patch size,
+        no bias (reading: the pages give no bias)
+    a3  `ln_pre` RMSNorm
+    a4..a10  per block: RMSNorm -> q,k,v -> 2D RoPE on q,k -> attention within
+        each image only -> o-projection + residual -> RMSNorm -> SiLU-gated MLP
+        + residual
+  patch-merging projector ("Mistral 3", API: `Mistral3Model`:
+  `spatial_merge_size` 2, `projector_bias` False)
+    a12 RMSNorm per patch, a13 2x2 unfold + concat -> merge linear,
+    a14 linear -> GELU -> linear
+  a15 masked scatter of the image rows into the text embeddings at
+      `image_token_id` positions (vllm.cpp issue "Mistral3ForConditionalGeneration
+      ...", "What we would contribute", item 2: gated so text rows stay
+      byte-identical)
+
+Readings taken where the pages are silent (each one is listed in the design
+notes): no biases anywhere; eps 1e-5 for every vision RMSNorm (the pages give
+1e-5 for the text model only); `ln_pre` plus pre-norm blocks and no final
+norm; SiLU-gated MLP; RoPE frequencies w_k = theta^(-2k/64), even k to the
+patch row, odd k to the patch column, rotation pairs (i, i+32); positions
+restart at (0, 0) in every image or tile; the projector RMSNorm is applied per
+patch before the merge; merged features in `unfold` channel-major order
+c*m*m + dy*m + dx; GELU in its erf form.
+
+Every function below is pinned by `tests/test_oracle_pins.py` against closed
+forms, library routines or brute force (no function here is "parity
+unpinned" except the end-to-end numbers of real trained weights, which do not
+exist in this environment).
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+from scipy.special import erf as _erf
+
+# "Mistral 3" (KerasFormers), API table `Mistral3Model`: vision_embed_dim 1024,
+# vision_mlp_dim 4096, vision_num_layers 24, vision_num_heads 16, patch_size 14,
+# vision_rope_theta 10000, spatial_merge_size 2, image_token_id 10; text
+# embed_dim 5120 is the projector's output width.
+MISTRAL3 = dict(layers=24, width=1024, heads=16, head_dim=64, mlp=4096, patch=14,
+                merge=2, proj_out=5120, image_token_id=10, rope_theta=1.0e4, eps=1.0e-5)
+
+# "Pixtral-12B-2409": ViT, 24 layers, hidden 1024, 16 heads, patch_size 16,
+# image_size 1024, intermediate 4096, rope_theta 1e4, no spatial merge.
+PIXTRAL12B = dict(MISTRAL3, patch=16, merge=1)
+
+# "Mistral 3" (KerasFormers), API table `Mistral3ImageProcessor`.
+IMAGE_MEAN = (0.48145466, 0.4578275, 0.40821073)
+IMAGE_STD = (0.26862954, 0.26130258, 0.27577711)
+LONGEST_EDGE = 1540
+PIXTRAL_TILE = 1024
+
+
+# ---------------------------------------------------------------------------
+# a0: shapes and positions
+# ---------------------------------------------------------------------------
+
+def patch_grid(height: int, width: int, patch: int) -> tuple:
+    """(h, w) patches of an image that lies on the patch grid.
+
+    "Mistral 3" intro: images are resized so they stay on the patch grid;
+    off-grid sizes are rejected here (reading: no padding or cropping).
+    """
+    if height <= 0 or width <= 0 or height % patch or width % patch:
+        raise ValueError(f"image {height}x{width} is not on the {patch}-pixel patch grid")
+    return height // patch, width // patch
+
+
+def merged_grid(h: int, w: int, merge: int) -> tuple:
+    """(h/m, w/m) merged tokens; `spatial_merge_size` m ("Mistral 3", `Mistral3Model`)."""
+    if h % merge or w % merge:
+        raise ValueError(f"patch grid {h}x{w} is not divisible by merge {merge}")
+    return h // merge, w // merge
+
+
+def tile_count(height: int, width: int, tile: int = PIXTRAL_TILE) -> int:
+    """Number of tile x tile tiles ("Pixtral-12B-2409", VISION TOKENS: 4096^2 -> 4x4 grid)."""
+    if height % tile or width % tile:
+        raise ValueError("image is not a whole number of tiles")
+    return (height // tile) * (width // tile)
+
+
+def positions(grids) -> tuple:
+    """Per-token (row, col) patch positions and block boundaries.
+
+    Patches are concatenated image after image, row-major inside each image
+    ("Mistral 3", `Mistral3VisionModel`: packed variable-resolution sequence).
+    Positions restart at (0, 0) in each image (reading).
+    Returns (rows int64 [T], cols int64 [T], cu_seqlens int64 [n+1]).
+    """
+    rows, cols, cu = [], [], [0]
+    for h, w in grids:
+        rr, cc = np.meshgrid(np.arange(h), np.arange(w), indexing="ij")
+        rows.append(rr.reshape(-1))
+        cols.append(cc.reshape(-1))
+        cu.append(cu[-1] + h * w)
+    return (np.concatenate(rows).astype(np.int64), np.concatenate(cols).astype(np.int64),
+            np.asarray(cu, dtype=np.int64))
+
+
+# ---------------------------------------------------------------------------
+# a1, a2: processor normalisation and patch embedding
+# ---------------------------------------------------------------------------
+
+def normalize_pixels(image: np.ndarray) -> np.ndarray:
+    """(x - mean_c) / std_c per channel ("Mistral 3", `Mistral3ImageProcessor`)."""
+    x = np.asarray(image, dtype=np.float64)
+    mean = np.asarray(IMAGE_MEAN, dtype=np.float64)[:, None, None]
+    std = np.asarray(IMAGE_STD, dtype=np.float64)[:, None, None]
+    return (x - mean) / std
+
+
+def im2col(image: np.ndarray, patch: int) -> np.ndarray:
+    """[h*w, 3*p*p] patch rows; row = r*w + c, column = ch*p*p + ky*p + kx."""
+    c, height, width = image.shape
+    h, w = patch_grid(height, width, patch)
+    x = np.asarray(image, dtype=np.float64).reshape(c, h, patch, w, patch)
+    return x.transpose(1, 3, 0, 2, 4).reshape(h * w, c * patch * patch)
+
+
+def patch_embed(image: np.ndarray, w_pe: np.ndarray) -> np.ndarray:
+    """Conv with kernel = stride = p and no bias, as im2col . W_pe^T.
+
+    "Mistral 3", `Mistral3VisionModel`: conv patch embed. w_pe is [D, 3, p, p].
+    """
+    d, _, p, _ = w_pe.shape
+    return im2col(image, p) @ np.asarray(w_pe, dtype=np.float64).reshape(d, -1).T
+
+
+# ---------------------------------------------------------------------------
+# a3/a4/a9/a12: RMSNorm
+# ---------------------------------------------------------------------------
+
+def rms_norm(x: np.ndarray, gain: np.ndarray, eps: float) -> np.ndarray:
+    """x / sqrt(mean(x^2) + eps) * gain over the last axis ("RMS pre-norm")."""
+    x = np.asarray(x, dtype=np.float64)
+    return x / np.sqrt(np.mean(x * x, axis=-1, keepdims=True) + eps) * np.asarray(gain, dtype=np.float64)
+
+
+# ---------------------------------------------------------------------------
+# a6: 2D rotary position embedding
+# ---------------------------------------------------------------------------
+
+def rope_frequencies(theta: float, head_dim: int) -> np.ndarray:
+    """w_k = theta^(-2k/head_dim), k = 0 .. head_dim/2 - 1 (vision_rope_theta 1e4)."""
+    k = np.arange(head_dim // 2, dtype=np.float64)
+    return theta ** (-2.0 * k / head_dim)
+
+
+def rope_angles(rows, cols, theta: float, head_dim: int) -> np.ndarray:
+    """[T, head_dim/2] angles: pair i < head_dim/4 turns by row * w_{2i},
+    pair i >= head_dim/4 by col * w_{2(i - head_dim/4) + 1} (reading: frequencies
+    split between the patch's row and column index, even ones to the row)."""
+    omega = rope_frequencies(theta, head_dim)
+    rows = np.asarray(rows, dtype=np.float64)
+    cols = np.asarray(cols, dtype=np.float64)
+    return np.concatenate([np.outer(rows, omega[0::2]), np.outer(cols, omega[1::2])], axis=1)
+
+
+def apply_rope(x: np.ndarray, angles: np.ndarray) -> np.ndarray:
+    """Rotate each pair (x_i, x_{i+half}) of every head by angles[:, i].
+
+    x is [T, heads, head_dim]; angles is [T, head_dim/2].
+    """
+    x = np.asarray(x, dtype=np.float64)
+    half = x.shape[-1] // 2
+    cos = np.cos(angles)[:, None, :]
+    sin = np.sin(angles)[:, None, :]
+    a, b = x[..., :half], x[..., half:]
+    return np.concatenate([a * cos - b * sin, b * cos + a * sin], axis=-1)
+
+
+# ---------------------------------------------------------------------------
+# a7: block-diagonal attention
+# ---------------------------------------------------------------------------
+
+def attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, cu_seqlens) -> np.ndarray:
+    """Bidirectional softmax attention where token t attends only to tokens of
+    its own block [cu[b], cu[b+1]) (one block per image or tile).
+
+    q, k, v are [T, heads, head_dim]; scores are scaled by 1/sqrt(head_dim);
+    the softmax subtracts the row maximum before exponentiating.
+    Returns [T, heads * head_dim], heads concatenated in order.
+    """
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    t_total, heads, dh = q.shape
+    out = np.zeros((t_total, heads, dh), dtype=np.float64)
+    scale = 1.0 / math.sqrt(dh)
+    for b in range(len(cu_seqlens) - 1):
+        lo, hi = int(cu_seqlens[b]), int(cu_seqlens[b + 1])
+        for h in range(heads):
+            kb, vb = k[lo:hi, h, :], v[lo:hi, h, :]
+            for q0 in range(lo, hi, 2048):  # query chunks bound the score matrix's memory
+                q1 = min(q0 + 2048, hi)
+                s = (q[q0:q1, h, :] @ kb.T) * scale
+                s -= s.max(axis=1, keepdims=True)
+                p = np.exp(s)
+                p /= p.sum(axis=1, keepdims=True)
+                out[q0:q1, h, :] = p @ vb
+    return out.reshape(t_total, heads * dh)
+
+
+def attention_rows(q, k, v, cu_seqlens, rows) -> np.ndarray:
+    """attention() evaluated for the listed query rows only (for sampled checks)."""
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    _, heads, dh = q.shape
+    cu = np.asarray(cu_seqlens)
+    scale = 1.0 / math.sqrt(dh)
+    out = np.zeros((len(rows), heads * dh), dtype=np.float64)
+    for i, t in enumerate(rows):
+        b = int(np.searchsorted(cu, t, side="right") - 1)
+        lo, hi = int(cu[b]), int(cu[b + 1])
+        for h in range(heads):
+            s = (k[lo:hi, h, :] @ q[t, h, :]) * scale
+            s -= s.max()
+            p = np.exp(s)
+            p /= p.sum()
+            out[i, h * dh:(h + 1) * dh] = p @ v[lo:hi, h, :]
+    return out
+
+
+# ---------------------------------------------------------------------------
+# a10, a14: activations
+# ---------------------------------------------------------------------------
+
+def silu(z):
+    """z * sigmoid(z) = z / (1 + e^-z)."""
+    z = np.asarray(z, dtype=np.float64)
+    return z / (1.0 + np.exp(-z))
+
+
+def gelu(z):
+    """Exact (erf) GELU: z * (1 + erf(z / sqrt 2)) / 2 (reading: the form is unstated)."""
+    z = np.asarray(z, dtype=np.float64)
+    return 0.5 * z * (1.0 + _erf(z / math.sqrt(2.0)))
+
+
+# ---------------------------------------------------------------------------
+# a4..a10: one tower block, and the tower
+# ---------------------------------------------------------------------------
+
+def tower_block(x: np.ndarray, lw: dict, angles: np.ndarray, cu_seqlens, cfg: dict) -> np.ndarray:
+    """x + attn(norm(x)), then + MLP(norm(.)) with pre-norm RMSNorms.
+
+    lw holds wq, wk, wv, wo [D, D], w_gate, w_up [F, D], w_down [D, F],
+    g_attn, g_ffn [D] (nn.Linear [out, in] layouts, y = x W^T).
+    """
+    t_total = x.shape[0]
+    heads, dh, eps = cfg["heads"], cfg["head_dim"], cfg["eps"]
+    xn = rms_norm(x, lw["g_attn"], eps)
+    q = (xn @ lw["wq"].T).reshape(t_total, heads, dh)
+    k = (xn @ lw["wk"].T).reshape(t_total, heads, dh)
+    v = (xn @ lw["wv"].T).reshape(t_total, heads, dh)
+    q = apply_rope(q, angles)
+    k = apply_rope(k, angles)
+    x = x + attention(q, k, v, cu_seqlens) @ lw["wo"].T
+    xn = rms_norm(x, lw["g_ffn"], eps)
+    hidden = silu(xn @ lw["w_gate"].T) * (xn @ lw["w_up"].T)
+    return x + hidden @ lw["w_down"].T
+
+
+def layer_weights(tw: dict, layer: int) -> dict:
+    names = ("wq", "wk", "wv", "wo", "w_gate", "w_up", "w_down", "g_attn", "g_ffn")
+    return {n: np.asarray(tw[n][layer], dtype=np.float64) for n in names}
+
+
+def tower(images, tw: dict, cfg: dict, layers: int | None = None, normalize: bool = True) -> np.ndarray:
+    """Vision tower over a packed sequence of images.
+
+    images: list of fp [3, H, W] arrays (raw U[0,1) pixels if `normalize`).
+    tw: w_pe [D,3,p,p], g_pre [D], stacked per-layer tensors [L, ...].
+    Returns the residual stream after the last block, [T, D] (no final norm).
+    """
+    p, eps = cfg["patch"], cfg["eps"]
+    n_layers = cfg["layers"] if layers is None else layers
+    grids = [patch_grid(im.shape[1], im.shape[2], p) for im in images]
+    rows, cols, cu = positions(grids)
+    w_pe = np.asarray(tw["w_pe"], dtype=np.float64)
+    x = np.concatenate([patch_embed(normalize_pixels(im) if normalize else np.asarray(im, np.float64), w_pe)
+                        for im in images], axis=0)
+    x = rms_norm(x, tw["g_pre"], eps)
+    angles = rope_angles(rows, cols, cfg["rope_theta"], cfg["head_dim"])
+    for layer in range(n_layers):
+        x = tower_block(x, layer_weights(tw, layer), angles, cu, cfg)
+    return x
+
+
+# ---------------------------------------------------------------------------
+# a12..a14: patch-merging projector
+# ---------------------------------------------------------------------------
+
+def merge_unfold(x: np.ndarray, grids, merge: int) -> np.ndarray:
+    """2x2 (m x m) unfold + concat per image.
+
+    For image b with patch grid (h, w) and merged position (i, j):
+    z[c*m*m + dy*m + dx] = x[off_b + (m*i + dy)*w + (m*j + dx), c]
+    (channel-major order of an unfold with kernel = stride = m). Merged tokens
+    are row-major per image, images concatenated.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    d = x.shape[1]
+    out, off = [], 0
+    for h, w in grids:
+        hm, wm = merged_grid(h, w, merge)
+        img = x[off:off + h * w].reshape(hm, merge, wm, merge, d)  # [i, dy, j, dx, c]
+        out.append(img.transpose(0, 2, 4, 1, 3).reshape(hm * wm, d * merge * merge))
+        off += h * w
+    return np.concatenate(out, axis=0)
+
+
+def projector(x_tower: np.ndarray, grids, pw: dict, cfg: dict) -> np.ndarray:
+    """RMSNorm per patch -> m x m merge -> merge linear -> W1 -> GELU -> W2, no biases.
+
+    ("Mistral 3", `Mistral3Model`: 2x2 patch-merging projector, projector_bias
+    False, text width 5120.) pw: g_proj [D], w_merge [D, m*m*D], w1 [E, D],
+    w2 [E, E].
+    """
+    xn = rms_norm(x_tower, pw["g_proj"], cfg["eps"])
+    z = merge_unfold(xn, grids, cfg["merge"]) if cfg["merge"] > 1 else xn
+    y = z @ np.asarray(pw["w_merge"], dtype=np.float64).T if cfg["merge"] > 1 else z
+    return gelu(y @ np.asarray(pw["w1"], dtype=np.float64).T) @ np.asarray(pw["w2"], dtype=np.float64).T
+
+
+# ---------------------------------------------------------------------------
+# a15: masked scatter
+# ---------------------------------------------------------------------------
+
+def scatter(input_ids: np.ndarray, image_rows: np.ndarray, text_rows: np.ndarray,
+            image_token_id: int) -> np.ndarray:
+    """Copy image row k into the k-th position whose id equals image_token_id.
+
+    Rows are copied as raw bits (any dtype); every other row is left as it
+    was. Raises if the placeholder count differs from the number of image rows.
+    """
+    ids = np.asarray(input_ids).reshape(-1)
+    out = np.array(text_rows, copy=True)
+    k = 0
+    for i in range(ids.shape[0]):
+        if ids[i] == image_token_id:
+            if k < image_rows.shape[0]:
+                out[i] = image_rows[k]
+            k += 1
+    if k != image_rows.shape[0]:
+        raise ValueError(f"{k} placeholders for {image_rows.shape[0]} image rows")
+    return out
+
+
+# ---------------------------------------------------------------------------
+# The whole image half
+# ---------------------------------------------------------------------------
+
+def encode_merge_project(images, tw: dict, pw: dict, cfg: dict, layers: int | None = None,
+                         normalize: bool = True) -> tuple:
+    """(tower output [T, D], projected image embeddings [T_m, E])."""
+    grids = [patch_grid(im.shape[1], im.shape[2], cfg["patch"]) for im in images]
+    xt = tower(images, tw, cfg, layers=layers, normalize=normalize)
+    return xt, projector(xt, grids, pw, cfg)
+
+
+def flops(cfg: dict, grids, layers: int | None = None) -> float:
+    """Algorithmic FLOPs (2 per multiply-add) of tower + merge + projector.
+
+    Attention is counted over each block's own L_b^2 query-key pairs only.
+    """
+    d, f, e, m, p = cfg["width"], cfg["mlp"], cfg["proj_out"], cfg["merge"], cfg["patch"]
+    n_layers = cfg["layers"] if layers is None else layers
+    total = 0.0
+    for h, w in grids:
+        lb = h * w
+        per_layer = lb * 2 * (3 * d * d + d * d + 3 * d * f) + 4 * lb * lb * d
+        total += n_layers * per_layer + lb * 2 * 3 * p * p * d
+        tm = lb // (m * m)
+        total += tm * (2 * (m * m * d) * d if m > 1 else 0) + tm * 2 * (d * e + e * e)
+    return total

@@ -1,0 +1,391 @@
+"""Pins of the CPU oracle against things other than itself.
+
+Each test ties one oracle function to a closed form, a value the pages print
+(tests/golden/), a library routine that computes the same definition by
+another route, a special case, or brute force on a tiny input. The last block
+plants plausible mistakes into the oracle (on the CPU) and checks that a pin
+catches each one.
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+import torch.nn.functional as F
+
+from oracle import vlm_oracle as O
+from vision_language_model_b200 import synth
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+RNG = np.random.default_rng(1234)
+
+
+def _golden(name):
+    with open(os.path.join(GOLDEN, name)) as fh:
+        return json.load(fh)
+
+
+# ---------------------------------------------------------------------------
+# a0 / a13 counts: values printed on the pages
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("case", _golden("token_counts.json")["cases"], ids=lambda c: c["name"])
+def test_token_counts_match_pages(case):
+    h, w = O.patch_grid(case["height"], case["width"], case["patch"])
+    assert h * w == case["patches"]
+    hm, wm = O.merged_grid(h, w, case["merge"])
+    assert hm * wm == case["merged"]
+
+
+@pytest.mark.parametrize("case", _golden("token_counts.json")["tiled"], ids=lambda c: c["name"])
+def test_tiled_token_counts_match_pages(case):
+    n = O.tile_count(case["height"], case["width"], case["tile"])
+    assert n == case["tiles"]
+    h, w = O.patch_grid(case["tile"], case["tile"], case["patch"])
+    assert n * h * w == case["tokens"]
+
+
+def test_hparams_match_pages():
+    g = _golden("hparams.json")
+    for preset, ref in (("mistral3", O.MISTRAL3), ("pixtral12b", O.PIXTRAL12B)):
+        for key in ("width", "mlp", "layers", "heads", "patch", "rope_theta", "merge"):
+            assert ref[key] == g[preset][key], (preset, key)
+    assert O.MISTRAL3["image_token_id"] == g["mistral3"]["image_token_id"]
+    assert O.MISTRAL3["proj_out"] == g["mistral3"]["proj_out"]
+    assert list(O.IMAGE_MEAN) == g["processor"]["image_mean"]
+    assert list(O.IMAGE_STD) == g["processor"]["image_std"]
+    assert O.LONGEST_EDGE == g["processor"]["longest_edge"]
+
+
+def test_off_grid_sizes_rejected():
+    with pytest.raises(ValueError):
+        O.patch_grid(225, 224, 14)
+    with pytest.raises(ValueError):
+        O.merged_grid(15, 16, 2)
+    assert O.merged_grid(15, 16, 1) == (15, 16)
+
+
+def test_positions_restart_per_image():
+    rows, cols, cu = O.positions([(2, 3), (1, 2)])
+    assert cu.tolist() == [0, 6, 8]
+    assert rows.tolist() == [0, 0, 0, 1, 1, 1, 0, 0]
+    assert cols.tolist() == [0, 1, 2, 0, 1, 2, 0, 1]
+
+
+# ---------------------------------------------------------------------------
+# a1, a2: normalisation and patch embedding
+# ---------------------------------------------------------------------------
+
+def test_normalize_constants():
+    img = np.ones((3, 2, 2))
+    got = O.normalize_pixels(img)
+    for c in range(3):
+        assert got[c, 0, 0] == pytest.approx((1.0 - O.IMAGE_MEAN[c]) / O.IMAGE_STD[c], rel=1e-15)
+
+
+@pytest.mark.parametrize("patch,hw", [(14, (28, 42)), (16, (32, 48)), (3, (9, 6))])
+def test_patch_embed_equals_strided_conv2d(patch, hw):
+    d = 8
+    img = RNG.standard_normal((3, *hw))
+    w = RNG.standard_normal((d, 3, patch, patch))
+    got = O.patch_embed(img, w)
+    ref = F.conv2d(torch.from_numpy(img)[None], torch.from_numpy(w), stride=patch)[0]  # [D, h, w]
+    ref = ref.permute(1, 2, 0).reshape(-1, d).numpy()
+    np.testing.assert_allclose(got, ref, rtol=1e-12, atol=1e-12)
+
+
+def test_patch_embed_p1_identity_is_passthrough():
+    img = RNG.standard_normal((3, 4, 5))
+    w = np.eye(3).reshape(3, 3, 1, 1)
+    got = O.patch_embed(img, w)
+    np.testing.assert_array_equal(got, img.transpose(1, 2, 0).reshape(20, 3))
+
+
+# ---------------------------------------------------------------------------
+# RMSNorm
+# ---------------------------------------------------------------------------
+
+def test_rmsnorm_constant_vector_gives_sign_times_gain():
+    g = RNG.standard_normal(64)
+    for cval in (3.5, -0.25):
+        y = O.rms_norm(np.full((1, 64), cval), g, 0.0)
+        np.testing.assert_allclose(y[0], math.copysign(1.0, cval) * g, rtol=1e-14)
+
+
+def test_rmsnorm_matches_torch():
+    x = RNG.standard_normal((7, 1024)) * 3
+    g = RNG.standard_normal(1024)
+    ref = F.rms_norm(torch.from_numpy(x), (1024,), torch.from_numpy(g), eps=1e-5).numpy()
+    np.testing.assert_allclose(O.rms_norm(x, g, 1e-5), ref, rtol=1e-12, atol=1e-12)
+
+
+# ---------------------------------------------------------------------------
+# 2D RoPE
+# ---------------------------------------------------------------------------
+
+def test_rope_frequencies_closed_form():
+    om = O.rope_frequencies(1e4, 64)
+    assert om[0] == 1.0
+    assert om[2] == pytest.approx(10.0 ** -0.25, rel=1e-14)   # 1e4^(-4/64)
+    assert om[31] == pytest.approx(1e4 ** (-62 / 64), rel=1e-14)
+    # pair 1 at (row 1, col 0) turns by w_2; pair 16 at (row 0, col 1) by w_1
+    ang = O.rope_angles([1, 0], [0, 1], 1e4, 64)
+    assert ang[0, 1] == pytest.approx(10.0 ** -0.25, rel=1e-14)
+    assert ang[1, 16] == pytest.approx(1e4 ** (-2 / 64), rel=1e-14)
+    assert np.all(ang[0, 16:] == 0) and np.all(ang[1, :16] == 0)
+
+
+def test_rope_is_complex_rotation():
+    x = RNG.standard_normal((5, 2, 64))
+    ang = O.rope_angles(np.arange(5), np.arange(5)[::-1], 1e4, 64)
+    got = O.apply_rope(x, ang)
+    z = (x[..., :32] + 1j * x[..., 32:]) * np.exp(1j * ang)[:, None, :]
+    np.testing.assert_allclose(got[..., :32], z.real, rtol=1e-13, atol=1e-13)
+    np.testing.assert_allclose(got[..., 32:], z.imag, rtol=1e-13, atol=1e-13)
+
+
+def test_rope_preserves_norm_and_origin_is_identity():
+    x = RNG.standard_normal((16, 3, 64))
+    rows, cols, _ = O.positions([(4, 4)])
+    y = O.apply_rope(x, O.rope_angles(rows, cols, 1e4, 64))
+    np.testing.assert_allclose(np.linalg.norm(y, axis=-1), np.linalg.norm(x, axis=-1), rtol=1e-6)
+    np.testing.assert_array_equal(y[0], x[0])  # position (0, 0)
+
+
+def test_rope_scores_depend_only_on_relative_position_bruteforce_4x4():
+    q = RNG.standard_normal(64)
+    k = RNG.standard_normal(64)
+    grid = [(r, c) for r in range(4) for c in range(4)]
+    seen = {}
+    for r1, c1 in grid:
+        for r2, c2 in grid:
+            qa = O.apply_rope(q[None, None], O.rope_angles([r1], [c1], 1e4, 64))[0, 0]
+            ka = O.apply_rope(k[None, None], O.rope_angles([r2], [c2], 1e4, 64))[0, 0]
+            seen.setdefault((r1 - r2, c1 - c2), []).append(float(qa @ ka))
+    assert len(seen) == 49
+    for vals in seen.values():
+        assert max(vals) - min(vals) < 1e-5 * max(1.0, max(abs(v) for v in vals))
+    # different offsets give different scores in general
+    assert abs(seen[(1, 0)][0] - seen[(0, 1)][0]) > 1e-6
+
+
+def test_rope_row_shift_changes_only_row_half():
+    x = RNG.standard_normal((1, 1, 64))
+    a = O.apply_rope(x, O.rope_angles([0], [2], 1e4, 64))
+    b = O.apply_rope(x, O.rope_angles([3], [2], 1e4, 64))
+    pairs_changed = np.abs(a - b)[0, 0]
+    changed = (pairs_changed[:32] > 0) | (pairs_changed[32:] > 0)
+    assert changed[:16].all() and not changed[16:].any()
+
+
+# ---------------------------------------------------------------------------
+# Attention
+# ---------------------------------------------------------------------------
+
+def _sdpa_blockdiag(q, k, v, cu):
+    t = q.shape[0]
+    mask = torch.zeros(t, t, dtype=torch.bool)
+    for b in range(len(cu) - 1):
+        mask[cu[b]:cu[b + 1], cu[b]:cu[b + 1]] = True
+    qt, kt, vt = (torch.from_numpy(a).permute(1, 0, 2)[None] for a in (q, k, v))
+    o = F.scaled_dot_product_attention(qt, kt, vt, attn_mask=mask)[0]  # [H, T, dh]
+    return o.permute(1, 0, 2).reshape(t, -1).numpy()
+
+
+def test_attention_matches_sdpa_block_diagonal():
+    cu = [0, 5, 6, 19, 40]
+    q, k, v = (RNG.standard_normal((40, 3, 64)) * 2 for _ in range(3))
+    np.testing.assert_allclose(O.attention(q, k, v, cu), _sdpa_blockdiag(q, k, v, cu), rtol=1e-11, atol=1e-12)
+    rows = [0, 5, 18, 39]
+    np.testing.assert_allclose(O.attention_rows(q, k, v, cu, rows), O.attention(q, k, v, cu)[rows], rtol=1e-12)
+
+
+def test_attention_single_patch_returns_v_and_zero_q_gives_mean():
+    q, k, v = (RNG.standard_normal((1, 2, 64)) for _ in range(3))
+    np.testing.assert_array_equal(O.attention(q, k, v, [0, 1]), v.reshape(1, -1))
+    q0 = np.zeros((9, 2, 64))
+    k, v = RNG.standard_normal((9, 2, 64)), RNG.standard_normal((9, 2, 64))
+    out = O.attention(q0, k, v, [0, 9])
+    np.testing.assert_allclose(out, np.broadcast_to(v.mean(axis=0).reshape(1, -1), (9, 128)), rtol=1e-13)
+
+
+# ---------------------------------------------------------------------------
+# Activations and MLP
+# ---------------------------------------------------------------------------
+
+def test_activations_special_values_and_library():
+    z = np.linspace(-8, 8, 101)
+    assert O.silu(0.0) == 0.0 and O.gelu(0.0) == 0.0
+    np.testing.assert_allclose(O.silu(z), F.silu(torch.from_numpy(z)).numpy(), rtol=1e-13, atol=1e-15)
+    np.testing.assert_allclose(O.gelu(z), F.gelu(torch.from_numpy(z)).numpy(), rtol=1e-13, atol=1e-15)
+    assert O.gelu(30.0) == pytest.approx(30.0, rel=1e-15)
+    assert O.gelu(1.0) == pytest.approx(0.5 * (1 + math.erf(1 / math.sqrt(2))), rel=1e-15)
+
+
+def _tiny_tower(seed=0, layers=2, width=64, mlp=128, patch=14, heads=4):
+    cfg = dict(O.MISTRAL3, layers=layers, width=width, mlp=mlp, heads=heads, head_dim=width // heads)
+    tw = {k: v.double().numpy() for k, v in synth.tower_weights(seed, layers, width, mlp, patch).items()}
+    return cfg, tw
+
+
+def test_mlp_with_zero_up_is_identity_block_on_ffn_half():
+    cfg, tw = _tiny_tower(layers=1, heads=1)
+    cfg["head_dim"] = 64
+    lw = O.layer_weights(tw, 0)
+    lw["w_up"][:] = 0.0
+    lw["wo"][:] = 0.0  # attention branch off too
+    x = RNG.standard_normal((6, 64))
+    rows, cols, cu = O.positions([(2, 3)])
+    y = O.tower_block(x, lw, O.rope_angles(rows, cols, 1e4, 64), cu, cfg)
+    np.testing.assert_array_equal(y, x)
+
+
+# ---------------------------------------------------------------------------
+# Tower-level invariants: isolation and packing
+# ---------------------------------------------------------------------------
+
+def test_tower_isolation_and_packed_equals_separate():
+    cfg, tw = _tiny_tower(heads=1)
+    cfg["head_dim"] = 64
+    imgs = [synth.pixels_u01(0, f"iso{i}", h, w).double().numpy() for i, (h, w) in enumerate([(28, 42), (14, 14), (42, 28)])]
+    packed = O.tower(imgs, tw, cfg)
+    sep = np.concatenate([O.tower([im], tw, cfg) for im in imgs], axis=0)
+    np.testing.assert_allclose(packed, sep, rtol=1e-12, atol=1e-12)
+    pert = [im.copy() for im in imgs]
+    pert[1] += 0.5
+    out2 = O.tower(pert, tw, cfg)
+    n0, n1 = 6, 1
+    np.testing.assert_array_equal(out2[:n0], packed[:n0])
+    np.testing.assert_array_equal(out2[n0 + n1:], packed[n0 + n1:])
+    assert np.abs(out2[n0:n0 + n1] - packed[n0:n0 + n1]).max() > 1e-3
+
+
+# ---------------------------------------------------------------------------
+# Merge
+# ---------------------------------------------------------------------------
+
+def test_merge_matches_torch_unfold():
+    d = 5
+    grids = [(4, 6), (2, 2)]
+    x = RNG.standard_normal((28, d))
+    got = O.merge_unfold(x, grids, 2)
+    ref, off = [], 0
+    for h, w in grids:
+        img = torch.from_numpy(x[off:off + h * w]).reshape(h, w, d).permute(2, 0, 1)[None]  # [1, D, h, w]
+        ref.append(F.unfold(img, kernel_size=2, stride=2)[0].T.numpy())  # [L, D*4] channel-major
+        off += h * w
+    np.testing.assert_array_equal(got, np.concatenate(ref))
+
+
+def test_merge_selector_weights_pick_the_right_patch():
+    d, h, w = 3, 4, 4
+    x = RNG.standard_normal((h * w, d))
+    z = O.merge_unfold(x, [(h, w)], 2)
+    for c in range(d):
+        for dy in range(2):
+            for dx in range(2):
+                sel = np.zeros(4 * d)
+                sel[c * 4 + dy * 2 + dx] = 1.0
+                for i in range(2):
+                    for j in range(2):
+                        assert z[i * 2 + j] @ sel == x[(2 * i + dy) * w + (2 * j + dx), c]
+
+
+# ---------------------------------------------------------------------------
+# Scatter
+# ---------------------------------------------------------------------------
+
+def test_scatter_matches_masked_scatter_bit_exact():
+    ids = synth.text_sequences(3, 2, 64, [[5], [7, 2]])
+    n_img = int((ids == 10).sum())
+    assert n_img == 14
+    img = synth.randn_bf16(3, "img", (n_img, 32), 1.0)
+    text = synth.text_embeddings(3, 128, 32)
+    got = O.scatter(ids.numpy(), img.view(torch.int16).numpy(), text.view(torch.int16).numpy(), 10)
+    mask = (ids.reshape(-1) == 10)[:, None].expand(-1, 32)
+    ref = text.masked_scatter(mask, img)
+    assert np.array_equal(got, ref.view(torch.int16).numpy())
+    untouched = ~(ids.reshape(-1) == 10).numpy()
+    assert np.array_equal(got[untouched], text.view(torch.int16).numpy()[untouched])
+
+
+def test_scatter_count_mismatch_raises():
+    ids = np.array([1, 10, 10, 3])
+    with pytest.raises(ValueError):
+        O.scatter(ids, np.zeros((3, 4), np.int16), np.zeros((4, 4), np.int16), 10)
+    with pytest.raises(ValueError):
+        O.scatter(ids, np.zeros((1, 4), np.int16), np.zeros((4, 4), np.int16), 10)
+
+
+def test_text_placeholder_runs_count():
+    ids = synth.text_sequences(0, 4, 4096, [[1536]] * 4)
+    assert ((ids == 10).sum(dim=1) == 1536).all()
+    # one contiguous run per sequence
+    for s in range(4):
+        pos = torch.nonzero(ids[s] == 10).reshape(-1)
+        assert int(pos[-1] - pos[0]) == 1535
+
+
+# ---------------------------------------------------------------------------
+# FLOP counter: closed form of the config-2 total
+# ---------------------------------------------------------------------------
+
+def test_flop_count_closed_form():
+    total = O.flops(O.MISTRAL3, [(110, 110)])
+    t, d, f = 12100, 1024, 4096
+    tower = 24 * (t * 2 * (4 * d * d + 3 * d * f) + 4 * t * t * d)
+    assert total == pytest.approx(tower + t * 2 * 588 * d + 3025 * 2 * (4096 * d + d * 5120 + 5120 * 5120), rel=1e-15)
+    assert total == pytest.approx(2.437e13, rel=2e-3)
+
+
+# ---------------------------------------------------------------------------
+# Planted mistakes: each must be caught by one of the pins above
+# ---------------------------------------------------------------------------
+
+def test_planted_rope_sign_error_is_caught(monkeypatch):
+    def bad(x, angles):
+        half = x.shape[-1] // 2
+        cos, sin = np.cos(angles)[:, None, :], np.sin(angles)[:, None, :]
+        a, b = x[..., :half], x[..., half:]
+        return np.concatenate([a * cos + b * sin, b * cos + a * sin], axis=-1)
+    monkeypatch.setattr(O, "apply_rope", bad)
+    with pytest.raises(AssertionError):
+        test_rope_preserves_norm_and_origin_is_identity()
+
+
+def test_planted_missing_attention_scale_is_caught(monkeypatch):
+    orig = O.attention
+
+    def bad(q, k, v, cu):
+        return orig(np.asarray(q) * 8.0, k, v, cu)
+    monkeypatch.setattr(O, "attention", bad)
+    with pytest.raises(AssertionError):
+        test_attention_matches_sdpa_block_diagonal()
+
+
+def test_planted_merge_order_swap_is_caught(monkeypatch):
+    def bad(x, grids, merge):
+        x = np.asarray(x, dtype=np.float64)
+        d = x.shape[1]
+        out, off = [], 0
+        for h, w in grids:
+            hm, wm = h // merge, w // merge
+            img = x[off:off + h * w].reshape(hm, merge, wm, merge, d)
+            out.append(img.transpose(0, 2, 4, 3, 1).reshape(hm * wm, d * merge * merge))  # dx, dy swapped
+            off += h * w
+        return np.concatenate(out, axis=0)
+    monkeypatch.setattr(O, "merge_unfold", bad)
+    with pytest.raises(AssertionError):
+        test_merge_matches_torch_unfold()
+
+
+def test_planted_rope_frequency_split_swap_is_caught(monkeypatch):
+    orig = O.rope_angles
+
+    def bad(rows, cols, theta, head_dim):
+        return orig(cols, rows, theta, head_dim)
+    monkeypatch.setattr(O, "rope_angles", bad)
+    with pytest.raises(AssertionError):
+        test_rope_frequencies_closed_form()
