@@ -1,0 +1,446 @@
+#!/usr/bin/env python
+"""Throughput of the image half of the Mistral 3 / Pixtral forward on B200.
+
+One step = the whole path on one batch of synthetic input: the 24-layer
+vision tower (vlm_encode), the 2x2 merge + projector (vlm_merge_project) and
+the masked scatter of the image embeddings into a text-embedding sequence
+(vlm_scatter). Metric: vision patches per second (whole job, all ranks).
+
+    python bench.py [--gpus N --steps K --warmup W] [--workload NAME] [--impl reference]
+
+N > 1 runs one independent replica per GPU (launched by torch.distributed.run;
+no collective on the data path; a NCCL all-reduce only takes the max of the
+ranks' timings).
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "vision patches/sec through 24-layer tower+merger+projector; % BF16 TC peak"
+
+# Workloads: image sizes (H, W) of one step and the text sequences the
+# embeddings are scattered into.
+WORKLOADS = {
+    "mistral3_1540": dict(preset="mistral3", sizes=[(1540, 1540)], n_seq=1, seq_len=4096,
+                          desc="one 1540x1540 image (110x110 = 12,100 patches -> 3,025 merged tokens), "
+                               "24-layer tower + 2x2 merge + projector 1024->5120->5120 + scatter into "
+                               "4,096 text tokens"),
+    "packed8": dict(preset="mistral3", sizes="packed", n_seq=1, seq_len=16384,
+                    desc="8 images, sides 28*U{10..55} (seed 0), packed into one sequence"),
+    "pixtral_4096": dict(preset="pixtral12b", sizes=[(1024, 1024)] * 16, n_seq=16, seq_len=4352,
+                         desc="Pixtral-12B-style: one 4096x4096 image as 16 tiles of 1024x1024 = 65,536 patches, "
+                              "no merge, projector 1024->5120->5120"),
+    "e2e4": dict(preset="mistral3", sizes=[(896, 1344)] * 4, n_seq=4, seq_len=4096,
+                 desc="4 x 896x1344 images (6,144 patches -> 1,536 placeholders each) scattered into 4 x 4,096 ids"),
+}
+
+
+def parse_args():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=20)
+    p.add_argument("--warmup", type=int, default=3)
+    p.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    p.add_argument("--workload", default="mistral3_1540", choices=sorted(WORKLOADS))
+    p.add_argument("--seed", type=int, default=0)
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--profile-steps", type=int, default=0,
+                   help="for ncu: run this many plain steps after warmup and exit (no JSON)")
+    return p.parse_args()
+
+
+def sizes_of(wl: dict, seed: int):
+    from vision_language_model_b200 import synth
+    return synth.packed_sizes(seed, 8) if wl["sizes"] == "packed" else list(wl["sizes"])
+
+
+def measured_peaks() -> dict:
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as fh:
+            d = json.load(fh)
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d["bf16_tflops_sustained"], "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+# ---------------------------------------------------------------------------
+# FLOP accounting (2 FLOPs per multiply-add; attention over each block's own L_b^2 pairs)
+# ---------------------------------------------------------------------------
+
+def flops_breakdown(cfg, sizes) -> dict:
+    D, F, E, m, p, L = cfg.width, cfg.mlp, cfg.proj_out, cfg.merge, cfg.patch, cfg.layers
+    lens = [(h // p) * (w // p) for h, w in sizes]
+    T = sum(lens)
+    Tm = sum(n // (m * m) for n in lens)
+    gemm = 2.0 * T * 3 * p * p * D
+    gemm += L * 2.0 * T * (3 * D * D + D * D + 2 * F * D + F * D)
+    gemm += (2.0 * Tm * m * m * D * D if m > 1 else 0.0) + 2.0 * Tm * (D * E + E * E)
+    attn_per_launch = sum(4.0 * n * n * D for n in lens)
+    return {"T": T, "Tm": Tm, "gemm": gemm, "attn_per_launch": attn_per_launch, "attn": L * attn_per_launch,
+            "total": gemm + L * attn_per_launch}
+
+
+# ---------------------------------------------------------------------------
+# Clocks sampled during the timed region
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.proc = None
+        self.lines = []
+        try:
+            uuid = "GPU-" + str(torch.cuda.get_device_properties(device_index).uuid)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", uuid, f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                smax.append(float(parts[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[3:7]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# Distributed plumbing (replicas; the all-reduce only takes max over ranks)
+# ---------------------------------------------------------------------------
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=180),
+                                device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(world, value: float) -> float:
+    if world == 1:
+        return value
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------------------
+# CPU baseline: the oracle, on a bounded sample of the same workload
+# ---------------------------------------------------------------------------
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return int(max(n)) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+class OracleSample:
+    """Times the oracle on the workload: patch embed + ln_pre on all patches,
+    one tower block (keys/values of all patches once, then every per-row step
+    on a strided slice of 1/`frac` of the patches), and the projector on all
+    merged tokens; the tower time is extrapolated to all rows and all layers."""
+
+    def __init__(self, wl: dict, seed: int, frac: int):
+        from oracle import vlm_oracle as O
+        from vision_language_model_b200 import synth
+        self.O = O
+        self.sizes = sizes_of(wl, seed)
+        base = O.MISTRAL3 if wl["preset"] == "mistral3" else O.PIXTRAL12B
+        self.cfg = dict(base)
+        self.frac = frac
+        tw = synth.tower_weights(seed, 1, base["width"], base["mlp"], base["patch"])
+        self.tw = {k: v.double().numpy() for k, v in tw.items()}
+        self.lw = O.layer_weights(self.tw, 0)
+        pw = synth.projector_weights(seed, base["width"], base["merge"], base["proj_out"])
+        self.pw = {k: v.double().numpy() for k, v in pw.items()}
+        self.imgs = [im.double().numpy() for im in synth.images(seed, self.sizes)]
+        self.grids = [O.patch_grid(h, w, base["patch"]) for h, w in self.sizes]
+        self.T = sum(h * w for h, w in self.grids)
+        self.step_i = 0
+
+    def prepare(self):
+        O = self.O
+        t0 = time.perf_counter()
+        x = np.concatenate([O.patch_embed(O.normalize_pixels(im), self.tw["w_pe"]) for im in self.imgs])
+        self.x = O.rms_norm(x, self.tw["g_pre"], self.cfg["eps"])
+        t1 = time.perf_counter()
+        rows, cols, self.cu = O.positions(self.grids)
+        self.ang = O.rope_angles(rows, cols, self.cfg["rope_theta"], self.cfg["head_dim"])
+        self.kv = O.block_keys_values(self.x, self.lw, self.ang, self.cfg)
+        t2 = time.perf_counter()
+        O.projector(self.x, self.grids, self.pw, self.cfg)
+        t3 = time.perf_counter()
+        self.t_embed, self.t_kv, self.t_proj = t1 - t0, t2 - t1, t3 - t2
+
+    def step(self) -> float:
+        rows = np.arange(self.step_i % self.frac, self.T, self.frac)
+        self.step_i += 1
+        t0 = time.perf_counter()
+        self.O.tower_block_rows(self.x, self.lw, self.ang, self.cu, self.cfg, rows, kv=self.kv)
+        return (time.perf_counter() - t0) * self.T / len(rows)
+
+    def patches_per_s(self, t_rows_full: float, layers: int) -> float:
+        return self.T / (self.t_embed + layers * (self.t_kv + t_rows_full) + self.t_proj)
+
+    def describe(self) -> str:
+        return (f"oracle (numpy fp64): patch embed of all {self.T} patches, keys/values of one tower block for all "
+                f"patches, the rest of that block on every {self.frac}th patch, projector on all merged tokens; "
+                f"tower time extrapolated to all patches and 24 layers")
+
+
+def cpu_baseline(wl, seed) -> dict:
+    s = OracleSample(wl, seed, frac=4)
+    s.prepare()
+    t_rows = s.step()
+    return {"value": s.patches_per_s(t_rows, 24), "unit": "patches/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": s.describe()}
+
+
+def run_reference(args, wl):
+    world, rank, _ = int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")), 0
+    if rank != 0:
+        return
+    s = OracleSample(wl, args.seed, frac=16)
+    s.prepare()
+    for _ in range(args.warmup):
+        s.step()
+    t0 = time.perf_counter()
+    per = [s.step() for _ in range(args.steps)]
+    wall = time.perf_counter() - t0
+    value = s.patches_per_s(float(np.mean(per)), 24)
+    cfg_out = {"workload": wl["desc"], "patches": s.T, "layers": 24}
+    line = {"metric": METRIC, "value": value, "unit": "patches/s", "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": 1000.0 * wall / max(1, args.steps), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": cfg_out,
+            "cpu_baseline": {"value": value, "unit": "patches/s", "cores": blas_threads(), "kind": "oracle",
+                             "sample": s.describe() + "; each step = one 1/16 row slice of the block"},
+            "e2e": {"value": value, "unit": "patches/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------
+# Our arm
+# ---------------------------------------------------------------------------
+
+def source_hash(*names) -> str:
+    h = hashlib.sha1()
+    for n in names:
+        with open(os.path.join(ROOT, "vision_language_model_b200", "csrc", n), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:12]
+
+
+def ncu_traffic(kernel: str) -> float | None:
+    """DRAM bytes per launch from the committed ncu summary, if it was taken
+    on the current source of that kernel."""
+    path = os.path.join(ROOT, "profiles", "traffic_per_launch.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as fh:
+        table = json.load(fh)
+    ent = table.get(kernel)
+    if not ent or ent.get("source_hash") != source_hash(*ent.get("sources", [])):
+        return None
+    return float(ent["bytes_per_launch"])
+
+
+KERNEL_SOURCES = {"attention": ["attention_mma.cu", "common.cuh", "kernels.cuh"],
+                  "gemm": ["gemm_tcgen05.cu", "common.cuh", "kernels.cuh"]}
+
+
+def run_ours(args, wl):
+    from vision_language_model_b200 import synth, vlm
+
+    world, rank, local = dist_setup()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    sizes = sizes_of(wl, args.seed)
+    cfg = vlm.preset(wl["preset"])
+    fl = flops_breakdown(cfg, sizes)
+    T, Tm = fl["T"], fl["Tm"]
+
+    tw = {k: v.to(dev) for k, v in synth.tower_weights(args.seed, cfg.layers, cfg.width, cfg.mlp, cfg.patch).items()}
+    pw = {k: v.to(dev) for k, v in synth.projector_weights(args.seed, cfg.width, cfg.merge, cfg.proj_out).items()}
+    pipe = vlm.ImagePipeline(cfg, tw, pw, sizes, device=dev)
+    del tw, pw
+    imgs = synth.images(args.seed + rank, sizes)
+    pix_host = torch.cat([im.reshape(-1) for im in imgs]).pin_memory()
+    pix = pix_host.to(dev)
+    per_seq = [[] for _ in range(wl["n_seq"])]
+    lens_m = [(h // cfg.patch) * (w // cfg.patch) // (cfg.merge * cfg.merge) for h, w in sizes]
+    for i, n in enumerate(lens_m):
+        per_seq[i % wl["n_seq"]].append(n)
+    ids_host = synth.text_sequences(args.seed, wl["n_seq"], wl["seq_len"], per_seq).reshape(-1).pin_memory()
+    ids = ids_host.to(dev)
+    text = synth.text_embeddings(args.seed, ids.numel(), cfg.proj_out).to(dev)
+    scatter_ws = torch.empty(max(256, vlm.scatter_workspace_size(ids.numel())), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        emb = pipe(pix)
+        vlm.scatter(ids, emb, text, cfg.image_token_id, workspace=scatter_ws, status=pipe.status)
+
+    for _ in range(args.warmup):
+        step()
+    rc = vlm.status_sync(pipe.status)
+    if rc != vlm.OK:
+        raise RuntimeError(f"device status after warm-up: {vlm.status_string(rc)}")
+
+    if args.profile_steps:
+        for _ in range(args.profile_steps):
+            step()
+        torch.cuda.synchronize()
+        return
+
+    # ---- timed region: inputs resident in HBM ----
+    clocks = ClockSampler(local)
+    time.sleep(0.3)
+    vlm.profile_enable(True)
+    launches0 = vlm.launch_count()
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    start.record(stream)
+    for _ in range(args.steps):
+        step()
+    stop.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    ms = start.elapsed_time(stop)
+    launches = vlm.launch_count() - launches0
+    clk = clocks.stop()
+    n_gemm, ms_gemm = vlm.profile_query("gemm")
+    n_attn, ms_attn = vlm.profile_query("attention")
+    n_norm, ms_norm = vlm.profile_query("rmsnorm")
+    vlm.profile_enable(False)
+    rc = vlm.status_sync(pipe.status)
+    if rc != vlm.OK:
+        raise RuntimeError(f"device status after timed steps: {vlm.status_string(rc)}")
+    ms_max = max_over_ranks(world, ms)
+
+    # ---- e2e: host buffers in and out every step ----
+    out_host = torch.empty(text.shape, dtype=text.dtype, pin_memory=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    e_start, e_stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e_start.record(stream)
+    for _ in range(args.steps):
+        pix.copy_(pix_host, non_blocking=True)
+        ids.copy_(ids_host, non_blocking=True)
+        step()
+        out_host.copy_(text, non_blocking=True)
+    e_stop.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    e_ms = max_over_ranks(world, e_start.elapsed_time(e_stop))
+
+    peaks = measured_peaks()
+    value = T * world * args.steps / (ms_max / 1000.0)
+    # dominant kernel of the step
+    if ms_attn >= ms_gemm:
+        kern, achieved = "attention", fl["attn_per_launch"] / (ms_attn / n_attn / 1000.0) / 1e12
+    else:
+        kern, achieved = "gemm", fl["gemm"] * args.steps / (ms_gemm / 1000.0) / 1e12
+    peak = peaks["bf16_tflops_sustained"]
+    step_tflops = fl["total"] / (ms / args.steps / 1000.0) / 1e12
+    line = {
+        "metric": METRIC, "value": value, "unit": "patches/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": wl["desc"], "patches": T, "merged_tokens": Tm, "layers": cfg.layers,
+                   "images": len(sizes), "text_tokens": int(ids.numel()), "parallelism": f"replicas{world}",
+                   "l2": "inputs larger than L2 (weights 0.88 GB + activations per step)"},
+        "roofline": {"kernel": kern, "bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": achieved / peak, "peak_source": f"bf16_tflops_sustained ({peaks['source']})",
+                     "traffic": ncu_traffic(kern)},
+        "step_tflops": step_tflops,
+        "step_frac_of_bf16_peak": {"measured_sustained": step_tflops / peak,
+                                   "measured_burst": step_tflops / peaks["bf16_tflops"],
+                                   "nominal_2250": step_tflops / 2250.0},
+        "kernels_ms_per_step": {"gemm": ms_gemm / args.steps, "attention": ms_attn / args.steps,
+                                "rmsnorm": ms_norm / args.steps},
+        "e2e": {"value": T * world * args.steps / (e_ms / 1000.0), "unit": "patches/s",
+                "h2d_bytes_per_step": int(pix_host.numel() * 4 + ids_host.numel() * 8),
+                "d2h_bytes_per_step": int(out_host.numel() * out_host.element_size())},
+        "gpu_launches": int(launches),
+        "clocks": clk,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(wl, args.seed)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def main():
+    args = parse_args()
+    wl = WORKLOADS[args.workload]
+    if args.impl == "reference":
+        run_reference(args, wl)
+    else:
+        run_ours(args, wl)
+
+
+if __name__ == "__main__":
+    main()

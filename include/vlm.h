@@ -1,0 +1,216 @@
+/*
+ * vlm.h -- C ABI of the B200 (sm_100a) image half of the Mistral 3 / Pixtral
+ * multimodal forward: vision tower, 2x2 patch-merging projector, and the
+ * masked scatter of image embeddings into the text-embedding sequence.
+ *
+ * Sources (web pages, cited by title and section):
+ *   [K] "Mistral 3" (KerasFormers): intro; API tables Mistral3Model,
+ *       Mistral3VisionModel, Mistral3ImageProcessor; "Several images in one
+ *       conversation" (one placeholder run per image).
+ *   [P] "Pixtral-12B-2409" (inference-research): vision dimensions, patch 16,
+ *       no spatial merge, 1024x1024 tiles (VISION TOKENS).
+ *   [I] vllm.cpp issue "Mistral3ForConditionalGeneration ...", section
+ *       "What we would contribute", item 2: projector plus masked-scatter merge
+ *       into the decoder, gated so text rows stay byte-identical.
+ *   [N] NeMo AutoModel mistral3_vlm, Mistral3FP8VLMForConditionalGeneration.forward:
+ *       input_ids [B, S], pixel_values, image_sizes.
+ *
+ * Conventions shared by every call:
+ *   - Every pointer named d_* or documented as "device" is CUDA device memory
+ *     owned by the caller. The library never allocates, frees or keeps device
+ *     memory and never synchronises the stream (except vlm_status_sync).
+ *     Host arrays (image_hw) are read during the call only.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *   - A negative return value means the arguments were rejected on the host and
+ *     nothing was launched. VLM_OK means the work was enqueued; errors found on
+ *     the device (a placeholder-count mismatch, a barrier wait that ran out of
+ *     its time budget) are written to the caller's int32 status word d_status
+ *     (first error wins; the library never clears it: zero it before a call
+ *     sequence) and read back with vlm_status_sync.
+ *   - Matrices are row-major. Weights use nn.Linear's [out, in] layout.
+ *     bf16 means IEEE bfloat16 with round-to-nearest-even conversions.
+ *   - Calls keep no state between them (apart from the optional profiling
+ *     counters); concurrent calls on different streams must use different
+ *     workspaces.
+ */
+#ifndef VLM_B200_H
+#define VLM_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define VLM_API __attribute__((visibility("default")))
+#else
+#define VLM_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  VLM_OK = 0,
+  VLM_ERR_INVALID_ARG = -1,    /* null pointer, bad config value */
+  VLM_ERR_BAD_SHAPE = -2,      /* image off the patch grid / merge grid, empty batch, too many tokens */
+  VLM_ERR_WORKSPACE = -3,      /* workspace or packed buffer smaller than the size function returns */
+  VLM_ERR_COUNT_MISMATCH = -4, /* device: placeholder count != number of image rows */
+  VLM_ERR_TIMEOUT = -5,        /* device: a barrier wait exceeded its time budget */
+  VLM_ERR_CUDA = -6,           /* a CUDA runtime call failed */
+  VLM_ERR_UNSUPPORTED = -7     /* shape the kernels do not implement (e.g. head_dim != 64) */
+} vlm_status;
+
+/* Hyperparameters of the vision side. [K] Mistral3Model: vision_embed_dim
+ * (width) 1024, vision_mlp_dim 4096, vision_num_layers 24, vision_num_heads 16,
+ * patch_size 14, vision_rope_theta 1e4, spatial_merge_size 2, image_token_id 10,
+ * text embed_dim 5120 (proj_out). [P]: patch 16, merge 1.
+ * eps: RMSNorm epsilon (reading: 1e-5, the only norm_eps the pages give).
+ * normalize: 1 = `pixels` hold raw [0,1] values and the processor's per-channel
+ * (x - mean)/std ([K] Mistral3ImageProcessor) is applied while gathering
+ * patches; 0 = `pixels` are already normalised. */
+typedef struct {
+  int32_t layers, width, heads, head_dim, mlp, patch, merge, proj_out, image_token_id;
+  float rope_theta, eps;
+  int32_t normalize;
+} vlm_config;
+
+/* Tower weights, device pointers, stacked over layers (L = cfg.layers,
+ * D = width, F = mlp, p = patch):
+ *   w_pe   bf16 [D, 3, p, p]  patch-embed conv weight (no bias: reading)
+ *   g_pre  fp32 [D]           ln_pre RMSNorm gain
+ *   wq, wk, wv, wo bf16 [L, D, D]
+ *   w_gate, w_up   bf16 [L, F, D]
+ *   w_down         bf16 [L, D, F]
+ *   g_attn, g_ffn  fp32 [L, D] pre-attention / pre-MLP RMSNorm gains */
+typedef struct {
+  const void* w_pe;
+  const float* g_pre;
+  const void *wq, *wk, *wv, *wo, *w_gate, *w_up, *w_down;
+  const float *g_attn, *g_ffn;
+} vlm_tower_weights;
+
+/* Projector weights, device pointers (E = proj_out, m = merge):
+ *   g_proj  fp32 [D]            RMSNorm gain, applied per patch before the merge (reading)
+ *   w_merge bf16 [D, m*m*D]     merge linear; input column c*m*m + dy*m + dx is
+ *                               channel c of patch (m*i+dy, m*j+dx) (unfold order).
+ *                               Ignored when merge == 1.
+ *   w1      bf16 [E, D]; w2 bf16 [E, E]   ([K] Mistral3Model: projector_bias False) */
+typedef struct {
+  const float* g_proj;
+  const void *w_merge, *w1, *w2;
+} vlm_projector_weights;
+
+/* Status name for a vlm_status value (static string). */
+VLM_API const char* vlm_status_string(int status);
+
+/* Synchronises `stream`, then returns *d_status (an int32 on the device).
+ * Returns VLM_ERR_CUDA if the synchronisation itself failed. */
+VLM_API int vlm_status_sync(const int32_t* d_status, void* stream);
+
+/* Presets: fills *cfg with [K]'s Mistral 3 vision values (preset 0) or [P]'s
+ * Pixtral-12B values (preset 1); normalize = 1. Returns VLM_ERR_INVALID_ARG
+ * for an unknown preset. */
+VLM_API int vlm_config_preset(int preset, vlm_config* cfg);
+
+/* ---------------------------------------------------------------------------
+ * Weight packing (one-time, exact: only copies and reorders values)
+ *
+ * The packed tower holds per layer: [wq;wk;wv] [3D, D]; wo; gate/up rows
+ * interleaved in groups of 16 [2F, D]; w_down; the two gains; plus w_pe
+ * zero-padded to [D, Kp] (Kp = 3p^2 rounded up to 64) and g_pre.
+ * The packed projector holds g_proj, w_merge with its columns reordered to
+ * patch-major (dy*m+dx)*D + c, w1, w2.
+ * Returns VLM_ERR_WORKSPACE if packed_bytes is smaller than the size function.
+ * ------------------------------------------------------------------------- */
+VLM_API size_t vlm_tower_packed_bytes(const vlm_config* cfg);
+VLM_API int vlm_pack_tower(const vlm_config* cfg, const vlm_tower_weights* w, void* d_packed,
+                   size_t packed_bytes, void* stream);
+VLM_API size_t vlm_projector_packed_bytes(const vlm_config* cfg);
+VLM_API int vlm_pack_projector(const vlm_config* cfg, const vlm_projector_weights* w, void* d_packed,
+                       size_t packed_bytes, void* stream);
+
+/* Number of patches T of a batch, or a negative vlm_status if an image is off
+ * the patch grid (H or W not a multiple of p), its patch grid is not a multiple
+ * of the merge size, or the batch is empty. image_hw is host int32 [n, 2] of
+ * (H, W) in pixels ([N] image_sizes). */
+VLM_API int64_t vlm_num_patches(const vlm_config* cfg, const int32_t* image_hw, int n_images);
+/* Number of merged tokens T_m = sum_b (h_b/m)(w_b/m), or a negative vlm_status. */
+VLM_API int64_t vlm_num_merged(const vlm_config* cfg, const int32_t* image_hw, int n_images);
+
+/* ---------------------------------------------------------------------------
+ * vlm_encode -- the vision tower ([K] Mistral3VisionModel: conv patch embed ->
+ * RMS pre-norm -> 2D-rotary blocks over a packed variable-resolution patch
+ * sequence).
+ *
+ * pixels: device fp32, the images' [3, H_b, W_b] CHW blocks concatenated in
+ *   call order, no padding. A large Pixtral image is passed as its 1024x1024
+ *   tiles, each tile one image ([P] VISION TOKENS).
+ * image_hw: host int32 [n_images, 2].
+ * d_packed_tower: output of vlm_pack_tower.
+ * d_out: device bf16 [T, width], patches concatenated image after image,
+ *   row-major within an image; the residual stream after the last block (no
+ *   final norm: reading).
+ * Attention is bidirectional within each image only; RoPE positions restart
+ *   at (0,0) in each image (reading).
+ * d_workspace: device scratch of at least vlm_encode_workspace_size bytes,
+ *   256-byte aligned. Overwritten.
+ * ------------------------------------------------------------------------- */
+VLM_API size_t vlm_encode_workspace_size(const vlm_config* cfg, const int32_t* image_hw, int n_images);
+VLM_API int vlm_encode(const vlm_config* cfg, const float* pixels, const int32_t* image_hw, int n_images,
+               const void* d_packed_tower, void* d_out, void* d_workspace, size_t ws_bytes,
+               int32_t* d_status, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * vlm_merge_project -- the patch-merging projector ([K] Mistral3Model: 2x2
+ * patch-merging projector, spatial_merge_size, projector_bias False):
+ * RMSNorm per patch, m x m unfold + concat, merge linear (m*m*D -> D), then
+ * W1 (D -> E), exact GELU, W2 (E -> E). With merge == 1 ([P]) the unfold and
+ * merge linear are skipped.
+ *
+ * d_tower_out: device bf16 [T, width] from vlm_encode with the same image_hw.
+ * d_out: device bf16 [T_m, proj_out], merged tokens row-major per image,
+ *   images concatenated.
+ * ------------------------------------------------------------------------- */
+VLM_API size_t vlm_merge_project_workspace_size(const vlm_config* cfg, const int32_t* image_hw, int n_images);
+VLM_API int vlm_merge_project(const vlm_config* cfg, const void* d_tower_out, const int32_t* image_hw,
+                      int n_images, const void* d_packed_projector, void* d_out, void* d_workspace,
+                      size_t ws_bytes, int32_t* d_status, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * vlm_scatter -- masked scatter ([I] item 2; [K] image_token_id 10 and
+ * "Several images in one conversation"): the k-th position i (in order) with
+ * input_ids[i] == image_token_id receives row k of image_embeds; all other
+ * rows of text_embeds are left untouched (bit-identical).
+ *
+ * d_input_ids: device int64 [n_tokens] ([N] input_ids [B, S], flattened).
+ * d_image_embeds: device, n_image_tokens rows of row_bytes bytes.
+ * d_text_embeds: device, n_tokens rows of row_bytes bytes, updated in place.
+ * row_bytes: bytes per row (e.g. 5120 * 2 for bf16), a multiple of 16.
+ * If the number of placeholders differs from n_image_tokens the call writes
+ *   no row and sets *d_status = VLM_ERR_COUNT_MISMATCH.
+ * d_workspace: at least vlm_scatter_workspace_size(n_tokens) bytes.
+ * ------------------------------------------------------------------------- */
+VLM_API size_t vlm_scatter_workspace_size(int64_t n_tokens);
+VLM_API int vlm_scatter(const int64_t* d_input_ids, int64_t n_tokens, int64_t image_token_id,
+                const void* d_image_embeds, int64_t n_image_tokens, void* d_text_embeds,
+                int64_t row_bytes, void* d_workspace, size_t ws_bytes, int32_t* d_status,
+                void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Instrumentation (host-side, not thread-safe)
+ * ------------------------------------------------------------------------- */
+/* Total kernels this library has launched in the process. */
+VLM_API int64_t vlm_launch_count(void);
+/* Turns per-kernel CUDA-event timing on (1) or off (0) and clears it. */
+VLM_API int vlm_profile_enable(int on);
+/* Kernel classes: 0 GEMM, 1 attention, 2 RMSNorm, 3 patch gather, 4 merge
+ * gather, 5 scatter, 6 index setup, 7 weight packing. Synchronises on the last
+ * recorded event, then returns the launches and summed device milliseconds
+ * recorded for `kclass` since profiling was enabled. */
+VLM_API int vlm_profile_query(int kclass, int64_t* launches, double* total_ms);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* VLM_B200_H */

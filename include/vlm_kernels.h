@@ -1,0 +1,90 @@
+/*
+ * vlm_kernels.h -- per-kernel entry points of the B200 image-half library.
+ *
+ * vlm_encode / vlm_merge_project / vlm_scatter (vlm.h) chain these kernels;
+ * they are exported on their own so each can be checked against the CPU
+ * oracle at full size. Conventions (ownership, status word, streams, error
+ * returns) are those of vlm.h. Page citations use the same keys:
+ * [K] "Mistral 3" (KerasFormers), [P] "Pixtral-12B-2409".
+ */
+#ifndef VLM_B200_KERNELS_H
+#define VLM_B200_KERNELS_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#include "vlm.h"
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Epilogues of vlm_gemm (what is done with the fp32 accumulator acc[M, N]):
+ *   BF16   c = bf16(acc)                                  c: bf16 [M, N]
+ *   F32    c = acc                                        c: fp32 [M, N]
+ *   RESID  c += acc (fp32 residual update in place);      c: fp32 [M, N]
+ *          if c_bf16 != NULL also c_bf16 = bf16(new c)    c_bf16: bf16 [M, N]
+ *   SWIGLU with B rows interleaved in groups of 16 (rows 32j..32j+15 gate
+ *          rows 16j.., rows 32j+16..32j+31 up rows 16j..):
+ *          c[:, 16j+i] = bf16(silu(acc[:, 32j+i]) * acc[:, 32j+16+i]),
+ *          silu(z) = z / (1 + e^-z)                       c: bf16 [M, N/2]
+ *          (the gated-SiLU MLP's first half; [K]/[P] give its width 4096)
+ *   ROPE   c = bf16(acc) after rotating, in columns [0, rope_cols), each
+ *          64-column head's pairs (i, i+32) by the angle table entry of the
+ *          row's position: pairs i < 16 use the patch row r, pairs i >= 16
+ *          the patch column c ([K] Mistral3VisionModel "2D-rotary")
+ *                                                          c: bf16 [M, N]
+ *          d_pos: int32 [M] = (r << 16) | c; d_rope_table: from vlm_rope_table
+ *   GELU   c = bf16(gelu(acc)), gelu(z) = z (1 + erf(z / sqrt 2)) / 2
+ *                                                          c: bf16 [M, N]
+ */
+enum {
+  VLM_EPI_BF16 = 0,
+  VLM_EPI_F32 = 1,
+  VLM_EPI_RESID = 2,
+  VLM_EPI_SWIGLU = 3,
+  VLM_EPI_ROPE = 4,
+  VLM_EPI_GELU = 5
+};
+
+/* acc = A . B^T on the sm_100a tensor cores (tcgen05.mma kind::f16, fp32
+ * accumulation in TMEM, operands staged by TMA), followed by `epilogue`.
+ * A: device bf16 [M, K]; B: device bf16 [N, K]; both row-major, 16-byte
+ * aligned. Requires K % 64 == 0, N % 128 == 0 (N % 256 == 0 for SWIGLU and
+ * ROPE), M >= 1. Returns VLM_ERR_UNSUPPORTED otherwise. */
+VLM_API int vlm_gemm(int epilogue, const void* d_a, const void* d_b, int64_t M, int64_t N, int64_t K,
+             void* d_c, void* d_c_bf16, const int32_t* d_pos, const void* d_rope_table,
+             int64_t rope_cols, int32_t* d_status, void* stream);
+
+/* 2D RoPE angle table ([K] vision_rope_theta): entry [p][i] (float2 cos, sin)
+ * of the angle p * w, w = theta^(-2k/head_dim) with k = 2i for i < head_dim/4
+ * (row frequencies) and k = 2(i - head_dim/4) + 1 otherwise (column
+ * frequencies). d_table: device float2 [max_pos, head_dim/2]. */
+VLM_API int vlm_rope_table(float theta, int head_dim, int max_pos, void* d_table, void* stream);
+
+/* Block-diagonal bidirectional attention over a packed sequence:
+ * out[t, h*64:(h+1)*64] = softmax_u(q_t . k_u / 8) v_u over the keys u of
+ * t's own block [cu[b], cu[b+1]) only ([K] Mistral3VisionModel, packed
+ * variable-resolution sequence; one block per image or per [P] tile).
+ * d_qkv: device bf16 [T, 3 * heads * 64] with q, k, v column blocks (RoPE
+ * already applied). cu_seqlens: HOST int32 [n_blocks + 1], cu[0] = 0,
+ * cu[n_blocks] = T, non-decreasing. d_out: device bf16 [T, heads * 64].
+ * head_dim must be 64. */
+VLM_API size_t vlm_attention_workspace_size(int n_blocks);
+VLM_API int vlm_attention(const void* d_qkv, int64_t T, int heads, int head_dim, const int32_t* cu_seqlens,
+                  int n_blocks, void* d_out, void* d_workspace, size_t ws_bytes, int32_t* d_status,
+                  void* stream);
+
+/* RMSNorm over rows of width `width` (a multiple of 128, <= 2048):
+ * y = x / sqrt(mean(x^2) + eps) * g. If d_g0 != NULL the row is first
+ * normalised with gain g0 and written back to d_x (fp32, in place), and the
+ * bf16 output is the RMSNorm of that result with gain g1; otherwise
+ * d_out = bf16(rmsnorm(x) * g1). d_x: fp32 [rows, width]. */
+VLM_API int vlm_rmsnorm(float* d_x, const float* d_g0, const float* d_g1, void* d_out, int64_t rows,
+                int width, float eps, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* VLM_B200_KERNELS_H */

@@ -279,6 +279,34 @@ def tower_block(x: np.ndarray, lw: dict, angles: np.ndarray, cu_seqlens, cfg: di
     return x + hidden @ lw["w_down"].T
 
 
+def block_keys_values(x: np.ndarray, lw: dict, angles: np.ndarray, cfg: dict) -> tuple:
+    """The part of tower_block shared by every query row: the attention-norm
+    input of all rows and their rotated keys and values ([T, heads, head_dim])."""
+    t_total = x.shape[0]
+    heads, dh = cfg["heads"], cfg["head_dim"]
+    xn = rms_norm(x, lw["g_attn"], cfg["eps"])
+    k = apply_rope((xn @ lw["wk"].T).reshape(t_total, heads, dh), angles)
+    v = (xn @ lw["wv"].T).reshape(t_total, heads, dh)
+    return xn, k, v
+
+
+def tower_block_rows(x: np.ndarray, lw: dict, angles: np.ndarray, cu_seqlens, cfg: dict, rows,
+                     kv: tuple | None = None) -> np.ndarray:
+    """tower_block() evaluated for the listed rows only: every step of the block
+    is row-wise except attention, whose keys and values come from all rows of
+    the row's block (pass `kv` from block_keys_values to reuse them)."""
+    rows = np.asarray(rows)
+    heads, dh, eps = cfg["heads"], cfg["head_dim"], cfg["eps"]
+    xn, k, v = block_keys_values(x, lw, angles, cfg) if kv is None else kv
+    q = apply_rope((xn[rows] @ lw["wq"].T).reshape(len(rows), heads, dh), angles[rows])
+    qfull = np.zeros((x.shape[0], heads, dh))
+    qfull[rows] = q
+    xr = x[rows] + attention_rows(qfull, k, v, cu_seqlens, rows) @ lw["wo"].T
+    xrn = rms_norm(xr, lw["g_ffn"], eps)
+    hidden = silu(xrn @ lw["w_gate"].T) * (xrn @ lw["w_up"].T)
+    return xr + hidden @ lw["w_down"].T
+
+
 def layer_weights(tw: dict, layer: int) -> dict:
     names = ("wq", "wk", "wv", "wo", "w_gate", "w_up", "w_down", "g_attn", "g_ffn")
     return {n: np.asarray(tw[n][layer], dtype=np.float64) for n in names}

@@ -1,0 +1,120 @@
+"""Host-side checks of the C-ABI library (no GPU needed).
+
+The library must load, export every function that include/*.h declares, and
+reject bad arguments on the host before launching anything.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+from vision_language_model_b200 import vlm
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", fn)).read()
+            names |= set(re.findall(r"VLM_API\s+[\w\s\*]+?\b(vlm_\w+)\s*\(", text))
+    return names
+
+
+@pytest.fixture(scope="module")
+def L():
+    if not os.path.exists(vlm.lib_path()):
+        from vision_language_model_b200 import build
+        build.build()
+    return vlm.lib()
+
+
+def test_every_declared_symbol_is_exported(L):
+    names = _declared()
+    assert {"vlm_encode", "vlm_merge_project", "vlm_scatter", "vlm_gemm", "vlm_attention"} <= names
+    for n in sorted(names):
+        assert hasattr(L, n), n
+
+
+def test_presets_match_pages(L):
+    m = vlm.preset("mistral3")
+    assert (m.layers, m.width, m.heads, m.head_dim, m.mlp, m.patch, m.merge, m.proj_out, m.image_token_id) == \
+        (24, 1024, 16, 64, 4096, 14, 2, 5120, 10)
+    assert m.rope_theta == 10000.0 and abs(m.eps - 1e-5) < 1e-12
+    p = vlm.preset("pixtral12b")
+    assert (p.patch, p.merge) == (16, 1)
+
+
+def test_patch_and_merged_counts(L):
+    m = vlm.preset("mistral3")
+    assert vlm.num_patches(m, [(1540, 1540)]) == 12100
+    assert vlm.num_merged(m, [(1540, 1540)]) == 3025
+    assert vlm.num_patches(m, [(896, 1344)] * 4) == 4 * 6144
+    assert vlm.num_merged(m, [(896, 1344)] * 4) == 4 * 1536
+    p = vlm.preset("pixtral12b")
+    assert vlm.num_patches(p, [(1024, 1024)] * 16) == 65536
+    assert vlm.num_merged(p, [(1024, 1024)] * 16) == 65536
+
+
+@pytest.mark.parametrize("hw", [[(225, 224)], [(14 * 3, 28)], []])
+def test_bad_shapes_rejected_on_host(L, hw):
+    m = vlm.preset("mistral3")
+    with pytest.raises(vlm.VlmError) as e:
+        vlm.num_patches(m, hw)
+    assert e.value.rc == vlm.ERR_BAD_SHAPE
+
+
+def test_unsupported_config_rejected(L):
+    with pytest.raises(vlm.VlmError) as e:
+        vlm.num_patches(vlm.preset("mistral3", head_dim=128, heads=8), [(28, 28)])
+    assert e.value.rc == vlm.ERR_UNSUPPORTED
+    assert L.vlm_tower_packed_bytes(ctypes.byref(vlm.preset("mistral3", width=1000))) == 0
+
+
+def test_workspace_sizes_cover_buffers(L):
+    m = vlm.preset("mistral3")
+    ws = vlm.encode_workspace_size(m, [(1540, 1540)])
+    T, D, F = 12100, 1024, 4096
+    assert ws >= T * D * 4 + T * D * 2 * 2 + T * 3 * D * 2 + T * F * 2
+    assert vlm.merge_project_workspace_size(m, [(1540, 1540)]) >= 3025 * 5120 * 2
+    assert vlm.scatter_workspace_size(16384) >= 16384 * 8
+
+
+def test_scatter_argument_errors_return_before_launch(L):
+    null = None
+    # row_bytes not a multiple of 16
+    rc = L.vlm_scatter(null, 4, 10, null, 0, null, 10, null, 0, null, null)
+    assert rc == vlm.ERR_INVALID_ARG
+    # empty id list with image rows
+    rc = L.vlm_scatter(null, 0, 10, null, 3, null, 16, null, 0, null, null)
+    assert rc == vlm.ERR_BAD_SHAPE
+    # null pointers
+    rc = L.vlm_scatter(null, 4, 10, null, 1, null, 16, null, 1 << 20, null, null)
+    assert rc == vlm.ERR_INVALID_ARG
+
+
+def test_status_strings(L):
+    assert vlm.status_string(vlm.ERR_COUNT_MISMATCH) == "VLM_ERR_COUNT_MISMATCH"
+    assert vlm.status_string(vlm.ERR_TIMEOUT) == "VLM_ERR_TIMEOUT"
+    assert vlm.status_string(123) == "VLM_ERR_UNKNOWN"
+
+
+def test_gemm_shape_checks_return_before_launch(L):
+    fake = ctypes.c_void_p(256)
+    st = None
+    assert L.vlm_gemm(0, fake, fake, 128, 100, 64, fake, None, None, None, 0, st, None) == vlm.ERR_UNSUPPORTED
+    assert L.vlm_gemm(0, fake, fake, 128, 128, 60, fake, None, None, None, 0, st, None) == vlm.ERR_UNSUPPORTED
+    assert L.vlm_gemm(3, fake, fake, 128, 384, 64, fake, None, None, None, 0, st, None) == vlm.ERR_UNSUPPORTED
+    assert L.vlm_gemm(0, None, fake, 128, 128, 64, fake, None, None, None, 0, st, None) == vlm.ERR_INVALID_ARG
+    assert L.vlm_gemm(0, fake, fake, 0, 128, 64, fake, None, None, None, 0, st, None) == vlm.ERR_BAD_SHAPE
+
+
+def test_package_import_does_not_load_library():
+    import importlib
+    import sys
+    for k in [k for k in sys.modules if k.startswith("vision_language_model_b200")]:
+        sys.modules.pop(k)
+    pkg = importlib.import_module("vision_language_model_b200")
+    assert not hasattr(pkg, "_lib")

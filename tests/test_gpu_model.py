@@ -1,0 +1,132 @@
+"""End-to-end parity of vlm_encode / vlm_merge_project / vlm_scatter with the
+CPU oracle, plus the invariants that hold at any size (block isolation,
+packed == separate, determinism) checked at full size.
+"""
+import numpy as np
+import pytest
+import torch
+
+from oracle import vlm_oracle as O
+from tests.gpu_util import compare, pixels_to_device, to_np, to_oracle, tower_to_device
+from vision_language_model_b200 import synth, vlm
+
+pytestmark = pytest.mark.gpu
+
+
+def _setup(preset, layers, sizes, seed=0, qk_scale=1.0):
+    cfg = vlm.preset(preset, layers=layers)
+    tw = synth.tower_weights(seed, layers, cfg.width, cfg.mlp, cfg.patch, qk_scale=qk_scale)
+    pw = synth.projector_weights(seed, cfg.width, cfg.merge, cfg.proj_out)
+    imgs = synth.images(seed, sizes)
+    return cfg, tw, pw, imgs
+
+
+def _run_gpu(cfg, tw, pw, imgs, sizes):
+    pipe = vlm.ImagePipeline(cfg, tower_to_device(tw), tower_to_device(pw), sizes)
+    emb = pipe(pixels_to_device(imgs))
+    assert vlm.status_sync(pipe.status) == vlm.OK
+    return pipe.tower_out.clone(), emb.clone()
+
+
+def _oracle_cfg(cfg):
+    d = dict(O.MISTRAL3 if cfg.merge == 2 else O.PIXTRAL12B)
+    d.update(layers=cfg.layers, patch=cfg.patch, merge=cfg.merge)
+    return d
+
+
+def _run_oracle(cfg, tw, pw, imgs):
+    ocfg = _oracle_cfg(cfg)
+    return O.encode_merge_project([im.double().numpy() for im in imgs], to_oracle(tw), to_oracle(pw), ocfg)
+
+
+CASES = [
+    ("tiny_224", "mistral3", 2, [(224, 224)], 1.0),
+    ("packed3", "mistral3", 2, [(84, 140), (28, 28), (112, 56)], 1.0),
+    ("packed3_peaked", "mistral3", 2, [(84, 140), (28, 28), (112, 56)], 8.0),
+    ("pixtral_2tiles", "pixtral12b", 2, [(128, 128), (128, 128)], 1.0),
+    ("deep24_112", "mistral3", 24, [(112, 140)], 1.0),
+]
+
+
+@pytest.mark.parametrize("name,preset,layers,sizes,qk", CASES, ids=[c[0] for c in CASES])
+def test_encode_merge_project_vs_oracle(name, preset, layers, sizes, qk):
+    cfg, tw, pw, imgs = _setup(preset, layers, sizes, qk_scale=qk)
+    tower, emb = _run_gpu(cfg, tw, pw, imgs, sizes)
+    ref_tower, ref_emb = _run_oracle(cfg, tw, pw, imgs)
+    compare(tower, ref_tower, what=f"{name} tower")
+    compare(emb, ref_emb, what=f"{name} projector")
+
+
+def test_gpu_block_isolation_and_packed_equals_separate():
+    sizes = [(84, 140), (56, 56), (112, 84)]
+    cfg, tw, pw, imgs = _setup("mistral3", 2, sizes, seed=3)
+    tower, emb = _run_gpu(cfg, tw, pw, imgs, sizes)
+    # perturb image 1 only
+    imgs2 = [im.clone() for im in imgs]
+    imgs2[1] = (imgs2[1] + 0.25).clamp(0, 1)
+    tower2, emb2 = _run_gpu(cfg, tw, pw, imgs2, sizes)
+    n0 = (84 // 14) * (140 // 14)
+    n1 = (56 // 14) ** 2
+    assert torch.equal(tower2[:n0], tower[:n0]) and torch.equal(tower2[n0 + n1:], tower[n0 + n1:])
+    assert not torch.equal(tower2[n0:n0 + n1], tower[n0:n0 + n1])
+    m0, m1 = n0 // 4, n1 // 4
+    assert torch.equal(emb2[:m0], emb[:m0]) and torch.equal(emb2[m0 + m1:], emb[m0 + m1:])
+    # packed == separate, bit for bit
+    outs = [_run_gpu(cfg, tw, pw, [im], [hw]) for im, hw in zip(imgs, sizes)]
+    assert torch.equal(torch.cat([o[0] for o in outs]), tower)
+    assert torch.equal(torch.cat([o[1] for o in outs]), emb)
+
+
+def test_full_size_1540_deterministic_and_finite():
+    """The 24-layer tower on one 1540x1540 image, as the bench runs it."""
+    sizes = [(1540, 1540)]
+    cfg, tw, pw, imgs = _setup("mistral3", 24, sizes, seed=0)
+    pipe = vlm.ImagePipeline(cfg, tower_to_device(tw), tower_to_device(pw), sizes)
+    pix = pixels_to_device(imgs)
+    e1 = pipe(pix).clone()
+    t1 = pipe.tower_out.clone()
+    e2 = pipe(pix).clone()
+    assert vlm.status_sync(pipe.status) == vlm.OK
+    assert e1.shape == (3025, 5120) and t1.shape == (12100, 1024)
+    assert torch.isfinite(e1.float()).all() and torch.isfinite(t1.float()).all()
+    assert torch.equal(e1, e2) and torch.equal(t1, pipe.tower_out)
+    # the output depends on the input: a different image gives different embeddings
+    e3 = pipe(pixels_to_device(synth.images(1, sizes))).clone()
+    assert not torch.equal(e1, e3)
+
+
+def test_full_size_packed_batch_isolation():
+    """Packed variable-resolution batch of 8 images (sides 28*U{10..55}), 24 layers."""
+    sizes = synth.packed_sizes(0, 8)
+    cfg, tw, pw, imgs = _setup("mistral3", 24, sizes, seed=0)
+    pipe = vlm.ImagePipeline(cfg, tower_to_device(tw), tower_to_device(pw), sizes)
+    e1 = pipe(pixels_to_device(imgs)).clone()
+    imgs2 = [im.clone() for im in imgs]
+    imgs2[3] = imgs2[3].flip(-1).contiguous()
+    e2 = pipe(pixels_to_device(imgs2)).clone()
+    assert vlm.status_sync(pipe.status) == vlm.OK
+    m = [(h // 28) * (w // 28) for h, w in sizes]
+    off = np.concatenate([[0], np.cumsum(m)])
+    for b in range(8):
+        same = torch.equal(e1[off[b]:off[b + 1]], e2[off[b]:off[b + 1]])
+        assert same == (b != 3), b
+
+
+def test_encode_then_scatter_end_to_end():
+    """4 sequences x 4,096 ids, one 896x1344 image each (1,536 placeholders), 2 layers."""
+    sizes = [(896, 1344)] * 4
+    cfg, tw, pw, imgs = _setup("mistral3", 2, sizes, seed=5)
+    tower, emb = _run_gpu(cfg, tw, pw, imgs, sizes)
+    ids = synth.text_sequences(5, 4, 4096, [[1536]] * 4)
+    text = synth.text_embeddings(5, 4 * 4096, 5120)
+    t_gpu = text.cuda()
+    status = vlm.new_status()
+    vlm.scatter(ids.reshape(-1).cuda(), emb, t_gpu, 10, status=status)
+    assert vlm.status_sync(status) == vlm.OK
+    mask = (ids.reshape(-1) == 10).cuda()
+    # non-image rows bit-identical, image rows are exactly the embeddings in order
+    assert torch.equal(t_gpu[~mask].cpu().view(torch.int16), text[~mask.cpu()].view(torch.int16))
+    assert torch.equal(t_gpu[mask], emb)
+    # and the embeddings themselves match the oracle on one of the four images
+    ref_tower, ref_emb = _run_oracle(cfg, tw, pw, imgs[:1])
+    compare(emb[:1536], ref_emb, what="e2e projector image 0")

@@ -242,6 +242,21 @@ def test_mlp_with_zero_up_is_identity_block_on_ffn_half():
     np.testing.assert_array_equal(y, x)
 
 
+def test_block_rows_equals_full_block_on_those_rows():
+    cfg, tw = _tiny_tower(layers=1, heads=1)
+    cfg["head_dim"] = 64
+    lw = O.layer_weights(tw, 0)
+    grids = [(3, 4), (2, 2)]
+    rows_, cols_, cu = O.positions(grids)
+    ang = O.rope_angles(rows_, cols_, 1e4, 64)
+    x = RNG.standard_normal((16, 64))
+    full = O.tower_block(x, lw, ang, cu, cfg)
+    sel = [0, 5, 11, 12, 15]
+    np.testing.assert_allclose(O.tower_block_rows(x, lw, ang, cu, cfg, sel), full[sel], rtol=1e-12, atol=1e-12)
+    kv = O.block_keys_values(x, lw, ang, cfg)
+    np.testing.assert_allclose(O.tower_block_rows(x, lw, ang, cu, cfg, [3], kv=kv), full[[3]], rtol=1e-12)
+
+
 # ---------------------------------------------------------------------------
 # Tower-level invariants: isolation and packing
 # ---------------------------------------------------------------------------

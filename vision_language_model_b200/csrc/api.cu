@@ -1,0 +1,626 @@
+// C-ABI layer: argument validation, workspace layout, and the kernel chains of
+// vlm_encode / vlm_merge_project / vlm_scatter (declared in include/vlm.h and
+// include/vlm_kernels.h).
+#include <algorithm>
+#include <atomic>
+#include <vector>
+
+#include "../../include/vlm_kernels.h"
+#include "kernels.cuh"
+
+namespace vlm {
+
+// ---------------------------------------------------------------------------
+// Launch bookkeeping and optional per-kernel event timing
+// ---------------------------------------------------------------------------
+namespace {
+std::atomic<int64_t> g_launches{0};
+bool g_profile = false;
+struct EventRec { int kclass; cudaEvent_t start, stop; };
+std::vector<EventRec> g_records;
+std::vector<cudaEvent_t> g_pool;
+cudaEvent_t g_pending_start = nullptr;
+
+cudaEvent_t take_event() {
+  if (!g_pool.empty()) {
+    cudaEvent_t e = g_pool.back();
+    g_pool.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  cudaEventCreate(&e);
+  return e;
+}
+}  // namespace
+
+void launch_begin(int kclass, cudaStream_t s) {
+  (void)kclass;
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  if (g_profile) {
+    g_pending_start = take_event();
+    cudaEventRecord(g_pending_start, s);
+  }
+}
+
+void launch_end(int kclass, cudaStream_t s) {
+  if (g_profile && g_pending_start != nullptr) {
+    cudaEvent_t stop = take_event();
+    cudaEventRecord(stop, s);
+    g_records.push_back({kclass, g_pending_start, stop});
+    g_pending_start = nullptr;
+  }
+}
+
+void note_extra_launches(int n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
+
+int num_sms() {
+  static int cache[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 64) dev = 63;
+  if (cache[dev] == 0) {
+    int n = 0;
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    cache[dev] = n > 0 ? n : 148;
+  }
+  return cache[dev];
+}
+
+namespace {
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Bump allocator over a caller-provided workspace (sizes only when base == nullptr).
+struct Carver {
+  uint8_t* base;
+  size_t used = 0;
+  explicit Carver(void* b) : base(static_cast<uint8_t*>(b)) {}
+  template <typename T>
+  T* take(size_t count) {
+    used = align_up(used, 256);
+    T* p = base ? reinterpret_cast<T*>(base + used) : nullptr;
+    used += count * sizeof(T);
+    return p;
+  }
+};
+
+int check_config(const vlm_config* c) {
+  if (c == nullptr) return VLM_ERR_INVALID_ARG;
+  if (c->layers < 0 || c->width <= 0 || c->heads <= 0 || c->head_dim <= 0 || c->mlp <= 0 || c->patch <= 0 ||
+      c->merge <= 0 || c->proj_out <= 0 || !(c->rope_theta > 0.f) || !(c->eps >= 0.f))
+    return VLM_ERR_INVALID_ARG;
+  if (c->head_dim != 64 || c->heads * c->head_dim != c->width) return VLM_ERR_UNSUPPORTED;
+  if (c->width % 256 || c->width > 2048 || c->mlp % 128 || c->proj_out % 256) return VLM_ERR_UNSUPPORTED;
+  if (c->patch > 64) return VLM_ERR_UNSUPPORTED;
+  return VLM_OK;
+}
+
+inline int64_t kpad(int p) { return align_up(static_cast<size_t>(3 * p * p), 64); }
+
+// Host-side per-image tables of a batch.
+struct Batch {
+  int n = 0;
+  int64_t T = 0, Tm = 0;
+  int total_qtiles = 0;
+  int max_pos = 0;
+  std::vector<int32_t> h, w, H, W, tok_off, m_off, qt_off;
+  std::vector<int64_t> pix_off;
+};
+
+int make_batch(const vlm_config* c, const int32_t* hw, int n, Batch* b) {
+  if (hw == nullptr || n <= 0) return VLM_ERR_BAD_SHAPE;
+  b->n = n;
+  b->h.resize(n); b->w.resize(n); b->H.resize(n); b->W.resize(n);
+  b->tok_off.resize(n + 1); b->m_off.resize(n + 1); b->qt_off.resize(n + 1); b->pix_off.resize(n);
+  int64_t t = 0, tm = 0, qt = 0, pix = 0;
+  int maxp = 1;
+  for (int i = 0; i < n; ++i) {
+    const int Hh = hw[2 * i], Ww = hw[2 * i + 1];
+    if (Hh <= 0 || Ww <= 0 || Hh % c->patch || Ww % c->patch) return VLM_ERR_BAD_SHAPE;
+    const int hp = Hh / c->patch, wp = Ww / c->patch;
+    if (hp % c->merge || wp % c->merge) return VLM_ERR_BAD_SHAPE;
+    if (hp >= 32768 || wp >= 32768) return VLM_ERR_BAD_SHAPE;
+    b->H[i] = Hh; b->W[i] = Ww; b->h[i] = hp; b->w[i] = wp;
+    b->tok_off[i] = static_cast<int32_t>(t);
+    b->m_off[i] = static_cast<int32_t>(tm);
+    b->qt_off[i] = static_cast<int32_t>(qt);
+    b->pix_off[i] = pix;
+    const int64_t L = static_cast<int64_t>(hp) * wp;
+    t += L;
+    tm += L / (c->merge * c->merge);
+    qt += (L + kAttnBQ - 1) / kAttnBQ;
+    pix += 3LL * Hh * Ww;
+    maxp = std::max(maxp, std::max(hp, wp));
+    if (t > (1LL << 31) - 1 || qt > (1LL << 31) - 1) return VLM_ERR_BAD_SHAPE;
+  }
+  b->tok_off[n] = static_cast<int32_t>(t);
+  b->m_off[n] = static_cast<int32_t>(tm);
+  b->qt_off[n] = static_cast<int32_t>(qt);
+  b->T = t;
+  b->Tm = tm;
+  b->total_qtiles = static_cast<int>(qt);
+  b->max_pos = maxp;
+  return VLM_OK;
+}
+
+// Device tables of a batch, carved from a workspace.
+struct BatchDev {
+  ImgInfo* info;
+  int32_t* cu;
+  int32_t* qt;
+  int32_t* pos;
+  float2* rope;
+};
+
+BatchDev carve_batch(Carver& cv, const Batch& b, bool with_pos, int head_dim) {
+  BatchDev d;
+  d.info = cv.take<ImgInfo>(b.n);
+  d.cu = cv.take<int32_t>(b.n + 1);
+  d.qt = cv.take<int32_t>(b.n + 1);
+  d.pos = with_pos ? cv.take<int32_t>(b.T) : nullptr;
+  d.rope = with_pos ? cv.take<float2>(static_cast<size_t>(b.max_pos) * head_dim / 2) : nullptr;
+  return d;
+}
+
+int upload_batch(const Batch& b, const BatchDev& d, cudaStream_t s) {
+  for (int first = 0; first < b.n; first += kChunk) {
+    ImageChunk ch;
+    ch.first = first;
+    ch.count = std::min(kChunk, b.n - first);
+    for (int i = 0; i < ch.count; ++i) {
+      ch.h[i] = b.h[first + i]; ch.w[i] = b.w[first + i];
+      ch.H[i] = b.H[first + i]; ch.W[i] = b.W[first + i];
+      ch.tok_off[i] = b.tok_off[first + i];
+      ch.m_off[i] = b.m_off[first + i];
+      ch.qt_off[i] = b.qt_off[first + i];
+      ch.pix_off[i] = b.pix_off[first + i];
+    }
+    ch.tok_off[ch.count] = b.tok_off[first + ch.count];
+    ch.m_off[ch.count] = b.m_off[first + ch.count];
+    ch.qt_off[ch.count] = b.qt_off[first + ch.count];
+    const int rc = launch_setup(ch, d.info, d.cu, d.qt, d.pos, b.n, s);
+    if (rc != VLM_OK) return rc;
+  }
+  return VLM_OK;
+}
+
+// Packed tower layout (byte offsets).
+struct TowerLayout {
+  size_t w_pe, g_pre, layer0, layer_stride;
+  size_t wqkv, wo, wgu, wdown, g_attn, g_ffn;  // offsets inside a layer
+  size_t total;
+};
+
+TowerLayout tower_layout(const vlm_config* c) {
+  TowerLayout L;
+  const size_t D = c->width, F = c->mlp;
+  size_t off = 0;
+  L.w_pe = off; off = align_up(off + D * kpad(c->patch) * 2, 256);
+  L.g_pre = off; off = align_up(off + D * 4, 256);
+  L.layer0 = off;
+  size_t lo = 0;
+  L.wqkv = lo; lo = align_up(lo + 3 * D * D * 2, 256);
+  L.wo = lo; lo = align_up(lo + D * D * 2, 256);
+  L.wgu = lo; lo = align_up(lo + 2 * F * D * 2, 256);
+  L.wdown = lo; lo = align_up(lo + D * F * 2, 256);
+  L.g_attn = lo; lo = align_up(lo + D * 4, 256);
+  L.g_ffn = lo; lo = align_up(lo + D * 4, 256);
+  L.layer_stride = lo;
+  L.total = off + lo * static_cast<size_t>(c->layers);
+  return L;
+}
+
+struct ProjLayout { size_t g_proj, w_merge, w1, w2, total; };
+
+ProjLayout proj_layout(const vlm_config* c) {
+  ProjLayout L;
+  const size_t D = c->width, E = c->proj_out, mm = static_cast<size_t>(c->merge) * c->merge;
+  size_t off = 0;
+  L.g_proj = off; off = align_up(off + D * 4, 256);
+  L.w_merge = off; off = align_up(off + (c->merge > 1 ? D * mm * D * 2 : 0), 256);
+  L.w1 = off; off = align_up(off + E * D * 2, 256);
+  L.w2 = off; off = align_up(off + E * E * 2, 256);
+  L.total = off;
+  return L;
+}
+
+// Encode workspace layout.
+struct EncodeWs {
+  BatchDev bd;
+  float* x;
+  __nv_bfloat16 *xn, *qkv, *attn, *hbuf, *cols;
+  size_t used;
+};
+
+EncodeWs carve_encode(void* ws, const vlm_config* c, const Batch& b) {
+  Carver cv(ws);
+  EncodeWs e;
+  e.bd = carve_batch(cv, b, true, c->head_dim);
+  const size_t T = b.T, D = c->width, F = c->mlp;
+  e.x = cv.take<float>(T * D);
+  e.xn = cv.take<__nv_bfloat16>(T * D);
+  e.qkv = cv.take<__nv_bfloat16>(T * 3 * D);
+  e.attn = cv.take<__nv_bfloat16>(T * D);
+  const size_t hsz = std::max(T * F, T * static_cast<size_t>(kpad(c->patch)));
+  e.hbuf = cv.take<__nv_bfloat16>(hsz);
+  e.cols = e.hbuf;  // the patch gather is consumed before the first MLP
+  e.used = align_up(cv.used, 256);
+  return e;
+}
+
+struct ProjWs {
+  BatchDev bd;
+  __nv_bfloat16 *z, *y, *g;
+  size_t used;
+};
+
+ProjWs carve_proj(void* ws, const vlm_config* c, const Batch& b) {
+  Carver cv(ws);
+  ProjWs p;
+  p.bd = carve_batch(cv, b, false, c->head_dim);
+  const size_t D = c->width, E = c->proj_out;
+  p.z = cv.take<__nv_bfloat16>(b.T * D);  // [T_m, m*m*D] == [T, D] elements
+  p.y = c->merge > 1 ? cv.take<__nv_bfloat16>(b.Tm * D) : nullptr;
+  p.g = cv.take<__nv_bfloat16>(b.Tm * E);
+  p.used = align_up(cv.used, 256);
+  return p;
+}
+
+ScatterWs carve_scatter(void* ws, int64_t n_tokens, size_t* used) {
+  Carver cv(ws);
+  const int64_t n_chunks = (n_tokens + 255) / 256;
+  ScatterWs s;
+  s.ok_flag = cv.take<int32_t>(1);
+  s.chunk_count = cv.take<int32_t>(n_chunks);
+  s.chunk_base = cv.take<int64_t>(n_chunks);
+  s.dst_rows = cv.take<int64_t>(n_tokens);
+  if (used) *used = align_up(cv.used, 256);
+  return s;
+}
+
+inline cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
+
+#define VLM_TRY(expr)             \
+  do {                            \
+    const int _rc = (expr);       \
+    if (_rc != VLM_OK) return _rc; \
+  } while (0)
+
+}  // namespace
+}  // namespace vlm
+
+using namespace vlm;
+
+extern "C" {
+
+const char* vlm_status_string(int status) {
+  switch (status) {
+    case VLM_OK: return "VLM_OK";
+    case VLM_ERR_INVALID_ARG: return "VLM_ERR_INVALID_ARG";
+    case VLM_ERR_BAD_SHAPE: return "VLM_ERR_BAD_SHAPE";
+    case VLM_ERR_WORKSPACE: return "VLM_ERR_WORKSPACE";
+    case VLM_ERR_COUNT_MISMATCH: return "VLM_ERR_COUNT_MISMATCH";
+    case VLM_ERR_TIMEOUT: return "VLM_ERR_TIMEOUT";
+    case VLM_ERR_CUDA: return "VLM_ERR_CUDA";
+    case VLM_ERR_UNSUPPORTED: return "VLM_ERR_UNSUPPORTED";
+    default: return "VLM_ERR_UNKNOWN";
+  }
+}
+
+int vlm_status_sync(const int32_t* d_status, void* stream) {
+  if (d_status == nullptr) return VLM_ERR_INVALID_ARG;
+  int32_t h = 0;
+  if (cudaMemcpyAsync(&h, d_status, sizeof(h), cudaMemcpyDeviceToHost, as_stream(stream)) != cudaSuccess)
+    return VLM_ERR_CUDA;
+  if (cudaStreamSynchronize(as_stream(stream)) != cudaSuccess) return VLM_ERR_CUDA;
+  return h;
+}
+
+int vlm_config_preset(int preset, vlm_config* cfg) {
+  if (cfg == nullptr || (preset != 0 && preset != 1)) return VLM_ERR_INVALID_ARG;
+  cfg->layers = 24;
+  cfg->width = 1024;
+  cfg->heads = 16;
+  cfg->head_dim = 64;
+  cfg->mlp = 4096;
+  cfg->patch = preset == 0 ? 14 : 16;
+  cfg->merge = preset == 0 ? 2 : 1;
+  cfg->proj_out = 5120;
+  cfg->image_token_id = 10;
+  cfg->rope_theta = 10000.0f;
+  cfg->eps = 1e-5f;
+  cfg->normalize = 1;
+  return VLM_OK;
+}
+
+int64_t vlm_num_patches(const vlm_config* cfg, const int32_t* image_hw, int n_images) {
+  const int rc = check_config(cfg);
+  if (rc != VLM_OK) return rc;
+  Batch b;
+  const int rb = make_batch(cfg, image_hw, n_images, &b);
+  return rb != VLM_OK ? rb : b.T;
+}
+
+int64_t vlm_num_merged(const vlm_config* cfg, const int32_t* image_hw, int n_images) {
+  const int rc = check_config(cfg);
+  if (rc != VLM_OK) return rc;
+  Batch b;
+  const int rb = make_batch(cfg, image_hw, n_images, &b);
+  return rb != VLM_OK ? rb : b.Tm;
+}
+
+size_t vlm_tower_packed_bytes(const vlm_config* cfg) {
+  return check_config(cfg) == VLM_OK ? tower_layout(cfg).total : 0;
+}
+
+size_t vlm_projector_packed_bytes(const vlm_config* cfg) {
+  return check_config(cfg) == VLM_OK ? proj_layout(cfg).total : 0;
+}
+
+int vlm_pack_tower(const vlm_config* cfg, const vlm_tower_weights* w, void* d_packed, size_t packed_bytes,
+                   void* stream) {
+  VLM_TRY(check_config(cfg));
+  if (w == nullptr || d_packed == nullptr || !w->w_pe || !w->g_pre || !w->wq || !w->wk || !w->wv || !w->wo ||
+      !w->w_gate || !w->w_up || !w->w_down || !w->g_attn || !w->g_ffn)
+    return VLM_ERR_INVALID_ARG;
+  const TowerLayout L = tower_layout(cfg);
+  if (packed_bytes < L.total) return VLM_ERR_WORKSPACE;
+  cudaStream_t s = as_stream(stream);
+  uint8_t* dst = static_cast<uint8_t*>(d_packed);
+  const size_t D = cfg->width, F = cfg->mlp;
+  const int p = cfg->patch;
+  VLM_TRY(launch_pack_cols(w->w_pe, dst + L.w_pe, D, 3 * p * p, kpad(p), 0, 1, s));
+  if (cudaMemcpyAsync(dst + L.g_pre, w->g_pre, D * 4, cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+    return VLM_ERR_CUDA;
+  for (int l = 0; l < cfg->layers; ++l) {
+    uint8_t* ly = dst + L.layer0 + L.layer_stride * l;
+    const uint8_t* wq = static_cast<const uint8_t*>(w->wq) + l * D * D * 2;
+    const uint8_t* wk = static_cast<const uint8_t*>(w->wk) + l * D * D * 2;
+    const uint8_t* wv = static_cast<const uint8_t*>(w->wv) + l * D * D * 2;
+    const uint8_t* wo = static_cast<const uint8_t*>(w->wo) + l * D * D * 2;
+    const uint8_t* wg = static_cast<const uint8_t*>(w->w_gate) + l * F * D * 2;
+    const uint8_t* wu = static_cast<const uint8_t*>(w->w_up) + l * F * D * 2;
+    const uint8_t* wd = static_cast<const uint8_t*>(w->w_down) + l * D * F * 2;
+    bool ok = cudaMemcpyAsync(ly + L.wqkv, wq, D * D * 2, cudaMemcpyDeviceToDevice, s) == cudaSuccess;
+    ok = ok && cudaMemcpyAsync(ly + L.wqkv + D * D * 2, wk, D * D * 2, cudaMemcpyDeviceToDevice, s) == cudaSuccess;
+    ok = ok && cudaMemcpyAsync(ly + L.wqkv + 2 * D * D * 2, wv, D * D * 2, cudaMemcpyDeviceToDevice, s) == cudaSuccess;
+    ok = ok && cudaMemcpyAsync(ly + L.wo, wo, D * D * 2, cudaMemcpyDeviceToDevice, s) == cudaSuccess;
+    ok = ok && cudaMemcpyAsync(ly + L.wdown, wd, D * F * 2, cudaMemcpyDeviceToDevice, s) == cudaSuccess;
+    ok = ok && cudaMemcpyAsync(ly + L.g_attn, w->g_attn + l * D, D * 4, cudaMemcpyDeviceToDevice, s) == cudaSuccess;
+    ok = ok && cudaMemcpyAsync(ly + L.g_ffn, w->g_ffn + l * D, D * 4, cudaMemcpyDeviceToDevice, s) == cudaSuccess;
+    if (!ok) return VLM_ERR_CUDA;
+    VLM_TRY(launch_pack_gate_up(wg, wu, ly + L.wgu, F, D, s));
+  }
+  return VLM_OK;
+}
+
+int vlm_pack_projector(const vlm_config* cfg, const vlm_projector_weights* w, void* d_packed,
+                       size_t packed_bytes, void* stream) {
+  VLM_TRY(check_config(cfg));
+  if (w == nullptr || d_packed == nullptr || !w->g_proj || !w->w1 || !w->w2 || (cfg->merge > 1 && !w->w_merge))
+    return VLM_ERR_INVALID_ARG;
+  const ProjLayout L = proj_layout(cfg);
+  if (packed_bytes < L.total) return VLM_ERR_WORKSPACE;
+  cudaStream_t s = as_stream(stream);
+  uint8_t* dst = static_cast<uint8_t*>(d_packed);
+  const size_t D = cfg->width, E = cfg->proj_out;
+  const int mm = cfg->merge * cfg->merge;
+  bool ok = cudaMemcpyAsync(dst + L.g_proj, w->g_proj, D * 4, cudaMemcpyDeviceToDevice, s) == cudaSuccess;
+  ok = ok && cudaMemcpyAsync(dst + L.w1, w->w1, E * D * 2, cudaMemcpyDeviceToDevice, s) == cudaSuccess;
+  ok = ok && cudaMemcpyAsync(dst + L.w2, w->w2, E * E * 2, cudaMemcpyDeviceToDevice, s) == cudaSuccess;
+  if (!ok) return VLM_ERR_CUDA;
+  if (cfg->merge > 1) VLM_TRY(launch_pack_cols(w->w_merge, dst + L.w_merge, D, D * mm, D * mm, 1, mm, s));
+  return VLM_OK;
+}
+
+size_t vlm_encode_workspace_size(const vlm_config* cfg, const int32_t* image_hw, int n_images) {
+  if (check_config(cfg) != VLM_OK) return 0;
+  Batch b;
+  if (make_batch(cfg, image_hw, n_images, &b) != VLM_OK) return 0;
+  return carve_encode(nullptr, cfg, b).used;
+}
+
+int vlm_encode(const vlm_config* cfg, const float* pixels, const int32_t* image_hw, int n_images,
+               const void* d_packed_tower, void* d_out, void* d_workspace, size_t ws_bytes, int32_t* d_status,
+               void* stream) {
+  VLM_TRY(check_config(cfg));
+  if (pixels == nullptr || d_packed_tower == nullptr || d_out == nullptr || d_workspace == nullptr)
+    return VLM_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(d_workspace) & 255) return VLM_ERR_INVALID_ARG;
+  Batch b;
+  VLM_TRY(make_batch(cfg, image_hw, n_images, &b));
+  const EncodeWs e = carve_encode(d_workspace, cfg, b);
+  if (ws_bytes < e.used) return VLM_ERR_WORKSPACE;
+  cudaStream_t s = as_stream(stream);
+  const TowerLayout L = tower_layout(cfg);
+  const uint8_t* pk = static_cast<const uint8_t*>(d_packed_tower);
+  const int64_t T = b.T, D = cfg->width, F = cfg->mlp, kp = kpad(cfg->patch);
+
+  VLM_TRY(upload_batch(b, e.bd, s));
+  VLM_TRY(launch_rope_table(cfg->rope_theta, cfg->head_dim, b.max_pos, e.bd.rope, s));
+  VLM_TRY(launch_im2col(pixels, e.bd.info, e.bd.cu, b.n, T, cfg->patch, static_cast<int>(kp), cfg->normalize,
+                        e.cols, s));
+  VLM_TRY(launch_gemm(VLM_EPI_F32, e.cols, pk + L.w_pe, T, D, kp, e.x, nullptr, nullptr, nullptr, 0, d_status, s));
+  for (int l = 0; l < cfg->layers; ++l) {
+    const uint8_t* ly = pk + L.layer0 + L.layer_stride * l;
+    const float* g_attn = reinterpret_cast<const float*>(ly + L.g_attn);
+    const float* g_ffn = reinterpret_cast<const float*>(ly + L.g_ffn);
+    // ln_pre is fused into the first block's attention norm
+    const float* g0 = l == 0 ? reinterpret_cast<const float*>(pk + L.g_pre) : nullptr;
+    VLM_TRY(launch_rmsnorm(e.x, g0, g_attn, e.xn, T, static_cast<int>(D), cfg->eps, s));
+    VLM_TRY(launch_gemm(VLM_EPI_ROPE, e.xn, ly + L.wqkv, T, 3 * D, D, e.qkv, nullptr, e.bd.pos, e.bd.rope, 2 * D,
+                        d_status, s));
+    VLM_TRY(launch_attention(e.qkv, T, cfg->heads, e.bd.cu, e.bd.qt, b.n, b.total_qtiles, e.attn, d_status, s));
+    VLM_TRY(launch_gemm(VLM_EPI_RESID, e.attn, ly + L.wo, T, D, D, e.x, nullptr, nullptr, nullptr, 0, d_status, s));
+    VLM_TRY(launch_rmsnorm(e.x, nullptr, g_ffn, e.xn, T, static_cast<int>(D), cfg->eps, s));
+    VLM_TRY(launch_gemm(VLM_EPI_SWIGLU, e.xn, ly + L.wgu, T, 2 * F, D, e.hbuf, nullptr, nullptr, nullptr, 0,
+                        d_status, s));
+    const bool last = l == cfg->layers - 1;
+    VLM_TRY(launch_gemm(VLM_EPI_RESID, e.hbuf, ly + L.wdown, T, D, F, e.x, last ? d_out : nullptr, nullptr,
+                        nullptr, 0, d_status, s));
+  }
+  if (cfg->layers == 0) {
+    // ln_pre alone: normalise in place, then convert
+    VLM_TRY(launch_rmsnorm(e.x, reinterpret_cast<const float*>(pk + L.g_pre),
+                           reinterpret_cast<const float*>(pk + L.g_pre), e.xn, T, static_cast<int>(D), cfg->eps, s));
+    VLM_TRY(launch_f32_to_bf16(e.x, static_cast<__nv_bfloat16*>(d_out), T * D, s));
+  }
+  return VLM_OK;
+}
+
+size_t vlm_merge_project_workspace_size(const vlm_config* cfg, const int32_t* image_hw, int n_images) {
+  if (check_config(cfg) != VLM_OK) return 0;
+  Batch b;
+  if (make_batch(cfg, image_hw, n_images, &b) != VLM_OK) return 0;
+  return carve_proj(nullptr, cfg, b).used;
+}
+
+int vlm_merge_project(const vlm_config* cfg, const void* d_tower_out, const int32_t* image_hw, int n_images,
+                      const void* d_packed_projector, void* d_out, void* d_workspace, size_t ws_bytes,
+                      int32_t* d_status, void* stream) {
+  VLM_TRY(check_config(cfg));
+  if (d_tower_out == nullptr || d_packed_projector == nullptr || d_out == nullptr || d_workspace == nullptr)
+    return VLM_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(d_workspace) & 255) return VLM_ERR_INVALID_ARG;
+  Batch b;
+  VLM_TRY(make_batch(cfg, image_hw, n_images, &b));
+  const ProjWs p = carve_proj(d_workspace, cfg, b);
+  if (ws_bytes < p.used) return VLM_ERR_WORKSPACE;
+  cudaStream_t s = as_stream(stream);
+  const ProjLayout L = proj_layout(cfg);
+  const uint8_t* pk = static_cast<const uint8_t*>(d_packed_projector);
+  const int64_t D = cfg->width, E = cfg->proj_out, mm = static_cast<int64_t>(cfg->merge) * cfg->merge;
+
+  VLM_TRY(upload_batch(b, p.bd, s));
+  VLM_TRY(launch_merge_norm(static_cast<const __nv_bfloat16*>(d_tower_out), reinterpret_cast<const float*>(pk + L.g_proj),
+                            p.bd.info, p.bd.cu, b.n, b.T, static_cast<int>(D), cfg->merge, cfg->eps, p.z, s));
+  const __nv_bfloat16* y = p.z;
+  if (cfg->merge > 1) {
+    VLM_TRY(launch_gemm(VLM_EPI_BF16, p.z, pk + L.w_merge, b.Tm, D, mm * D, p.y, nullptr, nullptr, nullptr, 0,
+                        d_status, s));
+    y = p.y;
+  }
+  VLM_TRY(launch_gemm(VLM_EPI_GELU, y, pk + L.w1, b.Tm, E, D, p.g, nullptr, nullptr, nullptr, 0, d_status, s));
+  VLM_TRY(launch_gemm(VLM_EPI_BF16, p.g, pk + L.w2, b.Tm, E, E, d_out, nullptr, nullptr, nullptr, 0, d_status, s));
+  return VLM_OK;
+}
+
+size_t vlm_scatter_workspace_size(int64_t n_tokens) {
+  if (n_tokens < 0) return 0;
+  size_t used = 0;
+  carve_scatter(nullptr, n_tokens, &used);
+  return used;
+}
+
+int vlm_scatter(const int64_t* d_input_ids, int64_t n_tokens, int64_t image_token_id, const void* d_image_embeds,
+                int64_t n_image_tokens, void* d_text_embeds, int64_t row_bytes, void* d_workspace, size_t ws_bytes,
+                int32_t* d_status, void* stream) {
+  if (n_tokens < 0 || n_image_tokens < 0 || row_bytes <= 0 || row_bytes % 16) return VLM_ERR_INVALID_ARG;
+  if (n_tokens == 0) return n_image_tokens == 0 ? VLM_OK : VLM_ERR_BAD_SHAPE;
+  if (d_input_ids == nullptr || d_text_embeds == nullptr || d_workspace == nullptr || d_status == nullptr ||
+      (n_image_tokens > 0 && d_image_embeds == nullptr))
+    return VLM_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(d_image_embeds) | reinterpret_cast<uintptr_t>(d_text_embeds)) & 15)
+    return VLM_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(d_workspace) & 255) return VLM_ERR_INVALID_ARG;
+  if (n_tokens > (1LL << 40)) return VLM_ERR_BAD_SHAPE;
+  size_t used = 0;
+  const ScatterWs ws = carve_scatter(d_workspace, n_tokens, &used);
+  if (ws_bytes < used) return VLM_ERR_WORKSPACE;
+  return launch_scatter(d_input_ids, n_tokens, image_token_id, d_image_embeds, n_image_tokens, d_text_embeds,
+                        row_bytes, ws, d_status, as_stream(stream));
+}
+
+int64_t vlm_launch_count(void) { return g_launches.load(); }
+
+int vlm_profile_enable(int on) {
+  for (auto& r : g_records) {
+    g_pool.push_back(r.start);
+    g_pool.push_back(r.stop);
+  }
+  g_records.clear();
+  g_profile = on != 0;
+  return VLM_OK;
+}
+
+int vlm_profile_query(int kclass, int64_t* launches, double* total_ms) {
+  if (launches == nullptr || total_ms == nullptr || kclass < 0 || kclass >= KC_COUNT) return VLM_ERR_INVALID_ARG;
+  *launches = 0;
+  *total_ms = 0.0;
+  if (!g_records.empty() && cudaEventSynchronize(g_records.back().stop) != cudaSuccess) return VLM_ERR_CUDA;
+  for (const auto& r : g_records) {
+    if (r.kclass != kclass) continue;
+    float ms = 0.f;
+    if (cudaEventElapsedTime(&ms, r.start, r.stop) != cudaSuccess) return VLM_ERR_CUDA;
+    *launches += 1;
+    *total_ms += ms;
+  }
+  return VLM_OK;
+}
+
+// ---------------------------------------------------------------------------
+// Per-kernel entry points (include/vlm_kernels.h)
+// ---------------------------------------------------------------------------
+int vlm_gemm(int epilogue, const void* d_a, const void* d_b, int64_t M, int64_t N, int64_t K, void* d_c,
+             void* d_c_bf16, const int32_t* d_pos, const void* d_rope_table, int64_t rope_cols, int32_t* d_status,
+             void* stream) {
+  return launch_gemm(epilogue, d_a, d_b, M, N, K, d_c, d_c_bf16, d_pos, static_cast<const float2*>(d_rope_table),
+                     rope_cols, d_status, as_stream(stream));
+}
+
+int vlm_rope_table(float theta, int head_dim, int max_pos, void* d_table, void* stream) {
+  if (d_table == nullptr || head_dim != 64 || max_pos <= 0 || !(theta > 0.f)) return VLM_ERR_INVALID_ARG;
+  return launch_rope_table(theta, head_dim, max_pos, static_cast<float2*>(d_table), as_stream(stream));
+}
+
+size_t vlm_attention_workspace_size(int n_blocks) {
+  if (n_blocks <= 0) return 0;
+  return align_up(static_cast<size_t>(n_blocks) * sizeof(ImgInfo), 256) + 2 * align_up((n_blocks + 1) * 4, 256);
+}
+
+int vlm_attention(const void* d_qkv, int64_t T, int heads, int head_dim, const int32_t* cu_seqlens, int n_blocks,
+                  void* d_out, void* d_workspace, size_t ws_bytes, int32_t* d_status, void* stream) {
+  if (d_qkv == nullptr || d_out == nullptr || cu_seqlens == nullptr || d_workspace == nullptr || n_blocks <= 0 ||
+      heads <= 0)
+    return VLM_ERR_INVALID_ARG;
+  if (head_dim != 64) return VLM_ERR_UNSUPPORTED;
+  if (ws_bytes < vlm_attention_workspace_size(n_blocks)) return VLM_ERR_WORKSPACE;
+  if (cu_seqlens[0] != 0 || cu_seqlens[n_blocks] != T || T > (1LL << 31) - 1) return VLM_ERR_BAD_SHAPE;
+  Batch b;
+  b.n = n_blocks;
+  b.T = T;
+  b.h.assign(n_blocks, 1); b.w.assign(n_blocks, 1); b.H.assign(n_blocks, 0); b.W.assign(n_blocks, 0);
+  b.tok_off.resize(n_blocks + 1); b.m_off.assign(n_blocks + 1, 0); b.qt_off.resize(n_blocks + 1);
+  b.pix_off.assign(n_blocks, 0);
+  int64_t qt = 0;
+  for (int i = 0; i < n_blocks; ++i) {
+    const int64_t L = static_cast<int64_t>(cu_seqlens[i + 1]) - cu_seqlens[i];
+    if (L < 0) return VLM_ERR_BAD_SHAPE;
+    b.tok_off[i] = cu_seqlens[i];
+    b.w[i] = L > 0 ? static_cast<int32_t>(L) : 1;
+    b.qt_off[i] = static_cast<int32_t>(qt);
+    qt += (L + kAttnBQ - 1) / kAttnBQ;
+  }
+  b.tok_off[n_blocks] = cu_seqlens[n_blocks];
+  b.qt_off[n_blocks] = static_cast<int32_t>(qt);
+  Carver cv(d_workspace);
+  BatchDev d;
+  d.info = cv.take<ImgInfo>(n_blocks);
+  d.cu = cv.take<int32_t>(n_blocks + 1);
+  d.qt = cv.take<int32_t>(n_blocks + 1);
+  d.pos = nullptr;
+  d.rope = nullptr;
+  cudaStream_t s = as_stream(stream);
+  VLM_TRY(upload_batch(b, d, s));
+  return launch_attention(static_cast<const __nv_bfloat16*>(d_qkv), T, heads, d.cu, d.qt, n_blocks,
+                          static_cast<int>(qt), static_cast<__nv_bfloat16*>(d_out), d_status, s);
+}
+
+int vlm_rmsnorm(float* d_x, const float* d_g0, const float* d_g1, void* d_out, int64_t rows, int width, float eps,
+                void* stream) {
+  if (d_x == nullptr || d_g1 == nullptr || d_out == nullptr || rows < 0) return VLM_ERR_INVALID_ARG;
+  if (rows == 0) return VLM_OK;
+  return launch_rmsnorm(d_x, d_g0, d_g1, static_cast<__nv_bfloat16*>(d_out), rows, width, eps, as_stream(stream));
+}
+
+}  // extern "C"

@@ -1,0 +1,64 @@
+// Internal declarations shared by the kernel files and the C-ABI layer.
+#pragma once
+
+#include "common.cuh"
+
+namespace vlm {
+
+// Per-image table kept on the device.
+struct ImgInfo {
+  int32_t h, w;        // patch grid
+  int32_t H, W;        // pixels
+  int32_t tok_off;     // first patch of the image in the packed sequence
+  int32_t m_off;       // first merged token of the image
+  int32_t qt_off;      // first attention query tile of the image
+  int32_t pad;
+  int64_t pix_off;     // first float of the image in the pixel buffer
+};
+
+// Up to kChunk images' host-computed tables, passed by value to the setup kernel.
+constexpr int kChunk = 64;
+struct ImageChunk {
+  int32_t first, count;
+  int32_t h[kChunk], w[kChunk], H[kChunk], W[kChunk];
+  int32_t tok_off[kChunk + 1], m_off[kChunk + 1], qt_off[kChunk + 1];
+  int64_t pix_off[kChunk];
+};
+
+struct ScatterWs {
+  int32_t* chunk_count;
+  int64_t* chunk_base;
+  int64_t* dst_rows;
+  int32_t* ok_flag;
+};
+
+// Query rows per attention CTA tile.
+constexpr int kAttnBQ = 128;
+
+void note_extra_launches(int n);
+
+int launch_setup(const ImageChunk& chunk, ImgInfo* info, int32_t* cu, int32_t* qt, int32_t* pos,
+                 int n_images, cudaStream_t s);
+int launch_rope_table(float theta, int head_dim, int max_pos, float2* tab, cudaStream_t s);
+int launch_im2col(const float* pix, const ImgInfo* info, const int32_t* cu, int n_images, int64_t T,
+                  int p, int kp, int normalize, __nv_bfloat16* out, cudaStream_t s);
+int launch_rmsnorm(float* x, const float* g0, const float* g1, __nv_bfloat16* out, int64_t rows,
+                   int width, float eps, cudaStream_t s);
+int launch_merge_norm(const __nv_bfloat16* x, const float* g, const ImgInfo* info, const int32_t* cu,
+                      int n_images, int64_t T, int width, int m, float eps, __nv_bfloat16* z,
+                      cudaStream_t s);
+int launch_scatter(const int64_t* ids, int64_t n, int64_t token, const void* img, int64_t n_img,
+                   void* text, int64_t row_bytes, ScatterWs ws, int32_t* status, cudaStream_t s);
+int launch_pack_gate_up(const void* gate, const void* up, void* dst, int64_t f, int64_t d, cudaStream_t s);
+int launch_pack_cols(const void* src, void* dst, int64_t rows, int64_t src_cols, int64_t dst_cols, int mode,
+                     int mm, cudaStream_t s);
+int launch_f32_to_bf16(const float* x, __nv_bfloat16* y, int64_t n, cudaStream_t s);
+
+int launch_gemm(int epi, const void* a, const void* b, int64_t M, int64_t N, int64_t K, void* c,
+                void* c_bf16, const int32_t* pos, const float2* rope, int64_t rope_cols, int32_t* status,
+                cudaStream_t s);
+
+int launch_attention(const __nv_bfloat16* qkv, int64_t T, int heads, const int32_t* cu, const int32_t* qt,
+                     int n_blocks, int total_qtiles, __nv_bfloat16* out, int32_t* status, cudaStream_t s);
+
+}  // namespace vlm

@@ -1,0 +1,467 @@
+// Memory-bound kernels of the image half: index setup, RoPE angle table,
+// patch gather (im2col with the processor normalisation), RMSNorm, merge
+// gather, masked scatter and weight packing. Every one is a coalesced,
+// vectorised streaming kernel; none uses the tensor cores.
+#include "kernels.cuh"
+
+namespace vlm {
+
+// ---------------------------------------------------------------------------
+// Index setup: per-image tables and per-token (row, col) positions.
+// ---------------------------------------------------------------------------
+__global__ void setup_kernel(ImageChunk chunk, ImgInfo* info, int32_t* cu, int32_t* qt,
+                             int32_t* pos, int n_images) {
+  const int tid = blockIdx.x * blockDim.x + threadIdx.x;
+  if (tid < chunk.count) {
+    const int b = chunk.first + tid;
+    ImgInfo in;
+    in.h = chunk.h[tid];
+    in.w = chunk.w[tid];
+    in.H = chunk.H[tid];
+    in.W = chunk.W[tid];
+    in.tok_off = chunk.tok_off[tid];
+    in.m_off = chunk.m_off[tid];
+    in.qt_off = chunk.qt_off[tid];
+    in.pad = 0;
+    in.pix_off = chunk.pix_off[tid];
+    info[b] = in;
+    cu[b] = chunk.tok_off[tid];
+    qt[b] = chunk.qt_off[tid];
+    if (b == n_images - 1) {
+      cu[n_images] = chunk.tok_off[tid + 1];
+      qt[n_images] = chunk.qt_off[tid + 1];
+    }
+  }
+  if (pos == nullptr) return;
+  const int t0 = chunk.tok_off[0], t1 = chunk.tok_off[chunk.count];
+  for (int t = t0 + tid; t < t1; t += gridDim.x * blockDim.x) {
+    int lo = 0, hi = chunk.count - 1;  // last image whose offset <= t
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (chunk.tok_off[mid] <= t) lo = mid; else hi = mid - 1;
+    }
+    const int local = t - chunk.tok_off[lo];
+    const int w = chunk.w[lo];
+    pos[t] = ((local / w) << 16) | (local % w);
+  }
+}
+
+// 2D RoPE angle table: tab[p][i] = (cos, sin)(p * w_k), w_k = theta^(-2k/dh),
+// k = 2i for the row half (i < dh/4) and k = 2(i - dh/4) + 1 for the column half.
+__global__ void rope_table_kernel(float theta, int head_dim, int max_pos, float2* tab) {
+  const int half = head_dim / 2, quarter = head_dim / 4;
+  const int idx = blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= max_pos * half) return;
+  const int p = idx / half, i = idx % half;
+  const int k = i < quarter ? 2 * i : 2 * (i - quarter) + 1;
+  const double omega = pow(static_cast<double>(theta), -2.0 * k / head_dim);
+  double s, c;
+  sincos(static_cast<double>(p) * omega, &s, &c);
+  tab[idx] = make_float2(static_cast<float>(c), static_cast<float>(s));
+}
+
+__device__ __forceinline__ int find_block(const int32_t* cu, int n, int t) {
+  int lo = 0, hi = n - 1;  // last b with cu[b] <= t
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (__ldg(cu + mid) <= t) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
+// ---------------------------------------------------------------------------
+// Patch gather: one warp per patch; column k = ch*p*p + ky*p + kx of the
+// conv weight; columns >= 3p^2 are zero padding.
+// ---------------------------------------------------------------------------
+__constant__ float c_mean[3] = {0.48145466f, 0.4578275f, 0.40821073f};
+__constant__ float c_std[3] = {0.26862954f, 0.26130258f, 0.27577711f};
+
+__global__ void im2col_kernel(const float* __restrict__ pix, const ImgInfo* __restrict__ info,
+                              const int32_t* __restrict__ cu, int n_images, int64_t T, int p, int kp,
+                              int normalize, __nv_bfloat16* __restrict__ out) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
+  const int pp = p * p, kreal = 3 * pp;
+  for (int64_t t = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; t < T; t += warps) {
+    const int b = find_block(cu, n_images, static_cast<int>(t));
+    const ImgInfo in = info[b];
+    const int local = static_cast<int>(t) - in.tok_off;
+    const int r = local / in.w, c = local % in.w;
+    const float* base = pix + in.pix_off;
+    uint32_t* orow = reinterpret_cast<uint32_t*>(out + t * kp);
+    for (int k2 = lane; k2 < kp / 2; k2 += 32) {
+      float v[2];
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int k = 2 * k2 + e;
+        float val = 0.f;
+        if (k < kreal) {
+          const int ch = k / pp, rem = k - ch * pp, ky = rem / p, kx = rem - ky * p;
+          val = __ldg(base + (static_cast<int64_t>(ch) * in.H + r * p + ky) * in.W + c * p + kx);
+          if (normalize) val = (val - c_mean[ch]) / c_std[ch];
+        }
+        v[e] = val;
+      }
+      orow[k2] = pack_bf16x2(v[0], v[1]);
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// RMSNorm, one warp per row of `width` fp32 values (width % 128 == 0, <= 2048).
+// With g0: y = norm(x) * g0 is written back to x, and out = bf16(norm(y) * g1).
+// Without g0: out = bf16(norm(x) * g1).
+// ---------------------------------------------------------------------------
+template <int NV>
+__global__ void rmsnorm_kernel(float* __restrict__ x, const float* __restrict__ g0,
+                               const float* __restrict__ g1, __nv_bfloat16* __restrict__ out,
+                               int64_t rows, float eps) {
+  constexpr int width = NV * 128;
+  const int lane = threadIdx.x & 31;
+  const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
+  for (int64_t row = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; row < rows;
+       row += warps) {
+    float4* xr = reinterpret_cast<float4*>(x + row * width);
+    float4 v[NV];
+    float ss = 0.f;
+#pragma unroll
+    for (int j = 0; j < NV; ++j) {
+      v[j] = xr[lane + 32 * j];
+      ss += v[j].x * v[j].x + v[j].y * v[j].y + v[j].z * v[j].z + v[j].w * v[j].w;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    float rs = rsqrtf(ss / width + eps);
+    if (g0 != nullptr) {
+      const float4* gr = reinterpret_cast<const float4*>(g0);
+      ss = 0.f;
+#pragma unroll
+      for (int j = 0; j < NV; ++j) {
+        const float4 g = __ldg(gr + lane + 32 * j);
+        v[j].x *= rs * g.x; v[j].y *= rs * g.y; v[j].z *= rs * g.z; v[j].w *= rs * g.w;
+        xr[lane + 32 * j] = v[j];
+        ss += v[j].x * v[j].x + v[j].y * v[j].y + v[j].z * v[j].z + v[j].w * v[j].w;
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+      rs = rsqrtf(ss / width + eps);
+    }
+    const float4* gr = reinterpret_cast<const float4*>(g1);
+    uint2* orow = reinterpret_cast<uint2*>(out + row * width);
+#pragma unroll
+    for (int j = 0; j < NV; ++j) {
+      const float4 g = __ldg(gr + lane + 32 * j);
+      uint2 o;
+      o.x = pack_bf16x2(v[j].x * rs * g.x, v[j].y * rs * g.y);
+      o.y = pack_bf16x2(v[j].z * rs * g.z, v[j].w * rs * g.w);
+      orow[lane + 32 * j] = o;
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Projector RMSNorm + m x m merge gather, one warp per patch (bf16 in/out).
+// Patch (r, c) of image b goes to merged token m_off_b + (r/m)(w/m) + c/m,
+// slot (r%m)*m + c%m, i.e. z[token, slot*D + ch] (patch-major).
+// ---------------------------------------------------------------------------
+template <int NV>
+__global__ void merge_norm_kernel(const __nv_bfloat16* __restrict__ x, const float* __restrict__ g,
+                                  const ImgInfo* __restrict__ info, const int32_t* __restrict__ cu,
+                                  int n_images, int64_t T, int m, float eps,
+                                  __nv_bfloat16* __restrict__ z) {
+  constexpr int width = NV * 128;
+  const int lane = threadIdx.x & 31;
+  const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
+  for (int64_t t = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; t < T; t += warps) {
+    const uint2* xr = reinterpret_cast<const uint2*>(x + t * width);
+    float v[NV][4];
+    float ss = 0.f;
+#pragma unroll
+    for (int j = 0; j < NV; ++j) {
+      const uint2 u = xr[lane + 32 * j];
+      const __nv_bfloat162 a = *reinterpret_cast<const __nv_bfloat162*>(&u.x);
+      const __nv_bfloat162 bb = *reinterpret_cast<const __nv_bfloat162*>(&u.y);
+      v[j][0] = __low2float(a); v[j][1] = __high2float(a);
+      v[j][2] = __low2float(bb); v[j][3] = __high2float(bb);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) ss += v[j][e] * v[j][e];
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    const float rs = rsqrtf(ss / width + eps);
+    const int b = find_block(cu, n_images, static_cast<int>(t));
+    const ImgInfo in = info[b];
+    const int local = static_cast<int>(t) - in.tok_off;
+    const int r = local / in.w, c = local % in.w;
+    const int64_t mt = in.m_off + (r / m) * (in.w / m) + c / m;
+    const int slot = (r % m) * m + c % m;
+    uint2* orow = reinterpret_cast<uint2*>(z + (mt * m * m + slot) * width);
+    const float4* gr = reinterpret_cast<const float4*>(g);
+#pragma unroll
+    for (int j = 0; j < NV; ++j) {
+      const float4 gg = __ldg(gr + lane + 32 * j);
+      uint2 o;
+      o.x = pack_bf16x2(v[j][0] * rs * gg.x, v[j][1] * rs * gg.y);
+      o.y = pack_bf16x2(v[j][2] * rs * gg.z, v[j][3] * rs * gg.w);
+      orow[lane + 32 * j] = o;
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Masked scatter: (1) placeholder count per 256-id chunk, (2) one-block scan
+// and total check, (3) destination row of every placeholder, (4) row copy.
+// Steps 3 and 4 do nothing unless step 2 found count == n_image_tokens.
+// ---------------------------------------------------------------------------
+__global__ void scatter_count_kernel(const int64_t* __restrict__ ids, int64_t n, int64_t token,
+                                     int32_t* __restrict__ chunk_count) {
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x;
+  const int flag = (i < n && ids[i] == token) ? 1 : 0;
+  const int wc = __popc(__ballot_sync(0xffffffffu, flag));
+  __shared__ int s[8];
+  if ((threadIdx.x & 31) == 0) s[threadIdx.x >> 5] = wc;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int tot = 0;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) tot += s[w];
+    chunk_count[blockIdx.x] = tot;
+  }
+}
+
+__global__ void scatter_scan_kernel(const int32_t* __restrict__ chunk_count, int64_t n_chunks,
+                                    int64_t expected, int64_t* __restrict__ chunk_base,
+                                    int32_t* __restrict__ ok_flag, int32_t* status) {
+  // 1024 threads; sequential over blocks of 1024 chunks with a running carry.
+  __shared__ int64_t warp_sums[32];
+  __shared__ int64_t carry;
+  if (threadIdx.x == 0) carry = 0;
+  __syncthreads();
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  for (int64_t base = 0; base < n_chunks; base += 1024) {
+    const int64_t i = base + threadIdx.x;
+    const int64_t v = i < n_chunks ? chunk_count[i] : 0;
+    int64_t incl = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int64_t y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    if (lane == 31) warp_sums[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+      int64_t ws = warp_sums[lane];
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int64_t y = __shfl_up_sync(0xffffffffu, ws, o);
+        if (lane >= o) ws += y;
+      }
+      warp_sums[lane] = ws;  // inclusive over warps
+    }
+    __syncthreads();
+    const int64_t before = carry + (warp > 0 ? warp_sums[warp - 1] : 0) + incl - v;
+    if (i < n_chunks) chunk_base[i] = before;
+    __syncthreads();
+    if (threadIdx.x == 0) carry += warp_sums[31];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) {
+    const int good = (carry == expected) ? 1 : 0;
+    *ok_flag = good;
+    if (!good) set_status(status, VLM_ERR_COUNT_MISMATCH);
+  }
+}
+
+__global__ void scatter_positions_kernel(const int64_t* __restrict__ ids, int64_t n, int64_t token,
+                                         const int64_t* __restrict__ chunk_base,
+                                         const int32_t* __restrict__ ok_flag,
+                                         int64_t* __restrict__ dst_rows) {
+  if (*ok_flag == 0) return;
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x;
+  const int flag = (i < n && ids[i] == token) ? 1 : 0;
+  const unsigned ballot = __ballot_sync(0xffffffffu, flag);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  __shared__ int s[8];
+  if (lane == 0) s[warp] = __popc(ballot);
+  __syncthreads();
+  int before = 0;
+  for (int w = 0; w < warp; ++w) before += s[w];
+  before += __popc(ballot & ((1u << lane) - 1u));
+  if (flag) dst_rows[chunk_base[blockIdx.x] + before] = i;
+}
+
+__global__ void scatter_copy_kernel(const uint4* __restrict__ img, uint4* __restrict__ text,
+                                    const int64_t* __restrict__ dst_rows,
+                                    const int32_t* __restrict__ ok_flag, int64_t n_rows,
+                                    int64_t vec_per_row) {
+  if (*ok_flag == 0) return;
+  const int64_t total = n_rows * vec_per_row;
+  for (int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; idx < total;
+       idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t k = idx / vec_per_row, j = idx - k * vec_per_row;
+    text[dst_rows[k] * vec_per_row + j] = __ldg(img + idx);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Weight packing (exact copies / reorderings of bf16 values)
+// ---------------------------------------------------------------------------
+// dst [2F, D]: rows 32j..32j+15 = gate rows 16j.., rows 32j+16..32j+31 = up rows 16j..
+__global__ void pack_gate_up_kernel(const uint4* __restrict__ gate, const uint4* __restrict__ up,
+                                    uint4* __restrict__ dst, int64_t f, int64_t vec_per_row) {
+  const int64_t total = 2 * f * vec_per_row;
+  for (int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; idx < total;
+       idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t row = idx / vec_per_row, j = idx - row * vec_per_row;
+    const int64_t grp = row >> 5, within = row & 31;
+    const int64_t src_row = grp * 16 + (within & 15);
+    dst[idx] = (within < 16 ? gate : up)[src_row * vec_per_row + j];
+  }
+}
+
+// dst [rows, dst_cols] from src [rows, src_cols], bf16:
+//   mode 0 (pad):     dst[r, k] = k < src_cols ? src[r, k] : 0
+//   mode 1 (permute): dst[r, slot*D + c] = src[r, c*mm + slot]  (D = src_cols / mm)
+__global__ void pack_cols_kernel(const __nv_bfloat16* __restrict__ src, __nv_bfloat16* __restrict__ dst,
+                                 int64_t rows, int64_t src_cols, int64_t dst_cols, int mode, int mm) {
+  const int64_t total = rows * dst_cols;
+  for (int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; idx < total;
+       idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t r = idx / dst_cols, k = idx - r * dst_cols;
+    __nv_bfloat16 v;
+    if (mode == 0) {
+      v = k < src_cols ? src[r * src_cols + k] : __float2bfloat16(0.f);
+    } else {
+      const int64_t d = src_cols / mm;
+      const int64_t slot = k / d, c = k - slot * d;
+      v = src[r * src_cols + c * mm + slot];
+    }
+    dst[idx] = v;
+  }
+}
+
+__global__ void f32_to_bf16_kernel(const float* __restrict__ x, __nv_bfloat16* __restrict__ y, int64_t n) {
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; 2 * i < n;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const float2 v = reinterpret_cast<const float2*>(x)[i];
+    reinterpret_cast<uint32_t*>(y)[i] = pack_bf16x2(v.x, v.y);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Host launchers
+// ---------------------------------------------------------------------------
+static int grid_for(int64_t work_items, int per_block) {
+  const int64_t blocks = (work_items + per_block - 1) / per_block;
+  const int64_t cap = static_cast<int64_t>(num_sms()) * 16;
+  return static_cast<int>(blocks < 1 ? 1 : (blocks > cap ? cap : blocks));
+}
+
+int launch_setup(const ImageChunk& chunk, ImgInfo* info, int32_t* cu, int32_t* qt, int32_t* pos,
+                 int n_images, cudaStream_t s) {
+  const int64_t tokens = chunk.tok_off[chunk.count] - chunk.tok_off[0];
+  const int grid = grid_for(tokens > chunk.count ? tokens : chunk.count, 256);
+  launch_begin(KC_SETUP, s);
+  setup_kernel<<<grid, 256, 0, s>>>(chunk, info, cu, qt, pos, n_images);
+  launch_end(KC_SETUP, s);
+  return cudaGetLastError() == cudaSuccess ? VLM_OK : VLM_ERR_CUDA;
+}
+
+int launch_rope_table(float theta, int head_dim, int max_pos, float2* tab, cudaStream_t s) {
+  const int n = max_pos * head_dim / 2;
+  launch_begin(KC_SETUP, s);
+  rope_table_kernel<<<(n + 255) / 256, 256, 0, s>>>(theta, head_dim, max_pos, tab);
+  launch_end(KC_SETUP, s);
+  return cudaGetLastError() == cudaSuccess ? VLM_OK : VLM_ERR_CUDA;
+}
+
+int launch_im2col(const float* pix, const ImgInfo* info, const int32_t* cu, int n_images, int64_t T,
+                  int p, int kp, int normalize, __nv_bfloat16* out, cudaStream_t s) {
+  launch_begin(KC_IM2COL, s);
+  im2col_kernel<<<grid_for(T * 32, 256), 256, 0, s>>>(pix, info, cu, n_images, T, p, kp, normalize, out);
+  launch_end(KC_IM2COL, s);
+  return cudaGetLastError() == cudaSuccess ? VLM_OK : VLM_ERR_CUDA;
+}
+
+int launch_rmsnorm(float* x, const float* g0, const float* g1, __nv_bfloat16* out, int64_t rows,
+                   int width, float eps, cudaStream_t s) {
+  if (width % 128 || width > 2048 || width <= 0) return VLM_ERR_UNSUPPORTED;
+  const int grid = grid_for(rows * 32, 256);
+  launch_begin(KC_NORM, s);
+  switch (width / 128) {
+#define VLM_NORM_CASE(nv) \
+  case nv: rmsnorm_kernel<nv><<<grid, 256, 0, s>>>(x, g0, g1, out, rows, eps); break;
+    VLM_NORM_CASE(1) VLM_NORM_CASE(2) VLM_NORM_CASE(3) VLM_NORM_CASE(4) VLM_NORM_CASE(5)
+    VLM_NORM_CASE(6) VLM_NORM_CASE(7) VLM_NORM_CASE(8) VLM_NORM_CASE(9) VLM_NORM_CASE(10)
+    VLM_NORM_CASE(11) VLM_NORM_CASE(12) VLM_NORM_CASE(13) VLM_NORM_CASE(14) VLM_NORM_CASE(15)
+    VLM_NORM_CASE(16)
+#undef VLM_NORM_CASE
+    default: break;
+  }
+  launch_end(KC_NORM, s);
+  return cudaGetLastError() == cudaSuccess ? VLM_OK : VLM_ERR_CUDA;
+}
+
+int launch_merge_norm(const __nv_bfloat16* x, const float* g, const ImgInfo* info, const int32_t* cu,
+                      int n_images, int64_t T, int width, int m, float eps, __nv_bfloat16* z,
+                      cudaStream_t s) {
+  if (width % 128 || width > 2048 || width <= 0) return VLM_ERR_UNSUPPORTED;
+  const int grid = grid_for(T * 32, 256);
+  launch_begin(KC_MERGE, s);
+  switch (width / 128) {
+#define VLM_MERGE_CASE(nv) \
+  case nv: merge_norm_kernel<nv><<<grid, 256, 0, s>>>(x, g, info, cu, n_images, T, m, eps, z); break;
+    VLM_MERGE_CASE(1) VLM_MERGE_CASE(2) VLM_MERGE_CASE(3) VLM_MERGE_CASE(4) VLM_MERGE_CASE(5)
+    VLM_MERGE_CASE(6) VLM_MERGE_CASE(7) VLM_MERGE_CASE(8) VLM_MERGE_CASE(9) VLM_MERGE_CASE(10)
+    VLM_MERGE_CASE(11) VLM_MERGE_CASE(12) VLM_MERGE_CASE(13) VLM_MERGE_CASE(14) VLM_MERGE_CASE(15)
+    VLM_MERGE_CASE(16)
+#undef VLM_MERGE_CASE
+    default: break;
+  }
+  launch_end(KC_MERGE, s);
+  return cudaGetLastError() == cudaSuccess ? VLM_OK : VLM_ERR_CUDA;
+}
+
+int launch_scatter(const int64_t* ids, int64_t n, int64_t token, const void* img, int64_t n_img,
+                   void* text, int64_t row_bytes, ScatterWs ws, int32_t* status, cudaStream_t s) {
+  const int64_t n_chunks = (n + 255) / 256;
+  launch_begin(KC_SCATTER, s);
+  scatter_count_kernel<<<static_cast<unsigned>(n_chunks), 256, 0, s>>>(ids, n, token, ws.chunk_count);
+  scatter_scan_kernel<<<1, 1024, 0, s>>>(ws.chunk_count, n_chunks, n_img, ws.chunk_base, ws.ok_flag, status);
+  scatter_positions_kernel<<<static_cast<unsigned>(n_chunks), 256, 0, s>>>(ids, n, token, ws.chunk_base,
+                                                                           ws.ok_flag, ws.dst_rows);
+  const int64_t vec = row_bytes / 16;
+  scatter_copy_kernel<<<grid_for(n_img * vec, 256), 256, 0, s>>>(
+      static_cast<const uint4*>(img), static_cast<uint4*>(text), ws.dst_rows, ws.ok_flag, n_img, vec);
+  launch_end(KC_SCATTER, s);
+  note_extra_launches(3);
+  return cudaGetLastError() == cudaSuccess ? VLM_OK : VLM_ERR_CUDA;
+}
+
+int launch_pack_gate_up(const void* gate, const void* up, void* dst, int64_t f, int64_t d, cudaStream_t s) {
+  const int64_t vec = d * 2 / 16;
+  launch_begin(KC_PACK, s);
+  pack_gate_up_kernel<<<grid_for(2 * f * vec, 256), 256, 0, s>>>(
+      static_cast<const uint4*>(gate), static_cast<const uint4*>(up), static_cast<uint4*>(dst), f, vec);
+  launch_end(KC_PACK, s);
+  return cudaGetLastError() == cudaSuccess ? VLM_OK : VLM_ERR_CUDA;
+}
+
+int launch_pack_cols(const void* src, void* dst, int64_t rows, int64_t src_cols, int64_t dst_cols, int mode,
+                     int mm, cudaStream_t s) {
+  launch_begin(KC_PACK, s);
+  pack_cols_kernel<<<grid_for(rows * dst_cols, 256), 256, 0, s>>>(
+      static_cast<const __nv_bfloat16*>(src), static_cast<__nv_bfloat16*>(dst), rows, src_cols, dst_cols,
+      mode, mm);
+  launch_end(KC_PACK, s);
+  return cudaGetLastError() == cudaSuccess ? VLM_OK : VLM_ERR_CUDA;
+}
+
+int launch_f32_to_bf16(const float* x, __nv_bfloat16* y, int64_t n, cudaStream_t s) {
+  launch_begin(KC_NORM, s);
+  f32_to_bf16_kernel<<<grid_for(n / 2, 256), 256, 0, s>>>(x, y, n);
+  launch_end(KC_NORM, s);
+  return cudaGetLastError() == cudaSuccess ? VLM_OK : VLM_ERR_CUDA;
+}
+
+}  // namespace vlm

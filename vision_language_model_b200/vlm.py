@@ -1,0 +1,366 @@
+"""Thin ctypes binding of libvlm_b200.so (include/vlm.h, include/vlm_kernels.h).
+
+Argument marshalling only: torch supplies device memory and the current CUDA
+stream; every step of the path runs in the library's sm_100a kernels. There
+is no fallback: if the library is missing or a tensor is not on a CUDA
+device, the call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libvlm_b200.so")
+_lib = None
+
+# vlm_status values (include/vlm.h)
+OK, ERR_INVALID_ARG, ERR_BAD_SHAPE, ERR_WORKSPACE, ERR_COUNT_MISMATCH, ERR_TIMEOUT, ERR_CUDA, ERR_UNSUPPORTED = \
+    0, -1, -2, -3, -4, -5, -6, -7
+# epilogues (include/vlm_kernels.h)
+EPI_BF16, EPI_F32, EPI_RESID, EPI_SWIGLU, EPI_ROPE, EPI_GELU = range(6)
+# profiling kernel classes
+KCLASS = {"gemm": 0, "attention": 1, "rmsnorm": 2, "im2col": 3, "merge": 4, "scatter": 5, "setup": 6, "pack": 7}
+
+
+class VlmError(RuntimeError):
+    def __init__(self, rc: int, what: str):
+        self.rc = rc
+        super().__init__(f"{what}: {status_string(rc)} ({rc})")
+
+
+class Config(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in
+                ("layers", "width", "heads", "head_dim", "mlp", "patch", "merge", "proj_out", "image_token_id")] + \
+               [("rope_theta", ctypes.c_float), ("eps", ctypes.c_float), ("normalize", ctypes.c_int32)]
+
+    def as_dict(self) -> dict:
+        return {n: getattr(self, n) for n, _ in self._fields_}
+
+
+class TowerWeights(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in
+                ("w_pe", "g_pre", "wq", "wk", "wv", "wo", "w_gate", "w_up", "w_down", "g_attn", "g_ffn")]
+
+
+class ProjectorWeights(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in ("g_proj", "w_merge", "w1", "w2")]
+
+
+def lib_path() -> str:
+    return _LIB_PATH
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded library; raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(_LIB_PATH):
+            raise RuntimeError(f"{_LIB_PATH} is missing: build it with `python -m vision_language_model_b200.build`")
+        L = ctypes.CDLL(_LIB_PATH)
+        P, I32, I64, SZ, F = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t, ctypes.c_float
+        CP = ctypes.POINTER(Config)
+        sig = {
+            "vlm_status_string": (ctypes.c_char_p, [I32]),
+            "vlm_status_sync": (I32, [P, P]),
+            "vlm_config_preset": (I32, [I32, CP]),
+            "vlm_tower_packed_bytes": (SZ, [CP]),
+            "vlm_pack_tower": (I32, [CP, ctypes.POINTER(TowerWeights), P, SZ, P]),
+            "vlm_projector_packed_bytes": (SZ, [CP]),
+            "vlm_pack_projector": (I32, [CP, ctypes.POINTER(ProjectorWeights), P, SZ, P]),
+            "vlm_num_patches": (I64, [CP, P, I32]),
+            "vlm_num_merged": (I64, [CP, P, I32]),
+            "vlm_encode_workspace_size": (SZ, [CP, P, I32]),
+            "vlm_encode": (I32, [CP, P, P, I32, P, P, P, SZ, P, P]),
+            "vlm_merge_project_workspace_size": (SZ, [CP, P, I32]),
+            "vlm_merge_project": (I32, [CP, P, P, I32, P, P, P, SZ, P, P]),
+            "vlm_scatter_workspace_size": (SZ, [I64]),
+            "vlm_scatter": (I32, [P, I64, I64, P, I64, P, I64, P, SZ, P, P]),
+            "vlm_launch_count": (I64, []),
+            "vlm_profile_enable": (I32, [I32]),
+            "vlm_profile_query": (I32, [I32, ctypes.POINTER(I64), ctypes.POINTER(ctypes.c_double)]),
+            "vlm_gemm": (I32, [I32, P, P, I64, I64, I64, P, P, P, P, I64, P, P]),
+            "vlm_rope_table": (I32, [F, I32, I32, P, P]),
+            "vlm_attention_workspace_size": (SZ, [I32]),
+            "vlm_attention": (I32, [P, I64, I32, I32, P, I32, P, P, SZ, P, P]),
+            "vlm_rmsnorm": (I32, [P, P, P, P, I64, I32, F, P]),
+        }
+        for name, (res, args) in sig.items():
+            fn = getattr(L, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = L
+    return _lib
+
+
+def status_string(rc: int) -> str:
+    return lib().vlm_status_string(int(rc)).decode()
+
+
+def _check(rc: int, what: str) -> None:
+    if rc != OK:
+        raise VlmError(rc, what)
+
+
+def _stream(stream=None) -> int:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+def _dev(t: torch.Tensor | None, name: str) -> int | None:
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t.data_ptr()
+
+
+def _hw_array(image_hw) -> tuple:
+    flat = [int(v) for hw in image_hw for v in hw]
+    arr = (ctypes.c_int32 * max(1, len(flat)))(*flat)
+    return arr, len(flat) // 2
+
+
+# ---------------------------------------------------------------------------
+# Configs
+# ---------------------------------------------------------------------------
+
+def preset(name: str = "mistral3", **overrides) -> Config:
+    cfg = Config()
+    _check(lib().vlm_config_preset({"mistral3": 0, "pixtral12b": 1}[name], ctypes.byref(cfg)), "vlm_config_preset")
+    for k, v in overrides.items():
+        setattr(cfg, k, v)
+    return cfg
+
+
+def num_patches(cfg: Config, image_hw) -> int:
+    arr, n = _hw_array(image_hw)
+    t = lib().vlm_num_patches(ctypes.byref(cfg), arr, n)
+    if t < 0:
+        raise VlmError(int(t), "vlm_num_patches")
+    return int(t)
+
+
+def num_merged(cfg: Config, image_hw) -> int:
+    arr, n = _hw_array(image_hw)
+    t = lib().vlm_num_merged(ctypes.byref(cfg), arr, n)
+    if t < 0:
+        raise VlmError(int(t), "vlm_num_merged")
+    return int(t)
+
+
+def new_status(device=None) -> torch.Tensor:
+    return torch.zeros(1, dtype=torch.int32, device=device or "cuda")
+
+
+def status_sync(status: torch.Tensor, stream=None) -> int:
+    return int(lib().vlm_status_sync(_dev(status, "status"), _stream(stream)))
+
+
+# ---------------------------------------------------------------------------
+# Weight packing
+# ---------------------------------------------------------------------------
+
+def pack_tower(cfg: Config, w: dict, stream=None) -> torch.Tensor:
+    """w: device tensors named as in vlm_tower_weights (bf16 matrices, fp32 gains)."""
+    L = lib()
+    tw = TowerWeights(**{k: _dev(w[k], k) for k, _ in TowerWeights._fields_})
+    nbytes = L.vlm_tower_packed_bytes(ctypes.byref(cfg))
+    if nbytes == 0:
+        raise VlmError(ERR_INVALID_ARG, "vlm_tower_packed_bytes")
+    packed = torch.empty(nbytes, dtype=torch.uint8, device=w["wq"].device)
+    _check(L.vlm_pack_tower(ctypes.byref(cfg), ctypes.byref(tw), packed.data_ptr(), nbytes, _stream(stream)),
+           "vlm_pack_tower")
+    return packed
+
+
+def pack_projector(cfg: Config, w: dict, stream=None) -> torch.Tensor:
+    L = lib()
+    pw = ProjectorWeights(g_proj=_dev(w["g_proj"], "g_proj"), w_merge=_dev(w.get("w_merge"), "w_merge"),
+                          w1=_dev(w["w1"], "w1"), w2=_dev(w["w2"], "w2"))
+    nbytes = L.vlm_projector_packed_bytes(ctypes.byref(cfg))
+    if nbytes == 0:
+        raise VlmError(ERR_INVALID_ARG, "vlm_projector_packed_bytes")
+    packed = torch.empty(nbytes, dtype=torch.uint8, device=w["w1"].device)
+    _check(L.vlm_pack_projector(ctypes.byref(cfg), ctypes.byref(pw), packed.data_ptr(), nbytes, _stream(stream)),
+           "vlm_pack_projector")
+    return packed
+
+
+# ---------------------------------------------------------------------------
+# The three calls of the path
+# ---------------------------------------------------------------------------
+
+def encode_workspace_size(cfg: Config, image_hw) -> int:
+    arr, n = _hw_array(image_hw)
+    return int(lib().vlm_encode_workspace_size(ctypes.byref(cfg), arr, n))
+
+
+def encode(cfg: Config, pixels: torch.Tensor, image_hw, packed_tower: torch.Tensor, out=None, workspace=None,
+           status=None, stream=None) -> torch.Tensor:
+    """Vision tower: pixels (device fp32, CHW blocks concatenated) -> bf16 [T, width]."""
+    L = lib()
+    arr, n = _hw_array(image_hw)
+    T = num_patches(cfg, image_hw)
+    dev = pixels.device
+    if out is None:
+        out = torch.empty((T, cfg.width), dtype=torch.bfloat16, device=dev)
+    ws_need = L.vlm_encode_workspace_size(ctypes.byref(cfg), arr, n)
+    if workspace is None:
+        workspace = torch.empty(ws_need, dtype=torch.uint8, device=dev)
+    if status is None:
+        status = new_status(dev)
+    _check(L.vlm_encode(ctypes.byref(cfg), _dev(pixels, "pixels"), arr, n, _dev(packed_tower, "packed_tower"),
+                        _dev(out, "out"), _dev(workspace, "workspace"), workspace.numel(), _dev(status, "status"),
+                        _stream(stream)), "vlm_encode")
+    return out
+
+
+def merge_project_workspace_size(cfg: Config, image_hw) -> int:
+    arr, n = _hw_array(image_hw)
+    return int(lib().vlm_merge_project_workspace_size(ctypes.byref(cfg), arr, n))
+
+
+def merge_project(cfg: Config, tower_out: torch.Tensor, image_hw, packed_projector: torch.Tensor, out=None,
+                  workspace=None, status=None, stream=None) -> torch.Tensor:
+    """Projector: bf16 [T, width] -> bf16 [T_m, proj_out]."""
+    L = lib()
+    arr, n = _hw_array(image_hw)
+    Tm = num_merged(cfg, image_hw)
+    dev = tower_out.device
+    if out is None:
+        out = torch.empty((Tm, cfg.proj_out), dtype=torch.bfloat16, device=dev)
+    if workspace is None:
+        workspace = torch.empty(L.vlm_merge_project_workspace_size(ctypes.byref(cfg), arr, n), dtype=torch.uint8,
+                                device=dev)
+    if status is None:
+        status = new_status(dev)
+    _check(L.vlm_merge_project(ctypes.byref(cfg), _dev(tower_out, "tower_out"), arr, n,
+                               _dev(packed_projector, "packed_projector"), _dev(out, "out"),
+                               _dev(workspace, "workspace"), workspace.numel(), _dev(status, "status"),
+                               _stream(stream)), "vlm_merge_project")
+    return out
+
+
+def scatter_workspace_size(n_tokens: int) -> int:
+    return int(lib().vlm_scatter_workspace_size(int(n_tokens)))
+
+
+def scatter(input_ids: torch.Tensor, image_embeds: torch.Tensor, text_embeds: torch.Tensor, image_token_id: int = 10,
+            workspace=None, status=None, stream=None) -> torch.Tensor:
+    """In place: rows of text_embeds at image_token_id positions <- image_embeds rows, in order."""
+    L = lib()
+    if input_ids.dtype != torch.int64:
+        raise ValueError("input_ids must be int64")
+    n = input_ids.numel()
+    if text_embeds.shape[0] != n:
+        raise ValueError("text_embeds must have one row per id")
+    row_bytes = text_embeds[0].numel() * text_embeds.element_size()
+    if image_embeds.numel() and image_embeds[0].numel() * image_embeds.element_size() != row_bytes:
+        raise ValueError("image and text rows differ in size")
+    dev = text_embeds.device
+    if workspace is None:
+        workspace = torch.empty(max(256, L.vlm_scatter_workspace_size(n)), dtype=torch.uint8, device=dev)
+    if status is None:
+        status = new_status(dev)
+    _check(L.vlm_scatter(_dev(input_ids, "input_ids"), n, int(image_token_id), _dev(image_embeds, "image_embeds"),
+                         image_embeds.shape[0], _dev(text_embeds, "text_embeds"), row_bytes,
+                         _dev(workspace, "workspace"), workspace.numel(), _dev(status, "status"), _stream(stream)),
+           "vlm_scatter")
+    return text_embeds
+
+
+# ---------------------------------------------------------------------------
+# Per-kernel entry points
+# ---------------------------------------------------------------------------
+
+def gemm(epilogue: int, a: torch.Tensor, b: torch.Tensor, out: torch.Tensor, out_bf16=None, pos=None,
+         rope_table=None, rope_cols: int = 0, status=None, stream=None) -> torch.Tensor:
+    M, K = a.shape
+    N = b.shape[0]
+    if status is None:
+        status = new_status(a.device)
+    _check(lib().vlm_gemm(epilogue, _dev(a, "a"), _dev(b, "b"), M, N, K, _dev(out, "out"), _dev(out_bf16, "out_bf16"),
+                          _dev(pos, "pos"), _dev(rope_table, "rope_table"), rope_cols, _dev(status, "status"),
+                          _stream(stream)), "vlm_gemm")
+    return out
+
+
+def rope_table(theta: float, head_dim: int, max_pos: int, device="cuda", stream=None) -> torch.Tensor:
+    tab = torch.empty((max_pos, head_dim // 2, 2), dtype=torch.float32, device=device)
+    _check(lib().vlm_rope_table(float(theta), head_dim, max_pos, tab.data_ptr(), _stream(stream)), "vlm_rope_table")
+    return tab
+
+
+def attention(qkv: torch.Tensor, cu_seqlens, heads: int, out=None, status=None, stream=None) -> torch.Tensor:
+    L = lib()
+    T = qkv.shape[0]
+    cu = (ctypes.c_int32 * len(cu_seqlens))(*[int(c) for c in cu_seqlens])
+    nb = len(cu_seqlens) - 1
+    if out is None:
+        out = torch.empty((T, heads * 64), dtype=torch.bfloat16, device=qkv.device)
+    ws = torch.empty(max(256, L.vlm_attention_workspace_size(nb)), dtype=torch.uint8, device=qkv.device)
+    if status is None:
+        status = new_status(qkv.device)
+    _check(L.vlm_attention(_dev(qkv, "qkv"), T, heads, 64, cu, nb, _dev(out, "out"), ws.data_ptr(), ws.numel(),
+                           _dev(status, "status"), _stream(stream)), "vlm_attention")
+    return out
+
+
+def rmsnorm(x: torch.Tensor, g1: torch.Tensor, g0=None, eps: float = 1e-5, out=None, stream=None) -> torch.Tensor:
+    rows, width = x.shape
+    if out is None:
+        out = torch.empty((rows, width), dtype=torch.bfloat16, device=x.device)
+    _check(lib().vlm_rmsnorm(_dev(x, "x"), _dev(g0, "g0"), _dev(g1, "g1"), _dev(out, "out"), rows, width, float(eps),
+                             _stream(stream)), "vlm_rmsnorm")
+    return out
+
+
+# ---------------------------------------------------------------------------
+# Instrumentation
+# ---------------------------------------------------------------------------
+
+def launch_count() -> int:
+    return int(lib().vlm_launch_count())
+
+
+def profile_enable(on: bool = True) -> None:
+    _check(lib().vlm_profile_enable(1 if on else 0), "vlm_profile_enable")
+
+
+def profile_query(kclass: str) -> tuple:
+    n = ctypes.c_int64()
+    ms = ctypes.c_double()
+    _check(lib().vlm_profile_query(KCLASS[kclass], ctypes.byref(n), ctypes.byref(ms)), "vlm_profile_query")
+    return int(n.value), float(ms.value)
+
+
+# ---------------------------------------------------------------------------
+# A reusable pipeline: packed weights + workspaces for repeated calls
+# ---------------------------------------------------------------------------
+
+class ImagePipeline:
+    """vlm_encode -> vlm_merge_project (-> vlm_scatter) with buffers kept between calls."""
+
+    def __init__(self, cfg: Config, tower: dict, projector: dict, image_hw, device="cuda"):
+        self.cfg = cfg
+        self.image_hw = [tuple(int(v) for v in hw) for hw in image_hw]
+        self.packed_tower = pack_tower(cfg, tower)
+        self.packed_proj = pack_projector(cfg, projector)
+        self.T = num_patches(cfg, self.image_hw)
+        self.Tm = num_merged(cfg, self.image_hw)
+        self.tower_out = torch.empty((self.T, cfg.width), dtype=torch.bfloat16, device=device)
+        self.embeds = torch.empty((self.Tm, cfg.proj_out), dtype=torch.bfloat16, device=device)
+        ws = max(encode_workspace_size(cfg, self.image_hw), merge_project_workspace_size(cfg, self.image_hw))
+        self.workspace = torch.empty(ws, dtype=torch.uint8, device=device)
+        self.status = new_status(device)
+
+    def __call__(self, pixels: torch.Tensor, stream=None) -> torch.Tensor:
+        encode(self.cfg, pixels, self.image_hw, self.packed_tower, out=self.tower_out, workspace=self.workspace,
+               status=self.status, stream=stream)
+        merge_project(self.cfg, self.tower_out, self.image_hw, self.packed_proj, out=self.embeds,
+                      workspace=self.workspace, status=self.status, stream=stream)
+        return self.embeds
