@@ -133,7 +133,7 @@ def _qkv(seed, T, heads=16, q_scale=1.0):
 
 
 @pytest.mark.parametrize("cu", [[0, 1], [0, 1, 65, 200, 457], [0, 128, 256], [0, 300], [0, 64, 64, 191]])
-@pytest.mark.parametrize("q_scale", [1.0, 0.3])
+@pytest.mark.parametrize("q_scale", [1.0, 0.3, 6.0])
 def test_attention_blocks(cu, q_scale):
     T = cu[-1]
     qkv, q, k, v = _qkv(7, T, q_scale=q_scale)
