@@ -197,6 +197,34 @@ VLM_API int vlm_scatter(const int64_t* d_input_ids, int64_t n_tokens, int64_t im
                 void* stream);
 
 /* ---------------------------------------------------------------------------
+ * vlm_scatter_noalloc -- vlm_scatter for callers that cannot allocate device
+ * memory. The pages have no counterpart: this is a library convenience.
+ *
+ * vlm_scatter takes its scratch (placeholder counts and destination rows) from
+ * a caller workspace. A serving engine that gives all free device memory to
+ * its own pools at start-up, or a plugin host that passes an operator only its
+ * input and output buffers, has no workspace to offer. This entry point keeps
+ * that scratch in a fixed array inside the library's device memory (about
+ * 2 MiB, held on every GPU that loads the library until the process exits),
+ * so the caller passes only inputs and outputs; no call allocates or frees
+ * anything.
+ *
+ * Arguments, layouts, results and device-side errors are those of vlm_scatter.
+ * n_tokens above VLM_SCATTER_NOALLOC_MAX_TOKENS returns VLM_ERR_BAD_SHAPE
+ * before anything is launched.
+ * All calls share the one array: calls that overlap on the GPU (other streams,
+ * other host threads on the same device) race and must be serialised by the
+ * caller. Each call writes all the scratch it reads, so nothing carries over.
+ * The first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress, with that device current) and caches it; make that
+ * first call before any stream capture begins.
+ * ------------------------------------------------------------------------- */
+#define VLM_SCATTER_NOALLOC_MAX_TOKENS 262144
+VLM_API int vlm_scatter_noalloc(const int64_t* d_input_ids, int64_t n_tokens, int64_t image_token_id,
+                                const void* d_image_embeds, int64_t n_image_tokens, void* d_text_embeds,
+                                int64_t row_bytes, int32_t* d_status, void* stream);
+
+/* ---------------------------------------------------------------------------
  * Instrumentation (host-side, not thread-safe)
  * ------------------------------------------------------------------------- */
 /* Total kernels this library has launched in the process. */
