@@ -1,0 +1,285 @@
+// Block-diagonal (per-image) bidirectional attention on the sm_100a tensor
+// cores, head_dim 64: for query t of block b,
+//   o_t = sum_u softmax_u(q_t . k_u / 8) v_u   over the keys u of block b only.
+//
+// One CTA = one 128-query tile of one block and one head; two CTAs share an
+// SM so one CTA's softmax overlaps the other's MMAs. 6 warps:
+//   warp 0      TMA: the Q tile once, then K and V tiles of 128 keys into a
+//               2-stage ring (128-byte swizzle).
+//   warp 1      allocates 256 TMEM columns; one thread issues
+//                 S  = Q K^T      (tcgen05.mma, M=128 N=128, A and B in smem)
+//                 O += P V        (tcgen05.mma, M=128 N=64, A = P in TMEM,
+//                                  B = V in smem, MN-major)
+//   warps 2..5  softmax, one thread per query row = TMEM lane: reads its S row
+//               (128 fp32), keeps a running max m (log2 units) and sum l,
+//               writes P = 2^(s*log2e/8 - m) as bf16 into TMEM, rescales its O
+//               row when m grows by more than 8 (otherwise the stale max is
+//               kept; P stays <= 2^8, exact after the final division by l),
+//               and finally writes O / l.
+// TMEM: S in columns [0,128), P in [128,192) (bf16 pairs), O in [192,256).
+// Keys past the block end are masked to -inf; their V rows are finite (rows of
+// the next block) or TMA zero fill (past the sequence). Query tiles never
+// straddle two blocks, so every block's result is independent of the others.
+#include "kernels.cuh"
+
+namespace vlm {
+
+namespace {
+
+constexpr int BQ = kAttnBQ;  // 128
+constexpr int BKV = 128;
+constexpr int DH = 64;
+constexpr int kStages = 2;
+constexpr int kTileBytes = 128 * DH * 2;  // 16 KiB: 128 rows x 128 bytes
+constexpr int kSmemBytes = (1 + 2 * kStages) * kTileBytes + 256 + 1024;
+constexpr uint32_t kColS = 0, kColP = 128, kColO = 192, kTmemCols = 256;
+constexpr float kRescaleThreshold = 8.0f;  // log2 units
+
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+struct AttnArgs {
+  const int32_t* cu;
+  const int32_t* qt;
+  int n_blocks;
+  int heads;
+  __nv_bfloat16* out;
+  int32_t* status;
+};
+
+__global__ void __launch_bounds__(192, 2)
+    attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, const AttnArgs args) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sQ = smem;
+  uint8_t* sK = smem + kTileBytes;                    // [kStages] tiles
+  uint8_t* sV = smem + (1 + kStages) * kTileBytes;    // [kStages] tiles
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (1 + 2 * kStages) * kTileBytes);
+  uint64_t* q_full = bars;
+  uint64_t* kv_full = bars + 1;               // [kStages]
+  uint64_t* kv_empty = bars + 1 + kStages;    // [kStages]
+  uint64_t* s_full = bars + 1 + 2 * kStages;
+  uint64_t* s_free = s_full + 1;
+  uint64_t* p_full = s_full + 2;
+  uint64_t* o_done = s_full + 3;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(o_done + 1);
+  int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  // this CTA's block, query tile and head
+  const int tile = blockIdx.x, h = blockIdx.y;
+  int lo = 0, hi = args.n_blocks - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (__ldg(args.qt + mid) <= tile) lo = mid; else hi = mid - 1;
+  }
+  const int kbeg = __ldg(args.cu + lo), kend = __ldg(args.cu + lo + 1);
+  const int q0 = kbeg + (tile - __ldg(args.qt + lo)) * BQ;
+  const int n_kv = (kend - kbeg + BKV - 1) / BKV;
+  const int D = args.heads * DH;
+
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(q_full), 1);
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(smem_u32(kv_full + s), 1);
+      mbar_init(smem_u32(kv_empty + s), 1);
+    }
+    mbar_init(smem_u32(s_full), 1);
+    mbar_init(smem_u32(s_free), 128);
+    mbar_init(smem_u32(p_full), 128);
+    mbar_init(smem_u32(o_done), 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) prefetch_tmap(&tm_qkv);
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  volatile int* abort_v = abort_flag;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      const uint32_t qb = smem_u32(q_full);
+      mbar_arrive_expect_tx(qb, kTileBytes);
+      tma_load_2d(smem_u32(sQ), &tm_qkv, qb, h * DH, q0);
+      for (int j = 0; j < n_kv; ++j) {
+        const int st = j % kStages;
+        if (!mbar_wait(smem_u32(kv_empty + st), ((j / kStages) & 1) ^ 1, abort_v, args.status)) break;
+        const uint32_t fb = smem_u32(kv_full + st);
+        mbar_arrive_expect_tx(fb, 2 * kTileBytes);
+        const int key0 = kbeg + j * BKV;
+        tma_load_2d(smem_u32(sK + st * kTileBytes), &tm_qkv, fb, D + h * DH, key0);
+        tma_load_2d(smem_u32(sV + st * kTileBytes), &tm_qkv, fb, 2 * D + h * DH, key0);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc_s = idesc_bf16(BQ, BKV);
+      constexpr uint32_t idesc_o = idesc_bf16(BQ, DH, /*b_mn_major=*/true);
+      bool ok = mbar_wait(smem_u32(q_full), 0, abort_v, args.status);
+      const uint64_t qdesc = smem_desc_sw128(smem_u32(sQ));
+      for (int j = 0; ok && j <= n_kv; ++j) {
+        if (j < n_kv) {
+          const int st = j % kStages;
+          if (!mbar_wait(smem_u32(kv_full + st), (j / kStages) & 1, abort_v, args.status)) break;
+          if (j > 0 && !mbar_wait(smem_u32(s_free), (j - 1) & 1, abort_v, args.status)) break;
+          tc_fence_after();
+          const uint64_t kdesc = smem_desc_sw128(smem_u32(sK + st * kTileBytes));
+#pragma unroll
+          for (int k = 0; k < DH / 16; ++k)
+            umma_bf16_ss(tmem + kColS, qdesc + 2 * k, kdesc + 2 * k, idesc_s, k > 0 ? 1u : 0u);
+          umma_commit(smem_u32(s_full));
+        }
+        if (j > 0) {
+          const int jp = j - 1, st = jp % kStages;
+          if (!mbar_wait(smem_u32(p_full), jp & 1, abort_v, args.status)) break;
+          tc_fence_after();
+          const uint64_t vdesc = smem_desc_sw128(smem_u32(sV + st * kTileBytes));
+#pragma unroll
+          for (int kk = 0; kk < BKV / 16; ++kk)  // 16 keys = 8 TMEM columns of bf16 pairs = 2048 smem bytes
+            umma_bf16_ts(tmem + kColO, tmem + kColP + 8 * kk, vdesc + 128 * kk, idesc_o,
+                         (jp > 0 || kk > 0) ? 1u : 0u);
+          umma_commit(smem_u32(kv_empty + st));
+          umma_commit(smem_u32(o_done));
+        }
+      }
+    }
+  } else {
+    // softmax: this thread owns query row r of the tile (TMEM lane r)
+    const int q = warp & 3;
+    const int r = q * 32 + lane;
+    const uint32_t trow = tmem + (static_cast<uint32_t>(q * 32) << 16);
+    const float sl2 = 1.4426950408889634f * 0.125f;  // log2(e) / sqrt(64)
+    float m = -INFINITY, l = 0.f;
+    bool ok = true;
+    for (int j = 0; j < n_kv; ++j) {
+      if (!mbar_wait_warp(smem_u32(s_full), j & 1, abort_v, args.status)) { ok = false; break; }
+      tc_fence_after();
+      float s[BKV];
+#pragma unroll
+      for (int c = 0; c < BKV; c += 32) {
+        uint32_t u[32];
+        tmem_ld32(trow + kColS + c, u);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) s[c + i] = __uint_as_float(u[i]);
+      }
+      tc_fence_before();
+      mbar_arrive(smem_u32(s_free));
+
+      const int nvalid = kend - (kbeg + j * BKV);
+      if (nvalid < BKV) {
+#pragma unroll
+        for (int c = 0; c < BKV; ++c)
+          if (c >= nvalid) s[c] = -INFINITY;
+      }
+      float mx = s[0];
+#pragma unroll
+      for (int c = 1; c < BKV; ++c) mx = fmaxf(mx, s[c]);
+      const float m_cand = mx * sl2;
+      const bool grow = m_cand > m + kRescaleThreshold;
+      const float m_new = grow ? m_cand : m;
+      const float corr = grow ? ex2(m - m_new) : 1.0f;
+      float sum = 0.f;
+      uint32_t pk[BKV / 2];
+#pragma unroll
+      for (int c = 0; c < BKV; c += 2) {
+        const float p0 = ex2(fmaf(s[c], sl2, -m_new));
+        const float p1 = ex2(fmaf(s[c + 1], sl2, -m_new));
+        sum += p0 + p1;
+        pk[c / 2] = pack_bf16x2(p0, p1);
+      }
+      l = l * corr + sum;
+      m = m_new;
+
+      if (j > 0) {
+        // PV of the previous tile must be done before O is rescaled and P overwritten
+        if (!mbar_wait_warp(smem_u32(o_done), (j - 1) & 1, abort_v, args.status)) { ok = false; break; }
+        tc_fence_after();
+        if (__any_sync(0xffffffffu, grow)) {
+#pragma unroll
+          for (int c = 0; c < DH; c += 32) {
+            uint32_t u[32];
+            tmem_ld32(trow + kColO + c, u);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) u[i] = __float_as_uint(__uint_as_float(u[i]) * corr);
+            tmem_st32(trow + kColO + c, u);
+          }
+        }
+      }
+#pragma unroll
+      for (int c = 0; c < BKV / 2; c += 32) {
+        uint32_t u[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) u[i] = pk[c + i];
+        tmem_st32(trow + kColP + c, u);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(smem_u32(p_full));
+    }
+    if (ok && mbar_wait_warp(smem_u32(o_done), (n_kv - 1) & 1, abort_v, args.status)) {
+      tc_fence_after();
+      const float inv = 1.0f / l;
+      const int row = q0 + r;
+      __nv_bfloat16* dst = args.out + static_cast<int64_t>(row) * D + h * DH;
+#pragma unroll
+      for (int c = 0; c < DH; c += 32) {
+        uint32_t u[32];
+        tmem_ld32(trow + kColO + c, u);
+        if (row < kend) {
+          uint4* d4 = reinterpret_cast<uint4*>(dst + c);
+#pragma unroll
+          for (int jj = 0; jj < 4; ++jj)
+            d4[jj] = make_uint4(pack_bf16x2(__uint_as_float(u[8 * jj]) * inv, __uint_as_float(u[8 * jj + 1]) * inv),
+                                pack_bf16x2(__uint_as_float(u[8 * jj + 2]) * inv, __uint_as_float(u[8 * jj + 3]) * inv),
+                                pack_bf16x2(__uint_as_float(u[8 * jj + 4]) * inv, __uint_as_float(u[8 * jj + 5]) * inv),
+                                pack_bf16x2(__uint_as_float(u[8 * jj + 6]) * inv, __uint_as_float(u[8 * jj + 7]) * inv));
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+}  // namespace
+
+int launch_attention(const __nv_bfloat16* qkv, int64_t T, int heads, const int32_t* cu, const int32_t* qt,
+                     int n_blocks, int total_qtiles, __nv_bfloat16* out, int32_t* status, cudaStream_t s) {
+  if (total_qtiles <= 0) return VLM_OK;
+  if (heads <= 0 || heads > 65535) return VLM_ERR_UNSUPPORTED;
+  CUtensorMap tm;
+  const uint64_t row = 3ull * heads * DH;
+  if (!make_tmap_2d_bf16(&tm, qkv, row, static_cast<uint64_t>(T), row * 2, DH, BQ)) return VLM_ERR_CUDA;
+  static bool attr_done[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !attr_done[dev]) {
+    if (cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) !=
+        cudaSuccess)
+      return VLM_ERR_CUDA;
+    attr_done[dev] = true;
+  }
+  AttnArgs args{cu, qt, n_blocks, heads, out, status};
+  dim3 grid(total_qtiles, heads);
+  launch_begin(KC_ATTN, s);
+  attn_tc_kernel<<<grid, 192, kSmemBytes, s>>>(tm, args);
+  launch_end(KC_ATTN, s);
+  return cudaGetLastError() == cudaSuccess ? VLM_OK : VLM_ERR_CUDA;
+}
+
+}  // namespace vlm

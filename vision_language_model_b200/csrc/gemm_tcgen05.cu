@@ -273,7 +273,7 @@ __global__ void __launch_bounds__(192, 1)
     uint32_t acc_phase = 0;
     for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x) {
       const int mt = tile / args.n_tiles, nt = tile - mt * args.n_tiles;
-      if (!mbar_wait(smem_u32(tfull + acc), acc_phase, abort_v, args.status)) break;
+      if (!mbar_wait_warp(smem_u32(tfull + acc), acc_phase, abort_v, args.status)) break;
       tc_fence_after();
       const int row = mt * GBM + q * 32 + lane;
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * BN);
@@ -291,33 +291,6 @@ __global__ void __launch_bounds__(192, 1)
     tc_fence_after();
     tmem_dealloc(tmem_base, S::TMEM_COLS);
   }
-}
-
-PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (fn == nullptr) {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  }
-  return fn;
-}
-
-// 2D bf16 tensor map over a row-major [outer, inner] matrix with a
-// box_outer x 64 box (128 bytes inner) and 128-byte swizzle.
-bool make_tmap_bf16(CUtensorMap* map, const void* ptr, uint64_t inner, uint64_t outer, uint32_t box_outer) {
-  auto enc = tensor_map_encoder();
-  if (enc == nullptr) return false;
-  cuuint64_t dims[2] = {inner, outer};
-  cuuint64_t strides[1] = {inner * 2};
-  cuuint32_t box[2] = {static_cast<cuuint32_t>(GBK), box_outer};
-  cuuint32_t estr[2] = {1, 1};
-  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box,
-                         estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
 }
 
 template <int BN, int EPI>
@@ -355,6 +328,34 @@ int dispatch_epi(int epi, const CUtensorMap& ta, const CUtensorMap& tb, const Ge
 
 }  // namespace
 
+namespace {
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (fn == nullptr) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+}  // namespace
+
+bool make_tmap_2d_bf16(CUtensorMap* map, const void* ptr, uint64_t inner, uint64_t outer, uint64_t row_bytes,
+                       uint32_t box_inner, uint32_t box_outer) {
+  auto enc = tensor_map_encoder();
+  if (enc == nullptr) return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {row_bytes};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box,
+                         estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 int launch_gemm(int epi, const void* a, const void* b, int64_t M, int64_t N, int64_t K, void* c, void* c_bf16,
                 const int32_t* pos, const float2* rope, int64_t rope_cols, int32_t* status, cudaStream_t s) {
   if (a == nullptr || b == nullptr || c == nullptr) return VLM_ERR_INVALID_ARG;
@@ -369,8 +370,8 @@ int launch_gemm(int epi, const void* a, const void* b, int64_t M, int64_t N, int
   const int bn = (needs256 || (N % 256 == 0 && N >= 2048)) ? 256 : 128;
 
   CUtensorMap ta, tb;
-  if (!make_tmap_bf16(&ta, a, K, M, GBM)) return VLM_ERR_CUDA;
-  if (!make_tmap_bf16(&tb, b, K, N, bn)) return VLM_ERR_CUDA;
+  if (!make_tmap_2d_bf16(&ta, a, K, M, K * 2, GBK, GBM)) return VLM_ERR_CUDA;
+  if (!make_tmap_2d_bf16(&tb, b, K, N, K * 2, GBK, bn)) return VLM_ERR_CUDA;
 
   GemmArgs args;
   args.M = static_cast<int>(M);

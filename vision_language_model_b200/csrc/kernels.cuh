@@ -54,6 +54,10 @@ int launch_pack_cols(const void* src, void* dst, int64_t rows, int64_t src_cols,
                      int mm, cudaStream_t s);
 int launch_f32_to_bf16(const float* x, __nv_bfloat16* y, int64_t n, cudaStream_t s);
 
+// 2D bf16 tensor map, 128-byte swizzle, box box_outer x box_inner (box_inner * 2 == 128 bytes).
+bool make_tmap_2d_bf16(CUtensorMap* map, const void* ptr, uint64_t inner, uint64_t outer, uint64_t row_bytes,
+                       uint32_t box_inner, uint32_t box_outer);
+
 int launch_gemm(int epi, const void* a, const void* b, int64_t M, int64_t N, int64_t K, void* c,
                 void* c_bf16, const int32_t* pos, const float2* rope, int64_t rope_cols, int32_t* status,
                 cudaStream_t s);
