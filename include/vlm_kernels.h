@@ -83,6 +83,14 @@ VLM_API int vlm_attention(const void* d_qkv, int64_t T, int heads, int head_dim,
 VLM_API int vlm_rmsnorm(float* d_x, const float* d_g0, const float* d_g1, void* d_out, int64_t rows,
                 int width, float eps, void* stream);
 
+/* Failure-detection self-test (no counterpart on the pages): launches one
+ * thread that waits on a shared-memory mbarrier nothing arrives on, using the
+ * same bounded wait as every barrier wait of the GEMM and attention kernels,
+ * with a budget of budget_cycles SM clocks (1 .. 2^32). The wait gives up,
+ * writes VLM_ERR_TIMEOUT to *d_status and the kernel returns; the CUDA context
+ * stays usable. Nothing faults, traps or hangs. */
+VLM_API int vlm_selftest_wait_timeout(int64_t budget_cycles, int32_t* d_status, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -144,6 +144,7 @@ def test_attention_blocks(cu, q_scale):
 def test_attention_single_patch_is_v():
     qkv, q, k, v = _qkv(8, 1)
     out = vlm.attention(qkv, [0, 1], 16)
+    # one key: probability exactly 1, so the output is v itself
     np.testing.assert_array_equal(to_np(out), v.reshape(1, -1))
 
 
@@ -214,3 +215,17 @@ def test_scatter_count_mismatch_writes_nothing():
     vlm.scatter(ids.reshape(-1).cuda(), img.cuda(), t_gpu, 10, status=status)
     assert vlm.status_sync(status) == vlm.ERR_COUNT_MISMATCH
     assert torch.equal(t_gpu.cpu().view(torch.int16), text.view(torch.int16))
+
+
+# ---------------------------------------------------------------------------
+# Failure detection: a barrier wait that runs out reports, it does not hang
+# ---------------------------------------------------------------------------
+
+def test_bounded_wait_times_out_into_status_and_context_survives():
+    status = vlm.new_status()
+    vlm.selftest_wait_timeout(2_000_000, status)  # ~1 ms of SM clocks
+    assert vlm.status_sync(status) == vlm.ERR_TIMEOUT
+    # the context is still usable: a normal call after it succeeds
+    qkv, q, k, v = _qkv(8, 1)
+    out = vlm.attention(qkv, [0, 1], 16)
+    np.testing.assert_array_equal(to_np(out), v.reshape(1, -1))

@@ -616,6 +616,11 @@ int vlm_attention(const void* d_qkv, int64_t T, int heads, int head_dim, const i
                           static_cast<int>(qt), static_cast<__nv_bfloat16*>(d_out), d_status, s);
 }
 
+int vlm_selftest_wait_timeout(int64_t budget_cycles, int32_t* d_status, void* stream) {
+  if (d_status == nullptr || budget_cycles <= 0 || budget_cycles > (1LL << 32)) return VLM_ERR_INVALID_ARG;
+  return launch_wait_timeout_selftest(budget_cycles, d_status, as_stream(stream));
+}
+
 int vlm_rmsnorm(float* d_x, const float* d_g0, const float* d_g1, void* d_out, int64_t rows, int width, float eps,
                 void* stream) {
   if (d_x == nullptr || d_g1 == nullptr || d_out == nullptr || rows < 0) return VLM_ERR_INVALID_ARG;

@@ -7,15 +7,18 @@
 //   warp 0      TMA: the Q tile once, then K and V tiles of 128 keys into a
 //               2-stage ring (128-byte swizzle).
 //   warp 1      allocates 256 TMEM columns; one thread issues
-//                 S  = Q K^T      (tcgen05.mma, M=128 N=128, A and B in smem)
-//                 O += P V        (tcgen05.mma, M=128 N=64, A = P in TMEM,
-//                                  B = V in smem, MN-major)
+//                 S  = Q K^T      (tcgen05.mma kind::f16, M=128 N=128, A and B in smem)
+//                 O += P V        (M=128 N=64, A = P in TMEM, B = V in smem, MN-major)
+//               S_{j+1} is issued as soon as the softmax has copied S_j out.
 //   warps 2..5  softmax, one thread per query row = TMEM lane: reads its S row
-//               (128 fp32), keeps a running max m (log2 units) and sum l,
-//               writes P = 2^(s*log2e/8 - m) as bf16 into TMEM, rescales its O
-//               row when m grows by more than 8 (otherwise the stale max is
-//               kept; P stays <= 2^8, exact after the final division by l),
-//               and finally writes O / l.
+//               (128 fp32), finds the tile max with four short 3-input-max
+//               chains, keeps a running max m (log2 units) that only moves when
+//               the tile max exceeds it by more than 8 (otherwise the stale max
+//               is kept; P stays <= 2^8 and the final division by l is exact),
+//               computes P = 2^(s*log2e/8 - m) with packed fp32x2 FMAs and MUFU
+//               ex2, writes P to TMEM as bf16, sums the fp32 values into l with
+//               packed adds, rescales its O row when m moved, and finally writes
+//               O / l.
 // TMEM: S in columns [0,128), P in [128,192) (bf16 pairs), O in [192,256).
 // Keys past the block end are masked to -inf; their V rows are finite (rows of
 // the next block) or TMA zero fill (past the sequence). Query tiles never
@@ -39,6 +42,66 @@ __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// Packed pairs of fp32 (first value in the low word) for the f32x2 instructions.
+__device__ __forceinline__ uint64_t pack2(uint32_t lo, uint32_t hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "r"(lo), "r"(hi));
+  return r;
+}
+__device__ __forceinline__ uint64_t pair_f32(float v) { return pack2(__float_as_uint(v), __float_as_uint(v)); }
+__device__ __forceinline__ void unpack2(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
+// Row maximum of 128 values with four independent chains of 3-input max.
+__device__ __forceinline__ float row_max(const uint32_t (&u)[BKV]) {
+  float m[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+  for (int c = 0; c < BKV; c += 8) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) m[i] = max3f(m[i], __uint_as_float(u[c + 2 * i]), __uint_as_float(u[c + 2 * i + 1]));
+  }
+  return fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3]));
+}
+
+// p_c = 2^(s_c * sl2 - m) for the row's 128 scores, packed as bf16 pairs into
+// pk; returns sum_c p_c (fp32, before rounding). The elements are independent.
+__device__ __forceinline__ float row_exp(const uint32_t (&u)[BKV], uint64_t sl2x2, float m, uint32_t (&pk)[BKV / 2]) {
+  const uint64_t negm2 = pair_f32(-m);
+  uint64_t acc[4] = {0, 0, 0, 0};
+#pragma unroll
+  for (int c = 0; c < BKV; c += 2) {
+    float x0, x1;
+    unpack2(fma2(pack2(u[c], u[c + 1]), sl2x2, negm2), x0, x1);
+    const float p0 = ex2(x0), p1 = ex2(x1);
+    const int i = (c >> 1) & 3;
+    acc[i] = add2(acc[i], pack2(__float_as_uint(p0), __float_as_uint(p1)));
+    pk[c >> 1] = pack_bf16x2(p0, p1);
+  }
+  float s0, s1, s2, s3, s4, s5, s6, s7;
+  unpack2(acc[0], s0, s1);
+  unpack2(acc[1], s2, s3);
+  unpack2(acc[2], s4, s5);
+  unpack2(acc[3], s6, s7);
+  return ((s0 + s1) + (s2 + s3)) + ((s4 + s5) + (s6 + s7));
 }
 
 struct AttnArgs {
@@ -159,68 +222,54 @@ __global__ void __launch_bounds__(192, 2)
     const int r = q * 32 + lane;
     const uint32_t trow = tmem + (static_cast<uint32_t>(q * 32) << 16);
     const float sl2 = 1.4426950408889634f * 0.125f;  // log2(e) / sqrt(64)
+    const uint64_t sl2x2 = pair_f32(sl2);
     float m = -INFINITY, l = 0.f;
     bool ok = true;
     for (int j = 0; j < n_kv; ++j) {
       if (!mbar_wait_warp(smem_u32(s_full), j & 1, abort_v, args.status)) { ok = false; break; }
       tc_fence_after();
-      float s[BKV];
-#pragma unroll
-      for (int c = 0; c < BKV; c += 32) {
-        uint32_t u[32];
-        tmem_ld32(trow + kColS + c, u);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) s[c + i] = __uint_as_float(u[i]);
-      }
+      uint32_t u[BKV];
+      tmem_ld128(trow + kColS, u);
       tc_fence_before();
       mbar_arrive(smem_u32(s_free));
 
       const int nvalid = kend - (kbeg + j * BKV);
-      if (nvalid < BKV) {
+      if (nvalid < BKV) {  // last tile of the block: keys past its end get probability 0
 #pragma unroll
         for (int c = 0; c < BKV; ++c)
-          if (c >= nvalid) s[c] = -INFINITY;
+          if (c >= nvalid) u[c] = __float_as_uint(-INFINITY);
       }
-      float mx = s[0];
-#pragma unroll
-      for (int c = 1; c < BKV; ++c) mx = fmaxf(mx, s[c]);
-      const float m_cand = mx * sl2;
+      const float m_cand = row_max(u) * sl2;
       const bool grow = m_cand > m + kRescaleThreshold;
       const float m_new = grow ? m_cand : m;
       const float corr = grow ? ex2(m - m_new) : 1.0f;
-      float sum = 0.f;
-      uint32_t pk[BKV / 2];
-#pragma unroll
-      for (int c = 0; c < BKV; c += 2) {
-        const float p0 = ex2(fmaf(s[c], sl2, -m_new));
-        const float p1 = ex2(fmaf(s[c + 1], sl2, -m_new));
-        sum += p0 + p1;
-        pk[c / 2] = pack_bf16x2(p0, p1);
-      }
-      l = l * corr + sum;
+      const bool any_grow = __any_sync(0xffffffffu, grow);
       m = m_new;
+      uint32_t pk[BKV / 2];
+      const float sum = row_exp(u, sl2x2, m, pk);
+      l = l * corr + sum;
 
       if (j > 0) {
         // PV of the previous tile must be done before O is rescaled and P overwritten
         if (!mbar_wait_warp(smem_u32(o_done), (j - 1) & 1, abort_v, args.status)) { ok = false; break; }
         tc_fence_after();
-        if (__any_sync(0xffffffffu, grow)) {
+        if (any_grow) {
 #pragma unroll
           for (int c = 0; c < DH; c += 32) {
-            uint32_t u[32];
-            tmem_ld32(trow + kColO + c, u);
+            uint32_t o[32];
+            tmem_ld32(trow + kColO + c, o);
 #pragma unroll
-            for (int i = 0; i < 32; ++i) u[i] = __float_as_uint(__uint_as_float(u[i]) * corr);
-            tmem_st32(trow + kColO + c, u);
+            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * corr);
+            tmem_st32(trow + kColO + c, o);
           }
         }
       }
 #pragma unroll
       for (int c = 0; c < BKV / 2; c += 32) {
-        uint32_t u[32];
+        uint32_t w[32];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) u[i] = pk[c + i];
-        tmem_st32(trow + kColP + c, u);
+        for (int i = 0; i < 32; ++i) w[i] = pk[c + i];
+        tmem_st32(trow + kColP + c, w);
       }
       tmem_st_wait();
       tc_fence_before();
@@ -233,16 +282,16 @@ __global__ void __launch_bounds__(192, 2)
       __nv_bfloat16* dst = args.out + static_cast<int64_t>(row) * D + h * DH;
 #pragma unroll
       for (int c = 0; c < DH; c += 32) {
-        uint32_t u[32];
-        tmem_ld32(trow + kColO + c, u);
+        uint32_t o[32];
+        tmem_ld32(trow + kColO + c, o);
         if (row < kend) {
           uint4* d4 = reinterpret_cast<uint4*>(dst + c);
 #pragma unroll
           for (int jj = 0; jj < 4; ++jj)
-            d4[jj] = make_uint4(pack_bf16x2(__uint_as_float(u[8 * jj]) * inv, __uint_as_float(u[8 * jj + 1]) * inv),
-                                pack_bf16x2(__uint_as_float(u[8 * jj + 2]) * inv, __uint_as_float(u[8 * jj + 3]) * inv),
-                                pack_bf16x2(__uint_as_float(u[8 * jj + 4]) * inv, __uint_as_float(u[8 * jj + 5]) * inv),
-                                pack_bf16x2(__uint_as_float(u[8 * jj + 6]) * inv, __uint_as_float(u[8 * jj + 7]) * inv));
+            d4[jj] = make_uint4(pack_bf16x2(__uint_as_float(o[8 * jj]) * inv, __uint_as_float(o[8 * jj + 1]) * inv),
+                                pack_bf16x2(__uint_as_float(o[8 * jj + 2]) * inv, __uint_as_float(o[8 * jj + 3]) * inv),
+                                pack_bf16x2(__uint_as_float(o[8 * jj + 4]) * inv, __uint_as_float(o[8 * jj + 5]) * inv),
+                                pack_bf16x2(__uint_as_float(o[8 * jj + 6]) * inv, __uint_as_float(o[8 * jj + 7]) * inv));
         }
       }
     }

@@ -8,8 +8,12 @@
 //               shared-memory ring of 128-byte-swizzled tiles.
 //   warp 1      allocates TMEM; one thread issues tcgen05.mma (M=128, N=BN,
 //               K=16 per instruction) and commits to mbarriers.
-//   warps 2..5  epilogue: tcgen05.ld of the accumulator (warp w reads TMEM
-//               lanes 32*(w%4)..+31), math, vectorised global stores.
+//   warps 2..5  epilogue: tcgen05.ld of the accumulator (warp w owns TMEM
+//               lanes = tile rows 32*(w%4)..+31), math, then each warp stages
+//               128-byte row chunks of its 32 rows in swizzled shared memory
+//               and writes them with TMA bulk tensor stores (rows past M are
+//               clipped by the tensor map). The fp32 residual of the RESID
+//               epilogue is read with coalesced loads, one chunk ahead.
 // Two TMEM accumulators (2 x BN columns) let the epilogue of tile i overlap the
 // MMAs of tile i+1. Tiles are handed out statically (tile += gridDim.x) over a
 // grid of one CTA per SM. No TMA multicast is used.
@@ -23,6 +27,9 @@ namespace {
 
 constexpr int GBM = 128;
 constexpr int GBK = 64;
+constexpr int kEpiWarps = 4;
+constexpr int kStageBufBytes = 32 * 128;  // one epilogue warp's 32 rows x 128 bytes
+constexpr int kStageBufs = 2;             // per epilogue warp (store of chunk i overlaps chunk i+1)
 
 struct GemmArgs {
   int M, N, K;
@@ -41,9 +48,45 @@ struct GemmShape {
   static constexpr int A_BYTES = GBM * GBK * 2;
   static constexpr int B_BYTES = BN * GBK * 2;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int EPI_BYTES = kEpiWarps * kStageBufs * kStageBufBytes;
   static constexpr int TMEM_COLS = 2 * BN;
   static constexpr int BAR_BYTES = 256;
-  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + BAR_BYTES + 1024;
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + EPI_BYTES + BAR_BYTES + 1024;
+};
+
+// One epilogue warp's pair of staging buffers and its TMA-store bookkeeping.
+struct Stager {
+  uint8_t* base;
+  const CUtensorMap* map;
+  int cur;
+  int lane;
+
+  // Buffer for the next chunk; the bulk store that last read it has finished.
+  __device__ __forceinline__ uint8_t* acquire() {
+    if (lane == 0) bulk_wait_read<kStageBufs - 1>();
+    __syncwarp();
+    return base + cur * kStageBufBytes;
+  }
+  // This lane's 128-byte row (row = lane) into the 128-byte-swizzled buffer.
+  __device__ __forceinline__ void write_row(uint8_t* buf, const uint32_t (&w)[32]) const {
+    uint4* r = reinterpret_cast<uint4*>(buf + lane * 128);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) r[j ^ (lane & 7)] = make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
+  }
+  // Stores the buffer's 32 rows at element (x, y) of the output tensor.
+  __device__ __forceinline__ void commit(uint8_t* buf, int x, int y) {
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+      tma_store_2d(map, smem_u32(buf), x, y);
+      bulk_commit();
+    }
+    cur ^= 1;
+  }
+  __device__ __forceinline__ void drain() {
+    if (lane == 0) bulk_wait<0>();
+    __syncwarp();
+  }
 };
 
 __device__ __forceinline__ float silu_f(float z) { return z / (1.0f + __expf(-z)); }
@@ -55,119 +98,137 @@ __device__ __forceinline__ float act(float v) {
   return v;
 }
 
-// Epilogue of one 128 x BN tile for this thread's row.
+// Epilogue of one 128 x BN tile: this warp's 32 rows (row0 = first of them;
+// this lane's row is row0 + lane), accumulator columns at TMEM address tbase.
 template <int BN, int EPI>
-__device__ __forceinline__ void epilogue_tile(const GemmArgs& args, uint32_t tbase, int row, int n0) {
+__device__ __forceinline__ void epilogue_tile(const GemmArgs& args, Stager& st, uint32_t tbase, int row0, int n0) {
+  const int lane = st.lane;
+  const int row = row0 + lane;
   const bool live = row < args.M;
   if constexpr (EPI == VLM_EPI_BF16 || EPI == VLM_EPI_GELU) {
-    __nv_bfloat16* out = static_cast<__nv_bfloat16*>(args.c) + static_cast<int64_t>(row) * args.N + n0;
 #pragma unroll 1
-    for (int c = 0; c < BN; c += 32) {
-      uint32_t r[32];
-      tmem_ld32(tbase + c, r);
-      if (live) {
-        uint4* dst = reinterpret_cast<uint4*>(out + c);
+    for (int c = 0; c < BN; c += 64) {
+      uint32_t a[32], b[32], w[32];
+      tmem_ld32(tbase + c, a);
+      tmem_ld32(tbase + c + 32, b);
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          uint4 v;
-          v.x = pack_bf16x2(act<EPI>(__uint_as_float(r[8 * j + 0])), act<EPI>(__uint_as_float(r[8 * j + 1])));
-          v.y = pack_bf16x2(act<EPI>(__uint_as_float(r[8 * j + 2])), act<EPI>(__uint_as_float(r[8 * j + 3])));
-          v.z = pack_bf16x2(act<EPI>(__uint_as_float(r[8 * j + 4])), act<EPI>(__uint_as_float(r[8 * j + 5])));
-          v.w = pack_bf16x2(act<EPI>(__uint_as_float(r[8 * j + 6])), act<EPI>(__uint_as_float(r[8 * j + 7])));
-          dst[j] = v;
-        }
+      for (int i = 0; i < 16; ++i) {
+        w[i] = pack_bf16x2(act<EPI>(__uint_as_float(a[2 * i])), act<EPI>(__uint_as_float(a[2 * i + 1])));
+        w[16 + i] = pack_bf16x2(act<EPI>(__uint_as_float(b[2 * i])), act<EPI>(__uint_as_float(b[2 * i + 1])));
       }
+      uint8_t* buf = st.acquire();
+      st.write_row(buf, w);
+      st.commit(buf, n0 + c, row0);
     }
-  } else if constexpr (EPI == VLM_EPI_F32 || EPI == VLM_EPI_RESID) {
-    float* out = static_cast<float*>(args.c) + static_cast<int64_t>(row) * args.N + n0;
-    __nv_bfloat16* outb = args.c_bf16 ? args.c_bf16 + static_cast<int64_t>(row) * args.N + n0 : nullptr;
+  } else if constexpr (EPI == VLM_EPI_F32) {
 #pragma unroll 1
     for (int c = 0; c < BN; c += 32) {
-      uint32_t r[32];
-      tmem_ld32(tbase + c, r);
-      if (live) {
-        float4* dst = reinterpret_cast<float4*>(out + c);
-        float4 v[8];
+      uint32_t a[32];
+      tmem_ld32(tbase + c, a);
+      uint8_t* buf = st.acquire();
+      st.write_row(buf, a);
+      st.commit(buf, n0 + c, row0);
+    }
+  } else if constexpr (EPI == VLM_EPI_RESID) {
+    // x[row, n0 + c ..] += acc: the warp reads the 32 x 32 fp32 residual chunk
+    // with coalesced 16-byte loads (lane -> row 4i + lane/8, 16-byte piece lane%8),
+    // one chunk ahead, and parks it in the staging buffer in swizzled order.
+    const float* x = static_cast<const float*>(args.c);
+    float4 pre[8];
+    auto load_res = [&](int c) {
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          v[j] = make_float4(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]),
-                             __uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3]));
-          if constexpr (EPI == VLM_EPI_RESID) {
-            const float4 o = dst[j];
-            v[j].x += o.x; v[j].y += o.y; v[j].z += o.z; v[j].w += o.w;
-          }
-          dst[j] = v[j];
-        }
-        if (outb != nullptr) {
-          uint4* db = reinterpret_cast<uint4*>(outb + c);
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            uint4 u;
-            u.x = pack_bf16x2(v[2 * j].x, v[2 * j].y);
-            u.y = pack_bf16x2(v[2 * j].z, v[2 * j].w);
-            u.z = pack_bf16x2(v[2 * j + 1].x, v[2 * j + 1].y);
-            u.w = pack_bf16x2(v[2 * j + 1].z, v[2 * j + 1].w);
-            db[j] = u;
-          }
-        }
+      for (int i = 0; i < 8; ++i) {
+        const int r = row0 + 4 * i + (lane >> 3);
+        pre[i] = r < args.M ? __ldg(reinterpret_cast<const float4*>(x + static_cast<int64_t>(r) * args.N + n0 + c) +
+                                    (lane & 7))
+                            : make_float4(0.f, 0.f, 0.f, 0.f);
       }
+    };
+    load_res(0);
+#pragma unroll 1
+    for (int c = 0; c < BN; c += 32) {
+      uint8_t* buf = st.acquire();
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int r = 4 * i + (lane >> 3), ch = lane & 7;
+        *reinterpret_cast<float4*>(buf + r * 128 + ((ch ^ (r & 7)) << 4)) = pre[i];
+      }
+      if (c + 32 < BN) load_res(c + 32);
+      uint32_t a[32];
+      tmem_ld32(tbase + c, a);
+      __syncwarp();
+      float4* rp = reinterpret_cast<float4*>(buf + lane * 128);
+      float v[32];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        float4 o = rp[j ^ (lane & 7)];
+        o.x += __uint_as_float(a[4 * j]);
+        o.y += __uint_as_float(a[4 * j + 1]);
+        o.z += __uint_as_float(a[4 * j + 2]);
+        o.w += __uint_as_float(a[4 * j + 3]);
+        rp[j ^ (lane & 7)] = o;
+        v[4 * j] = o.x; v[4 * j + 1] = o.y; v[4 * j + 2] = o.z; v[4 * j + 3] = o.w;
+      }
+      if (args.c_bf16 != nullptr && live) {
+        uint4* db = reinterpret_cast<uint4*>(args.c_bf16 + static_cast<int64_t>(row) * args.N + n0 + c);
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          db[j] = make_uint4(pack_bf16x2(v[8 * j], v[8 * j + 1]), pack_bf16x2(v[8 * j + 2], v[8 * j + 3]),
+                             pack_bf16x2(v[8 * j + 4], v[8 * j + 5]), pack_bf16x2(v[8 * j + 6], v[8 * j + 7]));
+      }
+      st.commit(buf, n0 + c, row0);
     }
   } else if constexpr (EPI == VLM_EPI_SWIGLU) {
-    // columns 32j..32j+15 are gate, 32j+16..32j+31 the matching up values
-    __nv_bfloat16* out = static_cast<__nv_bfloat16*>(args.c) + static_cast<int64_t>(row) * (args.N / 2) + n0 / 2;
+    // accumulator columns 32g..32g+15 are gate, 32g+16..32g+31 the matching up
+    // values of output columns 16g..16g+15; a 128-column chunk gives 64 outputs
 #pragma unroll 1
-    for (int c = 0; c < BN; c += 32) {
-      uint32_t r[32];
-      tmem_ld32(tbase + c, r);
-      if (live) {
-        uint4* dst = reinterpret_cast<uint4*>(out + c / 2);
+    for (int c = 0; c < BN; c += 128) {
+      uint32_t w[32];
 #pragma unroll
-        for (int j = 0; j < 2; ++j) {
-          uint32_t w[4];
+      for (int g = 0; g < 4; ++g) {
+        uint32_t r[32];
+        tmem_ld32(tbase + c + 32 * g, r);
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int i = 8 * j + 2 * e;
-            const float h0 = silu_f(__uint_as_float(r[i])) * __uint_as_float(r[16 + i]);
-            const float h1 = silu_f(__uint_as_float(r[i + 1])) * __uint_as_float(r[16 + i + 1]);
-            w[e] = pack_bf16x2(h0, h1);
-          }
-          dst[j] = make_uint4(w[0], w[1], w[2], w[3]);
+        for (int e = 0; e < 8; ++e) {
+          const float h0 = silu_f(__uint_as_float(r[2 * e])) * __uint_as_float(r[16 + 2 * e]);
+          const float h1 = silu_f(__uint_as_float(r[2 * e + 1])) * __uint_as_float(r[16 + 2 * e + 1]);
+          w[8 * g + e] = pack_bf16x2(h0, h1);
         }
       }
+      uint8_t* buf = st.acquire();
+      st.write_row(buf, w);
+      st.commit(buf, (n0 + c) / 2, row0);
     }
   } else if constexpr (EPI == VLM_EPI_ROPE) {
-    __nv_bfloat16* out = static_cast<__nv_bfloat16*>(args.c) + static_cast<int64_t>(row) * args.N + n0;
     const int pk = live ? __ldg(args.pos + row) : 0;
     const int pr = pk >> 16, pc = pk & 0xFFFF;
 #pragma unroll 1
     for (int c = 0; c < BN; c += 64) {
-      uint32_t a[32], b[32];
+      uint32_t a[32], b[32], w[32];
       tmem_ld32(tbase + c, a);
       tmem_ld32(tbase + c + 32, b);
-      if (live) {
-        float x[32], y[32];
+      float x[32], y[32];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) { x[i] = __uint_as_float(a[i]); y[i] = __uint_as_float(b[i]); }
-        if (n0 + c < args.rope_cols) {
-          const float2* tr = args.rope + pr * 32;
-          const float2* tc = args.rope + pc * 32;
+      for (int i = 0; i < 32; ++i) { x[i] = __uint_as_float(a[i]); y[i] = __uint_as_float(b[i]); }
+      if (n0 + c < args.rope_cols) {
+        const float2* tr = args.rope + pr * 32;
+        const float2* tc = args.rope + pc * 32;
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const float2 cs = __ldg(i < 16 ? tr + i : tc + i);
-            const float xi = x[i], yi = y[i];
-            x[i] = xi * cs.x - yi * cs.y;
-            y[i] = yi * cs.x + xi * cs.y;
-          }
-        }
-        uint4* dst = reinterpret_cast<uint4*>(out + c);
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          dst[j] = make_uint4(pack_bf16x2(x[8 * j], x[8 * j + 1]), pack_bf16x2(x[8 * j + 2], x[8 * j + 3]),
-                              pack_bf16x2(x[8 * j + 4], x[8 * j + 5]), pack_bf16x2(x[8 * j + 6], x[8 * j + 7]));
-          dst[4 + j] = make_uint4(pack_bf16x2(y[8 * j], y[8 * j + 1]), pack_bf16x2(y[8 * j + 2], y[8 * j + 3]),
-                                  pack_bf16x2(y[8 * j + 4], y[8 * j + 5]), pack_bf16x2(y[8 * j + 6], y[8 * j + 7]));
+        for (int i = 0; i < 32; ++i) {
+          const float2 cs = __ldg(i < 16 ? tr + i : tc + i);
+          const float xi = x[i], yi = y[i];
+          x[i] = xi * cs.x - yi * cs.y;
+          y[i] = yi * cs.x + xi * cs.y;
         }
       }
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        w[i] = pack_bf16x2(x[2 * i], x[2 * i + 1]);
+        w[16 + i] = pack_bf16x2(y[2 * i], y[2 * i + 1]);
+      }
+      uint8_t* buf = st.acquire();
+      st.write_row(buf, w);
+      st.commit(buf, n0 + c, row0);
     }
   }
 }
@@ -175,13 +236,14 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& args, uint32_t tba
 template <int BN, int EPI>
 __global__ void __launch_bounds__(192, 1)
     gemm_tcgen05_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                        const GemmArgs args) {
+                        const __grid_constant__ CUtensorMap tmC, const GemmArgs args) {
   using S = GemmShape<BN>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
   uint8_t* sB = smem + S::STAGES * S::A_BYTES;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::STAGES * S::STAGE_BYTES);
+  uint8_t* sEpi = smem + S::STAGES * S::STAGE_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sEpi + S::EPI_BYTES);
   uint64_t* full = bars;
   uint64_t* empty = bars + S::STAGES;
   uint64_t* tfull = bars + 2 * S::STAGES;
@@ -208,6 +270,7 @@ __global__ void __launch_bounds__(192, 1)
   if (warp == 0 && lane == 0) {
     prefetch_tmap(&tmA);
     prefetch_tmap(&tmB);
+    prefetch_tmap(&tmC);
   }
   if (warp == 1) {
     tmem_alloc(smem_u32(tmem_slot), S::TMEM_COLS);
@@ -269,20 +332,21 @@ __global__ void __launch_bounds__(192, 1)
     }
   } else {
     const int q = warp & 3;  // TMEM lane quadrant this warp may access
+    Stager st{sEpi + (warp - 2) * kStageBufs * kStageBufBytes, &tmC, 0, lane};
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x) {
       const int mt = tile / args.n_tiles, nt = tile - mt * args.n_tiles;
       if (!mbar_wait_warp(smem_u32(tfull + acc), acc_phase, abort_v, args.status)) break;
       tc_fence_after();
-      const int row = mt * GBM + q * 32 + lane;
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * BN);
-      epilogue_tile<BN, EPI>(args, tbase, row, nt * BN);
+      epilogue_tile<BN, EPI>(args, st, tbase, mt * GBM + q * 32, nt * BN);
       tc_fence_before();
       mbar_arrive(smem_u32(tempty + acc));
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1u;
     }
+    st.drain();
   }
 
   tc_fence_before();
@@ -294,7 +358,8 @@ __global__ void __launch_bounds__(192, 1)
 }
 
 template <int BN, int EPI>
-int run_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const GemmArgs& args, cudaStream_t s) {
+int run_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tc, const GemmArgs& args,
+             cudaStream_t s) {
   using S = GemmShape<BN>;
   auto kern = gemm_tcgen05_kernel<BN, EPI>;
   static bool attr_done[64] = {};
@@ -308,20 +373,21 @@ int run_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const GemmArgs& args,
   const int tiles = args.m_tiles * args.n_tiles;
   const int grid = tiles < num_sms() ? tiles : num_sms();
   launch_begin(KC_GEMM, s);
-  kern<<<grid, 192, S::SMEM_BYTES, s>>>(ta, tb, args);
+  kern<<<grid, 192, S::SMEM_BYTES, s>>>(ta, tb, tc, args);
   launch_end(KC_GEMM, s);
   return cudaGetLastError() == cudaSuccess ? VLM_OK : VLM_ERR_CUDA;
 }
 
 template <int BN>
-int dispatch_epi(int epi, const CUtensorMap& ta, const CUtensorMap& tb, const GemmArgs& args, cudaStream_t s) {
+int dispatch_epi(int epi, const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tc, const GemmArgs& args,
+                 cudaStream_t s) {
   switch (epi) {
-    case VLM_EPI_BF16: return run_gemm<BN, VLM_EPI_BF16>(ta, tb, args, s);
-    case VLM_EPI_F32: return run_gemm<BN, VLM_EPI_F32>(ta, tb, args, s);
-    case VLM_EPI_RESID: return run_gemm<BN, VLM_EPI_RESID>(ta, tb, args, s);
-    case VLM_EPI_SWIGLU: return run_gemm<BN, VLM_EPI_SWIGLU>(ta, tb, args, s);
-    case VLM_EPI_ROPE: return run_gemm<BN, VLM_EPI_ROPE>(ta, tb, args, s);
-    case VLM_EPI_GELU: return run_gemm<BN, VLM_EPI_GELU>(ta, tb, args, s);
+    case VLM_EPI_BF16: return run_gemm<BN, VLM_EPI_BF16>(ta, tb, tc, args, s);
+    case VLM_EPI_F32: return run_gemm<BN, VLM_EPI_F32>(ta, tb, tc, args, s);
+    case VLM_EPI_RESID: return run_gemm<BN, VLM_EPI_RESID>(ta, tb, tc, args, s);
+    case VLM_EPI_SWIGLU: return run_gemm<BN, VLM_EPI_SWIGLU>(ta, tb, tc, args, s);
+    case VLM_EPI_ROPE: return run_gemm<BN, VLM_EPI_ROPE>(ta, tb, tc, args, s);
+    case VLM_EPI_GELU: return run_gemm<BN, VLM_EPI_GELU>(ta, tb, tc, args, s);
     default: return VLM_ERR_INVALID_ARG;
   }
 }
@@ -342,18 +408,24 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
 }
 }  // namespace
 
-bool make_tmap_2d_bf16(CUtensorMap* map, const void* ptr, uint64_t inner, uint64_t outer, uint64_t row_bytes,
-                       uint32_t box_inner, uint32_t box_outer) {
+bool make_tmap_2d(CUtensorMap* map, const void* ptr, bool fp32, uint64_t inner, uint64_t outer, uint64_t row_bytes,
+                  uint32_t box_inner, uint32_t box_outer) {
   auto enc = tensor_map_encoder();
   if (enc == nullptr) return false;
   cuuint64_t dims[2] = {inner, outer};
   cuuint64_t strides[1] = {row_bytes};
   cuuint32_t box[2] = {box_inner, box_outer};
   cuuint32_t estr[2] = {1, 1};
-  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box,
-                         estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  const CUresult r =
+      enc(map, fp32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr),
+          dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
+}
+
+bool make_tmap_2d_bf16(CUtensorMap* map, const void* ptr, uint64_t inner, uint64_t outer, uint64_t row_bytes,
+                       uint32_t box_inner, uint32_t box_outer) {
+  return make_tmap_2d(map, ptr, false, inner, outer, row_bytes, box_inner, box_outer);
 }
 
 int launch_gemm(int epi, const void* a, const void* b, int64_t M, int64_t N, int64_t K, void* c, void* c_bf16,
@@ -367,11 +439,17 @@ int launch_gemm(int epi, const void* a, const void* b, int64_t M, int64_t N, int
   if (epi == VLM_EPI_ROPE && (pos == nullptr || rope == nullptr || rope_cols % 64 != 0)) return VLM_ERR_INVALID_ARG;
   if ((reinterpret_cast<uintptr_t>(a) | reinterpret_cast<uintptr_t>(b) | reinterpret_cast<uintptr_t>(c)) & 15)
     return VLM_ERR_INVALID_ARG;
-  const int bn = (needs256 || (N % 256 == 0 && N >= 2048)) ? 256 : 128;
+  const int bn = N % 256 == 0 ? 256 : 128;
 
   CUtensorMap ta, tb;
   if (!make_tmap_2d_bf16(&ta, a, K, M, K * 2, GBK, GBM)) return VLM_ERR_CUDA;
   if (!make_tmap_2d_bf16(&tb, b, K, N, K * 2, GBK, bn)) return VLM_ERR_CUDA;
+  // output: 32-row boxes of 128 bytes (64 bf16 or 32 fp32 columns)
+  CUtensorMap tc;
+  const bool out_f32 = epi == VLM_EPI_F32 || epi == VLM_EPI_RESID;
+  const uint64_t out_cols = epi == VLM_EPI_SWIGLU ? N / 2 : N;
+  if (!make_tmap_2d(&tc, c, out_f32, out_cols, M, out_cols * (out_f32 ? 4 : 2), out_f32 ? 32 : 64, 32))
+    return VLM_ERR_CUDA;
 
   GemmArgs args;
   args.M = static_cast<int>(M);
@@ -385,7 +463,7 @@ int launch_gemm(int epi, const void* a, const void* b, int64_t M, int64_t N, int
   args.rope = rope;
   args.rope_cols = static_cast<int>(rope_cols);
   args.status = status;
-  return bn == 256 ? dispatch_epi<256>(epi, ta, tb, args, s) : dispatch_epi<128>(epi, ta, tb, args, s);
+  return bn == 256 ? dispatch_epi<256>(epi, ta, tb, tc, args, s) : dispatch_epi<128>(epi, ta, tb, tc, args, s);
 }
 
 }  // namespace vlm

@@ -53,7 +53,11 @@ int launch_pack_gate_up(const void* gate, const void* up, void* dst, int64_t f, 
 int launch_pack_cols(const void* src, void* dst, int64_t rows, int64_t src_cols, int64_t dst_cols, int mode,
                      int mm, cudaStream_t s);
 int launch_f32_to_bf16(const float* x, __nv_bfloat16* y, int64_t n, cudaStream_t s);
+int launch_wait_timeout_selftest(long long budget_cycles, int32_t* status, cudaStream_t s);
 
+// 2D tensor map (bf16 or fp32 elements), 128-byte swizzle, box box_outer x box_inner.
+bool make_tmap_2d(CUtensorMap* map, const void* ptr, bool fp32, uint64_t inner, uint64_t outer, uint64_t row_bytes,
+                  uint32_t box_inner, uint32_t box_outer);
 // 2D bf16 tensor map, 128-byte swizzle, box box_outer x box_inner (box_inner * 2 == 128 bytes).
 bool make_tmap_2d_bf16(CUtensorMap* map, const void* ptr, uint64_t inner, uint64_t outer, uint64_t row_bytes,
                        uint32_t box_inner, uint32_t box_outer);

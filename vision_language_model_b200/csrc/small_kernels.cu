@@ -465,3 +465,38 @@ int launch_f32_to_bf16(const float* x, __nv_bfloat16* y, int64_t n, cudaStream_t
 }
 
 }  // namespace vlm
+
+namespace vlm {
+
+// ---------------------------------------------------------------------------
+// Self-test of the bounded barrier wait: one thread waits on an mbarrier that
+// nothing arrives on, with a budget of `budget_cycles`, exactly as the GEMM and
+// attention roles wait on theirs; the wait must give up, record
+// VLM_ERR_TIMEOUT in *status and let the kernel return normally.
+// ---------------------------------------------------------------------------
+__global__ void wait_timeout_selftest_kernel(long long budget_cycles, int32_t* status) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x != 0) return;
+  mbar_init(smem_u32(&bar), 1);
+  fence_mbar_init();
+  const uint32_t b = smem_u32(&bar);
+  // the phase of parity 0 never completes: nobody arrives
+  if (mbar_try_wait(b, 0)) return;
+  const long long t0 = clock64();
+  for (uint32_t i = 1;; ++i) {
+    if (mbar_try_wait(b, 0)) return;
+    if ((i & 255u) == 0 && clock64() - t0 > budget_cycles) {
+      set_status(status, VLM_ERR_TIMEOUT);
+      return;
+    }
+  }
+}
+
+int launch_wait_timeout_selftest(long long budget_cycles, int32_t* status, cudaStream_t s) {
+  launch_begin(KC_SETUP, s);
+  wait_timeout_selftest_kernel<<<1, 32, 0, s>>>(budget_cycles, status);
+  launch_end(KC_SETUP, s);
+  return cudaGetLastError() == cudaSuccess ? VLM_OK : VLM_ERR_CUDA;
+}
+
+}  // namespace vlm

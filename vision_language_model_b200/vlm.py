@@ -85,6 +85,7 @@ def lib() -> ctypes.CDLL:
             "vlm_attention_workspace_size": (SZ, [I32]),
             "vlm_attention": (I32, [P, I64, I32, I32, P, I32, P, P, SZ, P, P]),
             "vlm_rmsnorm": (I32, [P, P, P, P, I64, I32, F, P]),
+            "vlm_selftest_wait_timeout": (I32, [I64, P, P]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -317,6 +318,11 @@ def rmsnorm(x: torch.Tensor, g1: torch.Tensor, g0=None, eps: float = 1e-5, out=N
     _check(lib().vlm_rmsnorm(_dev(x, "x"), _dev(g0, "g0"), _dev(g1, "g1"), _dev(out, "out"), rows, width, float(eps),
                              _stream(stream)), "vlm_rmsnorm")
     return out
+
+
+def selftest_wait_timeout(budget_cycles: int, status: torch.Tensor, stream=None) -> None:
+    _check(lib().vlm_selftest_wait_timeout(int(budget_cycles), _dev(status, "status"), _stream(stream)),
+           "vlm_selftest_wait_timeout")
 
 
 # ---------------------------------------------------------------------------
