@@ -23,6 +23,7 @@
 // Keys past the block end are masked to -inf; their V rows are finite (rows of
 // the next block) or TMA zero fill (past the sequence). Query tiles never
 // straddle two blocks, so every block's result is independent of the others.
+#include "exp2_poly.cuh"
 #include "kernels.cuh"
 
 namespace vlm {
@@ -82,16 +83,59 @@ __device__ __forceinline__ float row_max(const uint32_t (&u)[BKV]) {
   return fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3]));
 }
 
+__device__ __forceinline__ uint64_t sub2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("sub.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
+// One pair of scores in kPolyPairEvery takes its two exponentials from
+// exp2_poly2 (FMA and ALU pipes) instead of ex2.approx (MUFU), so the two
+// kinds of pipe share the softmax's exponentials.
+#ifndef VLM_ATTN_POLY_PAIR_EVERY
+#define VLM_ATTN_POLY_PAIR_EVERY 0
+#endif
+constexpr int kPolyPairEvery = VLM_ATTN_POLY_PAIR_EVERY;
+
+// (2^x0, 2^x1) without MUFU: k = round(x) by adding 1.5 * 2^23, f = x - k in
+// [-1/2, 1/2], 2^f from the degree-3 minimax polynomial of exp2_poly.cuh
+// (relative error < 7.5e-5, fitted by fit_exp2_poly.py with the Remez
+// algorithm), then k added to the exponent field; packed fp32x2 arithmetic.
+// x is clamped to -126 so the exponent cannot wrap; the result is then ~1e-38
+// instead of 0, so keys that must weigh exactly 0 never take this path.
+__device__ __forceinline__ void exp2_poly2(float x0, float x1, float& p0, float& p1) {
+  const uint64_t x = pack2(__float_as_uint(fmaxf(x0, -126.0f)), __float_as_uint(fmaxf(x1, -126.0f)));
+  const uint64_t magic = pair_f32(12582912.0f);
+  const uint64_t j = add2(x, magic);
+  const uint64_t f = sub2(x, sub2(j, magic));
+  uint64_t p = fma2(pair_f32(kExp2C3), f, pair_f32(kExp2C2));
+  p = fma2(p, f, pair_f32(kExp2C1));
+  p = fma2(p, f, pair_f32(kExp2C0));
+  float pl, ph, jl, jh;
+  unpack2(p, pl, ph);
+  unpack2(j, jl, jh);
+  p0 = __int_as_float(__float_as_int(pl) + (__float_as_int(jl) << 23));
+  p1 = __int_as_float(__float_as_int(ph) + (__float_as_int(jh) << 23));
+}
+
 // p_c = 2^(s_c * sl2 - m) for the row's 128 scores, packed as bf16 pairs into
 // pk; returns sum_c p_c (fp32, before rounding). The elements are independent.
+// kPoly: let exp2_poly2 take one pair in kPolyPairEvery (never on a tile with
+// masked keys, whose weights must be exactly 0).
+template <bool kPoly>
 __device__ __forceinline__ float row_exp(const uint32_t (&u)[BKV], uint64_t sl2x2, float m, uint32_t (&pk)[BKV / 2]) {
   const uint64_t negm2 = pair_f32(-m);
   uint64_t acc[4] = {0, 0, 0, 0};
 #pragma unroll
   for (int c = 0; c < BKV; c += 2) {
-    float x0, x1;
+    float x0, x1, p0, p1;
     unpack2(fma2(pack2(u[c], u[c + 1]), sl2x2, negm2), x0, x1);
-    const float p0 = ex2(x0), p1 = ex2(x1);
+    if (kPoly && kPolyPairEvery > 0 && (c >> 1) % (kPolyPairEvery > 0 ? kPolyPairEvery : 1) == kPolyPairEvery - 1) {
+      exp2_poly2(x0, x1, p0, p1);
+    } else {
+      p0 = ex2(x0);
+      p1 = ex2(x1);
+    }
     const int i = (c >> 1) & 3;
     acc[i] = add2(acc[i], pack2(__float_as_uint(p0), __float_as_uint(p1)));
     pk[c >> 1] = pack_bf16x2(p0, p1);
@@ -246,7 +290,7 @@ __global__ void __launch_bounds__(192, 2)
       const bool any_grow = __any_sync(0xffffffffu, grow);
       m = m_new;
       uint32_t pk[BKV / 2];
-      const float sum = row_exp(u, sl2x2, m, pk);
+      const float sum = nvalid < BKV ? row_exp<false>(u, sl2x2, m, pk) : row_exp<true>(u, sl2x2, m, pk);
       l = l * corr + sum;
 
       if (j > 0) {
