@@ -298,12 +298,14 @@ def ncu_traffic(kernel: str) -> float | None:
     with open(path) as fh:
         table = json.load(fh)
     ent = table.get(kernel)
-    if not ent or ent.get("source_hash") != source_hash(*ent.get("sources", [])):
+    if not ent or ent.get("bytes_per_launch") is None:
         return None
+    if ent.get("source_hash") != source_hash(*ent.get("sources", [])):
+        return None  # the kernel changed since the counters were taken
     return float(ent["bytes_per_launch"])
 
 
-KERNEL_SOURCES = {"attention": ["attention_mma.cu", "common.cuh", "kernels.cuh"],
+KERNEL_SOURCES = {"attention": ["attention_tc.cu", "exp2_poly.cuh", "common.cuh", "kernels.cuh"],
                   "gemm": ["gemm_tcgen05.cu", "common.cuh", "kernels.cuh"]}
 
 
