@@ -73,12 +73,18 @@ struct Stager {
 #pragma unroll
     for (int j = 0; j < 8; ++j) r[j ^ (lane & 7)] = make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
   }
-  // Stores the buffer's 32 rows at element (x, y) of the output tensor.
+  // Stores the buffer's 32 rows at element (x, y) of the output tensor, or
+  // (reduce) adds them to what is there.
+  template <bool kReduce = false>
   __device__ __forceinline__ void commit(uint8_t* buf, int x, int y) {
     fence_proxy_async_smem();
     __syncwarp();
     if (lane == 0) {
-      tma_store_2d(map, smem_u32(buf), x, y);
+      if constexpr (kReduce) {
+        tma_reduce_add_2d(map, smem_u32(buf), x, y);
+      } else {
+        tma_store_2d(map, smem_u32(buf), x, y);
+      }
       bulk_commit();
     }
     cur ^= 1;
@@ -89,7 +95,13 @@ struct Stager {
   }
 };
 
-__device__ __forceinline__ float silu_f(float z) { return z / (1.0f + __expf(-z)); }
+// silu(z) = z / (1 + e^-z) with MUFU ex2 and rcp (about 1 ulp each); z -> -inf gives -0.
+__device__ __forceinline__ float silu_f(float z) {
+  float e, r;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e) : "f"(z * -1.4426950408889634f));
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(1.0f + e));
+  return z * r;
+}
 __device__ __forceinline__ float gelu_f(float z) { return 0.5f * z * (1.0f + erff(z * 0.70710678118654752f)); }
 
 template <int EPI>
@@ -130,6 +142,19 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& args, Stager& st, 
       st.commit(buf, n0 + c, row0);
     }
   } else if constexpr (EPI == VLM_EPI_RESID) {
+    if (args.c_bf16 == nullptr) {
+      // x[row, n0 + c ..] += acc by a bulk tensor reduce-add: no residual reads on the SM
+#pragma unroll 1
+      for (int c = 0; c < BN; c += 32) {
+        uint32_t a[32];
+        tmem_ld32(tbase + c, a);
+        uint8_t* buf = st.acquire();
+        st.write_row(buf, a);
+        st.template commit<true>(buf, n0 + c, row0);
+      }
+      return;
+    }
+    // with the bf16 copy the new values are needed here: read the residual.
     // x[row, n0 + c ..] += acc: the warp reads the 32 x 32 fp32 residual chunk
     // with coalesced 16-byte loads (lane -> row 4i + lane/8, 16-byte piece lane%8),
     // one chunk ahead, and parks it in the staging buffer in swizzled order.
@@ -357,6 +382,191 @@ __global__ void __launch_bounds__(192, 1)
   }
 }
 
+// ---------------------------------------------------------------------------
+// Two-SM variant (N % 256 == 0): a cluster of two CTAs computes a 256 x 256
+// tile with tcgen05.mma.cta_group::2 (M = 256). Each CTA stages its own 128
+// rows of A and its own half (128 rows) of the B tile, so per k-block an SM
+// reads 32 KiB instead of 48 KiB; the even CTA issues the MMAs and both CTAs'
+// TMEM receive their 128 x 256 accumulator rows. Both CTAs run the same
+// producer (TMA completion counted on the even CTA's barrier) and epilogue;
+// the odd CTA's epilogue hands the accumulator back with a remote arrive.
+// ---------------------------------------------------------------------------
+struct PairShape {
+  static constexpr int BN = 256;
+  static constexpr int STAGES = 6;
+  static constexpr int A_BYTES = GBM * GBK * 2;         // this CTA's 128 rows of A
+  static constexpr int B_BYTES = (BN / 2) * GBK * 2;    // this CTA's 128 rows of B
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int EPI_BYTES = kEpiWarps * kStageBufs * kStageBufBytes;
+  static constexpr int TMEM_COLS = 2 * BN;
+  static constexpr int BAR_BYTES = 256;
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + EPI_BYTES + BAR_BYTES + 1024;
+};
+
+template <int EPI>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
+    gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                     const __grid_constant__ CUtensorMap tmC, const GemmArgs args) {
+  using S = PairShape;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + S::STAGES * S::A_BYTES;
+  uint8_t* sEpi = smem + S::STAGES * S::STAGE_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sEpi + S::EPI_BYTES);
+  uint64_t* full = bars;                     // used on the even CTA
+  uint64_t* empty = bars + S::STAGES;        // both CTAs
+  uint64_t* tfull = bars + 2 * S::STAGES;    // both CTAs
+  uint64_t* tempty = tfull + 2;              // used on the even CTA (8 warp arrivals)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
+  int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const int pair = blockIdx.x >> 1, n_pairs = gridDim.x >> 1;
+  const int total_tiles = args.m_tiles * args.n_tiles;  // m_tiles counts 256-row pair tiles here
+  const int nk = args.K / GBK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S::STAGES; ++s) {
+      mbar_init(smem_u32(full + s), 1);
+      mbar_init(smem_u32(empty + s), 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(smem_u32(tfull + a), 1);
+      mbar_init(smem_u32(tempty + a), 2 * kEpiWarps);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tmA);
+    prefetch_tmap(&tmB);
+    prefetch_tmap(&tmC);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(smem_u32(tmem_slot), S::TMEM_COLS);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();  // both CTAs' barriers are initialised before any cross-CTA signal
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  volatile int* abort_v = abort_flag;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int tile = pair; tile < total_tiles && ok; tile += n_pairs) {
+        const int mt = tile / args.n_tiles, nt = tile - mt * args.n_tiles;
+        const int arow = mt * 256 + static_cast<int>(rank) * GBM;
+        const int brow = nt * S::BN + static_cast<int>(rank) * (S::BN / 2);
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!mbar_wait(smem_u32(empty + stage), phase ^ 1u, abort_v, args.status)) { ok = false; break; }
+          const uint32_t fb = smem_u32(full + stage) & kPeerBitMask;
+          if (rank == 0) mbar_arrive_expect_tx(smem_u32(full + stage), 2 * S::STAGE_BYTES);
+          tma_load_2d_pair(smem_u32(sA + stage * S::A_BYTES), &tmA, fb, kb * GBK, arow);
+          tma_load_2d_pair(smem_u32(sB + stage * S::B_BYTES), &tmB, fb, kb * GBK, brow);
+          if (++stage == S::STAGES) { stage = 0; phase ^= 1u; }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (rank == 0 && lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16(2 * GBM, S::BN);
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      for (int tile = pair; tile < total_tiles && ok; tile += n_pairs) {
+        if (!mbar_wait_cluster(smem_u32(tempty + acc), acc_phase ^ 1u, abort_v, args.status)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * S::BN);
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!mbar_wait(smem_u32(full + stage), phase, abort_v, args.status)) { ok = false; break; }
+          tc_fence_after();
+          const uint64_t adesc = smem_desc_sw128(smem_u32(sA + stage * S::A_BYTES));
+          const uint64_t bdesc = smem_desc_sw128(smem_u32(sB + stage * S::B_BYTES));
+#pragma unroll
+          for (int k = 0; k < GBK / 16; ++k)
+            umma_bf16_ss_pair(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, (kb | k) != 0 ? 1u : 0u);
+          umma_commit_pair_mc(smem_u32(empty + stage), 0x3);
+          if (++stage == S::STAGES) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        umma_commit_pair_mc(smem_u32(tfull + acc), 0x3);
+        acc ^= 1;
+        if (acc == 0) acc_phase ^= 1u;
+      }
+    }
+  } else {
+    const int q = warp & 3;  // TMEM lane quadrant this warp may access
+    Stager st{sEpi + (warp - 2) * kStageBufs * kStageBufBytes, &tmC, 0, lane};
+    const uint32_t leader_tempty = mapa_shared(smem_u32(tempty), 0);
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int tile = pair; tile < total_tiles; tile += n_pairs) {
+      const int mt = tile / args.n_tiles, nt = tile - mt * args.n_tiles;
+      if (!mbar_wait_warp(smem_u32(tfull + acc), acc_phase, abort_v, args.status)) break;
+      tc_fence_after();
+      const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * S::BN);
+      epilogue_tile<S::BN, EPI>(args, st, tbase, mt * 256 + static_cast<int>(rank) * GBM + q * 32, nt * S::BN);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(leader_tempty + static_cast<uint32_t>(acc * 8));
+      acc ^= 1;
+      if (acc == 0) acc_phase ^= 1u;
+    }
+    st.drain();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();  // neither CTA leaves while its pair may still signal or read it
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, S::TMEM_COLS);
+  }
+}
+
+template <int EPI>
+int run_gemm_pair(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tc, const GemmArgs& args,
+                  cudaStream_t s) {
+  auto kern = gemm_pair_kernel<EPI>;
+  static bool attr_done[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !attr_done[dev]) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, PairShape::SMEM_BYTES) !=
+        cudaSuccess)
+      return VLM_ERR_CUDA;
+    attr_done[dev] = true;
+  }
+  const int tiles = args.m_tiles * args.n_tiles;
+  const int pairs = tiles < num_sms() / 2 ? tiles : num_sms() / 2;
+  launch_begin(KC_GEMM, s);
+  kern<<<2 * pairs, 192, PairShape::SMEM_BYTES, s>>>(ta, tb, tc, args);
+  launch_end(KC_GEMM, s);
+  return cudaGetLastError() == cudaSuccess ? VLM_OK : VLM_ERR_CUDA;
+}
+
+int dispatch_pair(int epi, const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tc, const GemmArgs& args,
+                  cudaStream_t s) {
+  switch (epi) {
+    case VLM_EPI_BF16: return run_gemm_pair<VLM_EPI_BF16>(ta, tb, tc, args, s);
+    case VLM_EPI_F32: return run_gemm_pair<VLM_EPI_F32>(ta, tb, tc, args, s);
+    case VLM_EPI_RESID: return run_gemm_pair<VLM_EPI_RESID>(ta, tb, tc, args, s);
+    case VLM_EPI_SWIGLU: return run_gemm_pair<VLM_EPI_SWIGLU>(ta, tb, tc, args, s);
+    case VLM_EPI_ROPE: return run_gemm_pair<VLM_EPI_ROPE>(ta, tb, tc, args, s);
+    case VLM_EPI_GELU: return run_gemm_pair<VLM_EPI_GELU>(ta, tb, tc, args, s);
+    default: return VLM_ERR_INVALID_ARG;
+  }
+}
+
 template <int BN, int EPI>
 int run_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tc, const GemmArgs& args,
              cudaStream_t s) {
@@ -463,7 +673,14 @@ int launch_gemm(int epi, const void* a, const void* b, int64_t M, int64_t N, int
   args.rope = rope;
   args.rope_cols = static_cast<int>(rope_cols);
   args.status = status;
-  return bn == 256 ? dispatch_epi<256>(epi, ta, tb, tc, args, s) : dispatch_epi<128>(epi, ta, tb, tc, args, s);
+  if (bn == 256) {
+    // two-SM pairs: 256-row tiles of A (128 per CTA) and 128-row halves of the B tile
+    CUtensorMap tb2;
+    if (!make_tmap_2d_bf16(&tb2, b, K, N, K * 2, GBK, 128)) return VLM_ERR_CUDA;
+    args.m_tiles = static_cast<int>((M + 255) / 256);
+    return dispatch_pair(epi, ta, tb2, tc, args, s);
+  }
+  return dispatch_epi<128>(epi, ta, tb, tc, args, s);
 }
 
 }  // namespace vlm
