@@ -171,12 +171,19 @@ def barrier(world):
 
 
 def max_over_ranks(world, value: float) -> float:
+    """The largest of the ranks' values (every rank gets it)."""
     if world == 1:
         return value
     import torch.distributed as dist
-    t = torch.tensor([value], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([value], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_throughput(units_per_rank: int, world: int, steps: int, ms_max: float) -> float:
+    """Whole-job units per second: every rank's units over the slowest rank's time."""
+    return units_per_rank * world * steps / (ms_max / 1000.0)
 
 
 # ---------------------------------------------------------------------------
@@ -396,7 +403,7 @@ def run_ours(args, wl):
     e_ms = max_over_ranks(world, e_start.elapsed_time(e_stop))
 
     peaks = measured_peaks()
-    value = T * world * args.steps / (ms_max / 1000.0)
+    value = job_throughput(T, world, args.steps, ms_max)
     # dominant kernel of the step
     if ms_attn >= ms_gemm:
         kern, achieved = "attention", fl["attn_per_launch"] / (ms_attn / n_attn / 1000.0) / 1e12
@@ -420,7 +427,7 @@ def run_ours(args, wl):
                                    "nominal_2250": step_tflops / 2250.0},
         "kernels_ms_per_step": {"gemm": ms_gemm / args.steps, "attention": ms_attn / args.steps,
                                 "rmsnorm": ms_norm / args.steps},
-        "e2e": {"value": T * world * args.steps / (e_ms / 1000.0), "unit": "patches/s",
+        "e2e": {"value": job_throughput(T, world, args.steps, e_ms), "unit": "patches/s",
                 "h2d_bytes_per_step": int(pix_host.numel() * 4 + ids_host.numel() * 8),
                 "d2h_bytes_per_step": int(out_host.numel() * out_host.element_size())},
         "gpu_launches": int(launches),

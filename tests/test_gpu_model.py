@@ -134,3 +134,43 @@ def test_encode_then_scatter_end_to_end():
     # and the embeddings themselves match the oracle on one of the four images
     ref_tower, ref_emb = _run_oracle(cfg, tw, pw, imgs[:1])
     compare(emb[:1536], ref_emb, what="e2e projector image 0")
+
+
+def test_many_tiny_images_cross_the_setup_chunks():
+    """70 images (the per-image tables are uploaded 64 at a time) of 28x28 and
+    56x28: one merged token each or two; patches 4 or 8 per image."""
+    sizes = [(28, 28) if i % 3 else (56, 28) for i in range(70)]
+    cfg, tw, pw, imgs = _setup("mistral3", 2, sizes, seed=11)
+    tower, emb = _run_gpu(cfg, tw, pw, imgs, sizes)
+    ref_tower, ref_emb = _run_oracle(cfg, tw, pw, imgs)
+    compare(tower, ref_tower, what="70 images tower")
+    compare(emb, ref_emb, what="70 images projector")
+
+
+def test_pixtral_single_patch_tiles():
+    """Pixtral preset (patch 16, no merge) with 16x16 images: one patch per block."""
+    sizes = [(16, 16), (16, 32), (16, 16)]
+    cfg, tw, pw, imgs = _setup("pixtral12b", 2, sizes, seed=12)
+    tower, emb = _run_gpu(cfg, tw, pw, imgs, sizes)
+    ref_tower, ref_emb = _run_oracle(cfg, tw, pw, imgs)
+    compare(tower, ref_tower, what="single-patch tower")
+    compare(emb, ref_emb, what="single-patch projector")
+
+
+def test_full_size_pixtral_4096_as_16_tiles():
+    """Pixtral-12B-style: one 4096x4096 image as 16 tiles of 1024x1024 = 65,536
+    patches, 24 layers, no merge; isolation between tiles and determinism."""
+    sizes = [(1024, 1024)] * 16
+    cfg, tw, pw, imgs = _setup("pixtral12b", 24, sizes, seed=0)
+    pipe = vlm.ImagePipeline(cfg, tower_to_device(tw), tower_to_device(pw), sizes)
+    e1 = pipe(pixels_to_device(imgs)).clone()
+    assert e1.shape == (65536, 5120) and torch.isfinite(e1.float()).all()
+    imgs2 = [im.clone() for im in imgs]
+    imgs2[7] = imgs2[7].flip(-2).contiguous()
+    e2 = pipe(pixels_to_device(imgs2)).clone()
+    e3 = pipe(pixels_to_device(imgs)).clone()
+    assert vlm.status_sync(pipe.status) == vlm.OK
+    assert torch.equal(e1, e3)
+    for b in range(16):
+        same = torch.equal(e1[4096 * b:4096 * (b + 1)], e2[4096 * b:4096 * (b + 1)])
+        assert same == (b != 7), b
