@@ -177,17 +177,6 @@ __global__ void __launch_bounds__(192, 2)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  // this CTA's block, query tile and head
-  const int tile = blockIdx.x, h = blockIdx.y;
-  int lo = 0, hi = args.n_blocks - 1;
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if (__ldg(args.qt + mid) <= tile) lo = mid; else hi = mid - 1;
-  }
-  const int kbeg = __ldg(args.cu + lo), kend = __ldg(args.cu + lo + 1);
-  const int q0 = kbeg + (tile - __ldg(args.qt + lo)) * BQ;
-  const int n_kv = (kend - kbeg + BKV - 1) / BKV;
-  const int D = args.heads * DH;
 
   if (threadIdx.x == 0) {
     mbar_init(smem_u32(q_full), 1);
@@ -212,6 +201,20 @@ __global__ void __launch_bounds__(192, 2)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   volatile int* abort_v = abort_flag;
+  griddep_wait();  // the block tables, q, k, v and the output belong to the previous kernels until here
+  griddep_launch_dependents();
+
+  // this CTA's block, query tile and head
+  const int tile = blockIdx.x, h = blockIdx.y;
+  int lo = 0, hi = args.n_blocks - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (__ldg(args.qt + mid) <= tile) lo = mid; else hi = mid - 1;
+  }
+  const int kbeg = __ldg(args.cu + lo), kend = __ldg(args.cu + lo + 1);
+  const int q0 = kbeg + (tile - __ldg(args.qt + lo)) * BQ;
+  const int n_kv = (kend - kbeg + BKV - 1) / BKV;
+  const int D = args.heads * DH;
 
   if (warp == 0) {
     if (lane == 0) {
@@ -370,9 +373,9 @@ int launch_attention(const __nv_bfloat16* qkv, int64_t T, int heads, const int32
   AttnArgs args{cu, qt, n_blocks, heads, out, status};
   dim3 grid(total_qtiles, heads);
   launch_begin(KC_ATTN, s);
-  attn_tc_kernel<<<grid, 192, kSmemBytes, s>>>(tm, args);
+  const cudaError_t e = launch_pdl(attn_tc_kernel, grid, dim3(192), kSmemBytes, s, tm, args);
   launch_end(KC_ATTN, s);
-  return cudaGetLastError() == cudaSuccess ? VLM_OK : VLM_ERR_CUDA;
+  return e == cudaSuccess ? VLM_OK : VLM_ERR_CUDA;
 }
 
 }  // namespace vlm

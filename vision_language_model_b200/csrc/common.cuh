@@ -9,6 +9,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "../../include/vlm.h"
 #include "../../include/vlm_kernels.h"
 
@@ -26,6 +28,32 @@ enum KernelClass : int {
 void launch_begin(int kclass, cudaStream_t s);
 void launch_end(int kclass, cudaStream_t s);
 int num_sms();
+
+// Programmatic dependent launch: every kernel of the path is launched with
+// programmatic stream serialisation, signals early that the next kernel may be
+// scheduled (its prologue then overlaps this kernel's tail), and waits for the
+// previous kernel's completion (griddep_wait) before it reads or writes any
+// memory that another kernel touches.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                              Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
 
 // Per-row status codes written by kernels (sticky: first error wins).
 __device__ __forceinline__ void set_status(int32_t* status, int32_t code) {

@@ -306,6 +306,8 @@ __global__ void __launch_bounds__(192, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   volatile int* abort_v = abort_flag;
+  griddep_wait();  // A, C (and the residual) belong to the previous kernels until here
+  griddep_launch_dependents();
 
   if (warp == 0) {
     if (lane == 0) {
@@ -454,6 +456,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   volatile int* abort_v = abort_flag;
+  griddep_wait();  // A, C (and the residual) belong to the previous kernels until here
+  griddep_launch_dependents();
 
   if (warp == 0) {
     if (lane == 0) {
@@ -549,9 +553,9 @@ int run_gemm_pair(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMa
   const int tiles = args.m_tiles * args.n_tiles;
   const int pairs = tiles < num_sms() / 2 ? tiles : num_sms() / 2;
   launch_begin(KC_GEMM, s);
-  kern<<<2 * pairs, 192, PairShape::SMEM_BYTES, s>>>(ta, tb, tc, args);
+  const cudaError_t e = launch_pdl(kern, dim3(2 * pairs), dim3(192), PairShape::SMEM_BYTES, s, ta, tb, tc, args);
   launch_end(KC_GEMM, s);
-  return cudaGetLastError() == cudaSuccess ? VLM_OK : VLM_ERR_CUDA;
+  return e == cudaSuccess ? VLM_OK : VLM_ERR_CUDA;
 }
 
 int dispatch_pair(int epi, const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tc, const GemmArgs& args,
@@ -583,9 +587,9 @@ int run_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tc
   const int tiles = args.m_tiles * args.n_tiles;
   const int grid = tiles < num_sms() ? tiles : num_sms();
   launch_begin(KC_GEMM, s);
-  kern<<<grid, 192, S::SMEM_BYTES, s>>>(ta, tb, tc, args);
+  const cudaError_t e = launch_pdl(kern, dim3(grid), dim3(192), S::SMEM_BYTES, s, ta, tb, tc, args);
   launch_end(KC_GEMM, s);
-  return cudaGetLastError() == cudaSuccess ? VLM_OK : VLM_ERR_CUDA;
+  return e == cudaSuccess ? VLM_OK : VLM_ERR_CUDA;
 }
 
 template <int BN>

@@ -11,6 +11,8 @@ namespace vlm {
 // ---------------------------------------------------------------------------
 __global__ void setup_kernel(ImageChunk chunk, ImgInfo* info, int32_t* cu, int32_t* qt,
                              int32_t* pos, int n_images) {
+  griddep_wait();
+  griddep_launch_dependents();
   const int tid = blockIdx.x * blockDim.x + threadIdx.x;
   if (tid < chunk.count) {
     const int b = chunk.first + tid;
@@ -49,6 +51,8 @@ __global__ void setup_kernel(ImageChunk chunk, ImgInfo* info, int32_t* cu, int32
 // 2D RoPE angle table: tab[p][i] = (cos, sin)(p * w_k), w_k = theta^(-2k/dh),
 // k = 2i for the row half (i < dh/4) and k = 2(i - dh/4) + 1 for the column half.
 __global__ void rope_table_kernel(float theta, int head_dim, int max_pos, float2* tab) {
+  griddep_wait();
+  griddep_launch_dependents();
   const int half = head_dim / 2, quarter = head_dim / 4;
   const int idx = blockIdx.x * blockDim.x + threadIdx.x;
   if (idx >= max_pos * half) return;
@@ -79,6 +83,8 @@ __constant__ float c_std[3] = {0.26862954f, 0.26130258f, 0.27577711f};
 __global__ void im2col_kernel(const float* __restrict__ pix, const ImgInfo* __restrict__ info,
                               const int32_t* __restrict__ cu, int n_images, int64_t T, int p, int kp,
                               int normalize, __nv_bfloat16* __restrict__ out) {
+  griddep_wait();
+  griddep_launch_dependents();
   const int lane = threadIdx.x & 31;
   const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
   const int pp = p * p, kreal = 3 * pp;
@@ -116,6 +122,8 @@ template <int NV>
 __global__ void rmsnorm_kernel(float* __restrict__ x, const float* __restrict__ g0,
                                const float* __restrict__ g1, __nv_bfloat16* __restrict__ out,
                                int64_t rows, float eps) {
+  griddep_wait();
+  griddep_launch_dependents();
   constexpr int width = NV * 128;
   const int lane = threadIdx.x & 31;
   const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
@@ -169,6 +177,8 @@ __global__ void merge_norm_kernel(const __nv_bfloat16* __restrict__ x, const flo
                                   const ImgInfo* __restrict__ info, const int32_t* __restrict__ cu,
                                   int n_images, int64_t T, int m, float eps,
                                   __nv_bfloat16* __restrict__ z) {
+  griddep_wait();
+  griddep_launch_dependents();
   constexpr int width = NV * 128;
   const int lane = threadIdx.x & 31;
   const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
@@ -215,6 +225,8 @@ __global__ void merge_norm_kernel(const __nv_bfloat16* __restrict__ x, const flo
 // ---------------------------------------------------------------------------
 __global__ void scatter_count_kernel(const int64_t* __restrict__ ids, int64_t n, int64_t token,
                                      int32_t* __restrict__ chunk_count) {
+  griddep_wait();
+  griddep_launch_dependents();
   const int64_t i = static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x;
   const int flag = (i < n && ids[i] == token) ? 1 : 0;
   const int wc = __popc(__ballot_sync(0xffffffffu, flag));
@@ -232,6 +244,8 @@ __global__ void scatter_count_kernel(const int64_t* __restrict__ ids, int64_t n,
 __global__ void scatter_scan_kernel(const int32_t* __restrict__ chunk_count, int64_t n_chunks,
                                     int64_t expected, int64_t* __restrict__ chunk_base,
                                     int32_t* __restrict__ ok_flag, int32_t* status) {
+  griddep_wait();
+  griddep_launch_dependents();
   // 1024 threads; sequential over blocks of 1024 chunks with a running carry.
   __shared__ int64_t warp_sums[32];
   __shared__ int64_t carry;
@@ -276,6 +290,8 @@ __global__ void scatter_positions_kernel(const int64_t* __restrict__ ids, int64_
                                          const int64_t* __restrict__ chunk_base,
                                          const int32_t* __restrict__ ok_flag,
                                          int64_t* __restrict__ dst_rows) {
+  griddep_wait();
+  griddep_launch_dependents();
   if (*ok_flag == 0) return;
   const int64_t i = static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x;
   const int flag = (i < n && ids[i] == token) ? 1 : 0;
@@ -294,6 +310,8 @@ __global__ void scatter_copy_kernel(const uint4* __restrict__ img, uint4* __rest
                                     const int64_t* __restrict__ dst_rows,
                                     const int32_t* __restrict__ ok_flag, int64_t n_rows,
                                     int64_t vec_per_row) {
+  griddep_wait();
+  griddep_launch_dependents();
   if (*ok_flag == 0) return;
   const int64_t total = n_rows * vec_per_row;
   for (int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; idx < total;
@@ -341,6 +359,8 @@ __global__ void pack_cols_kernel(const __nv_bfloat16* __restrict__ src, __nv_bfl
 }
 
 __global__ void f32_to_bf16_kernel(const float* __restrict__ x, __nv_bfloat16* __restrict__ y, int64_t n) {
+  griddep_wait();
+  griddep_launch_dependents();
   for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; 2 * i < n;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
     const float2 v = reinterpret_cast<const float2*>(x)[i];
@@ -362,25 +382,26 @@ int launch_setup(const ImageChunk& chunk, ImgInfo* info, int32_t* cu, int32_t* q
   const int64_t tokens = chunk.tok_off[chunk.count] - chunk.tok_off[0];
   const int grid = grid_for(tokens > chunk.count ? tokens : chunk.count, 256);
   launch_begin(KC_SETUP, s);
-  setup_kernel<<<grid, 256, 0, s>>>(chunk, info, cu, qt, pos, n_images);
+  const cudaError_t e = launch_pdl(setup_kernel, dim3(grid), dim3(256), 0, s, chunk, info, cu, qt, pos, n_images);
   launch_end(KC_SETUP, s);
-  return cudaGetLastError() == cudaSuccess ? VLM_OK : VLM_ERR_CUDA;
+  return e == cudaSuccess ? VLM_OK : VLM_ERR_CUDA;
 }
 
 int launch_rope_table(float theta, int head_dim, int max_pos, float2* tab, cudaStream_t s) {
   const int n = max_pos * head_dim / 2;
   launch_begin(KC_SETUP, s);
-  rope_table_kernel<<<(n + 255) / 256, 256, 0, s>>>(theta, head_dim, max_pos, tab);
+  const cudaError_t e = launch_pdl(rope_table_kernel, dim3((n + 255) / 256), dim3(256), 0, s, theta, head_dim, max_pos, tab);
   launch_end(KC_SETUP, s);
-  return cudaGetLastError() == cudaSuccess ? VLM_OK : VLM_ERR_CUDA;
+  return e == cudaSuccess ? VLM_OK : VLM_ERR_CUDA;
 }
 
 int launch_im2col(const float* pix, const ImgInfo* info, const int32_t* cu, int n_images, int64_t T,
                   int p, int kp, int normalize, __nv_bfloat16* out, cudaStream_t s) {
   launch_begin(KC_IM2COL, s);
-  im2col_kernel<<<grid_for(T * 32, 256), 256, 0, s>>>(pix, info, cu, n_images, T, p, kp, normalize, out);
+  const cudaError_t e = launch_pdl(im2col_kernel, dim3(grid_for(T * 32, 256)), dim3(256), 0, s, pix, info, cu, n_images, T, p, kp,
+                                    normalize, out);
   launch_end(KC_IM2COL, s);
-  return cudaGetLastError() == cudaSuccess ? VLM_OK : VLM_ERR_CUDA;
+  return e == cudaSuccess ? VLM_OK : VLM_ERR_CUDA;
 }
 
 int launch_rmsnorm(float* x, const float* g0, const float* g1, __nv_bfloat16* out, int64_t rows,
@@ -388,9 +409,10 @@ int launch_rmsnorm(float* x, const float* g0, const float* g1, __nv_bfloat16* ou
   if (width % 128 || width > 2048 || width <= 0) return VLM_ERR_UNSUPPORTED;
   const int grid = grid_for(rows * 32, 256);
   launch_begin(KC_NORM, s);
+  cudaError_t e = cudaErrorInvalidValue;
   switch (width / 128) {
 #define VLM_NORM_CASE(nv) \
-  case nv: rmsnorm_kernel<nv><<<grid, 256, 0, s>>>(x, g0, g1, out, rows, eps); break;
+  case nv: e = launch_pdl(rmsnorm_kernel<nv>, dim3(grid), dim3(256), 0, s, x, g0, g1, out, rows, eps); break;
     VLM_NORM_CASE(1) VLM_NORM_CASE(2) VLM_NORM_CASE(3) VLM_NORM_CASE(4) VLM_NORM_CASE(5)
     VLM_NORM_CASE(6) VLM_NORM_CASE(7) VLM_NORM_CASE(8) VLM_NORM_CASE(9) VLM_NORM_CASE(10)
     VLM_NORM_CASE(11) VLM_NORM_CASE(12) VLM_NORM_CASE(13) VLM_NORM_CASE(14) VLM_NORM_CASE(15)
@@ -399,7 +421,7 @@ int launch_rmsnorm(float* x, const float* g0, const float* g1, __nv_bfloat16* ou
     default: break;
   }
   launch_end(KC_NORM, s);
-  return cudaGetLastError() == cudaSuccess ? VLM_OK : VLM_ERR_CUDA;
+  return e == cudaSuccess ? VLM_OK : VLM_ERR_CUDA;
 }
 
 int launch_merge_norm(const __nv_bfloat16* x, const float* g, const ImgInfo* info, const int32_t* cu,
@@ -408,9 +430,10 @@ int launch_merge_norm(const __nv_bfloat16* x, const float* g, const ImgInfo* inf
   if (width % 128 || width > 2048 || width <= 0) return VLM_ERR_UNSUPPORTED;
   const int grid = grid_for(T * 32, 256);
   launch_begin(KC_MERGE, s);
+  cudaError_t e = cudaErrorInvalidValue;
   switch (width / 128) {
 #define VLM_MERGE_CASE(nv) \
-  case nv: merge_norm_kernel<nv><<<grid, 256, 0, s>>>(x, g, info, cu, n_images, T, m, eps, z); break;
+  case nv: e = launch_pdl(merge_norm_kernel<nv>, dim3(grid), dim3(256), 0, s, x, g, info, cu, n_images, T, m, eps, z); break;
     VLM_MERGE_CASE(1) VLM_MERGE_CASE(2) VLM_MERGE_CASE(3) VLM_MERGE_CASE(4) VLM_MERGE_CASE(5)
     VLM_MERGE_CASE(6) VLM_MERGE_CASE(7) VLM_MERGE_CASE(8) VLM_MERGE_CASE(9) VLM_MERGE_CASE(10)
     VLM_MERGE_CASE(11) VLM_MERGE_CASE(12) VLM_MERGE_CASE(13) VLM_MERGE_CASE(14) VLM_MERGE_CASE(15)
@@ -419,23 +442,28 @@ int launch_merge_norm(const __nv_bfloat16* x, const float* g, const ImgInfo* inf
     default: break;
   }
   launch_end(KC_MERGE, s);
-  return cudaGetLastError() == cudaSuccess ? VLM_OK : VLM_ERR_CUDA;
+  return e == cudaSuccess ? VLM_OK : VLM_ERR_CUDA;
 }
 
 int launch_scatter(const int64_t* ids, int64_t n, int64_t token, const void* img, int64_t n_img,
                    void* text, int64_t row_bytes, ScatterWs ws, int32_t* status, cudaStream_t s) {
   const int64_t n_chunks = (n + 255) / 256;
   launch_begin(KC_SCATTER, s);
-  scatter_count_kernel<<<static_cast<unsigned>(n_chunks), 256, 0, s>>>(ids, n, token, ws.chunk_count);
-  scatter_scan_kernel<<<1, 1024, 0, s>>>(ws.chunk_count, n_chunks, n_img, ws.chunk_base, ws.ok_flag, status);
-  scatter_positions_kernel<<<static_cast<unsigned>(n_chunks), 256, 0, s>>>(ids, n, token, ws.chunk_base,
-                                                                           ws.ok_flag, ws.dst_rows);
+  const dim3 chunks(static_cast<unsigned>(n_chunks));
+  cudaError_t e = launch_pdl(scatter_count_kernel, chunks, dim3(256), 0, s, ids, n, token, ws.chunk_count);
+  if (e == cudaSuccess)
+    e = launch_pdl(scatter_scan_kernel, dim3(1), dim3(1024), 0, s, ws.chunk_count, n_chunks, n_img, ws.chunk_base,
+                   ws.ok_flag, status);
+  if (e == cudaSuccess)
+    e = launch_pdl(scatter_positions_kernel, chunks, dim3(256), 0, s, ids, n, token, ws.chunk_base, ws.ok_flag,
+                   ws.dst_rows);
   const int64_t vec = row_bytes / 16;
-  scatter_copy_kernel<<<grid_for(n_img * vec, 256), 256, 0, s>>>(
-      static_cast<const uint4*>(img), static_cast<uint4*>(text), ws.dst_rows, ws.ok_flag, n_img, vec);
+  if (e == cudaSuccess)
+    e = launch_pdl(scatter_copy_kernel, dim3(grid_for(n_img * vec, 256)), dim3(256), 0, s,
+                   static_cast<const uint4*>(img), static_cast<uint4*>(text), ws.dst_rows, ws.ok_flag, n_img, vec);
   launch_end(KC_SCATTER, s);
   note_extra_launches(3);
-  return cudaGetLastError() == cudaSuccess ? VLM_OK : VLM_ERR_CUDA;
+  return e == cudaSuccess ? VLM_OK : VLM_ERR_CUDA;
 }
 
 int launch_pack_gate_up(const void* gate, const void* up, void* dst, int64_t f, int64_t d, cudaStream_t s) {
@@ -459,9 +487,9 @@ int launch_pack_cols(const void* src, void* dst, int64_t rows, int64_t src_cols,
 
 int launch_f32_to_bf16(const float* x, __nv_bfloat16* y, int64_t n, cudaStream_t s) {
   launch_begin(KC_NORM, s);
-  f32_to_bf16_kernel<<<grid_for(n / 2, 256), 256, 0, s>>>(x, y, n);
+  const cudaError_t e = launch_pdl(f32_to_bf16_kernel, dim3(grid_for(n / 2, 256)), dim3(256), 0, s, x, y, n);
   launch_end(KC_NORM, s);
-  return cudaGetLastError() == cudaSuccess ? VLM_OK : VLM_ERR_CUDA;
+  return e == cudaSuccess ? VLM_OK : VLM_ERR_CUDA;
 }
 
 }  // namespace vlm
