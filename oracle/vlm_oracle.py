@@ -115,6 +115,79 @@ def positions(grids) -> tuple:
 
 
 # ---------------------------------------------------------------------------
+# Image front end (before the path): resize onto the grid, Pixtral tiling
+# ---------------------------------------------------------------------------
+
+def resized_hw(height: int, width: int, longest_edge: int, grid: int) -> tuple:
+    """Target size of the processor's resize.
+
+    "Mistral 3" intro: images are resized so the longest edge fits
+    longest_edge while staying on the patch grid. Reading: shrink (never
+    enlarge) by r = max(H, W) / longest_edge when r > 1, flooring each side,
+    then round each side up to a multiple of `grid` (patch size times the
+    merge size, so the merge always finds whole 2x2 blocks).
+    """
+    if height <= 0 or width <= 0 or longest_edge <= 0 or grid <= 0:
+        raise ValueError("sizes must be positive")
+    ratio = max(height, width) / longest_edge
+    if ratio > 1.0:
+        height, width = int(height // ratio), int(width // ratio)
+    height, width = max(height, 1), max(width, 1)
+    return -(-height // grid) * grid, -(-width // grid) * grid
+
+
+def resize_bilinear(image: np.ndarray, out_h: int, out_w: int) -> np.ndarray:
+    """Bilinear resampling with half-pixel centres (no antialiasing).
+
+    Output pixel (y, x) samples the input at ((y + 1/2) H/out_h - 1/2,
+    (x + 1/2) W/out_w - 1/2), clamped to the image, interpolating the four
+    neighbours (reading: the pages do not name the filter).
+    """
+    x = np.asarray(image, dtype=np.float64)
+    c, h, w = x.shape
+
+    def axis(n_out, n_in):
+        src = (np.arange(n_out) + 0.5) * (n_in / n_out) - 0.5
+        src = np.clip(src, 0.0, n_in - 1)
+        i0 = np.floor(src).astype(np.int64)
+        i1 = np.minimum(i0 + 1, n_in - 1)
+        return i0, i1, src - i0
+
+    y0, y1, fy = axis(out_h, h)
+    x0, x1, fx = axis(out_w, w)
+    top = x[:, y0][:, :, x0] * (1 - fx) + x[:, y0][:, :, x1] * fx
+    bot = x[:, y1][:, :, x0] * (1 - fx) + x[:, y1][:, :, x1] * fx
+    return top * (1 - fy)[None, :, None] + bot * fy[None, :, None]
+
+
+def tile_image(image: np.ndarray, tile: int = PIXTRAL_TILE) -> list:
+    """Split [3, H, W] into tile x tile tiles, row-major over the tile grid
+    ("Pixtral-12B-2409", VISION TOKENS: 4096^2 -> a 4x4 grid of 1024^2 tiles)."""
+    c, h, w = image.shape
+    tile_count(h, w, tile)
+    return [np.asarray(image[:, i:i + tile, j:j + tile]) for i in range(0, h, tile) for j in range(0, w, tile)]
+
+
+def expand_placeholders(input_ids, marker_id: int, counts, image_token_id: int) -> np.ndarray:
+    """Each occurrence of marker_id, in order, becomes counts[k] copies of
+    image_token_id; every other id is kept ("Mistral 3", "Several images in one
+    conversation": the processor expands each image marker to that image's own
+    token count). Raises if the number of markers differs from len(counts)."""
+    out, k = [], 0
+    for t in np.asarray(input_ids).reshape(-1):
+        if t == marker_id:
+            if k >= len(counts):
+                raise ValueError("more markers than images")
+            out.extend([image_token_id] * int(counts[k]))
+            k += 1
+        else:
+            out.append(int(t))
+    if k != len(counts):
+        raise ValueError(f"{k} markers for {len(counts)} images")
+    return np.asarray(out, dtype=np.int64)
+
+
+# ---------------------------------------------------------------------------
 # a1, a2: processor normalisation and patch embedding
 # ---------------------------------------------------------------------------
 

@@ -404,3 +404,52 @@ def test_planted_rope_frequency_split_swap_is_caught(monkeypatch):
     monkeypatch.setattr(O, "rope_angles", bad)
     with pytest.raises(AssertionError):
         test_rope_frequencies_closed_form()
+
+
+# ---------------------------------------------------------------------------
+# Front end: resize onto the grid, tiling, placeholder expansion
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("hw,expect", [((1540, 1540), (1540, 1540)), ((3080, 1540), (1540, 784)),
+                                       ((100, 50), (112, 56)), ((2000, 1000), (1540, 784)), ((27, 3000), (28, 1540))])
+def test_resized_hw_closed_form(hw, expect):
+    assert O.resized_hw(*hw, 1540, 28) == expect
+    h, w = O.resized_hw(*hw, 1540, 28)
+    assert h % 28 == 0 and w % 28 == 0 and max(h, w) <= 1540 + 27
+
+
+@pytest.mark.parametrize("src,dst", [((13, 17), (28, 56)), ((64, 48), (28, 28)), ((5, 5), (5, 5))])
+def test_resize_bilinear_matches_torch_interpolate(src, dst):
+    img = RNG.random((3, *src))
+    ref = F.interpolate(torch.from_numpy(img)[None], size=dst, mode="bilinear", align_corners=False,
+                        antialias=False)[0].numpy()
+    np.testing.assert_allclose(O.resize_bilinear(img, *dst), ref, rtol=1e-12, atol=1e-12)
+
+
+def test_resize_identity_and_constant():
+    img = RNG.random((3, 7, 9))
+    np.testing.assert_allclose(O.resize_bilinear(img, 7, 9), img, rtol=0, atol=1e-15)
+    const = np.full((3, 5, 6), 0.25)
+    np.testing.assert_allclose(O.resize_bilinear(const, 28, 14), 0.25, rtol=0, atol=1e-15)
+
+
+def test_tile_image_round_trip_and_count():
+    img = RNG.random((3, 8, 12))
+    tiles = O.tile_image(img, 4)
+    assert len(tiles) == 6
+    back = np.concatenate([np.concatenate(tiles[r * 3:(r + 1) * 3], axis=2) for r in range(2)], axis=1)
+    np.testing.assert_array_equal(back, img)
+    with pytest.raises(ValueError):
+        O.tile_image(np.zeros((3, 10, 8)), 4)
+
+
+def test_expand_placeholders_definition():
+    ids = np.array([1, 2, 99, 3, 99, 4])
+    got = O.expand_placeholders(ids, 99, [3, 1], 10)
+    assert got.tolist() == [1, 2, 10, 10, 10, 3, 10, 4]
+    assert O.expand_placeholders(np.array([5, 6]), 99, [], 10).tolist() == [5, 6]
+    with pytest.raises(ValueError):
+        O.expand_placeholders(ids, 99, [3], 10)
+    # the pages' count: one 896x1344 image is 1,536 placeholders
+    h, w = O.merged_grid(*O.patch_grid(896, 1344, 14), 2)
+    assert int((O.expand_placeholders(np.array([7, 99, 8]), 99, [h * w], 10) == 10).sum()) == 1536
