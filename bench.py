@@ -45,6 +45,11 @@ WORKLOADS = {
     "pixtral_4096": dict(preset="pixtral12b", sizes=[(1024, 1024)] * 16, n_seq=16, seq_len=4352,
                          desc="Pixtral-12B-style: one 4096x4096 image as 16 tiles of 1024x1024 = 65,536 patches, "
                               "no merge, projector 1024->5120->5120"),
+    "photo_4032x3024": dict(preset="mistral3", photo=(3024, 4032), sizes=[(1176, 1540)], n_seq=1, seq_len=4096,
+                            desc="one decoded 4032x3024 u8 RGB photo: GPU resize to 1176x1540 (longest edge 1540, "
+                                 "28-px grid; 84x110 = 9,240 patches -> 2,310 merged tokens), 24-layer tower + "
+                                 "merge + projector, device placeholder expansion of one marker, scatter into "
+                                 "4,096 ids"),
     "e2e4": dict(preset="mistral3", sizes=[(896, 1344)] * 4, n_seq=4, seq_len=4096,
                  desc="4 x 896x1344 images (6,144 patches -> 1,536 placeholders each) scattered into 4 x 4,096 ids"),
 }
@@ -313,7 +318,8 @@ def ncu_traffic(kernel: str) -> float | None:
 
 
 KERNEL_SOURCES = {"attention": ["attention_tc.cu", "exp2_poly.cuh", "common.cuh", "kernels.cuh"],
-                  "gemm": ["gemm_tcgen05.cu", "common.cuh", "kernels.cuh"]}
+                  "gemm": ["gemm_tcgen05.cu", "common.cuh", "kernels.cuh"],
+                  "resize": ["frontend.cu", "common.cuh", "kernels.cuh"]}
 
 
 def run_ours(args, wl):
@@ -331,21 +337,41 @@ def run_ours(args, wl):
     pw = {k: v.to(dev) for k, v in synth.projector_weights(args.seed, cfg.width, cfg.merge, cfg.proj_out).items()}
     pipe = vlm.ImagePipeline(cfg, tw, pw, sizes, device=dev)
     del tw, pw
-    imgs = synth.images(args.seed + rank, sizes)
-    pix_host = torch.cat([im.reshape(-1) for im in imgs]).pin_memory()
-    pix = pix_host.to(dev)
+    photo = wl.get("photo")
+    if photo:
+        assert sizes == [vlm.resize_target(*photo, 1540, cfg.patch * cfg.merge)]
+        pix_host = synth.photo_u8(args.seed + rank, "photo", *photo).reshape(-1).pin_memory()
+        photo_dev = pix_host.to(dev)
+        pix = torch.empty(sum(3 * h * w for h, w in sizes), dtype=torch.float32, device=dev)
+    else:
+        imgs = synth.images(args.seed + rank, sizes)
+        pix_host = torch.cat([im.reshape(-1) for im in imgs]).pin_memory()
+        pix = pix_host.to(dev)
     per_seq = [[] for _ in range(wl["n_seq"])]
     lens_m = [(h // cfg.patch) * (w // cfg.patch) // (cfg.merge * cfg.merge) for h, w in sizes]
     for i, n in enumerate(lens_m):
         per_seq[i % wl["n_seq"]].append(n)
-    ids_host = synth.text_sequences(args.seed, wl["n_seq"], wl["seq_len"], per_seq).reshape(-1).pin_memory()
-    ids = ids_host.to(dev)
+    if photo:
+        marker = 7
+        ids_host = synth.prompt_with_markers(args.seed, wl["seq_len"] - sum(lens_m), len(lens_m), marker).pin_memory()
+        marker_ids = ids_host.to(dev)
+        ids = torch.empty(wl["seq_len"], dtype=torch.int64, device=dev)
+        expand_ws = torch.empty(max(256, vlm.expand_placeholders_workspace_size(marker_ids.numel(), len(lens_m))),
+                                dtype=torch.uint8, device=dev)
+    else:
+        ids_host = synth.text_sequences(args.seed, wl["n_seq"], wl["seq_len"], per_seq).reshape(-1).pin_memory()
+        ids = ids_host.to(dev)
     text = synth.text_embeddings(args.seed, ids.numel(), cfg.proj_out).to(dev)
     scatter_ws = torch.empty(max(256, vlm.scatter_workspace_size(ids.numel())), dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
 
     def step():
+        if photo:
+            vlm.preprocess(photo_dev, [photo], sizes, out=pix)
         emb = pipe(pix)
+        if photo:
+            vlm.expand_placeholders(marker_ids, marker, lens_m, cfg.image_token_id, out=ids, workspace=expand_ws,
+                                    status=pipe.status)
         vlm.scatter(ids, emb, text, cfg.image_token_id, workspace=scatter_ws, status=pipe.status)
 
     for _ in range(args.warmup):
@@ -387,6 +413,8 @@ def run_ours(args, wl):
     n_gemm, ms_gemm = vlm.profile_query("gemm")
     n_attn, ms_attn = vlm.profile_query("attention")
     n_norm, ms_norm = vlm.profile_query("rmsnorm")
+    n_resize, ms_resize = vlm.profile_query("resize")
+    n_expand, ms_expand = vlm.profile_query("expand")
     vlm.profile_enable(False)
     rc = vlm.status_sync(pipe.status)
     if rc != vlm.OK:
@@ -399,8 +427,8 @@ def run_ours(args, wl):
     e_start, e_stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e_start.record(stream)
     for _ in range(args.steps):
-        pix.copy_(pix_host, non_blocking=True)
-        ids.copy_(ids_host, non_blocking=True)
+        (photo_dev if photo else pix).copy_(pix_host, non_blocking=True)
+        (marker_ids if photo else ids).copy_(ids_host, non_blocking=True)
         step()
         out_host.copy_(text, non_blocking=True)
     e_stop.record(stream)
@@ -437,11 +465,44 @@ def run_ours(args, wl):
                                 "note": "per-kernel CUDA events on the launch stream, in a second pass of the "
                                         "same steps"},
         "e2e": {"value": job_throughput(T, world, args.steps, e_ms), "unit": "patches/s",
-                "h2d_bytes_per_step": int(pix_host.numel() * 4 + ids_host.numel() * 8),
+                "h2d_bytes_per_step": int(pix_host.numel() * pix_host.element_size() + ids_host.numel() * 8),
                 "d2h_bytes_per_step": int(out_host.numel() * out_host.element_size())},
         "gpu_launches": int(launches),
         "clocks": clk,
     }
+    if photo:
+        # distinct source rows the vertical taps touch (half-pixel centres, clamped)
+        (sh, sw), (oh, _) = photo, sizes[0]
+        ys = np.clip((np.arange(oh) + 0.5) * (sh / oh) - 0.5, 0, sh - 1)
+        rows_read = len(set(np.floor(ys).astype(int)) | set(np.minimum(np.floor(ys).astype(int) + 1, sh - 1)))
+        src_bytes = rows_read * 3 * sw
+        out_bytes = sum(12 * h * w for h, w in sizes)
+        # the resize alone: 3 photo/output buffer pairs (174 MB, more than L2) in rotation,
+        # 30 launches back to back between two events on the launch stream
+        srcs = [photo_dev] + [synth.photo_u8(args.seed + 100 + k, "photo", *photo).reshape(-1).to(dev)
+                              for k in range(2)]
+        outs = [pix] + [torch.empty_like(pix) for _ in range(2)]
+        for k in range(3):
+            vlm.preprocess(srcs[k], [photo], sizes, out=outs[k])
+        r_start, r_stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        r_start.record(stream)
+        for k in range(30):
+            vlm.preprocess(srcs[k % 3], [photo], sizes, out=outs[k % 3])
+        r_stop.record(stream)
+        torch.cuda.synchronize()
+        r_ms = r_start.elapsed_time(r_stop) / 30
+        resize_gbs = (src_bytes + out_bytes) / (r_ms / 1000.0) / 1e9
+        line["front_end"] = {
+            "resize": {"ms_per_launch": r_ms, "in_step_ms_per_launch": ms_resize / max(n_resize, 1),
+                       "algorithmic_bytes": src_bytes + out_bytes, "achieved_gbs": resize_gbs,
+                       "peak_gbs": peaks["hbm_gbs"], "frac": resize_gbs / peaks["hbm_gbs"],
+                       "bytes_note": f"u8 source rows the taps touch ({rows_read} of {sh}) read once + fp32 CHW "
+                                     "output written once; timed alone, 30 launches over 3 rotating buffer pairs "
+                                     "larger than L2 together",
+                       "traffic": ncu_traffic("resize")},
+            "expand_ms_per_step": ms_expand / args.steps,
+        }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(wl, args.seed)
     if rank == 0:

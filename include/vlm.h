@@ -225,6 +225,69 @@ VLM_API int vlm_scatter_noalloc(const int64_t* d_input_ids, int64_t n_tokens, in
                                 int64_t row_bytes, int32_t* d_status, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * Image front end: the steps just before the path ([K] intro and
+ * Mistral3ImageProcessor: images are resized so the longest edge fits
+ * longest_edge = 1540 while staying on the patch grid; [P] VISION TOKENS:
+ * a large image is cut into 1024x1024 tiles).
+ *
+ * vlm_resize_target (host only, launches nothing): the processor's resize
+ *   size. Reading (the pages give no formula): when max(H, W) > longest_edge
+ *   both sides are divided by r = max(H, W) / longest_edge (in double) and
+ *   floored; images are never enlarged by this step; then each side is rounded
+ *   up to a multiple of `grid` (patch * merge, so the 2x2 merge always finds
+ *   whole blocks: 28 for [K]; the tile size 1024 for [P]'s tiling).
+ *   Returns VLM_ERR_INVALID_ARG for a non-positive argument.
+ *
+ * vlm_preprocess: bilinear resize of decoded images onto out_hw.
+ *   d_src: device uint8, the images' [H_b, W_b, 3] RGB (HWC, interleaved)
+ *     blocks concatenated in call order, no padding.
+ *   src_hw, out_hw: host int32 [n_images, 2] source and output (H, W);
+ *     every output width a multiple of 4.
+ *   tile: 0, or the tile edge (a multiple of 4 dividing every output H and W).
+ *   d_out: device fp32, 16-byte aligned; per image [3, oh, ow] CHW in call
+ *     order, values u8 / 255 in [0, 1] (reading: [K]'s mean/std are in these
+ *     units); with tile > 0 each image is instead written as its
+ *     (oh/tile)(ow/tile) tiles, row-major over the tile grid, each a
+ *     [3, tile, tile] block -- exactly the `pixels` vlm_encode takes with
+ *     every tile listed as one (tile, tile) image.
+ *   Resampling (reading: the pages name no filter): output pixel (y, x)
+ *   samples the source at ((y + 1/2) H / oh - 1/2, (x + 1/2) W / ow - 1/2),
+ *   clamped to the image, interpolating the 4 neighbours; no antialiasing.
+ *   Host-side errors only (VLM_ERR_BAD_SHAPE for a size rule above).
+ * ------------------------------------------------------------------------- */
+VLM_API int vlm_resize_target(int32_t height, int32_t width, int32_t longest_edge, int32_t grid, int32_t* out_h,
+                              int32_t* out_w);
+VLM_API int vlm_preprocess(const uint8_t* d_src, const int32_t* src_hw, int n_images, const int32_t* out_hw,
+                           int32_t tile, float* d_out, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * vlm_expand_placeholders -- the step between the projector and the scatter
+ * ([K] "Several images in one conversation": each image's marker in the
+ * prompt becomes as many image_token_id positions as that image has merged
+ * tokens).
+ *
+ * d_input_ids: device int64 [n_ids] holding one marker_id per image, in
+ *   image order.
+ * counts: host int64 [n_images], the merged-token count of each image
+ *   ((H/p/m)(W/p/m) for an image on the grid).
+ * d_out_ids: device int64, capacity out_capacity; receives the expanded ids:
+ *   the k-th marker replaced by counts[k] copies of image_token_id, every
+ *   other id copied in order.
+ * *out_len (host) is set to n_ids - n_images + sum(counts) before anything
+ *   is launched; VLM_ERR_WORKSPACE if that exceeds out_capacity.
+ * If the number of markers on the device differs from n_images, nothing is
+ *   written and *d_status = VLM_ERR_COUNT_MISMATCH.
+ * n_ids == 0 with n_images == 0 sets *out_len = 0 and launches nothing.
+ * d_workspace: 256-byte aligned, at least
+ *   vlm_expand_placeholders_workspace_size(n_ids, n_images) bytes.
+ * ------------------------------------------------------------------------- */
+VLM_API size_t vlm_expand_placeholders_workspace_size(int64_t n_ids, int n_images);
+VLM_API int vlm_expand_placeholders(const int64_t* d_input_ids, int64_t n_ids, int64_t marker_id,
+                                    const int64_t* counts, int n_images, int64_t image_token_id,
+                                    int64_t* d_out_ids, int64_t out_capacity, int64_t* out_len,
+                                    void* d_workspace, size_t ws_bytes, int32_t* d_status, void* stream);
+
+/* ---------------------------------------------------------------------------
  * Instrumentation (host-side, not thread-safe)
  * ------------------------------------------------------------------------- */
 /* Total kernels this library has launched in the process. */
@@ -232,7 +295,8 @@ VLM_API int64_t vlm_launch_count(void);
 /* Turns per-kernel CUDA-event timing on (1) or off (0) and clears it. */
 VLM_API int vlm_profile_enable(int on);
 /* Kernel classes: 0 GEMM, 1 attention, 2 RMSNorm, 3 patch gather, 4 merge
- * gather, 5 scatter, 6 index setup, 7 weight packing. Synchronises on the last
+ * gather, 5 scatter, 6 index setup, 7 weight packing, 8 image resize,
+ * 9 placeholder expansion. Synchronises on the last
  * recorded event, then returns the launches and summed device milliseconds
  * recorded for `kclass` since profiling was enabled. */
 VLM_API int vlm_profile_query(int kclass, int64_t* launches, double* total_ms);

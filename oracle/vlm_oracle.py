@@ -118,6 +118,18 @@ def positions(grids) -> tuple:
 # Image front end (before the path): resize onto the grid, Pixtral tiling
 # ---------------------------------------------------------------------------
 
+def pixels_from_u8(image_hwc: np.ndarray) -> np.ndarray:
+    """Decoded u8 RGB [H, W, 3] -> float [3, H, W] in [0, 1] (value / 255).
+
+    Reading: "Mistral 3", API `Mistral3ImageProcessor` gives the mean/std in
+    [0, 1] units, so pixels enter the normalisation as u8 / 255.
+    """
+    x = np.asarray(image_hwc)
+    if x.ndim != 3 or x.shape[2] != 3:
+        raise ValueError("expected [H, W, 3]")
+    return x.astype(np.float64).transpose(2, 0, 1) / 255.0
+
+
 def resized_hw(height: int, width: int, longest_edge: int, grid: int) -> tuple:
     """Target size of the processor's resize.
 

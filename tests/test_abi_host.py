@@ -118,3 +118,41 @@ def test_package_import_does_not_load_library():
         sys.modules.pop(k)
     pkg = importlib.import_module("vision_language_model_b200")
     assert not hasattr(pkg, "_lib")
+
+
+def test_resize_target_matches_oracle_sweep(L):
+    """vlm_resize_target (host only) against the oracle's resized_hw, exactly."""
+    from oracle import vlm_oracle as O
+    import numpy as np
+    rng = np.random.default_rng(7)
+    sizes = [(1540, 1540), (4032, 3024), (3024, 4032), (1, 1), (27, 3000), (1541, 1540), (200, 100)]
+    sizes += [tuple(int(v) for v in rng.integers(1, 9000, 2)) for _ in range(300)]
+    for (h, w) in sizes:
+        for edge, grid in ((1540, 28), (1540, 14), (4096, 1024), (1024, 16)):
+            assert vlm.resize_target(h, w, edge, grid) == O.resized_hw(h, w, edge, grid), (h, w, edge, grid)
+
+
+def test_front_end_argument_errors_return_before_launch(L):
+    fake = ctypes.c_void_p(256)  # never dereferenced: every case fails validation first
+    src = (ctypes.c_int32 * 2)(100, 100)
+    bad_w = (ctypes.c_int32 * 2)(28, 30)       # width not a multiple of 4
+    off_tile = (ctypes.c_int32 * 2)(1024, 1000)  # not a whole number of tiles
+    assert L.vlm_preprocess(fake, src, 1, bad_w, 0, fake, None) == vlm.ERR_BAD_SHAPE
+    assert L.vlm_preprocess(fake, src, 1, off_tile, 1024, fake, None) == vlm.ERR_BAD_SHAPE
+    assert L.vlm_preprocess(fake, src, 0, src, 0, fake, None) == vlm.ERR_INVALID_ARG
+    assert L.vlm_preprocess(fake, src, 1, src, 6, fake, None) == vlm.ERR_BAD_SHAPE  # tile % 4
+    assert L.vlm_preprocess(fake, src, 1, src, 0, ctypes.c_void_p(260), None) == vlm.ERR_INVALID_ARG  # unaligned
+    oh, ow = ctypes.c_int32(), ctypes.c_int32()
+    assert L.vlm_resize_target(0, 5, 1540, 28, ctypes.byref(oh), ctypes.byref(ow)) == vlm.ERR_INVALID_ARG
+    # placeholder expansion: output too small, and more images than ids
+    counts = (ctypes.c_int64 * 2)(100, 200)
+    n_out = ctypes.c_int64()
+    ws = ctypes.c_void_p(1 << 20)
+    assert L.vlm_expand_placeholders(fake, 10, 99, counts, 2, 10, fake, 100, ctypes.byref(n_out), ws, 1 << 20, fake,
+                                     None) == vlm.ERR_WORKSPACE
+    assert n_out.value == 0
+    zero = (ctypes.c_int64 * 2)(0, 0)
+    assert L.vlm_expand_placeholders(fake, 1, 99, zero, 2, 10, fake, 100, ctypes.byref(n_out), ws, 1 << 20, fake,
+                                     None) == vlm.ERR_BAD_SHAPE
+    assert L.vlm_expand_placeholders(fake, 0, 99, zero, 0, 10, fake, 0, ctypes.byref(n_out), ws, 0, fake,
+                                     None) == vlm.OK and n_out.value == 0

@@ -453,3 +453,12 @@ def test_expand_placeholders_definition():
     # the pages' count: one 896x1344 image is 1,536 placeholders
     h, w = O.merged_grid(*O.patch_grid(896, 1344, 14), 2)
     assert int((O.expand_placeholders(np.array([7, 99, 8]), 99, [h * w], 10) == 10).sum()) == 1536
+
+
+def test_pixels_from_u8_layout_and_scale():
+    img = np.zeros((2, 3, 3), dtype=np.uint8)
+    img[1, 2] = (255, 0, 51)   # pixel at row 1, column 2
+    x = O.pixels_from_u8(img)
+    assert x.shape == (3, 2, 3)
+    assert x[0, 1, 2] == 1.0 and x[1, 1, 2] == 0.0 and x[2, 1, 2] == pytest.approx(0.2, abs=1e-15)
+    assert np.count_nonzero(x) == 2

@@ -2,6 +2,8 @@
 // vlm_encode / vlm_merge_project / vlm_scatter (declared in include/vlm.h and
 // include/vlm_kernels.h).
 #include <algorithm>
+#include <climits>
+#include <cmath>
 #include <atomic>
 #include <vector>
 
@@ -529,6 +531,120 @@ int vlm_scatter(const int64_t* d_input_ids, int64_t n_tokens, int64_t image_toke
   if (ws_bytes < used) return VLM_ERR_WORKSPACE;
   return launch_scatter(d_input_ids, n_tokens, image_token_id, d_image_embeds, n_image_tokens, d_text_embeds,
                         row_bytes, ws, d_status, as_stream(stream));
+}
+
+int vlm_resize_target(int32_t height, int32_t width, int32_t longest_edge, int32_t grid, int32_t* out_h,
+                      int32_t* out_w) {
+  if (out_h == nullptr || out_w == nullptr || height <= 0 || width <= 0 || longest_edge <= 0 || grid <= 0)
+    return VLM_ERR_INVALID_ARG;
+  double h = height, w = width;
+  const double ratio = static_cast<double>(std::max(height, width)) / static_cast<double>(longest_edge);
+  if (ratio > 1.0) {
+    h = std::floor(h / ratio);
+    w = std::floor(w / ratio);
+  }
+  const int64_t hh = std::max<int64_t>(static_cast<int64_t>(h), 1), ww = std::max<int64_t>(static_cast<int64_t>(w), 1);
+  const int64_t rh = (hh + grid - 1) / grid * grid, rw = (ww + grid - 1) / grid * grid;
+  if (rh > (1LL << 30) || rw > (1LL << 30)) return VLM_ERR_BAD_SHAPE;
+  *out_h = static_cast<int32_t>(rh);
+  *out_w = static_cast<int32_t>(rw);
+  return VLM_OK;
+}
+
+int vlm_preprocess(const uint8_t* d_src, const int32_t* src_hw, int n_images, const int32_t* out_hw, int32_t tile,
+                   float* d_out, void* stream) {
+  if (d_src == nullptr || src_hw == nullptr || out_hw == nullptr || d_out == nullptr || n_images <= 0 || tile < 0)
+    return VLM_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(d_out) | reinterpret_cast<uintptr_t>(d_src)) & 15) return VLM_ERR_INVALID_ARG;
+  if (tile % 4) return VLM_ERR_BAD_SHAPE;
+  for (int i = 0; i < n_images; ++i) {
+    const int32_t sh = src_hw[2 * i], sw = src_hw[2 * i + 1], oh = out_hw[2 * i], ow = out_hw[2 * i + 1];
+    if (sh <= 0 || sw <= 0 || oh <= 0 || ow <= 0 || ow % 4) return VLM_ERR_BAD_SHAPE;
+    if (sh > 65536 || sw > 65536 || oh > 32768 || ow > 32768) return VLM_ERR_BAD_SHAPE;
+    if (tile > 0 && (oh % tile || ow % tile)) return VLM_ERR_BAD_SHAPE;
+  }
+  cudaStream_t s = as_stream(stream);
+  int64_t src_bytes = 0;
+  for (int i = 0; i < n_images; ++i) src_bytes += 3LL * src_hw[2 * i] * src_hw[2 * i + 1];
+  int64_t src_off = 0, dst_off = 0;
+  for (int first = 0; first < n_images; first += kResizeChunk) {
+    ResizeChunk ch;
+    ch.count = std::min(kResizeChunk, n_images - first);
+    ch.tile = tile;
+    ch.wide = 0;
+    int64_t units = 0, stage = 0;
+    for (int k = 0; k < ch.count; ++k) {
+      const int i = first + k;
+      const int64_t sh = src_hw[2 * i], sw = src_hw[2 * i + 1], oh = out_hw[2 * i], ow = out_hw[2 * i + 1];
+      ch.sh[k] = static_cast<int32_t>(sh); ch.sw[k] = static_cast<int32_t>(sw);
+      ch.oh[k] = static_cast<int32_t>(oh); ch.ow[k] = static_cast<int32_t>(ow);
+      const int64_t nseg = (ow + kResizeSegMax - 1) / kResizeSegMax;
+      const int64_t segw = ((ow + nseg - 1) / nseg + 3) / 4 * 4;
+      ch.nseg[k] = static_cast<int32_t>(nseg);
+      ch.segw[k] = static_cast<int32_t>(segw);
+      ch.sq[k] = static_cast<int32_t>((2 * sw) / (2 * ow));
+      ch.sr[k] = static_cast<int32_t>((2 * sw) % (2 * ow));
+      ch.inv_den_x[k] = static_cast<float>(1.0 / (2.0 * ow));
+      ch.inv_den_y[k] = static_cast<float>(1.0 / (2.0 * oh));
+      if ((2 * ow + 1) * sw > INT32_MAX || (2 * oh + 1) * sh > INT32_MAX) ch.wide = 1;
+      ch.unit_off[k] = static_cast<int32_t>(units);
+      ch.src_off[k] = src_off;
+      ch.dst_off[k] = dst_off;
+      units += oh * nseg;
+      // source columns one segment's taps can touch: floor((segw - 1) sw / ow) + 3
+      const int64_t cols = std::min<int64_t>((segw - 1) * sw / ow + 3, sw);
+      stage = std::max<int64_t>(stage, (3 * cols + 15 + 15) / 16 * 16);
+      src_off += 3 * sh * sw;
+      dst_off += 3 * oh * ow;
+    }
+    ch.unit_off[ch.count] = static_cast<int32_t>(units);
+    ch.stage_bytes = stage <= kResizeStageMax ? static_cast<int32_t>(stage) : 0;
+    VLM_TRY(launch_resize_tile(d_src, src_bytes, ch, d_out, s));
+  }
+  return VLM_OK;
+}
+
+size_t vlm_expand_placeholders_workspace_size(int64_t n_ids, int n_images) {
+  if (n_ids < 0 || n_images < 0) return 0;
+  Carver cv(nullptr);
+  const int64_t chunks = (n_ids + 255) / 256;
+  cv.take<int32_t>(chunks > 0 ? chunks : 1);
+  cv.take<int64_t>(chunks > 0 ? chunks : 1);
+  cv.take<int64_t>(static_cast<size_t>(n_images) + 1);
+  cv.take<int32_t>(1);
+  return cv.used;
+}
+
+int vlm_expand_placeholders(const int64_t* d_input_ids, int64_t n_ids, int64_t marker_id, const int64_t* counts,
+                            int n_images, int64_t image_token_id, int64_t* d_out_ids, int64_t out_capacity,
+                            int64_t* out_len, void* d_workspace, size_t ws_bytes, int32_t* d_status, void* stream) {
+  if (n_ids == 0 && n_images == 0 && out_len != nullptr) {
+    *out_len = 0;
+    return VLM_OK;
+  }
+  if (n_ids <= 0 || n_images < 0 || d_input_ids == nullptr || d_out_ids == nullptr || out_len == nullptr ||
+      d_workspace == nullptr || d_status == nullptr || (n_images > 0 && counts == nullptr))
+    return VLM_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(d_workspace) & 255) return VLM_ERR_INVALID_ARG;
+  if (n_ids > (1LL << 40)) return VLM_ERR_BAD_SHAPE;
+  int64_t total = n_ids - n_images;
+  for (int i = 0; i < n_images; ++i) {
+    if (counts[i] < 0 || counts[i] > (1LL << 40)) return VLM_ERR_BAD_SHAPE;
+    total += counts[i];
+  }
+  if (total < 0) return VLM_ERR_BAD_SHAPE;  // more images than ids
+  if (total > out_capacity) return VLM_ERR_WORKSPACE;
+  if (ws_bytes < vlm_expand_placeholders_workspace_size(n_ids, n_images)) return VLM_ERR_WORKSPACE;
+  Carver cv(d_workspace);
+  const int64_t chunks = (n_ids + 255) / 256;
+  ExpandWs ws;
+  ws.chunk_count = cv.take<int32_t>(chunks);
+  ws.chunk_base = cv.take<int64_t>(chunks);
+  ws.prefix = cv.take<int64_t>(static_cast<size_t>(n_images) + 1);
+  ws.ok_flag = cv.take<int32_t>(1);
+  *out_len = total;
+  return launch_expand(d_input_ids, n_ids, marker_id, counts, n_images, image_token_id, d_out_ids, ws, d_status,
+                       as_stream(stream));
 }
 
 int64_t vlm_launch_count(void) { return g_launches.load(); }

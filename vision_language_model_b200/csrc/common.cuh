@@ -21,7 +21,7 @@ namespace vlm {
 // ---------------------------------------------------------------------------
 enum KernelClass : int {
   KC_GEMM = 0, KC_ATTN = 1, KC_NORM = 2, KC_IM2COL = 3, KC_MERGE = 4,
-  KC_SCATTER = 5, KC_SETUP = 6, KC_PACK = 7, KC_COUNT = 8
+  KC_SCATTER = 5, KC_SETUP = 6, KC_PACK = 7, KC_FRONT = 8, KC_EXPAND = 9, KC_COUNT = 10
 };
 // Called around every launch: counts launches and, when profiling is on,
 // records a CUDA event pair on the launch stream.

@@ -32,6 +32,39 @@ struct ScatterWs {
   int32_t* ok_flag;
 };
 
+// Up to kResizeChunk images of one resize launch, passed by value.
+constexpr int kResizeChunk = 32;
+constexpr int kResizeSegMax = 512;        // output pixels per work unit (a row segment)
+constexpr int kResizeStageMax = 48 * 1024;  // largest staged source span per row
+struct ResizeChunk {
+  int32_t count;
+  int32_t tile;          // 0: no tiling
+  int32_t wide;          // 1: (2 out + 1) * in overflows int32 for some image: 64-bit coordinates
+  int32_t stage_bytes;   // shared memory per staged source row span; 0: taps read global memory
+  int32_t sh[kResizeChunk], sw[kResizeChunk];  // source size (pixels)
+  int32_t oh[kResizeChunk], ow[kResizeChunk];  // output size (pixels)
+  int32_t nseg[kResizeChunk], segw[kResizeChunk];  // row segments per output row, and their width
+  int32_t sq[kResizeChunk], sr[kResizeChunk];  // 2 sw = sq * (2 ow) + sr
+  float inv_den_x[kResizeChunk], inv_den_y[kResizeChunk];  // 1 / (2 ow), 1 / (2 oh)
+  int32_t unit_off[kResizeChunk + 1];          // first work unit of each image in this chunk
+  int64_t src_off[kResizeChunk];               // first byte of each source image
+  int64_t dst_off[kResizeChunk];               // first float of each output image
+};
+
+// Up to kI64Chunk int64 values written by one launch (table upload without a copy call).
+constexpr int kI64Chunk = 256;
+struct I64Chunk {
+  int32_t first, count;
+  int64_t v[kI64Chunk];
+};
+
+struct ExpandWs {
+  int32_t* chunk_count;
+  int64_t* chunk_base;
+  int64_t* prefix;
+  int32_t* ok_flag;
+};
+
 // Query rows per attention CTA tile.
 constexpr int kAttnBQ = 128;
 
@@ -49,6 +82,12 @@ int launch_merge_norm(const __nv_bfloat16* x, const float* g, const ImgInfo* inf
                       cudaStream_t s);
 int launch_scatter(const int64_t* ids, int64_t n, int64_t token, const void* img, int64_t n_img,
                    void* text, int64_t row_bytes, ScatterWs ws, int32_t* status, cudaStream_t s);
+int launch_marker_count(const int64_t* ids, int64_t n, int64_t token, int32_t* chunk_count, cudaStream_t s);
+int launch_marker_scan(const int32_t* chunk_count, int64_t n_chunks, int64_t expected, int64_t* chunk_base,
+                       int32_t* ok_flag, int32_t* status, cudaStream_t s);
+int launch_resize_tile(const uint8_t* src, int64_t src_bytes, const ResizeChunk& ch, float* dst, cudaStream_t s);
+int launch_expand(const int64_t* ids, int64_t n, int64_t marker, const int64_t* counts, int n_images,
+                  int64_t image_token, int64_t* out, ExpandWs ws, int32_t* status, cudaStream_t s);
 int launch_pack_gate_up(const void* gate, const void* up, void* dst, int64_t f, int64_t d, cudaStream_t s);
 int launch_pack_cols(const void* src, void* dst, int64_t rows, int64_t src_cols, int64_t dst_cols, int mode,
                      int mm, cudaStream_t s);

@@ -466,6 +466,20 @@ int launch_scatter(const int64_t* ids, int64_t n, int64_t token, const void* img
   return e == cudaSuccess ? VLM_OK : VLM_ERR_CUDA;
 }
 
+// The scatter's first two kernels, reused by the placeholder expansion (the
+// caller brackets them with its own launch_begin / launch_end).
+int launch_marker_count(const int64_t* ids, int64_t n, int64_t token, int32_t* chunk_count, cudaStream_t s) {
+  const dim3 chunks(static_cast<unsigned>((n + 255) / 256));
+  return launch_pdl(scatter_count_kernel, chunks, dim3(256), 0, s, ids, n, token, chunk_count) == cudaSuccess
+             ? VLM_OK : VLM_ERR_CUDA;
+}
+
+int launch_marker_scan(const int32_t* chunk_count, int64_t n_chunks, int64_t expected, int64_t* chunk_base,
+                       int32_t* ok_flag, int32_t* status, cudaStream_t s) {
+  return launch_pdl(scatter_scan_kernel, dim3(1), dim3(1024), 0, s, chunk_count, n_chunks, expected, chunk_base,
+                    ok_flag, status) == cudaSuccess ? VLM_OK : VLM_ERR_CUDA;
+}
+
 int launch_pack_gate_up(const void* gate, const void* up, void* dst, int64_t f, int64_t d, cudaStream_t s) {
   const int64_t vec = d * 2 / 16;
   launch_begin(KC_PACK, s);

@@ -70,6 +70,26 @@ def pixels_u01(seed: int, name: str, height: int, width: int) -> torch.Tensor:
     return torch.rand((3, height, width), generator=generator(seed, name), dtype=torch.float32)
 
 
+def photo_u8(seed: int, name: str, height: int, width: int) -> torch.Tensor:
+    """uint8 [H, W, 3] RGB image as a decoder returns it: per channel a mean
+    level plus three random low-frequency plane waves (1-4 periods across the
+    image, like the slow shading of a photograph) plus uniform +-24 grain,
+    rounded and clipped to [0, 255]."""
+    g = generator(seed, name)
+    y = torch.arange(height, dtype=torch.float64)[:, None] / height
+    x = torch.arange(width, dtype=torch.float64)[None, :] / width
+    chans = []
+    for _ in range(3):
+        p = torch.rand(10, generator=g, dtype=torch.float64)
+        field = 60.0 + 135.0 * p[0]
+        for k in range(3):
+            fy, fx, ph = 1.0 + 3.0 * p[1 + 3 * k], 1.0 + 3.0 * p[2 + 3 * k], 6.283185307179586 * p[3 + 3 * k]
+            field = field + 30.0 * torch.sin(6.283185307179586 * (fy * y + fx * x) + ph)
+        grain = (torch.rand((height, width), generator=g, dtype=torch.float64) - 0.5) * 48.0
+        chans.append(field + grain)
+    return torch.stack(chans, -1).clamp(0, 255).round().to(torch.uint8).contiguous()
+
+
 # ---------------------------------------------------------------------------
 # Model hyperparameters of the synthetic towers (shapes only)
 # ---------------------------------------------------------------------------
@@ -153,6 +173,18 @@ def text_sequences(seed: int, n_seq: int, seq_len: int, runs, image_token_id: in
             prev = cut
             ids[s, pos:pos + run] = image_token_id
             pos += run
+    return ids
+
+
+def prompt_with_markers(seed: int, n_text: int, n_images: int, marker_id: int, vocab: int = 131072,
+                        lo_id: int = 11) -> torch.Tensor:
+    """int64 [n_text + n_images] ids: U[lo_id, vocab) text with one marker_id
+    per image at seeded, distinct positions (a prompt before expansion)."""
+    g = generator(seed, "prompt_ids")
+    n = n_text + n_images
+    ids = torch.randint(lo_id, vocab, (n,), generator=g, dtype=torch.int64)
+    where = torch.randperm(n, generator=generator(seed, "marker_positions"))[:n_images]
+    ids[where] = marker_id
     return ids
 
 

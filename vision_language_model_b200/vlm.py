@@ -21,7 +21,8 @@ OK, ERR_INVALID_ARG, ERR_BAD_SHAPE, ERR_WORKSPACE, ERR_COUNT_MISMATCH, ERR_TIMEO
 # epilogues (include/vlm_kernels.h)
 EPI_BF16, EPI_F32, EPI_RESID, EPI_SWIGLU, EPI_ROPE, EPI_GELU = range(6)
 # profiling kernel classes
-KCLASS = {"gemm": 0, "attention": 1, "rmsnorm": 2, "im2col": 3, "merge": 4, "scatter": 5, "setup": 6, "pack": 7}
+KCLASS = {"gemm": 0, "attention": 1, "rmsnorm": 2, "im2col": 3, "merge": 4, "scatter": 5, "setup": 6, "pack": 7,
+          "resize": 8, "expand": 9}
 
 
 class VlmError(RuntimeError):
@@ -77,6 +78,11 @@ def lib() -> ctypes.CDLL:
             "vlm_merge_project": (I32, [CP, P, P, I32, P, P, P, SZ, P, P]),
             "vlm_scatter_workspace_size": (SZ, [I64]),
             "vlm_scatter": (I32, [P, I64, I64, P, I64, P, I64, P, SZ, P, P]),
+            "vlm_resize_target": (I32, [I32, I32, I32, I32, ctypes.POINTER(ctypes.c_int32),
+                                        ctypes.POINTER(ctypes.c_int32)]),
+            "vlm_preprocess": (I32, [P, P, I32, P, I32, P, P]),
+            "vlm_expand_placeholders_workspace_size": (SZ, [I64, I32]),
+            "vlm_expand_placeholders": (I32, [P, I64, I64, P, I32, I64, P, I64, ctypes.POINTER(I64), P, SZ, P, P]),
             "vlm_launch_count": (I64, []),
             "vlm_profile_enable": (I32, [I32]),
             "vlm_profile_query": (I32, [I32, ctypes.POINTER(I64), ctypes.POINTER(ctypes.c_double)]),
@@ -277,6 +283,75 @@ def scatter(input_ids: torch.Tensor, image_embeds: torch.Tensor, text_embeds: to
 # ---------------------------------------------------------------------------
 # Per-kernel entry points
 # ---------------------------------------------------------------------------
+
+# ---------------------------------------------------------------------------
+# Image front end and placeholder expansion
+# ---------------------------------------------------------------------------
+
+def resize_target(height: int, width: int, longest_edge: int = 1540, grid: int = 28) -> tuple:
+    """The processor's resize size (host only): see vlm_resize_target."""
+    oh, ow = ctypes.c_int32(), ctypes.c_int32()
+    _check(lib().vlm_resize_target(int(height), int(width), int(longest_edge), int(grid), ctypes.byref(oh),
+                                   ctypes.byref(ow)), "vlm_resize_target")
+    return oh.value, ow.value
+
+
+def preprocess(images_u8: torch.Tensor, src_hw, out_hw, tile: int = 0, out=None, stream=None) -> torch.Tensor:
+    """Bilinear resize of decoded u8 RGB HWC images (concatenated, flat) onto out_hw.
+
+    Returns fp32 [3*sum(oh*ow)] CHW blocks in [0, 1]; with tile > 0 each image
+    is written as its row-major tiles of [3, tile, tile].
+    """
+    if images_u8.dtype != torch.uint8:
+        raise ValueError("images_u8 must be uint8")
+    src_arr, n = _hw_array(src_hw)
+    out_arr, n_out = _hw_array(out_hw)
+    if n != n_out:
+        raise ValueError("src_hw and out_hw must list the same images")
+    need_src = sum(3 * int(h) * int(w) for h, w in src_hw)
+    if images_u8.numel() != need_src:
+        raise ValueError(f"images_u8 holds {images_u8.numel()} bytes, the sizes need {need_src}")
+    total = sum(3 * int(h) * int(w) for h, w in out_hw)
+    if out is None:
+        out = torch.empty(total, dtype=torch.float32, device=images_u8.device)
+    elif out.numel() < total or out.dtype != torch.float32:
+        raise ValueError("out must be fp32 with room for every output pixel")
+    _check(lib().vlm_preprocess(_dev(images_u8, "images_u8"), src_arr, n, out_arr, int(tile), _dev(out, "out"),
+                                _stream(stream)), "vlm_preprocess")
+    return out
+
+
+def tiled_hw(out_hw, tile: int) -> list:
+    """Image table that vlm_encode takes for the output of preprocess(..., tile)."""
+    return [(tile, tile)] * sum((int(h) // tile) * (int(w) // tile) for h, w in out_hw)
+
+
+def expand_placeholders_workspace_size(n_ids: int, n_images: int) -> int:
+    return int(lib().vlm_expand_placeholders_workspace_size(int(n_ids), int(n_images)))
+
+
+def expand_placeholders(input_ids: torch.Tensor, marker_id: int, counts, image_token_id: int = 10, out=None,
+                        workspace=None, status=None, stream=None) -> torch.Tensor:
+    """Each marker_id (in order) becomes counts[k] copies of image_token_id; returns int64 ids."""
+    L = lib()
+    n_ids = input_ids.numel()
+    n_img = len(counts)
+    carr = (ctypes.c_int64 * max(1, n_img))(*[int(c) for c in counts])
+    total = n_ids - n_img + sum(int(c) for c in counts)
+    if out is None:
+        out = torch.empty(max(total, 0), dtype=torch.int64, device=input_ids.device)
+    ws_need = L.vlm_expand_placeholders_workspace_size(n_ids, n_img)
+    if workspace is None:
+        workspace = torch.empty(max(ws_need, 256), dtype=torch.uint8, device=input_ids.device)
+    if status is None:
+        status = new_status(input_ids.device)
+    out_len = ctypes.c_int64()
+    _check(L.vlm_expand_placeholders(_dev(input_ids, "input_ids"), n_ids, int(marker_id), carr, n_img,
+                                     int(image_token_id), _dev(out, "out"), out.numel(), ctypes.byref(out_len),
+                                     _dev(workspace, "workspace"), workspace.numel(), _dev(status, "status"),
+                                     _stream(stream)), "vlm_expand_placeholders")
+    return out[:out_len.value]
+
 
 def gemm(epilogue: int, a: torch.Tensor, b: torch.Tensor, out: torch.Tensor, out_bf16=None, pos=None,
          rope_table=None, rope_cols: int = 0, status=None, stream=None) -> torch.Tensor:
