@@ -64,6 +64,10 @@ def parse_args():
     p.add_argument("--workload", default="mistral3_1540", choices=sorted(WORKLOADS))
     p.add_argument("--seed", type=int, default=0)
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--graph", action="store_true",
+                   help="replay each step as one captured CUDA graph (headline and e2e loops)")
+    p.add_argument("--side-stream", action="store_true",
+                   help="also measure the encoder on a side stream overlapped with a decode-like GEMV loop")
     p.add_argument("--profile-steps", type=int, default=0,
                    help="for ncu: run this many plain steps after warmup and exit (no JSON)")
     return p.parse_args()
@@ -322,6 +326,81 @@ KERNEL_SOURCES = {"attention": ["attention_tc.cu", "exp2_poly.cuh", "common.cuh"
                   "resize": ["frontend.cu", "common.cuh", "kernels.cuh"]}
 
 
+def side_stream_overlap(pipe, pix, ids, text, cfg, scatter_ws, dev, steps: int) -> dict:
+    """The image path on a side stream while another stream runs a decode-like
+    loop (bf16 GEMVs [8, 5120] x [5120, 5120]^T over 48 distinct weight
+    matrices, 2.5 GB read per pass: memory-bound, like a decoder step). Times
+    each alone, then both together with the decode loop on a default-priority
+    and on a high-priority stream; CUDA events on the launching streams."""
+    from vision_language_model_b200 import vlm
+
+    main = torch.cuda.current_stream(dev)
+    w = torch.empty((48, 5120, 5120), dtype=torch.bfloat16, device=dev).normal_(0, 0.02)
+    x = torch.empty((8, 5120), dtype=torch.bfloat16, device=dev).normal_()
+    y = torch.empty((8, 5120), dtype=torch.bfloat16, device=dev)
+
+    def decode_pass():
+        for i in range(48):
+            torch.matmul(x, w[i].t(), out=y)
+
+    side = vlm.EncoderSideStream(pipe)
+
+    def encode_request():
+        side.submit(pix)
+        side.scatter(ids, text, workspace=scatter_ws)
+
+    def time_it(fn, reps):
+        for _ in range(2):
+            fn()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(main)
+        for _ in range(reps):
+            fn()
+        b.record(main)
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / reps
+
+    enc_ms = time_it(encode_request, steps)
+    dec_ms = time_it(decode_pass, 20)
+    n_dec = max(1, round(enc_ms / dec_ms))
+
+    def concurrent(priority):
+        dstream = torch.cuda.Stream(device=dev, priority=priority)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        totals, decs = [], []
+        for rep in range(steps + 2):
+            torch.cuda.synchronize()
+            a.record(main)
+            side.submit(pix)
+            dstream.wait_stream(main)
+            with torch.cuda.stream(dstream):
+                d0.record(dstream)
+                for _ in range(n_dec):
+                    decode_pass()
+                d1.record(dstream)
+            main.wait_stream(dstream)
+            side.scatter(ids, text, workspace=scatter_ws)
+            b.record(main)
+            torch.cuda.synchronize()
+            if rep >= 2:
+                totals.append(a.elapsed_time(b))
+                decs.append(d0.elapsed_time(d1) / n_dec)
+        return sum(totals) / len(totals), sum(decs) / len(decs)
+
+    both_ms, dec_conc = concurrent(0)
+    both_hi_ms, dec_conc_hi = concurrent(-1)
+    serial = enc_ms + n_dec * dec_ms
+    del w
+    return {"encode_ms": enc_ms, "decode_pass_ms": dec_ms, "decode_passes": n_dec, "serial_ms": serial,
+            "overlapped_ms": both_ms, "decode_pass_ms_during_encode": dec_conc,
+            "overlapped_ms_decode_high_priority": both_hi_ms, "decode_pass_ms_during_encode_high_priority": dec_conc_hi,
+            "hidden_frac": (serial - both_ms) / min(enc_ms, n_dec * dec_ms),
+            "note": "encoder + scatter of one request on a side stream, decode-like GEMV passes on another stream; "
+                    "hidden_frac = time saved against running them one after the other / the shorter of the two"}
+
+
 def run_ours(args, wl):
     from vision_language_model_b200 import synth, vlm
 
@@ -386,6 +465,9 @@ def run_ours(args, wl):
         torch.cuda.synchronize()
         return
 
+    graph = vlm.GraphStep(step, warmup=0) if args.graph else None
+    run_step = graph if graph is not None else step
+
     def timed(profile: bool) -> float:
         """Device milliseconds of args.steps steps, bracketed by barrier + synchronize."""
         vlm.profile_enable(profile)
@@ -394,7 +476,7 @@ def run_ours(args, wl):
         torch.cuda.synchronize()
         start.record(stream)
         for _ in range(args.steps):
-            step()
+            (step if profile else run_step)()
         stop.record(stream)
         torch.cuda.synchronize()
         barrier(world)
@@ -406,6 +488,8 @@ def run_ours(args, wl):
     launches0 = vlm.launch_count()
     ms = timed(False)
     launches = vlm.launch_count() - launches0
+    if graph is not None:  # replays launch the captured kernels without calling the library
+        launches = graph.launches_per_replay * args.steps
     clk = clocks.stop()
     ms_max = max_over_ranks(world, ms)
     # ---- the same steps again with a CUDA event pair around every launch: per-kernel times ----
@@ -429,7 +513,7 @@ def run_ours(args, wl):
     for _ in range(args.steps):
         (photo_dev if photo else pix).copy_(pix_host, non_blocking=True)
         (marker_ids if photo else ids).copy_(ids_host, non_blocking=True)
-        step()
+        run_step()
         out_host.copy_(text, non_blocking=True)
     e_stop.record(stream)
     torch.cuda.synchronize()
@@ -503,6 +587,10 @@ def run_ours(args, wl):
                        "traffic": ncu_traffic("resize")},
             "expand_ms_per_step": ms_expand / args.steps,
         }
+    if args.graph:
+        line["config"]["launch"] = f"one CUDA graph per step ({graph.launches_per_replay} kernels)"
+    if args.side_stream:
+        line["side_stream"] = side_stream_overlap(pipe, pix, ids, text, cfg, scatter_ws, dev, args.steps)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(wl, args.seed)
     if rank == 0:

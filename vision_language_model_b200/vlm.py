@@ -445,3 +445,65 @@ class ImagePipeline:
         merge_project(self.cfg, self.tower_out, self.image_hw, self.packed_proj, out=self.embeds,
                       workspace=self.workspace, status=self.status, stream=stream)
         return self.embeds
+
+
+class GraphStep:
+    """Captures every kernel a callable launches on the current stream into one
+    CUDA graph and replays it: one host call per step instead of one per
+    kernel. The callable's buffers must stay at the same addresses (an
+    ImagePipeline's do); the kernels keep their programmatic-launch edges.
+    """
+
+    def __init__(self, fn, warmup: int = 1):
+        self.fn = fn
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            for _ in range(warmup):
+                fn()
+        torch.cuda.current_stream().wait_stream(side)
+        torch.cuda.synchronize()
+        self.graph = torch.cuda.CUDAGraph()
+        before = launch_count()
+        with torch.cuda.graph(self.graph):
+            fn()
+        self.launches_per_replay = launch_count() - before
+
+    def __call__(self) -> None:
+        self.graph.replay()
+
+
+class EncoderSideStream:
+    """Runs the image path (vlm_encode + vlm_merge_project) on its own CUDA
+    stream so it overlaps other work on the caller's stream; the caller's
+    stream waits on an event before the scatter reads the embeddings.
+
+    submit() orders the side stream after the caller's stream (the pixels were
+    written there) and after the previous scatter (which read the previous
+    embeddings from the same buffers), then enqueues the image path and
+    records `ready`. scatter() makes the caller's stream wait on `ready`,
+    scatters, and records `consumed`.
+    """
+
+    def __init__(self, pipeline: ImagePipeline, priority: int = 0):
+        self.pipe = pipeline
+        self.stream = torch.cuda.Stream(device=pipeline.embeds.device, priority=priority)
+        self.ready = torch.cuda.Event()
+        self.consumed = torch.cuda.Event()
+        self.consumed.record(torch.cuda.current_stream())
+
+    def submit(self, pixels: torch.Tensor) -> torch.cuda.Event:
+        self.stream.wait_stream(torch.cuda.current_stream())
+        self.stream.wait_event(self.consumed)
+        with torch.cuda.stream(self.stream):
+            self.pipe(pixels, stream=self.stream)
+            self.ready.record(self.stream)
+        pixels.record_stream(self.stream)
+        return self.ready
+
+    def scatter(self, input_ids: torch.Tensor, text_embeds: torch.Tensor, workspace=None, stream=None) -> None:
+        main = stream if stream is not None else torch.cuda.current_stream()
+        main.wait_event(self.ready)
+        scatter(input_ids, self.pipe.embeds, text_embeds, self.pipe.cfg.image_token_id, workspace=workspace,
+                status=self.pipe.status, stream=main)
+        self.consumed.record(main)
