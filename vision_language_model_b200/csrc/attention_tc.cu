@@ -4,8 +4,10 @@
 //
 // One CTA = one 128-query tile of one block and one head; two CTAs share an
 // SM so one CTA's softmax overlaps the other's MMAs. 6 warps:
-//   warp 0      TMA: the Q tile once, then K and V tiles of 128 keys into a
-//               2-stage ring (128-byte swizzle).
+//   warp 0      TMA: the Q tile once, then K and V tiles of 128 keys into two
+//               2-stage rings (128-byte swizzle). A K stage is released when
+//               S = Q K^T has read it and a V stage when O += P V has, so the
+//               next K load never waits for a P V product.
 //   warp 1      allocates 256 TMEM columns; one thread issues
 //                 S  = Q K^T      (tcgen05.mma kind::f16, M=128 N=128, A and B in smem)
 //                 O += P V        (M=128 N=64, A = P in TMEM, B = V in smem, MN-major)
@@ -33,9 +35,10 @@ namespace {
 constexpr int BQ = kAttnBQ;  // 128
 constexpr int BKV = 128;
 constexpr int DH = 64;
-constexpr int kStages = 2;
+constexpr int kKStages = 2;  // K ring: a stage is free once S = Q K^T has read it
+constexpr int kVStages = 2;  // V ring: a stage is free once O += P V has read it
 constexpr int kTileBytes = 128 * DH * 2;  // 16 KiB: 128 rows x 128 bytes
-constexpr int kSmemBytes = (1 + 2 * kStages) * kTileBytes + 256 + 1024;
+constexpr int kSmemBytes = (1 + kKStages + kVStages) * kTileBytes + 256 + 1024;
 constexpr uint32_t kColS = 0, kColP = 128, kColO = 192, kTmemCols = 256;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
@@ -162,13 +165,15 @@ __global__ void __launch_bounds__(192, 2)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem;
-  uint8_t* sK = smem + kTileBytes;                    // [kStages] tiles
-  uint8_t* sV = smem + (1 + kStages) * kTileBytes;    // [kStages] tiles
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (1 + 2 * kStages) * kTileBytes);
+  uint8_t* sK = smem + kTileBytes;                     // [kKStages] tiles
+  uint8_t* sV = smem + (1 + kKStages) * kTileBytes;    // [kVStages] tiles
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (1 + kKStages + kVStages) * kTileBytes);
   uint64_t* q_full = bars;
-  uint64_t* kv_full = bars + 1;               // [kStages]
-  uint64_t* kv_empty = bars + 1 + kStages;    // [kStages]
-  uint64_t* s_full = bars + 1 + 2 * kStages;
+  uint64_t* k_full = bars + 1;                          // [kKStages]
+  uint64_t* k_empty = k_full + kKStages;                // [kKStages]
+  uint64_t* v_full = k_empty + kKStages;                // [kVStages]
+  uint64_t* v_empty = v_full + kVStages;                // [kVStages]
+  uint64_t* s_full = v_empty + kVStages;
   uint64_t* s_free = s_full + 1;
   uint64_t* p_full = s_full + 2;
   uint64_t* o_done = s_full + 3;
@@ -180,9 +185,13 @@ __global__ void __launch_bounds__(192, 2)
 
   if (threadIdx.x == 0) {
     mbar_init(smem_u32(q_full), 1);
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(smem_u32(kv_full + s), 1);
-      mbar_init(smem_u32(kv_empty + s), 1);
+    for (int s = 0; s < kKStages; ++s) {
+      mbar_init(smem_u32(k_full + s), 1);
+      mbar_init(smem_u32(k_empty + s), 1);
+    }
+    for (int s = 0; s < kVStages; ++s) {
+      mbar_init(smem_u32(v_full + s), 1);
+      mbar_init(smem_u32(v_empty + s), 1);
     }
     mbar_init(smem_u32(s_full), 1);
     mbar_init(smem_u32(s_free), 128);
@@ -221,14 +230,23 @@ __global__ void __launch_bounds__(192, 2)
       const uint32_t qb = smem_u32(q_full);
       mbar_arrive_expect_tx(qb, kTileBytes);
       tma_load_2d(smem_u32(sQ), &tm_qkv, qb, h * DH, q0);
-      for (int j = 0; j < n_kv; ++j) {
-        const int st = j % kStages;
-        if (!mbar_wait(smem_u32(kv_empty + st), ((j / kStages) & 1) ^ 1, abort_v, args.status)) break;
-        const uint32_t fb = smem_u32(kv_full + st);
-        mbar_arrive_expect_tx(fb, 2 * kTileBytes);
-        const int key0 = kbeg + j * BKV;
-        tma_load_2d(smem_u32(sK + st * kTileBytes), &tm_qkv, fb, D + h * DH, key0);
-        tma_load_2d(smem_u32(sV + st * kTileBytes), &tm_qkv, fb, 2 * D + h * DH, key0);
+      // K tile j, then V tile j - 1: V is needed only after the softmax of its tile,
+      // so a V stage still being read never holds back the next K load
+      for (int j = 0; j <= n_kv; ++j) {
+        if (j < n_kv) {
+          const int st = j % kKStages;
+          if (!mbar_wait(smem_u32(k_empty + st), ((j / kKStages) & 1) ^ 1, abort_v, args.status)) break;
+          const uint32_t fb = smem_u32(k_full + st);
+          mbar_arrive_expect_tx(fb, kTileBytes);
+          tma_load_2d(smem_u32(sK + st * kTileBytes), &tm_qkv, fb, D + h * DH, kbeg + j * BKV);
+        }
+        if (j > 0) {
+          const int jv = j - 1, st = jv % kVStages;
+          if (!mbar_wait(smem_u32(v_empty + st), ((jv / kVStages) & 1) ^ 1, abort_v, args.status)) break;
+          const uint32_t fb = smem_u32(v_full + st);
+          mbar_arrive_expect_tx(fb, kTileBytes);
+          tma_load_2d(smem_u32(sV + st * kTileBytes), &tm_qkv, fb, 2 * D + h * DH, kbeg + jv * BKV);
+        }
       }
     }
   } else if (warp == 1) {
@@ -239,8 +257,8 @@ __global__ void __launch_bounds__(192, 2)
       const uint64_t qdesc = smem_desc_sw128(smem_u32(sQ));
       for (int j = 0; ok && j <= n_kv; ++j) {
         if (j < n_kv) {
-          const int st = j % kStages;
-          if (!mbar_wait(smem_u32(kv_full + st), (j / kStages) & 1, abort_v, args.status)) break;
+          const int st = j % kKStages;
+          if (!mbar_wait(smem_u32(k_full + st), (j / kKStages) & 1, abort_v, args.status)) break;
           if (j > 0 && !mbar_wait(smem_u32(s_free), (j - 1) & 1, abort_v, args.status)) break;
           tc_fence_after();
           const uint64_t kdesc = smem_desc_sw128(smem_u32(sK + st * kTileBytes));
@@ -248,17 +266,19 @@ __global__ void __launch_bounds__(192, 2)
           for (int k = 0; k < DH / 16; ++k)
             umma_bf16_ss(tmem + kColS, qdesc + 2 * k, kdesc + 2 * k, idesc_s, k > 0 ? 1u : 0u);
           umma_commit(smem_u32(s_full));
+          umma_commit(smem_u32(k_empty + st));
         }
         if (j > 0) {
-          const int jp = j - 1, st = jp % kStages;
+          const int jp = j - 1, st = jp % kVStages;
           if (!mbar_wait(smem_u32(p_full), jp & 1, abort_v, args.status)) break;
+          if (!mbar_wait(smem_u32(v_full + st), (jp / kVStages) & 1, abort_v, args.status)) break;
           tc_fence_after();
           const uint64_t vdesc = smem_desc_sw128(smem_u32(sV + st * kTileBytes));
 #pragma unroll
           for (int kk = 0; kk < BKV / 16; ++kk)  // 16 keys = 8 TMEM columns of bf16 pairs = 2048 smem bytes
             umma_bf16_ts(tmem + kColO, tmem + kColP + 8 * kk, vdesc + 128 * kk, idesc_o,
                          (jp > 0 || kk > 0) ? 1u : 0u);
-          umma_commit(smem_u32(kv_empty + st));
+          umma_commit(smem_u32(v_empty + st));
           umma_commit(smem_u32(o_done));
         }
       }
