@@ -419,6 +419,96 @@ def tower(images, tw: dict, cfg: dict, layers: int | None = None, normalize: boo
 
 
 # ---------------------------------------------------------------------------
+# FP8 (E4M3) tower GEMMs: the deployments the pages describe run FP8-native
+# checkpoints ("Mistral 3" intro; vllm.cpp issue). Reading: weights quantised
+# per output row with scale amax/448, activations with one static scale per
+# GEMM input; the four tower GEMMs of every block run on E4M3 operands with
+# fp32 accumulation; attention, norms, the patch embed and the projector stay
+# as in the bf16 path.
+# ---------------------------------------------------------------------------
+E4M3_MAX = 448.0
+
+
+def e4m3_round(x) -> np.ndarray:
+    """Nearest value of the OCP FP8 E4M3 format (finite variant: 4 exponent
+    bits with bias 7, 3 mantissa bits, largest finite 448, no infinities),
+    ties to even, saturating to +-448. Normals cover [2^-6, 448] with 8
+    steps per binade; below 2^-6 the step is the subnormal quantum 2^-9."""
+    x = np.asarray(x, dtype=np.float64)
+    a = np.abs(x)
+    _, e = np.frexp(a)                       # a = f * 2^e, f in [0.5, 1)
+    e = np.clip(e - 1, -6, 8)                # binade exponent, subnormals share 2^-6's step
+    quantum = np.ldexp(1.0, (e - 3).astype(np.int64))
+    q = np.minimum(np.round(a / quantum) * quantum, E4M3_MAX)  # np.round: half to even
+    return np.where(np.isnan(x), np.nan, np.copysign(q, x))
+
+
+def quantize_weight_rows(w) -> tuple:
+    """Per-output-row E4M3 weights: s[n] = fp32(amax_n / 448) (1 for an all-zero
+    row), q = e4m3(fp32(w / s[n])) with fp32 division. Returns (q, s) as
+    float64 [N, K] and float32 [N]."""
+    w32 = np.asarray(w, dtype=np.float32)
+    amax = np.max(np.abs(w32), axis=1)
+    sc = (amax / np.float32(E4M3_MAX)).astype(np.float32)
+    sc = np.where(sc > 0, sc, np.float32(1.0)).astype(np.float32)
+    return e4m3_round((w32 / sc[:, None]).astype(np.float32)), sc
+
+
+def fp8_linear(a, q_w: np.ndarray, s_w: np.ndarray, s_a: float) -> np.ndarray:
+    """y = x W^T with both operands in E4M3: q_a = e4m3(fp32(a) * fp32(1/s_a)),
+    y[:, n] = (q_a q_w^T)[:, n] * fp32(s_a * s_w[n])."""
+    inv = np.float32(1.0 / np.float64(np.float32(s_a)))
+    q_a = e4m3_round(np.asarray(a, dtype=np.float32) * inv)
+    colscale = (np.float32(s_a) * np.asarray(s_w, dtype=np.float32)).astype(np.float64)
+    return (q_a @ np.asarray(q_w, dtype=np.float64).T) * colscale[None, :]
+
+
+def quantize_layer(lw: dict) -> dict:
+    """E4M3 copies of one layer's GEMM weights (q and per-row scales)."""
+    out = dict(lw)
+    for n in ("wq", "wk", "wv", "wo", "w_gate", "w_up", "w_down"):
+        out[n + "_q"], out[n + "_s"] = quantize_weight_rows(lw[n])
+    return out
+
+
+def tower_block_fp8(x: np.ndarray, lq: dict, act_scales, angles: np.ndarray, cu_seqlens, cfg: dict) -> np.ndarray:
+    """tower_block() with its four GEMMs (QKV, O, gate/up, down) on E4M3
+    operands; act_scales = (s_attn_norm, s_attn_out, s_ffn_norm, s_hidden),
+    the static scales of those four GEMM inputs."""
+    t_total = x.shape[0]
+    heads, dh, eps = cfg["heads"], cfg["head_dim"], cfg["eps"]
+    xn = rms_norm(x, lq["g_attn"], eps)
+    q = fp8_linear(xn, lq["wq_q"], lq["wq_s"], act_scales[0]).reshape(t_total, heads, dh)
+    k = fp8_linear(xn, lq["wk_q"], lq["wk_s"], act_scales[0]).reshape(t_total, heads, dh)
+    v = fp8_linear(xn, lq["wv_q"], lq["wv_s"], act_scales[0]).reshape(t_total, heads, dh)
+    q = apply_rope(q, angles)
+    k = apply_rope(k, angles)
+    x = x + fp8_linear(attention(q, k, v, cu_seqlens), lq["wo_q"], lq["wo_s"], act_scales[1])
+    xn = rms_norm(x, lq["g_ffn"], eps)
+    hidden = silu(fp8_linear(xn, lq["w_gate_q"], lq["w_gate_s"], act_scales[2])) * \
+        fp8_linear(xn, lq["w_up_q"], lq["w_up_s"], act_scales[2])
+    return x + fp8_linear(hidden, lq["w_down_q"], lq["w_down_s"], act_scales[3])
+
+
+def tower_fp8(images, tw: dict, act_scales, cfg: dict, layers: int | None = None,
+              normalize: bool = True) -> np.ndarray:
+    """tower() with tower_block_fp8 blocks; act_scales[l] holds layer l's four
+    static activation scales."""
+    p, eps = cfg["patch"], cfg["eps"]
+    n_layers = cfg["layers"] if layers is None else layers
+    grids = [patch_grid(im.shape[1], im.shape[2], p) for im in images]
+    rows, cols, cu = positions(grids)
+    w_pe = np.asarray(tw["w_pe"], dtype=np.float64)
+    x = np.concatenate([patch_embed(normalize_pixels(im) if normalize else np.asarray(im, np.float64), w_pe)
+                        for im in images], axis=0)
+    x = rms_norm(x, tw["g_pre"], eps)
+    angles = rope_angles(rows, cols, cfg["rope_theta"], cfg["head_dim"])
+    for layer in range(n_layers):
+        x = tower_block_fp8(x, quantize_layer(layer_weights(tw, layer)), act_scales[layer], angles, cu, cfg)
+    return x
+
+
+# ---------------------------------------------------------------------------
 # a12..a14: patch-merging projector
 # ---------------------------------------------------------------------------
 

@@ -462,3 +462,118 @@ def test_pixels_from_u8_layout_and_scale():
     assert x.shape == (3, 2, 3)
     assert x[0, 1, 2] == 1.0 and x[1, 1, 2] == 0.0 and x[2, 1, 2] == pytest.approx(0.2, abs=1e-15)
     assert np.count_nonzero(x) == 2
+
+
+# ---------------------------------------------------------------------------
+# FP8 (E4M3) tower GEMMs
+# ---------------------------------------------------------------------------
+
+def _e4m3_codes():
+    """All finite E4M3 values from the bit layout s.eeee.mmm (bias 7, code 0x7F/0xFF are NaN)."""
+    vals = []
+    for code in range(256):
+        sign = -1.0 if code & 0x80 else 1.0
+        e, m = (code >> 3) & 0xF, code & 7
+        if e == 15 and m == 7:
+            continue
+        vals.append(sign * (m / 8.0) * 2.0 ** -6 if e == 0 else sign * (1 + m / 8.0) * 2.0 ** (e - 7))
+    return np.unique(np.array(vals))
+
+
+def test_e4m3_codes_are_fixed_points_and_range():
+    codes = _e4m3_codes()
+    assert codes.max() == 448.0 and codes.min() == -448.0
+    assert len(codes) == 253  # 254 finite codes, +0 and -0 collapse
+    np.testing.assert_array_equal(O.e4m3_round(codes), codes)
+
+
+def test_e4m3_midpoints_round_to_even_mantissa():
+    pos = _e4m3_codes()
+    pos = pos[pos >= 0]
+    mids = (pos[:-1] + pos[1:]) / 2
+    got = O.e4m3_round(mids)
+    for lo, hi, g in zip(pos[:-1], pos[1:], got):
+        # the even neighbour has an even mantissa field: its value / quantum is even
+        _, e = np.frexp(lo if lo > 0 else hi)
+        q = 2.0 ** (max(min(e - 1, 8), -6) - 3)
+        even = lo if round(lo / q) % 2 == 0 else hi
+        assert g == even, (lo, hi, g)
+
+
+def test_e4m3_matches_torch_float8_and_saturates():
+    rng = np.random.default_rng(8)
+    mag = np.exp2(rng.uniform(-12, np.log2(460), 200000))
+    x = (mag * rng.choice([-1.0, 1.0], mag.size)).astype(np.float32)
+    ref = torch.from_numpy(x).to(torch.float8_e4m3fn).to(torch.float64).numpy()
+    np.testing.assert_array_equal(O.e4m3_round(x), ref)
+    np.testing.assert_array_equal(O.e4m3_round([464.0001, 1e6, -1e30]), [448.0, 448.0, -448.0])
+    assert np.isnan(O.e4m3_round([np.nan]))[0]
+
+
+def test_quantize_weight_rows_scale_and_error_bound():
+    w = RNG.standard_normal((16, 96)).astype(np.float32) * 0.02
+    w[3] = 0.0
+    q, s = O.quantize_weight_rows(w)
+    assert s.dtype == np.float32 and s[3] == 1.0 and np.all(q[3] == 0)
+    amax_idx = np.argmax(np.abs(w), axis=1)
+    for n in range(16):
+        if n != 3:
+            assert abs(q[n, amax_idx[n]]) == 448.0
+    rec = q * s[:, None].astype(np.float64)
+    normal = np.abs(w) >= 2.0 ** -6 * s[:, None]
+    assert np.all(np.abs(rec - w)[normal] <= np.abs(w)[normal] * 2.0 ** -4 * (1 + 1e-6))
+
+
+def test_fp8_linear_exact_on_representable_inputs():
+    """With activations on the scaled E4M3 grid and a power-of-two scale the
+    activation quantisation is exact, so fp8_linear equals a plain matmul with
+    the dequantised weights."""
+    codes = _e4m3_codes()
+    a = RNG.choice(codes[np.abs(codes) <= 64], size=(5, 32)) * 0.25
+    w = RNG.standard_normal((7, 32)) * 0.05
+    q_w, s_w = O.quantize_weight_rows(w)
+    got = O.fp8_linear(a, q_w, s_w, 0.25)
+    ref = (a / 0.25) @ q_w.T * (np.float32(0.25) * s_w.astype(np.float32)).astype(np.float64)[None, :]
+    np.testing.assert_allclose(got, ref, rtol=1e-15, atol=0)
+    np.testing.assert_allclose(got, a @ (q_w * s_w[:, None].astype(np.float64)).T, rtol=1e-12, atol=1e-15)
+
+
+def test_tower_block_fp8_close_to_bf16_block():
+    """The E4M3 block stays within E4M3's quantisation error of the exact block
+    and differs from it (the quantisation is really applied)."""
+    t, d, f = 24, 64, 128
+    cfg = dict(O.MISTRAL3, width=d, heads=1, mlp=f)
+    lw = {n: RNG.standard_normal(sh) * 0.05 for n, sh in
+          (("wq", (d, d)), ("wk", (d, d)), ("wv", (d, d)), ("wo", (d, d)), ("w_gate", (f, d)), ("w_up", (f, d)),
+           ("w_down", (d, f)))}
+    lw["g_attn"] = 1 + 0.02 * RNG.standard_normal(d)
+    lw["g_ffn"] = 1 + 0.02 * RNG.standard_normal(d)
+    x = RNG.standard_normal((t, d))
+    rows, cols, cu = O.positions([(4, 6)])
+    ang = O.rope_angles(rows, cols, 1e4, d)
+    exact = O.tower_block(x, lw, ang, cu, cfg)
+    fp8 = O.tower_block_fp8(x, O.quantize_layer(lw), (8 / 448, 4 / 448, 8 / 448, 8 / 448), ang, cu, cfg)
+    err = np.abs(fp8 - exact).max() / np.abs(exact).max()
+    assert 1e-4 < err < 5e-2, err
+
+
+def test_planted_fp8_missing_weight_scale_is_caught(monkeypatch):
+    def bad(a, q_w, s_w, s_a):
+        inv = np.float32(1.0 / np.float64(np.float32(s_a)))
+        q_a = O.e4m3_round(np.asarray(a, dtype=np.float32) * inv)
+        return (q_a @ np.asarray(q_w, dtype=np.float64).T) * np.float64(s_a)  # per-row weight scale dropped
+    monkeypatch.setattr(O, "fp8_linear", bad)
+    with pytest.raises(AssertionError):
+        test_fp8_linear_exact_on_representable_inputs()
+
+
+def test_planted_e4m3_truncation_is_caught(monkeypatch):
+    def bad(x):
+        x = np.asarray(x, dtype=np.float64)
+        a = np.abs(x)
+        _, e = np.frexp(a)
+        q = np.ldexp(1.0, (np.clip(e - 1, -6, 8) - 3).astype(np.int64))
+        return np.copysign(np.minimum(np.floor(a / q) * q, 448.0), x)  # rounds toward zero
+    monkeypatch.setattr(O, "e4m3_round", bad)
+    with pytest.raises(AssertionError):
+        test_e4m3_matches_torch_float8_and_saturates()
