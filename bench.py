@@ -45,6 +45,10 @@ WORKLOADS = {
     "pixtral_4096": dict(preset="pixtral12b", sizes=[(1024, 1024)] * 16, n_seq=16, seq_len=4352,
                          desc="Pixtral-12B-style: one 4096x4096 image as 16 tiles of 1024x1024 = 65,536 patches, "
                               "no merge, projector 1024->5120->5120"),
+    "mistral3_1540_fp8": dict(preset="mistral3", sizes=[(1540, 1540)], n_seq=1, seq_len=4096, fp8=True,
+                              desc="one 1540x1540 image (12,100 patches -> 3,025 merged tokens), 24-layer tower with "
+                                   "E4M3 QKV/O/gate-up/down GEMMs (per-row weight scales, static activation scales; "
+                                   "bf16 attention, norms, patch embed) + 2x2 merge + bf16 projector + scatter"),
     "photo_4032x3024": dict(preset="mistral3", photo=(3024, 4032), sizes=[(1176, 1540)], n_seq=1, seq_len=4096,
                             desc="one decoded 4032x3024 u8 RGB photo: GPU resize to 1176x1540 (longest edge 1540, "
                                  "28-px grid; 84x110 = 9,240 patches -> 2,310 merged tokens), 24-layer tower + "
@@ -414,7 +418,8 @@ def run_ours(args, wl):
 
     tw = {k: v.to(dev) for k, v in synth.tower_weights(args.seed, cfg.layers, cfg.width, cfg.mlp, cfg.patch).items()}
     pw = {k: v.to(dev) for k, v in synth.projector_weights(args.seed, cfg.width, cfg.merge, cfg.proj_out).items()}
-    pipe = vlm.ImagePipeline(cfg, tw, pw, sizes, device=dev)
+    pipe = vlm.ImagePipeline(cfg, tw, pw, sizes, device=dev,
+                             fp8_act_scales=synth.fp8_act_scales(cfg.layers) if wl.get("fp8") else None)
     del tw, pw
     photo = wl.get("photo")
     if photo:
@@ -532,7 +537,7 @@ def run_ours(args, wl):
     line = {
         "metric": METRIC, "value": value, "unit": "patches/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "vs_baseline": None, "dtype": "e4m3+bf16" if wl.get("fp8") else "bf16", "data": "synthetic",
         "config": {"workload": wl["desc"], "patches": T, "merged_tokens": Tm, "layers": cfg.layers,
                    "images": len(sizes), "text_tokens": int(ids.numel()), "parallelism": f"replicas{world}",
                    "l2": "inputs larger than L2 (weights 0.88 GB + activations per step)"},

@@ -161,6 +161,36 @@ VLM_API int vlm_encode(const vlm_config* cfg, const float* pixels, const int32_t
                int32_t* d_status, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * FP8 tower: the four GEMMs of every block (QKV, O, gate/up, down) on E4M3
+ * operands with fp32 accumulation (tcgen05.mma kind::f8f6f4), for the
+ * FP8-native deployments the pages describe ([K] intro; [I]). The patch
+ * embed, norms, RoPE, attention (bf16 q, k, v) and the residual stream are as
+ * in vlm_encode.
+ *
+ * Quantisation (reading; the pages give no recipe):
+ *   - weights per output row: s_w[n] = fp32(amax_n / 448) (1 for a zero row),
+ *     q = E4M3(fp32(w / s_w[n])), round to nearest even, saturating;
+ *   - activations with one static scale per GEMM input: q = E4M3(fp32(a) *
+ *     fp32(1 / s_a)); act_scales is host fp32 [layers][4] = the scales of the
+ *     attention-norm output, the attention output, the MLP-norm output and the
+ *     gated hidden state, each > 0;
+ *   - acc[m, n] * fp32(s_a * s_w[n]) dequantises a GEMM result.
+ *
+ * vlm_pack_tower_fp8: quantises the bf16 weights of vlm_tower_weights (same
+ *   meaning as for vlm_pack_tower) into d_packed (device, at least
+ *   vlm_tower_fp8_packed_bytes) with the given act_scales.
+ * vlm_encode_fp8: vlm_encode with the packed FP8 tower; act_scales must be the
+ *   array the tower was packed with. Workspace: vlm_encode_workspace_size.
+ * Requires width % 256 == 0 and mlp % 256 == 0 (else VLM_ERR_UNSUPPORTED).
+ * ------------------------------------------------------------------------- */
+VLM_API size_t vlm_tower_fp8_packed_bytes(const vlm_config* cfg);
+VLM_API int vlm_pack_tower_fp8(const vlm_config* cfg, const vlm_tower_weights* w, const float* act_scales,
+                               void* d_packed, size_t packed_bytes, void* stream);
+VLM_API int vlm_encode_fp8(const vlm_config* cfg, const float* pixels, const int32_t* image_hw, int n_images,
+                           const void* d_packed_tower_fp8, const float* act_scales, void* d_out, void* d_workspace,
+                           size_t ws_bytes, int32_t* d_status, void* stream);
+
+/* ---------------------------------------------------------------------------
  * vlm_merge_project -- the patch-merging projector ([K] Mistral3Model: 2x2
  * patch-merging projector, spatial_merge_size, projector_bias False):
  * RMSNorm per patch, m x m unfold + concat, merge linear (m*m*D -> D), then

@@ -56,6 +56,18 @@ VLM_API int vlm_gemm(int epilogue, const void* d_a, const void* d_b, int64_t M, 
              void* d_c, void* d_c_bf16, const int32_t* d_pos, const void* d_rope_table,
              int64_t rope_cols, int32_t* d_status, void* stream);
 
+/* The same product with E4M3 operands (tcgen05.mma kind::f8f6f4, fp32
+ * accumulation), then the accumulator column n is multiplied by
+ * d_colscale[n] (device fp32 [N], 16-byte aligned) before `epilogue`.
+ * A: device E4M3 [M, K]; B: device E4M3 [N, K]. Requires K % 128 == 0,
+ * N % 256 == 0. Epilogues BF16, RESID, ROPE (as for vlm_gemm) and SWIGLU,
+ * whose output is E4M3 [M, N/2] holding the gated values times out_scale
+ * (round to nearest even, saturating to +-448); others return
+ * VLM_ERR_UNSUPPORTED. */
+VLM_API int vlm_gemm_fp8(int epilogue, const void* d_a, const void* d_b, const float* d_colscale, float out_scale,
+                         int64_t M, int64_t N, int64_t K, void* d_c, void* d_c_bf16, const int32_t* d_pos,
+                         const void* d_rope_table, int64_t rope_cols, int32_t* d_status, void* stream);
+
 /* 2D RoPE angle table ([K] vision_rope_theta): entry [p][i] (float2 cos, sin)
  * of the angle p * w, w = theta^(-2k/head_dim) with k = 2i for i < head_dim/4
  * (row frequencies) and k = 2(i - head_dim/4) + 1 otherwise (column
@@ -82,6 +94,11 @@ VLM_API int vlm_attention(const void* d_qkv, int64_t T, int heads, int head_dim,
  * d_out = bf16(rmsnorm(x) * g1). d_x: fp32 [rows, width]. */
 VLM_API int vlm_rmsnorm(float* d_x, const float* d_g0, const float* d_g1, void* d_out, int64_t rows,
                 int width, float eps, void* stream);
+
+/* vlm_rmsnorm with an E4M3 output: d_out holds norm(.) * g1 * f8_scale rounded
+ * to E4M3 (nearest even, saturating to +-448); f8_scale > 0. */
+VLM_API int vlm_rmsnorm_fp8(float* d_x, const float* d_g0, const float* d_g1, void* d_out, int64_t rows, int width,
+                            float eps, float f8_scale, void* stream);
 
 /* Failure-detection self-test (no counterpart on the pages): launches one
  * thread that waits on a shared-memory mbarrier nothing arrives on, using the

@@ -212,6 +212,48 @@ TowerLayout tower_layout(const vlm_config* c) {
   return L;
 }
 
+// Packed FP8 tower layout (byte offsets): w_pe and g_pre as in the bf16 layout;
+// per layer the four GEMM weights as E4M3 (same row orders), their fp32 column
+// scales (s_a * s_w[n]) and the two gains.
+struct TowerF8Layout {
+  size_t w_pe, g_pre, layer0, layer_stride;
+  size_t wqkv, wo, wgu, wdown, cs_qkv, cs_o, cs_gu, cs_down, g_attn, g_ffn;
+  size_t total;
+};
+
+TowerF8Layout tower_f8_layout(const vlm_config* c) {
+  TowerF8Layout L;
+  const size_t D = c->width, F = c->mlp;
+  size_t off = 0;
+  L.w_pe = off; off = align_up(off + D * kpad(c->patch) * 2, 256);
+  L.g_pre = off; off = align_up(off + D * 4, 256);
+  L.layer0 = off;
+  size_t lo = 0;
+  L.wqkv = lo; lo = align_up(lo + 3 * D * D, 256);
+  L.wo = lo; lo = align_up(lo + D * D, 256);
+  L.wgu = lo; lo = align_up(lo + 2 * F * D, 256);
+  L.wdown = lo; lo = align_up(lo + D * F, 256);
+  L.cs_qkv = lo; lo = align_up(lo + 3 * D * 4, 256);
+  L.cs_o = lo; lo = align_up(lo + D * 4, 256);
+  L.cs_gu = lo; lo = align_up(lo + 2 * F * 4, 256);
+  L.cs_down = lo; lo = align_up(lo + D * 4, 256);
+  L.g_attn = lo; lo = align_up(lo + D * 4, 256);
+  L.g_ffn = lo; lo = align_up(lo + D * 4, 256);
+  L.layer_stride = lo;
+  L.total = off + lo * static_cast<size_t>(c->layers);
+  return L;
+}
+
+// fp32(1 / s) of a static activation scale, computed in double.
+inline float inv_scale(float s) { return static_cast<float>(1.0 / static_cast<double>(s)); }
+
+int check_act_scales(const vlm_config* c, const float* act) {
+  if (act == nullptr) return VLM_ERR_INVALID_ARG;
+  for (int i = 0; i < 4 * c->layers; ++i)
+    if (!(act[i] > 0.f) || !(act[i] < 3.0e38f)) return VLM_ERR_INVALID_ARG;
+  return VLM_OK;
+}
+
 struct ProjLayout { size_t g_proj, w_merge, w1, w2, total; };
 
 ProjLayout proj_layout(const vlm_config* c) {
@@ -470,6 +512,99 @@ int vlm_encode(const vlm_config* cfg, const float* pixels, const int32_t* image_
   return VLM_OK;
 }
 
+size_t vlm_tower_fp8_packed_bytes(const vlm_config* cfg) {
+  return check_config(cfg) == VLM_OK ? tower_f8_layout(cfg).total : 0;
+}
+
+int vlm_pack_tower_fp8(const vlm_config* cfg, const vlm_tower_weights* w, const float* act_scales, void* d_packed,
+                       size_t packed_bytes, void* stream) {
+  VLM_TRY(check_config(cfg));
+  if (w == nullptr || d_packed == nullptr || !w->w_pe || !w->g_pre || !w->wq || !w->wk || !w->wv || !w->wo ||
+      !w->w_gate || !w->w_up || !w->w_down || !w->g_attn || !w->g_ffn)
+    return VLM_ERR_INVALID_ARG;
+  VLM_TRY(check_act_scales(cfg, act_scales));
+  if (cfg->mlp % 256 || cfg->width % 256) return VLM_ERR_UNSUPPORTED;
+  const TowerF8Layout L = tower_f8_layout(cfg);
+  if (packed_bytes < L.total) return VLM_ERR_WORKSPACE;
+  cudaStream_t s = as_stream(stream);
+  uint8_t* dst = static_cast<uint8_t*>(d_packed);
+  const size_t D = cfg->width, F = cfg->mlp;
+  const int p = cfg->patch;
+  VLM_TRY(launch_pack_cols(w->w_pe, dst + L.w_pe, D, 3 * p * p, kpad(p), 0, 1, s));
+  if (cudaMemcpyAsync(dst + L.g_pre, w->g_pre, D * 4, cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+    return VLM_ERR_CUDA;
+  for (int l = 0; l < cfg->layers; ++l) {
+    uint8_t* ly = dst + L.layer0 + L.layer_stride * l;
+    const float* act = act_scales + 4 * l;
+    auto at = [&](const void* base, size_t elems) { return static_cast<const uint8_t*>(base) + l * elems * 2; };
+    float* cs_qkv = reinterpret_cast<float*>(ly + L.cs_qkv);
+    VLM_TRY(launch_quant_rows(at(w->wq, D * D), nullptr, 0, D, D, ly + L.wqkv, cs_qkv, act[0], s));
+    VLM_TRY(launch_quant_rows(at(w->wk, D * D), nullptr, 0, D, D, ly + L.wqkv + D * D, cs_qkv + D, act[0], s));
+    VLM_TRY(launch_quant_rows(at(w->wv, D * D), nullptr, 0, D, D, ly + L.wqkv + 2 * D * D, cs_qkv + 2 * D, act[0], s));
+    VLM_TRY(launch_quant_rows(at(w->wo, D * D), nullptr, 0, D, D, ly + L.wo, reinterpret_cast<float*>(ly + L.cs_o),
+                              act[1], s));
+    VLM_TRY(launch_quant_rows(at(w->w_gate, F * D), at(w->w_up, F * D), 1, 2 * F, D, ly + L.wgu,
+                              reinterpret_cast<float*>(ly + L.cs_gu), act[2], s));
+    VLM_TRY(launch_quant_rows(at(w->w_down, D * F), nullptr, 0, D, F, ly + L.wdown,
+                              reinterpret_cast<float*>(ly + L.cs_down), act[3], s));
+    bool ok = cudaMemcpyAsync(ly + L.g_attn, w->g_attn + l * D, D * 4, cudaMemcpyDeviceToDevice, s) == cudaSuccess;
+    ok = ok && cudaMemcpyAsync(ly + L.g_ffn, w->g_ffn + l * D, D * 4, cudaMemcpyDeviceToDevice, s) == cudaSuccess;
+    if (!ok) return VLM_ERR_CUDA;
+  }
+  return VLM_OK;
+}
+
+int vlm_encode_fp8(const vlm_config* cfg, const float* pixels, const int32_t* image_hw, int n_images,
+                   const void* d_packed_tower_fp8, const float* act_scales, void* d_out, void* d_workspace,
+                   size_t ws_bytes, int32_t* d_status, void* stream) {
+  VLM_TRY(check_config(cfg));
+  if (pixels == nullptr || d_packed_tower_fp8 == nullptr || d_out == nullptr || d_workspace == nullptr)
+    return VLM_ERR_INVALID_ARG;
+  VLM_TRY(check_act_scales(cfg, act_scales));
+  if (cfg->mlp % 256 || cfg->width % 256) return VLM_ERR_UNSUPPORTED;
+  if (reinterpret_cast<uintptr_t>(d_workspace) & 255) return VLM_ERR_INVALID_ARG;
+  Batch b;
+  VLM_TRY(make_batch(cfg, image_hw, n_images, &b));
+  const EncodeWs e = carve_encode(d_workspace, cfg, b);  // the E4M3 operands fit the bf16 buffers
+  if (ws_bytes < e.used) return VLM_ERR_WORKSPACE;
+  cudaStream_t s = as_stream(stream);
+  const TowerF8Layout L = tower_f8_layout(cfg);
+  const uint8_t* pk = static_cast<const uint8_t*>(d_packed_tower_fp8);
+  const int64_t T = b.T, D = cfg->width, F = cfg->mlp, kp = kpad(cfg->patch);
+
+  VLM_TRY(upload_batch(b, e.bd, s));
+  VLM_TRY(launch_rope_table(cfg->rope_theta, cfg->head_dim, b.max_pos, e.bd.rope, s));
+  VLM_TRY(launch_im2col(pixels, e.bd.info, e.bd.cu, b.n, T, cfg->patch, static_cast<int>(kp), cfg->normalize,
+                        e.cols, s));
+  VLM_TRY(launch_gemm(VLM_EPI_F32, e.cols, pk + L.w_pe, T, D, kp, e.x, nullptr, nullptr, nullptr, 0, d_status, s));
+  for (int l = 0; l < cfg->layers; ++l) {
+    const uint8_t* ly = pk + L.layer0 + L.layer_stride * l;
+    const float* act = act_scales + 4 * l;
+    auto f32 = [&](size_t off) { return reinterpret_cast<const float*>(ly + off); };
+    const float* g0 = l == 0 ? reinterpret_cast<const float*>(pk + L.g_pre) : nullptr;
+    VLM_TRY(launch_rmsnorm(e.x, g0, f32(L.g_attn), e.xn, T, static_cast<int>(D), cfg->eps, s, inv_scale(act[0])));
+    VLM_TRY(launch_gemm_f8(VLM_EPI_ROPE, e.xn, ly + L.wqkv, f32(L.cs_qkv), 1.f, T, 3 * D, D, e.qkv, nullptr,
+                           e.bd.pos, e.bd.rope, 2 * D, d_status, s));
+    VLM_TRY(launch_attention(e.qkv, T, cfg->heads, e.bd.cu, e.bd.qt, b.n, b.total_qtiles, e.attn, d_status, s,
+                             inv_scale(act[1])));
+    VLM_TRY(launch_gemm_f8(VLM_EPI_RESID, e.attn, ly + L.wo, f32(L.cs_o), 1.f, T, D, D, e.x, nullptr, nullptr,
+                           nullptr, 0, d_status, s));
+    VLM_TRY(launch_rmsnorm(e.x, nullptr, f32(L.g_ffn), e.xn, T, static_cast<int>(D), cfg->eps, s,
+                           inv_scale(act[2])));
+    VLM_TRY(launch_gemm_f8(VLM_EPI_SWIGLU, e.xn, ly + L.wgu, f32(L.cs_gu), inv_scale(act[3]), T, 2 * F, D, e.hbuf,
+                           nullptr, nullptr, nullptr, 0, d_status, s));
+    const bool last = l == cfg->layers - 1;
+    VLM_TRY(launch_gemm_f8(VLM_EPI_RESID, e.hbuf, ly + L.wdown, f32(L.cs_down), 1.f, T, D, F, e.x,
+                           last ? d_out : nullptr, nullptr, nullptr, 0, d_status, s));
+  }
+  if (cfg->layers == 0) {
+    VLM_TRY(launch_rmsnorm(e.x, reinterpret_cast<const float*>(pk + L.g_pre),
+                           reinterpret_cast<const float*>(pk + L.g_pre), e.xn, T, static_cast<int>(D), cfg->eps, s));
+    VLM_TRY(launch_f32_to_bf16(e.x, static_cast<__nv_bfloat16*>(d_out), T * D, s));
+  }
+  return VLM_OK;
+}
+
 size_t vlm_merge_project_workspace_size(const vlm_config* cfg, const int32_t* image_hw, int n_images) {
   if (check_config(cfg) != VLM_OK) return 0;
   Batch b;
@@ -684,6 +819,21 @@ int vlm_gemm(int epilogue, const void* d_a, const void* d_b, int64_t M, int64_t 
                      rope_cols, d_status, as_stream(stream));
 }
 
+int vlm_gemm_fp8(int epilogue, const void* d_a, const void* d_b, const float* d_colscale, float out_scale,
+                 int64_t M, int64_t N, int64_t K, void* d_c, void* d_c_bf16, const int32_t* d_pos,
+                 const void* d_rope_table, int64_t rope_cols, int32_t* d_status, void* stream) {
+  return launch_gemm_f8(epilogue, d_a, d_b, d_colscale, out_scale, M, N, K, d_c, d_c_bf16, d_pos,
+                        static_cast<const float2*>(d_rope_table), rope_cols, d_status, as_stream(stream));
+}
+
+int vlm_rmsnorm_fp8(float* d_x, const float* d_g0, const float* d_g1, void* d_out, int64_t rows, int width,
+                    float eps, float f8_scale, void* stream) {
+  if (d_x == nullptr || d_g1 == nullptr || d_out == nullptr || rows < 0 || !(f8_scale > 0.f))
+    return VLM_ERR_INVALID_ARG;
+  if (rows == 0) return VLM_OK;
+  return launch_rmsnorm(d_x, d_g0, d_g1, d_out, rows, width, eps, as_stream(stream), f8_scale);
+}
+
 int vlm_rope_table(float theta, int head_dim, int max_pos, void* d_table, void* stream) {
   if (d_table == nullptr || head_dim != 64 || max_pos <= 0 || !(theta > 0.f)) return VLM_ERR_INVALID_ARG;
   return launch_rope_table(theta, head_dim, max_pos, static_cast<float2*>(d_table), as_stream(stream));
@@ -741,7 +891,7 @@ int vlm_rmsnorm(float* d_x, const float* d_g0, const float* d_g1, void* d_out, i
                 void* stream) {
   if (d_x == nullptr || d_g1 == nullptr || d_out == nullptr || rows < 0) return VLM_ERR_INVALID_ARG;
   if (rows == 0) return VLM_OK;
-  return launch_rmsnorm(d_x, d_g0, d_g1, static_cast<__nv_bfloat16*>(d_out), rows, width, eps, as_stream(stream));
+  return launch_rmsnorm(d_x, d_g0, d_g1, d_out, rows, width, eps, as_stream(stream));
 }
 
 }  // extern "C"

@@ -156,10 +156,12 @@ struct AttnArgs {
   const int32_t* qt;
   int n_blocks;
   int heads;
-  __nv_bfloat16* out;
+  void* out;        // bf16, or E4M3 when kF8Out
   int32_t* status;
+  float f8_scale;   // E4M3 output: O / l times this before rounding
 };
 
+template <bool kF8Out>
 __global__ void __launch_bounds__(192, 2)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, const AttnArgs args) {
   extern __shared__ uint8_t smem_raw[];
@@ -346,7 +348,28 @@ __global__ void __launch_bounds__(192, 2)
       tc_fence_after();
       const float inv = 1.0f / l;
       const int row = q0 + r;
-      __nv_bfloat16* dst = args.out + static_cast<int64_t>(row) * D + h * DH;
+      if constexpr (kF8Out) {
+        const float f = inv * args.f8_scale;
+        uint8_t* dst = static_cast<uint8_t*>(args.out) + static_cast<int64_t>(row) * D + h * DH;
+#pragma unroll
+        for (int c = 0; c < DH; c += 32) {
+          uint32_t o[32];
+          tmem_ld32(trow + kColO + c, o);
+          if (row < kend) {
+            uint4* d4 = reinterpret_cast<uint4*>(dst + c);
+#pragma unroll
+            for (int jj = 0; jj < 2; ++jj) {
+              uint32_t w[4];
+#pragma unroll
+              for (int k = 0; k < 4; ++k)
+                w[k] = pack_e4m3x4(__uint_as_float(o[16 * jj + 4 * k]) * f, __uint_as_float(o[16 * jj + 4 * k + 1]) * f,
+                                   __uint_as_float(o[16 * jj + 4 * k + 2]) * f, __uint_as_float(o[16 * jj + 4 * k + 3]) * f);
+              d4[jj] = make_uint4(w[0], w[1], w[2], w[3]);
+            }
+          }
+        }
+      } else {
+      __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(args.out) + static_cast<int64_t>(row) * D + h * DH;
 #pragma unroll
       for (int c = 0; c < DH; c += 32) {
         uint32_t o[32];
@@ -360,6 +383,7 @@ __global__ void __launch_bounds__(192, 2)
                                 pack_bf16x2(__uint_as_float(o[8 * jj + 4]) * inv, __uint_as_float(o[8 * jj + 5]) * inv),
                                 pack_bf16x2(__uint_as_float(o[8 * jj + 6]) * inv, __uint_as_float(o[8 * jj + 7]) * inv));
         }
+      }
       }
     }
   }
@@ -375,7 +399,7 @@ __global__ void __launch_bounds__(192, 2)
 }  // namespace
 
 int launch_attention(const __nv_bfloat16* qkv, int64_t T, int heads, const int32_t* cu, const int32_t* qt,
-                     int n_blocks, int total_qtiles, __nv_bfloat16* out, int32_t* status, cudaStream_t s) {
+                     int n_blocks, int total_qtiles, void* out, int32_t* status, cudaStream_t s, float f8_scale) {
   if (total_qtiles <= 0) return VLM_OK;
   if (heads <= 0 || heads > 65535) return VLM_ERR_UNSUPPORTED;
   CUtensorMap tm;
@@ -385,15 +409,18 @@ int launch_attention(const __nv_bfloat16* qkv, int64_t T, int heads, const int32
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 64 && !attr_done[dev]) {
-    if (cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) !=
-        cudaSuccess)
+    if (cudaFuncSetAttribute(attn_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) !=
+            cudaSuccess ||
+        cudaFuncSetAttribute(attn_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) !=
+            cudaSuccess)
       return VLM_ERR_CUDA;
     attr_done[dev] = true;
   }
-  AttnArgs args{cu, qt, n_blocks, heads, out, status};
+  AttnArgs args{cu, qt, n_blocks, heads, out, status, f8_scale};
   dim3 grid(total_qtiles, heads);
   launch_begin(KC_ATTN, s);
-  const cudaError_t e = launch_pdl(attn_tc_kernel, grid, dim3(192), kSmemBytes, s, tm, args);
+  const cudaError_t e = f8_scale > 0.f ? launch_pdl(attn_tc_kernel<true>, grid, dim3(192), kSmemBytes, s, tm, args)
+                                       : launch_pdl(attn_tc_kernel<false>, grid, dim3(192), kSmemBytes, s, tm, args);
   launch_end(KC_ATTN, s);
   return e == cudaSuccess ? VLM_OK : VLM_ERR_CUDA;
 }

@@ -252,6 +252,17 @@ __device__ __forceinline__ void umma_bf16_ss_pair(uint32_t d_tmem, uint64_t a_de
       "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
+// The same with E4M3 operands (kind::f8f6f4: K = 32 per instruction, 32 bytes
+// of each operand row, like K = 16 of bf16).
+__device__ __forceinline__ void umma_f8_ss_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                                uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
 // Arrive once on the mbarrier at this offset in every CTA of cta_mask when the
 // pair's prior tcgen05 ops complete.
 __device__ __forceinline__ void umma_commit_pair_mc(uint32_t bar, uint16_t cta_mask) {
@@ -320,6 +331,25 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int m, int n, bool b_mn_major 
          | ((b_mn_major ? 1u : 0u) << 16)           // B major
          | (static_cast<uint32_t>(n >> 3) << 17)    // N / 8
          | (static_cast<uint32_t>(m >> 4) << 24);   // M / 16
+}
+
+// Instruction descriptor of kind::f8f6f4 with E4M3 A and B (format code 0),
+// fp32 D, both operands K-major.
+__host__ __device__ constexpr uint32_t idesc_e4m3(int m, int n) {
+  return (1u << 4)                                  // D format: f32
+         | (0u << 7)                                // A format: E4M3
+         | (0u << 10)                               // B format: E4M3
+         | (static_cast<uint32_t>(n >> 3) << 17)    // N / 8
+         | (static_cast<uint32_t>(m >> 4) << 24);   // M / 16
+}
+
+// Four fp32 values -> four E4M3 bytes (round to nearest even, saturating to
+// +-448), v0 in the lowest byte.
+__device__ __forceinline__ uint32_t pack_e4m3x4(float v0, float v1, float v2, float v3) {
+  uint16_t lo, hi;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(lo) : "f"(v1), "f"(v0));
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(hi) : "f"(v3), "f"(v2));
+  return static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
 }
 
 // Shared-memory matrix descriptor for a 128-byte-swizzled tile whose rows are

@@ -40,6 +40,8 @@ struct GemmArgs {
   const float2* rope;
   int rope_cols;
   int32_t* status;
+  const float* colscale;  // E4M3 operands: per-output-column dequantisation factor (s_a * s_w[n])
+  float out_scale;        // E4M3 output (SwiGLU): values are multiplied by this before rounding
 };
 
 template <int BN>
@@ -110,19 +112,65 @@ __device__ __forceinline__ float act(float v) {
   return v;
 }
 
+// 32 consecutive column scales (the same for every lane: broadcast loads).
+__device__ __forceinline__ void load_cs32(const float* p, float (&cs)[32]) {
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const float4 v = __ldg(reinterpret_cast<const float4*>(p) + j);
+    cs[4 * j] = v.x; cs[4 * j + 1] = v.y; cs[4 * j + 2] = v.z; cs[4 * j + 3] = v.w;
+  }
+}
+
 // Epilogue of one 128 x BN tile: this warp's 32 rows (row0 = first of them;
 // this lane's row is row0 + lane), accumulator columns at TMEM address tbase.
-template <int BN, int EPI>
+// kF8: the accumulator holds sums of E4M3 products; every column is first
+// multiplied by its colscale (SwiGLU also writes E4M3).
+template <int BN, int EPI, bool kF8 = false>
 __device__ __forceinline__ void epilogue_tile(const GemmArgs& args, Stager& st, uint32_t tbase, int row0, int n0) {
   const int lane = st.lane;
   const int row = row0 + lane;
   const bool live = row < args.M;
-  if constexpr (EPI == VLM_EPI_BF16 || EPI == VLM_EPI_GELU) {
+  // dequantise 32 accumulator words in place (E4M3 operands only)
+  auto deq = [&](uint32_t (&v)[32], int col) {
+    if constexpr (kF8) {
+      float cs[32];
+      load_cs32(args.colscale + col, cs);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * cs[i]);
+    }
+  };
+  if constexpr (kF8 && EPI == VLM_EPI_SWIGLU) {
+    // 256 accumulator columns -> 128 E4M3 outputs = one 128-byte row chunk;
+    // columns 32g..32g+15 are gate and 32g+16..32g+31 up of outputs 16g..16g+15
+#pragma unroll 1
+    for (int c = 0; c < BN; c += 256) {
+      uint32_t w[32];
+#pragma unroll
+      for (int g = 0; g < 8; ++g) {
+        uint32_t r[32];
+        tmem_ld32(tbase + c + 32 * g, r);
+        deq(r, n0 + c + 32 * g);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          float h[4];
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            h[k] = silu_f(__uint_as_float(r[4 * e + k])) * __uint_as_float(r[16 + 4 * e + k]) * args.out_scale;
+          w[4 * g + e] = pack_e4m3x4(h[0], h[1], h[2], h[3]);
+        }
+      }
+      uint8_t* buf = st.acquire();
+      st.write_row(buf, w);
+      st.commit(buf, (n0 + c) / 2, row0);
+    }
+  } else if constexpr (EPI == VLM_EPI_BF16 || EPI == VLM_EPI_GELU) {
 #pragma unroll 1
     for (int c = 0; c < BN; c += 64) {
       uint32_t a[32], b[32], w[32];
       tmem_ld32(tbase + c, a);
       tmem_ld32(tbase + c + 32, b);
+      deq(a, n0 + c);
+      deq(b, n0 + c + 32);
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
         w[i] = pack_bf16x2(act<EPI>(__uint_as_float(a[2 * i])), act<EPI>(__uint_as_float(a[2 * i + 1])));
@@ -137,6 +185,7 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& args, Stager& st, 
     for (int c = 0; c < BN; c += 32) {
       uint32_t a[32];
       tmem_ld32(tbase + c, a);
+      deq(a, n0 + c);
       uint8_t* buf = st.acquire();
       st.write_row(buf, a);
       st.commit(buf, n0 + c, row0);
@@ -148,6 +197,7 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& args, Stager& st, 
       for (int c = 0; c < BN; c += 32) {
         uint32_t a[32];
         tmem_ld32(tbase + c, a);
+        deq(a, n0 + c);
         uint8_t* buf = st.acquire();
         st.write_row(buf, a);
         st.template commit<true>(buf, n0 + c, row0);
@@ -181,6 +231,7 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& args, Stager& st, 
       if (c + 32 < BN) load_res(c + 32);
       uint32_t a[32];
       tmem_ld32(tbase + c, a);
+      deq(a, n0 + c);
       __syncwarp();
       float4* rp = reinterpret_cast<float4*>(buf + lane * 128);
       float v[32];
@@ -232,6 +283,8 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& args, Stager& st, 
       uint32_t a[32], b[32], w[32];
       tmem_ld32(tbase + c, a);
       tmem_ld32(tbase + c + 32, b);
+      deq(a, n0 + c);
+      deq(b, n0 + c + 32);
       float x[32], y[32];
 #pragma unroll
       for (int i = 0; i < 32; ++i) { x[i] = __uint_as_float(a[i]); y[i] = __uint_as_float(b[i]); }
@@ -405,7 +458,7 @@ struct PairShape {
   static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + EPI_BYTES + BAR_BYTES + 1024;
 };
 
-template <int EPI>
+template <int EPI, bool kF8 = false>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
     gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                      const __grid_constant__ CUtensorMap tmC, const GemmArgs args) {
@@ -427,7 +480,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
   const uint32_t rank = cluster_ctarank();
   const int pair = blockIdx.x >> 1, n_pairs = gridDim.x >> 1;
   const int total_tiles = args.m_tiles * args.n_tiles;  // m_tiles counts 256-row pair tiles here
-  const int nk = args.K / GBK;
+  // a stage holds 128 bytes of every operand row: 64 bf16 or 128 E4M3 values of K
+  constexpr int kBK = kF8 ? 2 * GBK : GBK;
+  const int nk = args.K / kBK;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S::STAGES; ++s) {
@@ -472,15 +527,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
           if (!mbar_wait(smem_u32(empty + stage), phase ^ 1u, abort_v, args.status)) { ok = false; break; }
           const uint32_t fb = smem_u32(full + stage) & kPeerBitMask;
           if (rank == 0) mbar_arrive_expect_tx(smem_u32(full + stage), 2 * S::STAGE_BYTES);
-          tma_load_2d_pair(smem_u32(sA + stage * S::A_BYTES), &tmA, fb, kb * GBK, arow);
-          tma_load_2d_pair(smem_u32(sB + stage * S::B_BYTES), &tmB, fb, kb * GBK, brow);
+          tma_load_2d_pair(smem_u32(sA + stage * S::A_BYTES), &tmA, fb, kb * kBK, arow);
+          tma_load_2d_pair(smem_u32(sB + stage * S::B_BYTES), &tmB, fb, kb * kBK, brow);
           if (++stage == S::STAGES) { stage = 0; phase ^= 1u; }
         }
       }
     }
   } else if (warp == 1) {
     if (rank == 0 && lane == 0) {
-      constexpr uint32_t idesc = idesc_bf16(2 * GBM, S::BN);
+      constexpr uint32_t idesc = kF8 ? idesc_e4m3(2 * GBM, S::BN) : idesc_bf16(2 * GBM, S::BN);
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
@@ -496,8 +551,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
           const uint64_t adesc = smem_desc_sw128(smem_u32(sA + stage * S::A_BYTES));
           const uint64_t bdesc = smem_desc_sw128(smem_u32(sB + stage * S::B_BYTES));
 #pragma unroll
-          for (int k = 0; k < GBK / 16; ++k)
-            umma_bf16_ss_pair(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, (kb | k) != 0 ? 1u : 0u);
+          for (int k = 0; k < 4; ++k) {  // 32 bytes of K per instruction
+            if constexpr (kF8)
+              umma_f8_ss_pair(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, (kb | k) != 0 ? 1u : 0u);
+            else
+              umma_bf16_ss_pair(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, (kb | k) != 0 ? 1u : 0u);
+          }
           umma_commit_pair_mc(smem_u32(empty + stage), 0x3);
           if (++stage == S::STAGES) { stage = 0; phase ^= 1u; }
         }
@@ -518,7 +577,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
       if (!mbar_wait_warp(smem_u32(tfull + acc), acc_phase, abort_v, args.status)) break;
       tc_fence_after();
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * S::BN);
-      epilogue_tile<S::BN, EPI>(args, st, tbase, mt * 256 + static_cast<int>(rank) * GBM + q * 32, nt * S::BN);
+      epilogue_tile<S::BN, EPI, kF8>(args, st, tbase, mt * 256 + static_cast<int>(rank) * GBM + q * 32, nt * S::BN);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(leader_tempty + static_cast<uint32_t>(acc * 8));
@@ -537,10 +596,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
   }
 }
 
-template <int EPI>
+template <int EPI, bool kF8 = false>
 int run_gemm_pair(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tc, const GemmArgs& args,
                   cudaStream_t s) {
-  auto kern = gemm_pair_kernel<EPI>;
+  auto kern = gemm_pair_kernel<EPI, kF8>;
   static bool attr_done[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
@@ -568,6 +627,17 @@ int dispatch_pair(int epi, const CUtensorMap& ta, const CUtensorMap& tb, const C
     case VLM_EPI_ROPE: return run_gemm_pair<VLM_EPI_ROPE>(ta, tb, tc, args, s);
     case VLM_EPI_GELU: return run_gemm_pair<VLM_EPI_GELU>(ta, tb, tc, args, s);
     default: return VLM_ERR_INVALID_ARG;
+  }
+}
+
+int dispatch_pair_f8(int epi, const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tc,
+                     const GemmArgs& args, cudaStream_t s) {
+  switch (epi) {
+    case VLM_EPI_BF16: return run_gemm_pair<VLM_EPI_BF16, true>(ta, tb, tc, args, s);
+    case VLM_EPI_RESID: return run_gemm_pair<VLM_EPI_RESID, true>(ta, tb, tc, args, s);
+    case VLM_EPI_SWIGLU: return run_gemm_pair<VLM_EPI_SWIGLU, true>(ta, tb, tc, args, s);
+    case VLM_EPI_ROPE: return run_gemm_pair<VLM_EPI_ROPE, true>(ta, tb, tc, args, s);
+    default: return VLM_ERR_UNSUPPORTED;
   }
 }
 
@@ -642,6 +712,58 @@ bool make_tmap_2d_bf16(CUtensorMap* map, const void* ptr, uint64_t inner, uint64
   return make_tmap_2d(map, ptr, false, inner, outer, row_bytes, box_inner, box_outer);
 }
 
+bool make_tmap_2d_u8(CUtensorMap* map, const void* ptr, uint64_t inner, uint64_t outer, uint64_t row_bytes,
+                     uint32_t box_inner, uint32_t box_outer) {
+  auto enc = tensor_map_encoder();
+  if (enc == nullptr) return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {row_bytes};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int launch_gemm_f8(int epi, const void* a, const void* b, const float* colscale, float out_scale, int64_t M,
+                   int64_t N, int64_t K, void* c, void* c_bf16, const int32_t* pos, const float2* rope,
+                   int64_t rope_cols, int32_t* status, cudaStream_t s) {
+  if (a == nullptr || b == nullptr || c == nullptr || colscale == nullptr) return VLM_ERR_INVALID_ARG;
+  if (M <= 0 || N <= 0 || K <= 0 || M > (1LL << 31) - 1 || N > 65535 * 256LL || K > (1 << 20))
+    return VLM_ERR_BAD_SHAPE;
+  if (K % 128 != 0 || N % 256 != 0) return VLM_ERR_UNSUPPORTED;
+  if (epi != VLM_EPI_BF16 && epi != VLM_EPI_RESID && epi != VLM_EPI_SWIGLU && epi != VLM_EPI_ROPE)
+    return VLM_ERR_UNSUPPORTED;
+  if (epi == VLM_EPI_ROPE && (pos == nullptr || rope == nullptr || rope_cols % 64 != 0)) return VLM_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(a) | reinterpret_cast<uintptr_t>(b) | reinterpret_cast<uintptr_t>(c) |
+       reinterpret_cast<uintptr_t>(colscale)) & 15)
+    return VLM_ERR_INVALID_ARG;
+  CUtensorMap ta, tb, tc;
+  if (!make_tmap_2d_u8(&ta, a, K, M, K, 128, GBM)) return VLM_ERR_CUDA;
+  if (!make_tmap_2d_u8(&tb, b, K, N, K, 128, 128)) return VLM_ERR_CUDA;
+  // output: 32-row boxes of 128 bytes (64 bf16, 32 fp32 or, for SwiGLU, 128 E4M3 columns)
+  bool ok;
+  if (epi == VLM_EPI_SWIGLU) ok = make_tmap_2d_u8(&tc, c, N / 2, M, N / 2, 128, 32);
+  else if (epi == VLM_EPI_RESID) ok = make_tmap_2d(&tc, c, true, N, M, N * 4, 32, 32);
+  else ok = make_tmap_2d(&tc, c, false, N, M, N * 2, 64, 32);
+  if (!ok) return VLM_ERR_CUDA;
+  GemmArgs args;
+  args.M = static_cast<int>(M);
+  args.N = static_cast<int>(N);
+  args.K = static_cast<int>(K);
+  args.m_tiles = static_cast<int>((M + 255) / 256);
+  args.n_tiles = static_cast<int>(N / 256);
+  args.c = c;
+  args.c_bf16 = static_cast<__nv_bfloat16*>(c_bf16);
+  args.pos = pos;
+  args.rope = rope;
+  args.rope_cols = static_cast<int>(rope_cols);
+  args.status = status;
+  args.colscale = colscale;
+  args.out_scale = out_scale;
+  return dispatch_pair_f8(epi, ta, tb, tc, args, s);
+}
+
 int launch_gemm(int epi, const void* a, const void* b, int64_t M, int64_t N, int64_t K, void* c, void* c_bf16,
                 const int32_t* pos, const float2* rope, int64_t rope_cols, int32_t* status, cudaStream_t s) {
   if (a == nullptr || b == nullptr || c == nullptr) return VLM_ERR_INVALID_ARG;
@@ -677,6 +799,8 @@ int launch_gemm(int epi, const void* a, const void* b, int64_t M, int64_t N, int
   args.rope = rope;
   args.rope_cols = static_cast<int>(rope_cols);
   args.status = status;
+  args.colscale = nullptr;
+  args.out_scale = 1.0f;
   if (bn == 256) {
     // two-SM pairs: 256-row tiles of A (128 per CTA) and 128-row halves of the B tile
     CUtensorMap tb2;

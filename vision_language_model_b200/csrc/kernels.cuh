@@ -75,8 +75,9 @@ int launch_setup(const ImageChunk& chunk, ImgInfo* info, int32_t* cu, int32_t* q
 int launch_rope_table(float theta, int head_dim, int max_pos, float2* tab, cudaStream_t s);
 int launch_im2col(const float* pix, const ImgInfo* info, const int32_t* cu, int n_images, int64_t T,
                   int p, int kp, int normalize, __nv_bfloat16* out, cudaStream_t s);
-int launch_rmsnorm(float* x, const float* g0, const float* g1, __nv_bfloat16* out, int64_t rows,
-                   int width, float eps, cudaStream_t s);
+// f8_scale > 0: `out` is E4M3 holding the normalised values times f8_scale; else bf16.
+int launch_rmsnorm(float* x, const float* g0, const float* g1, void* out, int64_t rows, int width, float eps,
+                   cudaStream_t s, float f8_scale = 0.f);
 int launch_merge_norm(const __nv_bfloat16* x, const float* g, const ImgInfo* info, const int32_t* cu,
                       int n_images, int64_t T, int width, int m, float eps, __nv_bfloat16* z,
                       cudaStream_t s);
@@ -105,7 +106,23 @@ int launch_gemm(int epi, const void* a, const void* b, int64_t M, int64_t N, int
                 void* c_bf16, const int32_t* pos, const float2* rope, int64_t rope_cols, int32_t* status,
                 cudaStream_t s);
 
+// E4M3 x E4M3 -> fp32 GEMM on two-SM pairs (N % 256 == 0, K % 128 == 0): the
+// accumulator column n is multiplied by colscale[n]; epilogues BF16, RESID,
+// ROPE, and SWIGLU with E4M3 output (values times out_scale).
+int launch_gemm_f8(int epi, const void* a, const void* b, const float* colscale, float out_scale, int64_t M,
+                   int64_t N, int64_t K, void* c, void* c_bf16, const int32_t* pos, const float2* rope,
+                   int64_t rope_cols, int32_t* status, cudaStream_t s);
+
+// f8_scale > 0: `out` is E4M3 holding the attention output times f8_scale; else bf16.
 int launch_attention(const __nv_bfloat16* qkv, int64_t T, int heads, const int32_t* cu, const int32_t* qt,
-                     int n_blocks, int total_qtiles, __nv_bfloat16* out, int32_t* status, cudaStream_t s);
+                     int n_blocks, int total_qtiles, void* out, int32_t* status, cudaStream_t s,
+                     float f8_scale = 0.f);
+// Per-row E4M3 quantisation of bf16 weight rows for the FP8 tower GEMMs:
+// s[r] = amax_r / 448 (1 for a zero row), dst[r, :] = e4m3(src[r, :] / s[r]),
+// colscale[r] = act_scale * s[r]. mode 0: row r of src; mode 1: the gate/up
+// interleave of pack_gate_up (rows 32j..32j+15 from gate rows 16j.., 32j+16..
+// from up rows 16j..; src = gate, src2 = up).
+int launch_quant_rows(const void* src, const void* src2, int mode, int64_t rows, int64_t cols, void* dst,
+                      float* colscale, float act_scale, cudaStream_t s);
 
 }  // namespace vlm

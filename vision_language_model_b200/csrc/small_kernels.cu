@@ -117,11 +117,13 @@ __global__ void im2col_kernel(const float* __restrict__ pix, const ImgInfo* __re
 // RMSNorm, one warp per row of `width` fp32 values (width % 128 == 0, <= 2048).
 // With g0: y = norm(x) * g0 is written back to x, and out = bf16(norm(y) * g1).
 // Without g0: out = bf16(norm(x) * g1).
+// kF8: out is E4M3 instead, of norm(.) * g1 * f8_scale (round to nearest even,
+// saturating).
 // ---------------------------------------------------------------------------
-template <int NV>
+template <int NV, bool kF8 = false>
 __global__ void rmsnorm_kernel(float* __restrict__ x, const float* __restrict__ g0,
-                               const float* __restrict__ g1, __nv_bfloat16* __restrict__ out,
-                               int64_t rows, float eps) {
+                               const float* __restrict__ g1, void* __restrict__ out_v,
+                               int64_t rows, float eps, float f8_scale) {
   griddep_wait();
   griddep_launch_dependents();
   constexpr int width = NV * 128;
@@ -155,14 +157,24 @@ __global__ void rmsnorm_kernel(float* __restrict__ x, const float* __restrict__ 
       rs = rsqrtf(ss / width + eps);
     }
     const float4* gr = reinterpret_cast<const float4*>(g1);
-    uint2* orow = reinterpret_cast<uint2*>(out + row * width);
+    if constexpr (kF8) {
+      uint32_t* orow = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(out_v) + row * width);
 #pragma unroll
-    for (int j = 0; j < NV; ++j) {
-      const float4 g = __ldg(gr + lane + 32 * j);
-      uint2 o;
-      o.x = pack_bf16x2(v[j].x * rs * g.x, v[j].y * rs * g.y);
-      o.y = pack_bf16x2(v[j].z * rs * g.z, v[j].w * rs * g.w);
-      orow[lane + 32 * j] = o;
+      for (int j = 0; j < NV; ++j) {
+        const float4 g = __ldg(gr + lane + 32 * j);
+        orow[lane + 32 * j] = pack_e4m3x4(v[j].x * rs * g.x * f8_scale, v[j].y * rs * g.y * f8_scale,
+                                          v[j].z * rs * g.z * f8_scale, v[j].w * rs * g.w * f8_scale);
+      }
+    } else {
+      uint2* orow = reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(out_v) + row * width);
+#pragma unroll
+      for (int j = 0; j < NV; ++j) {
+        const float4 g = __ldg(gr + lane + 32 * j);
+        uint2 o;
+        o.x = pack_bf16x2(v[j].x * rs * g.x, v[j].y * rs * g.y);
+        o.y = pack_bf16x2(v[j].z * rs * g.z, v[j].w * rs * g.w);
+        orow[lane + 32 * j] = o;
+      }
     }
   }
 }
@@ -337,6 +349,35 @@ __global__ void pack_gate_up_kernel(const uint4* __restrict__ gate, const uint4*
   }
 }
 
+// Per-row E4M3 quantisation, one warp per destination row (see launch_quant_rows).
+__global__ void quant_rows_kernel(const __nv_bfloat16* __restrict__ src, const __nv_bfloat16* __restrict__ src2,
+                                  int mode, int64_t rows, int64_t cols, uint8_t* __restrict__ dst,
+                                  float* __restrict__ colscale, float act_scale) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
+  for (int64_t r = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; r < rows; r += warps) {
+    const __nv_bfloat16* sr;
+    if (mode == 1) {
+      const int64_t grp = r >> 5, within = r & 31;
+      sr = (within < 16 ? src : src2) + (grp * 16 + (within & 15)) * cols;
+    } else {
+      sr = src + r * cols;
+    }
+    float amax = 0.f;
+    for (int64_t k = lane; k < cols; k += 32) amax = fmaxf(amax, fabsf(__bfloat162float(sr[k])));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    float sc = __fdiv_rn(amax, 448.0f);
+    if (!(sc > 0.f)) sc = 1.0f;
+    uint8_t* dr = dst + r * cols;
+    for (int64_t k = 4 * lane; k < cols; k += 128)
+      *reinterpret_cast<uint32_t*>(dr + k) =
+          pack_e4m3x4(__fdiv_rn(__bfloat162float(sr[k]), sc), __fdiv_rn(__bfloat162float(sr[k + 1]), sc),
+                      __fdiv_rn(__bfloat162float(sr[k + 2]), sc), __fdiv_rn(__bfloat162float(sr[k + 3]), sc));
+    if (lane == 0) colscale[r] = __fmul_rn(act_scale, sc);
+  }
+}
+
 // dst [rows, dst_cols] from src [rows, src_cols], bf16:
 //   mode 0 (pad):     dst[r, k] = k < src_cols ? src[r, k] : 0
 //   mode 1 (permute): dst[r, slot*D + c] = src[r, c*mm + slot]  (D = src_cols / mm)
@@ -404,15 +445,19 @@ int launch_im2col(const float* pix, const ImgInfo* info, const int32_t* cu, int 
   return e == cudaSuccess ? VLM_OK : VLM_ERR_CUDA;
 }
 
-int launch_rmsnorm(float* x, const float* g0, const float* g1, __nv_bfloat16* out, int64_t rows,
-                   int width, float eps, cudaStream_t s) {
+int launch_rmsnorm(float* x, const float* g0, const float* g1, void* out, int64_t rows, int width, float eps,
+                   cudaStream_t s, float f8_scale) {
   if (width % 128 || width > 2048 || width <= 0) return VLM_ERR_UNSUPPORTED;
   const int grid = grid_for(rows * 32, 256);
   launch_begin(KC_NORM, s);
   cudaError_t e = cudaErrorInvalidValue;
+  const bool f8 = f8_scale > 0.f;
   switch (width / 128) {
-#define VLM_NORM_CASE(nv) \
-  case nv: e = launch_pdl(rmsnorm_kernel<nv>, dim3(grid), dim3(256), 0, s, x, g0, g1, out, rows, eps); break;
+#define VLM_NORM_CASE(nv)                                                                                       \
+  case nv:                                                                                                    \
+    e = f8 ? launch_pdl(rmsnorm_kernel<nv, true>, dim3(grid), dim3(256), 0, s, x, g0, g1, out, rows, eps, f8_scale) \
+           : launch_pdl(rmsnorm_kernel<nv, false>, dim3(grid), dim3(256), 0, s, x, g0, g1, out, rows, eps, 0.f); \
+    break;
     VLM_NORM_CASE(1) VLM_NORM_CASE(2) VLM_NORM_CASE(3) VLM_NORM_CASE(4) VLM_NORM_CASE(5)
     VLM_NORM_CASE(6) VLM_NORM_CASE(7) VLM_NORM_CASE(8) VLM_NORM_CASE(9) VLM_NORM_CASE(10)
     VLM_NORM_CASE(11) VLM_NORM_CASE(12) VLM_NORM_CASE(13) VLM_NORM_CASE(14) VLM_NORM_CASE(15)
@@ -478,6 +523,17 @@ int launch_marker_scan(const int32_t* chunk_count, int64_t n_chunks, int64_t exp
                        int32_t* ok_flag, int32_t* status, cudaStream_t s) {
   return launch_pdl(scatter_scan_kernel, dim3(1), dim3(1024), 0, s, chunk_count, n_chunks, expected, chunk_base,
                     ok_flag, status) == cudaSuccess ? VLM_OK : VLM_ERR_CUDA;
+}
+
+int launch_quant_rows(const void* src, const void* src2, int mode, int64_t rows, int64_t cols, void* dst,
+                      float* colscale, float act_scale, cudaStream_t s) {
+  if (cols % 128 != 0 || rows <= 0) return VLM_ERR_UNSUPPORTED;
+  launch_begin(KC_PACK, s);
+  quant_rows_kernel<<<grid_for(rows * 32, 256), 256, 0, s>>>(
+      static_cast<const __nv_bfloat16*>(src), static_cast<const __nv_bfloat16*>(src2), mode, rows, cols,
+      static_cast<uint8_t*>(dst), colscale, act_scale);
+  launch_end(KC_PACK, s);
+  return cudaGetLastError() == cudaSuccess ? VLM_OK : VLM_ERR_CUDA;
 }
 
 int launch_pack_gate_up(const void* gate, const void* up, void* dst, int64_t f, int64_t d, cudaStream_t s) {

@@ -118,6 +118,14 @@ def tower_weights(seed: int, layers: int, width: int, mlp: int, patch: int,
     return w
 
 
+def fp8_act_scales(layers: int) -> list:
+    """Static E4M3 activation scales per layer for the synthetic towers: the
+    GEMM inputs' ranges under N(0, 0.02) weights and ~1 gains are about
+    |normed x| <= 8, |attention output| <= 4 (the values of v) and |gated
+    hidden| <= 16; each scale maps that bound to 448."""
+    return [[8.0 / 448.0, 4.0 / 448.0, 8.0 / 448.0, 16.0 / 448.0] for _ in range(layers)]
+
+
 def projector_weights(seed: int, width: int, merge: int, proj_out: int) -> dict:
     d, e, m = width, proj_out, merge
     return {

@@ -83,6 +83,11 @@ def lib() -> ctypes.CDLL:
             "vlm_preprocess": (I32, [P, P, I32, P, I32, P, P]),
             "vlm_expand_placeholders_workspace_size": (SZ, [I64, I32]),
             "vlm_expand_placeholders": (I32, [P, I64, I64, P, I32, I64, P, I64, ctypes.POINTER(I64), P, SZ, P, P]),
+            "vlm_tower_fp8_packed_bytes": (SZ, [CP]),
+            "vlm_pack_tower_fp8": (I32, [CP, ctypes.POINTER(TowerWeights), P, P, SZ, P]),
+            "vlm_encode_fp8": (I32, [CP, P, P, I32, P, P, P, P, SZ, P, P]),
+            "vlm_gemm_fp8": (I32, [I32, P, P, P, F, I64, I64, I64, P, P, P, P, I64, P, P]),
+            "vlm_rmsnorm_fp8": (I32, [P, P, P, P, I64, I32, F, F, P]),
             "vlm_launch_count": (I64, []),
             "vlm_profile_enable": (I32, [I32]),
             "vlm_profile_query": (I32, [I32, ctypes.POINTER(I64), ctypes.POINTER(ctypes.c_double)]),
@@ -285,6 +290,73 @@ def scatter(input_ids: torch.Tensor, image_embeds: torch.Tensor, text_embeds: to
 # ---------------------------------------------------------------------------
 
 # ---------------------------------------------------------------------------
+# FP8 (E4M3) tower GEMMs
+# ---------------------------------------------------------------------------
+
+def _act_array(cfg: Config, act_scales):
+    flat = [float(v) for row in act_scales for v in row]
+    if len(flat) != 4 * cfg.layers:
+        raise ValueError(f"act_scales needs {cfg.layers} rows of 4 scales")
+    return (ctypes.c_float * max(1, len(flat)))(*flat)
+
+
+def pack_tower_fp8(cfg: Config, w: dict, act_scales, stream=None) -> torch.Tensor:
+    """E4M3 tower (per-row weight scales, static activation scales act_scales[l][0..3])."""
+    L = lib()
+    tw = TowerWeights(**{k: _dev(w[k], k) for k, _ in TowerWeights._fields_})
+    nbytes = L.vlm_tower_fp8_packed_bytes(ctypes.byref(cfg))
+    if nbytes == 0:
+        raise VlmError(ERR_INVALID_ARG, "vlm_tower_fp8_packed_bytes")
+    packed = torch.empty(nbytes, dtype=torch.uint8, device=w["wq"].device)
+    _check(L.vlm_pack_tower_fp8(ctypes.byref(cfg), ctypes.byref(tw), _act_array(cfg, act_scales), packed.data_ptr(),
+                                nbytes, _stream(stream)), "vlm_pack_tower_fp8")
+    return packed
+
+
+def encode_fp8(cfg: Config, pixels: torch.Tensor, image_hw, packed_tower_fp8: torch.Tensor, act_scales, out=None,
+               workspace=None, status=None, stream=None) -> torch.Tensor:
+    """vlm_encode with the E4M3 tower GEMMs."""
+    L = lib()
+    arr, n = _hw_array(image_hw)
+    T = num_patches(cfg, image_hw)
+    dev = pixels.device
+    if out is None:
+        out = torch.empty((T, cfg.width), dtype=torch.bfloat16, device=dev)
+    if workspace is None:
+        workspace = torch.empty(L.vlm_encode_workspace_size(ctypes.byref(cfg), arr, n), dtype=torch.uint8, device=dev)
+    if status is None:
+        status = new_status(dev)
+    _check(L.vlm_encode_fp8(ctypes.byref(cfg), _dev(pixels, "pixels"), arr, n, _dev(packed_tower_fp8, "packed"),
+                            _act_array(cfg, act_scales), _dev(out, "out"), _dev(workspace, "workspace"),
+                            workspace.numel(), _dev(status, "status"), _stream(stream)), "vlm_encode_fp8")
+    return out
+
+
+def gemm_fp8(epilogue: int, a: torch.Tensor, b: torch.Tensor, colscale: torch.Tensor, out: torch.Tensor,
+             out_scale: float = 1.0, out_bf16=None, pos=None, rope=None, rope_cols: int = 0, status=None,
+             stream=None) -> torch.Tensor:
+    """E4M3 GEMM: a [M, K], b [N, K] as uint8 or float8_e4m3fn tensors."""
+    M, K = a.shape
+    N = b.shape[0]
+    if status is None:
+        status = new_status(a.device)
+    _check(lib().vlm_gemm_fp8(epilogue, _dev(a, "a"), _dev(b, "b"), _dev(colscale, "colscale"), float(out_scale),
+                              M, N, K, _dev(out, "out"), _dev(out_bf16, "out_bf16"), _dev(pos, "pos"),
+                              _dev(rope, "rope"), rope_cols, _dev(status, "status"), _stream(stream)), "vlm_gemm_fp8")
+    return out
+
+
+def rmsnorm_fp8(x: torch.Tensor, g1: torch.Tensor, f8_scale: float, g0=None, eps: float = 1e-5, out=None,
+                stream=None) -> torch.Tensor:
+    rows, width = x.shape
+    if out is None:
+        out = torch.empty((rows, width), dtype=torch.uint8, device=x.device)
+    _check(lib().vlm_rmsnorm_fp8(_dev(x, "x"), _dev(g0, "g0"), _dev(g1, "g1"), _dev(out, "out"), rows, width,
+                                 float(eps), float(f8_scale), _stream(stream)), "vlm_rmsnorm_fp8")
+    return out
+
+
+# ---------------------------------------------------------------------------
 # Image front end and placeholder expansion
 # ---------------------------------------------------------------------------
 
@@ -426,10 +498,14 @@ def profile_query(kclass: str) -> tuple:
 class ImagePipeline:
     """vlm_encode -> vlm_merge_project (-> vlm_scatter) with buffers kept between calls."""
 
-    def __init__(self, cfg: Config, tower: dict, projector: dict, image_hw, device="cuda"):
+    def __init__(self, cfg: Config, tower: dict, projector: dict, image_hw, device="cuda", fp8_act_scales=None):
+        """fp8_act_scales: None for the bf16 tower, or [layers][4] static activation
+        scales for the E4M3 tower GEMMs (vlm_encode_fp8)."""
         self.cfg = cfg
         self.image_hw = [tuple(int(v) for v in hw) for hw in image_hw]
-        self.packed_tower = pack_tower(cfg, tower)
+        self.fp8_act_scales = fp8_act_scales
+        self.packed_tower = pack_tower(cfg, tower) if fp8_act_scales is None else \
+            pack_tower_fp8(cfg, tower, fp8_act_scales)
         self.packed_proj = pack_projector(cfg, projector)
         self.T = num_patches(cfg, self.image_hw)
         self.Tm = num_merged(cfg, self.image_hw)
@@ -440,8 +516,12 @@ class ImagePipeline:
         self.status = new_status(device)
 
     def __call__(self, pixels: torch.Tensor, stream=None) -> torch.Tensor:
-        encode(self.cfg, pixels, self.image_hw, self.packed_tower, out=self.tower_out, workspace=self.workspace,
-               status=self.status, stream=stream)
+        if self.fp8_act_scales is None:
+            encode(self.cfg, pixels, self.image_hw, self.packed_tower, out=self.tower_out, workspace=self.workspace,
+                   status=self.status, stream=stream)
+        else:
+            encode_fp8(self.cfg, pixels, self.image_hw, self.packed_tower, self.fp8_act_scales, out=self.tower_out,
+                       workspace=self.workspace, status=self.status, stream=stream)
         merge_project(self.cfg, self.tower_out, self.image_hw, self.packed_proj, out=self.embeds,
                       workspace=self.workspace, status=self.status, stream=stream)
         return self.embeds
