@@ -72,6 +72,10 @@ def parse_args():
                    help="replay each step as one captured CUDA graph (headline and e2e loops)")
     p.add_argument("--side-stream", action="store_true",
                    help="also measure the encoder on a side stream overlapped with a decode-like GEMV loop")
+    p.add_argument("--gemm-shapes", action="store_true",
+                   help="instead of a step: time the tower's GEMM shapes (12,100 rows), bf16 and E4M3, each with its "
+                        "fused epilogue and with a plain store, beside torch's cuBLAS / cuBLASLt GEMM; one JSON line "
+                        "per shape")
     p.add_argument("--profile-steps", type=int, default=0,
                    help="for ncu: run this many plain steps after warmup and exit (no JSON)")
     return p.parse_args()
@@ -328,6 +332,68 @@ def ncu_traffic(kernel: str) -> float | None:
 KERNEL_SOURCES = {"attention": ["attention_tc.cu", "exp2_poly.cuh", "common.cuh", "kernels.cuh"],
                   "gemm": ["gemm_tcgen05.cu", "common.cuh", "kernels.cuh"],
                   "resize": ["frontend.cu", "common.cuh", "kernels.cuh"]}
+
+
+def gemm_shapes(args) -> None:
+    """Per-shape GEMM throughput of the tower's four GEMMs at M = 12,100 rows,
+    CUDA events around 20 back-to-back launches after 3 warm-ups."""
+    from vision_language_model_b200 import vlm
+
+    def timeit(fn, n=20):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(n):
+            fn()
+        b.record()
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / n
+
+    M = 12100
+    g = torch.Generator(device="cuda")
+    g.manual_seed(args.seed)
+    pos = torch.zeros(M, dtype=torch.int32, device="cuda")
+    rope = vlm.rope_table(1e4, 64, 128)
+    st = vlm.new_status()
+    shapes = [("gate/up", 8192, 1024, vlm.EPI_SWIGLU), ("qkv", 3072, 1024, vlm.EPI_ROPE),
+              ("o", 1024, 1024, vlm.EPI_RESID), ("down", 1024, 4096, vlm.EPI_RESID)]
+    for name, N, K, epi in shapes:
+        fl = 2.0 * M * N * K
+        kw = dict(pos=pos, rope=rope, rope_cols=2048) if epi == vlm.EPI_ROPE else {}
+        for dt in ("bf16", "e4m3"):
+            if dt == "bf16":
+                a = (torch.randn((M, K), device="cuda", generator=g)).to(torch.bfloat16)
+                b = (torch.randn((N, K), device="cuda", generator=g) * 0.02).to(torch.bfloat16)
+            else:
+                a = (torch.randn((M, K), device="cuda", generator=g) * 20).to(torch.float8_e4m3fn)
+                b = (torch.randn((N, K), device="cuda", generator=g) * 20).to(torch.float8_e4m3fn)
+                cs = torch.full((N,), 1e-3, device="cuda")
+            if epi == vlm.EPI_RESID:
+                c = torch.zeros((M, N), dtype=torch.float32, device="cuda")
+            elif epi == vlm.EPI_SWIGLU:
+                c = torch.empty((M, N // 2), dtype=torch.bfloat16 if dt == "bf16" else torch.uint8, device="cuda")
+            else:
+                c = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+            plain = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+            if dt == "bf16":
+                kw16 = dict(pos=pos, rope_table=rope, rope_cols=2048) if epi == vlm.EPI_ROPE else {}
+                fused = timeit(lambda: vlm.gemm(epi, a, b, c, status=st, **kw16))
+                store = timeit(lambda: vlm.gemm(vlm.EPI_BF16, a, b, plain, status=st))
+                lib_ms = timeit(lambda: torch.matmul(a, b.t()))
+                lib = "torch.matmul (cuBLAS)"
+            else:
+                au, bu = a.view(torch.uint8), b.view(torch.uint8)
+                fused = timeit(lambda: vlm.gemm_fp8(epi, au, bu, cs, c, out_scale=28.0, status=st, **kw))
+                store = timeit(lambda: vlm.gemm_fp8(vlm.EPI_BF16, au, bu, cs, plain, status=st))
+                one = torch.ones((), device="cuda")
+                lib_ms = timeit(lambda: torch._scaled_mm(a, b.t(), scale_a=one, scale_b=one, out_dtype=torch.bfloat16))
+                lib = "torch._scaled_mm (cuBLASLt)"
+            print(json.dumps({"gemm": name, "dtype": dt, "M": M, "N": N, "K": K, "epilogue": epi,
+                              "fused_ms": fused, "fused_tflops": fl / fused / 1e9,
+                              "plain_store_ms": store, "plain_store_tflops": fl / store / 1e9,
+                              "library": lib, "library_ms": lib_ms, "library_tflops": fl / lib_ms / 1e9}), flush=True)
 
 
 def side_stream_overlap(pipe, pix, ids, text, cfg, scatter_ws, dev, steps: int) -> dict:
@@ -608,6 +674,9 @@ def run_ours(args, wl):
 def main():
     args = parse_args()
     wl = WORKLOADS[args.workload]
+    if args.gemm_shapes:
+        gemm_shapes(args)
+        return
     if args.impl == "reference":
         run_reference(args, wl)
     else:
