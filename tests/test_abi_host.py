@@ -156,3 +156,35 @@ def test_front_end_argument_errors_return_before_launch(L):
                                      None) == vlm.ERR_BAD_SHAPE
     assert L.vlm_expand_placeholders(fake, 0, 99, zero, 0, 10, fake, 0, ctypes.byref(n_out), ws, 0, fake,
                                      None) == vlm.OK and n_out.value == 0
+
+
+def test_fp8_argument_errors_return_before_launch(L):
+    fake = ctypes.c_void_p(256)  # never dereferenced: every case fails validation first
+    cs = ctypes.c_void_p(512)
+    st = ctypes.c_void_p(1024)
+    # K % 128, N % 256, null colscale, unaligned operand, BF16-only epilogue set
+    assert L.vlm_gemm_fp8(vlm.EPI_BF16, fake, fake, cs, 1.0, 256, 256, 64, fake, None, None, None, 0, st,
+                          None) == vlm.ERR_UNSUPPORTED
+    assert L.vlm_gemm_fp8(vlm.EPI_BF16, fake, fake, cs, 1.0, 256, 128, 128, fake, None, None, None, 0, st,
+                          None) == vlm.ERR_UNSUPPORTED
+    assert L.vlm_gemm_fp8(vlm.EPI_BF16, fake, fake, None, 1.0, 256, 256, 128, fake, None, None, None, 0, st,
+                          None) == vlm.ERR_INVALID_ARG
+    assert L.vlm_gemm_fp8(vlm.EPI_BF16, ctypes.c_void_p(264), fake, cs, 1.0, 256, 256, 128, fake, None, None, None,
+                          0, st, None) == vlm.ERR_INVALID_ARG
+    assert L.vlm_gemm_fp8(vlm.EPI_GELU, fake, fake, cs, 1.0, 256, 256, 128, fake, None, None, None, 0, st,
+                          None) == vlm.ERR_UNSUPPORTED
+    assert L.vlm_rmsnorm_fp8(fake, None, fake, fake, 4, 1024, 1e-5, 0.0, None) == vlm.ERR_INVALID_ARG
+    cfg = vlm.preset("mistral3", layers=2)
+    tw = vlm.TowerWeights(**{k: 256 for k, _ in vlm.TowerWeights._fields_})
+    good = (ctypes.c_float * 8)(*([0.02] * 8))
+    for bad_vals in ([0.02] * 7 + [0.0], [0.02] * 7 + [-1.0], [0.02] * 7 + [float("nan")], [0.02] * 7 + [float("inf")]):
+        bad = (ctypes.c_float * 8)(*bad_vals)
+        assert L.vlm_pack_tower_fp8(ctypes.byref(cfg), ctypes.byref(tw), bad, fake, 1 << 40, None) == \
+            vlm.ERR_INVALID_ARG
+    assert L.vlm_pack_tower_fp8(ctypes.byref(cfg), ctypes.byref(tw), None, fake, 1 << 40, None) == vlm.ERR_INVALID_ARG
+    assert L.vlm_pack_tower_fp8(ctypes.byref(cfg), ctypes.byref(tw), good, fake, 16, None) == vlm.ERR_WORKSPACE
+    hw = (ctypes.c_int32 * 2)(224, 224)
+    assert L.vlm_encode_fp8(ctypes.byref(cfg), fake, hw, 1, fake, None, fake, fake, 1 << 40, st, None) == \
+        vlm.ERR_INVALID_ARG
+    fp8_bytes = L.vlm_tower_fp8_packed_bytes(ctypes.byref(cfg))
+    assert 0 < fp8_bytes < L.vlm_tower_packed_bytes(ctypes.byref(cfg))
