@@ -1,7 +1,7 @@
-"""The software exp2 of the attention softmax (exp2_poly2 in attention_tc.cu).
+"""The software exp2 of the attention softmax (exp2_poly in attention_tc.cu).
 
-It replaces ex2.approx for a fixed fraction of the scores so the MUFU and FMA
-pipes share the work. Its result is rounded to bf16 (relative step 2^-8) right
+It replaces ex2.approx for one score pair in eight so the MUFU and FMA pipes
+share the work. Its result is rounded to bf16 (relative step 2^-8) right
 after, so the bar is 1/16 of a bf16 half-step: 2^-9 / 16 = 1.2e-4 relative
 error. (CUDA's exp2f is within 2 ulp, 2.4e-7; ex2.approx.ftz within about
 2^-22.) These tests re-run the Remez fit, and evaluate the kernel's exact fp32

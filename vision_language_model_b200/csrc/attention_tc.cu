@@ -18,7 +18,8 @@
 //               the tile max exceeds it by more than 8 (otherwise the stale max
 //               is kept; P stays <= 2^8 and the final division by l is exact),
 //               computes P = 2^(s*log2e/8 - m) with packed fp32x2 FMAs and MUFU
-//               ex2, writes P to TMEM as bf16, sums the fp32 values into l with
+//               ex2 (one pair in eight from an FMA-pipe polynomial), writes P
+//               to TMEM as bf16, sums the fp32 values into l with
 //               packed adds, rescales its O row when m moved, and finally writes
 //               O / l.
 // TMEM: S in columns [0,128), P in [128,192) (bf16 pairs), O in [192,256).
@@ -113,44 +114,35 @@ __device__ __forceinline__ void tmem_st64(uint32_t taddr, const uint32_t (&r)[64
       : "memory");
 }
 
-__device__ __forceinline__ uint64_t sub2(uint64_t a, uint64_t b) {
-  uint64_t d;
-  asm("sub.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-  return d;
-}
 
 // One pair of scores in kPolyPairEvery takes its two exponentials from
-// exp2_poly2 (FMA and ALU pipes) instead of ex2.approx (MUFU), so the two
-// kinds of pipe share the softmax's exponentials.
+// exp2_poly (FMA and ALU pipes) instead of ex2.approx (MUFU), so the two kinds
+// of pipe share the softmax's exponentials. MUFU is the softmax's bottleneck;
+// one pair in eight is the largest share that still fits the 168 registers a
+// thread has at 2 CTAs per SM without spilling.
 #ifndef VLM_ATTN_POLY_PAIR_EVERY
-#define VLM_ATTN_POLY_PAIR_EVERY 0
+#define VLM_ATTN_POLY_PAIR_EVERY 8
 #endif
 constexpr int kPolyPairEvery = VLM_ATTN_POLY_PAIR_EVERY;
 
-// (2^x0, 2^x1) without MUFU: k = round(x) by adding 1.5 * 2^23, f = x - k in
+// 2^x without MUFU: k = round(x) by adding 1.5 * 2^23, f = x - k in
 // [-1/2, 1/2], 2^f from the degree-3 minimax polynomial of exp2_poly.cuh
 // (relative error < 7.5e-5, fitted by fit_exp2_poly.py with the Remez
-// algorithm), then k added to the exponent field; packed fp32x2 arithmetic.
-// x is clamped to -126 so the exponent cannot wrap; the result is then ~1e-38
-// instead of 0, so keys that must weigh exactly 0 never take this path.
-__device__ __forceinline__ void exp2_poly2(float x0, float x1, float& p0, float& p1) {
-  const uint64_t x = pack2(__float_as_uint(fmaxf(x0, -126.0f)), __float_as_uint(fmaxf(x1, -126.0f)));
-  const uint64_t magic = pair_f32(12582912.0f);
-  const uint64_t j = add2(x, magic);
-  const uint64_t f = sub2(x, sub2(j, magic));
-  uint64_t p = fma2(pair_f32(kExp2C3), f, pair_f32(kExp2C2));
-  p = fma2(p, f, pair_f32(kExp2C1));
-  p = fma2(p, f, pair_f32(kExp2C0));
-  float pl, ph, jl, jh;
-  unpack2(p, pl, ph);
-  unpack2(j, jl, jh);
-  p0 = __int_as_float(__float_as_int(pl) + (__float_as_int(jl) << 23));
-  p1 = __int_as_float(__float_as_int(ph) + (__float_as_int(jh) << 23));
+// algorithm), then k added to the exponent field. Scalar arithmetic with
+// immediate constants (no register pairs). x is clamped to -126 so the
+// exponent cannot wrap; the result is then ~1e-38 instead of 0, so keys that
+// must weigh exactly 0 never take this path.
+__device__ __forceinline__ float exp2_poly(float x) {
+  x = fmaxf(x, -126.0f);
+  const float j = x + 12582912.0f;
+  const float f = x - (j - 12582912.0f);
+  const float p = fmaf(fmaf(fmaf(kExp2C3, f, kExp2C2), f, kExp2C1), f, kExp2C0);
+  return __int_as_float(__float_as_int(p) + (__float_as_int(j) << 23));
 }
 
 // p_c = 2^(s_c * sl2 - m) for the row's 128 scores, packed as bf16 pairs into
 // pk; returns sum_c p_c (fp32, before rounding). The elements are independent.
-// kPoly: let exp2_poly2 take one pair in kPolyPairEvery (never on a tile with
+// kPoly: let exp2_poly take one pair in kPolyPairEvery (never on a tile with
 // masked keys, whose weights must be exactly 0).
 template <bool kPoly>
 __device__ __forceinline__ float row_exp(const uint32_t (&u)[BKV], uint64_t sl2x2, float m, uint32_t (&pk)[BKV / 2]) {
@@ -161,7 +153,8 @@ __device__ __forceinline__ float row_exp(const uint32_t (&u)[BKV], uint64_t sl2x
     float x0, x1, p0, p1;
     unpack2(fma2(pack2(u[c], u[c + 1]), sl2x2, negm2), x0, x1);
     if (kPoly && kPolyPairEvery > 0 && (c >> 1) % (kPolyPairEvery > 0 ? kPolyPairEvery : 1) == kPolyPairEvery - 1) {
-      exp2_poly2(x0, x1, p0, p1);
+      p0 = exp2_poly(x0);
+      p1 = exp2_poly(x1);
     } else {
       p0 = ex2(x0);
       p1 = ex2(x1);
