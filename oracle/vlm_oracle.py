@@ -537,10 +537,17 @@ def projector(x_tower: np.ndarray, grids, pw: dict, cfg: dict) -> np.ndarray:
     ("Mistral 3", `Mistral3Model`: 2x2 patch-merging projector, projector_bias
     False, text width 5120.) pw: g_proj [D], w_merge [D, m*m*D], w1 [E, D],
     w2 [E, E].
+    cfg["norm_after_merge"] (default False) takes the other reading of the
+    pages' order: merge -> merge linear -> RMSNorm over the merged D-vector ->
+    W1 -> GELU -> W2 (the same g_proj; with merge 1 both readings coincide).
     """
-    xn = rms_norm(x_tower, pw["g_proj"], cfg["eps"])
-    z = merge_unfold(xn, grids, cfg["merge"]) if cfg["merge"] > 1 else xn
-    y = z @ np.asarray(pw["w_merge"], dtype=np.float64).T if cfg["merge"] > 1 else z
+    eps, m = cfg["eps"], cfg["merge"]
+    after = bool(cfg.get("norm_after_merge", False)) and m > 1
+    xn = np.asarray(x_tower, dtype=np.float64) if after else rms_norm(x_tower, pw["g_proj"], eps)
+    z = merge_unfold(xn, grids, m) if m > 1 else xn
+    y = z @ np.asarray(pw["w_merge"], dtype=np.float64).T if m > 1 else z
+    if after:
+        y = rms_norm(y, pw["g_proj"], eps)
     return gelu(y @ np.asarray(pw["w1"], dtype=np.float64).T) @ np.asarray(pw["w2"], dtype=np.float64).T
 
 

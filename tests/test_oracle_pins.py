@@ -577,3 +577,35 @@ def test_planted_e4m3_truncation_is_caught(monkeypatch):
     monkeypatch.setattr(O, "e4m3_round", bad)
     with pytest.raises(AssertionError):
         test_e4m3_matches_torch_float8_and_saturates()
+
+
+@pytest.mark.parametrize("after", [False, True])
+def test_projector_both_norm_orders_match_torch_composition(after):
+    """The projector in either reading of the norm's place equals the same
+    steps written with torch (rms_norm, unfold, linear, exact GELU)."""
+    d, e = 8, 12
+    grids = [(4, 6), (2, 2)]
+    x = RNG.standard_normal((28, d))
+    pw = {"g_proj": 1 + 0.1 * RNG.standard_normal(d), "w_merge": RNG.standard_normal((d, 4 * d)) * 0.3,
+          "w1": RNG.standard_normal((e, d)) * 0.3, "w2": RNG.standard_normal((e, e)) * 0.3}
+    cfg = dict(O.MISTRAL3, eps=1e-5, merge=2, norm_after_merge=after)
+    got = O.projector(x, grids, pw, cfg)
+    t = {k: torch.from_numpy(v) for k, v in pw.items()}
+    xt = torch.from_numpy(x)
+    if not after:
+        xt = F.rms_norm(xt, (d,), t["g_proj"], eps=1e-5)
+    zs, off = [], 0
+    for h, w in grids:
+        img = xt[off:off + h * w].reshape(h, w, d).permute(2, 0, 1)[None]
+        zs.append(F.unfold(img, kernel_size=2, stride=2)[0].T)
+        off += h * w
+    y = torch.cat(zs) @ t["w_merge"].T
+    if after:
+        y = F.rms_norm(y, (d,), t["g_proj"], eps=1e-5)
+    ref = F.gelu(y @ t["w1"].T, approximate="none") @ t["w2"].T
+    np.testing.assert_allclose(got, ref.numpy(), rtol=1e-12, atol=1e-12)
+    other = O.projector(x, grids, pw, dict(cfg, norm_after_merge=not after))
+    assert np.abs(other - got).max() > 1e-3  # the two readings really differ
+    # with merge 1 the flag changes nothing
+    cfg1 = dict(cfg, merge=1)
+    np.testing.assert_array_equal(O.projector(x, [(28, 1)], pw, cfg1), O.projector(x, [(28, 1)], pw, dict(cfg1, norm_after_merge=not after)))
