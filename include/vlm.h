@@ -67,11 +67,15 @@ typedef enum {
  * eps: RMSNorm epsilon (reading: 1e-5, the only norm_eps the pages give).
  * normalize: 1 = `pixels` hold raw [0,1] values and the processor's per-channel
  * (x - mean)/std ([K] Mistral3ImageProcessor) is applied while gathering
- * patches; 0 = `pixels` are already normalised. */
+ * patches; 0 = `pixels` are already normalised.
+ * norm_after_merge: 0 = the projector RMSNorm runs per patch before the merge
+ * (reading); 1 = the other reading of the pages' order: after the merge
+ * linear, on the merged width-vector (same gain). No effect with merge == 1. */
 typedef struct {
   int32_t layers, width, heads, head_dim, mlp, patch, merge, proj_out, image_token_id;
   float rope_theta, eps;
   int32_t normalize;
+  int32_t norm_after_merge;
 } vlm_config;
 
 /* Tower weights, device pointers, stacked over layers (L = cfg.layers,

@@ -66,6 +66,14 @@ def test_bad_shapes_rejected_on_host(L, hw):
     assert e.value.rc == vlm.ERR_BAD_SHAPE
 
 
+def test_norm_after_merge_flag_checked(L):
+    c = vlm.preset("mistral3")
+    assert c.norm_after_merge == 0
+    c.norm_after_merge = 2
+    hw = (ctypes.c_int32 * 2)(224, 224)
+    assert L.vlm_num_patches(ctypes.byref(c), hw, 1) == vlm.ERR_INVALID_ARG
+
+
 def test_unsupported_config_rejected(L):
     with pytest.raises(vlm.VlmError) as e:
         vlm.num_patches(vlm.preset("mistral3", head_dim=128, heads=8), [(28, 28)])

@@ -174,3 +174,20 @@ def test_full_size_pixtral_4096_as_16_tiles():
     for b in range(16):
         same = torch.equal(e1[4096 * b:4096 * (b + 1)], e2[4096 * b:4096 * (b + 1)])
         assert same == (b != 7), b
+
+
+def test_projector_norm_after_merge_vs_oracle():
+    """The other reading of the projector norm's place (after the merge linear)."""
+    sizes = [(84, 140), (56, 112)]
+    cfg, tw, pw, imgs = _setup("mistral3", 2, sizes, seed=4)
+    cfg.norm_after_merge = 1
+    tower, emb = _run_gpu(cfg, tw, pw, imgs, sizes)
+    ocfg = dict(_oracle_cfg(cfg), norm_after_merge=True)
+    ref_tower, ref_emb = O.encode_merge_project([im.double().numpy() for im in imgs], to_oracle(tw), to_oracle(pw),
+                                                ocfg)
+    compare(tower, ref_tower, what="tower")
+    compare(emb, ref_emb, what="projector, norm after merge")
+    # and it is not the default reading's result
+    _, ref_before = O.encode_merge_project([im.double().numpy() for im in imgs], to_oracle(tw), to_oracle(pw),
+                                           _oracle_cfg(cfg))
+    assert np.abs(to_np(emb) - ref_before).max() > 0.05 * np.abs(ref_before).max()

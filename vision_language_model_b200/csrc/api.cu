@@ -91,6 +91,7 @@ int check_config(const vlm_config* c) {
   if (c->layers < 0 || c->width <= 0 || c->heads <= 0 || c->head_dim <= 0 || c->mlp <= 0 || c->patch <= 0 ||
       c->merge <= 0 || c->proj_out <= 0 || !(c->rope_theta > 0.f) || !(c->eps >= 0.f))
     return VLM_ERR_INVALID_ARG;
+  if (c->norm_after_merge != 0 && c->norm_after_merge != 1) return VLM_ERR_INVALID_ARG;
   if (c->head_dim != 64 || c->heads * c->head_dim != c->width) return VLM_ERR_UNSUPPORTED;
   if (c->width % 256 || c->width > 2048 || c->mlp % 128 || c->proj_out % 256) return VLM_ERR_UNSUPPORTED;
   if (c->patch > 64) return VLM_ERR_UNSUPPORTED;
@@ -374,6 +375,7 @@ int vlm_config_preset(int preset, vlm_config* cfg) {
   cfg->rope_theta = 10000.0f;
   cfg->eps = 1e-5f;
   cfg->normalize = 1;
+  cfg->norm_after_merge = 0;
   return VLM_OK;
 }
 
@@ -628,14 +630,18 @@ int vlm_merge_project(const vlm_config* cfg, const void* d_tower_out, const int3
   const uint8_t* pk = static_cast<const uint8_t*>(d_packed_projector);
   const int64_t D = cfg->width, E = cfg->proj_out, mm = static_cast<int64_t>(cfg->merge) * cfg->merge;
 
+  const bool after = cfg->norm_after_merge != 0 && cfg->merge > 1;
+  const float* g_proj = reinterpret_cast<const float*>(pk + L.g_proj);
   VLM_TRY(upload_batch(b, p.bd, s));
-  VLM_TRY(launch_merge_norm(static_cast<const __nv_bfloat16*>(d_tower_out), reinterpret_cast<const float*>(pk + L.g_proj),
-                            p.bd.info, p.bd.cu, b.n, b.T, static_cast<int>(D), cfg->merge, cfg->eps, p.z, s));
+  // the merge gather, normalising each patch unless the norm follows the merge linear
+  VLM_TRY(launch_merge_norm(static_cast<const __nv_bfloat16*>(d_tower_out), after ? nullptr : g_proj, p.bd.info,
+                            p.bd.cu, b.n, b.T, static_cast<int>(D), cfg->merge, cfg->eps, p.z, s));
   const __nv_bfloat16* y = p.z;
   if (cfg->merge > 1) {
     VLM_TRY(launch_gemm(VLM_EPI_BF16, p.z, pk + L.w_merge, b.Tm, D, mm * D, p.y, nullptr, nullptr, nullptr, 0,
                         d_status, s));
     y = p.y;
+    if (after) VLM_TRY(launch_rmsnorm_bf16(p.y, g_proj, p.y, b.Tm, static_cast<int>(D), cfg->eps, s));
   }
   VLM_TRY(launch_gemm(VLM_EPI_GELU, y, pk + L.w1, b.Tm, E, D, p.g, nullptr, nullptr, nullptr, 0, d_status, s));
   VLM_TRY(launch_gemm(VLM_EPI_BF16, p.g, pk + L.w2, b.Tm, E, E, d_out, nullptr, nullptr, nullptr, 0, d_status, s));

@@ -78,6 +78,10 @@ int launch_im2col(const float* pix, const ImgInfo* info, const int32_t* cu, int 
 // f8_scale > 0: `out` is E4M3 holding the normalised values times f8_scale; else bf16.
 int launch_rmsnorm(float* x, const float* g0, const float* g1, void* out, int64_t rows, int width, float eps,
                    cudaStream_t s, float f8_scale = 0.f);
+// RMSNorm of bf16 rows [rows, width] into bf16 (out may equal x).
+int launch_rmsnorm_bf16(const __nv_bfloat16* x, const float* g, __nv_bfloat16* out, int64_t rows, int width,
+                        float eps, cudaStream_t s);
+// g == nullptr: gather only (no normalisation).
 int launch_merge_norm(const __nv_bfloat16* x, const float* g, const ImgInfo* info, const int32_t* cu,
                       int n_images, int64_t T, int width, int m, float eps, __nv_bfloat16* z,
                       cudaStream_t s);

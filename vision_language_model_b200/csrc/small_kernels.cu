@@ -210,7 +210,7 @@ __global__ void merge_norm_kernel(const __nv_bfloat16* __restrict__ x, const flo
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-    const float rs = rsqrtf(ss / width + eps);
+    const float rs = g != nullptr ? rsqrtf(ss / width + eps) : 1.0f;
     const int b = find_block(cu, n_images, static_cast<int>(t));
     const ImgInfo in = info[b];
     const int local = static_cast<int>(t) - in.tok_off;
@@ -218,6 +218,45 @@ __global__ void merge_norm_kernel(const __nv_bfloat16* __restrict__ x, const flo
     const int64_t mt = in.m_off + (r / m) * (in.w / m) + c / m;
     const int slot = (r % m) * m + c % m;
     uint2* orow = reinterpret_cast<uint2*>(z + (mt * m * m + slot) * width);
+    const float4* gr = reinterpret_cast<const float4*>(g);
+#pragma unroll
+    for (int j = 0; j < NV; ++j) {
+      const float4 gg = g != nullptr ? __ldg(gr + lane + 32 * j) : make_float4(1.f, 1.f, 1.f, 1.f);
+      uint2 o;
+      o.x = pack_bf16x2(v[j][0] * rs * gg.x, v[j][1] * rs * gg.y);
+      o.y = pack_bf16x2(v[j][2] * rs * gg.z, v[j][3] * rs * gg.w);
+      orow[lane + 32 * j] = o;
+    }
+  }
+}
+
+// RMSNorm of bf16 rows into bf16 (in place allowed), one warp per row.
+template <int NV>
+__global__ void rmsnorm_bf16_kernel(const __nv_bfloat16* x, const float* __restrict__ g, __nv_bfloat16* out,
+                                    int64_t rows, float eps) {
+  griddep_wait();
+  griddep_launch_dependents();
+  constexpr int width = NV * 128;
+  const int lane = threadIdx.x & 31;
+  const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
+  for (int64_t t = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; t < rows; t += warps) {
+    const uint2* xr = reinterpret_cast<const uint2*>(x + t * width);
+    float v[NV][4];
+    float ss = 0.f;
+#pragma unroll
+    for (int j = 0; j < NV; ++j) {
+      const uint2 u = xr[lane + 32 * j];
+      const __nv_bfloat162 a = *reinterpret_cast<const __nv_bfloat162*>(&u.x);
+      const __nv_bfloat162 bb = *reinterpret_cast<const __nv_bfloat162*>(&u.y);
+      v[j][0] = __low2float(a); v[j][1] = __high2float(a);
+      v[j][2] = __low2float(bb); v[j][3] = __high2float(bb);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) ss += v[j][e] * v[j][e];
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    const float rs = rsqrtf(ss / width + eps);
+    uint2* orow = reinterpret_cast<uint2*>(out + t * width);
     const float4* gr = reinterpret_cast<const float4*>(g);
 #pragma unroll
     for (int j = 0; j < NV; ++j) {
@@ -484,6 +523,26 @@ int launch_merge_norm(const __nv_bfloat16* x, const float* g, const ImgInfo* inf
     VLM_MERGE_CASE(11) VLM_MERGE_CASE(12) VLM_MERGE_CASE(13) VLM_MERGE_CASE(14) VLM_MERGE_CASE(15)
     VLM_MERGE_CASE(16)
 #undef VLM_MERGE_CASE
+    default: break;
+  }
+  launch_end(KC_MERGE, s);
+  return e == cudaSuccess ? VLM_OK : VLM_ERR_CUDA;
+}
+
+int launch_rmsnorm_bf16(const __nv_bfloat16* x, const float* g, __nv_bfloat16* out, int64_t rows, int width,
+                        float eps, cudaStream_t s) {
+  if (width % 128 || width > 2048 || width <= 0) return VLM_ERR_UNSUPPORTED;
+  const int grid = grid_for(rows * 32, 256);
+  launch_begin(KC_MERGE, s);
+  cudaError_t e = cudaErrorInvalidValue;
+  switch (width / 128) {
+#define VLM_NORM16_CASE(nv) \
+  case nv: e = launch_pdl(rmsnorm_bf16_kernel<nv>, dim3(grid), dim3(256), 0, s, x, g, out, rows, eps); break;
+    VLM_NORM16_CASE(1) VLM_NORM16_CASE(2) VLM_NORM16_CASE(3) VLM_NORM16_CASE(4) VLM_NORM16_CASE(5)
+    VLM_NORM16_CASE(6) VLM_NORM16_CASE(7) VLM_NORM16_CASE(8) VLM_NORM16_CASE(9) VLM_NORM16_CASE(10)
+    VLM_NORM16_CASE(11) VLM_NORM16_CASE(12) VLM_NORM16_CASE(13) VLM_NORM16_CASE(14) VLM_NORM16_CASE(15)
+    VLM_NORM16_CASE(16)
+#undef VLM_NORM16_CASE
     default: break;
   }
   launch_end(KC_MERGE, s);
