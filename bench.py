@@ -570,6 +570,9 @@ def run_ours(args, wl):
     n_norm, ms_norm = vlm.profile_query("rmsnorm")
     n_resize, ms_resize = vlm.profile_query("resize")
     n_expand, ms_expand = vlm.profile_query("expand")
+    n_im2col, ms_im2col = vlm.profile_query("im2col")
+    n_merge, ms_merge = vlm.profile_query("merge")
+    n_scatter, ms_scatter = vlm.profile_query("scatter")
     vlm.profile_enable(False)
     rc = vlm.status_sync(pipe.status)
     if rc != vlm.OK:
@@ -615,7 +618,8 @@ def run_ours(args, wl):
                                    "measured_burst": step_tflops / peaks["bf16_tflops"],
                                    "nominal_2250": step_tflops / 2250.0},
         "kernels_ms_per_step": {"gemm": ms_gemm / args.steps, "attention": ms_attn / args.steps,
-                                "rmsnorm": ms_norm / args.steps,
+                                "rmsnorm": ms_norm / args.steps, "patch_gather": ms_im2col / args.steps,
+                                "merge_gather": ms_merge / args.steps, "scatter": ms_scatter / args.steps,
                                 "step_with_events": ms_profiled / args.steps,
                                 "note": "per-kernel CUDA events on the launch stream, in a second pass of the "
                                         "same steps"},
@@ -658,6 +662,23 @@ def run_ours(args, wl):
                        "traffic": ncu_traffic("resize")},
             "expand_ms_per_step": ms_expand / args.steps,
         }
+    # memory-bound kernels: algorithmic bytes per step / their event-timed device time
+    D_, p_ = cfg.width, cfg.patch
+    kp_ = -(-3 * p_ * p_ // 64) * 64
+    row_bytes = cfg.proj_out * 2
+    mb = {
+        "rmsnorm": (2 * cfg.layers * T * D_ * (4 + 2) + T * D_ * 4, ms_norm,
+                    "per launch: fp32 row read + bf16 row written (+ the fp32 write-back of ln_pre once)"),
+        "patch_gather": (T * (3 * p_ * p_ * 4 + kp_ * 2), ms_im2col, "fp32 pixels read + bf16 patch rows written"),
+        "merge_gather": (2 * T * D_ * 2, ms_merge, "bf16 tower rows read + bf16 merged rows written"),
+        "scatter": (2 * Tm * row_bytes + ids.numel() * 8, ms_scatter,
+                    "image rows read + written into the text rows + ids read"),
+    }
+    line["memory_bound_kernels"] = {
+        k: {"bytes_per_step": int(b), "ms_per_step": t / args.steps,
+            "achieved_gbs": b / (t / args.steps / 1e3) / 1e9 if t > 0 else None,
+            "frac_of_hbm": b / (t / args.steps / 1e3) / 1e9 / peaks["hbm_gbs"] if t > 0 else None, "bytes": note}
+        for k, (b, t, note) in mb.items()}
     if args.graph:
         line["config"]["launch"] = f"one CUDA graph per step ({graph.launches_per_replay} kernels)"
     if args.side_stream:

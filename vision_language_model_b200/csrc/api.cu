@@ -106,7 +106,8 @@ struct Batch {
   int64_t T = 0, Tm = 0;
   int total_qtiles = 0;
   int max_pos = 0;
-  std::vector<int32_t> h, w, H, W, tok_off, m_off, qt_off;
+  int i2c_items = 0;
+  std::vector<int32_t> h, w, H, W, tok_off, m_off, qt_off, i2c_off;
   std::vector<int64_t> pix_off;
 };
 
@@ -115,7 +116,8 @@ int make_batch(const vlm_config* c, const int32_t* hw, int n, Batch* b) {
   b->n = n;
   b->h.resize(n); b->w.resize(n); b->H.resize(n); b->W.resize(n);
   b->tok_off.resize(n + 1); b->m_off.resize(n + 1); b->qt_off.resize(n + 1); b->pix_off.resize(n);
-  int64_t t = 0, tm = 0, qt = 0, pix = 0;
+  b->i2c_off.resize(n + 1);
+  int64_t t = 0, tm = 0, qt = 0, pix = 0, i2c = 0;
   int maxp = 1;
   for (int i = 0; i < n; ++i) {
     const int Hh = hw[2 * i], Ww = hw[2 * i + 1];
@@ -127,7 +129,9 @@ int make_batch(const vlm_config* c, const int32_t* hw, int n, Batch* b) {
     b->tok_off[i] = static_cast<int32_t>(t);
     b->m_off[i] = static_cast<int32_t>(tm);
     b->qt_off[i] = static_cast<int32_t>(qt);
+    b->i2c_off[i] = static_cast<int32_t>(i2c);
     b->pix_off[i] = pix;
+    i2c += static_cast<int64_t>(hp) * ((wp + kI2cPatches - 1) / kI2cPatches);
     const int64_t L = static_cast<int64_t>(hp) * wp;
     t += L;
     tm += L / (c->merge * c->merge);
@@ -139,6 +143,8 @@ int make_batch(const vlm_config* c, const int32_t* hw, int n, Batch* b) {
   b->tok_off[n] = static_cast<int32_t>(t);
   b->m_off[n] = static_cast<int32_t>(tm);
   b->qt_off[n] = static_cast<int32_t>(qt);
+  b->i2c_off[n] = static_cast<int32_t>(i2c);
+  b->i2c_items = static_cast<int>(i2c);
   b->T = t;
   b->Tm = tm;
   b->total_qtiles = static_cast<int>(qt);
@@ -151,6 +157,7 @@ struct BatchDev {
   ImgInfo* info;
   int32_t* cu;
   int32_t* qt;
+  int32_t* i2c;
   int32_t* pos;
   float2* rope;
 };
@@ -160,6 +167,7 @@ BatchDev carve_batch(Carver& cv, const Batch& b, bool with_pos, int head_dim) {
   d.info = cv.take<ImgInfo>(b.n);
   d.cu = cv.take<int32_t>(b.n + 1);
   d.qt = cv.take<int32_t>(b.n + 1);
+  d.i2c = with_pos ? cv.take<int32_t>(b.n + 1) : nullptr;
   d.pos = with_pos ? cv.take<int32_t>(b.T) : nullptr;
   d.rope = with_pos ? cv.take<float2>(static_cast<size_t>(b.max_pos) * head_dim / 2) : nullptr;
   return d;
@@ -176,12 +184,14 @@ int upload_batch(const Batch& b, const BatchDev& d, cudaStream_t s) {
       ch.tok_off[i] = b.tok_off[first + i];
       ch.m_off[i] = b.m_off[first + i];
       ch.qt_off[i] = b.qt_off[first + i];
+      ch.i2c_off[i] = b.i2c_off[first + i];
       ch.pix_off[i] = b.pix_off[first + i];
     }
     ch.tok_off[ch.count] = b.tok_off[first + ch.count];
     ch.m_off[ch.count] = b.m_off[first + ch.count];
     ch.qt_off[ch.count] = b.qt_off[first + ch.count];
-    const int rc = launch_setup(ch, d.info, d.cu, d.qt, d.pos, b.n, s);
+    ch.i2c_off[ch.count] = b.i2c_off[first + ch.count];
+    const int rc = launch_setup(ch, d.info, d.cu, d.qt, d.i2c, d.pos, b.n, s);
     if (rc != VLM_OK) return rc;
   }
   return VLM_OK;
@@ -484,8 +494,8 @@ int vlm_encode(const vlm_config* cfg, const float* pixels, const int32_t* image_
 
   VLM_TRY(upload_batch(b, e.bd, s));
   VLM_TRY(launch_rope_table(cfg->rope_theta, cfg->head_dim, b.max_pos, e.bd.rope, s));
-  VLM_TRY(launch_im2col(pixels, e.bd.info, e.bd.cu, b.n, T, cfg->patch, static_cast<int>(kp), cfg->normalize,
-                        e.cols, s));
+  VLM_TRY(launch_im2col(pixels, e.bd.info, e.bd.cu, e.bd.i2c, b.i2c_items, b.n, T, cfg->patch,
+                        static_cast<int>(kp), cfg->normalize, e.cols, s));
   VLM_TRY(launch_gemm(VLM_EPI_F32, e.cols, pk + L.w_pe, T, D, kp, e.x, nullptr, nullptr, nullptr, 0, d_status, s));
   for (int l = 0; l < cfg->layers; ++l) {
     const uint8_t* ly = pk + L.layer0 + L.layer_stride * l;
@@ -576,8 +586,8 @@ int vlm_encode_fp8(const vlm_config* cfg, const float* pixels, const int32_t* im
 
   VLM_TRY(upload_batch(b, e.bd, s));
   VLM_TRY(launch_rope_table(cfg->rope_theta, cfg->head_dim, b.max_pos, e.bd.rope, s));
-  VLM_TRY(launch_im2col(pixels, e.bd.info, e.bd.cu, b.n, T, cfg->patch, static_cast<int>(kp), cfg->normalize,
-                        e.cols, s));
+  VLM_TRY(launch_im2col(pixels, e.bd.info, e.bd.cu, e.bd.i2c, b.i2c_items, b.n, T, cfg->patch,
+                        static_cast<int>(kp), cfg->normalize, e.cols, s));
   VLM_TRY(launch_gemm(VLM_EPI_F32, e.cols, pk + L.w_pe, T, D, kp, e.x, nullptr, nullptr, nullptr, 0, d_status, s));
   for (int l = 0; l < cfg->layers; ++l) {
     const uint8_t* ly = pk + L.layer0 + L.layer_stride * l;
@@ -863,6 +873,7 @@ int vlm_attention(const void* d_qkv, int64_t T, int heads, int head_dim, const i
   b.T = T;
   b.h.assign(n_blocks, 1); b.w.assign(n_blocks, 1); b.H.assign(n_blocks, 0); b.W.assign(n_blocks, 0);
   b.tok_off.resize(n_blocks + 1); b.m_off.assign(n_blocks + 1, 0); b.qt_off.resize(n_blocks + 1);
+  b.i2c_off.assign(n_blocks + 1, 0);
   b.pix_off.assign(n_blocks, 0);
   int64_t qt = 0;
   for (int i = 0; i < n_blocks; ++i) {
@@ -880,6 +891,7 @@ int vlm_attention(const void* d_qkv, int64_t T, int heads, int head_dim, const i
   d.info = cv.take<ImgInfo>(n_blocks);
   d.cu = cv.take<int32_t>(n_blocks + 1);
   d.qt = cv.take<int32_t>(n_blocks + 1);
+  d.i2c = nullptr;
   d.pos = nullptr;
   d.rope = nullptr;
   cudaStream_t s = as_stream(stream);

@@ -22,8 +22,12 @@ struct ImageChunk {
   int32_t first, count;
   int32_t h[kChunk], w[kChunk], H[kChunk], W[kChunk];
   int32_t tok_off[kChunk + 1], m_off[kChunk + 1], qt_off[kChunk + 1];
+  int32_t i2c_off[kChunk + 1];  // first patch-gather work item of each image
   int64_t pix_off[kChunk];
 };
+
+// Patches per work item of the tiled patch gather (one patch row segment).
+constexpr int kI2cPatches = 8;
 
 struct ScatterWs {
   int32_t* chunk_count;
@@ -70,11 +74,13 @@ constexpr int kAttnBQ = 128;
 
 void note_extra_launches(int n);
 
-int launch_setup(const ImageChunk& chunk, ImgInfo* info, int32_t* cu, int32_t* qt, int32_t* pos,
+int launch_setup(const ImageChunk& chunk, ImgInfo* info, int32_t* cu, int32_t* qt, int32_t* i2c, int32_t* pos,
                  int n_images, cudaStream_t s);
 int launch_rope_table(float theta, int head_dim, int max_pos, float2* tab, cudaStream_t s);
-int launch_im2col(const float* pix, const ImgInfo* info, const int32_t* cu, int n_images, int64_t T,
-                  int p, int kp, int normalize, __nv_bfloat16* out, cudaStream_t s);
+// i2c / i2c_items: work items of the tiled gather (p 14 or 16); other patch
+// sizes use one warp per patch.
+int launch_im2col(const float* pix, const ImgInfo* info, const int32_t* cu, const int32_t* i2c, int i2c_items,
+                  int n_images, int64_t T, int p, int kp, int normalize, __nv_bfloat16* out, cudaStream_t s);
 // f8_scale > 0: `out` is E4M3 holding the normalised values times f8_scale; else bf16.
 int launch_rmsnorm(float* x, const float* g0, const float* g1, void* out, int64_t rows, int width, float eps,
                    cudaStream_t s, float f8_scale = 0.f);

@@ -9,7 +9,7 @@ namespace vlm {
 // ---------------------------------------------------------------------------
 // Index setup: per-image tables and per-token (row, col) positions.
 // ---------------------------------------------------------------------------
-__global__ void setup_kernel(ImageChunk chunk, ImgInfo* info, int32_t* cu, int32_t* qt,
+__global__ void setup_kernel(ImageChunk chunk, ImgInfo* info, int32_t* cu, int32_t* qt, int32_t* i2c,
                              int32_t* pos, int n_images) {
   griddep_wait();
   griddep_launch_dependents();
@@ -29,9 +29,11 @@ __global__ void setup_kernel(ImageChunk chunk, ImgInfo* info, int32_t* cu, int32
     info[b] = in;
     cu[b] = chunk.tok_off[tid];
     qt[b] = chunk.qt_off[tid];
+    if (i2c != nullptr) i2c[b] = chunk.i2c_off[tid];
     if (b == n_images - 1) {
       cu[n_images] = chunk.tok_off[tid + 1];
       qt[n_images] = chunk.qt_off[tid + 1];
+      if (i2c != nullptr) i2c[n_images] = chunk.i2c_off[tid + 1];
     }
   }
   if (pos == nullptr) return;
@@ -109,6 +111,63 @@ __global__ void im2col_kernel(const float* __restrict__ pix, const ImgInfo* __re
         v[e] = val;
       }
       orow[k2] = pack_bf16x2(v[0], v[1]);
+    }
+  }
+}
+
+// Tiled patch gather for patch size P (14 or 16): a work item is a segment of
+// up to kI2cPatches patches of one patch row. The item's 3 x P pixel-row
+// segments are read with coalesced loads into shared memory (normalised on the
+// way), then the item's patch rows are written as consecutive bf16 pairs.
+template <int P>
+__global__ void __launch_bounds__(256) im2col_tiled_kernel(const float* __restrict__ pix,
+                                                           const ImgInfo* __restrict__ info,
+                                                           const int32_t* __restrict__ i2c, int n_images,
+                                                           int items, int kp, int normalize,
+                                                           __nv_bfloat16* __restrict__ out) {
+  constexpr int PP = P * P, SEGMAX = kI2cPatches * P;
+  __shared__ float tile[3 * P * SEGMAX];
+  griddep_wait();
+  griddep_launch_dependents();
+  for (int g = blockIdx.x; g < items; g += gridDim.x) {
+    const int b = find_block(i2c, n_images, g);
+    const ImgInfo in = info[b];
+    const int nch = (in.w + kI2cPatches - 1) / kI2cPatches;
+    const int local = g - __ldg(i2c + b);
+    const int r = local / nch, c0 = (local - r * nch) * kI2cPatches;
+    const int npat = min(kI2cPatches, in.w - c0), seg = npat * P;
+    const float* base = pix + in.pix_off;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
+    __syncthreads();  // the previous item's readers are done with the tile
+    for (int row = warp; row < 3 * P; row += nwarps) {  // one pixel-row segment per warp
+      const int ch = row / P, ky = row - ch * P;
+      const float* src = base + (static_cast<int64_t>(ch) * in.H + r * P + ky) * in.W + c0 * P;
+      const float mean = c_mean[ch], sd = c_std[ch];
+      for (int x = lane; x < seg; x += 32) {
+        float v = __ldg(src + x);
+        if (normalize) v = (v - mean) / sd;
+        tile[row * SEGMAX + x] = v;
+      }
+    }
+    __syncthreads();
+    const int half = kp / 2;
+    const int64_t t0 = in.tok_off + static_cast<int64_t>(r) * in.w + c0;
+    for (int pi = warp; pi < npat; pi += nwarps) {  // one patch row per warp
+      uint32_t* orow = reinterpret_cast<uint32_t*>(out + (t0 + pi) * kp);
+      for (int k2 = lane; k2 < half; k2 += 32) {
+        float v[2];
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int kk = 2 * k2 + e;
+          float val = 0.f;
+          if (kk < 3 * PP) {
+            const int ch = kk / PP, rem = kk - ch * PP, ky = rem / P, kx = rem - ky * P;
+            val = tile[(ch * P + ky) * SEGMAX + pi * P + kx];
+          }
+          v[e] = val;
+        }
+        orow[k2] = pack_bf16x2(v[0], v[1]);
+      }
     }
   }
 }
@@ -457,12 +516,13 @@ static int grid_for(int64_t work_items, int per_block) {
   return static_cast<int>(blocks < 1 ? 1 : (blocks > cap ? cap : blocks));
 }
 
-int launch_setup(const ImageChunk& chunk, ImgInfo* info, int32_t* cu, int32_t* qt, int32_t* pos,
+int launch_setup(const ImageChunk& chunk, ImgInfo* info, int32_t* cu, int32_t* qt, int32_t* i2c, int32_t* pos,
                  int n_images, cudaStream_t s) {
   const int64_t tokens = chunk.tok_off[chunk.count] - chunk.tok_off[0];
   const int grid = grid_for(tokens > chunk.count ? tokens : chunk.count, 256);
   launch_begin(KC_SETUP, s);
-  const cudaError_t e = launch_pdl(setup_kernel, dim3(grid), dim3(256), 0, s, chunk, info, cu, qt, pos, n_images);
+  const cudaError_t e =
+      launch_pdl(setup_kernel, dim3(grid), dim3(256), 0, s, chunk, info, cu, qt, i2c, pos, n_images);
   launch_end(KC_SETUP, s);
   return e == cudaSuccess ? VLM_OK : VLM_ERR_CUDA;
 }
@@ -475,11 +535,20 @@ int launch_rope_table(float theta, int head_dim, int max_pos, float2* tab, cudaS
   return e == cudaSuccess ? VLM_OK : VLM_ERR_CUDA;
 }
 
-int launch_im2col(const float* pix, const ImgInfo* info, const int32_t* cu, int n_images, int64_t T,
-                  int p, int kp, int normalize, __nv_bfloat16* out, cudaStream_t s) {
+int launch_im2col(const float* pix, const ImgInfo* info, const int32_t* cu, const int32_t* i2c, int i2c_items,
+                  int n_images, int64_t T, int p, int kp, int normalize, __nv_bfloat16* out, cudaStream_t s) {
   launch_begin(KC_IM2COL, s);
-  const cudaError_t e = launch_pdl(im2col_kernel, dim3(grid_for(T * 32, 256)), dim3(256), 0, s, pix, info, cu, n_images, T, p, kp,
-                                    normalize, out);
+  cudaError_t e;
+  const int tgrid = i2c_items < num_sms() * 8 ? (i2c_items > 0 ? i2c_items : 1) : num_sms() * 8;
+  if (p == 14 && i2c != nullptr)
+    e = launch_pdl(im2col_tiled_kernel<14>, dim3(tgrid), dim3(256), 0, s, pix, info, i2c, n_images, i2c_items, kp,
+                   normalize, out);
+  else if (p == 16 && i2c != nullptr)
+    e = launch_pdl(im2col_tiled_kernel<16>, dim3(tgrid), dim3(256), 0, s, pix, info, i2c, n_images, i2c_items, kp,
+                   normalize, out);
+  else
+    e = launch_pdl(im2col_kernel, dim3(grid_for(T * 32, 256)), dim3(256), 0, s, pix, info, cu, n_images, T, p, kp,
+                   normalize, out);
   launch_end(KC_IM2COL, s);
   return e == cudaSuccess ? VLM_OK : VLM_ERR_CUDA;
 }
