@@ -85,7 +85,8 @@ typedef struct {
  *   wq, wk, wv, wo bf16 [L, D, D]
  *   w_gate, w_up   bf16 [L, F, D]
  *   w_down         bf16 [L, D, F]
- *   g_attn, g_ffn  fp32 [L, D] pre-attention / pre-MLP RMSNorm gains */
+ *   g_attn, g_ffn  fp32 [L, D] pre-attention / pre-MLP RMSNorm gains
+ * With layers == 0 the per-layer pointers may be NULL. */
 typedef struct {
   const void* w_pe;
   const float* g_pre;

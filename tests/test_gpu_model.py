@@ -191,3 +191,39 @@ def test_projector_norm_after_merge_vs_oracle():
     _, ref_before = O.encode_merge_project([im.double().numpy() for im in imgs], to_oracle(tw), to_oracle(pw),
                                            _oracle_cfg(cfg))
     assert np.abs(to_np(emb) - ref_before).max() > 0.05 * np.abs(ref_before).max()
+
+
+def test_zero_layer_tower_is_patch_embed_and_ln_pre():
+    sizes = [(56, 84), (28, 28)]
+    cfg, tw, pw, imgs = _setup("mistral3", 0, sizes, seed=5)
+    tower, emb = _run_gpu(cfg, tw, pw, imgs, sizes)
+    ref_tower, ref_emb = _run_oracle(cfg, tw, pw, imgs)
+    compare(tower, ref_tower, what="ln_pre only")
+    compare(emb, ref_emb, what="projector after ln_pre only")
+
+
+def test_extreme_aspect_and_smallest_images_vs_oracle():
+    """A 28x1540 sliver (2 x 110 patches, one merged row of 55), the smallest
+    image (28x28: 4 patches, 1 merged token) and a 56x84 image in one batch."""
+    sizes = [(28, 1540), (28, 28), (56, 84)]
+    cfg, tw, pw, imgs = _setup("mistral3", 2, sizes, seed=6)
+    tower, emb = _run_gpu(cfg, tw, pw, imgs, sizes)
+    ref_tower, ref_emb = _run_oracle(cfg, tw, pw, imgs)
+    compare(tower, ref_tower, what="tower")
+    compare(emb, ref_emb, what="projector")
+
+
+@pytest.mark.parametrize("width,heads,mlp,proj_out", [(256, 4, 512, 512), (512, 8, 1536, 768)])
+def test_other_widths_vs_oracle(width, heads, mlp, proj_out):
+    """Narrower towers and projectors: other head counts, widths and GEMM tile counts."""
+    sizes = [(84, 112), (56, 56)]
+    cfg = vlm.preset("mistral3", layers=2, width=width, heads=heads, mlp=mlp, proj_out=proj_out)
+    tw = synth.tower_weights(7, 2, width, mlp, cfg.patch)
+    pw = synth.projector_weights(7, width, cfg.merge, proj_out)
+    imgs = synth.images(7, sizes)
+    tower, emb = _run_gpu(cfg, tw, pw, imgs, sizes)
+    ocfg = dict(O.MISTRAL3, layers=2, width=width, heads=heads, mlp=mlp, proj_out=proj_out)
+    ref_tower, ref_emb = O.encode_merge_project([im.double().numpy() for im in imgs], to_oracle(tw), to_oracle(pw),
+                                                ocfg)
+    compare(tower, ref_tower, what=f"tower width {width}")
+    compare(emb, ref_emb, what=f"projector {width}->{proj_out}")

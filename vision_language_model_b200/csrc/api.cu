@@ -416,9 +416,10 @@ size_t vlm_projector_packed_bytes(const vlm_config* cfg) {
 int vlm_pack_tower(const vlm_config* cfg, const vlm_tower_weights* w, void* d_packed, size_t packed_bytes,
                    void* stream) {
   VLM_TRY(check_config(cfg));
-  if (w == nullptr || d_packed == nullptr || !w->w_pe || !w->g_pre || !w->wq || !w->wk || !w->wv || !w->wo ||
-      !w->w_gate || !w->w_up || !w->w_down || !w->g_attn || !w->g_ffn)
-    return VLM_ERR_INVALID_ARG;
+  if (w == nullptr || d_packed == nullptr || !w->w_pe || !w->g_pre) return VLM_ERR_INVALID_ARG;
+  if (cfg->layers > 0 && (!w->wq || !w->wk || !w->wv || !w->wo || !w->w_gate || !w->w_up || !w->w_down ||
+                          !w->g_attn || !w->g_ffn))
+    return VLM_ERR_INVALID_ARG;  // the per-layer stacks may be empty (null) only without layers
   const TowerLayout L = tower_layout(cfg);
   if (packed_bytes < L.total) return VLM_ERR_WORKSPACE;
   cudaStream_t s = as_stream(stream);
@@ -531,9 +532,10 @@ size_t vlm_tower_fp8_packed_bytes(const vlm_config* cfg) {
 int vlm_pack_tower_fp8(const vlm_config* cfg, const vlm_tower_weights* w, const float* act_scales, void* d_packed,
                        size_t packed_bytes, void* stream) {
   VLM_TRY(check_config(cfg));
-  if (w == nullptr || d_packed == nullptr || !w->w_pe || !w->g_pre || !w->wq || !w->wk || !w->wv || !w->wo ||
-      !w->w_gate || !w->w_up || !w->w_down || !w->g_attn || !w->g_ffn)
-    return VLM_ERR_INVALID_ARG;
+  if (w == nullptr || d_packed == nullptr || !w->w_pe || !w->g_pre) return VLM_ERR_INVALID_ARG;
+  if (cfg->layers > 0 && (!w->wq || !w->wk || !w->wv || !w->wo || !w->w_gate || !w->w_up || !w->w_down ||
+                          !w->g_attn || !w->g_ffn))
+    return VLM_ERR_INVALID_ARG;  // the per-layer stacks may be empty (null) only without layers
   VLM_TRY(check_act_scales(cfg, act_scales));
   if (cfg->mlp % 256 || cfg->width % 256) return VLM_ERR_UNSUPPORTED;
   const TowerF8Layout L = tower_f8_layout(cfg);
