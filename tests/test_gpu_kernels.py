@@ -229,3 +229,28 @@ def test_bounded_wait_times_out_into_status_and_context_survives():
     qkv, q, k, v = _qkv(8, 1)
     out = vlm.attention(qkv, [0, 1], 16)
     np.testing.assert_array_equal(to_np(out), v.reshape(1, -1))
+
+
+def test_attention_last_wave_rows_single_block():
+    """16 heads x 95 query tiles = 1,520 CTAs: rows of the CTAs of the partial
+    last wave (head 15, query tiles 55..94) and rows outside it, with peaked
+    scores."""
+    T = 12100
+    qkv, q, k, v = _qkv(12, T, q_scale=2.0)
+    out = vlm.attention(qkv, [0, T], 16)
+    rng = np.random.default_rng(3)
+    rows = np.concatenate([rng.choice(np.arange(55 * 128, T), 20, replace=False), rng.choice(55 * 128, 6), [T - 1]])
+    compare(out[rows], O.attention_rows(q, k, v, [0, T], rows), what="attention last wave")
+
+
+def test_attention_many_small_blocks_last_wave():
+    """300 blocks of 131 keys (2 key tiles each, the second one almost all
+    masked): rows of the last blocks (in the last wave) and others."""
+    cu = [131 * i for i in range(301)]
+    T = cu[-1]
+    qkv, q, k, v = _qkv(13, T, q_scale=2.0)
+    out = vlm.attention(qkv, cu, 16)
+    rng = np.random.default_rng(4)
+    rows = np.concatenate([rng.choice(np.arange(236 * 131, T), 24, replace=False), rng.choice(236 * 131, 6),
+                           [T - 1, 236 * 131, 299 * 131 + 128]])
+    compare(out[rows], O.attention_rows(q, k, v, cu, rows), what="attention small blocks")
