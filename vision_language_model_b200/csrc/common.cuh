@@ -122,7 +122,7 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
   }
 }
 
-// mbar_wait for all 32 lanes of a warp with one verdict, so the warp-wide
+// mbar_wait for all 32 lanes of a warp with one shared result, so the warp-wide
 // (.sync.aligned) tcgen05 instructions that follow never diverge.
 __device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity, volatile int* abort,
                                                int32_t* status) {
