@@ -94,3 +94,31 @@ def test_side_stream_overlaps_other_work_and_matches_eager():
     assert vlm.status_sync(pipe.status) == vlm.OK
     for got, want in zip(outs, ref):
         assert torch.equal(got, want)
+
+
+def test_host_fed_steps_match_eager():
+    """Inputs from pinned host memory, copies overlapped on a copy stream:
+    the host result equals the eager single-stream result, run after run."""
+    cfg, pipe = _pipeline()
+    ids, text0 = _text_setup(cfg, pipe)
+    results = []
+    for seed in (8, 9):
+        pix_host = torch.cat([im.reshape(-1) for im in synth.images(seed, SIZES)]).pin_memory()
+        ids_host = ids.cpu().pin_memory()
+        t = text0.clone()
+        pipe(pix_host.cuda())
+        vlm.scatter(ids, pipe.embeds, t, cfg.image_token_id, status=pipe.status)
+        torch.cuda.synchronize()
+
+        def step(inputs, result):
+            emb = pipe(inputs[0])
+            vlm.scatter(inputs[1], emb, result, cfg.image_token_id, status=pipe.status)
+
+        fed = vlm.HostFedSteps(step, [pix_host.cuda(), ids], text0)
+        out_host = torch.empty(text0.shape, dtype=text0.dtype, pin_memory=True)
+        fed.run([pix_host, ids_host], out_host, 3)
+        torch.cuda.synchronize()
+        assert vlm.status_sync(pipe.status) == vlm.OK
+        assert torch.equal(out_host, t.cpu())
+        results.append(out_host.clone())
+    assert not torch.equal(results[0], results[1])

@@ -588,3 +588,56 @@ class EncoderSideStream:
         scatter(input_ids, self.pipe.embeds, text_embeds, self.pipe.cfg.image_token_id, workspace=workspace,
                 status=self.pipe.status, stream=main)
         self.consumed.record(main)
+
+
+class HostFedSteps:
+    """Steps whose inputs come from pinned host memory and whose result goes
+    back to it, with the copies overlapped with the compute: while step i runs
+    on the current stream, a copy stream brings in step i+1's inputs and then
+    takes out step i's result, ordered by events. Every device input and the
+    result buffer are double-buffered, so a copy never touches a buffer a
+    running step uses.
+
+    step_fn(inputs, result) enqueues one step on the current stream, reading
+    the device tensors `inputs` and writing the device tensor `result`.
+    """
+
+    def __init__(self, step_fn, input_templates, result_template: torch.Tensor):
+        self.step_fn = step_fn
+        dev = result_template.device
+        self.inputs = [[torch.empty_like(t) for t in input_templates] for _ in range(2)]
+        self.results = [result_template.clone(), result_template.clone()]
+        self.copy = torch.cuda.Stream(device=dev)
+        self.ev_in = [torch.cuda.Event(), torch.cuda.Event()]
+        self.ev_done = [torch.cuda.Event(), torch.cuda.Event()]
+        self.ev_out = [torch.cuda.Event(), torch.cuda.Event()]
+
+    def run(self, host_inputs, host_result: torch.Tensor, steps: int) -> None:
+        """`steps` steps, each on a fresh copy of host_inputs (pinned host
+        tensors matching the input templates); each step's result is copied
+        into host_result. Returns when everything is enqueued; the last copy is
+        ordered before any later work on the current stream."""
+        main = torch.cuda.current_stream()
+        self.copy.wait_stream(main)
+        with torch.cuda.stream(self.copy):
+            for d, h in zip(self.inputs[0], host_inputs):
+                d.copy_(h, non_blocking=True)
+            self.ev_in[0].record(self.copy)
+        for i in range(steps):
+            b, nb = i % 2, 1 - i % 2
+            main.wait_event(self.ev_in[b])
+            if i >= 2:
+                main.wait_event(self.ev_out[b])  # step i-2's result has left this buffer
+            self.step_fn(self.inputs[b], self.results[b])
+            self.ev_done[b].record(main)
+            with torch.cuda.stream(self.copy):
+                if i + 1 < steps:
+                    if i >= 1:
+                        self.copy.wait_event(self.ev_done[nb])  # step i-1 is done with these inputs
+                    for d, h in zip(self.inputs[nb], host_inputs):
+                        d.copy_(h, non_blocking=True)
+                    self.ev_in[nb].record(self.copy)
+                self.copy.wait_event(self.ev_done[b])
+                host_result.copy_(self.results[b], non_blocking=True)
+                self.ev_out[b].record(self.copy)
+        main.wait_stream(self.copy)
