@@ -609,3 +609,49 @@ def test_projector_both_norm_orders_match_torch_composition(after):
     # with merge 1 the flag changes nothing
     cfg1 = dict(cfg, merge=1)
     np.testing.assert_array_equal(O.projector(x, [(28, 1)], pw, cfg1), O.projector(x, [(28, 1)], pw, dict(cfg1, norm_after_merge=not after)))
+
+
+def test_tower_block_fp8_scales_feed_the_right_gemms():
+    """Each static scale belongs to one GEMM input: a tiny scale saturates that
+    input to +-448 s, which all but removes that GEMM's contribution. With the
+    attention-output scale tiny the block equals the exact block without its
+    O projection (Wo = 0); with the hidden-state scale tiny, without its MLP
+    (W_down = 0); with either norm-output scale tiny the matching GEMMs see
+    inputs of size 448 s and their outputs shrink the same way."""
+    t, d, f = 12, 64, 128
+    cfg = dict(O.MISTRAL3, width=d, heads=1, mlp=f)
+    rng = np.random.default_rng(21)
+    lw = {n: rng.standard_normal(sh) * 0.05 for n, sh in
+          (("wq", (d, d)), ("wk", (d, d)), ("wv", (d, d)), ("wo", (d, d)), ("w_gate", (f, d)), ("w_up", (f, d)),
+           ("w_down", (d, f)))}
+    lw["g_attn"] = np.ones(d)
+    lw["g_ffn"] = np.ones(d)
+    x = rng.standard_normal((t, d))
+    rows, cols, cu = O.positions([(3, 4)])
+    ang = O.rope_angles(rows, cols, 1e4, d)
+    lq = O.quantize_layer(lw)
+    ok = (8 / 448, 4 / 448, 8 / 448, 16 / 448)
+    tiny = 1e-9
+    no_o = O.tower_block(x, dict(lw, wo=np.zeros((d, d))), ang, cu, cfg)
+    no_mlp = O.tower_block(x, dict(lw, w_down=np.zeros((d, f))), ang, cu, cfg)
+    exact = O.tower_block(x, lw, ang, cu, cfg)
+
+    def rel(a, b):
+        return np.abs(a - b).max() / np.abs(b).max()
+
+    # attention output crushed: the O projection adds ~0, the MLP then sees x (not x + attention)
+    got = O.tower_block_fp8(x, lq, (ok[0], tiny, ok[2], ok[3]), ang, cu, cfg)
+    xo = x.copy()
+    ref = xo + (O.silu(O.rms_norm(xo, lw["g_ffn"], 1e-5) @ lw["w_gate"].T) *
+                (O.rms_norm(xo, lw["g_ffn"], 1e-5) @ lw["w_up"].T)) @ lw["w_down"].T
+    assert rel(got, ref) < 5e-2 and rel(got, exact) > rel(got, ref)
+    # hidden state crushed: the block is x + attention only
+    got = O.tower_block_fp8(x, lq, (ok[0], ok[1], ok[2], tiny), ang, cu, cfg)
+    assert rel(got, no_mlp) < 5e-2 and rel(got, exact) > rel(got, no_mlp)
+    # MLP-norm output crushed: gate and up see ~0, so the MLP adds ~0 as well
+    got = O.tower_block_fp8(x, lq, (ok[0], ok[1], tiny, ok[3]), ang, cu, cfg)
+    assert rel(got, no_mlp) < 5e-2
+    # attention-norm output crushed: q, k, v ~0, so attention (and the O projection) add ~0
+    got = O.tower_block_fp8(x, lq, (tiny, ok[1], ok[2], ok[3]), ang, cu, cfg)
+    assert rel(got, ref) < 5e-2
+    assert no_o.shape == got.shape
