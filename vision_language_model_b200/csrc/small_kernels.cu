@@ -81,6 +81,11 @@ __device__ __forceinline__ int find_block(const int32_t* cu, int n, int t) {
 // ---------------------------------------------------------------------------
 __constant__ float c_mean[3] = {0.48145466f, 0.4578275f, 0.40821073f};
 __constant__ float c_std[3] = {0.26862954f, 0.26130258f, 0.27577711f};
+// (x - mean) / std as one fused multiply-add: x * (1 / std) + (-mean / std), both rounded once from double
+__constant__ float c_inv_std[3] = {static_cast<float>(1.0 / 0.26862954), static_cast<float>(1.0 / 0.26130258),
+                                   static_cast<float>(1.0 / 0.27577711)};
+__constant__ float c_shift[3] = {static_cast<float>(-0.48145466 / 0.26862954), static_cast<float>(-0.4578275 / 0.26130258),
+                                 static_cast<float>(-0.40821073 / 0.27577711)};
 
 __global__ void im2col_kernel(const float* __restrict__ pix, const ImgInfo* __restrict__ info,
                               const int32_t* __restrict__ cu, int n_images, int64_t T, int p, int kp,
@@ -126,7 +131,7 @@ __global__ void __launch_bounds__(256) im2col_tiled_kernel(const float* __restri
                                                            int items, int kp, int normalize,
                                                            __nv_bfloat16* __restrict__ out) {
   constexpr int PP = P * P, SEGMAX = kI2cPatches * P;
-  __shared__ float tile[3 * P * SEGMAX];
+  __shared__ __align__(16) float tile[3 * P * SEGMAX];
   griddep_wait();
   griddep_launch_dependents();
   for (int g = blockIdx.x; g < items; g += gridDim.x) {
@@ -142,31 +147,24 @@ __global__ void __launch_bounds__(256) im2col_tiled_kernel(const float* __restri
     for (int row = warp; row < 3 * P; row += nwarps) {  // one pixel-row segment per warp
       const int ch = row / P, ky = row - ch * P;
       const float* src = base + (static_cast<int64_t>(ch) * in.H + r * P + ky) * in.W + c0 * P;
-      const float mean = c_mean[ch], sd = c_std[ch];
-      for (int x = lane; x < seg; x += 32) {
-        float v = __ldg(src + x);
-        if (normalize) v = (v - mean) / sd;
-        tile[row * SEGMAX + x] = v;
-      }
+      const float scale = normalize ? c_inv_std[ch] : 1.0f, shift = normalize ? c_shift[ch] : 0.0f;
+      for (int x = lane; x < seg; x += 32) tile[row * SEGMAX + x] = fmaf(__ldg(src + x), scale, shift);
     }
     __syncthreads();
+    // each output bf16 pair (kx, kx + 1) of pixel row (ch, ky) is two adjacent tile floats
+    constexpr int HALF_P = P / 2, REAL_PAIRS = 3 * PP / 2;
     const int half = kp / 2;
     const int64_t t0 = in.tok_off + static_cast<int64_t>(r) * in.w + c0;
     for (int pi = warp; pi < npat; pi += nwarps) {  // one patch row per warp
       uint32_t* orow = reinterpret_cast<uint32_t*>(out + (t0 + pi) * kp);
       for (int k2 = lane; k2 < half; k2 += 32) {
-        float v[2];
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const int kk = 2 * k2 + e;
-          float val = 0.f;
-          if (kk < 3 * PP) {
-            const int ch = kk / PP, rem = kk - ch * PP, ky = rem / P, kx = rem - ky * P;
-            val = tile[(ch * P + ky) * SEGMAX + pi * P + kx];
-          }
-          v[e] = val;
+        uint32_t w = 0u;  // the zero padding past 3 P^2
+        if (k2 < REAL_PAIRS) {
+          const int row = k2 / HALF_P, pair = k2 - row * HALF_P;
+          const float2 v = *reinterpret_cast<const float2*>(&tile[row * SEGMAX + pi * P + 2 * pair]);
+          w = pack_bf16x2(v.x, v.y);
         }
-        orow[k2] = pack_bf16x2(v[0], v[1]);
+        orow[k2] = w;
       }
     }
   }
