@@ -509,6 +509,78 @@ def tower_fp8(images, tw: dict, act_scales, cfg: dict, layers: int | None = None
 
 
 # ---------------------------------------------------------------------------
+# NVFP4 (E2M1 with E4M3 block scales) GEMM operands: the deployment on the
+# vllm.cpp issue ("Why this one is smaller than it looks", the quantisation
+# loaders bullet) loads NVFP4 weights: packed 4-bit values with a scale per
+# block. Reading: a block is 16 consecutive values of a row along K, its
+# scale is one E4M3 number, and the tensor has one fp32 global scale, so
+# x ~ q * s_block * s_global. Both GEMM operands take this format (the
+# block-scaled FP4 tensor-core product needs both in FP4): weights with
+# s_global = amax(W) / (6 * 448), activations with a static s_global per GEMM
+# input and block scales computed from the data. Every scaling step below is
+# one fp32 operation, so an implementation in fp32 reaches the same codes.
+# ---------------------------------------------------------------------------
+E2M1_MAX = 6.0
+NVFP4_BLOCK = 16
+
+
+def e2m1_round(x) -> np.ndarray:
+    """Nearest value of the E2M1 format (1 sign, 2 exponent bits with bias 1,
+    1 mantissa bit: magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6), ties to the even
+    mantissa, saturating to +-6. Binade [2^e, 2^(e+1)) has step 2^(e-1);
+    below 1 the step is the subnormal quantum 0.5."""
+    x = np.asarray(x, dtype=np.float64)
+    a = np.abs(x)
+    _, e = np.frexp(a)                       # a = f * 2^e, f in [0.5, 1)
+    e = np.clip(e - 1, 0, 2)                 # binade exponent; subnormals share binade 0's step
+    quantum = np.ldexp(1.0, (e - 1).astype(np.int64))
+    q = np.minimum(np.round(a / quantum) * quantum, E2M1_MAX)  # np.round: half to even
+    return np.where(np.isnan(x), np.nan, np.copysign(q, x))
+
+
+def nvfp4_global_scale(x) -> np.float32:
+    """Per-tensor scale that maps the tensor's largest magnitude onto the
+    largest block scale times the largest element: fp32(amax / 2688)."""
+    amax = np.float32(np.max(np.abs(np.asarray(x, dtype=np.float32))))
+    return np.float32(amax / np.float32(E2M1_MAX * E4M3_MAX))
+
+
+def quantize_nvfp4(x, s_global) -> tuple:
+    """Rows of x [R, K] (K a multiple of 16) to NVFP4 with the given fp32
+    global scale. Per block of 16: s_b = e4m3(fp32(amax_b / fp32(6 s_g)));
+    r = fp32(1 / fp32(s_b s_g)) (0 when s_b is 0); q = e2m1(fp32(x r)).
+    Returns (q float64 [R, K] on the E2M1 grid, s_b float64 [R, K/16])."""
+    x32 = np.asarray(x, dtype=np.float32)
+    r_, k_ = x32.shape
+    assert k_ % NVFP4_BLOCK == 0
+    sg = np.float32(s_global)
+    blocks = x32.reshape(r_, k_ // NVFP4_BLOCK, NVFP4_BLOCK)
+    amax = np.max(np.abs(blocks), axis=2)
+    s_b = e4m3_round((amax / np.float32(np.float32(E2M1_MAX) * sg)).astype(np.float32))
+    denom = (s_b.astype(np.float32) * sg).astype(np.float32)
+    with np.errstate(divide="ignore"):
+        recip = np.where(denom > 0, np.float32(1.0) / np.where(denom > 0, denom, np.float32(1.0)),
+                         np.float32(0.0)).astype(np.float32)
+    q = e2m1_round((blocks * recip[:, :, None]).astype(np.float32))
+    return q.reshape(r_, k_), s_b
+
+
+def dequantize_nvfp4(q, s_b, s_global) -> np.ndarray:
+    """q * s_b (each scale repeated over its 16 values) * s_g, in float64."""
+    q = np.asarray(q, dtype=np.float64)
+    return q * np.repeat(np.asarray(s_b, dtype=np.float64), NVFP4_BLOCK, axis=1) * np.float64(np.float32(s_global))
+
+
+def nvfp4_linear(q_a, s_a, g_a, q_w, s_w, g_w) -> np.ndarray:
+    """y = A W^T on NVFP4 operands: the blocked products summed exactly, then
+    the one fp32 factor fp32(g_a * g_w) for both global scales."""
+    a = np.asarray(q_a, np.float64) * np.repeat(np.asarray(s_a, np.float64), NVFP4_BLOCK, axis=1)
+    w = np.asarray(q_w, np.float64) * np.repeat(np.asarray(s_w, np.float64), NVFP4_BLOCK, axis=1)
+    alpha = np.float64(np.float32(np.float32(g_a) * np.float32(g_w)))
+    return (a @ w.T) * alpha
+
+
+# ---------------------------------------------------------------------------
 # a12..a14: patch-merging projector
 # ---------------------------------------------------------------------------
 

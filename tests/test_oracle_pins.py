@@ -655,3 +655,144 @@ def test_tower_block_fp8_scales_feed_the_right_gemms():
     got = O.tower_block_fp8(x, lq, (tiny, ok[1], ok[2], ok[3]), ang, cu, cfg)
     assert rel(got, ref) < 5e-2
     assert no_o.shape == got.shape
+
+
+# ---------------------------------------------------------------------------
+# NVFP4 (E2M1 values, E4M3 scale per 16, fp32 global scale)
+# ---------------------------------------------------------------------------
+
+def _e2m1_codes():
+    """The 16 E2M1 codes decoded from the bit layout s.ee.m (bias 1; e = 0 is subnormal: m * 0.5)."""
+    out = []
+    for code in range(16):
+        sign = -1.0 if code & 8 else 1.0
+        e, m = (code >> 1) & 3, code & 1
+        out.append((code, sign * (0.5 * m if e == 0 else (1 + m / 2.0) * 2.0 ** (e - 1))))
+    return out
+
+
+def _e2m1_brute(x):
+    """Nearest code by exhaustive search; a tie goes to the code whose mantissa bit is 0."""
+    res = np.empty(len(x))
+    codes = _e2m1_codes()
+    for i, v in enumerate(x):
+        if v > 6.0 or v < -6.0:
+            res[i] = math.copysign(6.0, v)
+            continue
+        best = min(abs(v - c) for _, c in codes)
+        cands = [(code, c) for code, c in codes if abs(v - c) == best]
+        even = [c for code, c in cands if code & 1 == 0]
+        res[i] = even[0] if even else cands[0][1]
+    return res
+
+
+def test_e2m1_grid_fixed_points_and_range():
+    vals = np.unique([c for _, c in _e2m1_codes()])
+    np.testing.assert_array_equal(vals, [-6, -4, -3, -2, -1.5, -1, -0.5, 0, 0.5, 1, 1.5, 2, 3, 4, 6])
+    np.testing.assert_array_equal(O.e2m1_round(vals), vals)
+
+
+def test_e2m1_round_matches_brute_force_and_ties_to_even():
+    rng = np.random.default_rng(41)
+    grid = np.unique([abs(c) for _, c in _e2m1_codes()])
+    mids = (grid[:-1] + grid[1:]) / 2
+    x = np.concatenate([rng.uniform(-7.5, 7.5, 20000), mids, -mids, [6.0, 6.5, 1e9, -1e9, 0.0]])
+    np.testing.assert_array_equal(O.e2m1_round(x), _e2m1_brute(x))
+    # the ties, spelled out: 0.25->0, 0.75->1, 1.25->1, 1.75->2, 2.5->2, 3.5->4, 5->4
+    np.testing.assert_array_equal(O.e2m1_round(mids), [0, 1, 1, 2, 2, 4, 4])
+    assert np.isnan(O.e2m1_round([np.nan]))[0]
+
+
+def _nvfp4_representable(rows, k, rng, s_g):
+    """Codes on the grid, a +-6 in every block, power-of-two block scales: x = q s_b s_g exactly."""
+    q = rng.choice([c for _, c in _e2m1_codes()], size=(rows, k))
+    q[:, ::16] = rng.choice([-6.0, 6.0], size=(rows, k // 16))
+    s_b = np.exp2(rng.integers(-6, 8, size=(rows, k // 16))).astype(np.float64)
+    return q * np.repeat(s_b, 16, axis=1) * s_g, q, s_b
+
+
+def test_quantize_nvfp4_exact_on_representable_input():
+    rng = np.random.default_rng(42)
+    s_g = 2.0 ** -5
+    x, q, s_b = _nvfp4_representable(6, 96, rng, s_g)
+    got_q, got_s = O.quantize_nvfp4(x, s_g)
+    np.testing.assert_array_equal(got_s, s_b)
+    np.testing.assert_array_equal(got_q, q)
+    np.testing.assert_array_equal(O.dequantize_nvfp4(got_q, got_s, s_g), x)
+
+
+def test_quantize_nvfp4_zero_block_and_error_bound():
+    rng = np.random.default_rng(43)
+    x = (rng.standard_normal((40, 128)) * np.exp2(rng.uniform(-3, 3, (40, 1)))).astype(np.float32)
+    x[5, 16:32] = 0.0
+    s_g = O.nvfp4_global_scale(x)
+    q, s_b = O.quantize_nvfp4(x, s_g)
+    assert s_b[5, 1] == 0 and np.all(q[5, 16:32] == 0) and np.all(np.isfinite(q))
+    # the block holding the tensor's largest magnitude takes the largest scale
+    r, c = np.unravel_index(np.argmax(np.abs(x)), x.shape)
+    assert s_b[r, c // 16] == 448.0
+    # every nonzero block's largest value lands on +-6
+    blocks = np.abs(x).reshape(40, 8, 16)
+    top = np.argmax(blocks, axis=2)
+    qb = np.abs(q).reshape(40, 8, 16)
+    live = s_b > 2.0 ** -6   # normal E4M3 scales (relative step 1/16)
+    assert np.all(np.take_along_axis(qb, top[:, :, None], 2)[:, :, 0][live] == 6.0)
+    # elementwise: within half an E2M1 step of x / s (s = s_b s_g), where the block scale is normal
+    s = np.repeat(s_b * np.float64(s_g), 16, axis=1)
+    y = x / np.where(s > 0, s, 1)
+    err = np.abs(O.dequantize_nvfp4(q, s_b, s_g) - x)
+    bound = s * np.maximum(0.25, np.abs(y) / 4) * (1 + 1e-6)
+    ok = np.repeat(live, 16, axis=1)
+    assert np.all(err[ok] <= bound[ok])
+
+
+def test_nvfp4_linear_exact_against_fractions():
+    """Brute force with exact rationals on a small case."""
+    from fractions import Fraction
+    rng = np.random.default_rng(44)
+    xa, qa, sa = _nvfp4_representable(3, 64, rng, 2.0 ** -4)
+    xw, qw, sw = _nvfp4_representable(4, 64, rng, 2.0 ** -7)
+    got = O.nvfp4_linear(qa, sa, 2.0 ** -4, qw, sw, 2.0 ** -7)
+    for i in range(3):
+        for j in range(4):
+            acc = sum(Fraction(qa[i, k]) * Fraction(sa[i, k // 16]) * Fraction(qw[j, k]) * Fraction(sw[j, k // 16])
+                      for k in range(64))
+            assert Fraction(got[i, j]) == acc * Fraction(2.0 ** -4) * Fraction(2.0 ** -7)
+    np.testing.assert_array_equal(got, xa @ xw.T)
+
+
+def test_planted_e2m1_round_half_up_is_caught(monkeypatch):
+    def bad(x):
+        x = np.asarray(x, dtype=np.float64)
+        a = np.abs(x)
+        _, e = np.frexp(a)
+        quantum = np.ldexp(1.0, (np.clip(e - 1, 0, 2) - 1).astype(np.int64))
+        return np.copysign(np.minimum(np.floor(a / quantum + 0.5) * quantum, 6.0), x)
+    monkeypatch.setattr(O, "e2m1_round", bad)
+    with pytest.raises(AssertionError):
+        test_e2m1_round_matches_brute_force_and_ties_to_even()
+
+
+def test_planted_nvfp4_block_of_32_is_caught(monkeypatch):
+    def bad(x, s_global):
+        x = np.asarray(x, dtype=np.float32)
+        r_, k_ = x.shape
+        # one scale per 32 values: each pair of blocks shares the larger scale
+        blocks = np.abs(x).reshape(r_, k_ // 32, 32).max(axis=2)
+        s32 = O.e4m3_round((blocks / np.float32(6 * np.float32(s_global))).astype(np.float32))
+        s_b = np.repeat(s32, 2, axis=1)
+        recip = np.where(s_b > 0, 1.0 / np.where(s_b > 0, s_b * np.float64(s_global), 1.0), 0.0)
+        return O.e2m1_round(x * np.repeat(recip, 16, axis=1)), s_b
+    monkeypatch.setattr(O, "quantize_nvfp4", bad)
+    with pytest.raises(AssertionError):
+        test_quantize_nvfp4_exact_on_representable_input()
+
+
+def test_planted_nvfp4_missing_global_scale_is_caught(monkeypatch):
+    def bad(q_a, s_a, g_a, q_w, s_w, g_w):
+        a = np.asarray(q_a) * np.repeat(s_a, 16, axis=1)
+        w = np.asarray(q_w) * np.repeat(s_w, 16, axis=1)
+        return (a @ w.T) * np.float64(g_a)  # the weights' global scale dropped
+    monkeypatch.setattr(O, "nvfp4_linear", bad)
+    with pytest.raises(AssertionError):
+        test_nvfp4_linear_exact_against_fractions()
