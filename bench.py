@@ -394,6 +394,33 @@ def gemm_shapes(args) -> None:
                               "fused_ms": fused, "fused_tflops": fl / fused / 1e9,
                               "plain_store_ms": store, "plain_store_tflops": fl / store / 1e9,
                               "library": lib, "library_ms": lib_ms, "library_tflops": fl / lib_ms / 1e9}), flush=True)
+        # NVFP4: bf16 activations quantised with a static global scale, weights with their own
+        x = torch.randn((M, K), device="cuda", generator=g).to(torch.bfloat16)
+        w = (torch.randn((N, K), device="cuda", generator=g) * 0.02).to(torch.bfloat16)
+        ga = torch.full((1,), 12.0 / 2688.0, device="cuda")
+        gw = vlm.amax_scale(w)
+        qa, sfa = vlm.quant_nvfp4(x, ga)
+        qw, sfw = vlm.quant_nvfp4(w, gw)
+        quant = timeit(lambda: vlm.quant_nvfp4(x, ga, q=qa, sf=sfa))
+        plain = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+        store = timeit(lambda: vlm.gemm_nvfp4(vlm.EPI_BF16, (qa, sfa, ga), (qw, sfw, gw), plain, status=st))
+        fused = None
+        if epi == vlm.EPI_RESID:
+            c = torch.zeros((M, N), dtype=torch.float32, device="cuda")
+            fused = timeit(lambda: vlm.gemm_nvfp4(vlm.EPI_RESID, (qa, sfa, ga), (qw, sfw, gw), c, status=st))
+        lib, lib_ms = "torch._scaled_mm (cuBLASLt, NVFP4)", None
+        try:
+            fa, fw = qa.view(torch.float4_e2m1fn_x2), qw.view(torch.float4_e2m1fn_x2)
+            sa8, sw8 = sfa.view(torch.float8_e4m3fn), sfw.view(torch.float8_e4m3fn)
+            lib_ms = timeit(lambda: torch._scaled_mm(fa, fw.t(), scale_a=sa8, scale_b=sw8, out_dtype=torch.bfloat16))
+        except Exception as e:  # the library call is a comparison only
+            lib = f"torch._scaled_mm NVFP4 unavailable: {type(e).__name__}: {str(e)[:120]}"
+        print(json.dumps({"gemm": name, "dtype": "nvfp4", "M": M, "N": N, "K": K, "epilogue": vlm.EPI_RESID
+                          if fused is not None else vlm.EPI_BF16,
+                          "fused_ms": fused, "fused_tflops": fl / fused / 1e9 if fused else None,
+                          "plain_store_ms": store, "plain_store_tflops": fl / store / 1e9,
+                          "quantise_activations_ms": quant, "library": lib, "library_ms": lib_ms,
+                          "library_tflops": fl / lib_ms / 1e9 if lib_ms else None}), flush=True)
 
 
 def side_stream_overlap(pipe, pix, ids, text, cfg, scatter_ws, dev, steps: int) -> dict:

@@ -100,6 +100,49 @@ VLM_API int vlm_rmsnorm(float* d_x, const float* d_g0, const float* d_g1, void* 
 VLM_API int vlm_rmsnorm_fp8(float* d_x, const float* d_g0, const float* d_g1, void* d_out, int64_t rows, int width,
                             float eps, float f8_scale, void* stream);
 
+/* NVFP4 operands. The vllm.cpp issue ("Mistral3ForConditionalGeneration ...",
+ * "Why this one is smaller than it looks", quantisation loaders) loads NVFP4
+ * weights: 4-bit E2M1 values with one E4M3 scale per block. Reading: a block
+ * is 16 consecutive values of a row along K and the tensor has one fp32
+ * global scale s_g, so x ~ q * s_b * s_g; both GEMM operands use this format.
+ *
+ * Codes: uint8 [rows, K/2], value k of a row in byte k/2, the low nibble for
+ * even k (E2M1 code s.ee.m, magnitudes 0, .5, 1, 1.5, 2, 3, 4, 6).
+ * Block scales: vlm_nvfp4_sf_bytes(rows, K) bytes of E4M3 codes in 512-byte
+ * atoms: rows grouped by 128, K by 64; atom (row/128) * (K/64) + k/64; inside
+ * it, row r's scale of block k/16 is byte 16 (r % 32) + 4 ((r % 128) / 32)
+ * + (k/16) % 4. This is the order in which the block-scaled tensor-core
+ * product takes its scales. Rows past `rows` in the last group have scale 0.
+ * Returns 0 for a K that is not a positive multiple of 64 or rows < 1. */
+VLM_API size_t vlm_nvfp4_sf_bytes(int64_t rows, int64_t K);
+
+/* Element types of vlm_amax_scale and vlm_quant_nvfp4 inputs. */
+enum { VLM_DTYPE_BF16 = 0, VLM_DTYPE_F32 = 1 };
+
+/* d_out[0] = fp32(max |x| / divisor) over n values of d_x (dtype VLM_DTYPE_BF16
+ * or VLM_DTYPE_F32, device memory). With divisor 2688 (= 6 * 448) this is an
+ * NVFP4 global scale: the largest block of the tensor gets scale 448. */
+VLM_API int vlm_amax_scale(const void* d_x, int dtype, int64_t n, float divisor, float* d_out, void* stream);
+
+/* x [rows, K] (bf16 or fp32 by dtype, row-major, 16-byte aligned, K % 64 == 0)
+ * to NVFP4 with the global scale *d_sg (device fp32): per block of 16,
+ * s_b = e4m3(amax / fp32(6 s_g)); r = 1 / fp32(s_b s_g) (0 when s_b = 0);
+ * q = e2m1(x r); each step one IEEE fp32 operation, both roundings to nearest
+ * even and saturating (+-448, +-6). d_q: [rows, K/2] (8-byte aligned);
+ * d_sf: vlm_nvfp4_sf_bytes(rows, K) bytes. */
+VLM_API int vlm_quant_nvfp4(const void* d_x, int dtype, int64_t rows, int64_t K, const float* d_sg, void* d_q,
+                            void* d_sf, void* stream);
+
+/* acc = A . B^T on NVFP4 operands (tcgen05.mma kind::mxf4nvf4 with block
+ * scales, fp32 accumulation in TMEM), times fp32(*d_ga * *d_gb), then
+ * `epilogue`: BF16 (d_c bf16 [M, N]) or RESID (d_c fp32 [M, N], d_c += result).
+ * A: codes [M, K/2] and scales for M rows; B: codes [N, K/2] and scales for N
+ * rows; all 16-byte aligned. Requires K % 256 == 0, N % 128 == 0, M >= 1;
+ * other epilogues or shapes return VLM_ERR_UNSUPPORTED. */
+VLM_API int vlm_gemm_nvfp4(int epilogue, const void* d_a, const void* d_a_sf, const float* d_ga, const void* d_b,
+                           const void* d_b_sf, const float* d_gb, int64_t M, int64_t N, int64_t K, void* d_c,
+                           int32_t* d_status, void* stream);
+
 /* Failure-detection self-test (no counterpart on the pages): launches one
  * thread that waits on a shared-memory mbarrier nothing arrives on, using the
  * same bounded wait as every barrier wait of the GEMM and attention kernels,

@@ -196,3 +196,36 @@ def test_fp8_argument_errors_return_before_launch(L):
         vlm.ERR_INVALID_ARG
     fp8_bytes = L.vlm_tower_fp8_packed_bytes(ctypes.byref(cfg))
     assert 0 < fp8_bytes < L.vlm_tower_packed_bytes(ctypes.byref(cfg))
+
+
+def test_nvfp4_scale_sizes_and_argument_errors_return_before_launch(L):
+    # one 512-byte atom per 128 rows x 64 values of K
+    assert L.vlm_nvfp4_sf_bytes(1, 64) == 512
+    assert L.vlm_nvfp4_sf_bytes(128, 1024) == 16 * 512
+    assert L.vlm_nvfp4_sf_bytes(129, 1024) == 32 * 512
+    assert L.vlm_nvfp4_sf_bytes(12100, 4096) == 95 * 64 * 512
+    for rows, k in ((0, 64), (5, 0), (5, 48), (-1, 64)):
+        assert L.vlm_nvfp4_sf_bytes(rows, k) == 0
+    fake = ctypes.c_void_p(256)  # never dereferenced: every case fails validation first
+    st = ctypes.c_void_p(1024)
+    # K % 256, N % 128, a null scale pointer, an unaligned operand, an unsupported epilogue
+    assert L.vlm_gemm_nvfp4(vlm.EPI_BF16, fake, fake, fake, fake, fake, fake, 256, 128, 128, fake, st,
+                            None) == vlm.ERR_UNSUPPORTED
+    assert L.vlm_gemm_nvfp4(vlm.EPI_BF16, fake, fake, fake, fake, fake, fake, 256, 192, 256, fake, st,
+                            None) == vlm.ERR_UNSUPPORTED
+    assert L.vlm_gemm_nvfp4(vlm.EPI_BF16, fake, None, fake, fake, fake, fake, 256, 128, 256, fake, st,
+                            None) == vlm.ERR_INVALID_ARG
+    assert L.vlm_gemm_nvfp4(vlm.EPI_BF16, fake, fake, fake, ctypes.c_void_p(264), fake, fake, 256, 128, 256, fake,
+                            st, None) == vlm.ERR_INVALID_ARG
+    assert L.vlm_gemm_nvfp4(vlm.EPI_SWIGLU, fake, fake, fake, fake, fake, fake, 256, 128, 256, fake, st,
+                            None) == vlm.ERR_UNSUPPORTED
+    assert L.vlm_gemm_nvfp4(vlm.EPI_BF16, fake, fake, fake, fake, fake, fake, 0, 128, 256, fake, st,
+                            None) == vlm.ERR_BAD_SHAPE
+    # quantiser: K % 64, bad dtype, null global scale, unaligned input
+    assert L.vlm_quant_nvfp4(fake, vlm.DTYPE_BF16, 4, 96, fake, fake, fake, None) == vlm.ERR_UNSUPPORTED
+    assert L.vlm_quant_nvfp4(fake, 7, 4, 128, fake, fake, fake, None) == vlm.ERR_INVALID_ARG
+    assert L.vlm_quant_nvfp4(fake, vlm.DTYPE_F32, 4, 128, None, fake, fake, None) == vlm.ERR_INVALID_ARG
+    assert L.vlm_quant_nvfp4(ctypes.c_void_p(260), vlm.DTYPE_F32, 4, 128, fake, fake, fake, None) == \
+        vlm.ERR_INVALID_ARG
+    assert L.vlm_amax_scale(fake, vlm.DTYPE_BF16, 10, 0.0, fake, None) == vlm.ERR_BAD_SHAPE
+    assert L.vlm_amax_scale(None, vlm.DTYPE_BF16, 10, 2688.0, fake, None) == vlm.ERR_INVALID_ARG

@@ -17,7 +17,8 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libvlm_b200.so")
-SOURCES = ["api.cu", "gemm_tcgen05.cu", "attention_tc.cu", "small_kernels.cu", "scatter_noalloc.cu", "frontend.cu"]
+SOURCES = ["api.cu", "gemm_tcgen05.cu", "attention_tc.cu", "small_kernels.cu", "scatter_noalloc.cu", "frontend.cu",
+           "nvfp4.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

@@ -9,6 +9,7 @@
 
 #include "../../include/vlm_kernels.h"
 #include "kernels.cuh"
+#include "nvfp4.cuh"
 
 namespace vlm {
 
@@ -850,6 +851,29 @@ int vlm_rmsnorm_fp8(float* d_x, const float* d_g0, const float* d_g1, void* d_ou
     return VLM_ERR_INVALID_ARG;
   if (rows == 0) return VLM_OK;
   return launch_rmsnorm(d_x, d_g0, d_g1, d_out, rows, width, eps, as_stream(stream), f8_scale);
+}
+
+size_t vlm_nvfp4_sf_bytes(int64_t rows, int64_t K) {
+  if (rows < 1 || K < 64 || K % 64 != 0 || rows > (1LL << 31) - 1 || K > (1LL << 31) - 1) return 0;
+  return static_cast<size_t>(nvfp4_sf_bytes(rows, K));
+}
+
+int vlm_amax_scale(const void* d_x, int dtype, int64_t n, float divisor, float* d_out, void* stream) {
+  return launch_amax_scale(d_x, dtype, n, divisor, d_out, as_stream(stream));
+}
+
+int vlm_quant_nvfp4(const void* d_x, int dtype, int64_t rows, int64_t K, const float* d_sg, void* d_q, void* d_sf,
+                    void* stream) {
+  return launch_quant_nvfp4(d_x, dtype, rows, K, d_sg, static_cast<uint8_t*>(d_q), static_cast<uint8_t*>(d_sf),
+                            as_stream(stream));
+}
+
+int vlm_gemm_nvfp4(int epilogue, const void* d_a, const void* d_a_sf, const float* d_ga, const void* d_b,
+                   const void* d_b_sf, const float* d_gb, int64_t M, int64_t N, int64_t K, void* d_c,
+                   int32_t* d_status, void* stream) {
+  return launch_gemm_nvfp4(epilogue, static_cast<const uint8_t*>(d_a), static_cast<const uint8_t*>(d_a_sf), d_ga,
+                           static_cast<const uint8_t*>(d_b), static_cast<const uint8_t*>(d_b_sf), d_gb, M, N, K,
+                           d_c, d_status, as_stream(stream));
 }
 
 int vlm_rope_table(float theta, int head_dim, int max_pos, void* d_table, void* stream) {

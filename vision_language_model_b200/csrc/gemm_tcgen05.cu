@@ -20,6 +20,7 @@
 #include <cudaTypedefs.h>
 
 #include "kernels.cuh"
+#include "nvfp4.cuh"
 
 namespace vlm {
 
@@ -42,6 +43,8 @@ struct GemmArgs {
   int32_t* status;
   const float* colscale;  // E4M3 operands: per-output-column dequantisation factor (s_a * s_w[n])
   float out_scale;        // E4M3 output (SwiGLU): values are multiplied by this before rounding
+  const float* g_a = nullptr;  // NVFP4 operands: the two global scales (device memory); the
+  const float* g_b = nullptr;  // epilogue multiplies by fp32(g_a * g_b)
 };
 
 template <int BN>
@@ -641,6 +644,271 @@ int dispatch_pair_f8(int epi, const CUtensorMap& ta, const CUtensorMap& tb, cons
   }
 }
 
+// ---------------------------------------------------------------------------
+// NVFP4 two-SM variant: E2M1 operands with E4M3 block scales
+// (tcgen05.mma.kind::mxf4nvf4.block_scale.block16; M = 256, N = 128, K = 64
+// per instruction). A stage holds 128 bytes (256 values) of every operand row
+// and the stage's four scale atoms of each operand: this CTA's 128 rows of A,
+// and all 128 columns of B (each CTA loads its own copy; no multicast). The
+// even CTA copies the atoms into tensor memory with tcgen05.cp (one
+// 32x128b.warpx4 copy per atom, into both CTAs' TMEM from each CTA's own
+// shared memory) just before the stage's MMAs. Copies and MMAs issued by one
+// thread run in order, so one scale region serves every stage. TMEM: two
+// 128-column accumulators, then 16 columns of A scales and 16 of B scales
+// (4 per K = 64 step: row r's four scales sit in lane r % 32 of every lane
+// quarter, column (r % 128) / 32).
+// ---------------------------------------------------------------------------
+struct Fp4Shape {
+  static constexpr int BN = 128;
+  static constexpr int STAGES = 6;
+  static constexpr int A_BYTES = GBM * 128;        // this CTA's 128 rows x 256 values
+  static constexpr int B_BYTES = (BN / 2) * 128;   // this CTA's 64 rows of the B tile
+  static constexpr int SF_BYTES = 4 * 512;         // four 512-byte scale atoms
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + 2 * SF_BYTES;
+  static constexpr int EPI_BYTES = kEpiWarps * kStageBufs * kStageBufBytes;
+  static constexpr int SFA_COL = 2 * BN;
+  static constexpr int SFB_COL = 2 * BN + 16;
+  static constexpr int TMEM_COLS = 512;
+  static constexpr int BAR_BYTES = 256;
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + EPI_BYTES + BAR_BYTES + 1024;
+};
+
+// Instruction descriptor of kind::mxf4nvf4: E2M1 A and B (format code 1), E4M3
+// scales (scale format 0), scale-factor ids 0, both operands K-major.
+__host__ __device__ constexpr uint32_t idesc_nvfp4(int m, int n) {
+  return (1u << 7)                                  // A format: E2M1
+         | (1u << 10)                               // B format: E2M1
+         | (static_cast<uint32_t>(n >> 3) << 17)    // N / 8
+         | (0u << 23)                               // scale format: E4M3
+         | (static_cast<uint32_t>(m >> 4) << 24);   // M / 16
+}
+
+// Descriptor of one 512-byte scale atom as a tcgen05.cp source: 32 rows of 16
+// bytes, no swizzle, 8-row groups 128 bytes apart.
+__device__ __forceinline__ uint64_t smem_desc_sf_atom(uint32_t saddr) {
+  return static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4) | (static_cast<uint64_t>(128 >> 4) << 32) |
+         (1ull << 46);  // descriptor version (sm100); layout: no swizzle
+}
+__device__ __forceinline__ void tmem_cp_atom_pair(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+__device__ __forceinline__ void umma_nvfp4_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                                uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(
+          d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+      : "memory");
+}
+
+// This warp's 32 rows of a 128 x 128 tile, scaled by alpha: bf16 stores, or an
+// fp32 bulk reduce-add into c.
+template <int EPI>
+__device__ __forceinline__ void epilogue_nvfp4(Stager& st, uint32_t tbase, int row0, int n0, float alpha) {
+  if constexpr (EPI == VLM_EPI_BF16) {
+#pragma unroll 1
+    for (int c = 0; c < Fp4Shape::BN; c += 64) {
+      uint32_t a[32], b[32], w[32];
+      tmem_ld32(tbase + c, a);
+      tmem_ld32(tbase + c + 32, b);
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        w[i] = pack_bf16x2(__uint_as_float(a[2 * i]) * alpha, __uint_as_float(a[2 * i + 1]) * alpha);
+        w[16 + i] = pack_bf16x2(__uint_as_float(b[2 * i]) * alpha, __uint_as_float(b[2 * i + 1]) * alpha);
+      }
+      uint8_t* buf = st.acquire();
+      st.write_row(buf, w);
+      st.commit(buf, n0 + c, row0);
+    }
+  } else {
+#pragma unroll 1
+    for (int c = 0; c < Fp4Shape::BN; c += 32) {
+      uint32_t a[32];
+      tmem_ld32(tbase + c, a);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) a[i] = __float_as_uint(__uint_as_float(a[i]) * alpha);
+      uint8_t* buf = st.acquire();
+      st.write_row(buf, a);
+      st.template commit<true>(buf, n0 + c, row0);
+    }
+  }
+}
+
+template <int EPI>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
+    gemm_nvfp4_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                           const __grid_constant__ CUtensorMap tmSFA, const __grid_constant__ CUtensorMap tmSFB,
+                           const __grid_constant__ CUtensorMap tmC, const GemmArgs args) {
+  using S = Fp4Shape;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = sA + S::STAGES * S::A_BYTES;
+  uint8_t* sSFA = sB + S::STAGES * S::B_BYTES;
+  uint8_t* sSFB = sSFA + S::STAGES * S::SF_BYTES;
+  uint8_t* sEpi = sSFB + S::STAGES * S::SF_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sEpi + S::EPI_BYTES);
+  uint64_t* full = bars;                     // used on the even CTA
+  uint64_t* empty = bars + S::STAGES;        // both CTAs
+  uint64_t* tfull = bars + 2 * S::STAGES;    // both CTAs
+  uint64_t* tempty = tfull + 2;              // used on the even CTA (8 warp arrivals)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
+  int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const int pair = blockIdx.x >> 1, n_pairs = gridDim.x >> 1;
+  const int total_tiles = args.m_tiles * args.n_tiles;  // 256-row x 128-column pair tiles
+  const int nk = args.K / 256;                          // a stage holds 256 values of K
+  const int katoms = args.K / 64;                       // scale atoms per 128-row group
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S::STAGES; ++s) {
+      mbar_init(smem_u32(full + s), 1);
+      mbar_init(smem_u32(empty + s), 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(smem_u32(tfull + a), 1);
+      mbar_init(smem_u32(tempty + a), 2 * kEpiWarps);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tmA);
+    prefetch_tmap(&tmB);
+    prefetch_tmap(&tmSFA);
+    prefetch_tmap(&tmSFB);
+    prefetch_tmap(&tmC);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(smem_u32(tmem_slot), S::TMEM_COLS);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();  // both CTAs' barriers are initialised before any cross-CTA signal
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  volatile int* abort_v = abort_flag;
+  griddep_wait();  // operands and c belong to the previous kernels until here
+  griddep_launch_dependents();
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int tile = pair; tile < total_tiles && ok; tile += n_pairs) {
+        const int mt = tile / args.n_tiles, nt = tile - mt * args.n_tiles;
+        const int arow = mt * 256 + static_cast<int>(rank) * GBM;
+        const int brow = nt * S::BN + static_cast<int>(rank) * (S::BN / 2);
+        const int sfa_atom = (2 * mt + static_cast<int>(rank)) * katoms;
+        const int sfb_atom = nt * katoms;
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!mbar_wait(smem_u32(empty + stage), phase ^ 1u, abort_v, args.status)) { ok = false; break; }
+          const uint32_t fb = smem_u32(full + stage) & kPeerBitMask;
+          if (rank == 0) mbar_arrive_expect_tx(smem_u32(full + stage), 2 * S::STAGE_BYTES);
+          tma_load_2d_pair(smem_u32(sA + stage * S::A_BYTES), &tmA, fb, kb * 128, arow);
+          tma_load_2d_pair(smem_u32(sB + stage * S::B_BYTES), &tmB, fb, kb * 128, brow);
+          tma_load_2d_pair(smem_u32(sSFA + stage * S::SF_BYTES), &tmSFA, fb, 0, sfa_atom + 4 * kb);
+          tma_load_2d_pair(smem_u32(sSFB + stage * S::SF_BYTES), &tmSFB, fb, 0, sfb_atom + 4 * kb);
+          if (++stage == S::STAGES) { stage = 0; phase ^= 1u; }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (rank == 0 && lane == 0) {
+      constexpr uint32_t idesc = idesc_nvfp4(2 * GBM, S::BN);
+      const uint32_t sfa_t = tmem_base + S::SFA_COL, sfb_t = tmem_base + S::SFB_COL;
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      for (int tile = pair; tile < total_tiles && ok; tile += n_pairs) {
+        if (!mbar_wait_cluster(smem_u32(tempty + acc), acc_phase ^ 1u, abort_v, args.status)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * S::BN);
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!mbar_wait(smem_u32(full + stage), phase, abort_v, args.status)) { ok = false; break; }
+          tc_fence_after();
+          const uint64_t adesc = smem_desc_sw128(smem_u32(sA + stage * S::A_BYTES));
+          const uint64_t bdesc = smem_desc_sw128(smem_u32(sB + stage * S::B_BYTES));
+          const uint32_t sfa_s = smem_u32(sSFA + stage * S::SF_BYTES), sfb_s = smem_u32(sSFB + stage * S::SF_BYTES);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            tmem_cp_atom_pair(sfa_t + 4 * k, smem_desc_sf_atom(sfa_s + 512 * k));
+            tmem_cp_atom_pair(sfb_t + 4 * k, smem_desc_sf_atom(sfb_s + 512 * k));
+          }
+#pragma unroll
+          for (int k = 0; k < 4; ++k)  // 32 bytes (64 values) of K per instruction
+            umma_nvfp4_pair(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, sfa_t + 4 * k, sfb_t + 4 * k,
+                            (kb | k) != 0 ? 1u : 0u);
+          umma_commit_pair_mc(smem_u32(empty + stage), 0x3);
+          if (++stage == S::STAGES) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        umma_commit_pair_mc(smem_u32(tfull + acc), 0x3);
+        acc ^= 1;
+        if (acc == 0) acc_phase ^= 1u;
+      }
+    }
+  } else {
+    const int q = warp & 3;  // TMEM lane quadrant this warp may access
+    Stager st{sEpi + (warp - 2) * kStageBufs * kStageBufBytes, &tmC, 0, lane};
+    const uint32_t leader_tempty = mapa_shared(smem_u32(tempty), 0);
+    const float alpha = __ldg(args.g_a) * __ldg(args.g_b);
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int tile = pair; tile < total_tiles; tile += n_pairs) {
+      const int mt = tile / args.n_tiles, nt = tile - mt * args.n_tiles;
+      if (!mbar_wait_warp(smem_u32(tfull + acc), acc_phase, abort_v, args.status)) break;
+      tc_fence_after();
+      const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * S::BN);
+      epilogue_nvfp4<EPI>(st, tbase, mt * 256 + static_cast<int>(rank) * GBM + q * 32, nt * S::BN, alpha);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(leader_tempty + static_cast<uint32_t>(acc * 8));
+      acc ^= 1;
+      if (acc == 0) acc_phase ^= 1u;
+    }
+    st.drain();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();  // neither CTA leaves while its pair may still signal or read it
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, S::TMEM_COLS);
+  }
+}
+
+template <int EPI>
+int run_gemm_nvfp4(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tsa, const CUtensorMap& tsb,
+                   const CUtensorMap& tc, const GemmArgs& args, cudaStream_t s) {
+  auto kern = gemm_nvfp4_pair_kernel<EPI>;
+  static bool attr_done[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !attr_done[dev]) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Fp4Shape::SMEM_BYTES) !=
+        cudaSuccess)
+      return VLM_ERR_CUDA;
+    attr_done[dev] = true;
+  }
+  const int tiles = args.m_tiles * args.n_tiles;
+  const int pairs = tiles < num_sms() / 2 ? tiles : num_sms() / 2;
+  launch_begin(KC_GEMM, s);
+  const cudaError_t e =
+      launch_pdl(kern, dim3(2 * pairs), dim3(192), Fp4Shape::SMEM_BYTES, s, ta, tb, tsa, tsb, tc, args);
+  launch_end(KC_GEMM, s);
+  return e == cudaSuccess ? VLM_OK : VLM_ERR_CUDA;
+}
+
 template <int BN, int EPI>
 int run_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tc, const GemmArgs& args,
              cudaStream_t s) {
@@ -809,6 +1077,63 @@ int launch_gemm(int epi, const void* a, const void* b, int64_t M, int64_t N, int
     return dispatch_pair(epi, ta, tb2, tc, args, s);
   }
   return dispatch_epi<128>(epi, ta, tb, tc, args, s);
+}
+
+namespace {
+// Scale atoms as a 2D tensor of 32-bit words: one 512-byte atom per row, four
+// atoms (one stage) per box, no swizzle.
+bool make_tmap_sf(CUtensorMap* map, const void* ptr, uint64_t atoms) {
+  auto enc = tensor_map_encoder();
+  if (enc == nullptr) return false;
+  cuuint64_t dims[2] = {128, atoms};
+  cuuint64_t strides[1] = {512};
+  cuuint32_t box[2] = {128, 4};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+}  // namespace
+
+int launch_gemm_nvfp4(int epi, const uint8_t* a, const uint8_t* a_sf, const float* g_a, const uint8_t* b,
+                      const uint8_t* b_sf, const float* g_b, int64_t M, int64_t N, int64_t K, void* c,
+                      int32_t* status, cudaStream_t s) {
+  if (a == nullptr || a_sf == nullptr || g_a == nullptr || b == nullptr || b_sf == nullptr || g_b == nullptr ||
+      c == nullptr)
+    return VLM_ERR_INVALID_ARG;
+  if (M <= 0 || N <= 0 || K <= 0 || M > (1LL << 31) - 1 || N > 65535 * 128LL || K > (1 << 20))
+    return VLM_ERR_BAD_SHAPE;
+  if (K % 256 != 0 || N % 128 != 0) return VLM_ERR_UNSUPPORTED;
+  if (epi != VLM_EPI_BF16 && epi != VLM_EPI_RESID) return VLM_ERR_UNSUPPORTED;
+  if ((reinterpret_cast<uintptr_t>(a) | reinterpret_cast<uintptr_t>(b) | reinterpret_cast<uintptr_t>(a_sf) |
+       reinterpret_cast<uintptr_t>(b_sf) | reinterpret_cast<uintptr_t>(c)) & 15)
+    return VLM_ERR_INVALID_ARG;
+  CUtensorMap ta, tb, tsa, tsb, tc;
+  if (!make_tmap_2d_u8(&ta, a, K / 2, M, K / 2, 128, GBM)) return VLM_ERR_CUDA;
+  if (!make_tmap_2d_u8(&tb, b, K / 2, N, K / 2, 128, Fp4Shape::BN / 2)) return VLM_ERR_CUDA;
+  if (!make_tmap_sf(&tsa, a_sf, static_cast<uint64_t>((M + 127) / 128 * (K / 64)))) return VLM_ERR_CUDA;
+  if (!make_tmap_sf(&tsb, b_sf, static_cast<uint64_t>(N / 128 * (K / 64)))) return VLM_ERR_CUDA;
+  const bool ok = epi == VLM_EPI_RESID ? make_tmap_2d(&tc, c, true, N, M, N * 4, 32, 32)
+                                       : make_tmap_2d(&tc, c, false, N, M, N * 2, 64, 32);
+  if (!ok) return VLM_ERR_CUDA;
+  GemmArgs args;
+  args.M = static_cast<int>(M);
+  args.N = static_cast<int>(N);
+  args.K = static_cast<int>(K);
+  args.m_tiles = static_cast<int>((M + 255) / 256);
+  args.n_tiles = static_cast<int>(N / Fp4Shape::BN);
+  args.c = c;
+  args.c_bf16 = nullptr;
+  args.pos = nullptr;
+  args.rope = nullptr;
+  args.rope_cols = 0;
+  args.status = status;
+  args.colscale = nullptr;
+  args.out_scale = 1.0f;
+  args.g_a = g_a;
+  args.g_b = g_b;
+  return epi == VLM_EPI_RESID ? run_gemm_nvfp4<VLM_EPI_RESID>(ta, tb, tsa, tsb, tc, args, s)
+                              : run_gemm_nvfp4<VLM_EPI_BF16>(ta, tb, tsa, tsb, tc, args, s);
 }
 
 }  // namespace vlm

@@ -89,6 +89,10 @@ def lib() -> ctypes.CDLL:
             "vlm_encode_fp8": (I32, [CP, P, P, I32, P, P, P, P, SZ, P, P]),
             "vlm_gemm_fp8": (I32, [I32, P, P, P, F, I64, I64, I64, P, P, P, P, I64, P, P]),
             "vlm_rmsnorm_fp8": (I32, [P, P, P, P, I64, I32, F, F, P]),
+            "vlm_nvfp4_sf_bytes": (SZ, [I64, I64]),
+            "vlm_amax_scale": (I32, [P, I32, I64, F, P, P]),
+            "vlm_quant_nvfp4": (I32, [P, I32, I64, I64, P, P, P, P]),
+            "vlm_gemm_nvfp4": (I32, [I32, P, P, P, P, P, P, I64, I64, I64, P, P, P]),
             "vlm_launch_count": (I64, []),
             "vlm_profile_enable": (I32, [I32]),
             "vlm_profile_query": (I32, [I32, ctypes.POINTER(I64), ctypes.POINTER(ctypes.c_double)]),
@@ -354,6 +358,61 @@ def rmsnorm_fp8(x: torch.Tensor, g1: torch.Tensor, f8_scale: float, g0=None, eps
         out = torch.empty((rows, width), dtype=torch.uint8, device=x.device)
     _check(lib().vlm_rmsnorm_fp8(_dev(x, "x"), _dev(g0, "g0"), _dev(g1, "g1"), _dev(out, "out"), rows, width,
                                  float(eps), float(f8_scale), _stream(stream)), "vlm_rmsnorm_fp8")
+    return out
+
+
+# ---------------------------------------------------------------------------
+# NVFP4 operands (E2M1 codes, E4M3 block scales, fp32 global scale)
+# ---------------------------------------------------------------------------
+DTYPE_BF16, DTYPE_F32 = 0, 1
+NVFP4_GLOBAL_DIVISOR = 6.0 * 448.0
+
+
+def nvfp4_sf_bytes(rows: int, k: int) -> int:
+    """Bytes of block scales for `rows` rows of K values (host only)."""
+    return int(lib().vlm_nvfp4_sf_bytes(rows, k))
+
+
+def _dtype_code(x: torch.Tensor) -> int:
+    if x.dtype == torch.bfloat16:
+        return DTYPE_BF16
+    if x.dtype == torch.float32:
+        return DTYPE_F32
+    raise TypeError(f"bf16 or fp32 expected, got {x.dtype}")
+
+
+def amax_scale(x: torch.Tensor, divisor: float = NVFP4_GLOBAL_DIVISOR, out=None, stream=None) -> torch.Tensor:
+    """Device fp32 [1] = max |x| / divisor (an NVFP4 global scale by default)."""
+    if out is None:
+        out = torch.empty(1, dtype=torch.float32, device=x.device)
+    _check(lib().vlm_amax_scale(_dev(x, "x"), _dtype_code(x), x.numel(), float(divisor), _dev(out, "out"),
+                                _stream(stream)), "vlm_amax_scale")
+    return out
+
+
+def quant_nvfp4(x: torch.Tensor, s_global: torch.Tensor, q=None, sf=None, stream=None) -> tuple:
+    """x [rows, K] (bf16 or fp32) -> (codes uint8 [rows, K/2], block scales uint8
+    [nvfp4_sf_bytes(rows, K)]) with the device global scale s_global [1]."""
+    rows, k = x.shape
+    if q is None:
+        q = torch.empty((rows, k // 2), dtype=torch.uint8, device=x.device)
+    if sf is None:
+        sf = torch.empty(max(nvfp4_sf_bytes(rows, k), 1), dtype=torch.uint8, device=x.device)
+    _check(lib().vlm_quant_nvfp4(_dev(x, "x"), _dtype_code(x), rows, k, _dev(s_global, "s_global"), _dev(q, "q"),
+                                 _dev(sf, "sf"), _stream(stream)), "vlm_quant_nvfp4")
+    return q, sf
+
+
+def gemm_nvfp4(epilogue: int, a: tuple, b: tuple, out: torch.Tensor, status=None, stream=None) -> torch.Tensor:
+    """out (bf16, or fp32 += for EPI_RESID) = fp32(g_a g_b) * A . B^T, where a and
+    b are (codes [rows, K/2], block scales, global scale [1]) triples."""
+    (qa, sfa, ga), (qb, sfb, gb) = a, b
+    M, N, K = qa.shape[0], qb.shape[0], 2 * qa.shape[1]
+    if status is None:
+        status = new_status(qa.device)
+    _check(lib().vlm_gemm_nvfp4(epilogue, _dev(qa, "a"), _dev(sfa, "a_sf"), _dev(ga, "g_a"), _dev(qb, "b"),
+                                _dev(sfb, "b_sf"), _dev(gb, "g_b"), M, N, K, _dev(out, "out"), _dev(status, "status"),
+                                _stream(stream)), "vlm_gemm_nvfp4")
     return out
 
 
