@@ -646,31 +646,47 @@ int dispatch_pair_f8(int epi, const CUtensorMap& ta, const CUtensorMap& tb, cons
 
 // ---------------------------------------------------------------------------
 // NVFP4 two-SM variant: E2M1 operands with E4M3 block scales
-// (tcgen05.mma.kind::mxf4nvf4.block_scale.block16; M = 256, N = 128, K = 64
+// (tcgen05.mma.kind::mxf4nvf4.block_scale.block16; M = 256, N = BN, K = 64
 // per instruction). A stage holds 128 bytes (256 values) of every operand row
-// and the stage's four scale atoms of each operand: this CTA's 128 rows of A,
-// and all 128 columns of B (each CTA loads its own copy; no multicast). The
-// even CTA copies the atoms into tensor memory with tcgen05.cp (one
+// and the stage's scale atoms of each operand: this CTA's 128 rows of A, and
+// all BN columns of B (each CTA loads its own copy; no multicast). The even
+// CTA copies the atoms into tensor memory with tcgen05.cp (one
 // 32x128b.warpx4 copy per atom, into both CTAs' TMEM from each CTA's own
 // shared memory) just before the stage's MMAs. Copies and MMAs issued by one
-// thread run in order, so one scale region serves every stage. TMEM: two
-// 128-column accumulators, then 16 columns of A scales and 16 of B scales
-// (4 per K = 64 step: row r's four scales sit in lane r % 32 of every lane
-// quarter, column (r % 128) / 32).
+// thread run in order, so one scale region serves every stage. Per K = 64
+// step the A scales take 4 TMEM columns (row r's four scales sit in lane
+// r % 32 of every lane quarter, column (r % 128) / 32) and the B scales 4 per
+// 128 columns of the tile.
+//
+// TMEM (512 columns): BN = 128 keeps two 128-column accumulators side by side
+// and the scales behind them. BN = 256 would need 512 columns for two
+// accumulators alone, so the second one starts at column 192 and shares 64
+// columns with the first; the scales take columns 448..511. The epilogue
+// reads the shared 64 columns of a tile first and then signals `ovl`: the next
+// tile's MMAs (into the other accumulator) wait for that signal and for the
+// other accumulator's own release, so they start while the epilogue is still
+// working through the tile's other 192 columns.
 // ---------------------------------------------------------------------------
+template <int BN_>
 struct Fp4Shape {
-  static constexpr int BN = 128;
-  static constexpr int STAGES = 6;
+  static constexpr int BN = BN_;
+  static constexpr bool kOverlap = BN == 256;
+  static constexpr int STAGES = BN == 256 ? 5 : 6;
   static constexpr int A_BYTES = GBM * 128;        // this CTA's 128 rows x 256 values
-  static constexpr int B_BYTES = (BN / 2) * 128;   // this CTA's 64 rows of the B tile
-  static constexpr int SF_BYTES = 4 * 512;         // four 512-byte scale atoms
-  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + 2 * SF_BYTES;
+  static constexpr int B_BYTES = (BN / 2) * 128;   // this CTA's half of the B tile
+  static constexpr int SFA_BYTES = 4 * 512;        // four 512-byte scale atoms
+  static constexpr int SFB_BLOCKS = BN / 128;      // 128-column groups of B scales
+  static constexpr int SFB_BYTES = SFB_BLOCKS * 4 * 512;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
   static constexpr int EPI_BYTES = kEpiWarps * kStageBufs * kStageBufBytes;
-  static constexpr int SFA_COL = 2 * BN;
-  static constexpr int SFB_COL = 2 * BN + 16;
+  static constexpr int ACC_STRIDE = kOverlap ? 192 : BN;  // TMEM column of the second accumulator
+  static constexpr int SFA_COL = kOverlap ? 448 : 2 * BN;
+  static constexpr int SFB_COL = SFA_COL + 16;
   static constexpr int TMEM_COLS = 512;
   static constexpr int BAR_BYTES = 256;
   static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + EPI_BYTES + BAR_BYTES + 1024;
+  static_assert(SFB_COL + 16 * SFB_BLOCKS <= TMEM_COLS, "scale columns past the allocation");
+  static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
 };
 
 // Instruction descriptor of kind::mxf4nvf4: E2M1 A and B (format code 1), E4M3
@@ -703,20 +719,25 @@ __device__ __forceinline__ void umma_nvfp4_pair(uint32_t d_tmem, uint64_t a_desc
       : "memory");
 }
 
-// This warp's 32 rows of a 128 x 128 tile, scaled by alpha: bf16 stores, or an
-// fp32 bulk reduce-add into c.
-template <int EPI>
-__device__ __forceinline__ void epilogue_nvfp4(Stager& st, uint32_t tbase, int row0, int n0, float alpha) {
+// This warp's 32 rows of a 128 x BN tile held at TMEM address tbase, scaled by
+// alpha: bf16 stores, or an fp32 bulk reduce-add into c. Chunks start at tile
+// column `first` and wrap around; after the chunks covering the first 64
+// columns have been read from TMEM, on_first64() runs.
+template <int EPI, int BN, typename F>
+__device__ __forceinline__ void epilogue_nvfp4(Stager& st, uint32_t tbase, int row0, int n0, int first, float alpha,
+                                               F&& on_first64) {
   if constexpr (EPI == VLM_EPI_BF16) {
 #pragma unroll 1
-    for (int c = 0; c < Fp4Shape::BN; c += 64) {
+    for (int i = 0; i < BN / 64; ++i) {
+      const int c = (first + 64 * i) % BN;
       uint32_t a[32], b[32], w[32];
       tmem_ld32(tbase + c, a);
       tmem_ld32(tbase + c + 32, b);
+      if (i == 0) on_first64();
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        w[i] = pack_bf16x2(__uint_as_float(a[2 * i]) * alpha, __uint_as_float(a[2 * i + 1]) * alpha);
-        w[16 + i] = pack_bf16x2(__uint_as_float(b[2 * i]) * alpha, __uint_as_float(b[2 * i + 1]) * alpha);
+      for (int j = 0; j < 16; ++j) {
+        w[j] = pack_bf16x2(__uint_as_float(a[2 * j]) * alpha, __uint_as_float(a[2 * j + 1]) * alpha);
+        w[16 + j] = pack_bf16x2(__uint_as_float(b[2 * j]) * alpha, __uint_as_float(b[2 * j + 1]) * alpha);
       }
       uint8_t* buf = st.acquire();
       st.write_row(buf, w);
@@ -724,11 +745,13 @@ __device__ __forceinline__ void epilogue_nvfp4(Stager& st, uint32_t tbase, int r
     }
   } else {
 #pragma unroll 1
-    for (int c = 0; c < Fp4Shape::BN; c += 32) {
+    for (int i = 0; i < BN / 32; ++i) {
+      const int c = (first + 32 * i) % BN;
       uint32_t a[32];
       tmem_ld32(tbase + c, a);
+      if (i == 1) on_first64();
 #pragma unroll
-      for (int i = 0; i < 32; ++i) a[i] = __float_as_uint(__uint_as_float(a[i]) * alpha);
+      for (int j = 0; j < 32; ++j) a[j] = __float_as_uint(__uint_as_float(a[j]) * alpha);
       uint8_t* buf = st.acquire();
       st.write_row(buf, a);
       st.template commit<true>(buf, n0 + c, row0);
@@ -736,31 +759,32 @@ __device__ __forceinline__ void epilogue_nvfp4(Stager& st, uint32_t tbase, int r
   }
 }
 
-template <int EPI>
+template <int EPI, int BN>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
     gemm_nvfp4_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                            const __grid_constant__ CUtensorMap tmSFA, const __grid_constant__ CUtensorMap tmSFB,
                            const __grid_constant__ CUtensorMap tmC, const GemmArgs args) {
-  using S = Fp4Shape;
+  using S = Fp4Shape<BN>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
   uint8_t* sB = sA + S::STAGES * S::A_BYTES;
   uint8_t* sSFA = sB + S::STAGES * S::B_BYTES;
-  uint8_t* sSFB = sSFA + S::STAGES * S::SF_BYTES;
-  uint8_t* sEpi = sSFB + S::STAGES * S::SF_BYTES;
+  uint8_t* sSFB = sSFA + S::STAGES * S::SFA_BYTES;
+  uint8_t* sEpi = sSFB + S::STAGES * S::SFB_BYTES;
   uint64_t* bars = reinterpret_cast<uint64_t*>(sEpi + S::EPI_BYTES);
   uint64_t* full = bars;                     // used on the even CTA
   uint64_t* empty = bars + S::STAGES;        // both CTAs
   uint64_t* tfull = bars + 2 * S::STAGES;    // both CTAs
   uint64_t* tempty = tfull + 2;              // used on the even CTA (8 warp arrivals)
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
+  uint64_t* ovl = tempty + 2;                // used on the even CTA (8 warp arrivals)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ovl + 1);
   int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();
   const int pair = blockIdx.x >> 1, n_pairs = gridDim.x >> 1;
-  const int total_tiles = args.m_tiles * args.n_tiles;  // 256-row x 128-column pair tiles
+  const int total_tiles = args.m_tiles * args.n_tiles;  // 256-row x BN-column pair tiles
   const int nk = args.K / 256;                          // a stage holds 256 values of K
   const int katoms = args.K / 64;                       // scale atoms per 128-row group
 
@@ -773,6 +797,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
       mbar_init(smem_u32(tfull + a), 1);
       mbar_init(smem_u32(tempty + a), 2 * kEpiWarps);
     }
+    mbar_init(smem_u32(ovl), 2 * kEpiWarps);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -806,15 +831,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
         const int arow = mt * 256 + static_cast<int>(rank) * GBM;
         const int brow = nt * S::BN + static_cast<int>(rank) * (S::BN / 2);
         const int sfa_atom = (2 * mt + static_cast<int>(rank)) * katoms;
-        const int sfb_atom = nt * katoms;
+        const int sfb_atom = nt * S::SFB_BLOCKS * katoms;
         for (int kb = 0; kb < nk; ++kb) {
           if (!mbar_wait(smem_u32(empty + stage), phase ^ 1u, abort_v, args.status)) { ok = false; break; }
           const uint32_t fb = smem_u32(full + stage) & kPeerBitMask;
           if (rank == 0) mbar_arrive_expect_tx(smem_u32(full + stage), 2 * S::STAGE_BYTES);
           tma_load_2d_pair(smem_u32(sA + stage * S::A_BYTES), &tmA, fb, kb * 128, arow);
           tma_load_2d_pair(smem_u32(sB + stage * S::B_BYTES), &tmB, fb, kb * 128, brow);
-          tma_load_2d_pair(smem_u32(sSFA + stage * S::SF_BYTES), &tmSFA, fb, 0, sfa_atom + 4 * kb);
-          tma_load_2d_pair(smem_u32(sSFB + stage * S::SF_BYTES), &tmSFB, fb, 0, sfb_atom + 4 * kb);
+          tma_load_2d_pair(smem_u32(sSFA + stage * S::SFA_BYTES), &tmSFA, fb, 0, sfa_atom + 4 * kb);
+#pragma unroll
+          for (int j = 0; j < S::SFB_BLOCKS; ++j)
+            tma_load_2d_pair(smem_u32(sSFB + stage * S::SFB_BYTES + j * 2048), &tmSFB, fb, 0,
+                             sfb_atom + j * katoms + 4 * kb);
           if (++stage == S::STAGES) { stage = 0; phase ^= 1u; }
         }
       }
@@ -826,27 +854,34 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
-      uint32_t acc_phase = 0;
+      uint32_t acc_phase = 0, ovl_phase = 0;
       bool ok = true;
       for (int tile = pair; tile < total_tiles && ok; tile += n_pairs) {
         if (!mbar_wait_cluster(smem_u32(tempty + acc), acc_phase ^ 1u, abort_v, args.status)) break;
+        if constexpr (S::kOverlap) {
+          // the previous tile's epilogue has read the 64 columns both accumulators share
+          if (!mbar_wait_cluster(smem_u32(ovl), ovl_phase ^ 1u, abort_v, args.status)) break;
+          ovl_phase ^= 1u;
+        }
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * S::BN);
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * S::ACC_STRIDE);
         for (int kb = 0; kb < nk; ++kb) {
           if (!mbar_wait(smem_u32(full + stage), phase, abort_v, args.status)) { ok = false; break; }
           tc_fence_after();
           const uint64_t adesc = smem_desc_sw128(smem_u32(sA + stage * S::A_BYTES));
           const uint64_t bdesc = smem_desc_sw128(smem_u32(sB + stage * S::B_BYTES));
-          const uint32_t sfa_s = smem_u32(sSFA + stage * S::SF_BYTES), sfb_s = smem_u32(sSFB + stage * S::SF_BYTES);
+          const uint32_t sfa_s = smem_u32(sSFA + stage * S::SFA_BYTES), sfb_s = smem_u32(sSFB + stage * S::SFB_BYTES);
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
             tmem_cp_atom_pair(sfa_t + 4 * k, smem_desc_sf_atom(sfa_s + 512 * k));
-            tmem_cp_atom_pair(sfb_t + 4 * k, smem_desc_sf_atom(sfb_s + 512 * k));
+#pragma unroll
+            for (int j = 0; j < S::SFB_BLOCKS; ++j)
+              tmem_cp_atom_pair(sfb_t + 4 * (S::SFB_BLOCKS * k + j), smem_desc_sf_atom(sfb_s + 2048 * j + 512 * k));
           }
 #pragma unroll
           for (int k = 0; k < 4; ++k)  // 32 bytes (64 values) of K per instruction
-            umma_nvfp4_pair(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, sfa_t + 4 * k, sfb_t + 4 * k,
-                            (kb | k) != 0 ? 1u : 0u);
+            umma_nvfp4_pair(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, sfa_t + 4 * k,
+                            sfb_t + 4 * S::SFB_BLOCKS * k, (kb | k) != 0 ? 1u : 0u);
           umma_commit_pair_mc(smem_u32(empty + stage), 0x3);
           if (++stage == S::STAGES) { stage = 0; phase ^= 1u; }
         }
@@ -860,6 +895,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
     const int q = warp & 3;  // TMEM lane quadrant this warp may access
     Stager st{sEpi + (warp - 2) * kStageBufs * kStageBufBytes, &tmC, 0, lane};
     const uint32_t leader_tempty = mapa_shared(smem_u32(tempty), 0);
+    const uint32_t leader_ovl = mapa_shared(smem_u32(ovl), 0);
     const float alpha = __ldg(args.g_a) * __ldg(args.g_b);
     int acc = 0;
     uint32_t acc_phase = 0;
@@ -867,8 +903,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
       const int mt = tile / args.n_tiles, nt = tile - mt * args.n_tiles;
       if (!mbar_wait_warp(smem_u32(tfull + acc), acc_phase, abort_v, args.status)) break;
       tc_fence_after();
-      const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * S::BN);
-      epilogue_nvfp4<EPI>(st, tbase, mt * 256 + static_cast<int>(rank) * GBM + q * 32, nt * S::BN, alpha);
+      const uint32_t tbase =
+          tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * S::ACC_STRIDE);
+      // the shared columns are tile columns 192..255 of the first accumulator and 0..63 of the second
+      const int first = S::kOverlap && acc == 0 ? 192 : 0;
+      epilogue_nvfp4<EPI, S::BN>(st, tbase, mt * 256 + static_cast<int>(rank) * GBM + q * 32, nt * S::BN, first,
+                                 alpha, [&] {
+                                   if constexpr (S::kOverlap) {
+                                     tc_fence_before();
+                                     __syncwarp();
+                                     if (lane == 0) mbar_arrive_cluster(leader_ovl);
+                                   }
+                                 });
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(leader_tempty + static_cast<uint32_t>(acc * 8));
@@ -887,24 +933,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
   }
 }
 
-template <int EPI>
+template <int EPI, int BN>
 int run_gemm_nvfp4(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tsa, const CUtensorMap& tsb,
                    const CUtensorMap& tc, const GemmArgs& args, cudaStream_t s) {
-  auto kern = gemm_nvfp4_pair_kernel<EPI>;
+  using S = Fp4Shape<BN>;
+  auto kern = gemm_nvfp4_pair_kernel<EPI, BN>;
   static bool attr_done[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 64 && !attr_done[dev]) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Fp4Shape::SMEM_BYTES) !=
-        cudaSuccess)
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S::SMEM_BYTES) != cudaSuccess)
       return VLM_ERR_CUDA;
     attr_done[dev] = true;
   }
   const int tiles = args.m_tiles * args.n_tiles;
   const int pairs = tiles < num_sms() / 2 ? tiles : num_sms() / 2;
   launch_begin(KC_GEMM, s);
-  const cudaError_t e =
-      launch_pdl(kern, dim3(2 * pairs), dim3(192), Fp4Shape::SMEM_BYTES, s, ta, tb, tsa, tsb, tc, args);
+  const cudaError_t e = launch_pdl(kern, dim3(2 * pairs), dim3(192), S::SMEM_BYTES, s, ta, tb, tsa, tsb, tc, args);
   launch_end(KC_GEMM, s);
   return e == cudaSuccess ? VLM_OK : VLM_ERR_CUDA;
 }
@@ -1108,9 +1153,10 @@ int launch_gemm_nvfp4(int epi, const uint8_t* a, const uint8_t* a_sf, const floa
   if ((reinterpret_cast<uintptr_t>(a) | reinterpret_cast<uintptr_t>(b) | reinterpret_cast<uintptr_t>(a_sf) |
        reinterpret_cast<uintptr_t>(b_sf) | reinterpret_cast<uintptr_t>(c)) & 15)
     return VLM_ERR_INVALID_ARG;
+  const int bn = N % 256 == 0 ? 256 : 128;
   CUtensorMap ta, tb, tsa, tsb, tc;
   if (!make_tmap_2d_u8(&ta, a, K / 2, M, K / 2, 128, GBM)) return VLM_ERR_CUDA;
-  if (!make_tmap_2d_u8(&tb, b, K / 2, N, K / 2, 128, Fp4Shape::BN / 2)) return VLM_ERR_CUDA;
+  if (!make_tmap_2d_u8(&tb, b, K / 2, N, K / 2, 128, bn / 2)) return VLM_ERR_CUDA;
   if (!make_tmap_sf(&tsa, a_sf, static_cast<uint64_t>((M + 127) / 128 * (K / 64)))) return VLM_ERR_CUDA;
   if (!make_tmap_sf(&tsb, b_sf, static_cast<uint64_t>(N / 128 * (K / 64)))) return VLM_ERR_CUDA;
   const bool ok = epi == VLM_EPI_RESID ? make_tmap_2d(&tc, c, true, N, M, N * 4, 32, 32)
@@ -1121,7 +1167,7 @@ int launch_gemm_nvfp4(int epi, const uint8_t* a, const uint8_t* a_sf, const floa
   args.N = static_cast<int>(N);
   args.K = static_cast<int>(K);
   args.m_tiles = static_cast<int>((M + 255) / 256);
-  args.n_tiles = static_cast<int>(N / Fp4Shape::BN);
+  args.n_tiles = static_cast<int>(N / bn);
   args.c = c;
   args.c_bf16 = nullptr;
   args.pos = nullptr;
@@ -1132,8 +1178,11 @@ int launch_gemm_nvfp4(int epi, const uint8_t* a, const uint8_t* a_sf, const floa
   args.out_scale = 1.0f;
   args.g_a = g_a;
   args.g_b = g_b;
-  return epi == VLM_EPI_RESID ? run_gemm_nvfp4<VLM_EPI_RESID>(ta, tb, tsa, tsb, tc, args, s)
-                              : run_gemm_nvfp4<VLM_EPI_BF16>(ta, tb, tsa, tsb, tc, args, s);
+  if (bn == 256)
+    return epi == VLM_EPI_RESID ? run_gemm_nvfp4<VLM_EPI_RESID, 256>(ta, tb, tsa, tsb, tc, args, s)
+                                : run_gemm_nvfp4<VLM_EPI_BF16, 256>(ta, tb, tsa, tsb, tc, args, s);
+  return epi == VLM_EPI_RESID ? run_gemm_nvfp4<VLM_EPI_RESID, 128>(ta, tb, tsa, tsb, tc, args, s)
+                              : run_gemm_nvfp4<VLM_EPI_BF16, 128>(ta, tb, tsa, tsb, tc, args, s);
 }
 
 }  // namespace vlm
