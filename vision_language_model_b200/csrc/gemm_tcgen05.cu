@@ -17,6 +17,11 @@
 // Two TMEM accumulators (2 x BN columns) let the epilogue of tile i overlap the
 // MMAs of tile i+1. Tiles are handed out statically (tile += gridDim.x) over a
 // grid of one CTA per SM. No TMA multicast is used.
+//
+// Variants further down: gemm_pair_kernel, the same design on two-SM pairs
+// (cta_group::2, 256-row tiles) with bf16 or E4M3 operands, and
+// gemm_nvfp4_pair_kernel, the pair design on NVFP4 operands with block scales
+// copied into TMEM.
 #include <cudaTypedefs.h>
 
 #include "kernels.cuh"
