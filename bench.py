@@ -73,9 +73,9 @@ def parse_args():
     p.add_argument("--side-stream", action="store_true",
                    help="also measure the encoder on a side stream overlapped with a decode-like GEMV loop")
     p.add_argument("--gemm-shapes", action="store_true",
-                   help="instead of a step: time the tower's GEMM shapes (12,100 rows), bf16 and E4M3, each with its "
-                        "fused epilogue and with a plain store, beside torch's cuBLAS / cuBLASLt GEMM; one JSON line "
-                        "per shape")
+                   help="instead of a step: time the tower's GEMM shapes (12,100 rows), bf16, E4M3 and NVFP4, each "
+                        "with its fused epilogue and with a plain store, beside torch's cuBLAS / cuBLASLt GEMM; one "
+                        "JSON line per shape and dtype")
     p.add_argument("--profile-steps", type=int, default=0,
                    help="for ncu: run this many plain steps after warmup and exit (no JSON)")
     return p.parse_args()
@@ -332,6 +332,21 @@ def ncu_traffic(kernel: str) -> float | None:
 KERNEL_SOURCES = {"attention": ["attention_tc.cu", "exp2_poly.cuh", "common.cuh", "kernels.cuh"],
                   "gemm": ["gemm_tcgen05.cu", "common.cuh", "kernels.cuh"],
                   "resize": ["frontend.cu", "common.cuh", "kernels.cuh"]}
+
+
+def exp_unit_line(attn_flops_per_launch: float, ms_per_launch: float, clk, sms: int) -> dict:
+    """Attention's other bound: one exponential per score (4 * 64 FLOPs per score at
+    head_dim 64), 7 of every 8 on the MUFU pipe (the kernel computes one score pair
+    in eight with an FMA-pipe polynomial), against 16 MUFU ex2 per SM per clock (the
+    pipe's issue rate on sm_100, 15.9 measured) x the SM count x the median SM clock
+    sampled during the timed region."""
+    scores = attn_flops_per_launch / (4 * 64)
+    per_s = scores / (ms_per_launch / 1000.0)
+    mhz = (clk or {}).get("sm_mhz")
+    peak = 16 * sms * mhz * 1e6 if mhz else None
+    mufu = per_s * 7 / 8
+    return {"scores_per_s": per_s, "mufu_ex2_per_s": mufu, "peak_mufu_ex2_per_s": peak,
+            "frac": mufu / peak if peak else None, "clock_mhz": mhz}
 
 
 def gemm_shapes(args) -> None:
@@ -656,6 +671,8 @@ def run_ours(args, wl):
                      "frac": achieved / peak, "peak_source": f"bf16_tflops_sustained ({peaks['source']})",
                      "traffic": ncu_traffic(kern)},
         "step_tflops": step_tflops,
+        "attention_exp_unit": exp_unit_line(fl["attn_per_launch"], ms_attn / n_attn, clk,
+                                            torch.cuda.get_device_properties(dev).multi_processor_count),
         "step_frac_of_bf16_peak": {"measured_sustained": step_tflops / peak,
                                    "measured_burst": step_tflops / peaks["bf16_tflops"],
                                    "nominal_2250": step_tflops / 2250.0},
