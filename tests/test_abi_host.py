@@ -229,3 +229,18 @@ def test_nvfp4_scale_sizes_and_argument_errors_return_before_launch(L):
         vlm.ERR_INVALID_ARG
     assert L.vlm_amax_scale(fake, vlm.DTYPE_BF16, 10, 0.0, fake, None) == vlm.ERR_BAD_SHAPE
     assert L.vlm_amax_scale(None, vlm.DTYPE_BF16, 10, 2688.0, fake, None) == vlm.ERR_INVALID_ARG
+
+
+def test_gemm_tile_counts_that_overflow_32_bits_are_rejected(L):
+    """Tile indices and scale-atom rows are 32-bit in the kernels: shapes whose
+    counts would not fit are refused on the host before any launch."""
+    fake = ctypes.c_void_p(256)
+    st = ctypes.c_void_p(1024)
+    big_m = (1 << 31) - 1
+    assert L.vlm_gemm(vlm.EPI_BF16, fake, fake, big_m, 65535 * 256, 64, fake, None, None, None, 0, st,
+                      None) == vlm.ERR_BAD_SHAPE
+    assert L.vlm_gemm_fp8(vlm.EPI_BF16, fake, fake, fake, 1.0, big_m, 65535 * 256, 128, fake, None, None, None, 0,
+                          st, None) == vlm.ERR_BAD_SHAPE
+    # NVFP4: 16.8M row groups x 16,384 scale atoms per row group
+    assert L.vlm_gemm_nvfp4(vlm.EPI_BF16, fake, fake, fake, fake, fake, fake, big_m, 128, 1 << 20, fake, st,
+                            None) == vlm.ERR_BAD_SHAPE

@@ -1043,11 +1043,17 @@ bool make_tmap_2d_u8(CUtensorMap* map, const void* ptr, uint64_t inner, uint64_t
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+namespace {
+// Tile indices (and, for NVFP4, scale-atom rows) are 32-bit in the kernels and in TMA
+// coordinates: reject shapes whose 128 x 128 tile count would not fit.
+bool tiles_fit(int64_t M, int64_t N) { return (M + 127) / 128 * ((N + 127) / 128) <= INT32_MAX; }
+}  // namespace
+
 int launch_gemm_f8(int epi, const void* a, const void* b, const float* colscale, float out_scale, int64_t M,
                    int64_t N, int64_t K, void* c, void* c_bf16, const int32_t* pos, const float2* rope,
                    int64_t rope_cols, int32_t* status, cudaStream_t s) {
   if (a == nullptr || b == nullptr || c == nullptr || colscale == nullptr) return VLM_ERR_INVALID_ARG;
-  if (M <= 0 || N <= 0 || K <= 0 || M > (1LL << 31) - 1 || N > 65535 * 256LL || K > (1 << 20))
+  if (M <= 0 || N <= 0 || K <= 0 || M > (1LL << 31) - 1 || N > 65535 * 256LL || K > (1 << 20) || !tiles_fit(M, N))
     return VLM_ERR_BAD_SHAPE;
   if (K % 128 != 0 || N % 256 != 0) return VLM_ERR_UNSUPPORTED;
   if (epi != VLM_EPI_BF16 && epi != VLM_EPI_RESID && epi != VLM_EPI_SWIGLU && epi != VLM_EPI_ROPE)
@@ -1085,7 +1091,7 @@ int launch_gemm_f8(int epi, const void* a, const void* b, const float* colscale,
 int launch_gemm(int epi, const void* a, const void* b, int64_t M, int64_t N, int64_t K, void* c, void* c_bf16,
                 const int32_t* pos, const float2* rope, int64_t rope_cols, int32_t* status, cudaStream_t s) {
   if (a == nullptr || b == nullptr || c == nullptr) return VLM_ERR_INVALID_ARG;
-  if (M <= 0 || N <= 0 || K <= 0 || M > (1LL << 31) - 1 || N > 65535 * 256LL || K > (1 << 20))
+  if (M <= 0 || N <= 0 || K <= 0 || M > (1LL << 31) - 1 || N > 65535 * 256LL || K > (1 << 20) || !tiles_fit(M, N))
     return VLM_ERR_BAD_SHAPE;
   if (K % GBK != 0 || N % 128 != 0) return VLM_ERR_UNSUPPORTED;
   const bool needs256 = epi == VLM_EPI_SWIGLU || epi == VLM_EPI_ROPE;
@@ -1151,7 +1157,8 @@ int launch_gemm_nvfp4(int epi, const uint8_t* a, const uint8_t* a_sf, const floa
   if (a == nullptr || a_sf == nullptr || g_a == nullptr || b == nullptr || b_sf == nullptr || g_b == nullptr ||
       c == nullptr)
     return VLM_ERR_INVALID_ARG;
-  if (M <= 0 || N <= 0 || K <= 0 || M > (1LL << 31) - 1 || N > 65535 * 128LL || K > (1 << 20))
+  if (M <= 0 || N <= 0 || K <= 0 || M > (1LL << 31) - 1 || N > 65535 * 128LL || K > (1 << 20) || !tiles_fit(M, N) ||
+      (M + 127) / 128 * (K / 64) > INT32_MAX || N / 128 * (K / 64) > INT32_MAX)
     return VLM_ERR_BAD_SHAPE;
   if (K % 256 != 0 || N % 128 != 0) return VLM_ERR_UNSUPPORTED;
   if (epi != VLM_EPI_BF16 && epi != VLM_EPI_RESID) return VLM_ERR_UNSUPPORTED;
