@@ -580,6 +580,48 @@ def nvfp4_linear(q_a, s_a, g_a, q_w, s_w, g_w) -> np.ndarray:
     return (a @ w.T) * alpha
 
 
+# The four tower GEMMs as they are executed: [Wq; Wk; Wv], Wo, [W_gate; W_up], W_down.
+NVFP4_GEMMS = (("qkv", ("wq", "wk", "wv")), ("o", ("wo",)), ("gate_up", ("w_gate", "w_up")), ("down", ("w_down",)))
+
+
+def quantize_layer_nvfp4(lw: dict) -> dict:
+    """NVFP4 copies of one layer's GEMM weights: one global scale per executed
+    GEMM weight (QKV and gate/up each as one tensor), block scales per 16 values
+    of a row. Entry name -> (q, s_b, s_g)."""
+    out = dict(lw)
+    for name, parts in NVFP4_GEMMS:
+        w = np.concatenate([np.asarray(lw[n], dtype=np.float32) for n in parts])
+        g = nvfp4_global_scale(w)
+        q, sb = quantize_nvfp4(w, g)
+        out[name] = (q, sb, g)
+    return out
+
+
+def _nvfp4_gemm(a, lq: dict, name: str, g_a) -> np.ndarray:
+    q_w, s_w, g_w = lq[name]
+    q_a, s_a = quantize_nvfp4(np.asarray(a, dtype=np.float32), g_a)
+    return nvfp4_linear(q_a, s_a, g_a, q_w, s_w, g_w)
+
+
+def tower_block_nvfp4(x: np.ndarray, lq: dict, act_scales, angles: np.ndarray, cu_seqlens, cfg: dict) -> np.ndarray:
+    """tower_block() with its four GEMMs on NVFP4 operands: each GEMM input is
+    rounded to fp32 and quantised with its static global scale
+    act_scales = (g_attn_norm, g_attn_out, g_ffn_norm, g_hidden), the weights
+    as quantize_layer_nvfp4 left them. Attention, norms and RoPE as in bf16."""
+    t_total = x.shape[0]
+    heads, dh, eps, d = cfg["heads"], cfg["head_dim"], cfg["eps"], cfg["width"]
+    xn = rms_norm(x, lq["g_attn"], eps)
+    qkv = _nvfp4_gemm(xn, lq, "qkv", act_scales[0])
+    q = apply_rope(qkv[:, :d].reshape(t_total, heads, dh), angles)
+    k = apply_rope(qkv[:, d:2 * d].reshape(t_total, heads, dh), angles)
+    v = qkv[:, 2 * d:].reshape(t_total, heads, dh)
+    x = x + _nvfp4_gemm(attention(q, k, v, cu_seqlens), lq, "o", act_scales[1])
+    xn = rms_norm(x, lq["g_ffn"], eps)
+    gu = _nvfp4_gemm(xn, lq, "gate_up", act_scales[2])
+    f = gu.shape[1] // 2
+    return x + _nvfp4_gemm(silu(gu[:, :f]) * gu[:, f:], lq, "down", act_scales[3])
+
+
 # ---------------------------------------------------------------------------
 # a12..a14: patch-merging projector
 # ---------------------------------------------------------------------------

@@ -796,3 +796,89 @@ def test_planted_nvfp4_missing_global_scale_is_caught(monkeypatch):
     monkeypatch.setattr(O, "nvfp4_linear", bad)
     with pytest.raises(AssertionError):
         test_nvfp4_linear_exact_against_fractions()
+
+
+def _small_layer(rng, d=64, f=128, gains_one=False):
+    lw = {n: rng.standard_normal(sh) * 0.05 for n, sh in
+          (("wq", (d, d)), ("wk", (d, d)), ("wv", (d, d)), ("wo", (d, d)), ("w_gate", (f, d)), ("w_up", (f, d)),
+           ("w_down", (d, f)))}
+    lw["g_attn"] = np.ones(d) if gains_one else 1 + 0.02 * rng.standard_normal(d)
+    lw["g_ffn"] = np.ones(d) if gains_one else 1 + 0.02 * rng.standard_normal(d)
+    return lw
+
+
+NVFP4_ACT = (8 / 2688, 4 / 2688, 8 / 2688, 16 / 2688)
+
+
+def test_quantize_layer_nvfp4_one_global_scale_per_executed_gemm():
+    rng = np.random.default_rng(71)
+    lw = _small_layer(rng)
+    lq = O.quantize_layer_nvfp4(lw)
+    qkv = np.concatenate([lw["wq"], lw["wk"], lw["wv"]]).astype(np.float32)
+    q, sb, g = lq["qkv"]
+    assert g == O.nvfp4_global_scale(qkv) and q.shape == qkv.shape and sb.shape == (192, 4)
+    # the fused tensor's largest block takes scale 448, and every value is within half an E2M1 step
+    # of its block's grid (scale s = s_b s_g per block of 16)
+    assert sb.max() == 448.0
+    s_full = np.repeat(sb * np.float64(g), 16, axis=1)
+    err = np.abs(O.dequantize_nvfp4(q, sb, g) - qkv)
+    assert np.all(err <= s_full * np.maximum(0.25, np.abs(qkv) / s_full / 4) * (1 + 1e-6))
+
+
+def test_tower_block_nvfp4_close_to_exact_block():
+    """The NVFP4 block stays within NVFP4's quantisation error of the exact block
+    and differs from it (the quantisation is really applied)."""
+    rng = np.random.default_rng(72)
+    d = 64
+    cfg = dict(O.MISTRAL3, width=d, heads=1, mlp=128)
+    lw = _small_layer(rng)
+    x = rng.standard_normal((24, d))
+    rows, cols, cu = O.positions([(4, 6)])
+    ang = O.rope_angles(rows, cols, 1e4, d)
+    exact = O.tower_block(x, lw, ang, cu, cfg)
+    fp4 = O.tower_block_nvfp4(x, O.quantize_layer_nvfp4(lw), NVFP4_ACT, ang, cu, cfg)
+    err = np.abs(fp4 - exact).max() / np.abs(exact).max()
+    assert 1e-3 < err < 0.15, err
+
+
+def test_tower_block_nvfp4_scales_feed_the_right_gemms():
+    """A tiny global scale saturates every block of that GEMM input to +-6 at
+    scale 448, i.e. +-2688 g: the input all but vanishes. With the attention-
+    output scale tiny the block equals the exact block without its O projection;
+    with the hidden-state scale tiny, without its MLP; with the attention-norm
+    scale tiny, q = k = v ~ 0 and the attention output vanishes as well; with the
+    MLP-norm scale tiny, gate and up vanish and so does the MLP."""
+    rng = np.random.default_rng(73)
+    d, f = 64, 128
+    cfg = dict(O.MISTRAL3, width=d, heads=1, mlp=f)
+    lw = _small_layer(rng, gains_one=True)
+    x = rng.standard_normal((12, d))
+    rows, cols, cu = O.positions([(3, 4)])
+    ang = O.rope_angles(rows, cols, 1e4, d)
+    lq = O.quantize_layer_nvfp4(lw)
+    no_o = O.tower_block(x, dict(lw, wo=np.zeros((d, d))), ang, cu, cfg)
+    no_mlp = O.tower_block(x, dict(lw, w_down=np.zeros((d, f))), ang, cu, cfg)
+    exact = O.tower_block(x, lw, ang, cu, cfg)
+
+    def rel(a, b):
+        return np.abs(a - b).max() / np.abs(b).max()
+
+    tiny = 1e-12
+    for i, ref in ((0, no_o), (1, no_o), (2, no_mlp), (3, no_mlp)):
+        act = list(NVFP4_ACT)
+        act[i] = tiny
+        got = O.tower_block_nvfp4(x, lq, act, ang, cu, cfg)
+        assert rel(got, ref) < 0.1, (i, rel(got, ref))
+        assert rel(got, exact) > 3 * rel(got, ref), (i, rel(got, exact), rel(got, ref))
+
+
+def test_planted_nvfp4_act_scales_swapped_is_caught(monkeypatch):
+    real = O.tower_block_nvfp4
+
+    def bad(x, lq, act, angles, cu, cfg):
+        a = list(act)
+        a[1], a[3] = a[3], a[1]   # the attention-output and hidden-state scales exchanged
+        return real(x, lq, a, angles, cu, cfg)
+    monkeypatch.setattr(O, "tower_block_nvfp4", bad)
+    with pytest.raises(AssertionError):
+        test_tower_block_nvfp4_scales_feed_the_right_gemms()
