@@ -38,9 +38,13 @@ patch before the merge; merged features in `unfold` channel-major order
 c*m*m + dy*m + dx; GELU in its erf form.
 
 Every function below is pinned by `tests/test_oracle_pins.py` against closed
-forms, library routines or brute force (no function here is "parity
-unpinned" except the end-to-end numbers of real trained weights, which do not
-exist in this environment).
+forms, library routines or brute force. The composition (`tower_block`,
+`tower`, `encode_merge_project`) is pinned by `tests/test_oracle_tower_pin.py`
+against the same steps rebuilt from torch primitives (conv2d, rms_norm, a
+complex-rotation RoPE, masked scaled_dot_product_attention, silu, unfold,
+gelu), with planted composition mistakes that must fail. Nothing here is
+"parity unpinned" except the end-to-end numbers of real trained weights,
+which do not exist in this environment.
 """
 from __future__ import annotations
 
