@@ -251,8 +251,10 @@ VLM_API int vlm_scatter(const int64_t* d_input_ids, int64_t n_tokens, int64_t im
  * other host threads on the same device) race and must be serialised by the
  * caller. Each call writes all the scratch it reads, so nothing carries over.
  * The first call on a device looks up the array's device address
- * (cudaGetSymbolAddress, with that device current) and caches it; make that
- * first call before any stream capture begins.
+ * (cudaGetSymbolAddress, with that device current) and caches it under the
+ * device and its current context; make that first call before any stream
+ * capture begins. After a device reset the first call in the new context
+ * looks the address up again (so it, too, belongs before any capture).
  * ------------------------------------------------------------------------- */
 #define VLM_SCATTER_NOALLOC_MAX_TOKENS 262144
 VLM_API int vlm_scatter_noalloc(const int64_t* d_input_ids, int64_t n_tokens, int64_t image_token_id,

@@ -116,26 +116,6 @@ def test_full_size_packed_batch_isolation():
         assert same == (b != 3), b
 
 
-def test_encode_then_scatter_end_to_end():
-    """4 sequences x 4,096 ids, one 896x1344 image each (1,536 placeholders), 2 layers."""
-    sizes = [(896, 1344)] * 4
-    cfg, tw, pw, imgs = _setup("mistral3", 2, sizes, seed=5)
-    tower, emb = _run_gpu(cfg, tw, pw, imgs, sizes)
-    ids = synth.text_sequences(5, 4, 4096, [[1536]] * 4)
-    text = synth.text_embeddings(5, 4 * 4096, 5120)
-    t_gpu = text.cuda()
-    status = vlm.new_status()
-    vlm.scatter(ids.reshape(-1).cuda(), emb, t_gpu, 10, status=status)
-    assert vlm.status_sync(status) == vlm.OK
-    mask = (ids.reshape(-1) == 10).cuda()
-    # non-image rows bit-identical, image rows are exactly the embeddings in order
-    assert torch.equal(t_gpu[~mask].cpu().view(torch.int16), text[~mask.cpu()].view(torch.int16))
-    assert torch.equal(t_gpu[mask], emb)
-    # and the embeddings themselves match the oracle on one of the four images
-    ref_tower, ref_emb = _run_oracle(cfg, tw, pw, imgs[:1])
-    compare(emb[:1536], ref_emb, what="e2e projector image 0")
-
-
 def test_many_tiny_images_cross_the_setup_chunks():
     """70 images (the per-image tables are uploaded 64 at a time) of 28x28 and
     56x28: one merged token each or two; patches 4 or 8 per image."""

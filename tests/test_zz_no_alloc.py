@@ -4,18 +4,21 @@ Serving engines that give all free device memory to their own pools, and
 plugin hosts that pass an operator only its inputs and outputs, cannot lend
 vlm_scatter a workspace. vlm_scatter_noalloc keeps that scratch in a fixed
 array inside the library instead. These tests call it through the C ABI and
-check its result against vlm_scatter's, bit for bit (the scatter is a pure
-copy), on two calls in a row: the second call is smaller than the first, so
-positions left over from the first call would show up as wrong rows.
+check its result, bit for bit (the scatter is a pure copy), against the CPU
+oracle's scatter and against vlm_scatter's, on two calls in a row: the second
+call is smaller than the first, so positions left over from the first call
+would show up as wrong rows.
 
 This file is collected last on purpose, so a run that stops at its first
 failure has already run every other test.
 """
 import ctypes
 
+import numpy as np
 import pytest
 import torch
 
+from oracle import vlm_oracle as O
 from vision_language_model_b200 import synth, vlm
 
 pytestmark = pytest.mark.gpu
@@ -54,6 +57,9 @@ def test_noalloc_matches_workspace_scatter_on_two_calls(case):
         st = vlm.new_status()
         assert _call(ids, img, got, st) == vlm.OK
         assert vlm.status_sync(st) == vlm.OK and vlm.status_sync(st_ref) == vlm.OK
+        expect = O.scatter(ids.cpu().numpy(), img.cpu().view(torch.int16).numpy(),
+                           text.cpu().view(torch.int16).numpy(), 10)
+        np.testing.assert_array_equal(got.cpu().view(torch.int16).numpy(), expect)
         assert torch.equal(got.view(torch.int16), ref.view(torch.int16))
 
 

@@ -18,9 +18,12 @@
 // it, so nothing has to be cleared between calls.
 //
 // In host code `g_scatter_scratch` names a host-side stand-in, not device
-// memory; its device address comes from cudaGetSymbolAddress, looked up once
-// per device (with that device current) by the first call made on it, and
-// cached.
+// memory; its device address comes from cudaGetSymbolAddress, looked up by the
+// first call made on a device (with that device current) and cached under the
+// device and the current context's unique ID. A device reset (or any teardown
+// and re-creation of the context) reloads the module at a new address; the new
+// context has a new ID, so the next call looks the address up again instead of
+// using the stale one.
 #include <mutex>
 
 #include "kernels.cuh"
@@ -42,20 +45,56 @@ static __device__ __align__(256) uint8_t g_scatter_scratch[kScratchBytes];
 
 constexpr int kMaxDevices = 64;
 std::mutex g_mutex;
-void* g_scratch_addr[kMaxDevices] = {};
+struct CachedAddress {
+  unsigned long long ctx_id;  // unique ID of the context the address belongs to
+  void* addr;
+};
+CachedAddress g_scratch_addr[kMaxDevices] = {};
 
-// Device address of g_scatter_scratch on the current device.
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+
+// Unique ID of the calling thread's current context (0 when there is none).
+int current_context_id(unsigned long long* id) {
+  static CtxGetCurrentFn get_current = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  if (get_current == nullptr || get_id == nullptr) {
+    void* p = nullptr;
+    void* q = nullptr;
+    cudaDriverEntryPointQueryResult r1, r2;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &r1) != cudaSuccess ||
+        r1 != cudaDriverEntryPointSuccess ||
+        cudaGetDriverEntryPoint("cuCtxGetId", &q, cudaEnableDefault, &r2) != cudaSuccess ||
+        r2 != cudaDriverEntryPointSuccess)
+      return VLM_ERR_CUDA;
+    get_current = reinterpret_cast<CtxGetCurrentFn>(p);
+    get_id = reinterpret_cast<CtxGetIdFn>(q);
+  }
+  CUcontext ctx = nullptr;
+  if (get_current(&ctx) != CUDA_SUCCESS) return VLM_ERR_CUDA;
+  *id = 0;
+  if (ctx != nullptr && get_id(ctx, id) != CUDA_SUCCESS) return VLM_ERR_CUDA;
+  return VLM_OK;
+}
+
+// Device address of g_scatter_scratch on the current device and context.
 int scratch_address(void** out) {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess) return VLM_ERR_CUDA;
   if (dev < 0 || dev >= kMaxDevices) return VLM_ERR_UNSUPPORTED;
   std::lock_guard<std::mutex> lock(g_mutex);
-  if (g_scratch_addr[dev] == nullptr) {
-    void* p = nullptr;
+  unsigned long long id = 0;
+  int rc = current_context_id(&id);
+  if (rc != VLM_OK) return rc;
+  if (id == 0 || g_scratch_addr[dev].addr == nullptr || g_scratch_addr[dev].ctx_id != id) {
+    void* p = nullptr;  // the lookup also makes the device's primary context current if none was
     if (cudaGetSymbolAddress(&p, g_scatter_scratch) != cudaSuccess || p == nullptr) return VLM_ERR_CUDA;
-    g_scratch_addr[dev] = p;
+    rc = current_context_id(&id);
+    if (rc != VLM_OK) return rc;
+    if (id == 0) return VLM_ERR_CUDA;
+    g_scratch_addr[dev] = CachedAddress{id, p};
   }
-  *out = g_scratch_addr[dev];
+  *out = g_scratch_addr[dev].addr;
   return VLM_OK;
 }
 
