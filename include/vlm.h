@@ -263,9 +263,9 @@ VLM_API int vlm_scatter_noalloc(const int64_t* d_input_ids, int64_t n_tokens, in
 
 /* ---------------------------------------------------------------------------
  * Image front end: the steps just before the path ([K] intro and
- * Mistral3ImageProcessor: images are resized so the longest edge fits
- * longest_edge = 1540 while staying on the patch grid; [P] VISION TOKENS:
- * a large image is cut into 1024x1024 tiles).
+ * Mistral3ImageProcessor: the processor scales an image down until its longer
+ * side is at most longest_edge = 1540, with both sides kept on the patch grid;
+ * [P] VISION TOKENS: a large image is cut into 1024x1024 tiles).
  *
  * vlm_resize_target (host only, launches nothing): the processor's resize
  *   size. Reading (the pages give no formula): when max(H, W) > longest_edge
@@ -273,6 +273,9 @@ VLM_API int vlm_scatter_noalloc(const int64_t* d_input_ids, int64_t n_tokens, in
  *   floored; images are never enlarged by this step; then each side is rounded
  *   up to a multiple of `grid` (patch * merge, so the 2x2 merge always finds
  *   whole blocks: 28 for [K]; the tile size 1024 for [P]'s tiling).
+ *   Both sides then stay within longest_edge, which must itself be a
+ *   multiple of grid: any other longest_edge returns VLM_ERR_BAD_SHAPE (a
+ *   side rounded up could pass it).
  *   Returns VLM_ERR_INVALID_ARG for a non-positive argument.
  *
  * vlm_preprocess: bilinear resize of decoded images onto out_hw.

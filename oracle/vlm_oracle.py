@@ -137,14 +137,18 @@ def pixels_from_u8(image_hwc: np.ndarray) -> np.ndarray:
 def resized_hw(height: int, width: int, longest_edge: int, grid: int) -> tuple:
     """Target size of the processor's resize.
 
-    "Mistral 3" intro: images are resized so the longest edge fits
-    longest_edge while staying on the patch grid. Reading: shrink (never
-    enlarge) by r = max(H, W) / longest_edge when r > 1, flooring each side,
-    then round each side up to a multiple of `grid` (patch size times the
-    merge size, so the merge always finds whole 2x2 blocks).
+    "Mistral 3" intro: the processor scales an image down until its longer
+    side is at most longest_edge and keeps both sides on the patch grid.
+    Reading: shrink (never enlarge) by r = max(H, W) / longest_edge when
+    r > 1, flooring each side, then round each side up to a multiple of
+    `grid` (patch size times the merge size, so the merge always finds whole
+    2x2 blocks). Rounding up stays within longest_edge only when longest_edge
+    is itself a multiple of grid, so any other longest_edge is rejected.
     """
     if height <= 0 or width <= 0 or longest_edge <= 0 or grid <= 0:
         raise ValueError("sizes must be positive")
+    if longest_edge % grid:
+        raise ValueError(f"longest_edge {longest_edge} is not a multiple of the grid {grid}")
     ratio = max(height, width) / longest_edge
     if ratio > 1.0:
         height, width = int(height // ratio), int(width // ratio)

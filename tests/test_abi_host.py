@@ -152,6 +152,10 @@ def test_front_end_argument_errors_return_before_launch(L):
     assert L.vlm_preprocess(fake, src, 1, src, 0, ctypes.c_void_p(260), None) == vlm.ERR_INVALID_ARG  # unaligned
     oh, ow = ctypes.c_int32(), ctypes.c_int32()
     assert L.vlm_resize_target(0, 5, 1540, 28, ctypes.byref(oh), ctypes.byref(ow)) == vlm.ERR_INVALID_ARG
+    # a longest_edge off the grid: rounding up could exceed it, so it is refused
+    assert L.vlm_resize_target(2000, 1000, 1000, 28, ctypes.byref(oh), ctypes.byref(ow)) == vlm.ERR_BAD_SHAPE
+    assert L.vlm_resize_target(2000, 1000, 1008, 28, ctypes.byref(oh), ctypes.byref(ow)) == vlm.OK
+    assert (oh.value, ow.value) == (1008, 504)
     # placeholder expansion: output too small, and more images than ids
     counts = (ctypes.c_int64 * 2)(100, 200)
     n_out = ctypes.c_int64()

@@ -415,7 +415,15 @@ def test_planted_rope_frequency_split_swap_is_caught(monkeypatch):
 def test_resized_hw_closed_form(hw, expect):
     assert O.resized_hw(*hw, 1540, 28) == expect
     h, w = O.resized_hw(*hw, 1540, 28)
-    assert h % 28 == 0 and w % 28 == 0 and max(h, w) <= 1540 + 27
+    assert h % 28 == 0 and w % 28 == 0 and max(h, w) <= 1540
+
+
+def test_resized_hw_rejects_longest_edge_off_the_grid():
+    """With longest_edge not a multiple of the grid, rounding a side up could
+    carry it past longest_edge: rejected instead."""
+    with pytest.raises(ValueError):
+        O.resized_hw(2000, 1000, 1000, 28)
+    assert O.resized_hw(2000, 1000, 1008, 28) == (1008, 504)
 
 
 @pytest.mark.parametrize("src,dst", [((13, 17), (28, 56)), ((64, 48), (28, 28)), ((5, 5), (5, 5))])

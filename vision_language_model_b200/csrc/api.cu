@@ -691,6 +691,8 @@ int vlm_resize_target(int32_t height, int32_t width, int32_t longest_edge, int32
                       int32_t* out_w) {
   if (out_h == nullptr || out_w == nullptr || height <= 0 || width <= 0 || longest_edge <= 0 || grid <= 0)
     return VLM_ERR_INVALID_ARG;
+  // rounding up to the grid must not carry a side past longest_edge
+  if (longest_edge % grid) return VLM_ERR_BAD_SHAPE;
   double h = height, w = width;
   const double ratio = static_cast<double>(std::max(height, width)) / static_cast<double>(longest_edge);
   if (ratio > 1.0) {
