@@ -59,6 +59,21 @@ WORKLOADS = {
 }
 
 
+# (patch, merge, layers) of the two presets, for describing a workload without the library
+PRESET_SHAPES = {"mistral3": (14, 2, 24), "pixtral12b": (16, 1, 24)}
+
+
+def workload_config(wl: dict, sizes, world: int) -> dict:
+    """The JSON line's `config`: the same object for both arms of the bench."""
+    p, m, layers = PRESET_SHAPES[wl["preset"]]
+    patches = sum((h // p) * (w // p) for h, w in sizes)
+    merged = sum((h // p) * (w // p) // (m * m) for h, w in sizes)
+    return {"workload": wl["desc"], "patches": patches, "merged_tokens": merged, "layers": layers,
+            "images": len(sizes), "text_tokens": wl["n_seq"] * wl["seq_len"] if not wl.get("photo") else wl["seq_len"],
+            "parallelism": f"replicas{world}",
+            "l2": "inputs larger than L2 (weights 0.88 GB + activations per step)"}
+
+
 def parse_args():
     p = argparse.ArgumentParser()
     p.add_argument("--gpus", type=int, default=1)
@@ -290,7 +305,7 @@ def run_reference(args, wl):
     per = [s.step() for _ in range(args.steps)]
     wall = time.perf_counter() - t0
     value = s.patches_per_s(float(np.mean(per)), 24)
-    cfg_out = {"workload": wl["desc"], "patches": s.T, "layers": 24}
+    cfg_out = workload_config(wl, s.sizes, world)
     line = {"metric": METRIC, "value": value, "unit": "patches/s", "n_gpus": args.gpus, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": 1000.0 * wall / max(1, args.steps), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
@@ -658,17 +673,18 @@ def run_ours(args, wl):
         kern, achieved = "attention", fl["attn_per_launch"] / (ms_attn / n_attn / 1000.0) / 1e12
     else:
         kern, achieved = "gemm", fl["gemm"] * args.steps / (ms_gemm / 1000.0) / 1e12
-    peak = peaks["bf16_tflops_sustained"]
+    # the kernel is timed inside a loop of well under a second: the burst figure is its peak
+    peak = peaks["bf16_tflops"]
     step_tflops = fl["total"] / (ms / args.steps / 1000.0) / 1e12
+    wcfg = workload_config(wl, sizes, world)
+    assert (wcfg["patches"], wcfg["merged_tokens"], wcfg["text_tokens"]) == (T, Tm, int(ids.numel()))
     line = {
         "metric": METRIC, "value": value, "unit": "patches/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "e4m3+bf16" if wl.get("fp8") else "bf16", "data": "synthetic",
-        "config": {"workload": wl["desc"], "patches": T, "merged_tokens": Tm, "layers": cfg.layers,
-                   "images": len(sizes), "text_tokens": int(ids.numel()), "parallelism": f"replicas{world}",
-                   "l2": "inputs larger than L2 (weights 0.88 GB + activations per step)"},
+        "config": wcfg,
         "roofline": {"kernel": kern, "bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                     "frac": achieved / peak, "peak_source": f"bf16_tflops_sustained ({peaks['source']})",
+                     "frac": achieved / peak, "peak_source": f"bf16_tflops, burst ({peaks['source']})",
                      "traffic": ncu_traffic(kern)},
         "step_tflops": step_tflops,
         "attention_exp_unit": exp_unit_line(fl["attn_per_launch"], ms_attn / n_attn, clk,
