@@ -11,3 +11,27 @@ if ROOT not in sys.path:
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a B200 (sm_100a) GPU and the built CUDA library")
     config.addinivalue_line("markers", "slow: takes more than a few seconds on the CPU")
+
+
+@pytest.fixture(autouse=True)
+def _guard_bands(request):
+    """For GPU tests: every buffer the binding allocates gets guard bands,
+    checked after the test (see tests/gpu_util.py)."""
+    if request.node.get_closest_marker("gpu") is None:
+        yield
+        return
+    import torch
+    if not torch.cuda.is_available():
+        yield
+        return
+    from tests import gpu_util
+    from vision_language_model_b200 import vlm
+    guard = gpu_util.Guard()
+    old = vlm.set_allocator(guard)
+    gpu_util._active_guard = guard
+    try:
+        yield
+    finally:
+        vlm.set_allocator(old)
+        gpu_util._active_guard = None
+    guard.check()

@@ -41,3 +41,59 @@ def to_oracle(w: dict) -> dict:
 
 def pixels_to_device(images) -> torch.Tensor:
     return torch.cat([im.reshape(-1) for im in images]).to("cuda").contiguous()
+
+
+# ---------------------------------------------------------------------------
+# Guard bands: every device buffer the binding allocates during a GPU test (and
+# every buffer a test makes with `guarded` / `guarded_copy`) sits between two
+# 4 KiB bands of a known byte; after the test the bands must be unchanged, so
+# a kernel that writes past either end of a buffer fails the test.
+# ---------------------------------------------------------------------------
+GUARD_BYTES = 4096
+GUARD_FILL = 0xA5
+
+
+class Guard:
+    def __init__(self):
+        self.bufs = []
+
+    def __call__(self, shape, dtype, device):
+        shape = (shape,) if isinstance(shape, int) else tuple(shape)
+        n = 1
+        for d in shape:
+            n *= int(d)
+        nbytes = n * torch.empty((), dtype=dtype).element_size()
+        buf = torch.full((2 * GUARD_BYTES + nbytes,), GUARD_FILL, dtype=torch.uint8, device=device)
+        self.bufs.append(buf)
+        return buf[GUARD_BYTES:GUARD_BYTES + nbytes].view(dtype).view(shape)
+
+    def check(self):
+        torch.cuda.synchronize()
+        bad = []
+        for i, buf in enumerate(self.bufs):
+            for name, band in (("before", buf[:GUARD_BYTES]), ("after", buf[buf.numel() - GUARD_BYTES:])):
+                if not bool((band == GUARD_FILL).all()):
+                    bad.append(f"buffer {i} ({buf.numel() - 2 * GUARD_BYTES} bytes): guard band {name} overwritten")
+        self.bufs.clear()
+        assert not bad, "; ".join(bad)
+
+
+_active_guard = None
+
+
+def guarded(shape, dtype, device="cuda") -> torch.Tensor:
+    """An uninitialised device tensor inside guard bands (a plain tensor when no guard is active)."""
+    if _active_guard is None:
+        return torch.empty(shape, dtype=dtype, device=device)
+    return _active_guard(shape, dtype, device)
+
+
+def guarded_copy(t: torch.Tensor) -> torch.Tensor:
+    """A device copy of t inside guard bands."""
+    out = guarded(tuple(t.shape), t.dtype)
+    out.copy_(t)
+    return out
+
+
+def guarded_zeros(shape, dtype, device="cuda") -> torch.Tensor:
+    return guarded(shape, dtype, device).zero_()

@@ -11,7 +11,7 @@ import pytest
 import torch
 
 from oracle import vlm_oracle as O
-from tests.gpu_util import compare, pixels_to_device, to_np, to_oracle, tower_to_device
+from tests.gpu_util import compare, pixels_to_device, to_np, to_oracle, tower_to_device, guarded
 from vision_language_model_b200 import synth, vlm
 
 pytestmark = pytest.mark.gpu
@@ -80,7 +80,7 @@ def test_gemm_fp8_bf16_and_resid_epilogues(M, N, K):
     a, b = codes[:M], codes[M:]
     cs = (RNG.uniform(0.5, 2.0, N) * 1e-3).astype(np.float32)
     ref = (a @ b.T) * cs.astype(np.float64)[None, :]
-    out = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    out = guarded((M, N), dtype=torch.bfloat16)
     csd = torch.from_numpy(cs).cuda()
     vlm.gemm_fp8(vlm.EPI_BF16, _e4m3_tensor(a), _e4m3_tensor(b), csd, out)
     torch.cuda.synchronize()
@@ -102,7 +102,7 @@ def test_gemm_fp8_swiglu_e4m3_output():
     gate = np.concatenate([acc[:, 32 * j:32 * j + 16] for j in range(N // 32)], axis=1)
     up = np.concatenate([acc[:, 32 * j + 16:32 * j + 32] for j in range(N // 32)], axis=1)
     ref = O.e4m3_round(np.float32(O.silu(gate) * up) * np.float32(out_scale))
-    out = torch.empty((M, N // 2), dtype=torch.uint8, device="cuda")
+    out = guarded((M, N // 2), dtype=torch.uint8)
     vlm.gemm_fp8(vlm.EPI_SWIGLU, _e4m3_tensor(a), _e4m3_tensor(b), torch.from_numpy(cs).cuda(), out,
                  out_scale=out_scale)
     torch.cuda.synchronize()

@@ -12,7 +12,7 @@ import pytest
 import torch
 
 from oracle import vlm_oracle as O
-from tests.gpu_util import compare, to_np, to_oracle, tower_to_device
+from tests.gpu_util import compare, to_np, to_oracle, tower_to_device, guarded_copy
 from vision_language_model_b200 import synth, vlm
 
 pytestmark = pytest.mark.gpu
@@ -170,7 +170,7 @@ def test_expand_then_scatter_equals_oracle():
     ids = _ids_with_markers(rng, 50, 2)
     exp = vlm.expand_placeholders(torch.from_numpy(ids).cuda(), MARKER, counts)
     n = exp.numel()
-    text = synth.text_embeddings(11, n, 256).cuda()
+    text = guarded_copy(synth.text_embeddings(11, n, 256))
     img = synth.text_embeddings(12, sum(counts), 256).cuda()
     ref = O.scatter(O.expand_placeholders(ids, MARKER, counts, 10), to_np(img), to_np(text), 10)
     vlm.scatter(exp, img, text, image_token_id=10)

@@ -24,7 +24,7 @@ import pytest
 import torch
 
 from oracle import vlm_oracle as O
-from tests.gpu_util import compare, pixels_to_device, to_oracle
+from tests.gpu_util import compare, pixels_to_device, to_oracle, guarded_copy
 from tests.test_gpu_model import _oracle_cfg, _run_gpu, _run_oracle, _setup
 from vision_language_model_b200 import synth, vlm
 
@@ -73,7 +73,7 @@ def test_encode_scatter_four_sequences_every_row_vs_oracle():
     compare(emb, ref_emb, what="e2e projector, 4 images")
     ids = synth.text_sequences(5, 4, 4096, [[1536]] * 4).reshape(-1)
     text = synth.text_embeddings(5, ids.numel(), 5120)
-    t_gpu = text.cuda()
+    t_gpu = guarded_copy(text)
     status = vlm.new_status()
     vlm.scatter(ids.cuda(), emb, t_gpu, 10, status=status)
     assert vlm.status_sync(status) == vlm.OK

@@ -10,7 +10,7 @@ import pytest
 import torch
 
 from oracle import vlm_oracle as O
-from tests.gpu_util import compare, to_np
+from tests.gpu_util import compare, to_np, guarded, guarded_copy
 from vision_language_model_b200 import synth, vlm
 
 pytestmark = pytest.mark.gpu
@@ -29,7 +29,7 @@ def _randn(seed, name, shape, std=1.0):
 def test_gemm_bf16_store(M, N, K):
     a = _randn(1, "a", (M, K))
     b = _randn(1, "b", (N, K), 0.05)
-    c = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    c = guarded((M, N), dtype=torch.bfloat16)
     vlm.gemm(vlm.EPI_BF16, a, b, c)
     ref = to_np(a) @ to_np(b).T
     compare(c, ref, max_rel=1e-2, min_cos=0.9999, what="gemm bf16")
@@ -39,13 +39,13 @@ def test_gemm_bf16_store(M, N, K):
 def test_gemm_f32_and_resid(M, N, K):
     a = _randn(2, "a", (M, K))
     b = _randn(2, "b", (N, K), 0.05)
-    c = torch.empty((M, N), dtype=torch.float32, device="cuda")
+    c = guarded((M, N), dtype=torch.float32)
     vlm.gemm(vlm.EPI_F32, a, b, c)
     ref = to_np(a) @ to_np(b).T
     compare(c, ref, max_rel=1e-5, min_cos=0.999999, what="gemm f32")
     base = torch.randn((M, N), generator=synth.generator(2, "resid"), dtype=torch.float32).cuda()
     c2 = base.clone()
-    cb = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    cb = guarded((M, N), dtype=torch.bfloat16)
     vlm.gemm(vlm.EPI_RESID, a, b, c2, out_bf16=cb)
     ref2 = to_np(base) + ref
     compare(c2, ref2, max_rel=1e-5, min_cos=0.999999, what="gemm resid")
@@ -64,7 +64,7 @@ def test_gemm_swiglu(M, F, K):
     a = _randn(3, "a", (M, K))
     wg = _randn(3, "wg", (F, K), 0.05)
     wu = _randn(3, "wu", (F, K), 0.05)
-    c = torch.empty((M, F), dtype=torch.bfloat16, device="cuda")
+    c = guarded((M, F), dtype=torch.bfloat16)
     vlm.gemm(vlm.EPI_SWIGLU, a, _interleave(wg, wu), c)
     an = to_np(a)
     ref = O.silu(an @ to_np(wg).T) * (an @ to_np(wu).T)
@@ -74,7 +74,7 @@ def test_gemm_swiglu(M, F, K):
 def test_gemm_gelu():
     a = _randn(4, "a", (700, 512))
     b = _randn(4, "b", (1280, 512), 0.08)
-    c = torch.empty((700, 1280), dtype=torch.bfloat16, device="cuda")
+    c = guarded((700, 1280), dtype=torch.bfloat16)
     vlm.gemm(vlm.EPI_GELU, a, b, c)
     compare(c, O.gelu(to_np(a) @ to_np(b).T), what="gemm gelu")
 
@@ -88,7 +88,7 @@ def test_gemm_qkv_rope(h, w):
     rows, cols, _ = O.positions([(h, w)])
     pos = torch.from_numpy((rows << 16 | cols).astype(np.int32)).cuda()
     tab = vlm.rope_table(1e4, 64, max(h, w))
-    c = torch.empty((M, 3 * D), dtype=torch.bfloat16, device="cuda")
+    c = guarded((M, 3 * D), dtype=torch.bfloat16)
     vlm.gemm(vlm.EPI_ROPE, a, b, c, pos=pos, rope_table=tab, rope_cols=2 * D)
     acc = to_np(a) @ to_np(b).T
     ang = O.rope_angles(rows, cols, 1e4, 64)
@@ -112,7 +112,7 @@ def test_gemm_full_size_sampled():
     M, N, K = 12100, 3072, 1024
     a = _randn(6, "a", (M, K))
     b = _randn(6, "b", (N, K), 0.05)
-    c = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    c = guarded((M, N), dtype=torch.bfloat16)
     vlm.gemm(vlm.EPI_BF16, a, b, c)
     rows = np.random.default_rng(0).choice(M, 64, replace=False)
     rows = np.concatenate([rows, [0, 127, 128, M - 1]])
@@ -176,11 +176,11 @@ def test_rmsnorm(rows):
     x = torch.randn((rows, 1024), generator=synth.generator(11, "x"), dtype=torch.float32) * 3
     g0 = synth.gain(11, "g0", (1024,))
     g1 = synth.gain(11, "g1", (1024,))
-    xd = x.cuda()
+    xd = guarded_copy(x)
     out = vlm.rmsnorm(xd, g1.cuda())
     compare(out, O.rms_norm(x.double().numpy(), g1.double().numpy(), 1e-5), max_rel=8e-3, min_cos=0.9999,
             what="rmsnorm")
-    xd2 = x.cuda()
+    xd2 = guarded_copy(x)
     out2 = vlm.rmsnorm(xd2, g1.cuda(), g0=g0.cuda())
     y = O.rms_norm(x.double().numpy(), g0.double().numpy(), 1e-5)
     compare(xd2, y, max_rel=1e-5, min_cos=0.999999, what="rmsnorm in-place")
@@ -191,26 +191,31 @@ def test_rmsnorm(rows):
 # Scatter (bit-exact)
 # ---------------------------------------------------------------------------
 
-@pytest.mark.parametrize("n_seq,seq_len,runs,width", [(4, 4096, [[1536]] * 4, 5120), (1, 300, [[3, 50, 7]], 64),
-                                                       (2, 1, [[1], []], 16), (3, 257, [[0], [256], [1]], 128)])
+@pytest.mark.parametrize("n_seq,seq_len,runs,width", [
+    (4, 4096, [[1536]] * 4, 5120), (1, 300, [[3, 50, 7]], 64), (2, 1, [[1], []], 16), (3, 257, [[0], [256], [1]], 128),
+    (8, 4096, [[1536]] * 8, 256),                 # 32,768 ids: the largest single-launch scatter
+    (2, 20000, [[5000, 3000], [7000]], 64),       # 40,000 ids: the multi-kernel path
+])
 def test_scatter_bit_exact(n_seq, seq_len, runs, width):
     ids = synth.text_sequences(12, n_seq, seq_len, runs)
     n_img = int((ids == 10).sum())
     img = synth.randn_bf16(12, "img", (n_img, width), 1.0)
     text = synth.text_embeddings(12, n_seq * seq_len, width)
     ref = O.scatter(ids.numpy(), img.view(torch.int16).numpy(), text.view(torch.int16).numpy(), 10)
-    t_gpu = text.cuda()
+    t_gpu = guarded_copy(text)
     status = vlm.new_status()
     vlm.scatter(ids.reshape(-1).cuda(), img.cuda(), t_gpu, 10, status=status)
     assert vlm.status_sync(status) == vlm.OK
     assert np.array_equal(t_gpu.view(torch.int16).cpu().numpy(), ref)
 
 
-def test_scatter_count_mismatch_writes_nothing():
-    ids = synth.text_sequences(13, 1, 500, [[40]])
-    img = synth.randn_bf16(13, "img", (39, 256), 1.0)
-    text = synth.text_embeddings(13, 500, 256)
-    t_gpu = text.cuda()
+@pytest.mark.parametrize("seq_len,run,n_img", [(500, 40, 39), (500, 40, 41), (100, 10, 600), (40000, 900, 899)],
+                         ids=["fewer_rows", "more_rows", "more_rows_than_ids", "multi_kernel"])
+def test_scatter_count_mismatch_writes_nothing(seq_len, run, n_img):
+    ids = synth.text_sequences(13, 1, seq_len, [[run]])
+    img = synth.randn_bf16(13, "img", (n_img, 256), 1.0)
+    text = synth.text_embeddings(13, seq_len, 256)
+    t_gpu = guarded_copy(text)
     status = vlm.new_status()
     vlm.scatter(ids.reshape(-1).cuda(), img.cuda(), t_gpu, 10, status=status)
     assert vlm.status_sync(status) == vlm.ERR_COUNT_MISMATCH

@@ -12,7 +12,7 @@ import pytest
 import torch
 
 from oracle import vlm_oracle as O
-from tests.gpu_util import compare, to_np
+from tests.gpu_util import compare, to_np, guarded, guarded_zeros
 from vision_language_model_b200 import vlm
 
 pytestmark = pytest.mark.gpu
@@ -118,7 +118,7 @@ def test_gemm_nvfp4_exact_when_partial_sums_are_representable():
     sa = np.exp2(rng.integers(-2, 3, size=(M, K // 16))).astype(np.float64)
     sb = np.exp2(rng.integers(-2, 3, size=(N, K // 16))).astype(np.float64)
     ref = O.nvfp4_linear(qa, sa, 1.0, qb, sb, 1.0)
-    out = torch.zeros((M, N), dtype=torch.float32, device="cuda")
+    out = guarded_zeros((M, N), dtype=torch.float32)
     st = vlm.new_status()
     vlm.gemm_nvfp4(vlm.EPI_RESID, _operand(qa, sa, 1.0, K), _operand(qb, sb, 1.0, K), out, status=st)
     torch.cuda.synchronize()
@@ -136,7 +136,7 @@ def test_gemm_nvfp4_bf16_and_resid_epilogues(M, N, K):
     ref = O.nvfp4_linear(qa, sa, ga, qb, sb, gb)
     a, b = _operand(qa, sa, ga, K), _operand(qb, sb, gb, K)
     st = vlm.new_status()
-    out = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    out = guarded((M, N), dtype=torch.bfloat16)
     vlm.gemm_nvfp4(vlm.EPI_BF16, a, b, out, status=st)
     torch.cuda.synchronize()
     assert vlm.status_sync(st) == vlm.OK
@@ -165,7 +165,7 @@ def test_tower_shapes_quantise_and_multiply_on_sampled_rows(N, K):
     gw = vlm.amax_scale(wd)
     qa, sfa = vlm.quant_nvfp4(xd, ga)
     qw, sfw = vlm.quant_nvfp4(wd, gw)
-    out = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    out = guarded((M, N), dtype=torch.bfloat16)
     st = vlm.new_status()
     vlm.gemm_nvfp4(vlm.EPI_BF16, (qa, sfa, ga), (qw, sfw, gw), out, status=st)
     torch.cuda.synchronize()

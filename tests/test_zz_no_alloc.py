@@ -19,6 +19,7 @@ import pytest
 import torch
 
 from oracle import vlm_oracle as O
+from tests.gpu_util import guarded, guarded_copy, guarded_zeros
 from vision_language_model_b200 import synth, vlm
 
 pytestmark = pytest.mark.gpu
@@ -50,10 +51,10 @@ def test_noalloc_matches_workspace_scatter_on_two_calls(case):
         n_img = int((ids == 10).sum())
         img = synth.randn_bf16(seed, "img", (n_img, width), 1.0).cuda()
         text = synth.text_embeddings(seed, ids.numel(), width).cuda()
-        ref = text.clone()
+        ref = guarded_copy(text)
         st_ref = vlm.new_status()
         vlm.scatter(ids, img, ref, 10, status=st_ref)
-        got = text.clone()
+        got = guarded_copy(text)
         st = vlm.new_status()
         assert _call(ids, img, got, st) == vlm.OK
         assert vlm.status_sync(st) == vlm.OK and vlm.status_sync(st_ref) == vlm.OK
@@ -76,8 +77,8 @@ def test_noalloc_count_mismatch_writes_nothing():
 
 def test_noalloc_rejects_more_ids_than_its_scratch_holds():
     ids = torch.full((MAX_TOKENS + 1,), 11, dtype=torch.int64, device="cuda")
-    img = torch.empty((0, 8), dtype=torch.bfloat16, device="cuda")
-    text = torch.zeros((MAX_TOKENS + 1, 8), dtype=torch.bfloat16, device="cuda")
+    img = guarded((0, 8), dtype=torch.bfloat16)
+    text = guarded_zeros((MAX_TOKENS + 1, 8), dtype=torch.bfloat16)
     st = vlm.new_status()
     assert _call(ids, img, text, st) == vlm.ERR_BAD_SHAPE
     ids = ids[:MAX_TOKENS]

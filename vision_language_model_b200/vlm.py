@@ -50,6 +50,32 @@ class ProjectorWeights(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in ("g_proj", "w_merge", "w1", "w2")]
 
 
+def _torch_empty(shape, dtype, device) -> torch.Tensor:
+    return torch.empty(shape, dtype=dtype, device=device)
+
+
+# Every device buffer this module allocates (outputs, workspaces, packed
+# weights, status words) comes from here; a test harness may install its own
+# allocator, for example one that surrounds each buffer with guard bytes.
+_alloc = _torch_empty
+
+
+def set_allocator(fn=None):
+    """Install fn(shape, dtype, device) -> tensor as the allocator of this
+    module's device buffers (None restores torch.empty); returns the old one."""
+    global _alloc
+    old, _alloc = _alloc, (fn or _torch_empty)
+    return old
+
+
+def _empty(shape, dtype, device) -> torch.Tensor:
+    return _alloc(shape, dtype, device)
+
+
+def _zeros(shape, dtype, device) -> torch.Tensor:
+    return _alloc(shape, dtype, device).zero_()
+
+
 def lib_path() -> str:
     return _LIB_PATH
 
@@ -170,7 +196,7 @@ def num_merged(cfg: Config, image_hw) -> int:
 
 
 def new_status(device=None) -> torch.Tensor:
-    return torch.zeros(1, dtype=torch.int32, device=device or "cuda")
+    return _zeros(1, dtype=torch.int32, device=device or "cuda")
 
 
 def status_sync(status: torch.Tensor, stream=None) -> int:
@@ -188,7 +214,7 @@ def pack_tower(cfg: Config, w: dict, stream=None) -> torch.Tensor:
     nbytes = L.vlm_tower_packed_bytes(ctypes.byref(cfg))
     if nbytes == 0:
         raise VlmError(ERR_INVALID_ARG, "vlm_tower_packed_bytes")
-    packed = torch.empty(nbytes, dtype=torch.uint8, device=w["wq"].device)
+    packed = _empty(nbytes, dtype=torch.uint8, device=w["wq"].device)
     _check(L.vlm_pack_tower(ctypes.byref(cfg), ctypes.byref(tw), packed.data_ptr(), nbytes, _stream(stream)),
            "vlm_pack_tower")
     return packed
@@ -201,7 +227,7 @@ def pack_projector(cfg: Config, w: dict, stream=None) -> torch.Tensor:
     nbytes = L.vlm_projector_packed_bytes(ctypes.byref(cfg))
     if nbytes == 0:
         raise VlmError(ERR_INVALID_ARG, "vlm_projector_packed_bytes")
-    packed = torch.empty(nbytes, dtype=torch.uint8, device=w["w1"].device)
+    packed = _empty(nbytes, dtype=torch.uint8, device=w["w1"].device)
     _check(L.vlm_pack_projector(ctypes.byref(cfg), ctypes.byref(pw), packed.data_ptr(), nbytes, _stream(stream)),
            "vlm_pack_projector")
     return packed
@@ -224,10 +250,10 @@ def encode(cfg: Config, pixels: torch.Tensor, image_hw, packed_tower: torch.Tens
     T = num_patches(cfg, image_hw)
     dev = pixels.device
     if out is None:
-        out = torch.empty((T, cfg.width), dtype=torch.bfloat16, device=dev)
+        out = _empty((T, cfg.width), dtype=torch.bfloat16, device=dev)
     ws_need = L.vlm_encode_workspace_size(ctypes.byref(cfg), arr, n)
     if workspace is None:
-        workspace = torch.empty(ws_need, dtype=torch.uint8, device=dev)
+        workspace = _empty(ws_need, dtype=torch.uint8, device=dev)
     if status is None:
         status = new_status(dev)
     _check(L.vlm_encode(ctypes.byref(cfg), _dev(pixels, "pixels"), arr, n, _dev(packed_tower, "packed_tower"),
@@ -249,9 +275,9 @@ def merge_project(cfg: Config, tower_out: torch.Tensor, image_hw, packed_project
     Tm = num_merged(cfg, image_hw)
     dev = tower_out.device
     if out is None:
-        out = torch.empty((Tm, cfg.proj_out), dtype=torch.bfloat16, device=dev)
+        out = _empty((Tm, cfg.proj_out), dtype=torch.bfloat16, device=dev)
     if workspace is None:
-        workspace = torch.empty(L.vlm_merge_project_workspace_size(ctypes.byref(cfg), arr, n), dtype=torch.uint8,
+        workspace = _empty(L.vlm_merge_project_workspace_size(ctypes.byref(cfg), arr, n), dtype=torch.uint8,
                                 device=dev)
     if status is None:
         status = new_status(dev)
@@ -280,7 +306,7 @@ def scatter(input_ids: torch.Tensor, image_embeds: torch.Tensor, text_embeds: to
         raise ValueError("image and text rows differ in size")
     dev = text_embeds.device
     if workspace is None:
-        workspace = torch.empty(max(256, L.vlm_scatter_workspace_size(n)), dtype=torch.uint8, device=dev)
+        workspace = _empty(max(256, L.vlm_scatter_workspace_size(n)), dtype=torch.uint8, device=dev)
     if status is None:
         status = new_status(dev)
     _check(L.vlm_scatter(_dev(input_ids, "input_ids"), n, int(image_token_id), _dev(image_embeds, "image_embeds"),
@@ -312,7 +338,7 @@ def pack_tower_fp8(cfg: Config, w: dict, act_scales, stream=None) -> torch.Tenso
     nbytes = L.vlm_tower_fp8_packed_bytes(ctypes.byref(cfg))
     if nbytes == 0:
         raise VlmError(ERR_INVALID_ARG, "vlm_tower_fp8_packed_bytes")
-    packed = torch.empty(nbytes, dtype=torch.uint8, device=w["wq"].device)
+    packed = _empty(nbytes, dtype=torch.uint8, device=w["wq"].device)
     _check(L.vlm_pack_tower_fp8(ctypes.byref(cfg), ctypes.byref(tw), _act_array(cfg, act_scales), packed.data_ptr(),
                                 nbytes, _stream(stream)), "vlm_pack_tower_fp8")
     return packed
@@ -326,9 +352,9 @@ def encode_fp8(cfg: Config, pixels: torch.Tensor, image_hw, packed_tower_fp8: to
     T = num_patches(cfg, image_hw)
     dev = pixels.device
     if out is None:
-        out = torch.empty((T, cfg.width), dtype=torch.bfloat16, device=dev)
+        out = _empty((T, cfg.width), dtype=torch.bfloat16, device=dev)
     if workspace is None:
-        workspace = torch.empty(L.vlm_encode_workspace_size(ctypes.byref(cfg), arr, n), dtype=torch.uint8, device=dev)
+        workspace = _empty(L.vlm_encode_workspace_size(ctypes.byref(cfg), arr, n), dtype=torch.uint8, device=dev)
     if status is None:
         status = new_status(dev)
     _check(L.vlm_encode_fp8(ctypes.byref(cfg), _dev(pixels, "pixels"), arr, n, _dev(packed_tower_fp8, "packed"),
@@ -355,7 +381,7 @@ def rmsnorm_fp8(x: torch.Tensor, g1: torch.Tensor, f8_scale: float, g0=None, eps
                 stream=None) -> torch.Tensor:
     rows, width = x.shape
     if out is None:
-        out = torch.empty((rows, width), dtype=torch.uint8, device=x.device)
+        out = _empty((rows, width), dtype=torch.uint8, device=x.device)
     _check(lib().vlm_rmsnorm_fp8(_dev(x, "x"), _dev(g0, "g0"), _dev(g1, "g1"), _dev(out, "out"), rows, width,
                                  float(eps), float(f8_scale), _stream(stream)), "vlm_rmsnorm_fp8")
     return out
@@ -384,7 +410,7 @@ def _dtype_code(x: torch.Tensor) -> int:
 def amax_scale(x: torch.Tensor, divisor: float = NVFP4_GLOBAL_DIVISOR, out=None, stream=None) -> torch.Tensor:
     """Device fp32 [1] = max |x| / divisor (an NVFP4 global scale by default)."""
     if out is None:
-        out = torch.empty(1, dtype=torch.float32, device=x.device)
+        out = _empty(1, dtype=torch.float32, device=x.device)
     _check(lib().vlm_amax_scale(_dev(x, "x"), _dtype_code(x), x.numel(), float(divisor), _dev(out, "out"),
                                 _stream(stream)), "vlm_amax_scale")
     return out
@@ -395,9 +421,9 @@ def quant_nvfp4(x: torch.Tensor, s_global: torch.Tensor, q=None, sf=None, stream
     [nvfp4_sf_bytes(rows, K)]) with the device global scale s_global [1]."""
     rows, k = x.shape
     if q is None:
-        q = torch.empty((rows, k // 2), dtype=torch.uint8, device=x.device)
+        q = _empty((rows, k // 2), dtype=torch.uint8, device=x.device)
     if sf is None:
-        sf = torch.empty(max(nvfp4_sf_bytes(rows, k), 1), dtype=torch.uint8, device=x.device)
+        sf = _empty(max(nvfp4_sf_bytes(rows, k), 1), dtype=torch.uint8, device=x.device)
     _check(lib().vlm_quant_nvfp4(_dev(x, "x"), _dtype_code(x), rows, k, _dev(s_global, "s_global"), _dev(q, "q"),
                                  _dev(sf, "sf"), _stream(stream)), "vlm_quant_nvfp4")
     return q, sf
@@ -445,7 +471,7 @@ def preprocess(images_u8: torch.Tensor, src_hw, out_hw, tile: int = 0, out=None,
         raise ValueError(f"images_u8 holds {images_u8.numel()} bytes, the sizes need {need_src}")
     total = sum(3 * int(h) * int(w) for h, w in out_hw)
     if out is None:
-        out = torch.empty(total, dtype=torch.float32, device=images_u8.device)
+        out = _empty(total, dtype=torch.float32, device=images_u8.device)
     elif out.numel() < total or out.dtype != torch.float32:
         raise ValueError("out must be fp32 with room for every output pixel")
     _check(lib().vlm_preprocess(_dev(images_u8, "images_u8"), src_arr, n, out_arr, int(tile), _dev(out, "out"),
@@ -471,10 +497,10 @@ def expand_placeholders(input_ids: torch.Tensor, marker_id: int, counts, image_t
     carr = (ctypes.c_int64 * max(1, n_img))(*[int(c) for c in counts])
     total = n_ids - n_img + sum(int(c) for c in counts)
     if out is None:
-        out = torch.empty(max(total, 0), dtype=torch.int64, device=input_ids.device)
+        out = _empty(max(total, 0), dtype=torch.int64, device=input_ids.device)
     ws_need = L.vlm_expand_placeholders_workspace_size(n_ids, n_img)
     if workspace is None:
-        workspace = torch.empty(max(ws_need, 256), dtype=torch.uint8, device=input_ids.device)
+        workspace = _empty(max(ws_need, 256), dtype=torch.uint8, device=input_ids.device)
     if status is None:
         status = new_status(input_ids.device)
     out_len = ctypes.c_int64()
@@ -498,7 +524,7 @@ def gemm(epilogue: int, a: torch.Tensor, b: torch.Tensor, out: torch.Tensor, out
 
 
 def rope_table(theta: float, head_dim: int, max_pos: int, device="cuda", stream=None) -> torch.Tensor:
-    tab = torch.empty((max_pos, head_dim // 2, 2), dtype=torch.float32, device=device)
+    tab = _empty((max_pos, head_dim // 2, 2), dtype=torch.float32, device=device)
     _check(lib().vlm_rope_table(float(theta), head_dim, max_pos, tab.data_ptr(), _stream(stream)), "vlm_rope_table")
     return tab
 
@@ -509,8 +535,8 @@ def attention(qkv: torch.Tensor, cu_seqlens, heads: int, out=None, status=None, 
     cu = (ctypes.c_int32 * len(cu_seqlens))(*[int(c) for c in cu_seqlens])
     nb = len(cu_seqlens) - 1
     if out is None:
-        out = torch.empty((T, heads * 64), dtype=torch.bfloat16, device=qkv.device)
-    ws = torch.empty(max(256, L.vlm_attention_workspace_size(nb)), dtype=torch.uint8, device=qkv.device)
+        out = _empty((T, heads * 64), dtype=torch.bfloat16, device=qkv.device)
+    ws = _empty(max(256, L.vlm_attention_workspace_size(nb)), dtype=torch.uint8, device=qkv.device)
     if status is None:
         status = new_status(qkv.device)
     _check(L.vlm_attention(_dev(qkv, "qkv"), T, heads, 64, cu, nb, _dev(out, "out"), ws.data_ptr(), ws.numel(),
@@ -521,7 +547,7 @@ def attention(qkv: torch.Tensor, cu_seqlens, heads: int, out=None, status=None, 
 def rmsnorm(x: torch.Tensor, g1: torch.Tensor, g0=None, eps: float = 1e-5, out=None, stream=None) -> torch.Tensor:
     rows, width = x.shape
     if out is None:
-        out = torch.empty((rows, width), dtype=torch.bfloat16, device=x.device)
+        out = _empty((rows, width), dtype=torch.bfloat16, device=x.device)
     _check(lib().vlm_rmsnorm(_dev(x, "x"), _dev(g0, "g0"), _dev(g1, "g1"), _dev(out, "out"), rows, width, float(eps),
                              _stream(stream)), "vlm_rmsnorm")
     return out
@@ -569,10 +595,10 @@ class ImagePipeline:
         self.packed_proj = pack_projector(cfg, projector)
         self.T = num_patches(cfg, self.image_hw)
         self.Tm = num_merged(cfg, self.image_hw)
-        self.tower_out = torch.empty((self.T, cfg.width), dtype=torch.bfloat16, device=device)
-        self.embeds = torch.empty((self.Tm, cfg.proj_out), dtype=torch.bfloat16, device=device)
+        self.tower_out = _empty((self.T, cfg.width), dtype=torch.bfloat16, device=device)
+        self.embeds = _empty((self.Tm, cfg.proj_out), dtype=torch.bfloat16, device=device)
         ws = max(encode_workspace_size(cfg, self.image_hw), merge_project_workspace_size(cfg, self.image_hw))
-        self.workspace = torch.empty(ws, dtype=torch.uint8, device=device)
+        self.workspace = _empty(ws, dtype=torch.uint8, device=device)
         self.status = new_status(device)
 
     def __call__(self, pixels: torch.Tensor, stream=None) -> torch.Tensor:
