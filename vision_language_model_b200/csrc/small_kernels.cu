@@ -2,6 +2,8 @@
 // patch gather (im2col with the processor normalisation), RMSNorm, merge
 // gather, masked scatter and weight packing. Every one is a coalesced,
 // vectorised streaming kernel; none uses the tensor cores.
+#include <type_traits>
+
 #include "kernels.cuh"
 
 namespace vlm {
@@ -142,20 +144,44 @@ __global__ void __launch_bounds__(256) im2col_tiled_kernel(const float* __restri
     const int r = local / nch, c0 = (local - r * nch) * kI2cPatches;
     const int npat = min(kI2cPatches, in.w - c0), seg = npat * P;
     const float* base = pix + in.pix_off;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    // pixel-row segments warp, warp + 8, ...: every load of the lane is issued
+    // before the first one is used, so their latencies overlap
+    constexpr int NWARPS = 8, ROWS = 3 * P, RPW = (ROWS + NWARPS - 1) / NWARPS, XPL = (SEGMAX + 31) / 32;
+    float buf[RPW][XPL];
+#pragma unroll
+    for (int i = 0; i < RPW; ++i) {
+      const int row = warp + NWARPS * i;
+      if (row < ROWS) {
+        const int ch = row / P, ky = row - ch * P;
+        const float* src = base + (static_cast<int64_t>(ch) * in.H + r * P + ky) * in.W + c0 * P;
+#pragma unroll
+        for (int q = 0; q < XPL; ++q) {
+          const int x = lane + 32 * q;
+          buf[i][q] = x < seg ? __ldg(src + x) : 0.f;
+        }
+      }
+    }
     __syncthreads();  // the previous item's readers are done with the tile
-    for (int row = warp; row < 3 * P; row += nwarps) {  // one pixel-row segment per warp
-      const int ch = row / P, ky = row - ch * P;
-      const float* src = base + (static_cast<int64_t>(ch) * in.H + r * P + ky) * in.W + c0 * P;
-      const float scale = normalize ? c_inv_std[ch] : 1.0f, shift = normalize ? c_shift[ch] : 0.0f;
-      for (int x = lane; x < seg; x += 32) tile[row * SEGMAX + x] = fmaf(__ldg(src + x), scale, shift);
+#pragma unroll
+    for (int i = 0; i < RPW; ++i) {
+      const int row = warp + NWARPS * i;
+      if (row < ROWS) {
+        const int ch = row / P;
+        const float scale = normalize ? c_inv_std[ch] : 1.0f, shift = normalize ? c_shift[ch] : 0.0f;
+#pragma unroll
+        for (int q = 0; q < XPL; ++q) {
+          const int x = lane + 32 * q;
+          if (x < seg) tile[row * SEGMAX + x] = fmaf(buf[i][q], scale, shift);
+        }
+      }
     }
     __syncthreads();
     // each output bf16 pair (kx, kx + 1) of pixel row (ch, ky) is two adjacent tile floats
     constexpr int HALF_P = P / 2, REAL_PAIRS = 3 * PP / 2;
     const int half = kp / 2;
     const int64_t t0 = in.tok_off + static_cast<int64_t>(r) * in.w + c0;
-    for (int pi = warp; pi < npat; pi += nwarps) {  // one patch row per warp
+    for (int pi = warp; pi < npat; pi += NWARPS) {  // one patch row per warp
       uint32_t* orow = reinterpret_cast<uint32_t*>(out + (t0 + pi) * kp);
       for (int k2 = lane; k2 < half; k2 += 32) {
         uint32_t w = 0u;  // the zero padding past 3 P^2
@@ -249,39 +275,51 @@ __global__ void merge_norm_kernel(const __nv_bfloat16* __restrict__ x, const flo
   griddep_wait();
   griddep_launch_dependents();
   constexpr int width = NV * 128;
+  // 16-byte accesses (8 values per lane) when the row holds a whole number of
+  // 256-value warp chunks, 8-byte ones (4 values) otherwise
+  constexpr int VE = (NV % 2 == 0) ? 8 : 4, NL = width / (32 * VE);
+  using Vec = typename std::conditional<VE == 8, uint4, uint2>::type;
   const int lane = threadIdx.x & 31;
   const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
   for (int64_t t = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; t < T; t += warps) {
-    const uint2* xr = reinterpret_cast<const uint2*>(x + t * width);
-    float v[NV][4];
-    float ss = 0.f;
-#pragma unroll
-    for (int j = 0; j < NV; ++j) {
-      const uint2 u = xr[lane + 32 * j];
-      const __nv_bfloat162 a = *reinterpret_cast<const __nv_bfloat162*>(&u.x);
-      const __nv_bfloat162 bb = *reinterpret_cast<const __nv_bfloat162*>(&u.y);
-      v[j][0] = __low2float(a); v[j][1] = __high2float(a);
-      v[j][2] = __low2float(bb); v[j][3] = __high2float(bb);
-#pragma unroll
-      for (int e = 0; e < 4; ++e) ss += v[j][e] * v[j][e];
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-    const float rs = g != nullptr ? rsqrtf(ss / width + eps) : 1.0f;
+    // destination first: its table loads overlap the row loads below
     const int b = find_block(cu, n_images, static_cast<int>(t));
     const ImgInfo in = info[b];
     const int local = static_cast<int>(t) - in.tok_off;
     const int r = local / in.w, c = local % in.w;
     const int64_t mt = in.m_off + (r / m) * (in.w / m) + c / m;
     const int slot = (r % m) * m + c % m;
-    uint2* orow = reinterpret_cast<uint2*>(z + (mt * m * m + slot) * width);
+    const Vec* xr = reinterpret_cast<const Vec*>(x + t * width);
+    Vec u[NL];
+#pragma unroll
+    for (int j = 0; j < NL; ++j) u[j] = xr[lane + 32 * j];
+    float v[NL][VE];
+    float ss = 0.f;
+#pragma unroll
+    for (int j = 0; j < NL; ++j) {
+      const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&u[j]);
+#pragma unroll
+      for (int e = 0; e < VE / 2; ++e) {
+        v[j][2 * e] = __low2float(h2[e]);
+        v[j][2 * e + 1] = __high2float(h2[e]);
+        ss += v[j][2 * e] * v[j][2 * e] + v[j][2 * e + 1] * v[j][2 * e + 1];
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    const float rs = g != nullptr ? rsqrtf(ss / width + eps) : 1.0f;
+    Vec* orow = reinterpret_cast<Vec*>(z + (mt * m * m + slot) * width);
     const float4* gr = reinterpret_cast<const float4*>(g);
 #pragma unroll
-    for (int j = 0; j < NV; ++j) {
-      const float4 gg = g != nullptr ? __ldg(gr + lane + 32 * j) : make_float4(1.f, 1.f, 1.f, 1.f);
-      uint2 o;
-      o.x = pack_bf16x2(v[j][0] * rs * gg.x, v[j][1] * rs * gg.y);
-      o.y = pack_bf16x2(v[j][2] * rs * gg.z, v[j][3] * rs * gg.w);
+    for (int j = 0; j < NL; ++j) {
+      Vec o;
+      uint32_t* ow = reinterpret_cast<uint32_t*>(&o);
+#pragma unroll
+      for (int q = 0; q < VE / 4; ++q) {
+        const float4 gg = g != nullptr ? __ldg(gr + (lane + 32 * j) * (VE / 4) + q) : make_float4(1.f, 1.f, 1.f, 1.f);
+        ow[2 * q] = pack_bf16x2(v[j][4 * q] * rs * gg.x, v[j][4 * q + 1] * rs * gg.y);
+        ow[2 * q + 1] = pack_bf16x2(v[j][4 * q + 2] * rs * gg.z, v[j][4 * q + 3] * rs * gg.w);
+      }
       orow[lane + 32 * j] = o;
     }
   }
@@ -421,11 +459,114 @@ __global__ void scatter_copy_kernel(const uint4* __restrict__ img, uint4* __rest
   griddep_wait();
   griddep_launch_dependents();
   if (*ok_flag == 0) return;
-  const int64_t total = n_rows * vec_per_row;
-  for (int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; idx < total;
-       idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int64_t k = idx / vec_per_row, j = idx - k * vec_per_row;
-    text[dst_rows[k] * vec_per_row + j] = __ldg(img + idx);
+  const int lane = threadIdx.x & 31;
+  const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
+  for (int64_t k = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); k < n_rows;
+       k += warps) {
+    const uint4* src = img + k * vec_per_row;
+    uint4* dst = text + dst_rows[k] * vec_per_row;
+    int64_t j = lane;
+    for (; j + 96 < vec_per_row; j += 128) {
+      const uint4 a = __ldg(src + j), b = __ldg(src + j + 32), c = __ldg(src + j + 64), d = __ldg(src + j + 96);
+      dst[j] = a;
+      dst[j + 32] = b;
+      dst[j + 64] = c;
+      dst[j + 96] = d;
+    }
+    for (; j < vec_per_row; j += 32) dst[j] = __ldg(src + j);
+  }
+}
+
+// Single-launch masked scatter for up to kScatterFusedMaxIds ids. Every CTA
+// (1) turns the ids into a placeholder bitmask in shared memory with coalesced
+// loads, (2) counts the bits of a contiguous range of words per thread and
+// ranks them with one block scan, (3) records the text row of each image row
+// of its own slice [k0, k1) and (4) copies that slice, one row per warp, only
+// if the placeholder total equals n_img. All CTAs compute the same total, so
+// either every slice is copied or nothing is written; CTA 0 reports a mismatch.
+constexpr int kScatterFusedThreads = 512;
+constexpr int64_t kScatterFusedMaxIds = 32768;
+constexpr int kScatterFusedMaxRows = 2048;  // image rows per CTA slice
+
+__global__ void __launch_bounds__(kScatterFusedThreads)
+    scatter_fused_kernel(const int64_t* __restrict__ ids, int n, int64_t token, const uint4* __restrict__ img,
+                         uint4* __restrict__ text, int64_t n_img, int64_t vec_per_row, int rows_per_cta,
+                         int32_t* status) {
+  __shared__ uint32_t s_bits[kScatterFusedMaxIds / 32];
+  __shared__ int64_t s_dst[kScatterFusedMaxRows];
+  __shared__ int s_warp[kScatterFusedThreads / 32];
+  griddep_wait();
+  griddep_launch_dependents();
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  constexpr int kWarps = kScatterFusedThreads / 32;
+  const int n_words = (n + 31) / 32;
+  // (1) bitmask: id c + threadIdx.x -> bit lane of word (c + 32 warp) / 32
+#pragma unroll 4
+  for (int c = 0; c < n; c += kScatterFusedThreads) {
+    const int i = c + threadIdx.x;
+    const bool f = i < n && __ldg(ids + i) == token;
+    const uint32_t b = __ballot_sync(0xffffffffu, f);
+    if (lane == 0 && (c >> 5) + warp < n_words) s_bits[(c >> 5) + warp] = b;
+  }
+  __syncthreads();
+  // (2) thread t owns words [t * wpt, (t + 1) * wpt): contiguous ids, so an
+  // exclusive scan of the per-thread counts gives every placeholder's rank
+  const int wpt = (n_words + kScatterFusedThreads - 1) / kScatterFusedThreads;
+  const int w0 = min(n_words, static_cast<int>(threadIdx.x) * wpt), w1 = min(n_words, w0 + wpt);
+  int cnt = 0;
+  for (int w = w0; w < w1; ++w) cnt += __popc(s_bits[w]);
+  int incl = cnt;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) s_warp[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    int v = lane < kWarps ? s_warp[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, v, o);
+      if (lane >= o) v += y;
+    }
+    if (lane < kWarps) s_warp[lane] = v;
+  }
+  __syncthreads();
+  const int total = s_warp[kWarps - 1];
+  if (total != n_img) {
+    if (blockIdx.x == 0 && threadIdx.x == 0) set_status(status, VLM_ERR_COUNT_MISMATCH);
+    return;
+  }
+  // (3) text rows of this CTA's image rows
+  const int64_t k0 = static_cast<int64_t>(blockIdx.x) * rows_per_cta;
+  const int64_t k1 = min(n_img, k0 + rows_per_cta);
+  int64_t k = (warp > 0 ? s_warp[warp - 1] : 0) + incl - cnt;
+  if (k < k1 && k + cnt > k0) {
+    for (int w = w0; w < w1; ++w) {
+      uint32_t b = s_bits[w];
+      while (b) {
+        const int bit = __ffs(b) - 1;
+        b &= b - 1;
+        if (k >= k0 && k < k1) s_dst[k - k0] = static_cast<int64_t>(w) * 32 + bit;
+        ++k;
+      }
+    }
+  }
+  __syncthreads();
+  // (4) copy, one row per warp, four 16-byte loads in flight per lane
+  for (int64_t r = k0 + warp; r < k1; r += kWarps) {
+    const uint4* src = img + r * vec_per_row;
+    uint4* dst = text + s_dst[r - k0] * vec_per_row;
+    int64_t j = lane;
+    for (; j + 96 < vec_per_row; j += 128) {
+      const uint4 a = __ldg(src + j), b = __ldg(src + j + 32), c = __ldg(src + j + 64), d = __ldg(src + j + 96);
+      dst[j] = a;
+      dst[j + 32] = b;
+      dst[j + 64] = c;
+      dst[j + 96] = d;
+    }
+    for (; j < vec_per_row; j += 32) dst[j] = __ldg(src + j);
   }
 }
 
@@ -618,6 +759,20 @@ int launch_rmsnorm_bf16(const __nv_bfloat16* x, const float* g, __nv_bfloat16* o
 
 int launch_scatter(const int64_t* ids, int64_t n, int64_t token, const void* img, int64_t n_img,
                    void* text, int64_t row_bytes, ScatterWs ws, int32_t* status, cudaStream_t s) {
+  if (n <= kScatterFusedMaxIds) {
+    // one launch; the workspace is not used
+    const int64_t slots = 2LL * num_sms();
+    int64_t rows = n_img > n ? 1 : (n_img + slots - 1) / slots;  // more rows than ids can only mismatch
+    rows = rows < 1 ? 1 : (rows > kScatterFusedMaxRows ? kScatterFusedMaxRows : rows);
+    const int64_t grid = n_img > n ? 1 : (n_img + rows - 1) / rows;
+    launch_begin(KC_SCATTER, s);
+    const cudaError_t e = launch_pdl(scatter_fused_kernel, dim3(static_cast<unsigned>(grid < 1 ? 1 : grid)),
+                                     dim3(kScatterFusedThreads), 0, s, ids, static_cast<int>(n), token,
+                                     static_cast<const uint4*>(img), static_cast<uint4*>(text), n_img,
+                                     row_bytes / 16, static_cast<int>(rows), status);
+    launch_end(KC_SCATTER, s);
+    return e == cudaSuccess ? VLM_OK : VLM_ERR_CUDA;
+  }
   const int64_t n_chunks = (n + 255) / 256;
   launch_begin(KC_SCATTER, s);
   const dim3 chunks(static_cast<unsigned>(n_chunks));
@@ -630,7 +785,7 @@ int launch_scatter(const int64_t* ids, int64_t n, int64_t token, const void* img
                    ws.dst_rows);
   const int64_t vec = row_bytes / 16;
   if (e == cudaSuccess)
-    e = launch_pdl(scatter_copy_kernel, dim3(grid_for(n_img * vec, 256)), dim3(256), 0, s,
+    e = launch_pdl(scatter_copy_kernel, dim3(grid_for(n_img * 32, 256)), dim3(256), 0, s,
                    static_cast<const uint4*>(img), static_cast<uint4*>(text), ws.dst_rows, ws.ok_flag, n_img, vec);
   launch_end(KC_SCATTER, s);
   note_extra_launches(3);
