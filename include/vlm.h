@@ -202,7 +202,8 @@ VLM_API int vlm_encode_fp8(const vlm_config* cfg, const float* pixels, const int
  * W1 (D -> E), exact GELU, W2 (E -> E). With merge == 1 ([P]) the unfold and
  * merge linear are skipped.
  *
- * d_tower_out: device bf16 [T, width] from vlm_encode with the same image_hw.
+ * d_tower_out: device bf16 [T, width] from vlm_encode with the same image_hw,
+ *   16-byte aligned (VLM_ERR_INVALID_ARG otherwise).
  * d_out: device bf16 [T_m, proj_out], merged tokens row-major per image,
  *   images concatenated.
  * ------------------------------------------------------------------------- */

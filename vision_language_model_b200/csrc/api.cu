@@ -634,6 +634,7 @@ int vlm_merge_project(const vlm_config* cfg, const void* d_tower_out, const int3
   if (d_tower_out == nullptr || d_packed_projector == nullptr || d_out == nullptr || d_workspace == nullptr)
     return VLM_ERR_INVALID_ARG;
   if (reinterpret_cast<uintptr_t>(d_workspace) & 255) return VLM_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(d_tower_out) & 15) return VLM_ERR_INVALID_ARG;  // read by bulk copies
   Batch b;
   VLM_TRY(make_batch(cfg, image_hw, n_images, &b));
   const ProjWs p = carve_proj(d_workspace, cfg, b);
@@ -648,7 +649,7 @@ int vlm_merge_project(const vlm_config* cfg, const void* d_tower_out, const int3
   VLM_TRY(upload_batch(b, p.bd, s));
   // the merge gather, normalising each patch unless the norm follows the merge linear
   VLM_TRY(launch_merge_norm(static_cast<const __nv_bfloat16*>(d_tower_out), after ? nullptr : g_proj, p.bd.info,
-                            p.bd.cu, b.n, b.T, static_cast<int>(D), cfg->merge, cfg->eps, p.z, s));
+                            p.bd.cu, b.n, b.T, static_cast<int>(D), cfg->merge, cfg->eps, p.z, d_status, s));
   const __nv_bfloat16* y = p.z;
   if (cfg->merge > 1) {
     VLM_TRY(launch_gemm(VLM_EPI_BF16, p.z, pk + L.w_merge, b.Tm, D, mm * D, p.y, nullptr, nullptr, nullptr, 0,

@@ -89,7 +89,7 @@ int launch_rmsnorm_bf16(const __nv_bfloat16* x, const float* g, __nv_bfloat16* o
                         float eps, cudaStream_t s);
 // g == nullptr: gather only (no normalisation).
 int launch_merge_norm(const __nv_bfloat16* x, const float* g, const ImgInfo* info, const int32_t* cu,
-                      int n_images, int64_t T, int width, int m, float eps, __nv_bfloat16* z,
+                      int n_images, int64_t T, int width, int m, float eps, __nv_bfloat16* z, int32_t* status,
                       cudaStream_t s);
 int launch_scatter(const int64_t* ids, int64_t n, int64_t token, const void* img, int64_t n_img,
                    void* text, int64_t row_bytes, ScatterWs ws, int32_t* status, cudaStream_t s);

@@ -2,6 +2,7 @@
 // patch gather (im2col with the processor normalisation), RMSNorm, merge
 // gather, masked scatter and weight packing. Every one is a coalesced,
 // vectorised streaming kernel; none uses the tensor cores.
+#include <algorithm>
 #include <type_traits>
 
 #include "kernels.cuh"
@@ -126,8 +127,10 @@ __global__ void im2col_kernel(const float* __restrict__ pix, const ImgInfo* __re
 // up to kI2cPatches patches of one patch row. The item's 3 x P pixel-row
 // segments are read with coalesced loads into shared memory (normalised on the
 // way), then the item's patch rows are written as consecutive bf16 pairs.
+constexpr int kI2cThreads = 128;  // 4 warps: small CTAs, so several items per SM are in flight at once
+
 template <int P>
-__global__ void __launch_bounds__(256) im2col_tiled_kernel(const float* __restrict__ pix,
+__global__ void __launch_bounds__(kI2cThreads) im2col_tiled_kernel(const float* __restrict__ pix,
                                                            const ImgInfo* __restrict__ info,
                                                            const int32_t* __restrict__ i2c, int n_images,
                                                            int items, int kp, int normalize,
@@ -147,7 +150,7 @@ __global__ void __launch_bounds__(256) im2col_tiled_kernel(const float* __restri
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     // pixel-row segments warp, warp + 8, ...: every load of the lane is issued
     // before the first one is used, so their latencies overlap
-    constexpr int NWARPS = 8, ROWS = 3 * P, RPW = (ROWS + NWARPS - 1) / NWARPS, XPL = (SEGMAX + 31) / 32;
+    constexpr int NWARPS = kI2cThreads / 32, ROWS = 3 * P, RPW = (ROWS + NWARPS - 1) / NWARPS, XPL = (SEGMAX + 31) / 32;
     float buf[RPW][XPL];
 #pragma unroll
     for (int i = 0; i < RPW; ++i) {
@@ -181,16 +184,24 @@ __global__ void __launch_bounds__(256) im2col_tiled_kernel(const float* __restri
     constexpr int HALF_P = P / 2, REAL_PAIRS = 3 * PP / 2;
     const int half = kp / 2;
     const int64_t t0 = in.tok_off + static_cast<int64_t>(r) * in.w + c0;
+    // pair k2 of a patch row is (pixel row k2 / (P/2), pair k2 % (P/2)); a lane steps
+    // k2 by 32, i.e. the row by 32 / (P/2) and the pair by 32 % (P/2), with a carry
+    constexpr int STEP_ROW = 32 / HALF_P, STEP_PAIR = 32 % HALF_P;
+    const int row0 = lane / HALF_P, pair0 = lane % HALF_P;
     for (int pi = warp; pi < npat; pi += NWARPS) {  // one patch row per warp
       uint32_t* orow = reinterpret_cast<uint32_t*>(out + (t0 + pi) * kp);
+      const float* trow = tile + pi * P;
+      int row = row0, pair = pair0;
       for (int k2 = lane; k2 < half; k2 += 32) {
         uint32_t w = 0u;  // the zero padding past 3 P^2
         if (k2 < REAL_PAIRS) {
-          const int row = k2 / HALF_P, pair = k2 - row * HALF_P;
-          const float2 v = *reinterpret_cast<const float2*>(&tile[row * SEGMAX + pi * P + 2 * pair]);
+          const float2 v = *reinterpret_cast<const float2*>(&trow[row * SEGMAX + 2 * pair]);
           w = pack_bf16x2(v.x, v.y);
         }
         orow[k2] = w;
+        row += STEP_ROW;
+        pair += STEP_PAIR;
+        if (pair >= HALF_P) { pair -= HALF_P; ++row; }
       }
     }
   }
@@ -262,68 +273,6 @@ __global__ void rmsnorm_kernel(float* __restrict__ x, const float* __restrict__ 
   }
 }
 
-// ---------------------------------------------------------------------------
-// Projector RMSNorm + m x m merge gather, one warp per patch (bf16 in/out).
-// Patch (r, c) of image b goes to merged token m_off_b + (r/m)(w/m) + c/m,
-// slot (r%m)*m + c%m, i.e. z[token, slot*D + ch] (patch-major).
-// ---------------------------------------------------------------------------
-template <int NV>
-__global__ void merge_norm_kernel(const __nv_bfloat16* __restrict__ x, const float* __restrict__ g,
-                                  const ImgInfo* __restrict__ info, const int32_t* __restrict__ cu,
-                                  int n_images, int64_t T, int m, float eps,
-                                  __nv_bfloat16* __restrict__ z) {
-  griddep_wait();
-  griddep_launch_dependents();
-  constexpr int width = NV * 128;
-  // 16-byte accesses (8 values per lane) when the row holds a whole number of
-  // 256-value warp chunks, 8-byte ones (4 values) otherwise
-  constexpr int VE = (NV % 2 == 0) ? 8 : 4, NL = width / (32 * VE);
-  using Vec = typename std::conditional<VE == 8, uint4, uint2>::type;
-  const int lane = threadIdx.x & 31;
-  const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
-  for (int64_t t = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; t < T; t += warps) {
-    // destination first: its table loads overlap the row loads below
-    const int b = find_block(cu, n_images, static_cast<int>(t));
-    const ImgInfo in = info[b];
-    const int local = static_cast<int>(t) - in.tok_off;
-    const int r = local / in.w, c = local % in.w;
-    const int64_t mt = in.m_off + (r / m) * (in.w / m) + c / m;
-    const int slot = (r % m) * m + c % m;
-    const Vec* xr = reinterpret_cast<const Vec*>(x + t * width);
-    Vec u[NL];
-#pragma unroll
-    for (int j = 0; j < NL; ++j) u[j] = xr[lane + 32 * j];
-    float v[NL][VE];
-    float ss = 0.f;
-#pragma unroll
-    for (int j = 0; j < NL; ++j) {
-      const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&u[j]);
-#pragma unroll
-      for (int e = 0; e < VE / 2; ++e) {
-        v[j][2 * e] = __low2float(h2[e]);
-        v[j][2 * e + 1] = __high2float(h2[e]);
-        ss += v[j][2 * e] * v[j][2 * e] + v[j][2 * e + 1] * v[j][2 * e + 1];
-      }
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-    const float rs = g != nullptr ? rsqrtf(ss / width + eps) : 1.0f;
-    Vec* orow = reinterpret_cast<Vec*>(z + (mt * m * m + slot) * width);
-    const float4* gr = reinterpret_cast<const float4*>(g);
-#pragma unroll
-    for (int j = 0; j < NL; ++j) {
-      Vec o;
-      uint32_t* ow = reinterpret_cast<uint32_t*>(&o);
-#pragma unroll
-      for (int q = 0; q < VE / 4; ++q) {
-        const float4 gg = g != nullptr ? __ldg(gr + (lane + 32 * j) * (VE / 4) + q) : make_float4(1.f, 1.f, 1.f, 1.f);
-        ow[2 * q] = pack_bf16x2(v[j][4 * q] * rs * gg.x, v[j][4 * q + 1] * rs * gg.y);
-        ow[2 * q + 1] = pack_bf16x2(v[j][4 * q + 2] * rs * gg.z, v[j][4 * q + 3] * rs * gg.w);
-      }
-      orow[lane + 32 * j] = o;
-    }
-  }
-}
 
 // RMSNorm of bf16 rows into bf16 (in place allowed), one warp per row.
 template <int NV>
@@ -477,28 +426,76 @@ __global__ void scatter_copy_kernel(const uint4* __restrict__ img, uint4* __rest
   }
 }
 
-// Single-launch masked scatter for up to kScatterFusedMaxIds ids. Every CTA
-// (1) turns the ids into a placeholder bitmask in shared memory with coalesced
-// loads, (2) counts the bits of a contiguous range of words per thread and
-// ranks them with one block scan, (3) records the text row of each image row
-// of its own slice [k0, k1) and (4) copies that slice, one row per warp, only
-// if the placeholder total equals n_img. All CTAs compute the same total, so
-// either every slice is copied or nothing is written; CTA 0 reports a mismatch.
+// Single-launch masked scatter for up to kScatterFusedMaxIds ids. Each CTA
+// owns a slice [k0, k1) of the image rows. Its thread 0 first starts bulk
+// copies (cp.async.bulk, no multicast) of the slice's first rows into a ring
+// of row buffers in shared memory; meanwhile all threads (1) turn the ids into
+// a placeholder bitmask with coalesced loads, (2) count the bits of a
+// contiguous range of words per thread and rank them with one block scan and
+// (3) record the text row of each row of the slice. Only if the placeholder
+// total equals n_img does thread 0 then (4) store each buffered row to its
+// text row with a bulk copy and refill the buffer with the next row of the
+// slice. All CTAs compute the same total, so either every slice is copied or
+// nothing is written; CTA 0 reports a mismatch. Every wait is bounded.
 constexpr int kScatterFusedThreads = 512;
 constexpr int64_t kScatterFusedMaxIds = 32768;
-constexpr int kScatterFusedMaxRows = 2048;  // image rows per CTA slice
+constexpr int kScatterFusedMaxRows = 2048;      // image rows per CTA slice
+constexpr int kScatterRingBytes = 96 * 1024;    // row buffers per CTA
+constexpr int kScatterRingMaxRows = 8;
+
+__device__ __forceinline__ void bulk_load_row(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+               "l"(src), "r"(bytes), "r"(bar)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_store_row(void* dst, uint32_t src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst), "r"(src), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_wait_read_le(int n) {  // at most n of this thread's bulk groups still reading
+  if (n <= 0) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+  else if (n == 1) asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+  else if (n == 2) asm volatile("cp.async.bulk.wait_group.read 2;" ::: "memory");
+  else if (n == 3) asm volatile("cp.async.bulk.wait_group.read 3;" ::: "memory");
+  else if (n == 4) asm volatile("cp.async.bulk.wait_group.read 4;" ::: "memory");
+  else if (n == 5) asm volatile("cp.async.bulk.wait_group.read 5;" ::: "memory");
+  else if (n == 6) asm volatile("cp.async.bulk.wait_group.read 6;" ::: "memory");
+  else asm volatile("cp.async.bulk.wait_group.read 7;" ::: "memory");
+}
 
 __global__ void __launch_bounds__(kScatterFusedThreads)
-    scatter_fused_kernel(const int64_t* __restrict__ ids, int n, int64_t token, const uint4* __restrict__ img,
-                         uint4* __restrict__ text, int64_t n_img, int64_t vec_per_row, int rows_per_cta,
+    scatter_fused_kernel(const int64_t* __restrict__ ids, int n, int64_t token, const uint8_t* __restrict__ img,
+                         uint8_t* __restrict__ text, int64_t n_img, int64_t row_bytes, int rows_per_cta, int ring,
                          int32_t* status) {
+  extern __shared__ __align__(128) uint8_t s_ring[];  // ring x row_bytes
   __shared__ uint32_t s_bits[kScatterFusedMaxIds / 32];
   __shared__ int64_t s_dst[kScatterFusedMaxRows];
   __shared__ int s_warp[kScatterFusedThreads / 32];
-  griddep_wait();
-  griddep_launch_dependents();
+  __shared__ __align__(8) uint64_t s_full[kScatterRingMaxRows];
+  __shared__ int s_abort;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   constexpr int kWarps = kScatterFusedThreads / 32;
+  const int64_t k0 = static_cast<int64_t>(blockIdx.x) * rows_per_cta;
+  const int64_t k1 = min(n_img, k0 + rows_per_cta);
+  const int n_rows = static_cast<int>(k1 > k0 ? k1 - k0 : 0);
+  const uint32_t bytes = static_cast<uint32_t>(row_bytes);
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < ring; ++i) mbar_init(smem_u32(s_full + i), 1);
+    s_abort = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  griddep_wait();
+  griddep_launch_dependents();
+  volatile int* abort_v = &s_abort;
+  // the slice's first rows start loading now; the scan below hides their latency
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < min(ring, n_rows); ++i) {
+      mbar_arrive_expect_tx(smem_u32(s_full + i), bytes);
+      bulk_load_row(smem_u32(s_ring + static_cast<size_t>(i) * row_bytes), img + (k0 + i) * row_bytes, bytes,
+                    smem_u32(s_full + i));
+    }
+  }
   const int n_words = (n + 31) / 32;
   // (1) bitmask: id c + threadIdx.x -> bit lane of word (c + 32 warp) / 32
 #pragma unroll 4
@@ -534,40 +531,52 @@ __global__ void __launch_bounds__(kScatterFusedThreads)
   }
   __syncthreads();
   const int total = s_warp[kWarps - 1];
-  if (total != n_img) {
-    if (blockIdx.x == 0 && threadIdx.x == 0) set_status(status, VLM_ERR_COUNT_MISMATCH);
-    return;
-  }
+  const bool good = total == n_img;
   // (3) text rows of this CTA's image rows
-  const int64_t k0 = static_cast<int64_t>(blockIdx.x) * rows_per_cta;
-  const int64_t k1 = min(n_img, k0 + rows_per_cta);
-  int64_t k = (warp > 0 ? s_warp[warp - 1] : 0) + incl - cnt;
-  if (k < k1 && k + cnt > k0) {
-    for (int w = w0; w < w1; ++w) {
-      uint32_t b = s_bits[w];
-      while (b) {
-        const int bit = __ffs(b) - 1;
-        b &= b - 1;
-        if (k >= k0 && k < k1) s_dst[k - k0] = static_cast<int64_t>(w) * 32 + bit;
-        ++k;
+  if (good) {
+    int64_t k = (warp > 0 ? s_warp[warp - 1] : 0) + incl - cnt;
+    if (k < k1 && k + cnt > k0) {
+      for (int w = w0; w < w1; ++w) {
+        uint32_t b = s_bits[w];
+        while (b) {
+          const int bit = __ffs(b) - 1;
+          b &= b - 1;
+          if (k >= k0 && k < k1) s_dst[k - k0] = static_cast<int64_t>(w) * 32 + bit;
+          ++k;
+        }
+      }
+    }
+  } else if (blockIdx.x == 0 && threadIdx.x == 0) {
+    set_status(status, VLM_ERR_COUNT_MISMATCH);
+  }
+  __syncthreads();
+  if (threadIdx.x != 0) return;
+  // (4) thread 0: each buffered row to its text row. The buffer of the row
+  // stored `lag` rows earlier takes the row `ring` after it once that store
+  // has read it, so `lag` stores and ring - lag loads stay in flight.
+  const int lag = ring / 2;
+  int issued = min(ring, n_rows), done = 0;
+  if (good) {
+    for (int r = 0; r < n_rows; ++r) {
+      if (!mbar_wait(smem_u32(s_full + r % ring), (r / ring) & 1, abort_v, status)) break;
+      bulk_store_row(text + s_dst[r] * row_bytes, smem_u32(s_ring + static_cast<size_t>(r % ring) * row_bytes), bytes);
+      bulk_commit();
+      done = r + 1;
+      const int q = r - lag;  // its store is older than the newest `lag` ones
+      if (q >= 0 && q + ring < n_rows) {
+        bulk_wait_read_le(lag);
+        const int buf = q % ring;
+        mbar_arrive_expect_tx(smem_u32(s_full + buf), bytes);
+        bulk_load_row(smem_u32(s_ring + static_cast<size_t>(buf) * row_bytes), img + (k0 + q + ring) * row_bytes,
+                      bytes, smem_u32(s_full + buf));
+        issued = q + ring + 1;
       }
     }
   }
-  __syncthreads();
-  // (4) copy, one row per warp, four 16-byte loads in flight per lane
-  for (int64_t r = k0 + warp; r < k1; r += kWarps) {
-    const uint4* src = img + r * vec_per_row;
-    uint4* dst = text + s_dst[r - k0] * vec_per_row;
-    int64_t j = lane;
-    for (; j + 96 < vec_per_row; j += 128) {
-      const uint4 a = __ldg(src + j), b = __ldg(src + j + 32), c = __ldg(src + j + 64), d = __ldg(src + j + 96);
-      dst[j] = a;
-      dst[j + 32] = b;
-      dst[j + 64] = c;
-      dst[j + 96] = d;
-    }
-    for (; j < vec_per_row; j += 32) dst[j] = __ldg(src + j);
-  }
+  // loads still in flight must land before the CTA's shared memory goes away
+  for (int r = done; r < issued; ++r)
+    if (!mbar_wait(smem_u32(s_full + r % ring), (r / ring) & 1, abort_v, status)) break;
+  bulk_wait<0>();
 }
 
 // ---------------------------------------------------------------------------
@@ -678,13 +687,14 @@ int launch_im2col(const float* pix, const ImgInfo* info, const int32_t* cu, cons
                   int n_images, int64_t T, int p, int kp, int normalize, __nv_bfloat16* out, cudaStream_t s) {
   launch_begin(KC_IM2COL, s);
   cudaError_t e;
-  const int tgrid = i2c_items < num_sms() * 8 ? (i2c_items > 0 ? i2c_items : 1) : num_sms() * 8;
+  // one item per CTA up to 16 CTAs per SM, then a grid-stride loop
+  const int tgrid = i2c_items < num_sms() * 16 ? (i2c_items > 0 ? i2c_items : 1) : num_sms() * 16;
   if (p == 14 && i2c != nullptr)
-    e = launch_pdl(im2col_tiled_kernel<14>, dim3(tgrid), dim3(256), 0, s, pix, info, i2c, n_images, i2c_items, kp,
-                   normalize, out);
+    e = launch_pdl(im2col_tiled_kernel<14>, dim3(tgrid), dim3(kI2cThreads), 0, s, pix, info, i2c, n_images,
+                   i2c_items, kp, normalize, out);
   else if (p == 16 && i2c != nullptr)
-    e = launch_pdl(im2col_tiled_kernel<16>, dim3(tgrid), dim3(256), 0, s, pix, info, i2c, n_images, i2c_items, kp,
-                   normalize, out);
+    e = launch_pdl(im2col_tiled_kernel<16>, dim3(tgrid), dim3(kI2cThreads), 0, s, pix, info, i2c, n_images,
+                   i2c_items, kp, normalize, out);
   else
     e = launch_pdl(im2col_kernel, dim3(grid_for(T * 32, 256)), dim3(256), 0, s, pix, info, cu, n_images, T, p, kp,
                    normalize, out);
@@ -716,16 +726,156 @@ int launch_rmsnorm(float* x, const float* g0, const float* g1, void* out, int64_
   return e == cudaSuccess ? VLM_OK : VLM_ERR_CUDA;
 }
 
+// ---------------------------------------------------------------------------
+// Projector RMSNorm + m x m merge gather (bf16 in/out). Patch (r, c) of image
+// b goes to merged token m_off_b + (r/m)(w/m) + c/m, slot (r%m)*m + c%m, i.e.
+// z[token, slot*D + ch] (patch-major). A CTA takes kMergeRows consecutive
+// patches: one bulk copy brings their rows into shared memory; meanwhile each
+// warp finds its rows' destinations and holds the gains in registers; then it
+// normalises each row in place and one lane bulk-stores the row to its slot.
+// The bulk engine keeps many bytes in flight at few registers per thread.
+// g == nullptr: gather only (the merge-first reading normalises later).
+// ---------------------------------------------------------------------------
+constexpr int kMergeThreads = 256;
+constexpr int kMergeSmem = 64 * 1024;
+
+template <int NV>
+__global__ void __launch_bounds__(kMergeThreads, 3) merge_norm_kernel(const __nv_bfloat16* __restrict__ x,
+                                                                   const float* __restrict__ g,
+                                                                   const ImgInfo* __restrict__ info,
+                                                                   const int32_t* __restrict__ cu, int n_images,
+                                                                   int64_t T, int m, float eps, int rows_per_cta,
+                                                                   __nv_bfloat16* __restrict__ z, int32_t* status) {
+  extern __shared__ __align__(128) uint8_t s_rows[];  // rows_per_cta x width bf16
+  __shared__ __align__(8) uint64_t s_full;
+  __shared__ int s_abort;
+  constexpr int width = NV * 128;
+  constexpr uint32_t kRowBytes = width * 2;
+  constexpr int kWarps = kMergeThreads / 32;
+  constexpr int kMaxRowsPerWarp = kMergeSmem / kRowBytes / kWarps > 0 ? kMergeSmem / kRowBytes / kWarps : 1;
+  // 16-byte accesses (8 values per lane) when the row holds a whole number of
+  // 256-value warp chunks, 8-byte ones (4 values) otherwise
+  constexpr int VE = (NV % 2 == 0) ? 8 : 4, NL = width / (32 * VE);
+  using Vec = typename std::conditional<VE == 8, uint4, uint2>::type;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int64_t t0 = static_cast<int64_t>(blockIdx.x) * rows_per_cta;
+  const int nrows = static_cast<int>(min(static_cast<int64_t>(rows_per_cta), T - t0));
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&s_full), 1);
+    s_abort = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  griddep_wait();
+  griddep_launch_dependents();
+  if (threadIdx.x == 0) {
+    mbar_arrive_expect_tx(smem_u32(&s_full), nrows * kRowBytes);
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                     smem_u32(s_rows)),
+                 "l"(x + t0 * width), "r"(nrows * kRowBytes), "r"(smem_u32(&s_full))
+                 : "memory");
+  }
+  // while the rows arrive: their destinations and the gains
+  int64_t dst[kMaxRowsPerWarp];
+#pragma unroll
+  for (int i = 0; i < kMaxRowsPerWarp; ++i) {
+    const int lr = warp + kWarps * i;
+    dst[i] = -1;
+    if (lr < nrows) {
+      const int t = static_cast<int>(t0 + lr);
+      const int b = find_block(cu, n_images, t);
+      const ImgInfo in = info[b];
+      const int local = t - in.tok_off;
+      const int r = local / in.w, c = local % in.w;
+      const int64_t mt = in.m_off + (r / m) * (in.w / m) + c / m;
+      dst[i] = (mt * m * m + (r % m) * m + c % m) * width;
+    }
+  }
+  float gv[NL][VE];
+#pragma unroll
+  for (int j = 0; j < NL; ++j)
+#pragma unroll
+    for (int q = 0; q < VE / 4; ++q) {
+      const float4 gg = g != nullptr ? __ldg(reinterpret_cast<const float4*>(g) + (lane + 32 * j) * (VE / 4) + q)
+                                     : make_float4(1.f, 1.f, 1.f, 1.f);
+      gv[j][4 * q] = gg.x;
+      gv[j][4 * q + 1] = gg.y;
+      gv[j][4 * q + 2] = gg.z;
+      gv[j][4 * q + 3] = gg.w;
+    }
+  const bool ok = mbar_wait(smem_u32(&s_full), 0, &s_abort, status);
+  if (ok) {
+#pragma unroll
+    for (int i = 0; i < kMaxRowsPerWarp; ++i) {
+      if (dst[i] < 0) break;
+      Vec* row = reinterpret_cast<Vec*>(s_rows + static_cast<size_t>(warp + kWarps * i) * kRowBytes);
+      Vec u[NL];
+      float ss = 0.f;
+#pragma unroll
+      for (int j = 0; j < NL; ++j) {
+        u[j] = row[lane + 32 * j];
+        const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&u[j]);
+#pragma unroll
+        for (int e = 0; e < VE / 2; ++e) {
+          const float a0 = __low2float(h2[e]), a1 = __high2float(h2[e]);
+          ss += a0 * a0 + a1 * a1;
+        }
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+      const float rs = g != nullptr ? rsqrtf(ss / width + eps) : 1.0f;
+#pragma unroll
+      for (int j = 0; j < NL; ++j) {
+        const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&u[j]);
+        Vec o;
+        uint32_t* ow = reinterpret_cast<uint32_t*>(&o);
+#pragma unroll
+        for (int e = 0; e < VE / 2; ++e)
+          ow[e] = pack_bf16x2(__low2float(h2[e]) * rs * gv[j][2 * e], __high2float(h2[e]) * rs * gv[j][2 * e + 1]);
+        row[lane + 32 * j] = o;
+      }
+      fence_proxy_async_smem();  // the row's new values are visible to the bulk copy below
+      __syncwarp();
+      if (lane == 0) {
+        asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(z + dst[i]),
+                     "r"(smem_u32(row)), "r"(kRowBytes)
+                     : "memory");
+        asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+      }
+    }
+  }
+  if (lane == 0) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");  // stores done before the CTA ends
+}
+
 int launch_merge_norm(const __nv_bfloat16* x, const float* g, const ImgInfo* info, const int32_t* cu,
-                      int n_images, int64_t T, int width, int m, float eps, __nv_bfloat16* z,
+                      int n_images, int64_t T, int width, int m, float eps, __nv_bfloat16* z, int32_t* status,
                       cudaStream_t s) {
   if (width % 128 || width > 2048 || width <= 0) return VLM_ERR_UNSUPPORTED;
-  const int grid = grid_for(T * 32, 256);
+  if (T <= 0) return VLM_OK;
+  const int row_bytes = width * 2;
+  const int warps = kMergeThreads / 32;
+  // rows per CTA: as many as fit the shared buffer, a whole number per warp
+  const int per_warp = std::max(1, kMergeSmem / row_bytes / warps);
+  const int rows = per_warp * warps;
+  const int64_t grid = (T + rows - 1) / rows;
+  const size_t smem = static_cast<size_t>(rows) * row_bytes;
+  static bool attr_done[64][17] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
   launch_begin(KC_MERGE, s);
   cudaError_t e = cudaErrorInvalidValue;
   switch (width / 128) {
-#define VLM_MERGE_CASE(nv) \
-  case nv: e = launch_pdl(merge_norm_kernel<nv>, dim3(grid), dim3(256), 0, s, x, g, info, cu, n_images, T, m, eps, z); break;
+#define VLM_MERGE_CASE(nv)                                                                                         \
+  case nv:                                                                                                         \
+    if (dev < 64 && !attr_done[dev][nv]) {                                                                         \
+      if (cudaFuncSetAttribute(merge_norm_kernel<nv>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMergeSmem) != \
+          cudaSuccess)                                                                                             \
+        break;                                                                                                     \
+      attr_done[dev][nv] = true;                                                                                   \
+    }                                                                                                              \
+    e = launch_pdl(merge_norm_kernel<nv>, dim3(static_cast<unsigned>(grid)), dim3(kMergeThreads), smem, s, x, g,  \
+                   info, cu, n_images, T, m, eps, rows, z, status);                                                \
+    break;
     VLM_MERGE_CASE(1) VLM_MERGE_CASE(2) VLM_MERGE_CASE(3) VLM_MERGE_CASE(4) VLM_MERGE_CASE(5)
     VLM_MERGE_CASE(6) VLM_MERGE_CASE(7) VLM_MERGE_CASE(8) VLM_MERGE_CASE(9) VLM_MERGE_CASE(10)
     VLM_MERGE_CASE(11) VLM_MERGE_CASE(12) VLM_MERGE_CASE(13) VLM_MERGE_CASE(14) VLM_MERGE_CASE(15)
@@ -759,17 +909,28 @@ int launch_rmsnorm_bf16(const __nv_bfloat16* x, const float* g, __nv_bfloat16* o
 
 int launch_scatter(const int64_t* ids, int64_t n, int64_t token, const void* img, int64_t n_img,
                    void* text, int64_t row_bytes, ScatterWs ws, int32_t* status, cudaStream_t s) {
-  if (n <= kScatterFusedMaxIds) {
+  const int ring = static_cast<int>(row_bytes > 0 ? std::min<int64_t>(kScatterRingMaxRows, kScatterRingBytes / row_bytes) : 0);
+  if (n <= kScatterFusedMaxIds && ring >= 2) {
     // one launch; the workspace is not used
     const int64_t slots = 2LL * num_sms();
     int64_t rows = n_img > n ? 1 : (n_img + slots - 1) / slots;  // more rows than ids can only mismatch
     rows = rows < 1 ? 1 : (rows > kScatterFusedMaxRows ? kScatterFusedMaxRows : rows);
     const int64_t grid = n_img > n ? 1 : (n_img + rows - 1) / rows;
+    const size_t smem = static_cast<size_t>(ring) * static_cast<size_t>(row_bytes);
+    static bool attr_done[64] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 64 && !attr_done[dev]) {
+      if (cudaFuncSetAttribute(scatter_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kScatterRingBytes) !=
+          cudaSuccess)
+        return VLM_ERR_CUDA;
+      attr_done[dev] = true;
+    }
     launch_begin(KC_SCATTER, s);
     const cudaError_t e = launch_pdl(scatter_fused_kernel, dim3(static_cast<unsigned>(grid < 1 ? 1 : grid)),
-                                     dim3(kScatterFusedThreads), 0, s, ids, static_cast<int>(n), token,
-                                     static_cast<const uint4*>(img), static_cast<uint4*>(text), n_img,
-                                     row_bytes / 16, static_cast<int>(rows), status);
+                                     dim3(kScatterFusedThreads), smem, s, ids, static_cast<int>(n), token,
+                                     static_cast<const uint8_t*>(img), static_cast<uint8_t*>(text), n_img, row_bytes,
+                                     static_cast<int>(rows), ring, status);
     launch_end(KC_SCATTER, s);
     return e == cudaSuccess ? VLM_OK : VLM_ERR_CUDA;
   }
