@@ -207,3 +207,20 @@ def test_other_widths_vs_oracle(width, heads, mlp, proj_out):
                                                 ocfg)
     compare(tower, ref_tower, what=f"tower width {width}")
     compare(emb, ref_emb, what=f"projector {width}->{proj_out}")
+
+
+def test_patch_gather_widths_off_the_16_byte_grid_vs_oracle():
+    """Patch 14 without a merge: image widths of 42 and 70 pixels (not multiples
+    of 4, so pixel rows are not 16-byte aligned) and patch rows of 3 and 5
+    patches (segments that end mid-vector) take the gather's scalar path."""
+    sizes = [(28, 42), (14, 70), (42, 28)]
+    cfg = vlm.preset("mistral3", layers=1, merge=1)
+    tw = synth.tower_weights(9, 1, cfg.width, cfg.mlp, cfg.patch)
+    pw = synth.projector_weights(9, cfg.width, 1, cfg.proj_out)
+    imgs = synth.images(9, sizes)
+    tower, emb = _run_gpu(cfg, tw, pw, imgs, sizes)
+    ocfg = dict(O.MISTRAL3, layers=1, merge=1)
+    ref_tower, ref_emb = O.encode_merge_project([im.double().numpy() for im in imgs], to_oracle(tw), to_oracle(pw), ocfg)
+    compare(tower, ref_tower, what="tower, widths off the 16-byte grid")
+    compare(emb, ref_emb, what="projector, widths off the 16-byte grid")
+
