@@ -151,6 +151,29 @@ VLM_API int vlm_gemm_nvfp4(int epilogue, const void* d_a, const void* d_a_sf, co
  * stays usable. Nothing faults, traps or hangs. */
 VLM_API int vlm_selftest_wait_timeout(int64_t budget_cycles, int32_t* d_status, void* stream);
 
+/* Debug build (no counterpart on the pages). The library can be compiled with
+ * -DVLM_DEBUG (libvlm_b200_debug.so, built beside the release library): every
+ * index that a kernel computes from tables or data before a global access --
+ * token positions, patch-gather items and pixel rows, merge destinations,
+ * scatter and expansion destinations, resize source rows, attention output
+ * rows -- is checked; a failing check records a code (source file id << 16 |
+ * line) in a device word and the access is skipped. Nothing traps. TMA
+ * transfers need no check: their tensor maps bound them.
+ *
+ * vlm_debug_build: 1 in a debug build, 0 otherwise (no CUDA call).
+ * vlm_debug_checks: synchronises the device, writes the first failing check's
+ *   code to *first_failure (0 when none failed) and clears the record.
+ *   VLM_OK in a debug build; VLM_ERR_UNSUPPORTED (and 0 written) otherwise;
+ *   VLM_ERR_CUDA if the record cannot be read.
+ * vlm_debug_selftest_bounds: debug builds only; threads i < 2n would write
+ *   d_buf[i] (int32) behind the check i < n, so the check must fail for
+ *   i >= n and leave d_buf[n .. 2n) untouched (d_buf holds 2n values,
+ *   1 <= n <= 2^20). Release builds return VLM_ERR_UNSUPPORTED and launch
+ *   nothing. */
+VLM_API int vlm_debug_build(void);
+VLM_API int vlm_debug_checks(int32_t* first_failure);
+VLM_API int vlm_debug_selftest_bounds(int32_t* d_buf, int n, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

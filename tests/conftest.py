@@ -11,6 +11,7 @@ if ROOT not in sys.path:
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a B200 (sm_100a) GPU and the built CUDA library")
     config.addinivalue_line("markers", "slow: takes more than a few seconds on the CPU")
+    config.addinivalue_line("markers", "debug_failure_expected: the test makes an index check fail on purpose")
 
 
 @pytest.fixture(autouse=True)
@@ -35,3 +36,8 @@ def _guard_bands(request):
         vlm.set_allocator(old)
         gpu_util._active_guard = None
     guard.check()
+    # under the index-checked debug build (VLM_B200_LIBRARY=libvlm_b200_debug.so)
+    # no check may have failed during the test
+    if vlm._lib is not None and vlm.debug_build() and not request.node.get_closest_marker("debug_failure_expected"):
+        code = vlm.debug_checks()
+        assert code == 0, f"index check failed in file {code >> 16}, line {code & 0xFFFF}"

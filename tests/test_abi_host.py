@@ -248,3 +248,29 @@ def test_gemm_tile_counts_that_overflow_32_bits_are_rejected(L):
     # NVFP4: 16.8M row groups x 16,384 scale atoms per row group
     assert L.vlm_gemm_nvfp4(vlm.EPI_BF16, fake, fake, fake, fake, fake, fake, big_m, 128, 1 << 20, fake, st,
                             None) == vlm.ERR_BAD_SHAPE
+
+
+def test_release_library_has_no_debug_checks(L):
+    """The release build compiles every index check out: it says so, reads no
+    device record, and refuses the deliberate-failure self-test before any
+    launch (a non-null pointer it never dereferences)."""
+    assert L.vlm_debug_build() == 0
+    code = ctypes.c_int32(77)
+    assert L.vlm_debug_checks(ctypes.byref(code)) == vlm.ERR_UNSUPPORTED and code.value == 0
+    assert L.vlm_debug_selftest_bounds(ctypes.c_void_p(256), 4, None) == vlm.ERR_UNSUPPORTED
+
+
+def test_debug_library_loads_and_exports_every_symbol():
+    """The index-checked build (-DVLM_DEBUG) sits beside the release library,
+    exports the same C ABI and identifies itself (no CUDA call needed)."""
+    path = vlm.DEBUG_LIB_PATH
+    if not os.path.exists(path):
+        from vision_language_model_b200 import build
+        build.build(debug=True)
+    D = ctypes.CDLL(path, mode=ctypes.RTLD_LOCAL)
+    for n in sorted(_declared()):
+        assert hasattr(D, n), n
+    D.vlm_debug_build.restype = ctypes.c_int
+    assert D.vlm_debug_build() == 1
+    D.vlm_debug_checks.restype = ctypes.c_int
+    assert D.vlm_debug_checks(None) == vlm.ERR_INVALID_ARG

@@ -122,3 +122,61 @@ def test_host_fed_steps_match_eager():
         assert torch.equal(out_host, t.cpu())
         results.append(out_host.clone())
     assert not torch.equal(results[0], results[1])
+
+
+def test_side_stream_runs_concurrently_and_matches_oracle():
+    """NEXT row 1 (the encoder on its own stream): two requests of one 896x1344
+    image (2 layers) submitted to the side stream while bf16 GEMMs run on the
+    caller's stream. The encoder's interval (side-stream events around each
+    request) and the other work's interval (caller-stream events) overlap in
+    time, and every scattered row equals the oracle's embedding to tolerance,
+    the other rows staying bit-identical."""
+    import numpy as np
+    from oracle import vlm_oracle as O
+    from tests.gpu_util import compare, to_oracle
+
+    sizes = [(896, 1344)]
+    cfg = vlm.preset("mistral3", layers=2)
+    tw = synth.tower_weights(13, 2, cfg.width, cfg.mlp, cfg.patch)
+    pw = synth.projector_weights(13, cfg.width, cfg.merge, cfg.proj_out)
+    pipe = vlm.ImagePipeline(cfg, tower_to_device(tw), tower_to_device(pw), sizes)
+    ids = synth.text_sequences(13, 1, 4096, [[1536]]).reshape(-1).cuda()
+    text0 = synth.text_embeddings(13, ids.numel(), cfg.proj_out).cuda()
+    images = [synth.images(s, sizes) for s in (14, 15)]
+    requests = [pixels_to_device(im) for im in images]
+
+    side = vlm.EncoderSideStream(pipe)
+    main = torch.cuda.current_stream()
+    a = torch.randn(4096, 4096, device="cuda", dtype=torch.bfloat16)
+    busy = torch.empty_like(a)
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+    ref = ev()
+    ref.record(main)
+    outs, spans = [], []
+    for pix in requests:
+        e0 = ev()
+        e0.record(main)  # the side stream waits on the caller's stream, so this precedes its work
+        side.ready = ev()  # a timing event, one per request, for the check below
+        side.submit(pix)
+        m0, m1 = ev(), ev()
+        m0.record(main)
+        for _ in range(12):  # other work on the caller's stream while the encoder runs
+            torch.matmul(a, a, out=busy)
+        m1.record(main)
+        t = text0.clone()
+        side.scatter(ids, t)
+        outs.append(t)
+        spans.append((e0, side.ready, m0, m1))
+    torch.cuda.synchronize()
+    assert vlm.status_sync(pipe.status) == vlm.OK
+    for e0, ready, m0, m1 in spans:
+        enc = (ref.elapsed_time(e0), ref.elapsed_time(ready))
+        other = (ref.elapsed_time(m0), ref.elapsed_time(m1))
+        assert enc[0] < other[1] and other[0] < enc[1], (enc, other)  # the two intervals overlap
+    mask = (ids == 10).cpu()
+    for got, im in zip(outs, images):
+        _, ref_emb = O.encode_merge_project([x.double().numpy() for x in im], to_oracle(tw), to_oracle(pw),
+                                           dict(O.MISTRAL3, layers=2))
+        compare(got[mask.cuda()], ref_emb, what="side-stream scattered rows")
+        assert torch.equal(got[~mask.cuda()].view(torch.int16), text0[~mask.cuda()].view(torch.int16))
+    assert not np.array_equal(outs[0].cpu().float().numpy(), outs[1].cpu().float().numpy())

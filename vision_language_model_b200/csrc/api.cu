@@ -934,6 +934,34 @@ int vlm_selftest_wait_timeout(int64_t budget_cycles, int32_t* d_status, void* st
   return launch_wait_timeout_selftest(budget_cycles, d_status, as_stream(stream));
 }
 
+int vlm_debug_build(void) {
+#ifdef VLM_DEBUG
+  return 1;
+#else
+  return 0;
+#endif
+}
+
+int vlm_debug_checks(int32_t* first_failure) {
+  if (first_failure == nullptr) return VLM_ERR_INVALID_ARG;
+  *first_failure = 0;
+#ifdef VLM_DEBUG
+  if (cudaDeviceSynchronize() != cudaSuccess) return VLM_ERR_CUDA;
+  const int words[3] = {debug_word_small_kernels(true), debug_word_frontend(true), debug_word_attention(true)};
+  for (int w : words) {
+    if (w < 0) return VLM_ERR_CUDA;
+    if (w != 0 && *first_failure == 0) *first_failure = w;
+  }
+  return VLM_OK;
+#else
+  return VLM_ERR_UNSUPPORTED;
+#endif
+}
+
+int vlm_debug_selftest_bounds(int32_t* d_buf, int n, void* stream) {
+  return launch_debug_selftest(d_buf, n, as_stream(stream));
+}
+
 int vlm_rmsnorm(float* d_x, const float* d_g0, const float* d_g1, void* d_out, int64_t rows, int width, float eps,
                 void* stream) {
   if (d_x == nullptr || d_g1 == nullptr || d_out == nullptr || rows < 0) return VLM_ERR_INVALID_ARG;

@@ -29,7 +29,11 @@
 #include "exp2_poly.cuh"
 #include "kernels.cuh"
 
+#define VLM_DEBUG_FILE_ID 3
+
 namespace vlm {
+
+VLM_DEBUG_UNIT(debug_word_attention)
 
 namespace {
 
@@ -369,7 +373,7 @@ __global__ void __launch_bounds__(192, 2)
         for (int c = 0; c < DH; c += 32) {
           uint32_t o[32];
           tmem_ld32(trow + kColO + c, o);
-          if (row < kend) {
+          if (row < kend && VLM_DCHECK(kend <= __ldg(args.cu + args.n_blocks))) {
             uint4* d4 = reinterpret_cast<uint4*>(dst + c);
 #pragma unroll
             for (int jj = 0; jj < 2; ++jj) {
@@ -388,7 +392,7 @@ __global__ void __launch_bounds__(192, 2)
       for (int c = 0; c < DH; c += 32) {
         uint32_t o[32];
         tmem_ld32(trow + kColO + c, o);
-        if (row < kend) {
+        if (row < kend && VLM_DCHECK(kend <= __ldg(args.cu + args.n_blocks))) {
           uint4* d4 = reinterpret_cast<uint4*>(dst + c);
 #pragma unroll
           for (int jj = 0; jj < 4; ++jj)

@@ -60,6 +60,35 @@ __device__ __forceinline__ void set_status(int32_t* status, int32_t code) {
   if (status) atomicCAS(status, 0, code);
 }
 
+// ---------------------------------------------------------------------------
+// Debug builds (compiled with -DVLM_DEBUG; libvlm_b200_debug.so): every
+// VLM_DCHECK(cond) on an index computed from tables or data records the first
+// failing check of its source file (file id << 16 | line) in that file's debug
+// word and evaluates to false, so the access it guards is skipped -- nothing
+// traps. vlm_debug_checks() reads and clears the words. In release builds a
+// check is the constant true and costs nothing. A file that uses the checks
+// defines VLM_DEBUG_FILE_ID and places VLM_DEBUG_UNIT(accessor) once, inside
+// namespace vlm, before its kernels.
+// ---------------------------------------------------------------------------
+#ifdef VLM_DEBUG
+#define VLM_DCHECK(cond)                                                                         \
+  (__builtin_expect(!!(cond), 1) ? true                                                          \
+                                 : (atomicCAS(&g_vlm_debug_word, 0, (VLM_DEBUG_FILE_ID << 16) | __LINE__), false))
+#define VLM_DEBUG_UNIT(accessor)                                                                  \
+  static __device__ int g_vlm_debug_word = 0;                                                     \
+  int accessor(bool clear) {                                                                      \
+    int v = 0;                                                                                    \
+    if (cudaMemcpyFromSymbol(&v, g_vlm_debug_word, sizeof(int)) != cudaSuccess) return -1;       \
+    const int zero = 0;                                                                           \
+    if (clear && cudaMemcpyToSymbol(g_vlm_debug_word, &zero, sizeof(int)) != cudaSuccess) return -1; \
+    return v;                                                                                     \
+  }
+#else
+#define VLM_DCHECK(cond) true
+#define VLM_DEBUG_UNIT(accessor) \
+  int accessor(bool) { return 0; }
+#endif
+
 // Spin budget of every wait on a barrier: ~1 s of SM clocks at 2 GHz.
 constexpr long long kWaitBudgetCycles = 2000000000LL;
 

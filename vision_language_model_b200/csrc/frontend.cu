@@ -4,7 +4,11 @@
 // image_token_id placeholders.
 #include "kernels.cuh"
 
+#define VLM_DEBUG_FILE_ID 2
+
 namespace vlm {
+
+VLM_DEBUG_UNIT(debug_word_frontend)
 
 // ---------------------------------------------------------------------------
 // Bilinear resize, u8 RGB HWC -> fp32 CHW in [0, 1], optionally tiled.
@@ -110,6 +114,8 @@ __global__ void __launch_bounds__(128) resize_tile_kernel(const uint8_t* __restr
     const Tap ty = make_tap(q, r, sh, ch.inv_den_y[b]);
     const int64_t img = ch.src_off[b];
     const int64_t row_bytes = 3LL * sw;
+    // both source rows of the unit lie inside its image (uniform over the CTA)
+    if (!VLM_DCHECK(ty.i0 >= 0 && ty.i1 < sh && img >= 0 && img + sh * row_bytes <= src_bytes)) continue;
     const uint8_t* r0;
     const uint8_t* r1;
     if constexpr (kStaged) {
@@ -220,7 +226,7 @@ __global__ void __launch_bounds__(256) expand_kernel(const int64_t* __restrict__
                                                      const int64_t* __restrict__ chunk_base,
                                                      const int64_t* __restrict__ prefix,
                                                      const int32_t* __restrict__ ok_flag, int64_t image_token,
-                                                     int64_t* __restrict__ out) {
+                                                     int64_t* __restrict__ out, int64_t n_out, int n_images) {
   griddep_wait();
   griddep_launch_dependents();
   if (*ok_flag == 0) return;
@@ -242,11 +248,15 @@ __global__ void __launch_bounds__(256) expand_kernel(const int64_t* __restrict__
   before += __popc(ballot & ((1u << lane) - 1u));
   const int64_t r = chunk_base[blockIdx.x] + before;  // markers before i
   if (i < n) {
-    const int64_t at = (i - r) + prefix[r];
+    // a marker's run is [at, at + len); another id lands at `at` (checked in debug builds)
+    const bool ok_r = VLM_DCHECK(r >= 0 && r + flag <= n_images);
+    const int64_t at = ok_r ? (i - r) + prefix[r] : 0;
+    const int64_t len = (ok_r && flag) ? prefix[r + 1] - prefix[r] : 0;
+    const bool ok = ok_r && VLM_DCHECK(at >= 0 && (flag ? at + len <= n_out : at < n_out));
     if (flag) {
       run_start[before] = at;
-      run_len[before] = prefix[r + 1] - prefix[r];
-    } else {
+      run_len[before] = ok ? len : 0;
+    } else if (ok) {
       out[at] = id;
     }
   }
@@ -281,7 +291,7 @@ int launch_expand(const int64_t* ids, int64_t n, int64_t marker, const int64_t* 
   if (rc == VLM_OK) rc = launch_marker_scan(ws.chunk_count, n_chunks, n_images, ws.chunk_base, ws.ok_flag, status, s);
   if (rc == VLM_OK &&
       launch_pdl(expand_kernel, dim3(static_cast<unsigned>(n_chunks)), dim3(256), 0, s, ids, n, marker,
-                 ws.chunk_base, ws.prefix, ws.ok_flag, image_token, out) != cudaSuccess)
+                 ws.chunk_base, ws.prefix, ws.ok_flag, image_token, out, n - n_images + acc, n_images) != cudaSuccess)
     rc = VLM_ERR_CUDA;
   launch_end(KC_EXPAND, s);
   note_extra_launches(launches + 2);

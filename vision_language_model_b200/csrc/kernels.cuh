@@ -74,6 +74,13 @@ constexpr int kAttnBQ = 128;
 
 void note_extra_launches(int n);
 
+// Debug words of the files with index checks (see VLM_DCHECK): the first
+// failing check's code or 0 (-1 if the read failed); `clear` resets the word.
+int debug_word_small_kernels(bool clear);
+int debug_word_frontend(bool clear);
+int debug_word_attention(bool clear);
+int launch_debug_selftest(int32_t* buf, int n, cudaStream_t s);
+
 int launch_setup(const ImageChunk& chunk, ImgInfo* info, int32_t* cu, int32_t* qt, int32_t* i2c, int32_t* pos,
                  int n_images, cudaStream_t s);
 int launch_rope_table(float theta, int head_dim, int max_pos, float2* tab, cudaStream_t s);

@@ -7,7 +7,11 @@
 
 #include "kernels.cuh"
 
+#define VLM_DEBUG_FILE_ID 1
+
 namespace vlm {
+
+VLM_DEBUG_UNIT(debug_word_small_kernels)
 
 // ---------------------------------------------------------------------------
 // Index setup: per-image tables and per-token (row, col) positions.
@@ -49,7 +53,7 @@ __global__ void setup_kernel(ImageChunk chunk, ImgInfo* info, int32_t* cu, int32
     }
     const int local = t - chunk.tok_off[lo];
     const int w = chunk.w[lo];
-    pos[t] = ((local / w) << 16) | (local % w);
+    if (VLM_DCHECK(local >= 0 && local < chunk.h[lo] * w)) pos[t] = ((local / w) << 16) | (local % w);
   }
 }
 
@@ -102,6 +106,7 @@ __global__ void im2col_kernel(const float* __restrict__ pix, const ImgInfo* __re
     const int b = find_block(cu, n_images, static_cast<int>(t));
     const ImgInfo in = info[b];
     const int local = static_cast<int>(t) - in.tok_off;
+    if (!VLM_DCHECK(local >= 0 && local < in.h * in.w && in.h * p <= in.H && in.w * p <= in.W)) continue;
     const int r = local / in.w, c = local % in.w;
     const float* base = pix + in.pix_off;
     uint32_t* orow = reinterpret_cast<uint32_t*>(out + t * kp);
@@ -145,6 +150,8 @@ __global__ void __launch_bounds__(kI2cThreads) im2col_tiled_kernel(const float* 
     const int nch = (in.w + kI2cPatches - 1) / kI2cPatches;
     const int local = g - __ldg(i2c + b);
     const int r = local / nch, c0 = (local - r * nch) * kI2cPatches;
+    // the item lies inside its image (the same decision in every thread of the CTA)
+    if (!VLM_DCHECK(local >= 0 && r < in.h && c0 < in.w && in.h * P <= in.H && in.w * P <= in.W)) continue;
     const int npat = min(kI2cPatches, in.w - c0), seg = npat * P;
     const float* base = pix + in.pix_off;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -384,7 +391,7 @@ __global__ void scatter_scan_kernel(const int32_t* __restrict__ chunk_count, int
 __global__ void scatter_positions_kernel(const int64_t* __restrict__ ids, int64_t n, int64_t token,
                                          const int64_t* __restrict__ chunk_base,
                                          const int32_t* __restrict__ ok_flag,
-                                         int64_t* __restrict__ dst_rows) {
+                                         int64_t* __restrict__ dst_rows, int64_t n_img) {
   griddep_wait();
   griddep_launch_dependents();
   if (*ok_flag == 0) return;
@@ -398,13 +405,16 @@ __global__ void scatter_positions_kernel(const int64_t* __restrict__ ids, int64_
   int before = 0;
   for (int w = 0; w < warp; ++w) before += s[w];
   before += __popc(ballot & ((1u << lane) - 1u));
-  if (flag) dst_rows[chunk_base[blockIdx.x] + before] = i;
+  if (flag) {
+    const int64_t k = chunk_base[blockIdx.x] + before;
+    if (VLM_DCHECK(k >= 0 && k < n_img)) dst_rows[k] = i;
+  }
 }
 
 __global__ void scatter_copy_kernel(const uint4* __restrict__ img, uint4* __restrict__ text,
                                     const int64_t* __restrict__ dst_rows,
                                     const int32_t* __restrict__ ok_flag, int64_t n_rows,
-                                    int64_t vec_per_row) {
+                                    int64_t vec_per_row, int64_t n_text) {
   griddep_wait();
   griddep_launch_dependents();
   if (*ok_flag == 0) return;
@@ -412,8 +422,10 @@ __global__ void scatter_copy_kernel(const uint4* __restrict__ img, uint4* __rest
   const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
   for (int64_t k = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); k < n_rows;
        k += warps) {
+    const int64_t d = dst_rows[k];
+    if (!VLM_DCHECK(d >= 0 && d < n_text)) continue;
     const uint4* src = img + k * vec_per_row;
-    uint4* dst = text + dst_rows[k] * vec_per_row;
+    uint4* dst = text + d * vec_per_row;
     int64_t j = lane;
     for (; j + 96 < vec_per_row; j += 128) {
       const uint4 a = __ldg(src + j), b = __ldg(src + j + 32), c = __ldg(src + j + 64), d = __ldg(src + j + 96);
@@ -559,7 +571,10 @@ __global__ void __launch_bounds__(kScatterFusedThreads)
   if (good) {
     for (int r = 0; r < n_rows; ++r) {
       if (!mbar_wait(smem_u32(s_full + r % ring), (r / ring) & 1, abort_v, status)) break;
-      bulk_store_row(text + s_dst[r] * row_bytes, smem_u32(s_ring + static_cast<size_t>(r % ring) * row_bytes), bytes);
+      if (VLM_DCHECK(s_dst[r] >= 0 && s_dst[r] < n)) {
+        bulk_store_row(text + s_dst[r] * row_bytes, smem_u32(s_ring + static_cast<size_t>(r % ring) * row_bytes),
+                       bytes);
+      }
       bulk_commit();
       done = r + 1;
       const int q = r - lag;  // its store is older than the newest `lag` ones
@@ -788,7 +803,8 @@ __global__ void __launch_bounds__(kMergeThreads, 3) merge_norm_kernel(const __nv
       const int local = t - in.tok_off;
       const int r = local / in.w, c = local % in.w;
       const int64_t mt = in.m_off + (r / m) * (in.w / m) + c / m;
-      dst[i] = (mt * m * m + (r % m) * m + c % m) * width;
+      if (VLM_DCHECK(local >= 0 && local < in.h * in.w && (mt + 1) * m * m <= T))
+        dst[i] = (mt * m * m + (r % m) * m + c % m) * width;
     }
   }
   float gv[NL][VE];
@@ -943,11 +959,11 @@ int launch_scatter(const int64_t* ids, int64_t n, int64_t token, const void* img
                    ws.ok_flag, status);
   if (e == cudaSuccess)
     e = launch_pdl(scatter_positions_kernel, chunks, dim3(256), 0, s, ids, n, token, ws.chunk_base, ws.ok_flag,
-                   ws.dst_rows);
+                   ws.dst_rows, n_img);
   const int64_t vec = row_bytes / 16;
   if (e == cudaSuccess)
     e = launch_pdl(scatter_copy_kernel, dim3(grid_for(n_img * 32, 256)), dim3(256), 0, s,
-                   static_cast<const uint4*>(img), static_cast<uint4*>(text), ws.dst_rows, ws.ok_flag, n_img, vec);
+                   static_cast<const uint4*>(img), static_cast<uint4*>(text), ws.dst_rows, ws.ok_flag, n_img, vec, n);
   launch_end(KC_SCATTER, s);
   note_extra_launches(3);
   return e == cudaSuccess ? VLM_OK : VLM_ERR_CUDA;
@@ -1014,6 +1030,27 @@ namespace vlm {
 // attention roles wait on theirs; the wait must give up, record
 // VLM_ERR_TIMEOUT in *status and let the kernel return normally.
 // ---------------------------------------------------------------------------
+// Debug builds only: threads i < 2n would write buf[i] behind the check i < n,
+// so the check fails for every i >= n, records its code and skips the write.
+// (Release builds never launch it: the entry point refuses first.)
+__global__ void debug_selftest_kernel(int32_t* buf, int n) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < 2 * n && VLM_DCHECK(i < n)) buf[i] = i + 1;
+}
+
+int launch_debug_selftest(int32_t* buf, int n, cudaStream_t s) {
+#ifdef VLM_DEBUG
+  if (buf == nullptr || n <= 0 || n > (1 << 20)) return VLM_ERR_INVALID_ARG;
+  debug_selftest_kernel<<<(2 * n + 255) / 256, 256, 0, s>>>(buf, n);
+  return cudaGetLastError() == cudaSuccess ? VLM_OK : VLM_ERR_CUDA;
+#else
+  (void)buf;
+  (void)n;
+  (void)s;
+  return VLM_ERR_UNSUPPORTED;
+#endif
+}
+
 __global__ void wait_timeout_selftest_kernel(long long budget_cycles, int32_t* status) {
   __shared__ __align__(8) uint64_t bar;
   if (threadIdx.x != 0) return;

@@ -12,7 +12,11 @@ import os
 
 import torch
 
-_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libvlm_b200.so")
+# VLM_B200_LIBRARY selects another build of the library, such as the
+# index-checked libvlm_b200_debug.so beside this file.
+_LIB_PATH = os.environ.get("VLM_B200_LIBRARY") or os.path.join(os.path.dirname(os.path.abspath(__file__)),
+                                                                "libvlm_b200.so")
+DEBUG_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libvlm_b200_debug.so")
 _lib = None
 
 # vlm_status values (include/vlm.h)
@@ -128,6 +132,9 @@ def lib() -> ctypes.CDLL:
             "vlm_attention": (I32, [P, I64, I32, I32, P, I32, P, P, SZ, P, P]),
             "vlm_rmsnorm": (I32, [P, P, P, P, I64, I32, F, P]),
             "vlm_selftest_wait_timeout": (I32, [I64, P, P]),
+            "vlm_debug_build": (I32, []),
+            "vlm_debug_checks": (I32, [ctypes.POINTER(ctypes.c_int32)]),
+            "vlm_debug_selftest_bounds": (I32, [P, I32, P]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -556,6 +563,25 @@ def rmsnorm(x: torch.Tensor, g1: torch.Tensor, g0=None, eps: float = 1e-5, out=N
 def selftest_wait_timeout(budget_cycles: int, status: torch.Tensor, stream=None) -> None:
     _check(lib().vlm_selftest_wait_timeout(int(budget_cycles), _dev(status, "status"), _stream(stream)),
            "vlm_selftest_wait_timeout")
+
+
+def debug_build() -> bool:
+    """True when the loaded library is the index-checked debug build."""
+    return bool(lib().vlm_debug_build())
+
+
+def debug_checks() -> int:
+    """Synchronises the device; the first failing index check's code
+    (file id << 16 | line), or 0, and clears the record (debug builds only)."""
+    code = ctypes.c_int32(0)
+    _check(lib().vlm_debug_checks(ctypes.byref(code)), "vlm_debug_checks")
+    return int(code.value)
+
+
+def debug_selftest_bounds(buf: torch.Tensor, n: int, stream=None) -> None:
+    """Debug builds: the deliberate out-of-range writes into buf[n:2n] are
+    caught by the index check and skipped."""
+    _check(lib().vlm_debug_selftest_bounds(_dev(buf, "buf"), int(n), _stream(stream)), "vlm_debug_selftest_bounds")
 
 
 # ---------------------------------------------------------------------------
