@@ -182,3 +182,40 @@ def test_tower_shapes_quantise_and_multiply_on_sampled_rows(N, K):
     exact = x32[rows].astype(np.float64) @ w32.astype(np.float64).T
     rel = np.abs(ref - exact).max() / np.abs(exact).max()
     assert 1e-3 < rel < 0.25, rel
+
+
+def _pow2_operand(rng, rows, k):
+    q = rng.choice(np.concatenate([_MAGS, -_MAGS[1:]]), size=(rows, k))
+    s = np.exp2(rng.integers(-2, 1, size=(rows, k // 16))).astype(np.float64)
+    return q, s
+
+
+@pytest.mark.parametrize("N,K", [(1024, 4096), (8192, 1024)])
+def test_gemm_nvfp4_exact_and_repeatable_at_tower_shapes(N, K):
+    """The tower's row count with a long K loop (16 stages of 256 values per
+    tile) and with many tiles: block scales in {1/4, 1/2, 1} keep every term a
+    multiple of 2^-6 of magnitude <= 36, so every partial sum over K <= 4096 is
+    exact in fp32 and sampled rows must equal the oracle bit for bit. A block
+    scale read from tensor memory before its copy has landed, or from another
+    stage's scale slot, breaks that; 20 further launches must agree bit for bit
+    with the first."""
+    rng = np.random.default_rng(N + 3 * K)
+    M = 12100
+    qa, sa = _pow2_operand(rng, M, K)
+    qb, sb = _pow2_operand(rng, N, K)
+    a, b = _operand(qa, sa, 1.0, K), _operand(qb, sb, 1.0, K)
+    out = guarded_zeros((M, N), dtype=torch.float32)
+    st = vlm.new_status()
+    vlm.gemm_nvfp4(vlm.EPI_RESID, a, b, out, status=st)
+    torch.cuda.synchronize()
+    assert vlm.status_sync(st) == vlm.OK
+    rows = np.sort(np.concatenate([rng.choice(M, 60, replace=False), [0, 127, 128, 255, 256, 12031, M - 1]]))
+    ref = O.nvfp4_linear(qa[rows], sa[rows], 1.0, qb, sb, 1.0)
+    np.testing.assert_array_equal(to_np(out[torch.from_numpy(rows).cuda()]), ref)
+    first = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    vlm.gemm_nvfp4(vlm.EPI_BF16, a, b, first, status=st)
+    again = torch.empty_like(first)
+    for _ in range(20):
+        vlm.gemm_nvfp4(vlm.EPI_BF16, a, b, again, status=st)
+        assert torch.equal(again, first)
+    assert vlm.status_sync(st) == vlm.OK

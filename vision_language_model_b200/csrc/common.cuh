@@ -220,6 +220,13 @@ __device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
+// Relaxed arrive, for hand-offs that order only tcgen05 accesses (through
+// tcgen05.fence::before_thread_sync before it and after_thread_sync behind the
+// wait) and publish no other memory: a release at cluster scope would also
+// hold the thread until its outstanding memory operations are visible.
+__device__ __forceinline__ void mbar_arrive_cluster_relaxed(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
 // try_wait with cluster-scope acquire, for barriers that CTAs of the cluster arrive on
 __device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity) {
   uint32_t ok;

@@ -588,7 +588,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
       epilogue_tile<S::BN, EPI, kF8>(args, st, tbase, mt * 256 + static_cast<int>(rank) * GBM + q * 32, nt * S::BN);
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(leader_tempty + static_cast<uint32_t>(acc * 8));
+      if (lane == 0) mbar_arrive_cluster_relaxed(leader_tempty + static_cast<uint32_t>(acc * 8));
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1u;
     }
@@ -657,20 +657,33 @@ int dispatch_pair_f8(int epi, const CUtensorMap& ta, const CUtensorMap& tb, cons
 // all BN columns of B (each CTA loads its own copy; no multicast). The even
 // CTA copies the atoms into tensor memory with tcgen05.cp (one
 // 32x128b.warpx4 copy per atom, into both CTAs' TMEM from each CTA's own
-// shared memory) just before the stage's MMAs. Copies and MMAs issued by one
-// thread run in order, so one scale region serves every stage. Per K = 64
-// step the A scales take 4 TMEM columns (row r's four scales sit in lane
-// r % 32 of every lane quarter, column (r % 128) / 32) and the B scales 4 per
-// 128 columns of the tile.
+// shared memory). Per K = 64 step the A scales take 4 TMEM columns (row r's
+// four scales sit in lane r % 32 of every lane quarter, column (r % 128) / 32)
+// and the B scales 4 per 128 columns of the tile.
+//
+// Each tcgen05 instruction costs its issuing thread close to a hundred cycles,
+// not far from what one K = 64 MMA of this shape takes on the tensor pipe
+// (128 cycles), so one thread issuing a stage's 4 MMAs and its 12 scale copies
+// cannot keep the pipe busy. The copies are therefore issued by copy warps of
+// the even CTA (two for A and two per 128 columns of B, two copies each), into
+// two scale slots used in turn. A copy followed by an MMA is a pipelined pair
+// of tcgen05 instructions: the MMA executes after the copy when it is issued
+// after it, and tcgen05.fence::before_thread_sync / after_thread_sync around
+// an mbarrier hand-off carry that issue order across threads. So a copy warp
+// arrives on sf_full[slot] as soon as its copies are issued, and the MMA
+// thread issues the stage's MMAs behind them without waiting for the copies
+// to complete. An MMA followed by a copy is not such a pair: a copy warp
+// refills a slot only once the MMAs that last read it have completed, which
+// their commit to empty[] signals. The MMA thread issues only MMAs and commits.
 //
 // TMEM (512 columns): BN = 128 keeps two 128-column accumulators side by side
-// and the scales behind them. BN = 256 would need 512 columns for two
-// accumulators alone, so the second one starts at column 192 and shares 64
-// columns with the first; the scales take columns 448..511. The epilogue
-// reads the shared 64 columns of a tile first and then signals `ovl`: the next
+// and the scale slots behind them. BN = 256 would need 512 columns for two
+// accumulators alone, so the second one starts at column 160 and shares 96
+// columns with the first; the scale slots take columns 416..511. The epilogue
+// reads the shared columns of a tile first and then signals `ovl`: the next
 // tile's MMAs (into the other accumulator) wait for that signal and for the
 // other accumulator's own release, so they start while the epilogue is still
-// working through the tile's other 192 columns.
+// working through the tile's other columns.
 // ---------------------------------------------------------------------------
 template <int BN_>
 struct Fp4Shape {
@@ -684,13 +697,21 @@ struct Fp4Shape {
   static constexpr int SFB_BYTES = SFB_BLOCKS * 4 * 512;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
   static constexpr int EPI_BYTES = kEpiWarps * kStageBufs * kStageBufBytes;
-  static constexpr int ACC_STRIDE = kOverlap ? 192 : BN;  // TMEM column of the second accumulator
-  static constexpr int SFA_COL = kOverlap ? 448 : 2 * BN;
-  static constexpr int SFB_COL = SFA_COL + 16;
+  static constexpr int ACC_STRIDE = kOverlap ? 160 : BN;  // TMEM column of the second accumulator
+  // Two scale slots used in turn: the copies of stage g + 1 fill one while the
+  // MMAs of stage g read the other. A slot holds 4 columns per K = 64 step for
+  // A and 4 per step per 128 columns of B.
+  static constexpr int SF_SLOT_COLS = 16 + 16 * SFB_BLOCKS;
+  static constexpr int SF_BASE = kOverlap ? 416 : 2 * BN;
   static constexpr int TMEM_COLS = 512;
+  // copy warps of the even CTA: two for the A scales and two per 128-column
+  // group of B, each issuing the copies of two K = 64 steps
+  static constexpr int COPY_WARPS = 2 * (1 + SFB_BLOCKS);
+  static constexpr int THREADS = 192 + 32 * COPY_WARPS;
   static constexpr int BAR_BYTES = 256;
   static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + EPI_BYTES + BAR_BYTES + 1024;
-  static_assert(SFB_COL + 16 * SFB_BLOCKS <= TMEM_COLS, "scale columns past the allocation");
+  static_assert(SF_BASE + 2 * SF_SLOT_COLS <= TMEM_COLS, "scale columns past the allocation");
+  static_assert(!kOverlap || SF_BASE >= ACC_STRIDE + BN, "scale slots overlap the second accumulator");
   static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
 };
 
@@ -726,11 +747,13 @@ __device__ __forceinline__ void umma_nvfp4_pair(uint32_t d_tmem, uint64_t a_desc
 
 // This warp's 32 rows of a 128 x BN tile held at TMEM address tbase, scaled by
 // alpha: bf16 stores, or an fp32 bulk reduce-add into c. Chunks start at tile
-// column `first` and wrap around; after the chunks covering the first 64
-// columns have been read from TMEM, on_first64() runs.
-template <int EPI, int BN, typename F>
+// column `first` and wrap around; after the chunks covering the first SHARED
+// columns have been read from TMEM, on_shared() runs.
+template <int EPI, int BN, int SHARED, typename F>
 __device__ __forceinline__ void epilogue_nvfp4(Stager& st, uint32_t tbase, int row0, int n0, int first, float alpha,
-                                               F&& on_first64) {
+                                               F&& on_shared) {
+  static_assert(SHARED % 64 == 0 || EPI != VLM_EPI_BF16, "bf16 chunks are 64 columns");
+  static_assert(SHARED % 32 == 0 && SHARED > 0 && SHARED <= BN, "shared columns");
   if constexpr (EPI == VLM_EPI_BF16) {
 #pragma unroll 1
     for (int i = 0; i < BN / 64; ++i) {
@@ -738,7 +761,7 @@ __device__ __forceinline__ void epilogue_nvfp4(Stager& st, uint32_t tbase, int r
       uint32_t a[32], b[32], w[32];
       tmem_ld32(tbase + c, a);
       tmem_ld32(tbase + c + 32, b);
-      if (i == 0) on_first64();
+      if (i == SHARED / 64 - 1) on_shared();
 #pragma unroll
       for (int j = 0; j < 16; ++j) {
         w[j] = pack_bf16x2(__uint_as_float(a[2 * j]) * alpha, __uint_as_float(a[2 * j + 1]) * alpha);
@@ -754,7 +777,7 @@ __device__ __forceinline__ void epilogue_nvfp4(Stager& st, uint32_t tbase, int r
       const int c = (first + 32 * i) % BN;
       uint32_t a[32];
       tmem_ld32(tbase + c, a);
-      if (i == 1) on_first64();
+      if (i == SHARED / 32 - 1) on_shared();
 #pragma unroll
       for (int j = 0; j < 32; ++j) a[j] = __float_as_uint(__uint_as_float(a[j]) * alpha);
       uint8_t* buf = st.acquire();
@@ -765,11 +788,15 @@ __device__ __forceinline__ void epilogue_nvfp4(Stager& st, uint32_t tbase, int r
 }
 
 template <int EPI, int BN>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Fp4Shape<BN>::THREADS, 1)
     gemm_nvfp4_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                            const __grid_constant__ CUtensorMap tmSFA, const __grid_constant__ CUtensorMap tmSFB,
                            const __grid_constant__ CUtensorMap tmC, const GemmArgs args) {
   using S = Fp4Shape<BN>;
+  // columns each epilogue warp reads before the shared ones are free (64-column bf16 chunks, 32-column fp32 ones)
+  constexpr int kShared = EPI == VLM_EPI_BF16 ? 128 : 96;
+  static_assert(!S::kOverlap || (S::BN - S::ACC_STRIDE <= kShared && S::ACC_STRIDE >= S::BN - kShared),
+                "the first columns read must cover the shared ones");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
@@ -783,7 +810,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
   uint64_t* tfull = bars + 2 * S::STAGES;    // both CTAs
   uint64_t* tempty = tfull + 2;              // used on the even CTA (8 warp arrivals)
   uint64_t* ovl = tempty + 2;                // used on the even CTA (8 warp arrivals)
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ovl + 1);
+  uint64_t* sf_full = ovl + 1;               // used on the even CTA (copies issued into a scale slot)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sf_full + 2);
   int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -803,6 +831,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
       mbar_init(smem_u32(tempty + a), 2 * kEpiWarps);
     }
     mbar_init(smem_u32(ovl), 2 * kEpiWarps);
+    for (int b = 0; b < 2; ++b) mbar_init(smem_u32(sf_full + b), S::COPY_WARPS);  // one arrival per copy warp
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -855,40 +884,35 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
   } else if (warp == 1) {
     if (rank == 0 && lane == 0) {
       constexpr uint32_t idesc = idesc_nvfp4(2 * GBM, S::BN);
-      const uint32_t sfa_t = tmem_base + S::SFA_COL, sfb_t = tmem_base + S::SFB_COL;
       int stage = 0;
-      uint32_t phase = 0;
+      uint32_t g = 0;  // stages consumed so far: scale slot g & 1, its use (g >> 1)
       int acc = 0;
       uint32_t acc_phase = 0, ovl_phase = 0;
       bool ok = true;
       for (int tile = pair; tile < total_tiles && ok; tile += n_pairs) {
         if (!mbar_wait_cluster(smem_u32(tempty + acc), acc_phase ^ 1u, abort_v, args.status)) break;
         if constexpr (S::kOverlap) {
-          // the previous tile's epilogue has read the 64 columns both accumulators share
+          // the previous tile's epilogue has read the columns both accumulators share
           if (!mbar_wait_cluster(smem_u32(ovl), ovl_phase ^ 1u, abort_v, args.status)) break;
           ovl_phase ^= 1u;
         }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * S::ACC_STRIDE);
         for (int kb = 0; kb < nk; ++kb) {
-          if (!mbar_wait(smem_u32(full + stage), phase, abort_v, args.status)) { ok = false; break; }
+          // the copy warps arrive on sf_full only after they have seen the stage's operands land (full)
+          if (!mbar_wait(smem_u32(sf_full + (g & 1u)), (g >> 1) & 1u, abort_v, args.status)) { ok = false; break; }
           tc_fence_after();
           const uint64_t adesc = smem_desc_sw128(smem_u32(sA + stage * S::A_BYTES));
           const uint64_t bdesc = smem_desc_sw128(smem_u32(sB + stage * S::B_BYTES));
-          const uint32_t sfa_s = smem_u32(sSFA + stage * S::SFA_BYTES), sfb_s = smem_u32(sSFB + stage * S::SFB_BYTES);
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            tmem_cp_atom_pair(sfa_t + 4 * k, smem_desc_sf_atom(sfa_s + 512 * k));
-#pragma unroll
-            for (int j = 0; j < S::SFB_BLOCKS; ++j)
-              tmem_cp_atom_pair(sfb_t + 4 * (S::SFB_BLOCKS * k + j), smem_desc_sf_atom(sfb_s + 2048 * j + 512 * k));
-          }
+          const uint32_t sfa_t = tmem_base + S::SF_BASE + (g & 1u) * S::SF_SLOT_COLS, sfb_t = sfa_t + 16;
 #pragma unroll
           for (int k = 0; k < 4; ++k)  // 32 bytes (64 values) of K per instruction
             umma_nvfp4_pair(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, sfa_t + 4 * k,
                             sfb_t + 4 * S::SFB_BLOCKS * k, (kb | k) != 0 ? 1u : 0u);
+          // completes when the MMAs have read the stage's operands and its scale slot
           umma_commit_pair_mc(smem_u32(empty + stage), 0x3);
-          if (++stage == S::STAGES) { stage = 0; phase ^= 1u; }
+          ++g;
+          if (++stage == S::STAGES) stage = 0;
         }
         if (!ok) break;
         umma_commit_pair_mc(smem_u32(tfull + acc), 0x3);
@@ -896,7 +920,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
         if (acc == 0) acc_phase ^= 1u;
       }
     }
-  } else {
+  } else if (warp < 2 + kEpiWarps) {
     const int q = warp & 3;  // TMEM lane quadrant this warp may access
     Stager st{sEpi + (warp - 2) * kStageBufs * kStageBufBytes, &tmC, 0, lane};
     const uint32_t leader_tempty = mapa_shared(smem_u32(tempty), 0);
@@ -910,23 +934,63 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
       tc_fence_after();
       const uint32_t tbase =
           tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * S::ACC_STRIDE);
-      // the shared columns are tile columns 192..255 of the first accumulator and 0..63 of the second
-      const int first = S::kOverlap && acc == 0 ? 192 : 0;
-      epilogue_nvfp4<EPI, S::BN>(st, tbase, mt * 256 + static_cast<int>(rank) * GBM + q * 32, nt * S::BN, first,
-                                 alpha, [&] {
+      // the shared columns are tile columns ACC_STRIDE..BN-1 of the first
+      // accumulator and 0..BN-ACC_STRIDE-1 of the second; each is read first
+      const int first = S::kOverlap && acc == 0 ? S::BN - kShared : 0;
+      epilogue_nvfp4<EPI, S::BN, kShared>(st, tbase, mt * 256 + static_cast<int>(rank) * GBM + q * 32, nt * S::BN,
+                                          first, alpha, [&] {
                                    if constexpr (S::kOverlap) {
                                      tc_fence_before();
                                      __syncwarp();
-                                     if (lane == 0) mbar_arrive_cluster(leader_ovl);
+                                     if (lane == 0) mbar_arrive_cluster_relaxed(leader_ovl);
                                    }
                                  });
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(leader_tempty + static_cast<uint32_t>(acc * 8));
+      if (lane == 0) mbar_arrive_cluster_relaxed(leader_tempty + static_cast<uint32_t>(acc * 8));
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1u;
     }
     st.drain();
+  } else if (rank == 0 && lane == 0) {
+    // copy warp c: K = 64 steps 2 (c & 1) and 2 (c & 1) + 1 of the A scales
+    // (c < 2) or of the B scales of 128-column group c / 2 - 1
+    const int c = warp - 2 - kEpiWarps;
+    const int grp = c >> 1, k0 = 2 * (c & 1);
+    int stage = 0;
+    uint32_t phase = 0;
+    uint32_t g = 0;  // stages filled so far
+    bool ok = true;
+    for (int tile = pair; tile < total_tiles && ok; tile += n_pairs) {
+      for (int kb = 0; kb < nk; ++kb) {
+        if (!mbar_wait(smem_u32(full + stage), phase, abort_v, args.status)) { ok = false; break; }
+        if (g >= 2) {  // the slot's previous reader, stage g - 2, has completed its MMAs
+          const uint32_t h = g - 2;
+          if (!mbar_wait(smem_u32(empty + h % S::STAGES), (h / S::STAGES) & 1u, abort_v, args.status)) {
+            ok = false;
+            break;
+          }
+        }
+        tc_fence_after();
+        const uint32_t slot = tmem_base + S::SF_BASE + (g & 1u) * S::SF_SLOT_COLS;
+        if (grp == 0) {
+          const uint32_t sfa_s = smem_u32(sSFA + stage * S::SFA_BYTES);
+#pragma unroll
+          for (int k = k0; k < k0 + 2; ++k) tmem_cp_atom_pair(slot + 4 * k, smem_desc_sf_atom(sfa_s + 512 * k));
+        } else {
+          const int j = grp - 1;
+          const uint32_t sfb_s = smem_u32(sSFB + stage * S::SFB_BYTES + 2048 * j);
+#pragma unroll
+          for (int k = k0; k < k0 + 2; ++k)
+            tmem_cp_atom_pair(slot + 16 + 4 * (S::SFB_BLOCKS * k + j), smem_desc_sf_atom(sfb_s + 512 * k));
+        }
+        // issued, not completed: the MMAs that read the slot are issued behind these copies
+        tc_fence_before();
+        mbar_arrive(smem_u32(sf_full + (g & 1u)));
+        ++g;
+        if (++stage == S::STAGES) { stage = 0; phase ^= 1u; }
+      }
+    }
   }
 
   tc_fence_before();
@@ -954,7 +1018,8 @@ int run_gemm_nvfp4(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorM
   const int tiles = args.m_tiles * args.n_tiles;
   const int pairs = tiles < num_sms() / 2 ? tiles : num_sms() / 2;
   launch_begin(KC_GEMM, s);
-  const cudaError_t e = launch_pdl(kern, dim3(2 * pairs), dim3(192), S::SMEM_BYTES, s, ta, tb, tsa, tsb, tc, args);
+  const cudaError_t e =
+      launch_pdl(kern, dim3(2 * pairs), dim3(S::THREADS), S::SMEM_BYTES, s, ta, tb, tsa, tsb, tc, args);
   launch_end(KC_GEMM, s);
   return e == cudaSuccess ? VLM_OK : VLM_ERR_CUDA;
 }
