@@ -745,41 +745,105 @@ __device__ __forceinline__ void umma_nvfp4_pair(uint32_t d_tmem, uint64_t a_desc
       : "memory");
 }
 
-// This warp's 32 rows of a 128 x BN tile held at TMEM address tbase, scaled by
-// alpha: bf16 stores, or an fp32 bulk reduce-add into c. Chunks start at tile
-// column `first` and wrap around; after the chunks covering the first SHARED
-// columns have been read from TMEM, on_shared() runs.
-template <int EPI, int BN, int SHARED, typename F>
-__device__ __forceinline__ void epilogue_nvfp4(Stager& st, uint32_t tbase, int row0, int n0, int first, float alpha,
-                                               F&& on_shared) {
-  static_assert(SHARED % 64 == 0 || EPI != VLM_EPI_BF16, "bf16 chunks are 64 columns");
-  static_assert(SHARED % 32 == 0 && SHARED > 0 && SHARED <= BN, "shared columns");
-  if constexpr (EPI == VLM_EPI_BF16) {
-#pragma unroll 1
-    for (int i = 0; i < BN / 64; ++i) {
-      const int c = (first + 64 * i) % BN;
-      uint32_t a[32], b[32], w[32];
-      tmem_ld32(tbase + c, a);
-      tmem_ld32(tbase + c + 32, b);
-      if (i == SHARED / 64 - 1) on_shared();
+// 32 accumulator columns (fp32 bits) scaled by alpha, as 16 packed bf16 pairs at w[OFF..OFF+15].
+template <int OFF, int N>
+__device__ __forceinline__ void pack_scaled16(const uint32_t (&a)[32], uint32_t (&w)[N], float alpha) {
 #pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        w[j] = pack_bf16x2(__uint_as_float(a[2 * j]) * alpha, __uint_as_float(a[2 * j + 1]) * alpha);
-        w[16 + j] = pack_bf16x2(__uint_as_float(b[2 * j]) * alpha, __uint_as_float(b[2 * j + 1]) * alpha);
+  for (int j = 0; j < 16; ++j)
+    w[OFF + j] = pack_bf16x2(__uint_as_float(a[2 * j]) * alpha, __uint_as_float(a[2 * j + 1]) * alpha);
+}
+__device__ __forceinline__ void scale32(uint32_t (&a)[32], float alpha) {
+#pragma unroll
+  for (int j = 0; j < 32; ++j) a[j] = __float_as_uint(__uint_as_float(a[j]) * alpha);
+}
+
+// This warp's 32 rows of a 128 x BN tile held at TMEM address tbase, scaled by
+// alpha: bf16 stores (64-column chunks), or an fp32 bulk reduce-add into c
+// (32-column chunks). With overlapping accumulators (kOverlap: BN = 256, the
+// second accumulator 160 columns after the first) the 96 columns both share --
+// tile columns 160..255 of accumulator 0, 0..95 of accumulator 1 -- are read
+// from TMEM first and held in registers; on_shared() then releases them to
+// the next tile's MMAs before any of them is stored.
+template <int EPI, int BN, bool kOverlap, typename F>
+__device__ __forceinline__ void epilogue_nvfp4(Stager& st, uint32_t tbase, int row0, int n0, int acc, float alpha,
+                                               F&& on_shared) {
+  static_assert(!kOverlap || BN == 256, "the overlap layout is for 256-column tiles");
+  if constexpr (EPI == VLM_EPI_BF16) {
+    int c_rest = 0;  // first of the chunks outside the shared columns
+    if constexpr (kOverlap) {
+      // the shared columns: one whole chunk (cp) and one half of another (ch + ho)
+      const int cp = acc == 0 ? 192 : 0, ch = acc == 0 ? 128 : 64, ho = acc == 0 ? 32 : 0;
+      uint32_t a[32], wp[32], wh[16];
+      tmem_ld32(tbase + cp, a);
+      pack_scaled16<0>(a, wp, alpha);
+      tmem_ld32(tbase + cp + 32, a);
+      pack_scaled16<16>(a, wp, alpha);
+      tmem_ld32(tbase + ch + ho, a);
+      pack_scaled16<0>(a, wh, alpha);
+      on_shared();
+      uint8_t* buf = st.acquire();
+      st.write_row(buf, wp);
+      st.commit(buf, n0 + cp, row0);
+      // the chunk with one shared half
+      tmem_ld32(tbase + ch + (32 - ho), a);
+      uint32_t w[32];
+      if (ho == 0) {
+#pragma unroll
+        for (int j = 0; j < 16; ++j) w[j] = wh[j];
+        pack_scaled16<16>(a, w, alpha);
+      } else {
+        pack_scaled16<0>(a, w, alpha);
+#pragma unroll
+        for (int j = 0; j < 16; ++j) w[16 + j] = wh[j];
       }
+      buf = st.acquire();
+      st.write_row(buf, w);
+      st.commit(buf, n0 + ch, row0);
+      c_rest = acc == 0 ? 0 : 128;
+    }
+    constexpr int kRest = kOverlap ? 2 : BN / 64;
+#pragma unroll 1
+    for (int i = 0; i < kRest; ++i) {
+      const int c = c_rest + 64 * i;
+      uint32_t a[32], w[32];
+      tmem_ld32(tbase + c, a);
+      pack_scaled16<0>(a, w, alpha);
+      tmem_ld32(tbase + c + 32, a);
+      pack_scaled16<16>(a, w, alpha);
       uint8_t* buf = st.acquire();
       st.write_row(buf, w);
       st.commit(buf, n0 + c, row0);
     }
   } else {
+    int c_rest = 0;
+    if constexpr (kOverlap) {
+      const int cs = acc == 0 ? 160 : 0;  // the three shared 32-column chunks
+      uint32_t a0[32], a1[32], a2[32];
+      tmem_ld32(tbase + cs, a0);
+      tmem_ld32(tbase + cs + 32, a1);
+      tmem_ld32(tbase + cs + 64, a2);
+      on_shared();
+      scale32(a0, alpha);
+      uint8_t* buf = st.acquire();
+      st.write_row(buf, a0);
+      st.template commit<true>(buf, n0 + cs, row0);
+      scale32(a1, alpha);
+      buf = st.acquire();
+      st.write_row(buf, a1);
+      st.template commit<true>(buf, n0 + cs + 32, row0);
+      scale32(a2, alpha);
+      buf = st.acquire();
+      st.write_row(buf, a2);
+      st.template commit<true>(buf, n0 + cs + 64, row0);
+      c_rest = acc == 0 ? 0 : 96;
+    }
+    constexpr int kRest = kOverlap ? 5 : BN / 32;
 #pragma unroll 1
-    for (int i = 0; i < BN / 32; ++i) {
-      const int c = (first + 32 * i) % BN;
+    for (int i = 0; i < kRest; ++i) {
+      const int c = c_rest + 32 * i;
       uint32_t a[32];
       tmem_ld32(tbase + c, a);
-      if (i == SHARED / 32 - 1) on_shared();
-#pragma unroll
-      for (int j = 0; j < 32; ++j) a[j] = __float_as_uint(__uint_as_float(a[j]) * alpha);
+      scale32(a, alpha);
       uint8_t* buf = st.acquire();
       st.write_row(buf, a);
       st.template commit<true>(buf, n0 + c, row0);
@@ -793,10 +857,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Fp4Shape<BN>::THREAD
                            const __grid_constant__ CUtensorMap tmSFA, const __grid_constant__ CUtensorMap tmSFB,
                            const __grid_constant__ CUtensorMap tmC, const GemmArgs args) {
   using S = Fp4Shape<BN>;
-  // columns each epilogue warp reads before the shared ones are free (64-column bf16 chunks, 32-column fp32 ones)
-  constexpr int kShared = EPI == VLM_EPI_BF16 ? 128 : 96;
-  static_assert(!S::kOverlap || (S::BN - S::ACC_STRIDE <= kShared && S::ACC_STRIDE >= S::BN - kShared),
-                "the first columns read must cover the shared ones");
+  static_assert(!S::kOverlap || S::ACC_STRIDE == 160, "the epilogue reads the shared columns 160..255 / 0..95");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
@@ -934,11 +995,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Fp4Shape<BN>::THREAD
       tc_fence_after();
       const uint32_t tbase =
           tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * S::ACC_STRIDE);
-      // the shared columns are tile columns ACC_STRIDE..BN-1 of the first
-      // accumulator and 0..BN-ACC_STRIDE-1 of the second; each is read first
-      const int first = S::kOverlap && acc == 0 ? S::BN - kShared : 0;
-      epilogue_nvfp4<EPI, S::BN, kShared>(st, tbase, mt * 256 + static_cast<int>(rank) * GBM + q * 32, nt * S::BN,
-                                          first, alpha, [&] {
+      epilogue_nvfp4<EPI, S::BN, S::kOverlap>(st, tbase, mt * 256 + static_cast<int>(rank) * GBM + q * 32,
+                                              nt * S::BN, acc, alpha, [&] {
                                    if constexpr (S::kOverlap) {
                                      tc_fence_before();
                                      __syncwarp();
