@@ -196,6 +196,44 @@ VLM_API int vlm_encode_fp8(const vlm_config* cfg, const float* pixels, const int
                            size_t ws_bytes, int32_t* d_status, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * vlm_encode_nvfp4 -- vlm_encode with the four tower GEMMs (QKV, O, gate/up,
+ * down) on NVFP4 operands (E2M1 values, one E4M3 scale per 16 values of a
+ * row along K, one fp32 global scale per tensor) with fp32 accumulation
+ * (tcgen05.mma kind::mxf4nvf4, block16), for the NVFP4 checkpoints the
+ * deployments load ([I] "Why this one is smaller than it looks", the
+ * quantisation loaders). Patch embed, norms, RoPE, attention (bf16 q, k, v)
+ * and the residual stream are as in vlm_encode.
+ *
+ * Quantisation (reading; the pages name the format, not a recipe):
+ *   - a block of 16 fp32 values x with global scale s_g:
+ *     s_b = E4M3(fp32(amax_b / fp32(6 s_g))), q = E2M1(fp32(x *
+ *     fp32(1 / fp32(s_b s_g)))) (q = 0 when s_b is 0), each rounding to
+ *     nearest even with saturation;
+ *   - weights: s_g = fp32(amax(W) / 2688) over the weight the GEMM executes
+ *     ([Wq; Wk; Wv] and [W_gate; W_up] as one tensor each);
+ *   - activations: one static s_g per GEMM input, block scales from the data;
+ *     act_scales is host fp32 [layers][4] = the global scales of the
+ *     attention-norm output, the attention output, the MLP-norm output and
+ *     the gated hidden state, each > 0; every input is quantised from fp32
+ *     inside the kernel that produces it;
+ *   - a GEMM result is acc * fp32(s_g(A) * s_g(W)).
+ *
+ * vlm_pack_tower_nvfp4: quantises the bf16 weights of vlm_tower_weights (same
+ *   meaning as for vlm_pack_tower) into d_packed (device, 256-byte aligned, at
+ *   least vlm_tower_nvfp4_packed_bytes) and stores act_scales beside them.
+ * vlm_encode_nvfp4: act_scales must be the array the tower was packed with.
+ *   d_workspace: 256-byte aligned, at least vlm_encode_nvfp4_workspace_size.
+ * Requires width % 256 == 0 and mlp % 256 == 0 (else VLM_ERR_UNSUPPORTED).
+ * ------------------------------------------------------------------------- */
+VLM_API size_t vlm_tower_nvfp4_packed_bytes(const vlm_config* cfg);
+VLM_API int vlm_pack_tower_nvfp4(const vlm_config* cfg, const vlm_tower_weights* w, const float* act_scales,
+                                 void* d_packed, size_t packed_bytes, void* stream);
+VLM_API size_t vlm_encode_nvfp4_workspace_size(const vlm_config* cfg, const int32_t* image_hw, int n_images);
+VLM_API int vlm_encode_nvfp4(const vlm_config* cfg, const float* pixels, const int32_t* image_hw, int n_images,
+                             const void* d_packed_tower_nvfp4, const float* act_scales, void* d_out,
+                             void* d_workspace, size_t ws_bytes, int32_t* d_status, void* stream);
+
+/* ---------------------------------------------------------------------------
  * vlm_merge_project -- the patch-merging projector ([K] Mistral3Model: 2x2
  * patch-merging projector, spatial_merge_size, projector_bias False):
  * RMSNorm per patch, m x m unfold + concat, merge linear (m*m*D -> D), then

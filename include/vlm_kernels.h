@@ -143,6 +143,46 @@ VLM_API int vlm_gemm_nvfp4(int epilogue, const void* d_a, const void* d_a_sf, co
                            const void* d_b_sf, const float* d_gb, int64_t M, int64_t N, int64_t K, void* d_c,
                            int32_t* d_status, void* stream);
 
+/* vlm_gemm_nvfp4 with the two tower epilogues of vlm_encode_nvfp4, both for
+ * N % 256 == 0:
+ * ROPE: d_c bf16 [M, N]; the 2D rotary embedding (as vlm_gemm's ROPE: d_pos
+ *   int32 [M] = row << 16 | col, d_rope from vlm_rope_table) rotates columns
+ *   below rope_cols (a multiple of 64), pair (i, i + 32) of every 64.
+ * SWIGLU: accumulator columns 32g..32g+15 are gate and 32g+16..32g+31 up of
+ *   hidden columns 16g..16g+15; h = silu(gate) * up in fp32 is quantised to
+ *   NVFP4 with global scale out_sg > 0 as vlm_quant_nvfp4 does: d_c codes
+ *   [M, N/4] bytes, d_c_sf block scales of an [M, N/2] operand (4-byte
+ *   aligned; scales of rows >= M are not written).
+ * BF16 and RESID as vlm_gemm_nvfp4 (d_c_sf, out_sg, d_pos, d_rope unused). */
+VLM_API int vlm_gemm_nvfp4_ex(int epilogue, const void* d_a, const void* d_a_sf, const float* d_ga, const void* d_b,
+                              const void* d_b_sf, const float* d_gb, int64_t M, int64_t N, int64_t K, void* d_c,
+                              void* d_c_sf, float out_sg, const int32_t* d_pos, const void* d_rope, int64_t rope_cols,
+                              int32_t* d_status, void* stream);
+
+/* The first steps of vlm_encode alone: index setup, the normalising patch
+ * gather and the patch-embed GEMM ([K] Mistral3VisionModel: conv patch
+ * embed), d_x = fp32 [T, width] patch features before ln_pre. d_packed_tower:
+ * any packed tower (vlm_pack_tower, _fp8 or _nvfp4: each starts with w_pe).
+ * d_workspace: 256-byte aligned, at least vlm_encode_workspace_size bytes. */
+VLM_API int vlm_patch_embed(const vlm_config* cfg, const float* pixels, const int32_t* image_hw, int n_images,
+                            const void* d_packed_tower, float* d_x, void* d_workspace, size_t ws_bytes,
+                            int32_t* d_status, void* stream);
+
+/* vlm_rmsnorm whose output is NVFP4: the fp32 values norm(.) * g1 quantised
+ * with global scale s_global > 0 as vlm_quant_nvfp4 does; d_q codes
+ * [rows, width/2], d_sf vlm_nvfp4_sf_bytes(rows, width) bytes (scales of the
+ * padding rows are not written). */
+VLM_API int vlm_rmsnorm_nvfp4(float* d_x, const float* d_g0, const float* d_g1, void* d_q, void* d_sf, int64_t rows,
+                              int width, float eps, float s_global, void* stream);
+
+/* vlm_attention whose output is NVFP4: the fp32 attention output quantised
+ * with global scale s_global > 0 as vlm_quant_nvfp4 does; d_q codes
+ * [T, heads * 32] (16-byte aligned), d_sf vlm_nvfp4_sf_bytes(T, heads * 64)
+ * bytes (scales of the padding rows are not written). */
+VLM_API int vlm_attention_nvfp4(const void* d_qkv, int64_t T, int heads, int head_dim, const int32_t* cu_seqlens,
+                                int n_blocks, void* d_q, void* d_sf, float s_global, void* d_workspace,
+                                size_t ws_bytes, int32_t* d_status, void* stream);
+
 /* Failure-detection self-test (no counterpart on the pages): launches one
  * thread that waits on a shared-memory mbarrier nothing arrives on, using the
  * same bounded wait as every barrier wait of the GEMM and attention kernels,

@@ -630,6 +630,25 @@ def tower_block_nvfp4(x: np.ndarray, lq: dict, act_scales, angles: np.ndarray, c
     return x + _nvfp4_gemm(silu(gu[:, :f]) * gu[:, f:], lq, "down", act_scales[3])
 
 
+def tower_nvfp4(images, tw: dict, act_scales, cfg: dict, layers: int | None = None,
+                normalize: bool = True) -> np.ndarray:
+    """tower() with tower_block_nvfp4 blocks; act_scales[l] holds layer l's four
+    static activation global scales, the weights are quantised per layer as
+    quantize_layer_nvfp4 does."""
+    p, eps = cfg["patch"], cfg["eps"]
+    n_layers = cfg["layers"] if layers is None else layers
+    grids = [patch_grid(im.shape[1], im.shape[2], p) for im in images]
+    rows, cols, cu = positions(grids)
+    w_pe = np.asarray(tw["w_pe"], dtype=np.float64)
+    x = np.concatenate([patch_embed(normalize_pixels(im) if normalize else np.asarray(im, np.float64), w_pe)
+                        for im in images], axis=0)
+    x = rms_norm(x, tw["g_pre"], eps)
+    angles = rope_angles(rows, cols, cfg["rope_theta"], cfg["head_dim"])
+    for layer in range(n_layers):
+        x = tower_block_nvfp4(x, quantize_layer_nvfp4(layer_weights(tw, layer)), act_scales[layer], angles, cu, cfg)
+    return x
+
+
 # ---------------------------------------------------------------------------
 # a12..a14: patch-merging projector
 # ---------------------------------------------------------------------------

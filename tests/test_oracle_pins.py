@@ -890,3 +890,45 @@ def test_planted_nvfp4_act_scales_swapped_is_caught(monkeypatch):
     monkeypatch.setattr(O, "tower_block_nvfp4", bad)
     with pytest.raises(AssertionError):
         test_tower_block_nvfp4_scales_feed_the_right_gemms()
+
+
+def _identity_nvfp4(monkeypatch):
+    """Quantisation switched off: codes = the fp32 values, every scale 1."""
+    monkeypatch.setattr(O, "quantize_nvfp4",
+                        lambda x, g: (np.asarray(x, np.float32).astype(np.float64),
+                                      np.ones((np.shape(x)[0], np.shape(x)[1] // 16))))
+    monkeypatch.setattr(O, "nvfp4_global_scale", lambda w: np.float32(1.0))
+
+
+def _nvfp4_tower_setup():
+    cfg = dict(O.MISTRAL3, layers=2, width=64, heads=1, head_dim=64, mlp=128)
+    tw = {k: v.double().numpy() for k, v in synth.tower_weights(4, 2, 64, 128, 14).items()}
+    imgs = [synth.pixels_u01(4, f"nvfp4tower{i}", h, w).double().numpy()
+            for i, (h, w) in enumerate([(28, 42), (14, 28)])]
+    return cfg, tw, imgs
+
+
+def test_tower_nvfp4_without_quantisation_is_the_tower(monkeypatch):
+    """With quantisation switched off (codes = the fp32 values, unit block and
+    global scales) tower_nvfp4 must be the pinned tower() -- same patch embed,
+    ln_pre, blocks and positions -- up to the fp32 rounding of each GEMM input;
+    with it on, it must differ by NVFP4's error and no more."""
+    cfg, tw, imgs = _nvfp4_tower_setup()
+    ref = O.tower(imgs, tw, cfg)
+    quant = O.tower_nvfp4(imgs, tw, [NVFP4_ACT] * 2, cfg)
+    err_q = np.abs(quant - ref).max() / np.abs(ref).max()
+    assert 1e-3 < err_q < 0.2, err_q
+    _identity_nvfp4(monkeypatch)
+    got = O.tower_nvfp4(imgs, tw, [(1.0, 1.0, 1.0, 1.0)] * 2, cfg)
+    np.testing.assert_allclose(got, ref, rtol=0, atol=1e-5 * np.abs(ref).max())
+
+
+def test_planted_nvfp4_tower_without_ln_pre_is_caught(monkeypatch):
+    cfg, tw, imgs = _nvfp4_tower_setup()
+    ref = O.tower(imgs, tw, cfg)
+    _identity_nvfp4(monkeypatch)
+    g_pre = tw["g_pre"]
+    real = O.rms_norm
+    monkeypatch.setattr(O, "rms_norm", lambda x, g, eps: np.asarray(x, np.float64) if g is g_pre else real(x, g, eps))
+    got = O.tower_nvfp4(imgs, tw, [(1.0, 1.0, 1.0, 1.0)] * 2, cfg)
+    assert np.abs(got - ref).max() > 1e-2 * np.abs(ref).max()

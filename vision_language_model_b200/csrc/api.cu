@@ -259,6 +259,42 @@ TowerF8Layout tower_f8_layout(const vlm_config* c) {
 // fp32(1 / s) of a static activation scale, computed in double.
 inline float inv_scale(float s) { return static_cast<float>(1.0 / static_cast<double>(s)); }
 
+// Packed NVFP4 tower layout (byte offsets): w_pe and g_pre as in the bf16
+// layout; per layer the four GEMM weights as E2M1 codes (the executed row
+// orders: [Wq; Wk; Wv], Wo, gate / up interleaved, W_down) with their block
+// scales, the four weight global scales, the four activation global scales
+// (device copies of act_scales, the GEMMs' A-operand scales) and the gains.
+struct TowerF4Layout {
+  size_t w_pe, g_pre, layer0, layer_stride;
+  size_t qkv, qkv_sf, o, o_sf, gu, gu_sf, down, down_sf, gw, act, g_attn, g_ffn;
+  size_t total;
+};
+
+TowerF4Layout tower_f4_layout(const vlm_config* c) {
+  TowerF4Layout L;
+  const int64_t D = c->width, F = c->mlp;
+  size_t off = 0;
+  L.w_pe = off; off = align_up(off + D * kpad(c->patch) * 2, 256);
+  L.g_pre = off; off = align_up(off + D * 4, 256);
+  L.layer0 = off;
+  size_t lo = 0;
+  L.qkv = lo; lo = align_up(lo + 3 * D * D / 2, 256);
+  L.qkv_sf = lo; lo = align_up(lo + nvfp4_sf_bytes(3 * D, D), 256);
+  L.o = lo; lo = align_up(lo + D * D / 2, 256);
+  L.o_sf = lo; lo = align_up(lo + nvfp4_sf_bytes(D, D), 256);
+  L.gu = lo; lo = align_up(lo + 2 * F * D / 2, 256);
+  L.gu_sf = lo; lo = align_up(lo + nvfp4_sf_bytes(2 * F, D), 256);
+  L.down = lo; lo = align_up(lo + D * F / 2, 256);
+  L.down_sf = lo; lo = align_up(lo + nvfp4_sf_bytes(D, F), 256);
+  L.gw = lo; lo = align_up(lo + 4 * 4, 256);
+  L.act = lo; lo = align_up(lo + 4 * 4, 256);
+  L.g_attn = lo; lo = align_up(lo + D * 4, 256);
+  L.g_ffn = lo; lo = align_up(lo + D * 4, 256);
+  L.layer_stride = lo;
+  L.total = off + lo * static_cast<size_t>(c->layers);
+  return L;
+}
+
 int check_act_scales(const vlm_config* c, const float* act) {
   if (act == nullptr) return VLM_ERR_INVALID_ARG;
   for (int i = 0; i < 4 * c->layers; ++i)
@@ -302,6 +338,29 @@ EncodeWs carve_encode(void* ws, const vlm_config* c, const Batch& b) {
   e.cols = e.hbuf;  // the patch gather is consumed before the first MLP
   e.used = align_up(cv.used, 256);
   return e;
+}
+
+// The NVFP4 encode: the bf16 workspace (its bf16 buffers hold the E2M1 codes
+// of the GEMM inputs) plus the block scales of the three quantised inputs.
+struct EncodeF4Ws {
+  EncodeWs e;
+  uint8_t *xn_sf, *attn_sf, *h_sf;
+  size_t sf_bytes_d, sf_bytes_f;
+  size_t used;
+};
+
+EncodeF4Ws carve_encode_f4(void* ws, const vlm_config* c, const Batch& b) {
+  EncodeF4Ws f;
+  f.e = carve_encode(ws, c, b);
+  Carver cv(ws);
+  cv.used = f.e.used;
+  f.sf_bytes_d = nvfp4_sf_bytes(b.T, c->width);
+  f.sf_bytes_f = nvfp4_sf_bytes(b.T, c->mlp);
+  f.xn_sf = cv.take<uint8_t>(f.sf_bytes_d);
+  f.attn_sf = cv.take<uint8_t>(f.sf_bytes_d);
+  f.h_sf = cv.take<uint8_t>(f.sf_bytes_f);
+  f.used = align_up(cv.used, 256);
+  return f;
 }
 
 struct ProjWs {
@@ -620,6 +679,146 @@ int vlm_encode_fp8(const vlm_config* cfg, const float* pixels, const int32_t* im
   return VLM_OK;
 }
 
+int vlm_patch_embed(const vlm_config* cfg, const float* pixels, const int32_t* image_hw, int n_images,
+                    const void* d_packed_tower, float* d_x, void* d_workspace, size_t ws_bytes, int32_t* d_status,
+                    void* stream) {
+  VLM_TRY(check_config(cfg));
+  if (pixels == nullptr || d_packed_tower == nullptr || d_x == nullptr || d_workspace == nullptr)
+    return VLM_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(d_workspace) & 255) return VLM_ERR_INVALID_ARG;
+  Batch b;
+  VLM_TRY(make_batch(cfg, image_hw, n_images, &b));
+  const EncodeWs e = carve_encode(d_workspace, cfg, b);
+  if (ws_bytes < e.used) return VLM_ERR_WORKSPACE;
+  cudaStream_t s = as_stream(stream);
+  const int64_t T = b.T, D = cfg->width, kp = kpad(cfg->patch);
+  // every packed tower layout starts with w_pe at offset 0
+  const uint8_t* w_pe = static_cast<const uint8_t*>(d_packed_tower) + tower_layout(cfg).w_pe;
+  VLM_TRY(upload_batch(b, e.bd, s));
+  VLM_TRY(launch_im2col(pixels, e.bd.info, e.bd.cu, e.bd.i2c, b.i2c_items, b.n, T, cfg->patch,
+                        static_cast<int>(kp), cfg->normalize, e.cols, s));
+  return launch_gemm(VLM_EPI_F32, e.cols, w_pe, T, D, kp, d_x, nullptr, nullptr, nullptr, 0, d_status, s);
+}
+
+size_t vlm_tower_nvfp4_packed_bytes(const vlm_config* cfg) {
+  return check_config(cfg) == VLM_OK ? tower_f4_layout(cfg).total : 0;
+}
+
+int vlm_pack_tower_nvfp4(const vlm_config* cfg, const vlm_tower_weights* w, const float* act_scales,
+                         void* d_packed, size_t packed_bytes, void* stream) {
+  VLM_TRY(check_config(cfg));
+  if (w == nullptr || d_packed == nullptr || !w->w_pe || !w->g_pre) return VLM_ERR_INVALID_ARG;
+  if (cfg->layers > 0 && (!w->wq || !w->wk || !w->wv || !w->wo || !w->w_gate || !w->w_up || !w->w_down ||
+                          !w->g_attn || !w->g_ffn))
+    return VLM_ERR_INVALID_ARG;
+  VLM_TRY(check_act_scales(cfg, act_scales));
+  if (cfg->mlp % 256 || cfg->width % 256) return VLM_ERR_UNSUPPORTED;
+  if (reinterpret_cast<uintptr_t>(d_packed) & 255) return VLM_ERR_INVALID_ARG;
+  const TowerF4Layout L = tower_f4_layout(cfg);
+  if (packed_bytes < L.total) return VLM_ERR_WORKSPACE;
+  cudaStream_t s = as_stream(stream);
+  uint8_t* dst = static_cast<uint8_t*>(d_packed);
+  const int64_t D = cfg->width, F = cfg->mlp;
+  const int p = cfg->patch;
+  constexpr float kFp4Range = 6.0f * 448.0f;  // largest E2M1 value times largest E4M3 block scale
+  VLM_TRY(launch_pack_cols(w->w_pe, dst + L.w_pe, D, 3 * p * p, kpad(p), 0, 1, s));
+  if (cudaMemcpyAsync(dst + L.g_pre, w->g_pre, D * 4, cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+    return VLM_ERR_CUDA;
+  for (int l = 0; l < cfg->layers; ++l) {
+    uint8_t* ly = dst + L.layer0 + L.layer_stride * l;
+    float* gw = reinterpret_cast<float*>(ly + L.gw);
+    auto at = [&](const void* base, int64_t elems) { return static_cast<const uint8_t*>(base) + l * elems * 2; };
+    // [Wq; Wk; Wv] under one global scale; each part fills whole 128-row scale groups
+    const void* qkv_parts[3] = {at(w->wq, D * D), at(w->wk, D * D), at(w->wv, D * D)};
+    const int64_t dd[3] = {D * D, D * D, D * D};
+    VLM_TRY(launch_amax_scale_multi(qkv_parts, dd, 3, 0, kFp4Range, gw + 0, s));
+    for (int j = 0; j < 3; ++j)
+      VLM_TRY(launch_quant_nvfp4(qkv_parts[j], 0, D, D, gw + 0, ly + L.qkv + j * D * D / 2,
+                                 ly + L.qkv_sf + j * nvfp4_sf_bytes(D, D), s));
+    VLM_TRY(launch_amax_scale(at(w->wo, D * D), 0, D * D, kFp4Range, gw + 1, s));
+    VLM_TRY(launch_quant_nvfp4(at(w->wo, D * D), 0, D, D, gw + 1, ly + L.o, ly + L.o_sf, s));
+    const void* gu_parts[2] = {at(w->w_gate, F * D), at(w->w_up, F * D)};
+    const int64_t fd[2] = {F * D, F * D};
+    VLM_TRY(launch_amax_scale_multi(gu_parts, fd, 2, 0, kFp4Range, gw + 2, s));
+    VLM_TRY(launch_quant_nvfp4_rows(gu_parts[0], gu_parts[1], 0, 2 * F, D, gw + 2, ly + L.gu, ly + L.gu_sf, s));
+    VLM_TRY(launch_amax_scale(at(w->w_down, D * F), 0, D * F, kFp4Range, gw + 3, s));
+    VLM_TRY(launch_quant_nvfp4(at(w->w_down, D * F), 0, D, F, gw + 3, ly + L.down, ly + L.down_sf, s));
+    bool ok = cudaMemcpyAsync(ly + L.act, act_scales + 4 * l, 4 * 4, cudaMemcpyHostToDevice, s) == cudaSuccess;
+    ok = ok && cudaMemcpyAsync(ly + L.g_attn, w->g_attn + l * D, D * 4, cudaMemcpyDeviceToDevice, s) == cudaSuccess;
+    ok = ok && cudaMemcpyAsync(ly + L.g_ffn, w->g_ffn + l * D, D * 4, cudaMemcpyDeviceToDevice, s) == cudaSuccess;
+    if (!ok) return VLM_ERR_CUDA;
+  }
+  return VLM_OK;
+}
+
+size_t vlm_encode_nvfp4_workspace_size(const vlm_config* cfg, const int32_t* image_hw, int n_images) {
+  if (check_config(cfg) != VLM_OK) return 0;
+  Batch b;
+  if (make_batch(cfg, image_hw, n_images, &b) != VLM_OK) return 0;
+  return carve_encode_f4(nullptr, cfg, b).used;
+}
+
+int vlm_encode_nvfp4(const vlm_config* cfg, const float* pixels, const int32_t* image_hw, int n_images,
+                     const void* d_packed_tower_nvfp4, const float* act_scales, void* d_out, void* d_workspace,
+                     size_t ws_bytes, int32_t* d_status, void* stream) {
+  VLM_TRY(check_config(cfg));
+  if (pixels == nullptr || d_packed_tower_nvfp4 == nullptr || d_out == nullptr || d_workspace == nullptr)
+    return VLM_ERR_INVALID_ARG;
+  VLM_TRY(check_act_scales(cfg, act_scales));
+  if (cfg->mlp % 256 || cfg->width % 256) return VLM_ERR_UNSUPPORTED;
+  if ((reinterpret_cast<uintptr_t>(d_workspace) & 255) || (reinterpret_cast<uintptr_t>(d_packed_tower_nvfp4) & 255))
+    return VLM_ERR_INVALID_ARG;
+  Batch b;
+  VLM_TRY(make_batch(cfg, image_hw, n_images, &b));
+  const EncodeF4Ws f = carve_encode_f4(d_workspace, cfg, b);
+  if (ws_bytes < f.used) return VLM_ERR_WORKSPACE;
+  const EncodeWs& e = f.e;
+  cudaStream_t s = as_stream(stream);
+  const TowerF4Layout L = tower_f4_layout(cfg);
+  const uint8_t* pk = static_cast<const uint8_t*>(d_packed_tower_nvfp4);
+  const int64_t T = b.T, D = cfg->width, F = cfg->mlp, kp = kpad(cfg->patch);
+  uint8_t* xn_q = reinterpret_cast<uint8_t*>(e.xn);
+  uint8_t* attn_q = reinterpret_cast<uint8_t*>(e.attn);
+  uint8_t* h_q = reinterpret_cast<uint8_t*>(e.hbuf);
+
+  // the producers write the scales of real rows only: padding rows keep scale 0
+  bool ok = cudaMemsetAsync(f.xn_sf, 0, f.sf_bytes_d, s) == cudaSuccess;
+  ok = ok && cudaMemsetAsync(f.attn_sf, 0, f.sf_bytes_d, s) == cudaSuccess;
+  ok = ok && cudaMemsetAsync(f.h_sf, 0, f.sf_bytes_f, s) == cudaSuccess;
+  if (!ok) return VLM_ERR_CUDA;
+  VLM_TRY(upload_batch(b, e.bd, s));
+  VLM_TRY(launch_rope_table(cfg->rope_theta, cfg->head_dim, b.max_pos, e.bd.rope, s));
+  VLM_TRY(launch_im2col(pixels, e.bd.info, e.bd.cu, e.bd.i2c, b.i2c_items, b.n, T, cfg->patch,
+                        static_cast<int>(kp), cfg->normalize, e.cols, s));
+  VLM_TRY(launch_gemm(VLM_EPI_F32, e.cols, pk + L.w_pe, T, D, kp, e.x, nullptr, nullptr, nullptr, 0, d_status, s));
+  for (int l = 0; l < cfg->layers; ++l) {
+    const uint8_t* ly = pk + L.layer0 + L.layer_stride * l;
+    const float* act = act_scales + 4 * l;                       // host copies: kernel arguments
+    const float* act_d = reinterpret_cast<const float*>(ly + L.act);  // device copies: GEMM A scales
+    const float* gw = reinterpret_cast<const float*>(ly + L.gw);
+    auto f32 = [&](size_t off) { return reinterpret_cast<const float*>(ly + off); };
+    const float* g0 = l == 0 ? reinterpret_cast<const float*>(pk + L.g_pre) : nullptr;
+    VLM_TRY(launch_rmsnorm_nvfp4(e.x, g0, f32(L.g_attn), xn_q, f.xn_sf, T, static_cast<int>(D), cfg->eps, act[0], s));
+    VLM_TRY(launch_gemm_nvfp4_ex(VLM_EPI_ROPE, xn_q, f.xn_sf, act_d + 0, ly + L.qkv, ly + L.qkv_sf, gw + 0, T, 3 * D,
+                                 D, e.qkv, nullptr, 1.f, e.bd.pos, e.bd.rope, 2 * D, d_status, s));
+    VLM_TRY(launch_attention(e.qkv, T, cfg->heads, e.bd.cu, e.bd.qt, b.n, b.total_qtiles, attn_q, d_status, s,
+                             act[1], f.attn_sf));
+    VLM_TRY(launch_gemm_nvfp4(VLM_EPI_RESID, attn_q, f.attn_sf, act_d + 1, ly + L.o, ly + L.o_sf, gw + 1, T, D, D,
+                              e.x, d_status, s));
+    VLM_TRY(launch_rmsnorm_nvfp4(e.x, nullptr, f32(L.g_ffn), xn_q, f.xn_sf, T, static_cast<int>(D), cfg->eps, act[2],
+                                 s));
+    VLM_TRY(launch_gemm_nvfp4_ex(VLM_EPI_SWIGLU, xn_q, f.xn_sf, act_d + 2, ly + L.gu, ly + L.gu_sf, gw + 2, T, 2 * F,
+                                 D, h_q, f.h_sf, act[3], nullptr, nullptr, 0, d_status, s));
+    VLM_TRY(launch_gemm_nvfp4(VLM_EPI_RESID, h_q, f.h_sf, act_d + 3, ly + L.down, ly + L.down_sf, gw + 3, T, D, F,
+                              e.x, d_status, s));
+  }
+  if (cfg->layers == 0)
+    VLM_TRY(launch_rmsnorm(e.x, reinterpret_cast<const float*>(pk + L.g_pre),
+                           reinterpret_cast<const float*>(pk + L.g_pre), e.xn, T, static_cast<int>(D), cfg->eps, s));
+  VLM_TRY(launch_f32_to_bf16(e.x, static_cast<__nv_bfloat16*>(d_out), T * D, s));
+  return VLM_OK;
+}
+
 size_t vlm_merge_project_workspace_size(const vlm_config* cfg, const int32_t* image_hw, int n_images) {
   if (check_config(cfg) != VLM_OK) return 0;
   Batch b;
@@ -879,6 +1078,26 @@ int vlm_gemm_nvfp4(int epilogue, const void* d_a, const void* d_a_sf, const floa
                            d_c, d_status, as_stream(stream));
 }
 
+int vlm_gemm_nvfp4_ex(int epilogue, const void* d_a, const void* d_a_sf, const float* d_ga, const void* d_b,
+                      const void* d_b_sf, const float* d_gb, int64_t M, int64_t N, int64_t K, void* d_c, void* d_c_sf,
+                      float out_sg, const int32_t* d_pos, const void* d_rope, int64_t rope_cols, int32_t* d_status,
+                      void* stream) {
+  return launch_gemm_nvfp4_ex(epilogue, static_cast<const uint8_t*>(d_a), static_cast<const uint8_t*>(d_a_sf), d_ga,
+                              static_cast<const uint8_t*>(d_b), static_cast<const uint8_t*>(d_b_sf), d_gb, M, N, K,
+                              d_c, static_cast<uint8_t*>(d_c_sf), out_sg, d_pos, static_cast<const float2*>(d_rope),
+                              rope_cols, d_status, as_stream(stream));
+}
+
+int vlm_rmsnorm_nvfp4(float* d_x, const float* d_g0, const float* d_g1, void* d_q, void* d_sf, int64_t rows,
+                      int width, float eps, float s_global, void* stream) {
+  if (d_x == nullptr || d_g1 == nullptr || d_q == nullptr || d_sf == nullptr || rows < 0 || !(s_global > 0.f) ||
+      !(s_global < 3.0e38f))
+    return VLM_ERR_INVALID_ARG;
+  if (rows == 0) return VLM_OK;
+  return launch_rmsnorm_nvfp4(d_x, d_g0, d_g1, static_cast<uint8_t*>(d_q), static_cast<uint8_t*>(d_sf), rows, width,
+                              eps, s_global, as_stream(stream));
+}
+
 int vlm_rope_table(float theta, int head_dim, int max_pos, void* d_table, void* stream) {
   if (d_table == nullptr || head_dim != 64 || max_pos <= 0 || !(theta > 0.f)) return VLM_ERR_INVALID_ARG;
   return launch_rope_table(theta, head_dim, max_pos, static_cast<float2*>(d_table), as_stream(stream));
@@ -889,8 +1108,10 @@ size_t vlm_attention_workspace_size(int n_blocks) {
   return align_up(static_cast<size_t>(n_blocks) * sizeof(ImgInfo), 256) + 2 * align_up((n_blocks + 1) * 4, 256);
 }
 
-int vlm_attention(const void* d_qkv, int64_t T, int heads, int head_dim, const int32_t* cu_seqlens, int n_blocks,
-                  void* d_out, void* d_workspace, size_t ws_bytes, int32_t* d_status, void* stream) {
+namespace {
+int attention_host_blocks(const void* d_qkv, int64_t T, int heads, int head_dim, const int32_t* cu_seqlens,
+                          int n_blocks, void* d_out, void* d_workspace, size_t ws_bytes, int32_t* d_status,
+                          void* stream, float f8_scale, uint8_t* out_sf) {
   if (d_qkv == nullptr || d_out == nullptr || cu_seqlens == nullptr || d_workspace == nullptr || n_blocks <= 0 ||
       heads <= 0)
     return VLM_ERR_INVALID_ARG;
@@ -926,7 +1147,23 @@ int vlm_attention(const void* d_qkv, int64_t T, int heads, int head_dim, const i
   cudaStream_t s = as_stream(stream);
   VLM_TRY(upload_batch(b, d, s));
   return launch_attention(static_cast<const __nv_bfloat16*>(d_qkv), T, heads, d.cu, d.qt, n_blocks,
-                          static_cast<int>(qt), static_cast<__nv_bfloat16*>(d_out), d_status, s);
+                          static_cast<int>(qt), d_out, d_status, s, f8_scale, out_sf);
+}
+}  // namespace
+
+int vlm_attention(const void* d_qkv, int64_t T, int heads, int head_dim, const int32_t* cu_seqlens, int n_blocks,
+                  void* d_out, void* d_workspace, size_t ws_bytes, int32_t* d_status, void* stream) {
+  return attention_host_blocks(d_qkv, T, heads, head_dim, cu_seqlens, n_blocks, d_out, d_workspace, ws_bytes,
+                               d_status, stream, 0.f, nullptr);
+}
+
+int vlm_attention_nvfp4(const void* d_qkv, int64_t T, int heads, int head_dim, const int32_t* cu_seqlens,
+                        int n_blocks, void* d_q, void* d_sf, float s_global, void* d_workspace, size_t ws_bytes,
+                        int32_t* d_status, void* stream) {
+  if (d_sf == nullptr || !(s_global > 0.f) || !(s_global < 3.0e38f)) return VLM_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(d_q) & 15) || (reinterpret_cast<uintptr_t>(d_sf) & 1)) return VLM_ERR_INVALID_ARG;
+  return attention_host_blocks(d_qkv, T, heads, head_dim, cu_seqlens, n_blocks, d_q, d_workspace, ws_bytes, d_status,
+                               stream, s_global, static_cast<uint8_t*>(d_sf));
 }
 
 int vlm_selftest_wait_timeout(int64_t budget_cycles, int32_t* d_status, void* stream) {

@@ -28,6 +28,7 @@
 // straddle two blocks, so every block's result is independent of the others.
 #include "exp2_poly.cuh"
 #include "kernels.cuh"
+#include "nvfp4.cuh"
 
 #define VLM_DEBUG_FILE_ID 3
 
@@ -180,12 +181,14 @@ struct AttnArgs {
   const int32_t* qt;
   int n_blocks;
   int heads;
-  void* out;        // bf16, or E4M3 when kF8Out
+  void* out;        // bf16; E4M3 (OUT 1); NVFP4 codes (OUT 2)
   int32_t* status;
-  float f8_scale;   // E4M3 output: O / l times this before rounding
+  float f8_scale;   // E4M3 output: O / l times this before rounding; NVFP4: the global scale
+  uint8_t* out_sf;  // NVFP4 block scales
 };
 
-template <bool kF8Out>
+// OUT: 0 bf16, 1 E4M3, 2 NVFP4 output.
+template <int OUT>
 __global__ void __launch_bounds__(192, 2)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, const AttnArgs args) {
   extern __shared__ uint8_t smem_raw[];
@@ -366,7 +369,34 @@ __global__ void __launch_bounds__(192, 2)
       tc_fence_after();
       const float inv = 1.0f / l;
       const int row = q0 + r;
-      if constexpr (kF8Out) {
+      if constexpr (OUT == 2) {
+        // blocks of 16 values along the row: four per head, two per 32-column load
+        uint8_t* dst = static_cast<uint8_t*>(args.out) + static_cast<int64_t>(row) * (D / 2) + h * (DH / 2);
+        const float sg = args.f8_scale, six_sg = 6.0f * sg;
+#pragma unroll
+        for (int c = 0; c < DH; c += 32) {
+          uint32_t o[32];
+          tmem_ld32(trow + kColO + c, o);
+          if (row < kend && VLM_DCHECK(kend <= __ldg(args.cu + args.n_blocks))) {
+            uint32_t sbs = 0;
+            uint2 codes[2];
+#pragma unroll
+            for (int b = 0; b < 2; ++b) {
+              float v[16], amax = 0.0f;
+#pragma unroll
+              for (int k = 0; k < 16; ++k) {
+                v[k] = __uint_as_float(o[16 * b + k]) * inv;
+                amax = fmaxf(amax, fabsf(v[k]));
+              }
+              sbs |= nvfp4_quant16(v, amax, sg, six_sg, codes[b]) << (8 * b);
+            }
+            *reinterpret_cast<uint4*>(dst + c / 2) = make_uint4(codes[0].x, codes[0].y, codes[1].x, codes[1].y);
+            // blocks (h DH + c) / 16 and the next: two adjacent scale bytes
+            *reinterpret_cast<uint16_t*>(args.out_sf + nvfp4_sf_offset(row, (h * DH + c) / 16, D)) =
+                static_cast<uint16_t>(sbs);
+          }
+        }
+      } else if constexpr (OUT == 1) {
         const float f = inv * args.f8_scale;
         uint8_t* dst = static_cast<uint8_t*>(args.out) + static_cast<int64_t>(row) * D + h * DH;
 #pragma unroll
@@ -417,7 +447,8 @@ __global__ void __launch_bounds__(192, 2)
 }  // namespace
 
 int launch_attention(const __nv_bfloat16* qkv, int64_t T, int heads, const int32_t* cu, const int32_t* qt,
-                     int n_blocks, int total_qtiles, void* out, int32_t* status, cudaStream_t s, float f8_scale) {
+                     int n_blocks, int total_qtiles, void* out, int32_t* status, cudaStream_t s, float f8_scale,
+                     uint8_t* out_sf) {
   if (total_qtiles <= 0) return VLM_OK;
   if (heads <= 0 || heads > 65535) return VLM_ERR_UNSUPPORTED;
   CUtensorMap tm;
@@ -427,18 +458,23 @@ int launch_attention(const __nv_bfloat16* qkv, int64_t T, int heads, const int32
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 64 && !attr_done[dev]) {
-    if (cudaFuncSetAttribute(attn_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) !=
+    if (cudaFuncSetAttribute(attn_tc_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) !=
             cudaSuccess ||
-        cudaFuncSetAttribute(attn_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) !=
+        cudaFuncSetAttribute(attn_tc_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) !=
+            cudaSuccess ||
+        cudaFuncSetAttribute(attn_tc_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) !=
             cudaSuccess)
       return VLM_ERR_CUDA;
     attr_done[dev] = true;
   }
-  AttnArgs args{cu, qt, n_blocks, heads, out, status, f8_scale};
+  if (out_sf != nullptr && !(f8_scale > 0.f)) return VLM_ERR_INVALID_ARG;
+  AttnArgs args{cu, qt, n_blocks, heads, out, status, f8_scale, out_sf};
   dim3 grid(total_qtiles, heads);
   launch_begin(KC_ATTN, s);
-  const cudaError_t e = f8_scale > 0.f ? launch_pdl(attn_tc_kernel<true>, grid, dim3(192), kSmemBytes, s, tm, args)
-                                       : launch_pdl(attn_tc_kernel<false>, grid, dim3(192), kSmemBytes, s, tm, args);
+  const cudaError_t e =
+      out_sf != nullptr ? launch_pdl(attn_tc_kernel<2>, grid, dim3(192), kSmemBytes, s, tm, args)
+      : f8_scale > 0.f  ? launch_pdl(attn_tc_kernel<1>, grid, dim3(192), kSmemBytes, s, tm, args)
+                        : launch_pdl(attn_tc_kernel<0>, grid, dim3(192), kSmemBytes, s, tm, args);
   launch_end(KC_ATTN, s);
   return e == cudaSuccess ? VLM_OK : VLM_ERR_CUDA;
 }

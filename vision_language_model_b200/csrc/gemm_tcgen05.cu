@@ -50,6 +50,7 @@ struct GemmArgs {
   float out_scale;        // E4M3 output (SwiGLU): values are multiplied by this before rounding
   const float* g_a = nullptr;  // NVFP4 operands: the two global scales (device memory); the
   const float* g_b = nullptr;  // epilogue multiplies by fp32(g_a * g_b)
+  uint8_t* c_sf = nullptr;     // NVFP4 output (SwiGLU): block scales; out_scale is its global scale
 };
 
 template <int BN>
@@ -764,11 +765,116 @@ __device__ __forceinline__ void scale32(uint32_t (&a)[32], float alpha) {
 // tile columns 160..255 of accumulator 0, 0..95 of accumulator 1 -- are read
 // from TMEM first and held in registers; on_shared() then releases them to
 // the next tile's MMAs before any of them is stored.
+//
+// ROPE (kOverlap only): bf16 output like BF16, with the 2D rotary embedding
+// applied in fp32 to the columns below rope_cols: a 64-column chunk is one
+// head, pair (i, i + 32) rotated by the angle of the row's position (row
+// frequencies for i < 16, column frequencies above). The shared half-head
+// waits in fp32 registers for its partner half.
+// SWIGLU (kOverlap only): accumulator columns 32g..32g+15 hold gate and
+// 32g+16..32g+31 the matching up values of hidden columns 16g..16g+15, one
+// NVFP4 block: h = silu(gate) * up in fp32, quantised with global scale
+// args.out_scale; codes and block scales are stored straight from registers.
 template <int EPI, int BN, bool kOverlap, typename F>
-__device__ __forceinline__ void epilogue_nvfp4(Stager& st, uint32_t tbase, int row0, int n0, int acc, float alpha,
-                                               F&& on_shared) {
+__device__ __forceinline__ void epilogue_nvfp4(const GemmArgs& args, Stager& st, uint32_t tbase, int row0, int n0,
+                                               int acc, float alpha, F&& on_shared) {
   static_assert(!kOverlap || BN == 256, "the overlap layout is for 256-column tiles");
-  if constexpr (EPI == VLM_EPI_BF16) {
+  static_assert(kOverlap || (EPI != VLM_EPI_ROPE && EPI != VLM_EPI_SWIGLU), "rope / swiglu need 256-column tiles");
+  if constexpr (EPI == VLM_EPI_ROPE) {
+    const int lane = st.lane, row = row0 + lane;
+    const int pk = row < args.M ? __ldg(args.pos + row) : 0;
+    const float2* tr = args.rope + (pk >> 16) * 32;
+    const float2* tcol = args.rope + (pk & 0xFFFF) * 32;
+    auto finish = [&](float (&x)[32], float (&y)[32], int c) {
+      if (n0 + c < args.rope_cols) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const float2 cs = __ldg(i < 16 ? tr + i : tcol + i);
+          const float xi = x[i], yi = y[i];
+          x[i] = xi * cs.x - yi * cs.y;
+          y[i] = yi * cs.x + xi * cs.y;
+        }
+      }
+      uint32_t w[32];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        w[i] = pack_bf16x2(x[2 * i], x[2 * i + 1]);
+        w[16 + i] = pack_bf16x2(y[2 * i], y[2 * i + 1]);
+      }
+      uint8_t* buf = st.acquire();
+      st.write_row(buf, w);
+      st.commit(buf, n0 + c, row0);
+    };
+    auto load_scaled = [&](uint32_t col, float (&v)[32]) {
+      uint32_t a[32];
+      tmem_ld32(tbase + col, a);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(a[i]) * alpha;
+    };
+    // the shared columns: head cp whole, and half ho of head ch
+    const int cp = acc == 0 ? 192 : 0, ch = acc == 0 ? 128 : 64, ho = acc == 0 ? 32 : 0;
+    float x[32], y[32], hv[32];
+    load_scaled(cp, x);
+    load_scaled(cp + 32, y);
+    load_scaled(ch + ho, hv);
+    on_shared();
+    finish(x, y, cp);
+    load_scaled(ch + 32 - ho, x);
+    if (ho == 0) {
+      finish(hv, x, ch);
+    } else {
+      finish(x, hv, ch);
+    }
+    const int c_rest = acc == 0 ? 0 : 128;
+#pragma unroll 1
+    for (int i = 0; i < 2; ++i) {
+      const int c = c_rest + 64 * i;
+      load_scaled(c, x);
+      load_scaled(c + 32, y);
+      finish(x, y, c);
+    }
+  } else if constexpr (EPI == VLM_EPI_SWIGLU) {
+    const int lane = st.lane, row = row0 + lane;
+    const bool live = row < args.M;
+    const int kh = args.N / 2;  // hidden width: the K of the GEMM that reads these codes
+    uint8_t* codes_row = static_cast<uint8_t*>(args.c) + static_cast<int64_t>(row) * (kh / 2) + n0 / 4;
+    const float sg = args.out_scale, six_sg = 6.0f * sg;
+    uint32_t sf_lo = 0, sf_hi = 0;  // scale bytes of blocks g = 0..3 and 4..7 of the tile
+    auto block = [&](int g, const uint32_t (&r)[32]) {
+      float h[16], amax = 0.0f;
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        h[e] = silu_f(__uint_as_float(r[e]) * alpha) * (__uint_as_float(r[16 + e]) * alpha);
+        amax = fmaxf(amax, fabsf(h[e]));
+      }
+      uint2 q;
+      const uint32_t sb = nvfp4_quant16(h, amax, sg, six_sg, q);
+      if (g < 4) sf_lo |= sb << (8 * g);
+      else sf_hi |= sb << (8 * (g - 4));
+      if (live) *reinterpret_cast<uint2*>(codes_row + 8 * g) = q;
+    };
+    // the shared columns: blocks 5..7 of accumulator 0, 0..2 of accumulator 1
+    const int gs = acc == 0 ? 5 : 0;
+    uint32_t r0[32], r1[32], r2[32];
+    tmem_ld32(tbase + 32 * gs, r0);
+    tmem_ld32(tbase + 32 * (gs + 1), r1);
+    tmem_ld32(tbase + 32 * (gs + 2), r2);
+    on_shared();
+    block(gs, r0);
+    block(gs + 1, r1);
+    block(gs + 2, r2);
+    const int g_rest = acc == 0 ? 0 : 3;
+#pragma unroll 1
+    for (int i = 0; i < 5; ++i) {
+      tmem_ld32(tbase + 32 * (g_rest + i), r0);
+      block(g_rest + i, r0);
+    }
+    if (live) {
+      const int kb0 = n0 / 32;  // first block of the tile (a multiple of 8)
+      *reinterpret_cast<uint32_t*>(args.c_sf + nvfp4_sf_offset(row, kb0, kh)) = sf_lo;
+      *reinterpret_cast<uint32_t*>(args.c_sf + nvfp4_sf_offset(row, kb0 + 4, kh)) = sf_hi;
+    }
+  } else if constexpr (EPI == VLM_EPI_BF16) {
     int c_rest = 0;  // first of the chunks outside the shared columns
     if constexpr (kOverlap) {
       // the shared columns: one whole chunk (cp) and one half of another (ch + ho)
@@ -995,7 +1101,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Fp4Shape<BN>::THREAD
       tc_fence_after();
       const uint32_t tbase =
           tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * S::ACC_STRIDE);
-      epilogue_nvfp4<EPI, S::BN, S::kOverlap>(st, tbase, mt * 256 + static_cast<int>(rank) * GBM + q * 32,
+      epilogue_nvfp4<EPI, S::BN, S::kOverlap>(args, st, tbase, mt * 256 + static_cast<int>(rank) * GBM + q * 32,
                                               nt * S::BN, acc, alpha, [&] {
                                    if constexpr (S::kOverlap) {
                                      tc_fence_before();
@@ -1274,9 +1380,10 @@ bool make_tmap_sf(CUtensorMap* map, const void* ptr, uint64_t atoms) {
 }
 }  // namespace
 
-int launch_gemm_nvfp4(int epi, const uint8_t* a, const uint8_t* a_sf, const float* g_a, const uint8_t* b,
-                      const uint8_t* b_sf, const float* g_b, int64_t M, int64_t N, int64_t K, void* c,
-                      int32_t* status, cudaStream_t s) {
+int launch_gemm_nvfp4_ex(int epi, const uint8_t* a, const uint8_t* a_sf, const float* g_a, const uint8_t* b,
+                         const uint8_t* b_sf, const float* g_b, int64_t M, int64_t N, int64_t K, void* c,
+                         uint8_t* c_sf, float out_sg, const int32_t* pos, const float2* rope, int64_t rope_cols,
+                         int32_t* status, cudaStream_t s) {
   if (a == nullptr || a_sf == nullptr || g_a == nullptr || b == nullptr || b_sf == nullptr || g_b == nullptr ||
       c == nullptr)
     return VLM_ERR_INVALID_ARG;
@@ -1284,7 +1391,14 @@ int launch_gemm_nvfp4(int epi, const uint8_t* a, const uint8_t* a_sf, const floa
       (M + 127) / 128 * (K / 64) > INT32_MAX || N / 128 * (K / 64) > INT32_MAX)
     return VLM_ERR_BAD_SHAPE;
   if (K % 256 != 0 || N % 128 != 0) return VLM_ERR_UNSUPPORTED;
-  if (epi != VLM_EPI_BF16 && epi != VLM_EPI_RESID) return VLM_ERR_UNSUPPORTED;
+  if (epi != VLM_EPI_BF16 && epi != VLM_EPI_RESID && epi != VLM_EPI_ROPE && epi != VLM_EPI_SWIGLU)
+    return VLM_ERR_UNSUPPORTED;
+  const bool needs256 = epi == VLM_EPI_ROPE || epi == VLM_EPI_SWIGLU;
+  if (needs256 && N % 256 != 0) return VLM_ERR_UNSUPPORTED;
+  if (epi == VLM_EPI_ROPE && (pos == nullptr || rope == nullptr || rope_cols < 0 || rope_cols % 64 != 0))
+    return VLM_ERR_INVALID_ARG;
+  if (epi == VLM_EPI_SWIGLU && (c_sf == nullptr || !(out_sg > 0.f) || (reinterpret_cast<uintptr_t>(c_sf) & 3)))
+    return VLM_ERR_INVALID_ARG;
   if ((reinterpret_cast<uintptr_t>(a) | reinterpret_cast<uintptr_t>(b) | reinterpret_cast<uintptr_t>(a_sf) |
        reinterpret_cast<uintptr_t>(b_sf) | reinterpret_cast<uintptr_t>(c)) & 15)
     return VLM_ERR_INVALID_ARG;
@@ -1294,8 +1408,10 @@ int launch_gemm_nvfp4(int epi, const uint8_t* a, const uint8_t* a_sf, const floa
   if (!make_tmap_2d_u8(&tb, b, K / 2, N, K / 2, 128, bn / 2)) return VLM_ERR_CUDA;
   if (!make_tmap_sf(&tsa, a_sf, static_cast<uint64_t>((M + 127) / 128 * (K / 64)))) return VLM_ERR_CUDA;
   if (!make_tmap_sf(&tsb, b_sf, static_cast<uint64_t>(N / 128 * (K / 64)))) return VLM_ERR_CUDA;
-  const bool ok = epi == VLM_EPI_RESID ? make_tmap_2d(&tc, c, true, N, M, N * 4, 32, 32)
-                                       : make_tmap_2d(&tc, c, false, N, M, N * 2, 64, 32);
+  // the SwiGLU epilogue stores codes from registers: its output map is never used
+  const bool ok = epi == VLM_EPI_RESID    ? make_tmap_2d(&tc, c, true, N, M, N * 4, 32, 32)
+                  : epi == VLM_EPI_SWIGLU ? make_tmap_2d_u8(&tc, c, N / 4, M, N / 4, 64, 32)
+                                          : make_tmap_2d(&tc, c, false, N, M, N * 2, 64, 32);
   if (!ok) return VLM_ERR_CUDA;
   GemmArgs args;
   args.M = static_cast<int>(M);
@@ -1305,19 +1421,33 @@ int launch_gemm_nvfp4(int epi, const uint8_t* a, const uint8_t* a_sf, const floa
   args.n_tiles = static_cast<int>(N / bn);
   args.c = c;
   args.c_bf16 = nullptr;
-  args.pos = nullptr;
-  args.rope = nullptr;
-  args.rope_cols = 0;
+  args.pos = pos;
+  args.rope = rope;
+  args.rope_cols = static_cast<int>(rope_cols);
   args.status = status;
   args.colscale = nullptr;
-  args.out_scale = 1.0f;
+  args.out_scale = out_sg;
   args.g_a = g_a;
   args.g_b = g_b;
-  if (bn == 256)
-    return epi == VLM_EPI_RESID ? run_gemm_nvfp4<VLM_EPI_RESID, 256>(ta, tb, tsa, tsb, tc, args, s)
-                                : run_gemm_nvfp4<VLM_EPI_BF16, 256>(ta, tb, tsa, tsb, tc, args, s);
+  args.c_sf = c_sf;
+  if (bn == 256) {
+    switch (epi) {
+      case VLM_EPI_RESID: return run_gemm_nvfp4<VLM_EPI_RESID, 256>(ta, tb, tsa, tsb, tc, args, s);
+      case VLM_EPI_ROPE: return run_gemm_nvfp4<VLM_EPI_ROPE, 256>(ta, tb, tsa, tsb, tc, args, s);
+      case VLM_EPI_SWIGLU: return run_gemm_nvfp4<VLM_EPI_SWIGLU, 256>(ta, tb, tsa, tsb, tc, args, s);
+      default: return run_gemm_nvfp4<VLM_EPI_BF16, 256>(ta, tb, tsa, tsb, tc, args, s);
+    }
+  }
   return epi == VLM_EPI_RESID ? run_gemm_nvfp4<VLM_EPI_RESID, 128>(ta, tb, tsa, tsb, tc, args, s)
                               : run_gemm_nvfp4<VLM_EPI_BF16, 128>(ta, tb, tsa, tsb, tc, args, s);
+}
+
+int launch_gemm_nvfp4(int epi, const uint8_t* a, const uint8_t* a_sf, const float* g_a, const uint8_t* b,
+                      const uint8_t* b_sf, const float* g_b, int64_t M, int64_t N, int64_t K, void* c,
+                      int32_t* status, cudaStream_t s) {
+  if (epi != VLM_EPI_BF16 && epi != VLM_EPI_RESID) return VLM_ERR_UNSUPPORTED;
+  return launch_gemm_nvfp4_ex(epi, a, a_sf, g_a, b, b_sf, g_b, M, N, K, c, nullptr, 1.0f, nullptr, nullptr, 0,
+                              status, s);
 }
 
 }  // namespace vlm

@@ -131,9 +131,11 @@ int launch_gemm_f8(int epi, const void* a, const void* b, const float* colscale,
                    int64_t rope_cols, int32_t* status, cudaStream_t s);
 
 // f8_scale > 0: `out` is E4M3 holding the attention output times f8_scale; else bf16.
+// out_sf != nullptr: `out` is NVFP4 instead -- E2M1 codes [T, heads * 64 / 2] and
+// block scales in out_sf -- of the fp32 attention output with global scale f8_scale.
 int launch_attention(const __nv_bfloat16* qkv, int64_t T, int heads, const int32_t* cu, const int32_t* qt,
                      int n_blocks, int total_qtiles, void* out, int32_t* status, cudaStream_t s,
-                     float f8_scale = 0.f);
+                     float f8_scale = 0.f, uint8_t* out_sf = nullptr);
 // Per-row E4M3 quantisation of bf16 weight rows for the FP8 tower GEMMs:
 // s[r] = amax_r / 448 (1 for a zero row), dst[r, :] = e4m3(src[r, :] / s[r]),
 // colscale[r] = act_scale * s[r]. mode 0: row r of src; mode 1: the gate/up

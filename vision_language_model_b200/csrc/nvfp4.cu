@@ -33,27 +33,6 @@ __device__ __forceinline__ void load16(const void* x, int dtype, int64_t off, fl
   }
 }
 
-// fp32 -> E4M3 byte and back (exact), round to nearest even, saturating.
-__device__ __forceinline__ uint32_t e4m3_byte(float v) {
-  uint16_t r;
-  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(0.0f), "f"(v));
-  return r & 0xFFu;
-}
-__device__ __forceinline__ float e4m3_value(uint32_t byte) {
-  uint32_t h2;
-  const uint16_t b = static_cast<uint16_t>(byte);
-  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(b));
-  return __half2float(__ushort_as_half(static_cast<unsigned short>(h2 & 0xFFFFu)));
-}
-// Two fp32 values -> one byte of E2M1 codes, lo in the low nibble.
-__device__ __forceinline__ uint32_t e2m1x2(float lo, float hi) {
-  uint16_t r;
-  asm("{\n\t.reg .b8 t;\n\tcvt.rn.satfinite.e2m1x2.f32 t, %1, %2;\n\tcvt.u16.u8 %0, t;\n\t}"
-      : "=h"(r)
-      : "f"(hi), "f"(lo));
-  return r;
-}
-
 __global__ void amax_kernel(const void* __restrict__ x, int dtype, int64_t n, unsigned int* __restrict__ out_bits) {
   griddep_wait();
   griddep_launch_dependents();
@@ -86,8 +65,10 @@ __global__ void scale_finish_kernel(unsigned int* bits, float divisor) {
 // One thread per block of 16 values; threads of a warp take consecutive blocks
 // of a row (coalesced 32- or 64-byte reads and 8-byte code writes). Rows from
 // `rows` up to the end of the last 128-row group only write scale 0.
-__global__ void quant_nvfp4_kernel(const void* __restrict__ x, int dtype, int64_t rows, int64_t k,
-                                   const float* __restrict__ s_global, uint8_t* __restrict__ q,
+// x2 != nullptr: output rows 32j..32j+15 are rows 16j.. of x, rows
+// 32j+16..32j+31 rows 16j.. of x2 (the gate / up interleave).
+__global__ void quant_nvfp4_kernel(const void* __restrict__ x, const void* __restrict__ x2, int dtype, int64_t rows,
+                                   int64_t k, const float* __restrict__ s_global, uint8_t* __restrict__ q,
                                    uint8_t* __restrict__ sf) {
   griddep_wait();
   griddep_launch_dependents();
@@ -104,32 +85,45 @@ __global__ void quant_nvfp4_kernel(const void* __restrict__ x, int dtype, int64_
       continue;
     }
     float v[16];
-    load16(x, dtype, row * k + blk * kFp4Block, v);
+    if (x2 == nullptr) {
+      load16(x, dtype, row * k + blk * kFp4Block, v);
+    } else {
+      const int64_t src = (row >> 5) * 16 + (row & 15);
+      load16((row & 16) ? x2 : x, dtype, src * k + blk * kFp4Block, v);
+    }
     float amax = 0.0f;
 #pragma unroll
     for (int j = 0; j < 16; ++j) amax = fmaxf(amax, fabsf(v[j]));
-    const uint32_t code = six_sg > 0.0f ? e4m3_byte(__fdiv_rn(amax, six_sg)) : 0u;
-    const float denom = e4m3_value(code) * sg;
-    const float r = denom > 0.0f ? __fdiv_rn(1.0f, denom) : 0.0f;
-    uint32_t w[2] = {0u, 0u};
-#pragma unroll
-    for (int j = 0; j < 8; ++j) w[j >> 2] |= e2m1x2(v[2 * j] * r, v[2 * j + 1] * r) << (8 * (j & 3));
-    *reinterpret_cast<uint2*>(q + row * (k / 2) + blk * 8) = make_uint2(w[0], w[1]);
-    sf[nvfp4_sf_offset(row, blk, k)] = static_cast<uint8_t>(code);
+    uint2 codes;
+    const uint32_t sb = nvfp4_quant16(v, amax, sg, six_sg, codes);
+    *reinterpret_cast<uint2*>(q + row * (k / 2) + blk * 8) = codes;
+    sf[nvfp4_sf_offset(row, blk, k)] = static_cast<uint8_t>(sb);
   }
 }
 
 }  // namespace
 
 int launch_amax_scale(const void* x, int dtype, int64_t n, float divisor, float* out, cudaStream_t s) {
-  if (x == nullptr || out == nullptr || (dtype != 0 && dtype != 1)) return VLM_ERR_INVALID_ARG;
-  if (n <= 0 || !(divisor > 0.0f)) return VLM_ERR_BAD_SHAPE;
+  return launch_amax_scale_multi(&x, &n, 1, dtype, divisor, out, s);
+}
+
+int launch_amax_scale_multi(const void* const* xs, const int64_t* ns, int count, int dtype, float divisor, float* out,
+                            cudaStream_t s) {
+  if (xs == nullptr || ns == nullptr || count <= 0 || out == nullptr || (dtype != 0 && dtype != 1))
+    return VLM_ERR_INVALID_ARG;
+  if (!(divisor > 0.0f)) return VLM_ERR_BAD_SHAPE;
+  for (int i = 0; i < count; ++i) {
+    if (xs[i] == nullptr) return VLM_ERR_INVALID_ARG;
+    if (ns[i] <= 0) return VLM_ERR_BAD_SHAPE;
+  }
   if (cudaMemsetAsync(out, 0, sizeof(float), s) != cudaSuccess) return VLM_ERR_CUDA;
-  const int64_t want = (n + 255) / 256;
-  const int grid = static_cast<int>(want < 4 * num_sms() ? want : 4 * num_sms());
   launch_begin(KC_PACK, s);
-  cudaError_t e = launch_pdl(amax_kernel, dim3(grid), dim3(256), 0, s, x, dtype, n,
-                             reinterpret_cast<unsigned int*>(out));
+  cudaError_t e = cudaSuccess;
+  for (int i = 0; i < count && e == cudaSuccess; ++i) {
+    const int64_t want = (ns[i] + 255) / 256;
+    const int grid = static_cast<int>(want < 4 * num_sms() ? want : 4 * num_sms());
+    e = launch_pdl(amax_kernel, dim3(grid), dim3(256), 0, s, xs[i], dtype, ns[i], reinterpret_cast<unsigned int*>(out));
+  }
   if (e == cudaSuccess)
     e = launch_pdl(scale_finish_kernel, dim3(1), dim3(32), 0, s, reinterpret_cast<unsigned int*>(out), divisor);
   launch_end(KC_PACK, s);
@@ -138,16 +132,24 @@ int launch_amax_scale(const void* x, int dtype, int64_t n, float divisor, float*
 
 int launch_quant_nvfp4(const void* x, int dtype, int64_t rows, int64_t k, const float* s_global, uint8_t* q,
                        uint8_t* sf, cudaStream_t s) {
+  return launch_quant_nvfp4_rows(x, nullptr, dtype, rows, k, s_global, q, sf, s);
+}
+
+int launch_quant_nvfp4_rows(const void* x, const void* x2, int dtype, int64_t rows, int64_t k,
+                            const float* s_global, uint8_t* q, uint8_t* sf, cudaStream_t s) {
   if (x == nullptr || s_global == nullptr || q == nullptr || sf == nullptr || (dtype != 0 && dtype != 1))
     return VLM_ERR_INVALID_ARG;
   if (rows <= 0 || k <= 0 || rows > (1LL << 31) - 1) return VLM_ERR_BAD_SHAPE;
-  if (k % 64 != 0) return VLM_ERR_UNSUPPORTED;
-  if ((reinterpret_cast<uintptr_t>(x) & 15) || (reinterpret_cast<uintptr_t>(q) & 7)) return VLM_ERR_INVALID_ARG;
+  if (k % 64 != 0 || (x2 != nullptr && rows % 32 != 0)) return VLM_ERR_UNSUPPORTED;
+  if ((reinterpret_cast<uintptr_t>(x) & 15) || (reinterpret_cast<uintptr_t>(x2) & 15) ||
+      (reinterpret_cast<uintptr_t>(q) & 7))
+    return VLM_ERR_INVALID_ARG;
   const int64_t total = (rows + 127) / 128 * 128 * (k / kFp4Block);
   const int64_t want = (total + 255) / 256;
   const int grid = static_cast<int>(want < 8 * num_sms() ? want : 8 * num_sms());
   launch_begin(KC_PACK, s);
-  const cudaError_t e = launch_pdl(quant_nvfp4_kernel, dim3(grid), dim3(256), 0, s, x, dtype, rows, k, s_global, q, sf);
+  const cudaError_t e =
+      launch_pdl(quant_nvfp4_kernel, dim3(grid), dim3(256), 0, s, x, x2, dtype, rows, k, s_global, q, sf);
   launch_end(KC_PACK, s);
   return e == cudaSuccess ? VLM_OK : VLM_ERR_CUDA;
 }

@@ -6,6 +6,7 @@
 #include <type_traits>
 
 #include "kernels.cuh"
+#include "nvfp4.cuh"
 
 #define VLM_DEBUG_FILE_ID 1
 
@@ -218,13 +219,16 @@ __global__ void __launch_bounds__(kI2cThreads) im2col_tiled_kernel(const float* 
 // RMSNorm, one warp per row of `width` fp32 values (width % 128 == 0, <= 2048).
 // With g0: y = norm(x) * g0 is written back to x, and out = bf16(norm(y) * g1).
 // Without g0: out = bf16(norm(x) * g1).
-// kF8: out is E4M3 instead, of norm(.) * g1 * f8_scale (round to nearest even,
-// saturating).
+// OUT 1: out is E4M3 instead, of norm(.) * g1 * f8_scale (round to nearest
+// even, saturating). OUT 2: out is NVFP4 -- E2M1 codes [rows, width / 2] and
+// block scales in out_sf -- of the fp32 values norm(.) * g1 with global scale
+// f8_scale (a block of 16 spans four lanes).
 // ---------------------------------------------------------------------------
-template <int NV, bool kF8 = false>
+template <int NV, int OUT = 0>
 __global__ void rmsnorm_kernel(float* __restrict__ x, const float* __restrict__ g0,
                                const float* __restrict__ g1, void* __restrict__ out_v,
-                               int64_t rows, float eps, float f8_scale) {
+                               int64_t rows, float eps, float f8_scale, uint8_t* __restrict__ out_sf) {
+  constexpr bool kF8 = OUT == 1;
   griddep_wait();
   griddep_launch_dependents();
   constexpr int width = NV * 128;
@@ -258,7 +262,22 @@ __global__ void rmsnorm_kernel(float* __restrict__ x, const float* __restrict__ 
       rs = rsqrtf(ss / width + eps);
     }
     const float4* gr = reinterpret_cast<const float4*>(g1);
-    if constexpr (kF8) {
+    if constexpr (OUT == 2) {
+      uint16_t* orow = reinterpret_cast<uint16_t*>(static_cast<uint8_t*>(out_v) + row * (width / 2));
+      const float six_sg = 6.0f * f8_scale;
+#pragma unroll
+      for (int j = 0; j < NV; ++j) {
+        const float4 g = __ldg(gr + lane + 32 * j);
+        const float y0 = v[j].x * rs * g.x, y1 = v[j].y * rs * g.y, y2 = v[j].z * rs * g.z, y3 = v[j].w * rs * g.w;
+        float amax = fmaxf(fmaxf(fabsf(y0), fabsf(y1)), fmaxf(fabsf(y2), fabsf(y3)));
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+        float r;
+        const uint32_t sb = nvfp4_block_scale(amax, f8_scale, six_sg, r);
+        orow[lane + 32 * j] = static_cast<uint16_t>(e2m1x2(y0 * r, y1 * r) | (e2m1x2(y2 * r, y3 * r) << 8));
+        if ((lane & 3) == 0) out_sf[nvfp4_sf_offset(row, (lane + 32 * j) >> 2, width)] = static_cast<uint8_t>(sb);
+      }
+    } else if constexpr (kF8) {
       uint32_t* orow = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(out_v) + row * width);
 #pragma unroll
       for (int j = 0; j < NV; ++j) {
@@ -727,8 +746,34 @@ int launch_rmsnorm(float* x, const float* g0, const float* g1, void* out, int64_
   switch (width / 128) {
 #define VLM_NORM_CASE(nv)                                                                                       \
   case nv:                                                                                                    \
-    e = f8 ? launch_pdl(rmsnorm_kernel<nv, true>, dim3(grid), dim3(256), 0, s, x, g0, g1, out, rows, eps, f8_scale) \
-           : launch_pdl(rmsnorm_kernel<nv, false>, dim3(grid), dim3(256), 0, s, x, g0, g1, out, rows, eps, 0.f); \
+    e = f8 ? launch_pdl(rmsnorm_kernel<nv, 1>, dim3(grid), dim3(256), 0, s, x, g0, g1, out, rows, eps, f8_scale, \
+                        nullptr)                                                                          \
+           : launch_pdl(rmsnorm_kernel<nv, 0>, dim3(grid), dim3(256), 0, s, x, g0, g1, out, rows, eps, 0.f,  \
+                        nullptr);                                                                         \
+    break;
+    VLM_NORM_CASE(1) VLM_NORM_CASE(2) VLM_NORM_CASE(3) VLM_NORM_CASE(4) VLM_NORM_CASE(5)
+    VLM_NORM_CASE(6) VLM_NORM_CASE(7) VLM_NORM_CASE(8) VLM_NORM_CASE(9) VLM_NORM_CASE(10)
+    VLM_NORM_CASE(11) VLM_NORM_CASE(12) VLM_NORM_CASE(13) VLM_NORM_CASE(14) VLM_NORM_CASE(15)
+    VLM_NORM_CASE(16)
+#undef VLM_NORM_CASE
+    default: break;
+  }
+  launch_end(KC_NORM, s);
+  return e == cudaSuccess ? VLM_OK : VLM_ERR_CUDA;
+}
+
+int launch_rmsnorm_nvfp4(float* x, const float* g0, const float* g1, uint8_t* q, uint8_t* sf, int64_t rows,
+                         int width, float eps, float s_global, cudaStream_t s) {
+  if (width % 128 || width > 2048 || width <= 0) return VLM_ERR_UNSUPPORTED;
+  if (q == nullptr || sf == nullptr || !(s_global > 0.f)) return VLM_ERR_INVALID_ARG;
+  const int grid = grid_for(rows * 32, 256);
+  launch_begin(KC_NORM, s);
+  cudaError_t e = cudaErrorInvalidValue;
+  switch (width / 128) {
+#define VLM_NORM_CASE(nv)                                                                                      \
+  case nv:                                                                                                   \
+    e = launch_pdl(rmsnorm_kernel<nv, 2>, dim3(grid), dim3(256), 0, s, x, g0, g1, static_cast<void*>(q), rows, \
+                   eps, s_global, sf);                                                                       \
     break;
     VLM_NORM_CASE(1) VLM_NORM_CASE(2) VLM_NORM_CASE(3) VLM_NORM_CASE(4) VLM_NORM_CASE(5)
     VLM_NORM_CASE(6) VLM_NORM_CASE(7) VLM_NORM_CASE(8) VLM_NORM_CASE(9) VLM_NORM_CASE(10)

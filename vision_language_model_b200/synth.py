@@ -126,6 +126,13 @@ def fp8_act_scales(layers: int) -> list:
     return [[8.0 / 448.0, 4.0 / 448.0, 8.0 / 448.0, 16.0 / 448.0] for _ in range(layers)]
 
 
+def nvfp4_act_scales(layers: int) -> list:
+    """Static NVFP4 activation global scales per layer for the synthetic towers:
+    the same bounds as fp8_act_scales (8, 4, 8, 16), each mapped to the largest
+    E2M1 value times the largest E4M3 block scale, 6 * 448 = 2688."""
+    return [[8.0 / 2688.0, 4.0 / 2688.0, 8.0 / 2688.0, 16.0 / 2688.0] for _ in range(layers)]
+
+
 def projector_weights(seed: int, width: int, merge: int, proj_out: int) -> dict:
     d, e, m = width, proj_out, merge
     return {

@@ -117,12 +117,20 @@ def lib() -> ctypes.CDLL:
             "vlm_tower_fp8_packed_bytes": (SZ, [CP]),
             "vlm_pack_tower_fp8": (I32, [CP, ctypes.POINTER(TowerWeights), P, P, SZ, P]),
             "vlm_encode_fp8": (I32, [CP, P, P, I32, P, P, P, P, SZ, P, P]),
+            "vlm_tower_nvfp4_packed_bytes": (SZ, [CP]),
+            "vlm_pack_tower_nvfp4": (I32, [CP, ctypes.POINTER(TowerWeights), P, P, SZ, P]),
+            "vlm_encode_nvfp4_workspace_size": (SZ, [CP, P, I32]),
+            "vlm_encode_nvfp4": (I32, [CP, P, P, I32, P, P, P, P, SZ, P, P]),
             "vlm_gemm_fp8": (I32, [I32, P, P, P, F, I64, I64, I64, P, P, P, P, I64, P, P]),
             "vlm_rmsnorm_fp8": (I32, [P, P, P, P, I64, I32, F, F, P]),
             "vlm_nvfp4_sf_bytes": (SZ, [I64, I64]),
             "vlm_amax_scale": (I32, [P, I32, I64, F, P, P]),
             "vlm_quant_nvfp4": (I32, [P, I32, I64, I64, P, P, P, P]),
             "vlm_gemm_nvfp4": (I32, [I32, P, P, P, P, P, P, I64, I64, I64, P, P, P]),
+            "vlm_gemm_nvfp4_ex": (I32, [I32, P, P, P, P, P, P, I64, I64, I64, P, P, F, P, P, I64, P, P]),
+            "vlm_rmsnorm_nvfp4": (I32, [P, P, P, P, P, I64, I32, F, F, P]),
+            "vlm_attention_nvfp4": (I32, [P, I64, I32, I32, P, I32, P, P, F, P, SZ, P, P]),
+            "vlm_patch_embed": (I32, [CP, P, P, I32, P, P, P, SZ, P, P]),
             "vlm_launch_count": (I64, []),
             "vlm_profile_enable": (I32, [I32]),
             "vlm_profile_query": (I32, [I32, ctypes.POINTER(I64), ctypes.POINTER(ctypes.c_double)]),
@@ -370,6 +378,60 @@ def encode_fp8(cfg: Config, pixels: torch.Tensor, image_hw, packed_tower_fp8: to
     return out
 
 
+def pack_tower_nvfp4(cfg: Config, w: dict, act_scales, stream=None) -> torch.Tensor:
+    """NVFP4 tower (block-scaled E2M1 weights, static activation global scales act_scales[l][0..3])."""
+    L = lib()
+    tw = TowerWeights(**{k: _dev(w[k], k) for k, _ in TowerWeights._fields_})
+    nbytes = L.vlm_tower_nvfp4_packed_bytes(ctypes.byref(cfg))
+    if nbytes == 0:
+        raise VlmError(ERR_INVALID_ARG, "vlm_tower_nvfp4_packed_bytes")
+    packed = _empty(nbytes, dtype=torch.uint8, device=w["wq"].device)
+    _check(L.vlm_pack_tower_nvfp4(ctypes.byref(cfg), ctypes.byref(tw), _act_array(cfg, act_scales),
+                                  packed.data_ptr(), nbytes, _stream(stream)), "vlm_pack_tower_nvfp4")
+    return packed
+
+
+def patch_embed(cfg: Config, pixels: torch.Tensor, image_hw, packed_tower: torch.Tensor, status=None,
+                stream=None) -> torch.Tensor:
+    """The patch features fp32 [T, width] (gather + patch-embed GEMM, before ln_pre)."""
+    L = lib()
+    arr, n = _hw_array(image_hw)
+    T = num_patches(cfg, image_hw)
+    dev = pixels.device
+    x = _empty((T, cfg.width), dtype=torch.float32, device=dev)
+    ws = _empty(L.vlm_encode_workspace_size(ctypes.byref(cfg), arr, n), dtype=torch.uint8, device=dev)
+    if status is None:
+        status = new_status(dev)
+    _check(L.vlm_patch_embed(ctypes.byref(cfg), _dev(pixels, "pixels"), arr, n, _dev(packed_tower, "packed"),
+                             _dev(x, "x"), _dev(ws, "workspace"), ws.numel(), _dev(status, "status"), _stream(stream)),
+           "vlm_patch_embed")
+    return x
+
+
+def encode_nvfp4_workspace_size(cfg: Config, image_hw) -> int:
+    arr, n = _hw_array(image_hw)
+    return lib().vlm_encode_nvfp4_workspace_size(ctypes.byref(cfg), arr, n)
+
+
+def encode_nvfp4(cfg: Config, pixels: torch.Tensor, image_hw, packed_tower_nvfp4: torch.Tensor, act_scales,
+                 out=None, workspace=None, status=None, stream=None) -> torch.Tensor:
+    """vlm_encode with the NVFP4 tower GEMMs."""
+    L = lib()
+    arr, n = _hw_array(image_hw)
+    T = num_patches(cfg, image_hw)
+    dev = pixels.device
+    if out is None:
+        out = _empty((T, cfg.width), dtype=torch.bfloat16, device=dev)
+    if workspace is None:
+        workspace = _empty(encode_nvfp4_workspace_size(cfg, image_hw), dtype=torch.uint8, device=dev)
+    if status is None:
+        status = new_status(dev)
+    _check(L.vlm_encode_nvfp4(ctypes.byref(cfg), _dev(pixels, "pixels"), arr, n, _dev(packed_tower_nvfp4, "packed"),
+                              _act_array(cfg, act_scales), _dev(out, "out"), _dev(workspace, "workspace"),
+                              workspace.numel(), _dev(status, "status"), _stream(stream)), "vlm_encode_nvfp4")
+    return out
+
+
 def gemm_fp8(epilogue: int, a: torch.Tensor, b: torch.Tensor, colscale: torch.Tensor, out: torch.Tensor,
              out_scale: float = 1.0, out_bf16=None, pos=None, rope=None, rope_cols: int = 0, status=None,
              stream=None) -> torch.Tensor:
@@ -447,6 +509,50 @@ def gemm_nvfp4(epilogue: int, a: tuple, b: tuple, out: torch.Tensor, status=None
                                 _dev(sfb, "b_sf"), _dev(gb, "g_b"), M, N, K, _dev(out, "out"), _dev(status, "status"),
                                 _stream(stream)), "vlm_gemm_nvfp4")
     return out
+
+
+def gemm_nvfp4_rope(a: tuple, b: tuple, out: torch.Tensor, pos: torch.Tensor, rope_table: torch.Tensor,
+                    rope_cols: int, status=None, stream=None) -> torch.Tensor:
+    """gemm_nvfp4 with the ROPE epilogue: out bf16 [M, N], columns below
+    rope_cols rotated (pos: int32 [M] = row << 16 | col; rope_table from rope_table())."""
+    (qa, sfa, ga), (qb, sfb, gb) = a, b
+    M, N, K = qa.shape[0], qb.shape[0], 2 * qa.shape[1]
+    if status is None:
+        status = new_status(qa.device)
+    _check(lib().vlm_gemm_nvfp4_ex(EPI_ROPE, _dev(qa, "a"), _dev(sfa, "a_sf"), _dev(ga, "g_a"), _dev(qb, "b"),
+                                   _dev(sfb, "b_sf"), _dev(gb, "g_b"), M, N, K, _dev(out, "out"), None, 1.0,
+                                   _dev(pos, "pos"), _dev(rope_table, "rope"), int(rope_cols), _dev(status, "status"),
+                                   _stream(stream)), "vlm_gemm_nvfp4_ex")
+    return out
+
+
+def gemm_nvfp4_swiglu(a: tuple, b: tuple, out_sg: float, q=None, sf=None, status=None, stream=None) -> tuple:
+    """gemm_nvfp4 with the SWIGLU epilogue (B rows gate / up interleaved by 16):
+    returns the NVFP4 codes [M, N/4] and block scales of silu(gate) * up with
+    global scale out_sg (the scales of padding rows are zero when sf is None)."""
+    (qa, sfa, ga), (qb, sfb, gb) = a, b
+    M, N, K = qa.shape[0], qb.shape[0], 2 * qa.shape[1]
+    if q is None:
+        q = _empty((M, N // 4), dtype=torch.uint8, device=qa.device)
+    if sf is None:
+        sf = _zeros(nvfp4_sf_bytes(M, N // 2), dtype=torch.uint8, device=qa.device)
+    if status is None:
+        status = new_status(qa.device)
+    _check(lib().vlm_gemm_nvfp4_ex(EPI_SWIGLU, _dev(qa, "a"), _dev(sfa, "a_sf"), _dev(ga, "g_a"), _dev(qb, "b"),
+                                   _dev(sfb, "b_sf"), _dev(gb, "g_b"), M, N, K, _dev(q, "out"), _dev(sf, "out_sf"),
+                                   float(out_sg), None, None, 0, _dev(status, "status"), _stream(stream)),
+           "vlm_gemm_nvfp4_ex")
+    return q, sf
+
+
+def rmsnorm_nvfp4(x: torch.Tensor, g1: torch.Tensor, s_global: float, g0=None, eps: float = 1e-5, stream=None) -> tuple:
+    """rmsnorm whose output is NVFP4 with global scale s_global: (codes, block scales)."""
+    rows, width = x.shape
+    q = _empty((rows, width // 2), dtype=torch.uint8, device=x.device)
+    sf = _zeros(nvfp4_sf_bytes(rows, width), dtype=torch.uint8, device=x.device)
+    _check(lib().vlm_rmsnorm_nvfp4(_dev(x, "x"), _dev(g0, "g0"), _dev(g1, "g1"), _dev(q, "q"), _dev(sf, "sf"), rows,
+                                   width, float(eps), float(s_global), _stream(stream)), "vlm_rmsnorm_nvfp4")
+    return q, sf
 
 
 # ---------------------------------------------------------------------------
@@ -551,6 +657,23 @@ def attention(qkv: torch.Tensor, cu_seqlens, heads: int, out=None, status=None, 
     return out
 
 
+def attention_nvfp4(qkv: torch.Tensor, cu_seqlens, heads: int, s_global: float, status=None, stream=None) -> tuple:
+    """attention whose output is NVFP4 with global scale s_global: (codes, block scales)."""
+    L = lib()
+    T = qkv.shape[0]
+    cu = (ctypes.c_int32 * len(cu_seqlens))(*[int(c) for c in cu_seqlens])
+    nb = len(cu_seqlens) - 1
+    q = _empty((T, heads * 32), dtype=torch.uint8, device=qkv.device)
+    sf = _zeros(nvfp4_sf_bytes(T, heads * 64), dtype=torch.uint8, device=qkv.device)
+    ws = _empty(max(256, L.vlm_attention_workspace_size(nb)), dtype=torch.uint8, device=qkv.device)
+    if status is None:
+        status = new_status(qkv.device)
+    _check(L.vlm_attention_nvfp4(_dev(qkv, "qkv"), T, heads, 64, cu, nb, _dev(q, "q"), _dev(sf, "sf"), float(s_global),
+                                 ws.data_ptr(), ws.numel(), _dev(status, "status"), _stream(stream)),
+           "vlm_attention_nvfp4")
+    return q, sf
+
+
 def rmsnorm(x: torch.Tensor, g1: torch.Tensor, g0=None, eps: float = 1e-5, out=None, stream=None) -> torch.Tensor:
     rows, width = x.shape
     if out is None:
@@ -610,25 +733,40 @@ def profile_query(kclass: str) -> tuple:
 class ImagePipeline:
     """vlm_encode -> vlm_merge_project (-> vlm_scatter) with buffers kept between calls."""
 
-    def __init__(self, cfg: Config, tower: dict, projector: dict, image_hw, device="cuda", fp8_act_scales=None):
-        """fp8_act_scales: None for the bf16 tower, or [layers][4] static activation
-        scales for the E4M3 tower GEMMs (vlm_encode_fp8)."""
+    def __init__(self, cfg: Config, tower: dict, projector: dict, image_hw, device="cuda", fp8_act_scales=None,
+                 nvfp4_act_scales=None):
+        """fp8_act_scales: [layers][4] static activation scales for the E4M3 tower
+        GEMMs (vlm_encode_fp8); nvfp4_act_scales: [layers][4] static activation
+        global scales for the NVFP4 tower GEMMs (vlm_encode_nvfp4); neither: the
+        bf16 tower."""
+        if fp8_act_scales is not None and nvfp4_act_scales is not None:
+            raise ValueError("choose one of fp8_act_scales and nvfp4_act_scales")
         self.cfg = cfg
         self.image_hw = [tuple(int(v) for v in hw) for hw in image_hw]
         self.fp8_act_scales = fp8_act_scales
-        self.packed_tower = pack_tower(cfg, tower) if fp8_act_scales is None else \
-            pack_tower_fp8(cfg, tower, fp8_act_scales)
+        self.nvfp4_act_scales = nvfp4_act_scales
+        if nvfp4_act_scales is not None:
+            self.packed_tower = pack_tower_nvfp4(cfg, tower, nvfp4_act_scales)
+        elif fp8_act_scales is not None:
+            self.packed_tower = pack_tower_fp8(cfg, tower, fp8_act_scales)
+        else:
+            self.packed_tower = pack_tower(cfg, tower)
         self.packed_proj = pack_projector(cfg, projector)
         self.T = num_patches(cfg, self.image_hw)
         self.Tm = num_merged(cfg, self.image_hw)
         self.tower_out = _empty((self.T, cfg.width), dtype=torch.bfloat16, device=device)
         self.embeds = _empty((self.Tm, cfg.proj_out), dtype=torch.bfloat16, device=device)
-        ws = max(encode_workspace_size(cfg, self.image_hw), merge_project_workspace_size(cfg, self.image_hw))
+        enc_ws = encode_nvfp4_workspace_size(cfg, self.image_hw) if nvfp4_act_scales is not None else \
+            encode_workspace_size(cfg, self.image_hw)
+        ws = max(enc_ws, merge_project_workspace_size(cfg, self.image_hw))
         self.workspace = _empty(ws, dtype=torch.uint8, device=device)
         self.status = new_status(device)
 
     def __call__(self, pixels: torch.Tensor, stream=None) -> torch.Tensor:
-        if self.fp8_act_scales is None:
+        if self.nvfp4_act_scales is not None:
+            encode_nvfp4(self.cfg, pixels, self.image_hw, self.packed_tower, self.nvfp4_act_scales,
+                         out=self.tower_out, workspace=self.workspace, status=self.status, stream=stream)
+        elif self.fp8_act_scales is None:
             encode(self.cfg, pixels, self.image_hw, self.packed_tower, out=self.tower_out, workspace=self.workspace,
                    status=self.status, stream=stream)
         else:
