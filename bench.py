@@ -49,6 +49,12 @@ WORKLOADS = {
                               desc="one 1540x1540 image (12,100 patches -> 3,025 merged tokens), 24-layer tower with "
                                    "E4M3 QKV/O/gate-up/down GEMMs (per-row weight scales, static activation scales; "
                                    "bf16 attention, norms, patch embed) + 2x2 merge + bf16 projector + scatter"),
+    "mistral3_1540_nvfp4": dict(preset="mistral3", sizes=[(1540, 1540)], n_seq=1, seq_len=4096, nvfp4=True,
+                                desc="one 1540x1540 image (12,100 patches -> 3,025 merged tokens), 24-layer tower "
+                                     "with NVFP4 QKV/O/gate-up/down GEMMs (E2M1 with E4M3 block scales per 16 "
+                                     "values; weight global scales from the data, static activation global scales; "
+                                     "every GEMM input quantised in the kernel that produces it; bf16 attention, "
+                                     "norms, patch embed) + 2x2 merge + bf16 projector + scatter"),
     "photo_4032x3024": dict(preset="mistral3", photo=(3024, 4032), sizes=[(1176, 1540)], n_seq=1, seq_len=4096,
                             desc="one decoded 4032x3024 u8 RGB photo: GPU resize to 1176x1540 (longest edge 1540, "
                                  "28-px grid; 84x110 = 9,240 patches -> 2,310 merged tokens), 24-layer tower + "
@@ -251,6 +257,7 @@ class OracleSample:
         pw = synth.projector_weights(seed, base["width"], base["merge"], base["proj_out"])
         self.pw = {k: v.double().numpy() for k, v in pw.items()}
         self.imgs = [im.double().numpy() for im in synth.images(seed, self.sizes)]
+        self.quantised = bool(wl.get("fp8") or wl.get("nvfp4"))
         self.grids = [O.patch_grid(h, w, base["patch"]) for h, w in self.sizes]
         self.T = sum(h * w for h, w in self.grids)
         self.step_i = 0
@@ -280,9 +287,11 @@ class OracleSample:
         return self.T / (self.t_embed + layers * (self.t_kv + t_rows_full) + self.t_proj)
 
     def describe(self) -> str:
+        quant = (" (the unquantised block: the oracle's quantised block runs the same products plus its "
+                 "quantisation passes)" if self.quantised else "")
         return (f"oracle (numpy fp64): patch embed of all {self.T} patches, keys/values of one tower block for all "
-                f"patches, the rest of that block on every {self.frac}th patch, projector on all merged tokens; "
-                f"tower time extrapolated to all patches and 24 layers")
+                f"patches, the rest of that block on every {self.frac}th patch{quant}, projector on all merged "
+                f"tokens; tower time extrapolated to all patches and 24 layers")
 
 
 def cpu_baseline(wl, seed) -> dict:
@@ -542,7 +551,8 @@ def run_ours(args, wl):
     tw = {k: v.to(dev) for k, v in synth.tower_weights(args.seed, cfg.layers, cfg.width, cfg.mlp, cfg.patch).items()}
     pw = {k: v.to(dev) for k, v in synth.projector_weights(args.seed, cfg.width, cfg.merge, cfg.proj_out).items()}
     pipe = vlm.ImagePipeline(cfg, tw, pw, sizes, device=dev,
-                             fp8_act_scales=synth.fp8_act_scales(cfg.layers) if wl.get("fp8") else None)
+                             fp8_act_scales=synth.fp8_act_scales(cfg.layers) if wl.get("fp8") else None,
+                             nvfp4_act_scales=synth.nvfp4_act_scales(cfg.layers) if wl.get("nvfp4") else None)
     del tw, pw
     photo = wl.get("photo")
     if photo:
@@ -681,7 +691,7 @@ def run_ours(args, wl):
     line = {
         "metric": METRIC, "value": value, "unit": "patches/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "e4m3+bf16" if wl.get("fp8") else "bf16", "data": "synthetic",
+        "vs_baseline": None, "dtype": "e4m3+bf16" if wl.get("fp8") else "e2m1+bf16" if wl.get("nvfp4") else "bf16", "data": "synthetic",
         "config": wcfg,
         "roofline": {"kernel": kern, "bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": achieved / peak, "peak_source": f"bf16_tflops, burst ({peaks['source']})",

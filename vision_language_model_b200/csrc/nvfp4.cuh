@@ -46,7 +46,7 @@ __device__ __forceinline__ uint32_t e2m1x2(float lo, float hi) {
 __device__ __forceinline__ uint32_t nvfp4_block_scale(float amax, float sg, float six_sg, float& r) {
   const uint32_t sb = six_sg > 0.0f ? e4m3_byte(__fdiv_rn(amax, six_sg)) : 0u;
   const float denom = e4m3_value(sb) * sg;
-  r = denom > 0.0f ? __fdiv_rn(1.0f, denom) : 0.0f;
+  r = denom > 0.0f ? __frcp_rn(denom) : 0.0f;  // the correctly rounded reciprocal
   return sb;
 }
 __device__ __forceinline__ uint32_t nvfp4_quant16(const float (&v)[16], float amax, float sg, float six_sg,

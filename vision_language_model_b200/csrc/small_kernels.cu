@@ -762,8 +762,94 @@ int launch_rmsnorm(float* x, const float* g0, const float* g1, void* out, int64_
   return e == cudaSuccess ? VLM_OK : VLM_ERR_CUDA;
 }
 
+// RMSNorm to NVFP4 for widths that are a multiple of 512: lane l holds the 16
+// consecutive values of blocks l + 32 b (b < NB), so each block is quantised
+// by one lane (no shuffles, no repeated scale arithmetic across lanes) and its
+// 8 code bytes are one store. One warp per row; loads are 64 contiguous bytes
+// per lane.
+template <int NB>
+__global__ void rmsnorm_nvfp4_kernel(float* __restrict__ x, const float* __restrict__ g0,
+                                     const float* __restrict__ g1, uint8_t* __restrict__ q,
+                                     uint8_t* __restrict__ sf, int64_t rows, float eps, float sg) {
+  griddep_wait();
+  griddep_launch_dependents();
+  constexpr int width = NB * 512;
+  const int lane = threadIdx.x & 31;
+  const float six_sg = 6.0f * sg;
+  const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
+  for (int64_t row = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; row < rows;
+       row += warps) {
+    float4* xr = reinterpret_cast<float4*>(x + row * width);
+    float4 v[NB][4];
+    float ss = 0.f;
+#pragma unroll
+    for (int b = 0; b < NB; ++b)
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        v[b][t] = xr[4 * (lane + 32 * b) + t];
+        ss += v[b][t].x * v[b][t].x + v[b][t].y * v[b][t].y + v[b][t].z * v[b][t].z + v[b][t].w * v[b][t].w;
+      }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    float rs = rsqrtf(ss / width + eps);
+    if (g0 != nullptr) {
+      const float4* gr = reinterpret_cast<const float4*>(g0);
+      ss = 0.f;
+#pragma unroll
+      for (int b = 0; b < NB; ++b)
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+          const float4 g = __ldg(gr + 4 * (lane + 32 * b) + t);
+          float4& u = v[b][t];
+          u.x *= rs * g.x; u.y *= rs * g.y; u.z *= rs * g.z; u.w *= rs * g.w;
+          xr[4 * (lane + 32 * b) + t] = u;
+          ss += u.x * u.x + u.y * u.y + u.z * u.z + u.w * u.w;
+        }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+      rs = rsqrtf(ss / width + eps);
+    }
+    const float4* gr = reinterpret_cast<const float4*>(g1);
+#pragma unroll
+    for (int b = 0; b < NB; ++b) {
+      float y[16], amax = 0.0f;
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        const float4 g = __ldg(gr + 4 * (lane + 32 * b) + t);
+        y[4 * t] = v[b][t].x * rs * g.x;
+        y[4 * t + 1] = v[b][t].y * rs * g.y;
+        y[4 * t + 2] = v[b][t].z * rs * g.z;
+        y[4 * t + 3] = v[b][t].w * rs * g.w;
+      }
+#pragma unroll
+      for (int k = 0; k < 16; ++k) amax = fmaxf(amax, fabsf(y[k]));
+      uint2 codes;
+      const uint32_t sb = nvfp4_quant16(y, amax, sg, six_sg, codes);
+      const int blk = lane + 32 * b;
+      *reinterpret_cast<uint2*>(q + row * (width / 2) + 8 * blk) = codes;
+      sf[nvfp4_sf_offset(row, blk, width)] = static_cast<uint8_t>(sb);
+    }
+  }
+}
+
 int launch_rmsnorm_nvfp4(float* x, const float* g0, const float* g1, uint8_t* q, uint8_t* sf, int64_t rows,
                          int width, float eps, float s_global, cudaStream_t s) {
+  if (width % 512 == 0 && width <= 2048 && width > 0) {
+    if (q == nullptr || sf == nullptr || !(s_global > 0.f)) return VLM_ERR_INVALID_ARG;
+    if (reinterpret_cast<uintptr_t>(q) & 7) return VLM_ERR_INVALID_ARG;
+    const int grid = grid_for(rows * 32, 256);
+    launch_begin(KC_NORM, s);
+    cudaError_t e = cudaErrorInvalidValue;
+    switch (width / 512) {
+      case 1: e = launch_pdl(rmsnorm_nvfp4_kernel<1>, dim3(grid), dim3(256), 0, s, x, g0, g1, q, sf, rows, eps, s_global); break;
+      case 2: e = launch_pdl(rmsnorm_nvfp4_kernel<2>, dim3(grid), dim3(256), 0, s, x, g0, g1, q, sf, rows, eps, s_global); break;
+      case 3: e = launch_pdl(rmsnorm_nvfp4_kernel<3>, dim3(grid), dim3(256), 0, s, x, g0, g1, q, sf, rows, eps, s_global); break;
+      case 4: e = launch_pdl(rmsnorm_nvfp4_kernel<4>, dim3(grid), dim3(256), 0, s, x, g0, g1, q, sf, rows, eps, s_global); break;
+      default: break;
+    }
+    launch_end(KC_NORM, s);
+    return e == cudaSuccess ? VLM_OK : VLM_ERR_CUDA;
+  }
   if (width % 128 || width > 2048 || width <= 0) return VLM_ERR_UNSUPPORTED;
   if (q == nullptr || sf == nullptr || !(s_global > 0.f)) return VLM_ERR_INVALID_ARG;
   const int grid = grid_for(rows * 32, 256);
