@@ -443,10 +443,16 @@ def gemm_shapes(args) -> None:
         quant = timeit(lambda: vlm.quant_nvfp4(x, ga, q=qa, sf=sfa))
         plain = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
         store = timeit(lambda: vlm.gemm_nvfp4(vlm.EPI_BF16, (qa, sfa, ga), (qw, sfw, gw), plain, status=st))
-        fused = None
         if epi == vlm.EPI_RESID:
             c = torch.zeros((M, N), dtype=torch.float32, device="cuda")
             fused = timeit(lambda: vlm.gemm_nvfp4(vlm.EPI_RESID, (qa, sfa, ga), (qw, sfw, gw), c, status=st))
+        elif epi == vlm.EPI_SWIGLU:
+            hq = torch.empty((M, N // 4), dtype=torch.uint8, device="cuda")
+            hsf = torch.zeros(vlm.nvfp4_sf_bytes(M, N // 2), dtype=torch.uint8, device="cuda")
+            fused = timeit(lambda: vlm.gemm_nvfp4_swiglu((qa, sfa, ga), (qw, sfw, gw), 16.0 / 2688.0, q=hq, sf=hsf,
+                                                         status=st))
+        else:
+            fused = timeit(lambda: vlm.gemm_nvfp4_rope((qa, sfa, ga), (qw, sfw, gw), plain, pos, rope, 2048, status=st))
         lib, lib_ms = "torch._scaled_mm (cuBLASLt, NVFP4)", None
         try:
             fa, fw = qa.view(torch.float4_e2m1fn_x2), qw.view(torch.float4_e2m1fn_x2)
@@ -454,8 +460,7 @@ def gemm_shapes(args) -> None:
             lib_ms = timeit(lambda: torch._scaled_mm(fa, fw.t(), scale_a=sa8, scale_b=sw8, out_dtype=torch.bfloat16))
         except Exception as e:  # the library call is a comparison only
             lib = f"torch._scaled_mm NVFP4 unavailable: {type(e).__name__}: {str(e)[:120]}"
-        print(json.dumps({"gemm": name, "dtype": "nvfp4", "M": M, "N": N, "K": K, "epilogue": vlm.EPI_RESID
-                          if fused is not None else vlm.EPI_BF16,
+        print(json.dumps({"gemm": name, "dtype": "nvfp4", "M": M, "N": N, "K": K, "epilogue": epi,
                           "fused_ms": fused, "fused_tflops": fl / fused / 1e9 if fused else None,
                           "plain_store_ms": store, "plain_store_tflops": fl / store / 1e9,
                           "quantise_activations_ms": quant, "library": lib, "library_ms": lib_ms,

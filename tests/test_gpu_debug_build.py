@@ -60,9 +60,9 @@ def test_debug_build_check_fails_into_record_and_skips_access():
 
 def test_parity_suite_under_debug_build_trips_no_check():
     files = ["tests/test_gpu_kernels.py", "tests/test_gpu_model.py", "tests/test_gpu_frontend.py",
-             "tests/test_gpu_fp8.py", "tests/test_gpu_nvfp4.py"]
+             "tests/test_gpu_fp8.py", "tests/test_gpu_nvfp4.py", "tests/test_gpu_nvfp4_tower.py"]
     r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-x", "-m", "gpu", "-p", "no:cacheprovider",
-                        "-k", "not full_size"] + files,
+                        "-k", "not full_size and not 1540"] + files,
                        cwd=ROOT, env=_debug_env(), capture_output=True, text=True, timeout=1800)
     assert r.returncode == 0, r.stdout[-6000:] + r.stderr[-3000:]
     assert " passed" in r.stdout
