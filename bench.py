@@ -93,6 +93,10 @@ def parse_args():
                    help="replay each step as one captured CUDA graph (headline and e2e loops)")
     p.add_argument("--side-stream", action="store_true",
                    help="also measure the encoder on a side stream overlapped with a decode-like GEMV loop")
+    p.add_argument("--sm-budget", type=int, default=0,
+                   help="vlm_config.sm_budget: SMs the encoder's persistent kernels may hold and twice the CTAs of "
+                        "each attention grid (0 = every SM); with --side-stream the rest of the GPU is left to the "
+                        "other stream")
     p.add_argument("--gemm-shapes", action="store_true",
                    help="instead of a step: time the tower's GEMM shapes (12,100 rows), bf16, E4M3 and NVFP4, each "
                         "with its fused epilogue and with a plain store, beside torch's cuBLAS / cuBLASLt GEMM; one "
@@ -503,6 +507,11 @@ def side_stream_overlap(pipe, pix, ids, text, cfg, scatter_ws, dev, steps: int) 
         return a.elapsed_time(b) / reps
 
     enc_ms = time_it(encode_request, steps)
+    enc_full_ms = enc_ms
+    if cfg.sm_budget:  # the same request with every SM, for the comparison against serial full-GPU runs
+        budget, cfg.sm_budget = cfg.sm_budget, 0
+        enc_full_ms = time_it(encode_request, steps)
+        cfg.sm_budget = budget
     dec_ms = time_it(decode_pass, 20)
     n_dec = max(1, round(enc_ms / dec_ms))
 
@@ -538,8 +547,12 @@ def side_stream_overlap(pipe, pix, ids, text, cfg, scatter_ws, dev, steps: int) 
             "overlapped_ms": both_ms, "decode_pass_ms_during_encode": dec_conc,
             "overlapped_ms_decode_high_priority": both_hi_ms, "decode_pass_ms_during_encode_high_priority": dec_conc_hi,
             "hidden_frac": (serial - both_ms) / min(enc_ms, n_dec * dec_ms),
+            "encoder_sm_budget": cfg.sm_budget or None, "encode_ms_every_sm": enc_full_ms,
+            "gain_vs_serial_every_sm": 1.0 - min(both_ms, both_hi_ms) / (enc_full_ms + n_dec * dec_ms),
             "note": "encoder + scatter of one request on a side stream, decode-like GEMV passes on another stream; "
-                    "hidden_frac = time saved against running them one after the other / the shorter of the two"}
+                    "hidden_frac = time saved against running them one after the other / the shorter of the two; "
+                    "gain_vs_serial_every_sm = time saved against running them one after the other with the "
+                    "encoder on every SM"}
 
 
 def run_ours(args, wl):
@@ -549,7 +562,7 @@ def run_ours(args, wl):
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     sizes = sizes_of(wl, args.seed)
-    cfg = vlm.preset(wl["preset"])
+    cfg = vlm.preset(wl["preset"], sm_budget=args.sm_budget)
     fl = flops_breakdown(cfg, sizes)
     T, Tm = fl["T"], fl["Tm"]
 
@@ -692,6 +705,8 @@ def run_ours(args, wl):
     peak = peaks["bf16_tflops"]
     step_tflops = fl["total"] / (ms / args.steps / 1000.0) / 1e12
     wcfg = workload_config(wl, sizes, world)
+    if args.sm_budget:
+        wcfg["sm_budget"] = args.sm_budget
     assert (wcfg["patches"], wcfg["merged_tokens"], wcfg["text_tokens"]) == (T, Tm, int(ids.numel()))
     line = {
         "metric": METRIC, "value": value, "unit": "patches/s", "n_gpus": world, "steps": args.steps,

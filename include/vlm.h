@@ -76,6 +76,12 @@ typedef struct {
   float rope_theta, eps;
   int32_t normalize;
   int32_t norm_after_merge;
+  /* SM budget of the calls that take this config (0 = every SM): the
+   * persistent GEMMs hold at most this many SMs, and attention is launched in
+   * successive grids of at most 2 CTAs per budgeted SM, so that work on other
+   * streams keeps the rest of the GPU. Results are bit-identical for every
+   * budget; a budget above the SM count means every SM. Negative: rejected. */
+  int32_t sm_budget;
 } vlm_config;
 
 /* Tower weights, device pointers, stacked over layers (L = cfg.layers,

@@ -74,6 +74,14 @@ def test_norm_after_merge_flag_checked(L):
     assert L.vlm_num_patches(ctypes.byref(c), hw, 1) == vlm.ERR_INVALID_ARG
 
 
+def test_negative_sm_budget_rejected(L):
+    cfg = vlm.preset("mistral3", sm_budget=-1)
+    arr = (ctypes.c_int32 * 2)(224, 224)
+    assert L.vlm_num_patches(ctypes.byref(cfg), arr, 1) == vlm.ERR_INVALID_ARG
+    cfg.sm_budget = 64
+    assert L.vlm_num_patches(ctypes.byref(cfg), arr, 1) == 256
+
+
 def test_unsupported_config_rejected(L):
     with pytest.raises(vlm.VlmError) as e:
         vlm.num_patches(vlm.preset("mistral3", head_dim=128, heads=8), [(28, 28)])

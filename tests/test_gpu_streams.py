@@ -180,3 +180,36 @@ def test_side_stream_runs_concurrently_and_matches_oracle():
         compare(got[mask.cuda()], ref_emb, what="side-stream scattered rows")
         assert torch.equal(got[~mask.cuda()].view(torch.int16), text0[~mask.cuda()].view(torch.int16))
     assert not np.array_equal(outs[0].cpu().float().numpy(), outs[1].cpu().float().numpy())
+
+
+@pytest.mark.parametrize("kind", ["bf16", "fp8", "nvfp4"])
+def test_sm_budget_gives_the_same_bits(kind):
+    """vlm_config.sm_budget only changes how many SMs the persistent GEMMs hold
+    and splits attention into successive grids of at most 2 CTAs per budgeted
+    SM: every tile computes the same thing, so the results are bit-identical for
+    every budget (2 SMs, 40, 95, and above the SM count)."""
+    layers, seed = 2, 5
+    tw = tower_to_device(synth.tower_weights(seed, layers, 1024, 4096, 14))
+    pw = tower_to_device(synth.projector_weights(seed, 1024, 2, 5120))
+    extra = {"fp8": dict(fp8_act_scales=synth.fp8_act_scales(layers)),
+             "nvfp4": dict(nvfp4_act_scales=synth.nvfp4_act_scales(layers))}.get(kind, {})
+    pix = pixels_to_device(synth.images(seed, SIZES))
+    outs = []
+    for budget in (0, 2, 40, 95, 100000):
+        cfg = vlm.preset("mistral3", layers=layers, sm_budget=budget)
+        pipe = vlm.ImagePipeline(cfg, tw, pw, SIZES, **extra)
+        before = vlm.launch_count()
+        pipe(pix)
+        launches = vlm.launch_count() - before
+        assert vlm.status_sync(pipe.status) == vlm.OK
+        outs.append((budget, launches, pipe.tower_out.clone(), pipe.embeds.clone()))
+    base = outs[0]
+    qtiles = sum(((h // 14) * (w // 14) + 127) // 128 for h, w in SIZES)
+    for budget, launches, tower, emb in outs[1:]:
+        assert torch.equal(tower, base[2]), budget
+        assert torch.equal(emb, base[3]), budget
+        if 0 < budget < torch.cuda.get_device_properties(0).multi_processor_count:
+            chunk = max(1, 2 * budget // 16)
+            assert launches == base[1] + layers * (-(-qtiles // chunk) - 1), (budget, launches, base[1])
+        else:
+            assert launches == base[1]

@@ -56,6 +56,16 @@ void launch_end(int kclass, cudaStream_t s) {
 
 void note_extra_launches(int n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
 
+thread_local int g_sm_budget = 0;  // set by the entry points for the launches they issue
+
+int sm_budget() {
+  const int n = num_sms();
+  return g_sm_budget > 0 && g_sm_budget < n ? g_sm_budget : n;
+}
+
+SmBudgetScope::SmBudgetScope(int budget) : prev_(g_sm_budget) { g_sm_budget = budget; }
+SmBudgetScope::~SmBudgetScope() { g_sm_budget = prev_; }
+
 int num_sms() {
   static int cache[64] = {};
   int dev = 0;
@@ -93,6 +103,7 @@ int check_config(const vlm_config* c) {
       c->merge <= 0 || c->proj_out <= 0 || !(c->rope_theta > 0.f) || !(c->eps >= 0.f))
     return VLM_ERR_INVALID_ARG;
   if (c->norm_after_merge != 0 && c->norm_after_merge != 1) return VLM_ERR_INVALID_ARG;
+  if (c->sm_budget < 0) return VLM_ERR_INVALID_ARG;
   if (c->head_dim != 64 || c->heads * c->head_dim != c->width) return VLM_ERR_UNSUPPORTED;
   if (c->width % 256 || c->width > 2048 || c->mlp % 128 || c->proj_out % 256) return VLM_ERR_UNSUPPORTED;
   if (c->patch > 64) return VLM_ERR_UNSUPPORTED;
@@ -446,6 +457,7 @@ int vlm_config_preset(int preset, vlm_config* cfg) {
   cfg->eps = 1e-5f;
   cfg->normalize = 1;
   cfg->norm_after_merge = 0;
+  cfg->sm_budget = 0;
   return VLM_OK;
 }
 
@@ -541,6 +553,7 @@ int vlm_encode(const vlm_config* cfg, const float* pixels, const int32_t* image_
                const void* d_packed_tower, void* d_out, void* d_workspace, size_t ws_bytes, int32_t* d_status,
                void* stream) {
   VLM_TRY(check_config(cfg));
+  const SmBudgetScope budget(cfg->sm_budget);
   if (pixels == nullptr || d_packed_tower == nullptr || d_out == nullptr || d_workspace == nullptr)
     return VLM_ERR_INVALID_ARG;
   if (reinterpret_cast<uintptr_t>(d_workspace) & 255) return VLM_ERR_INVALID_ARG;
@@ -632,6 +645,7 @@ int vlm_encode_fp8(const vlm_config* cfg, const float* pixels, const int32_t* im
                    const void* d_packed_tower_fp8, const float* act_scales, void* d_out, void* d_workspace,
                    size_t ws_bytes, int32_t* d_status, void* stream) {
   VLM_TRY(check_config(cfg));
+  const SmBudgetScope budget(cfg->sm_budget);
   if (pixels == nullptr || d_packed_tower_fp8 == nullptr || d_out == nullptr || d_workspace == nullptr)
     return VLM_ERR_INVALID_ARG;
   VLM_TRY(check_act_scales(cfg, act_scales));
@@ -683,6 +697,7 @@ int vlm_patch_embed(const vlm_config* cfg, const float* pixels, const int32_t* i
                     const void* d_packed_tower, float* d_x, void* d_workspace, size_t ws_bytes, int32_t* d_status,
                     void* stream) {
   VLM_TRY(check_config(cfg));
+  const SmBudgetScope budget(cfg->sm_budget);
   if (pixels == nullptr || d_packed_tower == nullptr || d_x == nullptr || d_workspace == nullptr)
     return VLM_ERR_INVALID_ARG;
   if (reinterpret_cast<uintptr_t>(d_workspace) & 255) return VLM_ERR_INVALID_ARG;
@@ -762,6 +777,7 @@ int vlm_encode_nvfp4(const vlm_config* cfg, const float* pixels, const int32_t* 
                      const void* d_packed_tower_nvfp4, const float* act_scales, void* d_out, void* d_workspace,
                      size_t ws_bytes, int32_t* d_status, void* stream) {
   VLM_TRY(check_config(cfg));
+  const SmBudgetScope budget(cfg->sm_budget);
   if (pixels == nullptr || d_packed_tower_nvfp4 == nullptr || d_out == nullptr || d_workspace == nullptr)
     return VLM_ERR_INVALID_ARG;
   VLM_TRY(check_act_scales(cfg, act_scales));
@@ -830,6 +846,7 @@ int vlm_merge_project(const vlm_config* cfg, const void* d_tower_out, const int3
                       const void* d_packed_projector, void* d_out, void* d_workspace, size_t ws_bytes,
                       int32_t* d_status, void* stream) {
   VLM_TRY(check_config(cfg));
+  const SmBudgetScope budget(cfg->sm_budget);
   if (d_tower_out == nullptr || d_packed_projector == nullptr || d_out == nullptr || d_workspace == nullptr)
     return VLM_ERR_INVALID_ARG;
   if (reinterpret_cast<uintptr_t>(d_workspace) & 255) return VLM_ERR_INVALID_ARG;

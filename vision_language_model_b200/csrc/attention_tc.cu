@@ -26,6 +26,8 @@
 // Keys past the block end are masked to -inf; their V rows are finite (rows of
 // the next block) or TMA zero fill (past the sequence). Query tiles never
 // straddle two blocks, so every block's result is independent of the others.
+#include <algorithm>
+
 #include "exp2_poly.cuh"
 #include "kernels.cuh"
 #include "nvfp4.cuh"
@@ -185,6 +187,7 @@ struct AttnArgs {
   int32_t* status;
   float f8_scale;   // E4M3 output: O / l times this before rounding; NVFP4: the global scale
   uint8_t* out_sf;  // NVFP4 block scales
+  int tile_base;    // query tile of blockIdx.x == 0 (launches split along the query tiles)
 };
 
 // OUT: 0 bf16, 1 E4M3, 2 NVFP4 output.
@@ -243,7 +246,7 @@ __global__ void __launch_bounds__(192, 2)
   griddep_launch_dependents();
 
   // this CTA's block, query tile and head
-  const int tile = blockIdx.x, h = blockIdx.y;
+  const int tile = blockIdx.x + args.tile_base, h = blockIdx.y;
   int lo = 0, hi = args.n_blocks - 1;
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
@@ -468,13 +471,26 @@ int launch_attention(const __nv_bfloat16* qkv, int64_t T, int heads, const int32
     attr_done[dev] = true;
   }
   if (out_sf != nullptr && !(f8_scale > 0.f)) return VLM_ERR_INVALID_ARG;
-  AttnArgs args{cu, qt, n_blocks, heads, out, status, f8_scale, out_sf};
-  dim3 grid(total_qtiles, heads);
+  AttnArgs args{cu, qt, n_blocks, heads, out, status, f8_scale, out_sf, 0};
+  auto kern = out_sf != nullptr ? attn_tc_kernel<2> : f8_scale > 0.f ? attn_tc_kernel<1> : attn_tc_kernel<0>;
   launch_begin(KC_ATTN, s);
-  const cudaError_t e =
-      out_sf != nullptr ? launch_pdl(attn_tc_kernel<2>, grid, dim3(192), kSmemBytes, s, tm, args)
-      : f8_scale > 0.f  ? launch_pdl(attn_tc_kernel<1>, grid, dim3(192), kSmemBytes, s, tm, args)
-                        : launch_pdl(attn_tc_kernel<0>, grid, dim3(192), kSmemBytes, s, tm, args);
+  cudaError_t e = cudaSuccess;
+  if (sm_budget() >= num_sms()) {
+    e = launch_pdl(kern, dim3(total_qtiles, heads), dim3(192), kSmemBytes, s, tm, args);
+  } else {
+    // at most two CTAs per budgeted SM at a time: successive grids over the query
+    // tiles, plain launches (a programmatic launch would let the next grid's CTAs
+    // take SMs while they wait for this one)
+    const int chunk = std::max(1, 2 * sm_budget() / heads);
+    int launches = 0;
+    for (int t0 = 0; t0 < total_qtiles && e == cudaSuccess; t0 += chunk) {
+      args.tile_base = t0;
+      kern<<<dim3(std::min(chunk, total_qtiles - t0), heads), dim3(192), kSmemBytes, s>>>(tm, args);
+      e = cudaGetLastError();
+      ++launches;
+    }
+    note_extra_launches(launches - 1);
+  }
   launch_end(KC_ATTN, s);
   return e == cudaSuccess ? VLM_OK : VLM_ERR_CUDA;
 }

@@ -28,6 +28,18 @@ enum KernelClass : int {
 void launch_begin(int kclass, cudaStream_t s);
 void launch_end(int kclass, cudaStream_t s);
 int num_sms();
+// The SMs the current entry point's persistent kernels may hold (vlm_config.sm_budget, else every SM).
+int sm_budget();
+// Sets sm_budget() for the launches issued on this host thread until the scope ends.
+struct SmBudgetScope {
+  explicit SmBudgetScope(int budget);
+  ~SmBudgetScope();
+  SmBudgetScope(const SmBudgetScope&) = delete;
+  SmBudgetScope& operator=(const SmBudgetScope&) = delete;
+
+ private:
+  int prev_;
+};
 
 // Programmatic dependent launch: every kernel of the path is launched with
 // programmatic stream serialisation, signals early that the next kernel may be

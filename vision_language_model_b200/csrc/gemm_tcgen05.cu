@@ -619,7 +619,8 @@ int run_gemm_pair(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMa
     attr_done[dev] = true;
   }
   const int tiles = args.m_tiles * args.n_tiles;
-  const int pairs = tiles < num_sms() / 2 ? tiles : num_sms() / 2;
+  const int max_pairs = sm_budget() / 2 > 0 ? sm_budget() / 2 : 1;
+  const int pairs = tiles < max_pairs ? tiles : max_pairs;
   launch_begin(KC_GEMM, s);
   const cudaError_t e = launch_pdl(kern, dim3(2 * pairs), dim3(192), PairShape::SMEM_BYTES, s, ta, tb, tc, args);
   launch_end(KC_GEMM, s);
@@ -1180,7 +1181,8 @@ int run_gemm_nvfp4(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorM
     attr_done[dev] = true;
   }
   const int tiles = args.m_tiles * args.n_tiles;
-  const int pairs = tiles < num_sms() / 2 ? tiles : num_sms() / 2;
+  const int max_pairs = sm_budget() / 2 > 0 ? sm_budget() / 2 : 1;
+  const int pairs = tiles < max_pairs ? tiles : max_pairs;
   launch_begin(KC_GEMM, s);
   const cudaError_t e =
       launch_pdl(kern, dim3(2 * pairs), dim3(S::THREADS), S::SMEM_BYTES, s, ta, tb, tsa, tsb, tc, args);
@@ -1202,7 +1204,7 @@ int run_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tc
     attr_done[dev] = true;
   }
   const int tiles = args.m_tiles * args.n_tiles;
-  const int grid = tiles < num_sms() ? tiles : num_sms();
+  const int grid = tiles < sm_budget() ? tiles : sm_budget();
   launch_begin(KC_GEMM, s);
   const cudaError_t e = launch_pdl(kern, dim3(grid), dim3(192), S::SMEM_BYTES, s, ta, tb, tc, args);
   launch_end(KC_GEMM, s);

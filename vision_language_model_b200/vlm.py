@@ -39,7 +39,7 @@ class Config(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in
                 ("layers", "width", "heads", "head_dim", "mlp", "patch", "merge", "proj_out", "image_token_id")] + \
                [("rope_theta", ctypes.c_float), ("eps", ctypes.c_float), ("normalize", ctypes.c_int32),
-                ("norm_after_merge", ctypes.c_int32)]
+                ("norm_after_merge", ctypes.c_int32), ("sm_budget", ctypes.c_int32)]
 
     def as_dict(self) -> dict:
         return {n: getattr(self, n) for n, _ in self._fields_}
