@@ -16,16 +16,22 @@ compares every output row with the oracle:
   (vllm.cpp issue, "What we would contribute", item 2), all four compared,
   the scatter bit-exact against the oracle's.
 
+* the E4M3 tower on the 1540x1540 image, and the NVFP4 tower on the packed
+  batch of 8 and on the 16 Pixtral tiles (four compared).
+
 Tolerance: max|gpu - oracle| / max|oracle| <= 2e-2 and every row's cosine
->= 0.999 for floating point; integer and copied rows bit-exact.
+>= 0.999 for floating point (the NVFP4 tower: the end-to-end bounds measured
+from the oracle's own sensitivity, max relative 0.1 and row cosine 0.995);
+integer and copied rows bit-exact.
 """
 import numpy as np
 import pytest
 import torch
 
 from oracle import vlm_oracle as O
-from tests.gpu_util import compare, pixels_to_device, to_oracle, guarded_copy
+from tests.gpu_util import compare, pixels_to_device, to_oracle, tower_to_device, guarded_copy
 from tests.test_gpu_model import _oracle_cfg, _run_gpu, _run_oracle, _setup
+from tests.test_gpu_nvfp4_tower import E2E_MAX_REL, E2E_MIN_COS
 from vision_language_model_b200 import synth, vlm
 
 pytestmark = pytest.mark.gpu
@@ -83,3 +89,56 @@ def test_encode_scatter_four_sequences_every_row_vs_oracle():
     # and the merged sequence's image rows are the oracle's embeddings to tolerance
     mask = ids == 10
     compare(t_gpu[mask.cuda()], ref_emb, what="scattered image rows")
+
+
+# ---------------------------------------------------------------------------
+# The quantised towers at full size (2 layers, every compared row)
+# ---------------------------------------------------------------------------
+
+def _run_quantised(cfg, tw, pw, imgs, sizes, **scales):
+    pipe = vlm.ImagePipeline(cfg, tower_to_device(tw), tower_to_device(pw), sizes, **scales)
+    emb = pipe(pixels_to_device(imgs))
+    assert vlm.status_sync(pipe.status) == vlm.OK
+    return pipe.tower_out.clone(), emb.clone()
+
+
+def test_fp8_1540_image_two_layers_every_row_vs_oracle():
+    """The E4M3 tower on one 1540x1540 image against the oracle's tower_fp8."""
+    sizes = [(1540, 1540)]
+    cfg, tw, pw, imgs = _setup("mistral3", 2, sizes, seed=0)
+    act = synth.fp8_act_scales(2)
+    tower, emb = _run_quantised(cfg, tw, pw, imgs, sizes, fp8_act_scales=act)
+    ocfg = _oracle_cfg(cfg)
+    x_ref = O.tower_fp8([im.double().numpy() for im in imgs], to_oracle(tw), act, ocfg)
+    compare(tower, x_ref, what="fp8 1540 tower")
+    compare(emb, O.projector(x_ref, [(110, 110)], to_oracle(pw), ocfg), what="fp8 1540 projector")
+
+
+def test_nvfp4_packed8_two_layers_every_row_vs_oracle():
+    """The NVFP4 tower on the seeded packed batch of 8 images; the end-to-end
+    bounds are the ones measured from the oracle's own sensitivity (see
+    tests/test_gpu_nvfp4_tower.py, where exactness is checked step by step)."""
+    sizes = synth.packed_sizes(0, 8)
+    cfg, tw, pw, imgs = _setup("mistral3", 2, sizes, seed=0)
+    act = synth.nvfp4_act_scales(2)
+    tower, emb = _run_quantised(cfg, tw, pw, imgs, sizes, nvfp4_act_scales=act)
+    ocfg = _oracle_cfg(cfg)
+    x_ref = O.tower_nvfp4([im.double().numpy() for im in imgs], to_oracle(tw), act, ocfg)
+    compare(tower, x_ref, max_rel=E2E_MAX_REL, min_cos=E2E_MIN_COS, what="nvfp4 packed8 tower")
+    grids = [O.patch_grid(h, w, 14) for h, w in sizes]
+    compare(emb, O.projector(x_ref, grids, to_oracle(pw), ocfg), max_rel=E2E_MAX_REL, min_cos=E2E_MIN_COS,
+            what="nvfp4 packed8 projector")
+
+
+def test_nvfp4_pixtral_16_tiles_two_layers_vs_oracle_on_four():
+    sizes = [(1024, 1024)] * 16
+    cfg, tw, pw, imgs = _setup("pixtral12b", 2, sizes, seed=0)
+    act = synth.nvfp4_act_scales(2)
+    tower, emb = _run_quantised(cfg, tw, pw, imgs, sizes, nvfp4_act_scales=act)
+    picked = [0, 5, 10, 15]
+    ocfg = _oracle_cfg(cfg)
+    x_ref = O.tower_nvfp4([imgs[i].double().numpy() for i in picked], to_oracle(tw), act, ocfg)
+    rows = torch.cat([torch.arange(4096 * i, 4096 * (i + 1)) for i in picked]).cuda()
+    compare(tower[rows], x_ref, max_rel=E2E_MAX_REL, min_cos=E2E_MIN_COS, what=f"nvfp4 pixtral tiles {picked} tower")
+    compare(emb[rows], O.projector(x_ref, [(64, 64)] * 4, to_oracle(pw), ocfg), max_rel=E2E_MAX_REL,
+            min_cos=E2E_MIN_COS, what=f"nvfp4 pixtral tiles {picked} projector")
