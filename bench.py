@@ -773,9 +773,11 @@ def run_ours(args, wl):
     D_, p_ = cfg.width, cfg.patch
     kp_ = -(-3 * p_ * p_ // 64) * 64
     row_bytes = cfg.proj_out * 2
+    # the norm's output per value: bf16, E4M3, or E2M1 codes plus one E4M3 scale per 16 values
+    out_b, out_name = (1.0, "E4M3") if wl.get("fp8") else (0.5 + 1.0 / 16, "NVFP4") if wl.get("nvfp4") else (2.0, "bf16")
     mb = {
-        "rmsnorm": (2 * cfg.layers * T * D_ * (4 + 2) + T * D_ * 4, ms_norm,
-                    "per launch: fp32 row read + bf16 row written (+ the fp32 write-back of ln_pre once)"),
+        "rmsnorm": (2 * cfg.layers * T * D_ * (4 + out_b) + T * D_ * 4, ms_norm,
+                    f"per launch: fp32 row read + the {out_name} row written (+ the fp32 write-back of ln_pre once)"),
         "patch_gather": (T * (3 * p_ * p_ * 4 + kp_ * 2), ms_im2col, "fp32 pixels read + bf16 patch rows written"),
         "merge_gather": (2 * T * D_ * 2, ms_merge, "bf16 tower rows read + bf16 merged rows written"),
         "scatter": (2 * Tm * row_bytes + ids.numel() * 8, ms_scatter,
