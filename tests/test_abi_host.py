@@ -243,6 +243,60 @@ def test_nvfp4_scale_sizes_and_argument_errors_return_before_launch(L):
     assert L.vlm_amax_scale(None, vlm.DTYPE_BF16, 10, 2688.0, fake, None) == vlm.ERR_INVALID_ARG
 
 
+def test_nvfp4_tower_entry_points_reject_bad_arguments_before_launch(L):
+    """Every case fails validation before any CUDA call (the fake pointers are never dereferenced)."""
+    fake, st = ctypes.c_void_p(256), ctypes.c_void_p(1024)
+    gx = L.vlm_gemm_nvfp4_ex
+    args = lambda epi, n, c_sf=fake, sg=1.0, pos=fake, rope=fake, rc=256: (
+        epi, fake, fake, fake, fake, fake, fake, 256, n, 256, fake, c_sf, sg, pos, rope, rc, st, None)
+    assert gx(*args(vlm.EPI_ROPE, 512, pos=None)) == vlm.ERR_INVALID_ARG          # RoPE without positions
+    assert gx(*args(vlm.EPI_ROPE, 512, rc=32)) == vlm.ERR_INVALID_ARG             # rope_cols not whole heads
+    assert gx(*args(vlm.EPI_ROPE, 384)) == vlm.ERR_UNSUPPORTED                    # RoPE needs N % 256 == 0
+    assert gx(*args(vlm.EPI_SWIGLU, 384)) == vlm.ERR_UNSUPPORTED
+    assert gx(*args(vlm.EPI_SWIGLU, 512, c_sf=None)) == vlm.ERR_INVALID_ARG       # no hidden-state scales
+    assert gx(*args(vlm.EPI_SWIGLU, 512, sg=0.0)) == vlm.ERR_INVALID_ARG          # global scale not > 0
+    assert gx(*args(vlm.EPI_SWIGLU, 512, c_sf=ctypes.c_void_p(258))) == vlm.ERR_INVALID_ARG
+    assert gx(*args(vlm.EPI_GELU, 512)) == vlm.ERR_UNSUPPORTED
+    # RMSNorm to NVFP4: scale, scale buffer, width
+    assert L.vlm_rmsnorm_nvfp4(fake, None, fake, fake, fake, 8, 1024, 1e-5, 0.0, None) == vlm.ERR_INVALID_ARG
+    assert L.vlm_rmsnorm_nvfp4(fake, None, fake, fake, None, 8, 1024, 1e-5, 1.0, None) == vlm.ERR_INVALID_ARG
+    assert L.vlm_rmsnorm_nvfp4(fake, None, fake, fake, fake, 8, 100, 1e-5, 1.0, None) == vlm.ERR_UNSUPPORTED
+    assert L.vlm_rmsnorm_nvfp4(fake, None, fake, fake, fake, 0, 1024, 1e-5, 1.0, None) == vlm.OK
+    # attention to NVFP4: scale buffer, scale, alignment of the codes
+    cu = (ctypes.c_int32 * 2)(0, 128)
+    att = L.vlm_attention_nvfp4
+    assert att(fake, 128, 2, 64, cu, 1, fake, None, 1.0, fake, 4096, st, None) == vlm.ERR_INVALID_ARG
+    assert att(fake, 128, 2, 64, cu, 1, fake, fake, -1.0, fake, 4096, st, None) == vlm.ERR_INVALID_ARG
+    assert att(fake, 128, 2, 64, cu, 1, ctypes.c_void_p(264), fake, 1.0, fake, 4096, st, None) == vlm.ERR_INVALID_ARG
+    # packing and encoding
+    cfg = vlm.preset("mistral3", layers=1)
+    tw = vlm.TowerWeights(*([fake.value] * len(vlm.TowerWeights._fields_)))
+    good = (ctypes.c_float * 4)(1.0, 1.0, 1.0, 1.0)
+    bad = (ctypes.c_float * 4)(1.0, 0.0, 1.0, 1.0)
+    need = L.vlm_tower_nvfp4_packed_bytes(ctypes.byref(cfg))
+    assert need > 0
+    pk = L.vlm_pack_tower_nvfp4
+    assert pk(ctypes.byref(cfg), ctypes.byref(tw), bad, fake, need, None) == vlm.ERR_INVALID_ARG
+    assert pk(ctypes.byref(cfg), None, good, fake, need, None) == vlm.ERR_INVALID_ARG
+    assert pk(ctypes.byref(cfg), ctypes.byref(tw), good, ctypes.c_void_p(272), need, None) == vlm.ERR_INVALID_ARG
+    assert pk(ctypes.byref(cfg), ctypes.byref(tw), good, fake, need - 1, None) == vlm.ERR_WORKSPACE
+    hw = (ctypes.c_int32 * 2)(224, 224)
+    ws = L.vlm_encode_nvfp4_workspace_size(ctypes.byref(cfg), hw, 1)
+    assert ws > L.vlm_encode_workspace_size(ctypes.byref(cfg), hw, 1)   # plus the inputs' block scales
+    enc = L.vlm_encode_nvfp4
+    assert enc(ctypes.byref(cfg), None, hw, 1, fake, good, fake, fake, ws, st, None) == vlm.ERR_INVALID_ARG
+    assert enc(ctypes.byref(cfg), fake, hw, 1, fake, good, fake, ctypes.c_void_p(272), ws, st, None) == \
+        vlm.ERR_INVALID_ARG
+    assert enc(ctypes.byref(cfg), fake, hw, 1, fake, good, fake, fake, ws - 1, st, None) == vlm.ERR_WORKSPACE
+    assert enc(ctypes.byref(cfg), fake, hw, 1, fake, bad, fake, fake, ws, st, None) == vlm.ERR_INVALID_ARG
+    # the patch embed alone
+    pe = L.vlm_patch_embed
+    ws_pe = L.vlm_encode_workspace_size(ctypes.byref(cfg), hw, 1)
+    assert pe(ctypes.byref(cfg), fake, hw, 1, fake, None, fake, ws_pe, st, None) == vlm.ERR_INVALID_ARG
+    assert pe(ctypes.byref(cfg), fake, hw, 1, fake, fake, ctypes.c_void_p(272), ws_pe, st, None) == vlm.ERR_INVALID_ARG
+    assert pe(ctypes.byref(cfg), fake, hw, 1, fake, fake, fake, ws_pe - 1, st, None) == vlm.ERR_WORKSPACE
+
+
 def test_gemm_tile_counts_that_overflow_32_bits_are_rejected(L):
     """Tile indices and scale-atom rows are 32-bit in the kernels: shapes whose
     counts would not fit are refused on the host before any launch."""

@@ -363,3 +363,30 @@ def test_encode_nvfp4_rejects_bad_inputs():
     small = torch.empty(16, dtype=torch.uint8, device="cuda")
     with pytest.raises(vlm.VlmError):
         vlm.encode_nvfp4(cfg, pix, [(112, 112)], packed, act, workspace=small)
+
+
+def test_encode_nvfp4_zero_layers_is_the_bf16_encoder():
+    """Without blocks the NVFP4 encoder is patch embed + ln_pre, as the bf16 one."""
+    sizes = [(224, 224), (112, 168)]
+    cfg, tw, pw, act, imgs = _nvfp4_setup(sizes, layers=0)
+    twd, pix = tower_to_device(tw), pixels_to_device(imgs)
+    a = vlm.encode_nvfp4(cfg, pix, sizes, vlm.pack_tower_nvfp4(cfg, twd, act), act)
+    b = vlm.encode(cfg, pix, sizes, vlm.pack_tower(cfg, twd))
+    torch.cuda.synchronize()
+    assert torch.equal(a, b)
+
+
+def test_encode_nvfp4_tiny_batch_vs_oracle():
+    """28 patches: every GEMM's rows are a fraction of one 128-row scale group
+    (the padding rows' scales stay 0) and of one 256-row tile."""
+    sizes = [(28, 28), (56, 84)]
+    cfg, tw, pw, act, imgs = _nvfp4_setup(sizes, layers=2, seed=11)
+    pipe = vlm.ImagePipeline(cfg, tower_to_device(tw), tower_to_device(pw), sizes, nvfp4_act_scales=act)
+    emb = pipe(pixels_to_device(imgs))
+    assert vlm.status_sync(pipe.status) == vlm.OK
+    ocfg = dict(O.MISTRAL3, layers=2)
+    x_ref = O.tower_nvfp4([im.double().numpy() for im in imgs], to_oracle(tw), act, ocfg)
+    compare(pipe.tower_out, x_ref, max_rel=E2E_MAX_REL, min_cos=E2E_MIN_COS, what="nvfp4 tiny tower")
+    grids = [O.patch_grid(h, w, 14) for h, w in sizes]
+    compare(emb, O.projector(x_ref, grids, to_oracle(pw), ocfg), max_rel=E2E_MAX_REL, min_cos=E2E_MIN_COS,
+            what="nvfp4 tiny projector")
