@@ -3,7 +3,7 @@
 //   o_t = sum_u softmax_u(q_t . k_u / 8) v_u   over the keys u of block b only.
 //
 // One CTA = one 128-query tile of one block and one head; two CTAs share an
-// SM so one CTA's softmax overlaps the other's MMAs. 6 warps:
+// SM so one CTA's softmax overlaps the other's MMAs. 10 warps:
 //   warp 0      TMA: the Q tile once, then K and V tiles of 128 keys into two
 //               2-stage rings (128-byte swizzle). A K stage is released when
 //               S = Q K^T has read it and a V stage when O += P V has, so the
@@ -12,16 +12,20 @@
 //                 S  = Q K^T      (tcgen05.mma kind::f16, M=128 N=128, A and B in smem)
 //                 O += P V        (M=128 N=64, A = P in TMEM, B = V in smem, MN-major)
 //               S_{j+1} is issued as soon as the softmax has copied S_j out.
-//   warps 2..5  softmax, one thread per query row = TMEM lane: reads its S row
-//               (128 fp32), finds the tile max with four short 3-input-max
-//               chains, keeps a running max m (log2 units) that only moves when
-//               the tile max exceeds it by more than 8 (otherwise the stale max
-//               is kept; P stays <= 2^8 and the final division by l is exact),
-//               computes P = 2^(s*log2e/8 - m) with packed fp32x2 FMAs and MUFU
-//               ex2 (one pair in eight from an FMA-pipe polynomial), writes P
-//               to TMEM as bf16, sums the fp32 values into l with
-//               packed adds, rescales its O row when m moved, and finally writes
-//               O / l.
+//   warps 2..9  softmax, two threads per query row (TMEM lane): warp w and
+//               warp w + 4 read the same 32 lanes, keys [0,64) and [64,128) of
+//               the tile (64 fp32 each). Each finds its half's max with four
+//               short 3-input-max chains; the two halves exchange them through
+//               shared memory (a 64-thread named barrier per row group), so
+//               both keep the same running max m (log2 units), which only
+//               moves when the tile max exceeds it by more than 8 (otherwise
+//               the stale max is kept; P stays <= 2^8 and the final division
+//               by l is exact). Each computes its 64 P = 2^(s*log2e/8 - m) with
+//               packed fp32x2 FMAs and MUFU ex2 (one pair in eight from an
+//               FMA-pipe polynomial), writes them to TMEM as bf16, sums the
+//               fp32 values into its part of l with packed adds, rescales its
+//               32 O columns when m moved, and finally writes those columns
+//               of O / l (l = the sum of both parts).
 // TMEM: S in columns [0,128), P in [128,192) (bf16 pairs), O in [192,256).
 // Keys past the block end are masked to -inf; their V rows are finite (rows of
 // the next block) or TMA zero fill (past the sequence). Query tiles never
@@ -43,10 +47,13 @@ namespace {
 constexpr int BQ = kAttnBQ;  // 128
 constexpr int BKV = 128;
 constexpr int DH = 64;
+constexpr int HK = BKV / 2;  // keys per softmax thread
+constexpr int kThreads = 320;
 constexpr int kKStages = 2;  // K ring: a stage is free once S = Q K^T has read it
 constexpr int kVStages = 2;  // V ring: a stage is free once O += P V has read it
 constexpr int kTileBytes = 128 * DH * 2;  // 16 KiB: 128 rows x 128 bytes
-constexpr int kSmemBytes = (1 + kKStages + kVStages) * kTileBytes + 256 + 1024;
+constexpr int kXchOffset = (1 + kKStages + kVStages) * kTileBytes + 256;
+constexpr int kSmemBytes = kXchOffset + 3072 + 1024;
 constexpr uint32_t kColS = 0, kColP = 128, kColO = 192, kTmemCols = 256;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
@@ -83,14 +90,15 @@ __device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
   return d;
 }
 
-// Row maximum of 128 values with four independent chains of 3-input max.
-__device__ __forceinline__ float row_max(const uint32_t (&u)[BKV]) {
+// Row maximum of N values with four independent chains of 3-input max.
+template <int N>
+__device__ __forceinline__ float row_max(const uint32_t (&u)[N]) {
   constexpr int NC = 4;
   float m[NC];
 #pragma unroll
   for (int i = 0; i < NC; ++i) m[i] = -INFINITY;
 #pragma unroll
-  for (int c = 0; c < BKV; c += 2 * NC) {
+  for (int c = 0; c < N; c += 2 * NC) {
 #pragma unroll
     for (int i = 0; i < NC; ++i) m[i] = max3f(m[i], __uint_as_float(u[c + 2 * i]), __uint_as_float(u[c + 2 * i + 1]));
   }
@@ -101,32 +109,39 @@ __device__ __forceinline__ float row_max(const uint32_t (&u)[BKV]) {
   return m[0];
 }
 
-// The row's 64 packed bf16 P words in one store: storing them as two 32-column
-// halves from copies made the compiler keep both and spill.
-__device__ __forceinline__ void tmem_st64(uint32_t taddr, const uint32_t (&r)[64]) {
+// 32 lanes x 64 columns of 32-bit TMEM words into registers (one lane per
+// thread), waiting for completion inside the same asm block.
+__device__ __forceinline__ void tmem_ld64(uint32_t taddr, uint32_t (&r)[64]) {
   asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x64.b32 [%0], "
-      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, "
-      "%17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32, "
-      "%33, %34, %35, %36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47, %48, "
-      "%49, %50, %51, %52, %53, %54, %55, %56, %57, %58, %59, %60, %61, %62, %63, %64};" ::"r"(taddr),
-      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
-      "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]),
-      "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]),
-      "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31]), "r"(r[32]),
-      "r"(r[33]), "r"(r[34]), "r"(r[35]), "r"(r[36]), "r"(r[37]), "r"(r[38]), "r"(r[39]), "r"(r[40]),
-      "r"(r[41]), "r"(r[42]), "r"(r[43]), "r"(r[44]), "r"(r[45]), "r"(r[46]), "r"(r[47]), "r"(r[48]),
-      "r"(r[49]), "r"(r[50]), "r"(r[51]), "r"(r[52]), "r"(r[53]), "r"(r[54]), "r"(r[55]), "r"(r[56]),
-      "r"(r[57]), "r"(r[58]), "r"(r[59]), "r"(r[60]), "r"(r[61]), "r"(r[62]), "r"(r[63])
+      "tcgen05.ld.sync.aligned.32x32b.x64.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, "
+      "%32, %33, %34, %35, %36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47, "
+      "%48, %49, %50, %51, %52, %53, %54, %55, %56, %57, %58, %59, %60, %61, %62, %63}, [%64];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]),
+        "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]), "=r"(r[38]), "=r"(r[39]),
+        "=r"(r[40]), "=r"(r[41]), "=r"(r[42]), "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]),
+        "=r"(r[48]), "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]),
+        "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]), "=r"(r[62]), "=r"(r[63])
+      : "r"(taddr)
       : "memory");
 }
 
+// The two softmax warps of one row group (warps w and w + 4) meet here: a
+// named barrier of 64 threads, id 1 + the TMEM lane group.
+__device__ __forceinline__ void pair_sync(int q) {
+  asm volatile("bar.sync %0, 64;" ::"r"(1 + q) : "memory");
+}
 
 // One pair of scores in kPolyPairEvery takes its two exponentials from
 // exp2_poly (FMA and ALU pipes) instead of ex2.approx (MUFU), so the two kinds
 // of pipe share the softmax's exponentials. MUFU is the softmax's bottleneck;
-// one pair in eight is the largest share that still fits the 168 registers a
-// thread has at 2 CTAs per SM without spilling.
+// one pair in eight measured fastest: one in four fits the 96 registers a
+// thread has at 2 CTAs of 320 threads per SM but is no faster, one in three
+// spills.
 #ifndef VLM_ATTN_POLY_PAIR_EVERY
 #define VLM_ATTN_POLY_PAIR_EVERY 8
 #endif
@@ -147,16 +162,16 @@ __device__ __forceinline__ float exp2_poly(float x) {
   return __int_as_float(__float_as_int(p) + (__float_as_int(j) << 23));
 }
 
-// p_c = 2^(s_c * sl2 - m) for the row's 128 scores, packed as bf16 pairs into
+// p_c = 2^(s_c * sl2 - m) for the thread's N scores of the row, packed as bf16 pairs into
 // pk; returns sum_c p_c (fp32, before rounding). The elements are independent.
 // kPoly: let exp2_poly take one pair in kPolyPairEvery (never on a tile with
 // masked keys, whose weights must be exactly 0).
-template <bool kPoly>
-__device__ __forceinline__ float row_exp(const uint32_t (&u)[BKV], uint64_t sl2x2, float m, uint32_t (&pk)[BKV / 2]) {
+template <bool kPoly, int N>
+__device__ __forceinline__ float row_exp(const uint32_t (&u)[N], uint64_t sl2x2, float m, uint32_t (&pk)[N / 2]) {
   const uint64_t negm2 = pair_f32(-m);
   uint64_t acc[4] = {0, 0, 0, 0};
 #pragma unroll
-  for (int c = 0; c < BKV; c += 2) {
+  for (int c = 0; c < N; c += 2) {
     float x0, x1, p0, p1;
     unpack2(fma2(pack2(u[c], u[c + 1]), sl2x2, negm2), x0, x1);
     if (kPoly && kPolyPairEvery > 0 && (c >> 1) % (kPolyPairEvery > 0 ? kPolyPairEvery : 1) == kPolyPairEvery - 1) {
@@ -192,7 +207,7 @@ struct AttnArgs {
 
 // OUT: 0 bf16, 1 E4M3, 2 NVFP4 output.
 template <int OUT>
-__global__ void __launch_bounds__(192, 2)
+__global__ void __launch_bounds__(kThreads, 2)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, const AttnArgs args) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -226,8 +241,8 @@ __global__ void __launch_bounds__(192, 2)
       mbar_init(smem_u32(v_empty + s), 1);
     }
     mbar_init(smem_u32(s_full), 1);
-    mbar_init(smem_u32(s_free), 128);
-    mbar_init(smem_u32(p_full), 128);
+    mbar_init(smem_u32(s_free), 256);
+    mbar_init(smem_u32(p_full), 256);
     mbar_init(smem_u32(o_done), 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -316,113 +331,121 @@ __global__ void __launch_bounds__(192, 2)
       }
     }
   } else {
-    // softmax: this thread owns query row r of the tile (TMEM lane r)
+    // softmax, warps 2..9: warp w and warp w + 4 own the same 32 query rows
+    // (TMEM lanes 32 (w % 4) ..), keys [0, 64) and [64, 128) of every tile. The
+    // pair agrees on the row maximum through shared memory; each keeps its own
+    // part of the row sum and owns 32 of the 64 O columns.
     const int q = warp & 3;
+    const int hf = (warp - 2) >> 2;
     const int r = q * 32 + lane;
     const uint32_t trow = tmem + (static_cast<uint32_t>(q * 32) << 16);
+    float* xmax = reinterpret_cast<float*>(smem + kXchOffset);  // [tile parity][half][row]
+    float* xsum = xmax + 512;                                   // [half][row]
     const float sl2 = 1.4426950408889634f * 0.125f;  // log2(e) / sqrt(64)
     const uint64_t sl2x2 = pair_f32(sl2);
     float m = -INFINITY, l = 0.f;
     bool ok = true;
+    // A warp whose wait failed stays in the loop and keeps meeting its partner
+    // at pair_sync, doing nothing else, so the partner never waits for it.
     for (int j = 0; j < n_kv; ++j) {
-      if (!mbar_wait_warp(smem_u32(s_full), j & 1, abort_v, args.status)) { ok = false; break; }
+      if (ok) ok = mbar_wait_warp(smem_u32(s_full), j & 1, abort_v, args.status);
+      if (!ok) {
+        pair_sync(q);
+        continue;
+      }
       tc_fence_after();
-      uint32_t u[BKV];
-      tmem_ld128(trow + kColS, u);
+      uint32_t u[HK];
+      tmem_ld64(trow + kColS + HK * hf, u);
       tc_fence_before();
       mbar_arrive(smem_u32(s_free));
-
-      const int nvalid = kend - (kbeg + j * BKV);
-      if (nvalid < BKV) {  // last tile of the block: keys past its end get probability 0
+      const int nvalid = kend - (kbeg + j * BKV) - HK * hf;
+      if (nvalid < HK) {  // keys past the block end get probability 0
 #pragma unroll
-        for (int c = 0; c < BKV; ++c)
+        for (int c = 0; c < HK; ++c)
           if (c >= nvalid) u[c] = __float_as_uint(-INFINITY);
       }
-      const float m_cand = row_max(u) * sl2;
+      const float m_own = row_max(u) * sl2;
+      xmax[((j & 1) * 2 + hf) * BQ + r] = m_own;
+      pair_sync(q);
+      const float m_cand = fmaxf(m_own, xmax[((j & 1) * 2 + (hf ^ 1)) * BQ + r]);
       const bool grow = m_cand > m + kRescaleThreshold;
       const float m_new = grow ? m_cand : m;
       const float corr = grow ? ex2(m - m_new) : 1.0f;
       const bool any_grow = __any_sync(0xffffffffu, grow);
       m = m_new;
-      uint32_t pk[BKV / 2];
-      const float sum = nvalid < BKV ? row_exp<false>(u, sl2x2, m, pk) : row_exp<true>(u, sl2x2, m, pk);
+      uint32_t pk[HK / 2];
+      const float sum = nvalid < HK ? row_exp<false>(u, sl2x2, m, pk) : row_exp<true>(u, sl2x2, m, pk);
       l = l * corr + sum;
 
       if (j > 0) {
         // PV of the previous tile must be done before O is rescaled and P overwritten
-        if (!mbar_wait_warp(smem_u32(o_done), (j - 1) & 1, abort_v, args.status)) { ok = false; break; }
+        ok = mbar_wait_warp(smem_u32(o_done), (j - 1) & 1, abort_v, args.status);
+        if (!ok) continue;
         tc_fence_after();
-        if (any_grow) {
-#pragma unroll
-          for (int c = 0; c < DH; c += 32) {
-            uint32_t o[32];
-            tmem_ld32(trow + kColO + c, o);
-#pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * corr);
-            tmem_st32(trow + kColO + c, o);
-          }
-        }
       }
-      tmem_st64(trow + kColP, pk);
+      tmem_st32(trow + kColP + 32 * hf, pk);
+      if (j > 0 && any_grow) {
+        uint32_t o[32];
+        tmem_ld32(trow + kColO + 32 * hf, o);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * corr);
+        tmem_st32(trow + kColO + 32 * hf, o);
+      }
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(smem_u32(p_full));
     }
+    xsum[hf * BQ + r] = l;
+    pair_sync(q);
+    l += xsum[(hf ^ 1) * BQ + r];
     if (ok && mbar_wait_warp(smem_u32(o_done), (n_kv - 1) & 1, abort_v, args.status)) {
       tc_fence_after();
       const float inv = 1.0f / l;
       const int row = q0 + r;
+      const int c = 32 * hf;  // this thread's O columns
       if constexpr (OUT == 2) {
         // blocks of 16 values along the row: four per head, two per 32-column load
         uint8_t* dst = static_cast<uint8_t*>(args.out) + static_cast<int64_t>(row) * (D / 2) + h * (DH / 2);
         const float sg = args.f8_scale, six_sg = 6.0f * sg;
+        uint32_t o[32];
+        tmem_ld32(trow + kColO + c, o);
+        if (row < kend && VLM_DCHECK(kend <= __ldg(args.cu + args.n_blocks))) {
+          uint32_t sbs = 0;
+          uint2 codes[2];
 #pragma unroll
-        for (int c = 0; c < DH; c += 32) {
-          uint32_t o[32];
-          tmem_ld32(trow + kColO + c, o);
-          if (row < kend && VLM_DCHECK(kend <= __ldg(args.cu + args.n_blocks))) {
-            uint32_t sbs = 0;
-            uint2 codes[2];
+          for (int b = 0; b < 2; ++b) {
+            float v[16], amax = 0.0f;
 #pragma unroll
-            for (int b = 0; b < 2; ++b) {
-              float v[16], amax = 0.0f;
-#pragma unroll
-              for (int k = 0; k < 16; ++k) {
-                v[k] = __uint_as_float(o[16 * b + k]) * inv;
-                amax = fmaxf(amax, fabsf(v[k]));
-              }
-              sbs |= nvfp4_quant16(v, amax, sg, six_sg, codes[b]) << (8 * b);
+            for (int k = 0; k < 16; ++k) {
+              v[k] = __uint_as_float(o[16 * b + k]) * inv;
+              amax = fmaxf(amax, fabsf(v[k]));
             }
-            *reinterpret_cast<uint4*>(dst + c / 2) = make_uint4(codes[0].x, codes[0].y, codes[1].x, codes[1].y);
-            // blocks (h DH + c) / 16 and the next: two adjacent scale bytes
-            *reinterpret_cast<uint16_t*>(args.out_sf + nvfp4_sf_offset(row, (h * DH + c) / 16, D)) =
-                static_cast<uint16_t>(sbs);
+            sbs |= nvfp4_quant16(v, amax, sg, six_sg, codes[b]) << (8 * b);
           }
+          *reinterpret_cast<uint4*>(dst + c / 2) = make_uint4(codes[0].x, codes[0].y, codes[1].x, codes[1].y);
+          // blocks (h DH + c) / 16 and the next: two adjacent scale bytes
+          *reinterpret_cast<uint16_t*>(args.out_sf + nvfp4_sf_offset(row, (h * DH + c) / 16, D)) =
+              static_cast<uint16_t>(sbs);
         }
       } else if constexpr (OUT == 1) {
         const float f = inv * args.f8_scale;
         uint8_t* dst = static_cast<uint8_t*>(args.out) + static_cast<int64_t>(row) * D + h * DH;
+        uint32_t o[32];
+        tmem_ld32(trow + kColO + c, o);
+        if (row < kend && VLM_DCHECK(kend <= __ldg(args.cu + args.n_blocks))) {
+          uint4* d4 = reinterpret_cast<uint4*>(dst + c);
 #pragma unroll
-        for (int c = 0; c < DH; c += 32) {
-          uint32_t o[32];
-          tmem_ld32(trow + kColO + c, o);
-          if (row < kend && VLM_DCHECK(kend <= __ldg(args.cu + args.n_blocks))) {
-            uint4* d4 = reinterpret_cast<uint4*>(dst + c);
+          for (int jj = 0; jj < 2; ++jj) {
+            uint32_t w[4];
 #pragma unroll
-            for (int jj = 0; jj < 2; ++jj) {
-              uint32_t w[4];
-#pragma unroll
-              for (int k = 0; k < 4; ++k)
-                w[k] = pack_e4m3x4(__uint_as_float(o[16 * jj + 4 * k]) * f, __uint_as_float(o[16 * jj + 4 * k + 1]) * f,
-                                   __uint_as_float(o[16 * jj + 4 * k + 2]) * f, __uint_as_float(o[16 * jj + 4 * k + 3]) * f);
-              d4[jj] = make_uint4(w[0], w[1], w[2], w[3]);
-            }
+            for (int k = 0; k < 4; ++k)
+              w[k] = pack_e4m3x4(__uint_as_float(o[16 * jj + 4 * k]) * f, __uint_as_float(o[16 * jj + 4 * k + 1]) * f,
+                                 __uint_as_float(o[16 * jj + 4 * k + 2]) * f, __uint_as_float(o[16 * jj + 4 * k + 3]) * f);
+            d4[jj] = make_uint4(w[0], w[1], w[2], w[3]);
           }
         }
       } else {
-      __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(args.out) + static_cast<int64_t>(row) * D + h * DH;
-#pragma unroll
-      for (int c = 0; c < DH; c += 32) {
+        __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(args.out) + static_cast<int64_t>(row) * D + h * DH;
         uint32_t o[32];
         tmem_ld32(trow + kColO + c, o);
         if (row < kend && VLM_DCHECK(kend <= __ldg(args.cu + args.n_blocks))) {
@@ -434,7 +457,6 @@ __global__ void __launch_bounds__(192, 2)
                                 pack_bf16x2(__uint_as_float(o[8 * jj + 4]) * inv, __uint_as_float(o[8 * jj + 5]) * inv),
                                 pack_bf16x2(__uint_as_float(o[8 * jj + 6]) * inv, __uint_as_float(o[8 * jj + 7]) * inv));
         }
-      }
       }
     }
   }
@@ -476,7 +498,7 @@ int launch_attention(const __nv_bfloat16* qkv, int64_t T, int heads, const int32
   launch_begin(KC_ATTN, s);
   cudaError_t e = cudaSuccess;
   if (sm_budget() >= num_sms()) {
-    e = launch_pdl(kern, dim3(total_qtiles, heads), dim3(192), kSmemBytes, s, tm, args);
+    e = launch_pdl(kern, dim3(total_qtiles, heads), dim3(kThreads), kSmemBytes, s, tm, args);
   } else {
     // at most two CTAs per budgeted SM at a time: successive grids over the query
     // tiles, plain launches (a programmatic launch would let the next grid's CTAs
@@ -485,7 +507,7 @@ int launch_attention(const __nv_bfloat16* qkv, int64_t T, int heads, const int32
     int launches = 0;
     for (int t0 = 0; t0 < total_qtiles && e == cudaSuccess; t0 += chunk) {
       args.tile_base = t0;
-      kern<<<dim3(std::min(chunk, total_qtiles - t0), heads), dim3(192), kSmemBytes, s>>>(tm, args);
+      kern<<<dim3(std::min(chunk, total_qtiles - t0), heads), dim3(kThreads), kSmemBytes, s>>>(tm, args);
       e = cudaGetLastError();
       ++launches;
     }
