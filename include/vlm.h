@@ -277,6 +277,37 @@ VLM_API int vlm_scatter(const int64_t* d_input_ids, int64_t n_tokens, int64_t im
                 void* stream);
 
 /* ---------------------------------------------------------------------------
+ * vlm_merge_project_scatter -- vlm_merge_project followed by vlm_scatter in
+ * one call, without the [T_m, proj_out] embedding buffer between them: the
+ * projector's last linear (W2) writes each merged token's row straight to its
+ * placeholder row of text_embeds ([K] Mistral3Model: the image features
+ * replace the image_token_id positions of the token embeddings; [I] item 2).
+ *
+ * The rows written are bit-identical to those that vlm_merge_project followed
+ * by vlm_scatter(d_input_ids, n_tokens, cfg->image_token_id, ...) would write;
+ * all other rows of text_embeds are left untouched.
+ *
+ * d_tower_out, image_hw, n_images, d_packed_projector: as for
+ *   vlm_merge_project.
+ * d_input_ids: device int64 [n_tokens]; the placeholder is
+ *   cfg->image_token_id; n_tokens >= 1 (VLM_ERR_BAD_SHAPE otherwise).
+ * d_text_embeds: device bf16 [n_tokens, proj_out], 16-byte aligned, updated in
+ *   place.
+ * If the number of placeholders differs from T_m (vlm_num_merged) the call
+ *   writes no row and sets *d_status = VLM_ERR_COUNT_MISMATCH.
+ * d_workspace: 256-byte aligned, at least
+ *   vlm_merge_project_scatter_workspace_size(cfg, image_hw, n_images,
+ *   n_tokens) bytes (VLM_ERR_WORKSPACE otherwise). Host-side argument errors
+ *   are returned before anything is launched.
+ * ------------------------------------------------------------------------- */
+VLM_API size_t vlm_merge_project_scatter_workspace_size(const vlm_config* cfg, const int32_t* image_hw,
+                                                        int n_images, int64_t n_tokens);
+VLM_API int vlm_merge_project_scatter(const vlm_config* cfg, const void* d_tower_out, const int32_t* image_hw,
+                                      int n_images, const void* d_packed_projector, const int64_t* d_input_ids,
+                                      int64_t n_tokens, void* d_text_embeds, void* d_workspace, size_t ws_bytes,
+                                      int32_t* d_status, void* stream);
+
+/* ---------------------------------------------------------------------------
  * vlm_scatter_noalloc -- vlm_scatter for callers that cannot allocate device
  * memory. The pages have no counterpart: this is a library convenience.
  *

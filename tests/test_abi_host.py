@@ -336,3 +336,29 @@ def test_debug_library_loads_and_exports_every_symbol():
     assert D.vlm_debug_build() == 1
     D.vlm_debug_checks.restype = ctypes.c_int
     assert D.vlm_debug_checks(None) == vlm.ERR_INVALID_ARG
+
+
+def test_merge_project_scatter_rejects_bad_arguments_before_launch(L):
+    """Every case fails validation before any CUDA call (the fake pointers are never dereferenced)."""
+    fake, st = ctypes.c_void_p(256), ctypes.c_void_p(1024)
+    cfg = vlm.preset("mistral3", layers=1)
+    hw = (ctypes.c_int32 * 2)(224, 224)
+    n = 300
+    ws = L.vlm_merge_project_scatter_workspace_size(ctypes.byref(cfg), hw, 1, n)
+    assert ws >= L.vlm_merge_project_workspace_size(ctypes.byref(cfg), hw, 1) + L.vlm_scatter_workspace_size(n)
+    assert L.vlm_merge_project_scatter_workspace_size(ctypes.byref(cfg), hw, 1, 0) == 0
+    base = [ctypes.byref(cfg), fake, hw, 1, fake, fake, n, fake, fake, ws, st, None]
+
+    def call(i=None, v=None):
+        a = list(base)
+        if i is not None:
+            a[i] = v
+        return L.vlm_merge_project_scatter(*a)
+
+    for i in (1, 4, 5, 7, 8, 10):                          # tower_out, projector, ids, text, workspace, status
+        assert call(i, None) == vlm.ERR_INVALID_ARG, i
+    assert call(6, 0) == vlm.ERR_BAD_SHAPE                 # no ids
+    assert call(8, ctypes.c_void_p(384)) == vlm.ERR_INVALID_ARG   # workspace not 256-byte aligned
+    assert call(7, ctypes.c_void_p(264)) == vlm.ERR_INVALID_ARG   # text rows not 16-byte aligned
+    assert call(9, ws - 1) == vlm.ERR_WORKSPACE
+    assert call(2, (ctypes.c_int32 * 2)(225, 224)) != vlm.OK      # not on the merged-patch grid

@@ -8,6 +8,7 @@
 #include <vector>
 
 #include "../../include/vlm_kernels.h"
+#include "gemm_rows.cuh"
 #include "kernels.cuh"
 #include "nvfp4.cuh"
 
@@ -835,6 +836,30 @@ int vlm_encode_nvfp4(const vlm_config* cfg, const float* pixels, const int32_t* 
   return VLM_OK;
 }
 
+namespace {
+// The projector up to its last linear ("Mistral 3", Mistral3MultiModalProjector:
+// RMSNorm, the 2x2 patch merger, linear_1 + GELU): merge gather (normalising
+// each patch unless the norm follows the merge linear), merge linear, W1 with
+// GELU into p.g.
+int projector_head(const vlm_config* cfg, const void* d_tower_out, const Batch& b, const ProjWs& p, const uint8_t* pk,
+                   const ProjLayout& L, int32_t* d_status, cudaStream_t s) {
+  const int64_t D = cfg->width, E = cfg->proj_out, mm = static_cast<int64_t>(cfg->merge) * cfg->merge;
+  const bool after = cfg->norm_after_merge != 0 && cfg->merge > 1;
+  const float* g_proj = reinterpret_cast<const float*>(pk + L.g_proj);
+  VLM_TRY(upload_batch(b, p.bd, s));
+  VLM_TRY(launch_merge_norm(static_cast<const __nv_bfloat16*>(d_tower_out), after ? nullptr : g_proj, p.bd.info,
+                            p.bd.cu, b.n, b.T, static_cast<int>(D), cfg->merge, cfg->eps, p.z, d_status, s));
+  const __nv_bfloat16* y = p.z;
+  if (cfg->merge > 1) {
+    VLM_TRY(launch_gemm(VLM_EPI_BF16, p.z, pk + L.w_merge, b.Tm, D, mm * D, p.y, nullptr, nullptr, nullptr, 0,
+                        d_status, s));
+    y = p.y;
+    if (after) VLM_TRY(launch_rmsnorm_bf16(p.y, g_proj, p.y, b.Tm, static_cast<int>(D), cfg->eps, s));
+  }
+  return launch_gemm(VLM_EPI_GELU, y, pk + L.w1, b.Tm, E, D, p.g, nullptr, nullptr, nullptr, 0, d_status, s);
+}
+}  // namespace
+
 size_t vlm_merge_project_workspace_size(const vlm_config* cfg, const int32_t* image_hw, int n_images) {
   if (check_config(cfg) != VLM_OK) return 0;
   Batch b;
@@ -858,24 +883,51 @@ int vlm_merge_project(const vlm_config* cfg, const void* d_tower_out, const int3
   cudaStream_t s = as_stream(stream);
   const ProjLayout L = proj_layout(cfg);
   const uint8_t* pk = static_cast<const uint8_t*>(d_packed_projector);
-  const int64_t D = cfg->width, E = cfg->proj_out, mm = static_cast<int64_t>(cfg->merge) * cfg->merge;
-
-  const bool after = cfg->norm_after_merge != 0 && cfg->merge > 1;
-  const float* g_proj = reinterpret_cast<const float*>(pk + L.g_proj);
-  VLM_TRY(upload_batch(b, p.bd, s));
-  // the merge gather, normalising each patch unless the norm follows the merge linear
-  VLM_TRY(launch_merge_norm(static_cast<const __nv_bfloat16*>(d_tower_out), after ? nullptr : g_proj, p.bd.info,
-                            p.bd.cu, b.n, b.T, static_cast<int>(D), cfg->merge, cfg->eps, p.z, d_status, s));
-  const __nv_bfloat16* y = p.z;
-  if (cfg->merge > 1) {
-    VLM_TRY(launch_gemm(VLM_EPI_BF16, p.z, pk + L.w_merge, b.Tm, D, mm * D, p.y, nullptr, nullptr, nullptr, 0,
-                        d_status, s));
-    y = p.y;
-    if (after) VLM_TRY(launch_rmsnorm_bf16(p.y, g_proj, p.y, b.Tm, static_cast<int>(D), cfg->eps, s));
-  }
-  VLM_TRY(launch_gemm(VLM_EPI_GELU, y, pk + L.w1, b.Tm, E, D, p.g, nullptr, nullptr, nullptr, 0, d_status, s));
+  const int64_t E = cfg->proj_out;
+  VLM_TRY(projector_head(cfg, d_tower_out, b, p, pk, L, d_status, s));
   VLM_TRY(launch_gemm(VLM_EPI_BF16, p.g, pk + L.w2, b.Tm, E, E, d_out, nullptr, nullptr, nullptr, 0, d_status, s));
   return VLM_OK;
+}
+
+size_t vlm_merge_project_scatter_workspace_size(const vlm_config* cfg, const int32_t* image_hw, int n_images,
+                                                int64_t n_tokens) {
+  if (check_config(cfg) != VLM_OK || n_tokens <= 0 || n_tokens > (1LL << 40)) return 0;
+  Batch b;
+  if (make_batch(cfg, image_hw, n_images, &b) != VLM_OK) return 0;
+  size_t sc = 0;
+  carve_scatter(nullptr, n_tokens, &sc);
+  return carve_proj(nullptr, cfg, b).used + sc;
+}
+
+int vlm_merge_project_scatter(const vlm_config* cfg, const void* d_tower_out, const int32_t* image_hw, int n_images,
+                              const void* d_packed_projector, const int64_t* d_input_ids, int64_t n_tokens,
+                              void* d_text_embeds, void* d_workspace, size_t ws_bytes, int32_t* d_status,
+                              void* stream) {
+  VLM_TRY(check_config(cfg));
+  const SmBudgetScope budget(cfg->sm_budget);
+  if (d_tower_out == nullptr || d_packed_projector == nullptr || d_input_ids == nullptr || d_text_embeds == nullptr ||
+      d_workspace == nullptr || d_status == nullptr)
+    return VLM_ERR_INVALID_ARG;
+  if (n_tokens <= 0 || n_tokens > (1LL << 40)) return VLM_ERR_BAD_SHAPE;
+  if ((reinterpret_cast<uintptr_t>(d_workspace) & 255) ||
+      ((reinterpret_cast<uintptr_t>(d_tower_out) | reinterpret_cast<uintptr_t>(d_text_embeds)) & 15))
+    return VLM_ERR_INVALID_ARG;
+  Batch b;
+  VLM_TRY(make_batch(cfg, image_hw, n_images, &b));
+  const ProjWs p = carve_proj(d_workspace, cfg, b);
+  size_t sc = 0;
+  const ScatterWs sw = carve_scatter(static_cast<uint8_t*>(d_workspace) + p.used, n_tokens, &sc);
+  if (ws_bytes < p.used + sc) return VLM_ERR_WORKSPACE;
+  cudaStream_t s = as_stream(stream);
+  const ProjLayout L = proj_layout(cfg);
+  const uint8_t* pk = static_cast<const uint8_t*>(d_packed_projector);
+  const int64_t E = cfg->proj_out;
+  // the placeholders' rows first: on a count mismatch ok_flag stays 0 and the
+  // last linear writes nothing
+  VLM_TRY(launch_scatter_rows(d_input_ids, n_tokens, cfg->image_token_id, b.Tm, sw, d_status, s));
+  VLM_TRY(projector_head(cfg, d_tower_out, b, p, pk, L, d_status, s));
+  return launch_gemm_rows(p.g, pk + L.w2, b.Tm, E, E, d_text_embeds, n_tokens, sw.dst_rows, sw.ok_flag, d_status,
+                          s);
 }
 
 size_t vlm_scatter_workspace_size(int64_t n_tokens) {
@@ -1201,7 +1253,8 @@ int vlm_debug_checks(int32_t* first_failure) {
   *first_failure = 0;
 #ifdef VLM_DEBUG
   if (cudaDeviceSynchronize() != cudaSuccess) return VLM_ERR_CUDA;
-  const int words[3] = {debug_word_small_kernels(true), debug_word_frontend(true), debug_word_attention(true)};
+  const int words[4] = {debug_word_small_kernels(true), debug_word_frontend(true), debug_word_attention(true),
+                        debug_word_gemm(true)};
   for (int w : words) {
     if (w < 0) return VLM_ERR_CUDA;
     if (w != 0 && *first_failure == 0) *first_failure = w;

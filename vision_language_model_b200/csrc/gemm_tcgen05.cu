@@ -24,10 +24,15 @@
 // copied into TMEM.
 #include <cudaTypedefs.h>
 
+#define VLM_DEBUG_FILE_ID 4
+
+#include "gemm_rows.cuh"
 #include "kernels.cuh"
 #include "nvfp4.cuh"
 
 namespace vlm {
+
+VLM_DEBUG_UNIT(debug_word_gemm)
 
 namespace {
 
@@ -51,6 +56,9 @@ struct GemmArgs {
   const float* g_a = nullptr;  // NVFP4 operands: the two global scales (device memory); the
   const float* g_b = nullptr;  // epilogue multiplies by fp32(g_a * g_b)
   uint8_t* c_sf = nullptr;     // NVFP4 output (SwiGLU): block scales; out_scale is its global scale
+  const int64_t* dst_rows = nullptr;  // row-scattered store: destination row of each output row
+  const int32_t* ok_flag = nullptr;   // row-scattered store: nothing is written while *ok_flag == 0
+  int64_t c_rows = 0;                 // row-scattered store: rows of the destination table
 };
 
 template <int BN>
@@ -325,6 +333,33 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& args, Stager& st, 
       uint8_t* buf = st.acquire();
       st.write_row(buf, w);
       st.commit(buf, n0 + c, row0);
+    }
+  } else if constexpr (EPI == kEpiRows) {
+    // the masked scatter fused in: this lane's bf16 row goes to row
+    // dst_rows[row] of the table, 128 bytes per 64 columns; the lanes write 32
+    // different rows, which the output's small share of the kernel's traffic
+    // (one bf16 row per K columns of A read) absorbs
+    const int64_t dst = live && *args.ok_flag != 0 ? __ldg(args.dst_rows + row) : -1;
+    const bool put = dst >= 0 && VLM_DCHECK(dst < args.c_rows);
+#pragma unroll 1
+    for (int c = 0; c < BN; c += 64) {
+      uint32_t a[32], b[32];
+      tmem_ld32(tbase + c, a);
+      tmem_ld32(tbase + c + 32, b);
+      if (put) {
+        uint4* d = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(args.c) + dst * args.N + n0 + c);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          d[j] = make_uint4(pack_bf16x2(__uint_as_float(a[8 * j]), __uint_as_float(a[8 * j + 1])),
+                            pack_bf16x2(__uint_as_float(a[8 * j + 2]), __uint_as_float(a[8 * j + 3])),
+                            pack_bf16x2(__uint_as_float(a[8 * j + 4]), __uint_as_float(a[8 * j + 5])),
+                            pack_bf16x2(__uint_as_float(a[8 * j + 6]), __uint_as_float(a[8 * j + 7])));
+          d[4 + j] = make_uint4(pack_bf16x2(__uint_as_float(b[8 * j]), __uint_as_float(b[8 * j + 1])),
+                                pack_bf16x2(__uint_as_float(b[8 * j + 2]), __uint_as_float(b[8 * j + 3])),
+                                pack_bf16x2(__uint_as_float(b[8 * j + 4]), __uint_as_float(b[8 * j + 5])),
+                                pack_bf16x2(__uint_as_float(b[8 * j + 6]), __uint_as_float(b[8 * j + 7])));
+        }
+      }
     }
   }
 }
@@ -645,6 +680,7 @@ int dispatch_pair(int epi, const CUtensorMap& ta, const CUtensorMap& tb, const C
     case VLM_EPI_SWIGLU: return run_gemm_pair<VLM_EPI_SWIGLU>(ta, tb, tc, args, s);
     case VLM_EPI_ROPE: return run_gemm_pair<VLM_EPI_ROPE>(ta, tb, tc, args, s);
     case VLM_EPI_GELU: return run_gemm_pair<VLM_EPI_GELU>(ta, tb, tc, args, s);
+    case kEpiRows: return run_gemm_pair<kEpiRows>(ta, tb, tc, args, s);
     default: return VLM_ERR_INVALID_ARG;
   }
 }
@@ -1230,6 +1266,7 @@ int dispatch_epi(int epi, const CUtensorMap& ta, const CUtensorMap& tb, const CU
     case VLM_EPI_SWIGLU: return run_gemm<BN, VLM_EPI_SWIGLU>(ta, tb, tc, args, s);
     case VLM_EPI_ROPE: return run_gemm<BN, VLM_EPI_ROPE>(ta, tb, tc, args, s);
     case VLM_EPI_GELU: return run_gemm<BN, VLM_EPI_GELU>(ta, tb, tc, args, s);
+    case kEpiRows: return run_gemm<BN, kEpiRows>(ta, tb, tc, args, s);
     default: return VLM_ERR_INVALID_ARG;
   }
 }
@@ -1331,6 +1368,7 @@ int launch_gemm_f8(int epi, const void* a, const void* b, const float* colscale,
 int launch_gemm(int epi, const void* a, const void* b, int64_t M, int64_t N, int64_t K, void* c, void* c_bf16,
                 const int32_t* pos, const float2* rope, int64_t rope_cols, int32_t* status, cudaStream_t s) {
   if (a == nullptr || b == nullptr || c == nullptr) return VLM_ERR_INVALID_ARG;
+  if (epi < VLM_EPI_BF16 || epi > VLM_EPI_GELU) return VLM_ERR_INVALID_ARG;  // launch_gemm_rows has its own entry
   if (M <= 0 || N <= 0 || K <= 0 || M > (1LL << 31) - 1 || N > 65535 * 256LL || K > (1 << 20) || !tiles_fit(M, N))
     return VLM_ERR_BAD_SHAPE;
   if (K % GBK != 0 || N % 128 != 0) return VLM_ERR_UNSUPPORTED;
@@ -1373,6 +1411,43 @@ int launch_gemm(int epi, const void* a, const void* b, int64_t M, int64_t N, int
     return dispatch_pair(epi, ta, tb2, tc, args, s);
   }
   return dispatch_epi<128>(epi, ta, tb, tc, args, s);
+}
+
+int launch_gemm_rows(const void* a, const void* b, int64_t M, int64_t N, int64_t K, void* c, int64_t c_rows,
+                     const int64_t* dst_rows, const int32_t* ok_flag, int32_t* status, cudaStream_t s) {
+  if (a == nullptr || b == nullptr || c == nullptr || dst_rows == nullptr || ok_flag == nullptr)
+    return VLM_ERR_INVALID_ARG;
+  if (M <= 0 || N <= 0 || K <= 0 || c_rows <= 0 || M > (1LL << 31) - 1 || N > 65535 * 256LL || K > (1 << 20) ||
+      !tiles_fit(M, N))
+    return VLM_ERR_BAD_SHAPE;
+  if (K % GBK != 0 || N % 128 != 0) return VLM_ERR_UNSUPPORTED;
+  if ((reinterpret_cast<uintptr_t>(a) | reinterpret_cast<uintptr_t>(b) | reinterpret_cast<uintptr_t>(c)) & 15)
+    return VLM_ERR_INVALID_ARG;
+  const int bn = N % 256 == 0 ? 256 : 128;
+  CUtensorMap ta, tb, tc;
+  if (!make_tmap_2d_bf16(&ta, a, K, M, K * 2, GBK, GBM)) return VLM_ERR_CUDA;
+  if (!make_tmap_2d_bf16(&tb, b, K, N, K * 2, GBK, bn == 256 ? 128 : bn)) return VLM_ERR_CUDA;
+  // the kernels take an output map; this epilogue stores without it
+  if (!make_tmap_2d(&tc, c, false, N, c_rows, N * 2, 64, 1)) return VLM_ERR_CUDA;
+  GemmArgs args;
+  args.M = static_cast<int>(M);
+  args.N = static_cast<int>(N);
+  args.K = static_cast<int>(K);
+  args.m_tiles = static_cast<int>(bn == 256 ? (M + 255) / 256 : (M + GBM - 1) / GBM);
+  args.n_tiles = static_cast<int>(N / bn);
+  args.c = c;
+  args.c_bf16 = nullptr;
+  args.pos = nullptr;
+  args.rope = nullptr;
+  args.rope_cols = 0;
+  args.status = status;
+  args.colscale = nullptr;
+  args.out_scale = 1.0f;
+  args.dst_rows = dst_rows;
+  args.ok_flag = ok_flag;
+  args.c_rows = c_rows;
+  if (bn == 256) return dispatch_pair(kEpiRows, ta, tb, tc, args, s);
+  return dispatch_epi<128>(kEpiRows, ta, tb, tc, args, s);
 }
 
 namespace {

@@ -5,6 +5,7 @@
 #include <algorithm>
 #include <type_traits>
 
+#include "gemm_rows.cuh"
 #include "kernels.cuh"
 #include "nvfp4.cuh"
 
@@ -1097,6 +1098,24 @@ int launch_scatter(const int64_t* ids, int64_t n, int64_t token, const void* img
                    static_cast<const uint4*>(img), static_cast<uint4*>(text), ws.dst_rows, ws.ok_flag, n_img, vec, n);
   launch_end(KC_SCATTER, s);
   note_extra_launches(3);
+  return e == cudaSuccess ? VLM_OK : VLM_ERR_CUDA;
+}
+
+int launch_scatter_rows(const int64_t* ids, int64_t n, int64_t token, int64_t n_img, const ScatterWs& ws,
+                        int32_t* status, cudaStream_t s) {
+  if (n <= 0) return VLM_ERR_BAD_SHAPE;
+  const int64_t n_chunks = (n + 255) / 256;
+  const dim3 chunks(static_cast<unsigned>(n_chunks));
+  launch_begin(KC_SCATTER, s);
+  cudaError_t e = launch_pdl(scatter_count_kernel, chunks, dim3(256), 0, s, ids, n, token, ws.chunk_count);
+  if (e == cudaSuccess)
+    e = launch_pdl(scatter_scan_kernel, dim3(1), dim3(1024), 0, s, ws.chunk_count, n_chunks, n_img, ws.chunk_base,
+                   ws.ok_flag, status);
+  if (e == cudaSuccess)
+    e = launch_pdl(scatter_positions_kernel, chunks, dim3(256), 0, s, ids, n, token, ws.chunk_base, ws.ok_flag,
+                   ws.dst_rows, n_img);
+  launch_end(KC_SCATTER, s);
+  note_extra_launches(2);
   return e == cudaSuccess ? VLM_OK : VLM_ERR_CUDA;
 }
 

@@ -107,6 +107,8 @@ def lib() -> ctypes.CDLL:
             "vlm_encode": (I32, [CP, P, P, I32, P, P, P, SZ, P, P]),
             "vlm_merge_project_workspace_size": (SZ, [CP, P, I32]),
             "vlm_merge_project": (I32, [CP, P, P, I32, P, P, P, SZ, P, P]),
+            "vlm_merge_project_scatter_workspace_size": (SZ, [CP, P, I32, I64]),
+            "vlm_merge_project_scatter": (I32, [CP, P, P, I32, P, P, I64, P, P, SZ, P, P]),
             "vlm_scatter_workspace_size": (SZ, [I64]),
             "vlm_scatter": (I32, [P, I64, I64, P, I64, P, I64, P, SZ, P, P]),
             "vlm_resize_target": (I32, [I32, I32, I32, I32, ctypes.POINTER(ctypes.c_int32),
@@ -301,6 +303,38 @@ def merge_project(cfg: Config, tower_out: torch.Tensor, image_hw, packed_project
                                _dev(workspace, "workspace"), workspace.numel(), _dev(status, "status"),
                                _stream(stream)), "vlm_merge_project")
     return out
+
+
+def merge_project_scatter_workspace_size(cfg: Config, image_hw, n_tokens: int) -> int:
+    arr, n = _hw_array(image_hw)
+    return int(lib().vlm_merge_project_scatter_workspace_size(ctypes.byref(cfg), arr, n, int(n_tokens)))
+
+
+def merge_project_scatter(cfg: Config, tower_out: torch.Tensor, image_hw, packed_projector: torch.Tensor,
+                          input_ids: torch.Tensor, text_embeds: torch.Tensor, workspace=None, status=None,
+                          stream=None) -> torch.Tensor:
+    """Projector with the masked scatter fused into its last linear: rows of
+    text_embeds (bf16 [n_tokens, proj_out]) at cfg.image_token_id positions <-
+    the projected merged tokens, in order; no [T_m, proj_out] buffer."""
+    L = lib()
+    if input_ids.dtype != torch.int64:
+        raise ValueError("input_ids must be int64")
+    n = input_ids.numel()
+    if text_embeds.dtype != torch.bfloat16 or text_embeds.dim() != 2 or tuple(text_embeds.shape) != (n, cfg.proj_out):
+        raise ValueError("text_embeds must be bf16 [n_tokens, proj_out]")
+    arr, n_img = _hw_array(image_hw)
+    dev = text_embeds.device
+    if workspace is None:
+        workspace = _empty(max(256, L.vlm_merge_project_scatter_workspace_size(ctypes.byref(cfg), arr, n_img, n)),
+                           dtype=torch.uint8, device=dev)
+    if status is None:
+        status = new_status(dev)
+    _check(L.vlm_merge_project_scatter(ctypes.byref(cfg), _dev(tower_out, "tower_out"), arr, n_img,
+                                       _dev(packed_projector, "packed_projector"), _dev(input_ids, "input_ids"), n,
+                                       _dev(text_embeds, "text_embeds"), _dev(workspace, "workspace"),
+                                       workspace.numel(), _dev(status, "status"), _stream(stream)),
+           "vlm_merge_project_scatter")
+    return text_embeds
 
 
 def scatter_workspace_size(n_tokens: int) -> int:
@@ -761,8 +795,10 @@ class ImagePipeline:
         ws = max(enc_ws, merge_project_workspace_size(cfg, self.image_hw))
         self.workspace = _empty(ws, dtype=torch.uint8, device=device)
         self.status = new_status(device)
+        self._fused_ws = None  # vlm_merge_project_scatter's workspace, sized on first use
 
-    def __call__(self, pixels: torch.Tensor, stream=None) -> torch.Tensor:
+    def encode(self, pixels: torch.Tensor, stream=None) -> torch.Tensor:
+        """The tower alone: pixels -> self.tower_out."""
         if self.nvfp4_act_scales is not None:
             encode_nvfp4(self.cfg, pixels, self.image_hw, self.packed_tower, self.nvfp4_act_scales,
                          out=self.tower_out, workspace=self.workspace, status=self.status, stream=stream)
@@ -772,9 +808,27 @@ class ImagePipeline:
         else:
             encode_fp8(self.cfg, pixels, self.image_hw, self.packed_tower, self.fp8_act_scales, out=self.tower_out,
                        workspace=self.workspace, status=self.status, stream=stream)
+        return self.tower_out
+
+    def __call__(self, pixels: torch.Tensor, stream=None) -> torch.Tensor:
+        self.encode(pixels, stream)
         merge_project(self.cfg, self.tower_out, self.image_hw, self.packed_proj, out=self.embeds,
                       workspace=self.workspace, status=self.status, stream=stream)
         return self.embeds
+
+    def embed_into(self, pixels: torch.Tensor, input_ids: torch.Tensor, text_embeds: torch.Tensor,
+                   stream=None) -> torch.Tensor:
+        """The whole image path written into the token embeddings in place:
+        vlm_encode, then vlm_merge_project_scatter (the masked scatter fused
+        into the projector's last linear; self.embeds is not written). Rows of
+        text_embeds at cfg.image_token_id positions receive this batch's
+        projected merged tokens in order; the others are left untouched."""
+        self.encode(pixels, stream)
+        need = merge_project_scatter_workspace_size(self.cfg, self.image_hw, input_ids.numel())
+        if self._fused_ws is None or self._fused_ws.numel() < need:
+            self._fused_ws = _empty(max(256, need), dtype=torch.uint8, device=self.tower_out.device)
+        return merge_project_scatter(self.cfg, self.tower_out, self.image_hw, self.packed_proj, input_ids, text_embeds,
+                                     workspace=self._fused_ws, status=self.status, stream=stream)
 
 
 class GraphStep:
