@@ -101,6 +101,9 @@ def parse_args():
                    help="instead of a step: time the tower's GEMM shapes (12,100 rows), bf16, E4M3 and NVFP4, each "
                         "with its fused epilogue and with a plain store, beside torch's cuBLAS / cuBLASLt GEMM; one "
                         "JSON line per shape and dtype")
+    p.add_argument("--scatter", default="fused", choices=["fused", "separate"],
+                   help="fused (default): vlm_merge_project_scatter, the masked scatter in the projector's last "
+                        "linear, no embedding buffer; separate: vlm_merge_project then vlm_scatter")
     p.add_argument("--profile-steps", type=int, default=0,
                    help="for ncu: run this many plain steps after warmup and exit (no JSON)")
     return p.parse_args()
@@ -600,9 +603,17 @@ def run_ours(args, wl):
     scatter_ws = torch.empty(max(256, vlm.scatter_workspace_size(ids.numel())), dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
 
+    fused = args.scatter == "fused"
+
     def step():
         if photo:
             vlm.preprocess(photo_dev, [photo], sizes, out=pix)
+        if fused:
+            if photo:
+                vlm.expand_placeholders(marker_ids, marker, lens_m, cfg.image_token_id, out=ids, workspace=expand_ws,
+                                        status=pipe.status)
+            pipe.embed_into(pix, ids, text)
+            return
         emb = pipe(pix)
         if photo:
             vlm.expand_placeholders(marker_ids, marker, lens_m, cfg.image_token_id, out=ids, workspace=expand_ws,
@@ -671,10 +682,17 @@ def run_ours(args, wl):
         pix_in, ids_in = inputs
         if photo:
             vlm.preprocess(pix_in, [photo], sizes, out=pix)
+            if fused:
+                vlm.expand_placeholders(ids_in, marker, lens_m, cfg.image_token_id, out=ids, workspace=expand_ws,
+                                        status=pipe.status)
+                pipe.embed_into(pix, ids, result)
+                return
             emb = pipe(pix)
             vlm.expand_placeholders(ids_in, marker, lens_m, cfg.image_token_id, out=ids, workspace=expand_ws,
                                     status=pipe.status)
             vlm.scatter(ids, emb, result, cfg.image_token_id, workspace=scatter_ws, status=pipe.status)
+        elif fused:
+            pipe.embed_into(pix_in, ids_in, result)
         else:
             emb = pipe(pix_in)
             vlm.scatter(ids_in, emb, result, cfg.image_token_id, workspace=scatter_ws, status=pipe.status)
@@ -780,14 +798,22 @@ def run_ours(args, wl):
                     f"per launch: fp32 row read + the {out_name} row written (+ the fp32 write-back of ln_pre once)"),
         "patch_gather": (T * (3 * p_ * p_ * 4 + kp_ * 2), ms_im2col, "fp32 pixels read + bf16 patch rows written"),
         "merge_gather": (2 * T * D_ * 2, ms_merge, "bf16 tower rows read + bf16 merged rows written"),
-        "scatter": (2 * Tm * row_bytes + ids.numel() * 8, ms_scatter,
-                    "image rows read + written into the text rows + ids read"),
     }
+    if not fused:
+        mb["scatter"] = (2 * Tm * row_bytes + ids.numel() * 8, ms_scatter,
+                         "image rows read + written into the text rows + ids read")
     line["memory_bound_kernels"] = {
         k: {"bytes_per_step": int(b), "ms_per_step": t / args.steps,
             "achieved_gbs": b / (t / args.steps / 1e3) / 1e9 if t > 0 else None,
             "frac_of_hbm": b / (t / args.steps / 1e3) / 1e9 / peaks["hbm_gbs"] if t > 0 else None, "bytes": note}
         for k, (b, t, note) in mb.items()}
+    if fused:
+        line["config"]["scatter"] = "fused into the projector's last linear (vlm_merge_project_scatter)"
+        line["scatter_fused"] = {
+            "positions_ms_per_step": ms_scatter / args.steps,
+            "note": "the image rows go from the last projector GEMM's epilogue straight to their text rows (counted "
+                    "with the GEMMs); what is left of the scatter is its placeholder count, scan and positions "
+                    "kernels over the ids"}
     if args.graph:
         line["config"]["launch"] = f"one CUDA graph per step ({graph.launches_per_replay} kernels)"
     if args.side_stream:

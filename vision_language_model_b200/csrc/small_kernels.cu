@@ -1101,9 +1101,65 @@ int launch_scatter(const int64_t* ids, int64_t n, int64_t token, const void* img
   return e == cudaSuccess ? VLM_OK : VLM_ERR_CUDA;
 }
 
+// The placeholder positions of up to kScatterRowsOneCta ids in one CTA: each
+// thread counts a contiguous run of ids, one block scan ranks the runs, and
+// the runs' placeholders are written in order once the total is known to
+// equal n_img (otherwise ok_flag = 0 and nothing is written).
+constexpr int kScatterRowsOneCta = 32768;
+__global__ void __launch_bounds__(1024) scatter_rows_one_cta_kernel(const int64_t* __restrict__ ids, int n,
+                                                                      int64_t token, int64_t n_img,
+                                                                      int64_t* __restrict__ dst_rows,
+                                                                      int32_t* __restrict__ ok_flag, int32_t* status) {
+  griddep_wait();
+  griddep_launch_dependents();
+  __shared__ int warp_sums[32];
+  const int per = (n + 1023) / 1024;
+  const int beg = min(n, static_cast<int>(threadIdx.x) * per), end = min(n, beg + per);
+  int cnt = 0;
+  for (int i = beg; i < end; ++i) cnt += __ldg(ids + i) == token ? 1 : 0;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int incl = cnt;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) warp_sums[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    int w = warp_sums[lane];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w += y;
+    }
+    warp_sums[lane] = w;  // inclusive over warps
+  }
+  __syncthreads();
+  const int total = warp_sums[31];
+  if (total != n_img) {
+    if (threadIdx.x == 0) {
+      *ok_flag = 0;
+      set_status(status, VLM_ERR_COUNT_MISMATCH);
+    }
+    return;
+  }
+  int64_t k = (warp > 0 ? warp_sums[warp - 1] : 0) + incl - cnt;
+  for (int i = beg; i < end; ++i)
+    if (__ldg(ids + i) == token && VLM_DCHECK(k >= 0 && k < n_img)) dst_rows[k++] = i;
+  if (threadIdx.x == 0) *ok_flag = 1;
+}
+
 int launch_scatter_rows(const int64_t* ids, int64_t n, int64_t token, int64_t n_img, const ScatterWs& ws,
                         int32_t* status, cudaStream_t s) {
   if (n <= 0) return VLM_ERR_BAD_SHAPE;
+  if (n <= kScatterRowsOneCta) {
+    launch_begin(KC_SCATTER, s);
+    const cudaError_t e = launch_pdl(scatter_rows_one_cta_kernel, dim3(1), dim3(1024), 0, s, ids, static_cast<int>(n),
+                                     token, n_img, ws.dst_rows, ws.ok_flag, status);
+    launch_end(KC_SCATTER, s);
+    return e == cudaSuccess ? VLM_OK : VLM_ERR_CUDA;
+  }
   const int64_t n_chunks = (n + 255) / 256;
   const dim3 chunks(static_cast<unsigned>(n_chunks));
   launch_begin(KC_SCATTER, s);
