@@ -812,8 +812,8 @@ def run_ours(args, wl):
         line["scatter_fused"] = {
             "positions_ms_per_step": ms_scatter / args.steps,
             "note": "the image rows go from the last projector GEMM's epilogue straight to their text rows (counted "
-                    "with the GEMMs); what is left of the scatter is its placeholder count, scan and positions "
-                    "kernels over the ids"}
+                    "with the GEMMs); what is left of the scatter is the kernel that finds the placeholders' rows "
+                    "(one launch up to 32,768 ids; count, scan and positions kernels above that)"}
     if args.graph:
         line["config"]["launch"] = f"one CUDA graph per step ({graph.launches_per_replay} kernels)"
     if args.side_stream:
