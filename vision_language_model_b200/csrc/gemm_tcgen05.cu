@@ -336,9 +336,10 @@ __device__ __forceinline__ void epilogue_tile(const GemmArgs& args, Stager& st, 
     }
   } else if constexpr (EPI == kEpiRows) {
     // the masked scatter fused in: this lane's bf16 row goes to row
-    // dst_rows[row] of the table, 128 bytes per 64 columns; the lanes write 32
-    // different rows, which the output's small share of the kernel's traffic
-    // (one bf16 row per K columns of A read) absorbs
+    // dst_rows[row] of the table, 128 bytes per 64 columns with 16-byte
+    // stores. The 32 lanes write 32 different rows (no TMA box fits scattered
+    // rows), but the output is a small share of this GEMM's traffic (each
+    // output row costs K values of A read), and the stores are not waited on
     const int64_t dst = live && *args.ok_flag != 0 ? __ldg(args.dst_rows + row) : -1;
     const bool put = dst >= 0 && VLM_DCHECK(dst < args.c_rows);
 #pragma unroll 1
