@@ -125,6 +125,9 @@ def test_gemm_shape_checks_return_before_launch(L):
     assert L.vlm_gemm(3, fake, fake, 128, 384, 64, fake, None, None, None, 0, st, None) == vlm.ERR_UNSUPPORTED
     assert L.vlm_gemm(0, None, fake, 128, 128, 64, fake, None, None, None, 0, st, None) == vlm.ERR_INVALID_ARG
     assert L.vlm_gemm(0, fake, fake, 0, 128, 64, fake, None, None, None, 0, st, None) == vlm.ERR_BAD_SHAPE
+    # epilogue codes outside the public set (6 is the projector's internal row-scattered store)
+    for epi in (-1, 6, 7):
+        assert L.vlm_gemm(epi, fake, fake, 128, 256, 64, fake, None, None, None, 0, st, None) == vlm.ERR_INVALID_ARG
 
 
 def test_package_import_does_not_load_library():
