@@ -213,3 +213,29 @@ def test_sm_budget_gives_the_same_bits(kind):
             assert launches == base[1] + layers * (-(-qtiles // chunk) - 1), (budget, launches, base[1])
         else:
             assert launches == base[1]
+
+
+def test_fused_scatter_under_graph_replay_and_sm_budgets():
+    """ImagePipeline.embed_into (the scatter fused into the projector's last
+    linear) replayed as one CUDA graph, and run with the encoder confined to 2
+    and 40 SMs, writes the same rows as the eager separate calls."""
+    cfg, pipe = _pipeline()
+    ids, text0 = _text_setup(cfg, pipe)
+    pix = pixels_to_device(synth.images(3, SIZES))
+    ref = text0.clone()
+    vlm.scatter(ids, pipe(pix), ref, cfg.image_token_id, status=pipe.status)
+    text = text0.clone()
+    g = vlm.GraphStep(lambda: pipe.embed_into(pix, ids, text))  # one eager call first, then the capture
+    text.copy_(text0)
+    g()
+    torch.cuda.synchronize()
+    assert vlm.status_sync(pipe.status) == vlm.OK
+    assert torch.equal(text, ref)
+    tw = tower_to_device(synth.tower_weights(3, cfg.layers, cfg.width, cfg.mlp, cfg.patch))
+    pw = tower_to_device(synth.projector_weights(3, cfg.width, cfg.merge, cfg.proj_out))
+    for budget in (2, 40):
+        pb = vlm.ImagePipeline(vlm.preset("mistral3", layers=cfg.layers, sm_budget=budget), tw, pw, SIZES)
+        t = text0.clone()
+        pb.embed_into(pix, ids, t)
+        assert vlm.status_sync(pb.status) == vlm.OK
+        assert torch.equal(t, ref), budget
