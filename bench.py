@@ -807,10 +807,10 @@ def run_ours(args, wl):
             "achieved_gbs": b / (t / args.steps / 1e3) / 1e9 if t > 0 else None,
             "frac_of_hbm": b / (t / args.steps / 1e3) / 1e9 / peaks["hbm_gbs"] if t > 0 else None, "bytes": note}
         for k, (b, t, note) in mb.items()}
-    if fused:
-        line["config"]["scatter"] = "fused into the projector's last linear (vlm_merge_project_scatter)"
+    if fused:  # (config stays the workload's own keys, the same as the reference arm's)
         line["scatter_fused"] = {
             "positions_ms_per_step": ms_scatter / args.steps,
+            "entry": "vlm_merge_project_scatter (the masked scatter fused into the projector's last linear)",
             "note": "the image rows go from the last projector GEMM's epilogue straight to their text rows (counted "
                     "with the GEMMs); what is left of the scatter is the kernel that finds the placeholders' rows "
                     "(one launch up to 32,768 ids; count, scan and positions kernels above that)"}
