@@ -90,3 +90,27 @@ def test_fused_full_size_1540_equals_separate():
     pipe.embed_into(pix, ids, fused)
     assert vlm.status_sync(pipe.status) == vlm.OK
     assert torch.equal(fused, sep)
+
+
+def test_fused_above_one_cta_id_limit():
+    """More than 32,768 ids: the placeholder rows come from the count, scan and
+    positions kernels instead of the one-CTA kernel; same rows, and a count
+    mismatch still writes nothing."""
+    sizes = [(224, 224), (84, 112)]
+    cfg, _, _, imgs, pipe = _setup("mistral3", sizes, seed=14)
+    pix = pixels_to_device(imgs)
+    Tm = vlm.num_merged(cfg, sizes)
+    ids = _ids(40000 - Tm, Tm, seed=15, token=cfg.image_token_id)
+    text0 = _text(ids.numel(), cfg.proj_out, seed=16)
+    sep = text0.clone()
+    vlm.scatter(ids, pipe(pix).clone(), sep, image_token_id=cfg.image_token_id)
+    fused = text0.clone()
+    pipe.embed_into(pix, ids, fused)
+    assert vlm.status_sync(pipe.status) == vlm.OK
+    assert torch.equal(fused, sep)
+    bad = ids.clone()
+    bad[torch.nonzero(bad == cfg.image_token_id)[0]] = cfg.image_token_id + 1   # one placeholder too few
+    fused = text0.clone()
+    pipe.embed_into(pix, bad, fused)
+    assert vlm.status_sync(pipe.status) == vlm.ERR_COUNT_MISMATCH
+    assert torch.equal(fused, text0)
