@@ -365,3 +365,19 @@ def test_merge_project_scatter_rejects_bad_arguments_before_launch(L):
     assert call(7, ctypes.c_void_p(264)) == vlm.ERR_INVALID_ARG   # text rows not 16-byte aligned
     assert call(9, ws - 1) == vlm.ERR_WORKSPACE
     assert call(2, (ctypes.c_int32 * 2)(225, 224)) != vlm.OK      # not on the merged-patch grid
+
+
+def test_merge_project_scatter_wrapper_checks_dtypes_and_shapes():
+    """The binding rejects a wrong id dtype or token-table shape before calling the library."""
+    import torch
+    cfg = vlm.preset("mistral3", layers=1)
+    tower_out = torch.zeros(256, cfg.width, dtype=torch.bfloat16)
+    proj = torch.zeros(16, dtype=torch.uint8)
+    ids = torch.full((100,), cfg.image_token_id, dtype=torch.int64)
+    good_text = torch.zeros(100, cfg.proj_out, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        vlm.merge_project_scatter(cfg, tower_out, [(224, 224)], proj, ids.to(torch.int32), good_text)
+    for bad in (torch.zeros(99, cfg.proj_out, dtype=torch.bfloat16), torch.zeros(100, 1024, dtype=torch.bfloat16),
+                torch.zeros(100, cfg.proj_out, dtype=torch.float32)):
+        with pytest.raises(ValueError):
+            vlm.merge_project_scatter(cfg, tower_out, [(224, 224)], proj, ids, bad)
