@@ -813,7 +813,7 @@ def run_ours(args, wl):
             "entry": "vlm_merge_project_scatter (the masked scatter fused into the projector's last linear)",
             "note": "the image rows go from the last projector GEMM's epilogue straight to their text rows (counted "
                     "with the GEMMs); what is left of the scatter is the kernel that finds the placeholders' rows "
-                    "(one launch up to 32,768 ids; count, scan and positions kernels above that)"}
+                    "(one launch up to 4,096 ids; count, scan and positions kernels above that)"}
     if args.graph:
         line["config"]["launch"] = f"one CUDA graph per step ({graph.launches_per_replay} kernels)"
     if args.side_stream:

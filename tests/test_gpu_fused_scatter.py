@@ -93,8 +93,8 @@ def test_fused_full_size_1540_equals_separate():
 
 
 def test_fused_above_one_cta_id_limit():
-    """More than 32,768 ids: the placeholder rows come from the count, scan and
-    positions kernels instead of the one-CTA kernel; same rows, and a count
+    """40,000 ids, above the one-CTA kernel's 4,096: the placeholder rows come
+    from the count, scan and positions kernels; same rows, and a count
     mismatch still writes nothing."""
     sizes = [(224, 224), (84, 112)]
     cfg, _, _, imgs, pipe = _setup("mistral3", sizes, seed=14)

@@ -22,7 +22,7 @@ int launch_gemm_rows(const void* a, const void* b, int64_t M, int64_t N, int64_t
                      const int64_t* dst_rows, const int32_t* ok_flag, int32_t* status, cudaStream_t s);
 
 // The masked scatter's placeholder positions without its copy, over ids[0, n)
-// (one kernel up to 32,768 ids, else the count, scan and positions kernels). dst_rows[k] = the position of the k-th
+// (one kernel up to 4,096 ids, else the count, scan and positions kernels). dst_rows[k] = the position of the k-th
 // id equal to `token`; *ok_flag = 1 when there are exactly n_img of them,
 // otherwise 0 (dst_rows is then not written) and *status takes
 // VLM_ERR_COUNT_MISMATCH. Uses ws.chunk_count, ws.chunk_base, ws.dst_rows and

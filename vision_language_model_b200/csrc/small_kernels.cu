@@ -1104,8 +1104,11 @@ int launch_scatter(const int64_t* ids, int64_t n, int64_t token, const void* img
 // The placeholder positions of up to kScatterRowsOneCta ids in one CTA: each
 // thread counts a contiguous run of ids, one block scan ranks the runs, and
 // the runs' placeholders are written in order once the total is known to
-// equal n_img (otherwise ok_flag = 0 and nothing is written).
-constexpr int kScatterRowsOneCta = 32768;
+// equal n_img (otherwise ok_flag = 0 and nothing is written). A thread's run
+// is read one id after another, so longer id sequences go to the count, scan
+// and positions kernels, which spread them over many CTAs (16,384 ids: 33 us
+// in one CTA).
+constexpr int kScatterRowsOneCta = 4096;
 __global__ void __launch_bounds__(1024) scatter_rows_one_cta_kernel(const int64_t* __restrict__ ids, int n,
                                                                       int64_t token, int64_t n_img,
                                                                       int64_t* __restrict__ dst_rows,
